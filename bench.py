@@ -1,0 +1,377 @@
+#!/usr/bin/env python
+"""Benchmark: causal RACE attention forward + backward on one B200 per rank.
+
+Default workload: B1 H1 N=4,194,304 d64 bf16, L16 P4 tau 0.5, clustered Q/K (the
+sequence-length headline).  One step = race_attn_forward + race_attn_backward through the
+C ABI on device-resident inputs (each input tensor is 512 MiB, larger than the 126 MB L2,
+so no L2 flush is needed between steps).  Prints one JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+With N > 1 (torchrun) every rank runs its own independent sequence (weak scaling, no
+collective on the data path); the timed region is bracketed by barriers and the time is
+the max over ranks.  ``--impl reference`` times the fp64 CPU oracle instead, on a bounded
+prefix of the same workload, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import race_inputs  # noqa: E402
+
+METRIC = "causal RACE attn fwd+bwd tokens/s at N=4M,d=64 (1 B200); % of roofline"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "sm_max_mhz": 1965.0}
+FP32_LANES_PER_SM = 128  # FMA units per SM (4 partitions x 32)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        d["source"] = "measured"
+        return d
+    d = dict(PEAKS_FALLBACK)
+    d["source"] = "fallback"
+    return d
+
+
+# ---- algorithmic work (per token per head; s = element size; M = L*2^P) ---------------
+def step_work(w: race_inputs.Workload):
+    s = 4 if w.dtype == "f32" else 2
+    M, d, LP = w.L * w.R, w.d, w.L * w.P
+    byts = 12 * d * s + 8
+    flops = 12 * M * (d + 1) + 12 * LP * d
+    return byts, flops
+
+
+def kernel_work(name: str, w: race_inputs.Workload):
+    """(algorithmic bytes, algorithmic flops) per token per head of one kernel launch."""
+    s = 4 if w.dtype == "f32" else 2
+    M, d, LP, D = w.L * w.R, w.d, w.L * w.P, w.d + 1
+    table = {
+        "agg_kv": (2 * d * s, 2 * M * D + 2 * LP * d),
+        "fwd_walk": (4 * d * s + 4, 4 * M * D + 4 * LP * d),
+        "bwd_q_walk": (6 * d * s + 4, 4 * M * D + 6 * LP * d),
+        "agg_qdy": (3 * d * s + 4, 2 * M * D + 2 * LP * d),
+        "bwd_kv_walk": (7 * d * s + 4, 6 * M * D + 6 * LP * d),
+        "bwd_walk": (10 * d * s + 4, 10 * M * D + 12 * LP * d),
+    }
+    for key, val in table.items():
+        if name.endswith(key):
+            return val
+    return None
+
+
+def is_tensor_core_kernel(name: str) -> bool:
+    return name.startswith("tc_")
+
+
+# ---- clocks ----------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---- CPU baseline (the fp64 oracle) -----------------------------------------------------
+def oracle_step(inp_cpu, w, n):
+    import numpy as np
+    import oracle
+    q, k, v, do = (inp_cpu[x][0, 0, :n].to(torch.float64).numpy() for x in ("q", "k", "v", "do"))
+    W = inp_cpu["W"].to(torch.float64).numpy()
+    t0 = time.perf_counter()
+    oracle.forward(q, k, v, W, w.tau, w.causal)
+    oracle.backward(q, k, v, W, do, w.tau, w.causal)
+    return time.perf_counter() - t0
+
+
+def oracle_sample_size(inp_cpu, w, target_s):
+    n = 2048
+    t = oracle_step(inp_cpu, w, n)
+    n2 = int(n * target_s / max(t, 1e-3))
+    n2 = max(1024, min(n2, w.N, 1 << 20))
+    return n2
+
+
+def cpu_baseline(w, target_s=12.0):
+    import oracle
+    small = race_inputs.make_inputs(w.with_n(min(w.N, 1 << 20)), "cpu")
+    n = oracle_sample_size(small, w, target_s)
+    t = oracle_step(small, w, n)
+    return {"value": n / t, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": "causal fwd+bwd of the first %d tokens of head 0 (inputs drawn with the "
+                      "workload's recipe), fp64, wall clock %.1f s" % (n, t)}
+
+
+def run_reference(args, w):
+    """Time the fp64 oracle, as it stands, on a bounded prefix of the workload."""
+    import oracle
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    small = race_inputs.make_inputs(w.with_n(min(w.N, 1 << 20)), "cpu")
+    n = oracle_sample_size(small, w, min(10.0, budget))
+    for _ in range(args.warmup):
+        oracle_step(small, w, min(n, 2048))
+    times = [oracle_step(small, w, n) for _ in range(args.steps)]
+    t = statistics.mean(times)
+    val = n / t
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "L": w.L,
+                       "P": w.P, "tau": w.tau, "causal": w.causal,
+                       "sample_tokens_per_step": n},
+            "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": oracle.num_threads(),
+                             "kind": "oracle",
+                             "sample": "causal fwd+bwd of the first %d tokens of head 0 per step"
+                                       % n},
+            "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---- the CUDA library -------------------------------------------------------------------
+def run_ours(args, w):
+    import linear_attention_soft_b200 as ra
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    peaks = load_peaks()
+    # each rank draws its own independent sequence (weak scaling)
+    import dataclasses
+    wr = dataclasses.replace(w, seed=w.seed + 1000 * rank)
+    inp = race_inputs.make_inputs(wr, dev)
+    q, k, v, W, do = inp["q"], inp["k"], inp["v"], inp["W"], inp["do"]
+    B, H, N, d = q.shape
+    L, P = w.L, w.P
+    out = torch.empty_like(q)
+    den = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    code = ra.RACE_F32 if w.dtype == "f32" else ra.RACE_BF16
+    ws_f = torch.empty(ra.race_attn_workspace_size(B, H, N, d, L, P, w.causal, 0, code),
+                       dtype=torch.uint8, device=dev)
+    ws_b = torch.empty(ra.race_attn_workspace_size(B, H, N, d, L, P, w.causal, 1, code),
+                       dtype=torch.uint8, device=dev)
+    ctx = torch.empty(ra.race_attn_ctx_size(B, H, N, d, L, P, w.causal) // 4,
+                      dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(qq=q, kk=k, vv=v, dd=do):
+        ra.race_attn_forward(qq, kk, vv, W, out, den, ctx, w.tau, w.causal, ws_f, stream)
+        ra.race_attn_backward(qq, kk, vv, W, out, den, dd, ctx, dq, dk, dv, w.tau, w.causal,
+                              ws_b, stream)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    barrier()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    ra.race_attn_profile_reset()
+    ra.race_attn_profile_enable(True)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    ra.race_attn_profile_enable(False)
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    prof = ra.race_attn_profile_read()
+    ms_t = torch.tensor([ms], device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(ms_t, op=torch.distributed.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+    tokens_all = B * N * world
+    value = tokens_all / (ms_max / 1e3)
+
+    # ---- end to end through the C ABI with host buffers --------------------------------
+    host = {n: t.cpu().pin_memory() for n, t in (("q", q), ("k", k), ("v", v), ("do", do))}
+    host_out = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+                for n, t in (("out", out), ("dq", dq), ("dk", dk), ("dv", dv))}
+    dq_in = {n: torch.empty_like(host[n], device=dev) for n in host}
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+    e2e_steps = max(2, min(args.steps, 5))
+
+    def e2e_step():
+        for n in host:
+            dq_in[n].copy_(host[n], non_blocking=True)
+        step(dq_in["q"], dq_in["k"], dq_in["v"], dq_in["do"])
+        host_out["out"].copy_(out, non_blocking=True)
+        host_out["dq"].copy_(dq, non_blocking=True)
+        host_out["dk"].copy_(dk, non_blocking=True)
+        host_out["dv"].copy_(dv, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = torch.tensor([e0.elapsed_time(e1) / e2e_steps], device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(e2e_ms, op=torch.distributed.ReduceOp.MAX)
+    e2e_val = tokens_all / (float(e2e_ms.item()) / 1e3)
+
+    # ---- roofline of the dominant kernel and of the whole step ------------------------
+    launches = sum(c for _, c in prof.values())
+    top = max(prof.items(), key=lambda kv: kv[1][0]) if prof else None
+    roof = None
+    if top:
+        name, (tot_ms, cnt) = top
+        per_launch_s = tot_ms / cnt / 1e3
+        work = kernel_work(name, w)
+        units = B * H * N
+        share = tot_ms / sum(t for t, _ in prof.values())
+        if work:
+            byts, flops = work[0] * units, work[1] * units
+            if is_tensor_core_kernel(name):
+                peak_c = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+                t_c = flops / (peak_c * 1e12)
+            else:
+                peak_c = (torch.cuda.get_device_properties(dev).multi_processor_count
+                          * FP32_LANES_PER_SM * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12)
+                t_c = flops / (peak_c * 1e12)
+            t_m = byts / (peaks["hbm_gbs"] * 1e9)
+            if t_m >= t_c:
+                roof = {"bound": "hbm", "achieved": byts / per_launch_s / 1e9,
+                        "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+            else:
+                roof = {"bound": "tensor" if is_tensor_core_kernel(name) else "alu",
+                        "achieved": flops / per_launch_s / 1e12, "peak": peak_c, "unit": "TFLOP/s"}
+            roof["frac"] = roof["achieved"] / roof["peak"]
+            roof["traffic"] = None
+            roof.update({"kernel": name, "ms_per_launch": per_launch_s * 1e3,
+                         "share_of_step": share, "peak_source": peaks["source"]})
+    sb, sf = step_work(w)
+    t_step_roof = max(sb * B * H * N / (peaks["hbm_gbs"] * 1e9),
+                      sf * B * H * N / (peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * 1e12))
+    step_roof = {"bytes_per_token": sb, "flops_per_token": sf, "roofline_ms": t_step_roof * 1e3,
+                 "frac": t_step_roof * 1e3 / ms_max}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w)
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
+                "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+                           "L": w.L, "P": w.P, "tau": w.tau, "causal": w.causal,
+                           "dist": w.dist, "l2": "inputs larger than L2 (no flush)",
+                           "head_tokens_per_s": B * H * N * world / (ms_max / 1e3)},
+                "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                        "d2h_bytes_per_step": d2h},
+                "gpu_launches": launches,
+                "roofline": roof, "step_roofline": step_roof,
+                "kernels": {n: {"ms_total": t, "launches": c} for n, (t, c) in prof.items()},
+                "clocks": clk, "cpu_baseline": cpu}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="c3_causal_n4m_clusters",
+                    choices=sorted(race_inputs.WORKLOADS))
+    ap.add_argument("--n", type=int, default=0, help="override the sequence length")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    w = race_inputs.WORKLOADS[args.workload]
+    if args.n:
+        w = w.with_n(args.n)
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_ours(args, w)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,152 @@
+/*
+ * race_attn.h -- C ABI of the RACE Attention library for NVIDIA B200 (sm_100a).
+ *
+ * RACE Attention ("RACE Attention: A Strictly Linear-Time Attention for Long-Sequence
+ * Training", arXiv 2510.04008; sections cited below are those of its gist.science
+ * summaries: zh = Chinese page, es = Spanish page) replaces softmax attention by a
+ * sketch of the sharpened angular kernel (1 - arccos(q.k / |q||k|)/pi)^P (es §2.1,
+ * zh §2.1).  Per head, with x^ = x/|x|, L tables of P Gaussian hyperplanes W[L,P,d],
+ * u_l = tanh(W_l x^) and R = 2^P hypercube corners (zh §2.2):
+ *
+ *     phi_l(x)[r] = softmax_r( beta * c_r . u_l ),  c_rp = +1 if bit p of r is set else -1,
+ *     Y_i   = sum_l sum_{j in M(i)} (phi_l(q_i) . phi_l(k_j)) [v_j, 1],
+ *     out_i = Y_i[0:d] / Y_i[d],   den_i = Y_i[d],
+ *
+ * with M(i) = every key (Algorithm 1, zh §2.2) or keys j <= i (Algorithm 2, causal
+ * streaming statistics, zh §2.3).  beta = 1/tau; tau = 0 selects hard sign hashing
+ * (phi_l one-hot at r* = sum_p [W_lp . x > 0] 2^p).
+ *
+ * Conventions shared by every entry point
+ *   - Layout: q, k, v, out, dout, dq, dk, dv are [B, H, N, d] row-major (d fastest),
+ *     contiguous; den is [B, H, N]; W is [L, P, d] fp32 and is shared by every (b, h).
+ *   - Every pointer named "device" must point to memory of the current CUDA device,
+ *     16-byte aligned.  The caller owns all buffers, workspaces included; the library
+ *     allocates no memory and keeps no state between calls.
+ *   - Execution is asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream).  Nothing synchronises the host.
+ *   - Arguments are validated before anything is launched; a rejected call launches
+ *     nothing and returns RACE_ERR_INVALID_ARG, RACE_ERR_UNSUPPORTED or
+ *     RACE_ERR_WORKSPACE.  A launch failure reported by the CUDA runtime returns
+ *     RACE_ERR_CUDA (the runtime's own error stays readable with cudaGetLastError()).
+ *   - Supported: B, H >= 1; N >= 0 (N = 0 is a no-op); d a multiple of 8 in [8, 128];
+ *     1 <= P <= 5; L >= 1 with L * 2^P <= 1024; tau >= 0 and finite; dtype RACE_F32 or
+ *     RACE_BF16 (arithmetic is fp32 either way, with fp32 accumulation).
+ */
+#ifndef RACE_ATTN_H
+#define RACE_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t, declared here so the header needs no CUDA include. */
+typedef struct CUstream_st *race_stream_t;
+
+typedef enum {
+    RACE_OK = 0,
+    RACE_ERR_INVALID_ARG = 1, /* null pointer, negative size, misaligned pointer, bad tau */
+    RACE_ERR_UNSUPPORTED = 2, /* valid but outside the supported set (d, P, L*2^P, tau=0 backward) */
+    RACE_ERR_WORKSPACE = 3,   /* workspace or ctx buffer smaller than the size query says */
+    RACE_ERR_CUDA = 4         /* the CUDA runtime reported an error while launching */
+} race_status_t;
+
+typedef enum { RACE_F32 = 0, RACE_BF16 = 1 } race_dtype_t;
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char *race_status_string(race_status_t status);
+
+/*
+ * Device workspace, in bytes, that race_attn_forward (backward = 0) or
+ * race_attn_backward (backward = 1) needs for these sizes, written to *bytes.
+ * The workspace holds the per-segment bucket statistics of the chunked scan
+ * (fp32, L*2^P x (d+1) per segment and head); it is scratch: its contents on entry
+ * are ignored and on exit are unspecified.
+ */
+race_status_t race_attn_workspace_size(int B, int H, int64_t N, int d, int L, int P, int causal,
+                                       int backward, race_dtype_t dtype, size_t *bytes);
+
+/*
+ * Size, in bytes, of the optional saved-state buffer `ctx` (fp32 device memory).
+ * race_attn_forward can leave in it the key-side bucket statistics of every sequence
+ * segment (the running sums A_cum, B_cum of Algorithm 2, zh §2.3, at each segment
+ * start; for the bidirectional form, the totals A, B of Algorithm 1); handing the same
+ * buffer to race_attn_backward with the same q, k, v, W and sizes saves the backward
+ * pass one read of k and v.
+ */
+race_status_t race_attn_ctx_size(int B, int H, int64_t N, int d, int L, int P, int causal,
+                                 size_t *bytes);
+
+/*
+ * Forward pass (Algorithm 1 when causal = 0, Algorithm 2 when causal = 1; zh §2.2-2.3).
+ *   q, k, v    device, [B,H,N,d] of `dtype`, read only.  q and k need not be normalised:
+ *              rows are scaled to unit norm inside (|x| floored at 1e-12).
+ *   W          device, [L,P,d] fp32, read only: the Gaussian hyperplanes.
+ *   out        device, [B,H,N,d] of `dtype`, written.
+ *   den        device, [B,H,N] fp32, written: the denominator Y_i[d] (needed by the
+ *              backward pass); may be NULL.  Hard hashing can leave a query with no key
+ *              in any of its buckets: then den_i = 0 and out_i = 0.
+ *   ctx        device or NULL; if not NULL, ctx_bytes >= race_attn_ctx_size(...) and the
+ *              saved state is written there.
+ *   tau        temperature; beta = 1/tau scales the corner logits; tau = 0 = hard hash.
+ *   workspace  device, workspace_bytes >= race_attn_workspace_size(..., backward = 0).
+ */
+race_status_t race_attn_forward(const void *q, const void *k, const void *v, const float *W,
+                                void *out, float *den, float *ctx, size_t ctx_bytes, int B,
+                                int H, int64_t N, int d, int L, int P, float tau, int causal,
+                                race_dtype_t dtype, void *workspace, size_t workspace_bytes,
+                                race_stream_t stream);
+
+/*
+ * Backward pass: gradients of sum(out * dout) with respect to q, k and v, by the chain
+ * rule through the forward above (the pages state the method is differentiable end to
+ * end, es §2.3; they print no gradient formula).  W gets no gradient: it is a fixed
+ * random projection (zh §2.2).
+ *   q, k, v, W, out, den   the forward's inputs and outputs (den must not be NULL).
+ *   dout       device, [B,H,N,d] of `dtype`.
+ *   ctx        NULL, or the buffer a forward call with the same arguments filled.
+ *   dq, dk, dv device, [B,H,N,d] of `dtype`, overwritten.
+ *   tau        must be > 0 (hard hashing has no gradient: RACE_ERR_UNSUPPORTED).
+ *   workspace  device, workspace_bytes >= race_attn_workspace_size(..., backward = 1).
+ */
+race_status_t race_attn_backward(const void *q, const void *k, const void *v, const float *W,
+                                 const void *out, const float *den, const void *dout,
+                                 const float *ctx, size_t ctx_bytes, void *dq, void *dk,
+                                 void *dv, int B, int H, int64_t N, int d, int L, int P,
+                                 float tau, int causal, race_dtype_t dtype, void *workspace,
+                                 size_t workspace_bytes, race_stream_t stream);
+
+/*
+ * Hard sign-hash bucket of every row in every table (the one-hot assignment the soft
+ * hash tends to as beta grows; es §2.3 contrasts the two):
+ *   idx[b,h,n,l] = sum_p [W[l,p,:] . x[b,h,n,:] > 0] * 2^p,   int32, device, written.
+ *   x          device, [B,H,N,d] of `dtype`.
+ */
+race_status_t race_attn_hash_indices(const void *x, const float *W, int32_t *idx, int B, int H,
+                                     int64_t N, int d, int L, int P, race_dtype_t dtype,
+                                     race_stream_t stream);
+
+/*
+ * Opt-in kernel timing (a measurement aid; the method has no counterpart).  While enabled,
+ * every kernel the library launches is bracketed by a pair of CUDA events recorded on the
+ * launch stream; race_attn_profile_read waits for the recorded events, adds each
+ * kernel's elapsed time to its running total and reports the totals.  Off by default;
+ * costs two event records per launch when on.  Not thread-safe.
+ */
+void race_attn_profile_enable(int on);
+void race_attn_profile_reset(void);
+/*
+ * Writes up to max_kernels entries: names[i] (NUL-terminated, at most 63 chars, in a
+ * caller buffer of max_kernels * 64 chars), total milliseconds ms[i] and launch counts
+ * launches[i]; returns the number of distinct kernels seen (may exceed max_kernels), or
+ * -1 if a recorded event reports an error.
+ */
+int race_attn_profile_read(char *names, float *ms, int64_t *launches, int max_kernels);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RACE_ATTN_H */

@@ -1,0 +1,228 @@
+"""RACE Attention for NVIDIA B200: Python binding of the C ABI in ``include/race_attn.h``.
+
+Argument marshalling only: each function below passes torch tensors' device pointers, the
+sizes read from their shapes and the current CUDA stream to the entry point of the same
+name in ``librace_attn.so``.  Every step of the computation runs in that library's
+kernels.  There is no CPU fallback: if the library is missing, importing the functions
+works but the first call raises.
+
+Method: "RACE Attention: A Strictly Linear-Time Attention for Long-Sequence Training"
+(zh §2.2 Algorithm 1, zh §2.3 Algorithm 2).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+__all__ = [
+    "RACE_OK", "RACE_ERR_INVALID_ARG", "RACE_ERR_UNSUPPORTED", "RACE_ERR_WORKSPACE",
+    "RACE_ERR_CUDA", "RACE_F32", "RACE_BF16", "RaceError", "library_path", "load_library",
+    "race_status_string", "race_attn_workspace_size", "race_attn_ctx_size",
+    "race_attn_forward", "race_attn_backward", "race_attn_hash_indices",
+    "forward", "backward", "race_attn_profile_enable", "race_attn_profile_reset",
+    "race_attn_profile_read",
+]
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_NAME = "librace_attn.so"
+
+RACE_OK, RACE_ERR_INVALID_ARG, RACE_ERR_UNSUPPORTED, RACE_ERR_WORKSPACE, RACE_ERR_CUDA = range(5)
+RACE_F32, RACE_BF16 = 0, 1
+
+_vp = ctypes.c_void_p
+_i64 = ctypes.c_int64
+_int = ctypes.c_int
+_sz = ctypes.c_size_t
+_lib = None
+
+
+class RaceError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__("%s failed: %s" % (what, race_status_string(status)))
+
+
+def library_path() -> str:
+    return os.path.join(HERE, _LIB_NAME)
+
+
+def load_library():
+    """Load ``librace_attn.so`` (built in place by ``build.py``); raise if it is absent."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = library_path()
+    if not os.path.exists(path):
+        raise RuntimeError("%s is not built; run `python linear_attention_soft_b200/build.py`"
+                           % path)
+    lib = ctypes.CDLL(path)
+    lib.race_status_string.argtypes = [_int]
+    lib.race_status_string.restype = ctypes.c_char_p
+    lib.race_attn_workspace_size.argtypes = [_int, _int, _i64, _int, _int, _int, _int, _int, _int,
+                                             ctypes.POINTER(_sz)]
+    lib.race_attn_workspace_size.restype = _int
+    lib.race_attn_ctx_size.argtypes = [_int, _int, _i64, _int, _int, _int, _int,
+                                       ctypes.POINTER(_sz)]
+    lib.race_attn_ctx_size.restype = _int
+    lib.race_attn_forward.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _int, _int, _i64,
+                                      _int, _int, _int, ctypes.c_float, _int, _int, _vp, _sz, _vp]
+    lib.race_attn_forward.restype = _int
+    lib.race_attn_backward.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp, _vp,
+                                       _int, _int, _i64, _int, _int, _int, ctypes.c_float, _int,
+                                       _int, _vp, _sz, _vp]
+    lib.race_attn_backward.restype = _int
+    lib.race_attn_hash_indices.argtypes = [_vp, _vp, _vp, _int, _int, _i64, _int, _int, _int, _int,
+                                           _vp]
+    lib.race_attn_hash_indices.restype = _int
+    lib.race_attn_profile_enable.argtypes = [_int]
+    lib.race_attn_profile_enable.restype = None
+    lib.race_attn_profile_reset.argtypes = []
+    lib.race_attn_profile_reset.restype = None
+    lib.race_attn_profile_read.argtypes = [ctypes.c_char_p, ctypes.POINTER(ctypes.c_float),
+                                           ctypes.POINTER(_i64), _int]
+    lib.race_attn_profile_read.restype = _int
+    _lib = lib
+    return lib
+
+
+def race_status_string(status: int) -> str:
+    return load_library().race_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str):
+    if status != RACE_OK:
+        raise RaceError(status, what)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return RACE_F32
+    if t.dtype == torch.bfloat16:
+        return RACE_BF16
+    raise TypeError("RACE attention takes float32 or bfloat16 tensors, got %s" % t.dtype)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return t.data_ptr()
+
+
+def _nbytes(t: Optional[torch.Tensor]) -> int:
+    return 0 if t is None else t.numel() * t.element_size()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _dims(q: torch.Tensor, W: torch.Tensor) -> Tuple[int, int, int, int, int, int]:
+    B, H, N, d = q.shape
+    L, P, dw = W.shape
+    if dw != d:
+        raise ValueError("W is [L, P, d] with the d of q")
+    return B, H, N, d, L, P
+
+
+def race_attn_workspace_size(B, H, N, d, L, P, causal, backward, dtype) -> int:
+    out = _sz()
+    _check(load_library().race_attn_workspace_size(B, H, N, d, L, P, int(causal), int(backward),
+                                                   int(dtype), ctypes.byref(out)),
+           "race_attn_workspace_size")
+    return out.value
+
+
+def race_attn_ctx_size(B, H, N, d, L, P, causal) -> int:
+    out = _sz()
+    _check(load_library().race_attn_ctx_size(B, H, N, d, L, P, int(causal), ctypes.byref(out)),
+           "race_attn_ctx_size")
+    return out.value
+
+
+def race_attn_forward(q, k, v, W, out, den, ctx, tau: float, causal: bool, workspace,
+                      stream=None) -> None:
+    """C ABI forward on torch tensors ([B,H,N,d] q/k/v/out, [B,H,N] fp32 den, [L,P,d] W)."""
+    B, H, N, d, L, P = _dims(q, W)
+    _check(load_library().race_attn_forward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(W), _ptr(out), _ptr(den), _ptr(ctx), _nbytes(ctx),
+        B, H, N, d, L, P, float(tau), int(bool(causal)), _dtype_code(q), _ptr(workspace),
+        _nbytes(workspace), _stream(stream)), "race_attn_forward")
+
+
+def race_attn_backward(q, k, v, W, out, den, dout, ctx, dq, dk, dv, tau: float, causal: bool,
+                       workspace, stream=None) -> None:
+    """C ABI backward on torch tensors; dq/dk/dv are overwritten."""
+    B, H, N, d, L, P = _dims(q, W)
+    _check(load_library().race_attn_backward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(W), _ptr(out), _ptr(den), _ptr(dout), _ptr(ctx),
+        _nbytes(ctx), _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, L, P, float(tau),
+        int(bool(causal)), _dtype_code(q), _ptr(workspace), _nbytes(workspace), _stream(stream)),
+        "race_attn_backward")
+
+
+def race_attn_hash_indices(x, W, idx, stream=None) -> None:
+    """C ABI hard sign-hash indices: idx is [B,H,N,L] int32."""
+    B, H, N, d, L, P = _dims(x, W)
+    _check(load_library().race_attn_hash_indices(
+        _ptr(x), _ptr(W), _ptr(idx), B, H, N, d, L, P, _dtype_code(x), _stream(stream)),
+        "race_attn_hash_indices")
+
+
+def race_attn_profile_enable(on: bool) -> None:
+    load_library().race_attn_profile_enable(int(bool(on)))
+
+
+def race_attn_profile_reset() -> None:
+    load_library().race_attn_profile_reset()
+
+
+def race_attn_profile_read(max_kernels: int = 32):
+    """{kernel name: (total ms, launches)} accumulated since the last reset."""
+    names = ctypes.create_string_buffer(64 * max_kernels)
+    ms = (ctypes.c_float * max_kernels)()
+    cnt = (_i64 * max_kernels)()
+    n = load_library().race_attn_profile_read(names, ms, cnt, max_kernels)
+    if n < 0:
+        raise RuntimeError("race_attn_profile_read: a recorded event reported an error")
+    out = {}
+    for i in range(min(n, max_kernels)):
+        nm = names.raw[64 * i: 64 * i + 64].split(b"\0", 1)[0].decode()
+        out[nm] = (float(ms[i]), int(cnt[i]))
+    return out
+
+
+# ---- conveniences that allocate with torch (device memory is plumbing) ---------------
+
+def _workspace(q, W, causal, backward) -> torch.Tensor:
+    B, H, N, d, L, P = _dims(q, W)
+    n = race_attn_workspace_size(B, H, N, d, L, P, causal, backward, _dtype_code(q))
+    return torch.empty(max(n, 16), dtype=torch.uint8, device=q.device)
+
+
+def forward(q, k, v, W, tau: float, causal: bool, save_ctx: bool = False, stream=None):
+    """Allocate and run the forward: returns (out, den, ctx or None)."""
+    B, H, N, d, L, P = _dims(q, W)
+    out = torch.empty_like(q)
+    den = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    ctx = None
+    if save_ctx:
+        ctx = torch.empty(race_attn_ctx_size(B, H, N, d, L, P, causal) // 4, dtype=torch.float32,
+                          device=q.device)
+    race_attn_forward(q, k, v, W, out, den, ctx, tau, causal, _workspace(q, W, causal, False),
+                      stream)
+    return out, den, ctx
+
+
+def backward(q, k, v, W, out, den, dout, tau: float, causal: bool, ctx=None, stream=None):
+    """Allocate and run the backward: returns (dq, dk, dv)."""
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    race_attn_backward(q, k, v, W, out, den, dout, ctx, dq, dk, dv, tau, causal,
+                       _workspace(q, W, causal, True), stream)
+    return dq, dk, dv

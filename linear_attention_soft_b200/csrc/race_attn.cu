@@ -1,0 +1,446 @@
+// race_attn.cu -- C ABI of the RACE Attention library: argument checks, work planning and
+// kernel launches on the caller's stream.  Declarations and argument contracts are in
+// include/race_attn.h.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "race_attn.h"
+#include "race_generic.cuh"
+#include "race_tc.cuh"
+
+namespace {
+
+// ---- opt-in kernel timing -------------------------------------------------------------
+struct ProfEntry {
+    std::string name;
+    double ms;
+    int64_t launches;
+};
+struct ProfPending {
+    int entry;
+    cudaEvent_t a, b;
+};
+bool g_prof_on = false;
+std::vector<ProfEntry> g_prof;
+std::vector<ProfPending> g_pending;
+std::vector<cudaEvent_t> g_event_pool;
+
+cudaEvent_t prof_event()
+{
+    if (!g_event_pool.empty()) {
+        cudaEvent_t e = g_event_pool.back();
+        g_event_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+}
+
+int prof_entry(const char *name)
+{
+    for (size_t i = 0; i < g_prof.size(); ++i)
+        if (g_prof[i].name == name) return (int)i;
+    g_prof.push_back({name, 0.0, 0});
+    return (int)g_prof.size() - 1;
+}
+
+// Run `fn` (which launches one kernel on st) between two recorded events when enabled.
+template <typename Fn>
+cudaError_t timed(const char *name, cudaStream_t st, Fn fn)
+{
+    if (!g_prof_on) return fn();
+    ProfPending p{prof_entry(name), prof_event(), prof_event()};
+    if (p.a) cudaEventRecord(p.a, st);
+    cudaError_t e = fn();
+    if (p.b) cudaEventRecord(p.b, st);
+    if (p.a && p.b)
+        g_pending.push_back(p);
+    g_prof[p.entry].launches += 1;
+    return e;
+}
+
+using race::generic::Args;
+namespace gk = race::generic;
+
+constexpr int64_t kSegAlign = 128;     // segment lengths are multiples of this many tokens
+constexpr int64_t kMinSegTokens = 512;  // no segment shorter than this (unless N is)
+
+struct Plan {
+    int BH;
+    int64_t N;
+    int d, L, P, R, M, D, G;
+    int64_t seg_len;
+    int nseg;
+    size_t state_elems;  // one [BH][nseg][M][D] fp32 state buffer
+};
+
+int device_sm_count()
+{
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+        cudaGetLastError();  // no device here: plan for a full B200
+        return 148;
+    }
+    return n;
+}
+
+race_status_t check_sizes(int B, int H, int64_t N, int d, int L, int P)
+{
+    if (B < 1 || H < 1 || N < 0 || d < 1 || L < 1 || P < 1) return RACE_ERR_INVALID_ARG;
+    if ((int64_t)B * H > 65535) return RACE_ERR_UNSUPPORTED;
+    if (d % 8 != 0 || d > 128) return RACE_ERR_UNSUPPORTED;
+    if (P > 5) return RACE_ERR_UNSUPPORTED;
+    if ((int64_t)L << P > (int64_t)gk::MG * gk::MAXG) return RACE_ERR_UNSUPPORTED;
+    return RACE_OK;
+}
+
+Plan make_plan(int B, int H, int64_t N, int d, int L, int P)
+{
+    Plan p;
+    p.BH = B * H;
+    p.N = N;
+    p.d = d;
+    p.L = L;
+    p.P = P;
+    p.R = 1 << P;
+    p.M = L * p.R;
+    p.D = d + 1;
+    p.G = (p.M + gk::MG - 1) / gk::MG;
+    // Segments per sequence: about two CTAs per SM over all heads, none shorter than
+    // kMinSegTokens, lengths a multiple of kSegAlign.
+    const int64_t target = 2 * (int64_t)device_sm_count();
+    int64_t nseg = (target + p.BH - 1) / p.BH;
+    const int64_t maxseg = (N + kMinSegTokens - 1) / kMinSegTokens;
+    if (nseg > maxseg) nseg = maxseg;
+    if (nseg < 1) nseg = 1;
+    int64_t len = (N + nseg - 1) / nseg;
+    len = (len + kSegAlign - 1) / kSegAlign * kSegAlign;
+    if (len < kSegAlign) len = kSegAlign;
+    p.seg_len = len;
+    p.nseg = (int)((N + len - 1) / len);
+    if (p.nseg < 1) p.nseg = 1;
+    p.state_elems = (size_t)p.BH * p.nseg * p.M * p.D;
+    return p;
+}
+
+bool aligned16(const void *ptr) { return ((uintptr_t)ptr & 15u) == 0; }
+
+Args base_args(const Plan &p, const float *W, float tau)
+{
+    Args a;
+    std::memset(&a, 0, sizeof(a));
+    a.W = W;
+    a.N = p.N;
+    a.d = p.d;
+    a.L = p.L;
+    a.P = p.P;
+    a.M = p.M;
+    a.G = p.G;
+    a.hard = tau == 0.f;
+    a.beta = a.hard ? 0.f : 1.f / tau;
+    a.seg_len = p.seg_len;
+    a.nseg = p.nseg;
+    return a;
+}
+
+template <typename Kern>
+cudaError_t launch(Kern kernel, dim3 grid, int cluster_x, size_t smem, cudaStream_t st,
+                   const Args &a)
+{
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(gk::NT);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cluster_x;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, a);
+}
+
+cudaError_t launch_scan(float *buf, const Plan &p, int mode, cudaStream_t st)
+{
+    const int64_t MD = (int64_t)p.M * p.D;
+    dim3 grid((unsigned)((MD + gk::NT - 1) / gk::NT), (unsigned)p.BH);
+    return timed("segment_scan", st, [&] {
+        gk::race_scan<<<grid, gk::NT, 0, st>>>(buf, p.nseg, MD, mode);
+        return cudaGetLastError();
+    });
+}
+
+// ---- the general path (every shape and dtype) ----------------------------------------
+
+template <typename DT, int T>
+cudaError_t generic_forward(const Plan &p, Args a, float *states, int causal, cudaStream_t st)
+{
+    const size_t smem = gk::Smem(T, p.d, p.P).total * sizeof(float);
+    const dim3 grid((unsigned)p.G, (unsigned)p.nseg, (unsigned)p.BH);
+    a.causal = causal;
+    a.agg_out = states;
+    cudaError_t e = timed("generic_agg_kv", st, [&] {
+        return launch(gk::race_agg<DT, T, gk::AGG_KV>, grid, 1, smem, st, a);
+    });
+    if (e != cudaSuccess) return e;
+    e = launch_scan(states, p, causal ? gk::SCAN_EXCL_PREFIX : gk::SCAN_TOTAL, st);
+    if (e != cudaSuccess) return e;
+    a.state = states;
+    a.state_seg_stride = causal ? (int64_t)p.M * p.D : 0;
+    return timed("generic_fwd_walk", st,
+                 [&] { return launch(gk::race_fwd_walk<DT, T>, grid, p.G, smem, st, a); });
+}
+
+template <typename DT, int T>
+cudaError_t generic_backward(const Plan &p, Args a, const float *hstates, bool have_ctx,
+                             float *hbuf, float *gbuf, int causal, cudaStream_t st)
+{
+    const size_t smem = gk::Smem(T, p.d, p.P).total * sizeof(float);
+    const dim3 grid((unsigned)p.G, (unsigned)p.nseg, (unsigned)p.BH);
+    a.causal = causal;
+    cudaError_t e;
+    if (!have_ctx) {
+        a.agg_out = hbuf;
+        e = timed("generic_agg_kv", st, [&] {
+            return launch(gk::race_agg<DT, T, gk::AGG_KV>, grid, 1, smem, st, a);
+        });
+        if (e != cudaSuccess) return e;
+        e = launch_scan(hbuf, p, causal ? gk::SCAN_EXCL_PREFIX : gk::SCAN_TOTAL, st);
+        if (e != cudaSuccess) return e;
+        hstates = hbuf;
+    }
+    a.state = hstates;
+    a.state_seg_stride = causal ? (int64_t)p.M * p.D : 0;
+    e = timed("generic_bwd_q_walk", st,
+              [&] { return launch(gk::race_bwd_q_walk<DT, T>, grid, p.G, smem, st, a); });
+    if (e != cudaSuccess) return e;
+    a.agg_out = gbuf;
+    e = timed("generic_agg_qdy", st, [&] {
+        return launch(gk::race_agg<DT, T, gk::AGG_QDY>, grid, 1, smem, st, a);
+    });
+    if (e != cudaSuccess) return e;
+    e = launch_scan(gbuf, p, causal ? gk::SCAN_EXCL_SUFFIX : gk::SCAN_TOTAL, st);
+    if (e != cudaSuccess) return e;
+    a.state = gbuf;
+    return timed("generic_bwd_kv_walk", st,
+                 [&] { return launch(gk::race_bwd_kv_walk<DT, T>, grid, p.G, smem, st, a); });
+}
+
+template <typename DT>
+cudaError_t dispatch_forward(const Plan &p, const Args &a, float *states, int causal,
+                             cudaStream_t st)
+{
+    if (p.d <= 64) return generic_forward<DT, 32>(p, a, states, causal, st);
+    return generic_forward<DT, 16>(p, a, states, causal, st);
+}
+
+template <typename DT>
+cudaError_t dispatch_backward(const Plan &p, const Args &a, const float *ctx, float *hbuf,
+                              float *gbuf, int causal, cudaStream_t st)
+{
+    if (p.d <= 64) return generic_backward<DT, 32>(p, a, ctx, ctx != nullptr, hbuf, gbuf, causal, st);
+    return generic_backward<DT, 16>(p, a, ctx, ctx != nullptr, hbuf, gbuf, causal, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *race_status_string(race_status_t s)
+{
+    switch (s) {
+    case RACE_OK: return "RACE_OK";
+    case RACE_ERR_INVALID_ARG: return "RACE_ERR_INVALID_ARG";
+    case RACE_ERR_UNSUPPORTED: return "RACE_ERR_UNSUPPORTED";
+    case RACE_ERR_WORKSPACE: return "RACE_ERR_WORKSPACE";
+    case RACE_ERR_CUDA: return "RACE_ERR_CUDA";
+    }
+    return "RACE_ERR_UNKNOWN";
+}
+
+race_status_t race_attn_workspace_size(int B, int H, int64_t N, int d, int L, int P, int causal,
+                                       int backward, race_dtype_t dtype, size_t *bytes)
+{
+    (void)causal;
+    if (!bytes) return RACE_ERR_INVALID_ARG;
+    if (dtype != RACE_F32 && dtype != RACE_BF16) return RACE_ERR_INVALID_ARG;
+    race_status_t s = check_sizes(B, H, N, d, L, P);
+    if (s != RACE_OK) return s;
+    const Plan p = make_plan(B, H, N, d, L, P);
+    *bytes = p.state_elems * sizeof(float) * (backward ? 2 : 1);
+    return RACE_OK;
+}
+
+race_status_t race_attn_ctx_size(int B, int H, int64_t N, int d, int L, int P, int causal,
+                                 size_t *bytes)
+{
+    (void)causal;
+    if (!bytes) return RACE_ERR_INVALID_ARG;
+    race_status_t s = check_sizes(B, H, N, d, L, P);
+    if (s != RACE_OK) return s;
+    *bytes = make_plan(B, H, N, d, L, P).state_elems * sizeof(float);
+    return RACE_OK;
+}
+
+race_status_t race_attn_forward(const void *q, const void *k, const void *v, const float *W,
+                                void *out, float *den, float *ctx, size_t ctx_bytes, int B,
+                                int H, int64_t N, int d, int L, int P, float tau, int causal,
+                                race_dtype_t dtype, void *workspace, size_t workspace_bytes,
+                                race_stream_t stream)
+{
+    if (dtype != RACE_F32 && dtype != RACE_BF16) return RACE_ERR_INVALID_ARG;
+    if (!(tau >= 0.f) || !std::isfinite(tau)) return RACE_ERR_INVALID_ARG;
+    race_status_t s = check_sizes(B, H, N, d, L, P);
+    if (s != RACE_OK) return s;
+    if (N == 0) return RACE_OK;
+    if (!q || !k || !v || !W || !out || !workspace) return RACE_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(W) || !aligned16(out) ||
+        !aligned16(workspace) || (den && !aligned16(den)) || (ctx && !aligned16(ctx)))
+        return RACE_ERR_INVALID_ARG;
+    const Plan p = make_plan(B, H, N, d, L, P);
+    const size_t need = p.state_elems * sizeof(float);
+    if (workspace_bytes < need) return RACE_ERR_WORKSPACE;
+    if (ctx && ctx_bytes < need) return RACE_ERR_WORKSPACE;
+    Args a = base_args(p, W, tau);
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.out = out;
+    a.den_out = den;
+    float *states = ctx ? ctx : (float *)workspace;
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e;
+    if (race::tc::fast_path_ok(dtype, d, L, P, tau))
+        e = race::tc::forward(q, k, v, W, out, den, states, B * H, N, p.seg_len, p.nseg, tau,
+                              causal, st);
+    else if (dtype == RACE_F32)
+        e = dispatch_forward<float>(p, a, states, causal, st);
+    else
+        e = dispatch_forward<__nv_bfloat16>(p, a, states, causal, st);
+    return e == cudaSuccess ? RACE_OK : RACE_ERR_CUDA;
+}
+
+race_status_t race_attn_backward(const void *q, const void *k, const void *v, const float *W,
+                                 const void *out, const float *den, const void *dout,
+                                 const float *ctx, size_t ctx_bytes, void *dq, void *dk,
+                                 void *dv, int B, int H, int64_t N, int d, int L, int P,
+                                 float tau, int causal, race_dtype_t dtype, void *workspace,
+                                 size_t workspace_bytes, race_stream_t stream)
+{
+    if (dtype != RACE_F32 && dtype != RACE_BF16) return RACE_ERR_INVALID_ARG;
+    if (!(tau >= 0.f) || !std::isfinite(tau)) return RACE_ERR_INVALID_ARG;
+    race_status_t s = check_sizes(B, H, N, d, L, P);
+    if (s != RACE_OK) return s;
+    if (tau == 0.f) return RACE_ERR_UNSUPPORTED;
+    if (N == 0) return RACE_OK;
+    if (!q || !k || !v || !W || !out || !den || !dout || !dq || !dk || !dv || !workspace)
+        return RACE_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, W, out, den, dout, dq, dk, dv, workspace};
+    for (const void *ptr : ptrs)
+        if (!aligned16(ptr)) return RACE_ERR_INVALID_ARG;
+    if (ctx && !aligned16(ctx)) return RACE_ERR_INVALID_ARG;
+    const Plan p = make_plan(B, H, N, d, L, P);
+    const size_t one = p.state_elems * sizeof(float);
+    if (workspace_bytes < 2 * one) return RACE_ERR_WORKSPACE;
+    if (ctx && ctx_bytes < one) return RACE_ERR_WORKSPACE;
+    Args a = base_args(p, W, tau);
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.o = out;
+    a.den_in = den;
+    a.dout = dout;
+    a.dq = dq;
+    a.dk = dk;
+    a.dv = dv;
+    float *hbuf = (float *)workspace;
+    float *gbuf = hbuf + p.state_elems;
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e;
+    if (race::tc::fast_path_ok(dtype, d, L, P, tau))
+        e = race::tc::backward(q, k, v, W, out, den, dout, ctx, hbuf, gbuf, dq, dk, dv, B * H, N,
+                               p.seg_len, p.nseg, tau, causal, st);
+    else if (dtype == RACE_F32)
+        e = dispatch_backward<float>(p, a, ctx, hbuf, gbuf, causal, st);
+    else
+        e = dispatch_backward<__nv_bfloat16>(p, a, ctx, hbuf, gbuf, causal, st);
+    return e == cudaSuccess ? RACE_OK : RACE_ERR_CUDA;
+}
+
+race_status_t race_attn_hash_indices(const void *x, const float *W, int32_t *idx, int B, int H,
+                                     int64_t N, int d, int L, int P, race_dtype_t dtype,
+                                     race_stream_t stream)
+{
+    if (dtype != RACE_F32 && dtype != RACE_BF16) return RACE_ERR_INVALID_ARG;
+    if (B < 1 || H < 1 || N < 0 || d < 1 || L < 1 || P < 1) return RACE_ERR_INVALID_ARG;
+    if (d % 8 != 0 || d > 128 || P > 5) return RACE_ERR_UNSUPPORTED;
+    if (N == 0) return RACE_OK;
+    if (!x || !W || !idx) return RACE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(W) || !aligned16(idx)) return RACE_ERR_INVALID_ARG;
+    const int64_t rows = (int64_t)B * H * N;
+    const int64_t n = rows * L;
+    const unsigned blocks = (unsigned)((n + gk::NT - 1) / gk::NT);
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e = timed("hash_indices", st, [&] {
+        if (dtype == RACE_F32)
+            gk::race_hash<float><<<blocks, gk::NT, 0, st>>>((const float *)x, W, idx, rows, d, L, P);
+        else
+            gk::race_hash<__nv_bfloat16>
+                <<<blocks, gk::NT, 0, st>>>((const __nv_bfloat16 *)x, W, idx, rows, d, L, P);
+        return cudaGetLastError();
+    });
+    return e == cudaSuccess ? RACE_OK : RACE_ERR_CUDA;
+}
+
+void race_attn_profile_enable(int on) { g_prof_on = on != 0; }
+
+void race_attn_profile_reset(void)
+{
+    for (auto &p : g_pending) {
+        cudaEventSynchronize(p.b);
+        g_event_pool.push_back(p.a);
+        g_event_pool.push_back(p.b);
+    }
+    g_pending.clear();
+    g_prof.clear();
+}
+
+int race_attn_profile_read(char *names, float *ms, int64_t *launches, int max_kernels)
+{
+    int rc = 0;
+    for (auto &p : g_pending) {
+        float t = 0.f;
+        if (cudaEventSynchronize(p.b) != cudaSuccess || cudaEventElapsedTime(&t, p.a, p.b) != cudaSuccess)
+            rc = -1;
+        g_prof[p.entry].ms += t;
+        g_event_pool.push_back(p.a);
+        g_event_pool.push_back(p.b);
+    }
+    g_pending.clear();
+    if (rc) return rc;
+    const int n = (int)g_prof.size();
+    for (int i = 0; i < n && i < max_kernels; ++i) {
+        if (names) {
+            std::strncpy(names + 64 * i, g_prof[i].name.c_str(), 63);
+            names[64 * i + 63] = 0;
+        }
+        if (ms) ms[i] = (float)g_prof[i].ms;
+        if (launches) launches[i] = g_prof[i].launches;
+    }
+    return n;
+}
+
+}  // extern "C"

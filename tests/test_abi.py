@@ -1,0 +1,139 @@
+"""The C-ABI library loads, exports every entry point its header declares, and rejects bad
+arguments before touching the GPU (these calls launch nothing, so they run without one)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from linear_attention_soft_b200 import build
+    build.build()
+    import linear_attention_soft_b200 as ra
+    return ra.load_library()
+
+
+def declared_functions():
+    names = []
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if not h.endswith(".h"):
+            continue
+        src = open(os.path.join(ROOT, "include", h)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        names += re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*(race_[A-Za-z0-9_]+)\s*\(",
+                            src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("race_attn_forward", "race_attn_backward", "race_attn_hash_indices",
+              "race_attn_workspace_size", "race_attn_ctx_size", "race_status_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for n in declared_functions():
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(lib):
+    import linear_attention_soft_b200 as ra
+    assert ra.race_status_string(ra.RACE_OK) == "RACE_OK"
+    assert ra.race_status_string(ra.RACE_ERR_WORKSPACE) == "RACE_ERR_WORKSPACE"
+    assert ra.race_status_string(99) == "RACE_ERR_UNKNOWN"
+
+
+def test_workspace_queries(lib):
+    import linear_attention_soft_b200 as ra
+    fw = ra.race_attn_workspace_size(1, 1, 4096, 64, 16, 4, 1, 0, ra.RACE_BF16)
+    bw = ra.race_attn_workspace_size(1, 1, 4096, 64, 16, 4, 1, 1, ra.RACE_BF16)
+    cx = ra.race_attn_ctx_size(1, 1, 4096, 64, 16, 4, 1)
+    assert fw > 0 and bw == 2 * fw and cx == fw
+    # state is [segments][L*R][d+1] fp32 per head: a multiple of that size
+    assert fw % (256 * 65 * 4) == 0
+    with pytest.raises(ra.RaceError) as e:
+        ra.race_attn_workspace_size(1, 1, 4096, 60, 16, 4, 1, 0, ra.RACE_BF16)
+    assert e.value.status == ra.RACE_ERR_UNSUPPORTED
+    with pytest.raises(ra.RaceError) as e:
+        ra.race_attn_workspace_size(1, 1, 4096, 64, 16, 6, 1, 0, ra.RACE_BF16)
+    assert e.value.status == ra.RACE_ERR_UNSUPPORTED
+    with pytest.raises(ra.RaceError) as e:
+        ra.race_attn_workspace_size(1, 1, 4096, 64, 64, 5, 1, 0, ra.RACE_BF16)  # L*R = 2048
+    assert e.value.status == ra.RACE_ERR_UNSUPPORTED
+    with pytest.raises(ra.RaceError) as e:
+        ra.race_attn_workspace_size(0, 1, 4096, 64, 16, 4, 1, 0, ra.RACE_BF16)
+    assert e.value.status == ra.RACE_ERR_INVALID_ARG
+
+
+def _fwd(lib, **kw):
+    a = dict(q=16, k=16, v=16, W=16, out=16, den=16, ctx=None, ctx_bytes=0, B=1, H=1, N=256, d=64,
+             L=16, P=4, tau=0.5, causal=1, dtype=1, ws=16, ws_bytes=1 << 40, stream=None)
+    a.update(kw)
+    return lib.race_attn_forward(a["q"], a["k"], a["v"], a["W"], a["out"], a["den"], a["ctx"],
+                                 a["ctx_bytes"], a["B"], a["H"], a["N"], a["d"], a["L"], a["P"],
+                                 ctypes.c_float(a["tau"]), a["causal"], a["dtype"], a["ws"],
+                                 a["ws_bytes"], a["stream"])
+
+
+def _bwd(lib, **kw):
+    a = dict(q=16, k=16, v=16, W=16, out=16, den=16, dout=16, ctx=None, ctx_bytes=0, dq=16, dk=16,
+             dv=16, B=1, H=1, N=256, d=64, L=16, P=4, tau=0.5, causal=1, dtype=1, ws=16,
+             ws_bytes=1 << 40, stream=None)
+    a.update(kw)
+    return lib.race_attn_backward(a["q"], a["k"], a["v"], a["W"], a["out"], a["den"], a["dout"],
+                                  a["ctx"], a["ctx_bytes"], a["dq"], a["dk"], a["dv"], a["B"],
+                                  a["H"], a["N"], a["d"], a["L"], a["P"], ctypes.c_float(a["tau"]),
+                                  a["causal"], a["dtype"], a["ws"], a["ws_bytes"], a["stream"])
+
+
+def test_forward_rejects_bad_arguments_without_launching(lib):
+    import linear_attention_soft_b200 as ra
+    assert _fwd(lib, q=None) == ra.RACE_ERR_INVALID_ARG
+    assert _fwd(lib, out=None) == ra.RACE_ERR_INVALID_ARG
+    assert _fwd(lib, ws=None) == ra.RACE_ERR_INVALID_ARG
+    assert _fwd(lib, k=24) == ra.RACE_ERR_INVALID_ARG            # not 16-byte aligned
+    assert _fwd(lib, tau=-1.0) == ra.RACE_ERR_INVALID_ARG
+    assert _fwd(lib, tau=float("nan")) == ra.RACE_ERR_INVALID_ARG
+    assert _fwd(lib, tau=float("inf")) == ra.RACE_ERR_INVALID_ARG
+    assert _fwd(lib, dtype=7) == ra.RACE_ERR_INVALID_ARG
+    assert _fwd(lib, N=-1) == ra.RACE_ERR_INVALID_ARG
+    assert _fwd(lib, d=12) == ra.RACE_ERR_UNSUPPORTED
+    assert _fwd(lib, d=136) == ra.RACE_ERR_UNSUPPORTED
+    assert _fwd(lib, P=0) == ra.RACE_ERR_INVALID_ARG
+    assert _fwd(lib, P=6) == ra.RACE_ERR_UNSUPPORTED
+    assert _fwd(lib, ws_bytes=1024) == ra.RACE_ERR_WORKSPACE
+    assert _fwd(lib, ctx=16, ctx_bytes=1024) == ra.RACE_ERR_WORKSPACE
+    assert _fwd(lib, N=0, q=None) == ra.RACE_OK                  # empty input: nothing to do
+
+
+def test_backward_rejects_bad_arguments_without_launching(lib):
+    import linear_attention_soft_b200 as ra
+    assert _bwd(lib, tau=0.0) == ra.RACE_ERR_UNSUPPORTED        # hard hash has no gradient
+    assert _bwd(lib, den=None) == ra.RACE_ERR_INVALID_ARG
+    assert _bwd(lib, dv=None) == ra.RACE_ERR_INVALID_ARG
+    assert _bwd(lib, dq=8) == ra.RACE_ERR_INVALID_ARG
+    assert _bwd(lib, L=128, P=4) == ra.RACE_ERR_UNSUPPORTED     # L*R = 2048 > 1024
+    need = ra.race_attn_workspace_size(1, 1, 256, 64, 16, 4, 1, 1, ra.RACE_BF16)
+    assert _bwd(lib, ws_bytes=need - 1) == ra.RACE_ERR_WORKSPACE
+    assert _bwd(lib, N=0) == ra.RACE_OK
+
+
+def test_hash_indices_rejects_bad_arguments(lib):
+    import linear_attention_soft_b200 as ra
+    f = lib.race_attn_hash_indices
+    assert f(None, 16, 16, 1, 1, 8, 64, 4, 3, 1, None) == ra.RACE_ERR_INVALID_ARG
+    assert f(16, 16, 16, 1, 1, 8, 66, 4, 3, 1, None) == ra.RACE_ERR_UNSUPPORTED
+    assert f(16, 16, 16, 1, 1, 0, 64, 4, 3, 1, None) == ra.RACE_OK
+
+
+def test_product_path_has_no_cpu_fallback():
+    """The binding refuses to run without the CUDA library and never imports the oracle."""
+    src = open(os.path.join(ROOT, "linear_attention_soft_b200", "__init__.py")).read()
+    assert "oracle" not in src.replace("oracle.", "")
+    for f in os.listdir(os.path.join(ROOT, "linear_attention_soft_b200", "csrc")):
+        assert "oracle" not in open(os.path.join(ROOT, "linear_attention_soft_b200", "csrc", f)).read().lower()
