@@ -26,6 +26,7 @@ struct ProfPending {
     cudaEvent_t a, b;
 };
 bool g_prof_on = false;
+bool g_tc_forward = true;  // tensor-core forward for the shapes it covers
 std::vector<ProfEntry> g_prof;
 std::vector<ProfPending> g_pending;
 std::vector<cudaEvent_t> g_event_pool;
@@ -239,6 +240,48 @@ cudaError_t generic_backward(const Plan &p, Args a, const float *hstates, bool h
                  [&] { return launch(gk::race_bwd_kv_walk<DT, T>, grid, p.G, smem, st, a); });
 }
 
+// ---- the tensor-core path (bf16, d = 64, L = 16, P = 4) --------------------------------
+
+cudaError_t tc_forward(const Plan &p, const void *q, const void *k, const void *v, const float *W,
+                       void *out, float *den, float *states, float tau, int causal, cudaStream_t st)
+{
+    namespace tc = race::tc;
+    tc::Args a;
+    std::memset(&a, 0, sizeof(a));
+    a.q = (const __nv_bfloat16 *)q;
+    a.k = (const __nv_bfloat16 *)k;
+    a.v = (const __nv_bfloat16 *)v;
+    a.W = W;
+    a.out = (__nv_bfloat16 *)out;
+    a.den = den;
+    a.N = p.N;
+    a.seg_len = p.seg_len;
+    a.nseg = p.nseg;
+    a.beta = 1.f / tau;
+    a.causal = causal;
+    a.agg_out = states;
+    const dim3 grid((unsigned)p.nseg, (unsigned)p.BH);
+    const size_t sm_agg = tc::smem_bytes(tc::agg_smem::TOTAL);
+    const size_t sm_walk = tc::smem_bytes(tc::fwd_smem::TOTAL);
+    cudaError_t e = cudaFuncSetAttribute(tc::tc_agg_kv, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_agg);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(tc::tc_fwd_walk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_walk);
+    if (e != cudaSuccess) return e;
+    e = timed("tc_agg_kv", st, [&] {
+        tc::tc_agg_kv<<<grid, tc::NTH, sm_agg, st>>>(a);
+        return cudaGetLastError();
+    });
+    if (e != cudaSuccess) return e;
+    e = launch_scan(states, p, causal ? gk::SCAN_EXCL_PREFIX : gk::SCAN_TOTAL, st);
+    if (e != cudaSuccess) return e;
+    a.state = states;
+    a.state_seg_stride = causal ? (int64_t)p.M * p.D : 0;
+    return timed("tc_fwd_walk", st, [&] {
+        tc::tc_fwd_walk<<<grid, tc::NTH, sm_walk, st>>>(a);
+        return cudaGetLastError();
+    });
+}
+
 template <typename DT>
 cudaError_t dispatch_forward(const Plan &p, const Args &a, float *states, int causal,
                              cudaStream_t st)
@@ -323,9 +366,8 @@ race_status_t race_attn_forward(const void *q, const void *k, const void *v, con
     float *states = ctx ? ctx : (float *)workspace;
     cudaStream_t st = (cudaStream_t)stream;
     cudaError_t e;
-    if (race::tc::fast_path_ok(dtype, d, L, P, tau))
-        e = race::tc::forward(q, k, v, W, out, den, states, B * H, N, p.seg_len, p.nseg, tau,
-                              causal, st);
+    if (race::tc::fast_path_ok(dtype, d, L, P, tau) && g_tc_forward)
+        e = tc_forward(p, q, k, v, W, out, den, states, tau, causal, st);
     else if (dtype == RACE_F32)
         e = dispatch_forward<float>(p, a, states, causal, st);
     else
@@ -370,10 +412,7 @@ race_status_t race_attn_backward(const void *q, const void *k, const void *v, co
     float *gbuf = hbuf + p.state_elems;
     cudaStream_t st = (cudaStream_t)stream;
     cudaError_t e;
-    if (race::tc::fast_path_ok(dtype, d, L, P, tau))
-        e = race::tc::backward(q, k, v, W, out, den, dout, ctx, hbuf, gbuf, dq, dk, dv, B * H, N,
-                               p.seg_len, p.nseg, tau, causal, st);
-    else if (dtype == RACE_F32)
+    if (dtype == RACE_F32)
         e = dispatch_backward<float>(p, a, ctx, hbuf, gbuf, causal, st);
     else
         e = dispatch_backward<__nv_bfloat16>(p, a, ctx, hbuf, gbuf, causal, st);

@@ -1,28 +1,562 @@
-// race_tc.cuh -- tensor-core (tcgen05) path for the bf16, d = 64, L*2^P = 256 shape.
+// race_tc.cuh -- tcgen05 (5th-generation tensor core) path of RACE Attention for the shape
+// bf16 inputs, d = 64, L = 16 tables of P = 4 hyperplanes (L * 2^P = 256 features).
+//
+// Method ("RACE Attention: A Strictly Linear-Time Attention for Long-Sequence Training"):
+// soft bucket assignment per token (zh §2.2), bucket statistics A, B (zh §2.2), the global
+// read-out sum_l phi_l(q)^T B_l / sum_l phi_l(q)^T A_l (Algorithm 1) and its causal form
+// with cumulative statistics (Algorithm 2, zh §2.3), evaluated chunk by chunk:
+//
+//   per chunk of T = 128 tokens, with V~ = [V | 1] (80 columns, 15 of them zero):
+//     proj   = X W^T                        (X = raw q or k rows; W split as bf16 hi + lo)
+//     Phi    = soft hash of proj / |x|      (CUDA cores: tanh, sigmoid products)
+//     S      = Phi_Q Phi_K^T                (causal only; masked to j <= i)
+//     Y      = Phi_Q H_prev  (+ S V~)       (H_prev: state before the chunk, staged as bf16)
+//     H     += Phi_K^T V~                   (causal; fp32 master copy stays in TMEM)
+//     out    = Y[:, :64] / Y[:, 64],  den = Y[:, 64]
+//
+// Every GEMM above is a tcgen05.mma with operands in shared memory (SW128 / SW32 swizzled
+// tiles) and the accumulator in tensor memory; one thread issues them, completion is
+// signalled through an mbarrier that the other threads wait on with a bounded poll.
+// One CTA of 256 threads walks one segment of one (b, h) sequence; thread t owns token
+// row t % 128 and the tables of half t / 128 (tables 0-7 or 8-15).
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
 #include "race_attn.h"
+#include "race_common.cuh"
+#include "race_tc_util.cuh"
 
 namespace race {
 namespace tc {
 
-inline bool fast_path_ok(race_dtype_t, int, int, int, float) { return false; }
+constexpr int T = 128;      // tokens per chunk (MMA M)
+constexpr int NTH = 256;    // threads per CTA
+constexpr int DH = 64;      // head dimension
+constexpr int NPROJ = 64;   // L * P projections
+constexpr int MF = 256;     // L * 2^P features
+constexpr int NV = 80;      // value columns: 64 of V, the ones column, 15 zero
+constexpr int DS = 65;      // state row length in global memory (64 + ones column)
+constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s: far above any chunk's MMA time
 
-inline cudaError_t forward(const void *, const void *, const void *, const float *, void *, float *,
-                           float *, int, int64_t, int64_t, int, float, int, cudaStream_t)
+constexpr uint32_t TILE = 16384;  // one [128][64] bf16 SW128 tile
+
+// error word shared by all launches of this path (1 = an MMA completion wait timed out)
+__device__ int g_tc_error;
+
+struct Args {
+    const __nv_bfloat16 *q, *k, *v;
+    const float *W;
+    __nv_bfloat16 *out;
+    float *den;
+    const float *state;        // walk start states [BH][nseg][256][65]
+    int64_t state_seg_stride;  // floats between segments' states (0 = one shared state)
+    float *agg_out;            // aggregate output [BH][nseg][256][65]
+    int64_t N, seg_len;
+    int nseg;
+    float beta;
+    int causal;
+};
+
+// ---- shared memory maps (byte offsets from a 1024-aligned base) -------------------------
+namespace fwd_smem {
+constexpr uint32_t PHQ = 0;                 // Phi_Q [128][256]: 4 SW128 tiles
+constexpr uint32_t XQ = PHQ;                // q rows during the projection
+constexpr uint32_t XK = PHQ + TILE;         // k rows during the projection
+constexpr uint32_t SB = PHQ;                // masked S as bf16 [128][128]: 2 tiles
+constexpr uint32_t PHK = PHQ + 4 * TILE;    // Phi_K [128][256]
+constexpr uint32_t HS128 = PHK + 4 * TILE;  // staged H[:, 0:64] as [256][64] SW128 (2 tiles)
+constexpr uint32_t HS32 = HS128 + 2 * TILE; // staged H[:, 64:80] as [256][16] SW32 (8 KB)
+constexpr uint32_t V = HS32 + 8192;         // v rows [128][64]
+constexpr uint32_t ONES = V + TILE;         // ones column block [128][16] SW32 (4 KB)
+constexpr uint32_t WHI = ONES + 4096;       // W hi [64][64]
+constexpr uint32_t WLO = WHI + 8192;        // W lo [64][64]
+constexpr uint32_t BAR = WLO + 8192;        // mbarrier, TMEM address, abort flag
+constexpr uint32_t TOTAL = BAR + 64;
+}  // namespace fwd_smem
+
+namespace agg_smem {
+constexpr uint32_t PHK = 0;                 // Phi_K, also k rows during the projection
+constexpr uint32_t XK = PHK;
+constexpr uint32_t V = PHK + 4 * TILE;
+constexpr uint32_t ONES = V + TILE;
+constexpr uint32_t WHI = ONES + 4096;
+constexpr uint32_t WLO = WHI + 8192;
+constexpr uint32_t BAR = WLO + 8192;
+constexpr uint32_t TOTAL = BAR + 64;
+}  // namespace agg_smem
+
+// TMEM columns
+namespace fwd_tmem {
+constexpr uint32_t PROJ = 0;    // [128][64] q projections, [128][64] k projections at +64
+constexpr uint32_t S = 0;       // [128][128] (reuses PROJ once the features are formed)
+constexpr uint32_t Y = 128;     // [128][80]
+constexpr uint32_t HTOP = 256;  // H rows 0..127   [128][80]
+constexpr uint32_t HBOT = 336;  // H rows 128..255 [128][80]
+constexpr uint32_t NCOLS = 512;
+}  // namespace fwd_tmem
+namespace agg_tmem {
+constexpr uint32_t PROJ = 0;
+constexpr uint32_t HTOP = 64;
+constexpr uint32_t HBOT = 144;
+constexpr uint32_t NCOLS = 256;
+}  // namespace agg_tmem
+
+struct Ctl {
+    uint64_t bar;
+    uint32_t tmem;
+    uint32_t abort;
+};
+
+__device__ __forceinline__ uint8_t *aligned_base(uint8_t *raw)
 {
-    return cudaErrorNotSupported;
+    const uint32_t a = smem_u32(raw);
+    return raw + (((a + 1023u) & ~1023u) - a);
 }
 
-inline cudaError_t backward(const void *, const void *, const void *, const float *, const void *,
-                            const float *, const void *, const float *, float *, float *, void *,
-                            void *, void *, int, int64_t, int64_t, int, float, int, cudaStream_t)
+__device__ __forceinline__ uint32_t lane_base() { return (uint32_t)((threadIdx.x >> 5) & 3) * 32u; }
+
+// W [64][64] fp32 -> two SW128 tiles of bf16 (hi = round(W), lo = round(W - hi)).
+__device__ void load_w_split(const float *W, uint8_t *whi, uint8_t *wlo)
 {
-    return cudaErrorNotSupported;
+    for (int e = threadIdx.x; e < NPROJ * DH; e += NTH) {
+        const int n = e >> 6, c = e & 63;
+        const float w = W[e];
+        const __nv_bfloat16 hi = __float2bfloat16_rn(w);
+        const __nv_bfloat16 lo = __float2bfloat16_rn(w - __bfloat162float(hi));
+        const uint32_t off = sw128_off(n, c >> 3) + (c & 7) * 2;
+        *reinterpret_cast<__nv_bfloat16 *>(whi + off) = hi;
+        *reinterpret_cast<__nv_bfloat16 *>(wlo + off) = lo;
+    }
 }
+
+// Ones column block: row j holds 1 in column 0 when j < nvalid, zeros elsewhere.
+__device__ void write_ones(uint8_t *ones, int nvalid)
+{
+    if (threadIdx.x < T) {
+        const int j = threadIdx.x;
+        const uint32_t one = j < nvalid ? 0x3F80u : 0u;  // bf16 1.0 in the low half
+        const uint32_t a = smem_u32(ones);
+        st_shared_v4(a + sw32_off(j, 0), one, 0u, 0u, 0u);
+        st_shared_v4(a + sw32_off(j, 1), 0u, 0u, 0u, 0u);
+    }
+}
+
+// Wait for the MMAs committed to ctl->bar; one thread polls (bounded), all learn the outcome.
+__device__ __forceinline__ bool wait_mma(Ctl *ctl, uint32_t &phase)
+{
+    if (threadIdx.x == 0) {
+        if (!mbar_wait(&ctl->bar, phase & 1u, WAIT_LIMIT_NS)) {
+            ctl->abort = 1u;
+            atomicExch(&g_tc_error, 1);
+        }
+    }
+    ++phase;
+    __syncthreads();
+    fence_after_sync();
+    return *(volatile uint32_t *)&ctl->abort == 0u;
+}
+
+// Hand the shared-memory tiles written so far to the tensor core and sync the CTA.
+__device__ __forceinline__ void publish_smem()
+{
+    fence_smem_async();
+    fence_before_sync();
+    __syncthreads();
+}
+
+// Squared L2 norm of row r of a [128][64] SW128 tile.
+__device__ __forceinline__ float row_sqnorm(const uint8_t *tile, int r)
+{
+    const uint32_t a = smem_u32(tile);
+    float s = 0.f;
+#pragma unroll
+    for (int ch = 0; ch < 8; ++ch) {
+        const uint4 w = ld_shared_v4(a + sw128_off(r, ch));
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float x0 = bf16_lo(ws[i]), x1 = bf16_hi(ws[i]);
+            s = fmaf(x0, x0, s);
+            s = fmaf(x1, x1, s);
+        }
+    }
+    return s;
+}
+
+// Soft bucket assignment of the 8 tables of half h for token row r, from the 32
+// projections in TMEM (columns col0 + 32h ..), written as bf16 into the Phi tile
+// [128][256].  phi_l[r] = prod_p sigmoid(2 beta c_rp u_p) with u = tanh(proj / |x|): the
+// corner softmax of zh §2.2 in factorised form; sigmoid(2z) = (1 + tanh z) / 2.
+__device__ __forceinline__ void features_half(uint32_t tmem, uint32_t col0, int r, int h, float inv_norm,
+                                              float beta, bool valid, uint8_t *phi)
+{
+    float pr[32];
+    {
+        float a[16], b[16];
+        const uint32_t t = tmem + (lane_base() << 16) + col0 + 32u * h;
+        tmem_ld16(t, a);
+        tmem_ld16(t + 16, b);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            pr[i] = a[i];
+            pr[16 + i] = b[i];
+        }
+    }
+    const uint32_t base = smem_u32(phi);
+#pragma unroll
+    for (int l = 0; l < 8; ++l) {
+        float f[16];
+        f[0] = 1.f;
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            const float u = tanh_fast(pr[4 * l + p] * inv_norm);
+            const float t = tanh_fast(beta * u);
+            const float s1 = 0.5f + 0.5f * t, s0 = 0.5f - 0.5f * t;
+            const int hh = 1 << p;
+#pragma unroll
+            for (int c = 0; c < hh; ++c) {
+                f[c + hh] = f[c] * s1;
+                f[c] *= s0;
+            }
+        }
+        uint32_t w[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) w[i] = valid ? pack_bf16x2(f[2 * i], f[2 * i + 1]) : 0u;
+        const int tl = 8 * h + l;            // table 0..15 -> features 16 tl .. 16 tl + 15
+        const uint32_t blk = base + (uint32_t)(tl >> 2) * TILE;
+        const int ch = (tl & 3) * 2;
+        st_shared_v4(blk + sw128_off(r, ch), w[0], w[1], w[2], w[3]);
+        st_shared_v4(blk + sw128_off(r, ch + 1), w[4], w[5], w[6], w[7]);
+    }
+}
+
+// proj[128][64] (+)= X[128][64] (W_hi + W_lo)^T
+__device__ __forceinline__ void issue_proj(uint32_t d, uint32_t x, uint32_t whi, uint32_t wlo)
+{
+    constexpr uint32_t id = idesc_bf16(128, 64, 0, 0);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t a = sdesc(x + kk * 32, 16, 1024, LAYOUT_SW128);
+        mma_bf16(d, a, sdesc(whi + kk * 32, 16, 1024, LAYOUT_SW128), id, kk > 0);
+        mma_bf16(d, a, sdesc(wlo + kk * 32, 16, 1024, LAYOUT_SW128), id, 1);
+    }
+}
+
+// D[128][80] (+)= A * [V | 1] with A given per K-step (16 tokens) by a_at(kk); B from the
+// V tile (MN-major SW128) and the ones block (MN-major SW32).
+template <typename AF>
+__device__ __forceinline__ void issue_times_vt(uint32_t d, AF a_at, int a_mn, uint32_t vt, uint32_t ones,
+                                               bool acc_first)
+{
+    const uint32_t i64 = idesc_bf16(128, 64, a_mn, 1), i16 = idesc_bf16(128, 16, a_mn, 1);
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+        const uint64_t a = a_at(kk);
+        const uint32_t acc = (kk > 0 || acc_first) ? 1u : 0u;
+        mma_bf16(d, a, sdesc(vt + kk * 2048, TILE, 1024, LAYOUT_SW128), i64, acc);
+        mma_bf16(d + 64, a, sdesc(ones + kk * 512, 4096, 256, LAYOUT_SW32), i16, acc);
+    }
+}
+
+// H (both halves) += Phi_K^T [V | 1]
+__device__ __forceinline__ void issue_state_update(uint32_t tm, uint32_t htop, uint32_t hbot, uint32_t phk,
+                                                   uint32_t vt, uint32_t ones)
+{
+    issue_times_vt(tm + htop, [&](int kk) { return sdesc(phk + kk * 2048, TILE, 1024, LAYOUT_SW128); }, 1,
+                   vt, ones, true);
+    issue_times_vt(tm + hbot,
+                   [&](int kk) { return sdesc(phk + 2 * TILE + kk * 2048, TILE, 1024, LAYOUT_SW128); }, 1,
+                   vt, ones, true);
+}
+
+// Row of the state (lane r of the H half h: feature m = 128h + r), 80 columns -> regs.
+__device__ __forceinline__ void read_state_row(uint32_t tmem, uint32_t col, float (&hv)[80])
+{
+    const uint32_t t = tmem + (lane_base() << 16) + col;
+#pragma unroll
+    for (int c = 0; c < 5; ++c) {
+        float x[16];
+        tmem_ld16(t + 16 * c, x);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) hv[16 * c + i] = x[i];
+    }
+    tmem_wait_ld();
+}
+
+// Stage one state row (feature m) as bf16 into the [256][64] SW128 + [256][16] SW32 tiles.
+__device__ __forceinline__ void stage_state_row(const float (&hv)[80], int m, uint8_t *hs128, uint8_t *hs32)
+{
+    const uint32_t b128 = smem_u32(hs128) + (uint32_t)(m >> 7) * TILE;
+    const int rr = m & 127;
+#pragma unroll
+    for (int ch = 0; ch < 8; ++ch)
+        st_shared_v4(b128 + sw128_off(rr, ch), pack_bf16x2(hv[8 * ch], hv[8 * ch + 1]),
+                     pack_bf16x2(hv[8 * ch + 2], hv[8 * ch + 3]), pack_bf16x2(hv[8 * ch + 4], hv[8 * ch + 5]),
+                     pack_bf16x2(hv[8 * ch + 6], hv[8 * ch + 7]));
+    const uint32_t b32 = smem_u32(hs32);
+#pragma unroll
+    for (int ch = 0; ch < 2; ++ch)
+        st_shared_v4(b32 + sw32_off(m, ch), pack_bf16x2(hv[64 + 8 * ch], hv[65 + 8 * ch]),
+                     pack_bf16x2(hv[66 + 8 * ch], hv[67 + 8 * ch]), pack_bf16x2(hv[68 + 8 * ch], hv[69 + 8 * ch]),
+                     pack_bf16x2(hv[70 + 8 * ch], hv[71 + 8 * ch]));
+}
+
+__device__ __forceinline__ void seg_bounds(const Args &a, int seg, int64_t &t0, int64_t &t1)
+{
+    t0 = (int64_t)seg * a.seg_len;
+    t1 = t0 + a.seg_len;
+    if (t1 > a.N) t1 = a.N;
+}
+
+// ------------------------------------------------------------------------------------------
+// Segment totals: H_seg = sum_{j in segment} phi(k_j) [v_j, 1]^T   (grid: nseg x BH)
+// ------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(NTH, 2) tc_agg_kv(Args a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = aligned_base(smem_raw);
+    using namespace agg_smem;
+    Ctl *ctl = reinterpret_cast<Ctl *>(sm + BAR);
+    const int seg = blockIdx.x, bh = blockIdx.y;
+    const int r = threadIdx.x & 127, h = threadIdx.x >> 7;
+    const uint32_t sb = smem_u32(sm);
+    if (threadIdx.x == 0) {
+        mbar_init(&ctl->bar, 1);
+        ctl->abort = 0;
+    }
+    if (threadIdx.x < 32) tmem_alloc(&ctl->tmem, agg_tmem::NCOLS);
+    load_w_split(a.W, sm + WHI, sm + WLO);
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tm = ctl->tmem;
+    {  // zero state
+        float z[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) z[i] = 0.f;
+        const uint32_t t = tm + (lane_base() << 16) + (h ? agg_tmem::HBOT : agg_tmem::HTOP);
+#pragma unroll
+        for (int c = 0; c < 5; ++c) tmem_st16(t + 16 * c, z);
+        tmem_wait_st();
+    }
+    int64_t t0, t1;
+    seg_bounds(a, seg, t0, t1);
+    const int64_t base = (int64_t)bh * a.N;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int64_t c0 = t0; c0 < t1 && ok; c0 += T) {
+        const int nv = (int)(t1 - c0 < T ? t1 - c0 : T);
+        load_tile_async<NTH>(sm + XK, a.k + (base + c0) * DH, nv);
+        load_tile_async<NTH>(sm + V, a.v + (base + c0) * DH, nv);
+        cp_async_commit();
+        write_ones(sm + ONES, nv);
+        cp_async_wait_all();
+        publish_smem();
+        if (threadIdx.x == 0) {
+            fence_after_sync();
+            issue_proj(tm + agg_tmem::PROJ, sb + XK, sb + WHI, sb + WLO);
+            mma_commit(&ctl->bar);
+        }
+        const float inv = 1.f / fmaxf(sqrtf(row_sqnorm(sm + XK, r)), kNormEps);
+        if (!(ok = wait_mma(ctl, phase))) break;
+        features_half(tm, agg_tmem::PROJ, r, h, inv, a.beta, r < nv, sm + PHK);
+        publish_smem();
+        if (threadIdx.x == 0) {
+            fence_after_sync();
+            issue_state_update(tm, agg_tmem::HTOP, agg_tmem::HBOT, sb + PHK, sb + V, sb + ONES);
+            mma_commit(&ctl->bar);
+        }
+        ok = wait_mma(ctl, phase);
+    }
+    if (ok) {
+        float hv[80];
+        read_state_row(tm, h ? agg_tmem::HBOT : agg_tmem::HTOP, hv);
+        const int m = 128 * h + r;
+        float *dst = a.agg_out + (((int64_t)bh * a.nseg + seg) * MF + m) * DS;
+#pragma unroll
+        for (int c = 0; c < DS; ++c) dst[c] = hv[c];
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (threadIdx.x < 32) tmem_dealloc(tm, agg_tmem::NCOLS);
+}
+
+// ------------------------------------------------------------------------------------------
+// Walk: causal (Algorithm 2) or bidirectional read-out (Algorithm 1).  grid: nseg x BH
+// ------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(NTH, 1) tc_fwd_walk(Args a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = aligned_base(smem_raw);
+    using namespace fwd_smem;
+    Ctl *ctl = reinterpret_cast<Ctl *>(sm + BAR);
+    const int seg = blockIdx.x, bh = blockIdx.y;
+    const int r = threadIdx.x & 127, h = threadIdx.x >> 7;
+    const uint32_t sb = smem_u32(sm);
+    const bool causal = a.causal != 0;
+    if (threadIdx.x == 0) {
+        mbar_init(&ctl->bar, 1);
+        ctl->abort = 0;
+    }
+    if (threadIdx.x < 32) tmem_alloc(&ctl->tmem, fwd_tmem::NCOLS);
+    load_w_split(a.W, sm + WHI, sm + WLO);
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tm = ctl->tmem;
+    {  // start state: fp32 master into TMEM, bf16 copy into the staging tiles
+        const int m = 128 * h + r;
+        const float *src = a.state + (int64_t)bh * a.nseg * MF * DS + seg * a.state_seg_stride + (int64_t)m * DS;
+        float hv[80];
+#pragma unroll
+        for (int c = 0; c < 80; ++c) hv[c] = c < DS ? src[c] : 0.f;
+        const uint32_t t = tm + (lane_base() << 16) + (h ? fwd_tmem::HBOT : fwd_tmem::HTOP);
+#pragma unroll
+        for (int c = 0; c < 5; ++c) {
+            float x[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) x[i] = hv[16 * c + i];
+            tmem_st16(t + 16 * c, x);
+        }
+        tmem_wait_st();
+        stage_state_row(hv, m, sm + HS128, sm + HS32);
+    }
+    int64_t t0, t1;
+    seg_bounds(a, seg, t0, t1);
+    const int64_t base = (int64_t)bh * a.N;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int64_t c0 = t0; c0 < t1 && ok; c0 += T) {
+        const int nv = (int)(t1 - c0 < T ? t1 - c0 : T);
+        load_tile_async<NTH>(sm + XQ, a.q + (base + c0) * DH, nv);
+        if (causal) {
+            load_tile_async<NTH>(sm + XK, a.k + (base + c0) * DH, nv);
+            load_tile_async<NTH>(sm + V, a.v + (base + c0) * DH, nv);
+        }
+        cp_async_commit();
+        if (causal) write_ones(sm + ONES, nv);
+        cp_async_wait_all();
+        publish_smem();
+        if (threadIdx.x == 0) {
+            fence_after_sync();
+            issue_proj(tm + fwd_tmem::PROJ, sb + XQ, sb + WHI, sb + WLO);
+            if (causal) issue_proj(tm + fwd_tmem::PROJ + 64, sb + XK, sb + WHI, sb + WLO);
+            mma_commit(&ctl->bar);
+        }
+        const float inv_q = 1.f / fmaxf(sqrtf(row_sqnorm(sm + XQ, r)), kNormEps);
+        const float inv_k = causal ? 1.f / fmaxf(sqrtf(row_sqnorm(sm + XK, r)), kNormEps) : 0.f;
+        if (!(ok = wait_mma(ctl, phase))) break;
+        features_half(tm, fwd_tmem::PROJ, r, h, inv_q, a.beta, r < nv, sm + PHQ);
+        if (causal) features_half(tm, fwd_tmem::PROJ + 64, r, h, inv_k, a.beta, r < nv, sm + PHK);
+        publish_smem();
+        if (threadIdx.x == 0) {
+            fence_after_sync();
+            if (causal) {  // S = Phi_Q Phi_K^T
+                constexpr uint32_t id = idesc_bf16(128, 128, 0, 0);
+#pragma unroll
+                for (int kk = 0; kk < 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * TILE + (kk & 3) * 32;
+                    mma_bf16(tm + fwd_tmem::S, sdesc(sb + PHQ + off, 16, 1024, LAYOUT_SW128),
+                             sdesc(sb + PHK + off, 16, 1024, LAYOUT_SW128), id, kk > 0);
+                }
+            }
+            {  // Y = Phi_Q H_prev
+                constexpr uint32_t i64 = idesc_bf16(128, 64, 0, 1), i16 = idesc_bf16(128, 16, 0, 1);
+#pragma unroll
+                for (int kk = 0; kk < 16; ++kk) {
+                    const uint64_t aq = sdesc(sb + PHQ + (kk >> 2) * TILE + (kk & 3) * 32, 16, 1024, LAYOUT_SW128);
+                    mma_bf16(tm + fwd_tmem::Y, aq, sdesc(sb + HS128 + kk * 2048, TILE, 1024, LAYOUT_SW128), i64,
+                             kk > 0);
+                    mma_bf16(tm + fwd_tmem::Y + 64, aq, sdesc(sb + HS32 + kk * 512, 8192, 256, LAYOUT_SW32), i16,
+                             kk > 0);
+                }
+            }
+            mma_commit(&ctl->bar);
+        }
+        if (!(ok = wait_mma(ctl, phase))) break;
+        if (causal) {
+            // masked S (j <= i) as bf16: row r, columns 64h .. 64h+63
+            const uint32_t t = tm + (lane_base() << 16) + fwd_tmem::S + 64u * h;
+            const uint32_t blk = sb + SB + (uint32_t)h * TILE;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                float x[16];
+                tmem_ld16(t + 16 * c, x);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    if (64 * h + 16 * c + i > r) x[i] = 0.f;
+                st_shared_v4(blk + sw128_off(r, 2 * c), pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]),
+                             pack_bf16x2(x[4], x[5]), pack_bf16x2(x[6], x[7]));
+                st_shared_v4(blk + sw128_off(r, 2 * c + 1), pack_bf16x2(x[8], x[9]), pack_bf16x2(x[10], x[11]),
+                             pack_bf16x2(x[12], x[13]), pack_bf16x2(x[14], x[15]));
+            }
+            publish_smem();
+            if (threadIdx.x == 0) {
+                fence_after_sync();
+                // Y += S [V | 1]
+                issue_times_vt(tm + fwd_tmem::Y,
+                               [&](int kk) {
+                                   return sdesc(sb + SB + (kk >> 2) * TILE + (kk & 3) * 32, 16, 1024,
+                                                LAYOUT_SW128);
+                               },
+                               0, sb + V, sb + ONES, true);
+                // H += Phi_K^T [V | 1]
+                issue_state_update(tm, fwd_tmem::HTOP, fwd_tmem::HBOT, sb + PHK, sb + V, sb + ONES);
+                mma_commit(&ctl->bar);
+            }
+            if (!(ok = wait_mma(ctl, phase))) break;
+        }
+        {  // out = Y[:, :64] / Y[:, 64]: this thread writes columns 32h .. 32h+31 of row r
+            float y[32], dn[16];
+            const uint32_t t = tm + (lane_base() << 16) + fwd_tmem::Y;
+            float y0[16], y1[16];
+            tmem_ld16(t + 32u * h, y0);
+            tmem_ld16(t + 32u * h + 16, y1);
+            tmem_ld16(t + 64, dn);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                y[i] = y0[i];
+                y[16 + i] = y1[i];
+            }
+            if (r < nv) {
+                const float d = dn[0];
+                const float inv = d != 0.f ? 1.f / d : 0.f;
+                uint4 *dst = reinterpret_cast<uint4 *>(a.out + (base + c0 + r) * DH + 32 * h);
+#pragma unroll
+                for (int v4 = 0; v4 < 4; ++v4)
+                    dst[v4] = make_uint4(pack_bf16x2(y[8 * v4] * inv, y[8 * v4 + 1] * inv),
+                                         pack_bf16x2(y[8 * v4 + 2] * inv, y[8 * v4 + 3] * inv),
+                                         pack_bf16x2(y[8 * v4 + 4] * inv, y[8 * v4 + 5] * inv),
+                                         pack_bf16x2(y[8 * v4 + 6] * inv, y[8 * v4 + 7] * inv));
+                if (h == 0 && a.den) a.den[base + c0 + r] = d;
+            }
+        }
+        if (causal) {  // stage the updated state for the next chunk's read-out
+            float hv[80];
+            read_state_row(tm, h ? fwd_tmem::HBOT : fwd_tmem::HTOP, hv);
+            stage_state_row(hv, 128 * h + r, sm + HS128, sm + HS32);
+        }
+        publish_smem();
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (threadIdx.x < 32) tmem_dealloc(tm, fwd_tmem::NCOLS);
+}
+
+// ---- host side ---------------------------------------------------------------------------
+
+inline bool fast_path_ok(race_dtype_t dtype, int d, int L, int P, float tau)
+{
+    return dtype == RACE_BF16 && d == 64 && L == 16 && P == 4 && tau > 0.f;
+}
+
+inline size_t smem_bytes(uint32_t total) { return total + 1024; }
 
 }  // namespace tc
 }  // namespace race
