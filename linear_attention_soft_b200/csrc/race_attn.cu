@@ -26,7 +26,8 @@ struct ProfPending {
     cudaEvent_t a, b;
 };
 bool g_prof_on = false;
-bool g_tc_forward = true;  // tensor-core forward for the shapes it covers
+bool g_tc_forward = true;   // tensor-core forward for the shapes it covers
+bool g_tc_backward = true;  // tensor-core backward for the shapes it covers
 std::vector<ProfEntry> g_prof;
 std::vector<ProfPending> g_pending;
 std::vector<cudaEvent_t> g_event_pool;
@@ -282,6 +283,88 @@ cudaError_t tc_forward(const Plan &p, const void *q, const void *k, const void *
     });
 }
 
+cudaError_t tc_backward(const Plan &p, const void *q, const void *k, const void *v, const float *W,
+                        const void *out, const float *den, const void *dout, const float *ctx, float *hbuf,
+                        float *gbuf, void *dq, void *dk, void *dv, float tau, int causal, cudaStream_t st)
+{
+    namespace tc = race::tc;
+    const dim3 grid((unsigned)p.nseg, (unsigned)p.BH);
+    cudaError_t e;
+    const float *hstates = ctx;
+    if (!hstates) {  // key-side prefix statistics, as the forward computes them
+        tc::Args fa;
+        std::memset(&fa, 0, sizeof(fa));
+        fa.k = (const __nv_bfloat16 *)k;
+        fa.v = (const __nv_bfloat16 *)v;
+        fa.W = W;
+        fa.N = p.N;
+        fa.seg_len = p.seg_len;
+        fa.nseg = p.nseg;
+        fa.beta = 1.f / tau;
+        fa.causal = causal;
+        fa.agg_out = hbuf;
+        const size_t sm_agg = tc::smem_bytes(tc::agg_smem::TOTAL);
+        e = cudaFuncSetAttribute(tc::tc_agg_kv, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_agg);
+        if (e != cudaSuccess) return e;
+        e = timed("tc_agg_kv", st, [&] {
+            tc::tc_agg_kv<<<grid, tc::NTH, sm_agg, st>>>(fa);
+            return cudaGetLastError();
+        });
+        if (e != cudaSuccess) return e;
+        e = launch_scan(hbuf, p, causal ? gk::SCAN_EXCL_PREFIX : gk::SCAN_TOTAL, st);
+        if (e != cudaSuccess) return e;
+        hstates = hbuf;
+    }
+    tc::BwdArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.q = (const __nv_bfloat16 *)q;
+    a.k = (const __nv_bfloat16 *)k;
+    a.v = (const __nv_bfloat16 *)v;
+    a.o = (const __nv_bfloat16 *)out;
+    a.dout = (const __nv_bfloat16 *)dout;
+    a.den = den;
+    a.W = W;
+    a.dq = (__nv_bfloat16 *)dq;
+    a.dk = (__nv_bfloat16 *)dk;
+    a.dv = (__nv_bfloat16 *)dv;
+    a.N = p.N;
+    a.seg_len = p.seg_len;
+    a.nseg = p.nseg;
+    a.beta = 1.f / tau;
+    a.causal = causal;
+    const int64_t stride = causal ? (int64_t)p.M * p.D : 0;
+    const size_t sm_q = tc::smem_bytes(tc::bq_smem::TOTAL);
+    const size_t sm_aq = tc::smem_bytes(tc::aggq_smem::TOTAL);
+    const size_t sm_kv = tc::smem_bytes(tc::bkv_smem::TOTAL);
+    if ((e = cudaFuncSetAttribute(tc::tc_bwd_q_walk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_q)) !=
+            cudaSuccess ||
+        (e = cudaFuncSetAttribute(tc::tc_agg_qdy, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_aq)) !=
+            cudaSuccess ||
+        (e = cudaFuncSetAttribute(tc::tc_bwd_kv_walk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_kv)) !=
+            cudaSuccess)
+        return e;
+    a.state = hstates;
+    a.state_seg_stride = stride;
+    e = timed("tc_bwd_q_walk", st, [&] {
+        tc::tc_bwd_q_walk<<<grid, tc::NTH, sm_q, st>>>(a);
+        return cudaGetLastError();
+    });
+    if (e != cudaSuccess) return e;
+    a.agg_out = gbuf;
+    e = timed("tc_agg_qdy", st, [&] {
+        tc::tc_agg_qdy<<<grid, tc::NTH, sm_aq, st>>>(a);
+        return cudaGetLastError();
+    });
+    if (e != cudaSuccess) return e;
+    e = launch_scan(gbuf, p, causal ? gk::SCAN_EXCL_SUFFIX : gk::SCAN_TOTAL, st);
+    if (e != cudaSuccess) return e;
+    a.state = gbuf;
+    return timed("tc_bwd_kv_walk", st, [&] {
+        tc::tc_bwd_kv_walk<<<grid, tc::NTH, sm_kv, st>>>(a);
+        return cudaGetLastError();
+    });
+}
+
 template <typename DT>
 cudaError_t dispatch_forward(const Plan &p, const Args &a, float *states, int causal,
                              cudaStream_t st)
@@ -412,7 +495,9 @@ race_status_t race_attn_backward(const void *q, const void *k, const void *v, co
     float *gbuf = hbuf + p.state_elems;
     cudaStream_t st = (cudaStream_t)stream;
     cudaError_t e;
-    if (dtype == RACE_F32)
+    if (race::tc::fast_path_ok(dtype, d, L, P, tau) && g_tc_backward)
+        e = tc_backward(p, q, k, v, W, out, den, dout, ctx, hbuf, gbuf, dq, dk, dv, tau, causal, st);
+    else if (dtype == RACE_F32)
         e = dispatch_backward<float>(p, a, ctx, hbuf, gbuf, causal, st);
     else
         e = dispatch_backward<__nv_bfloat16>(p, a, ctx, hbuf, gbuf, causal, st);

@@ -549,6 +549,697 @@ __global__ void __launch_bounds__(NTH, 1) tc_fwd_walk(Args a)
     if (threadIdx.x < 32) tmem_dealloc(tm, fwd_tmem::NCOLS);
 }
 
+// ==========================================================================================
+// Backward.  With dY_i = [dO_i / den_i, -(dO_i . o_i) / den_i] (80 columns, 15 zero):
+//   dq side (prefix state H):   dPhi_Q = dY H_prev^T + tril(dY V~^T) Phi_K,   H += Phi_K^T V~
+//   dk/dv side (suffix state G, chunks walked backwards):
+//     dV~   = Phi_K G_next + triu(Phi_K Phi_Q^T) dY          (dv = dV~[:, :64])
+//     dPhi_K = V~ G_next^T + triu(V~ dY^T) Phi_Q,              G += Phi_Q^T dY
+//   feature-map VJP per table (CUDA cores): dz = phi (dphi - phi.dphi),
+//   du_p = beta sum_r c_rp dz_r, dp~ = du (1 - u^2); then dX^ = dP~ W (tcgen05) and
+//   dx = (dX^ - x^ (x^ . dX^)) / |x|.
+// ==========================================================================================
+
+struct BwdArgs {
+    const __nv_bfloat16 *q, *k, *v, *o, *dout;
+    const float *den, *W;
+    __nv_bfloat16 *dq, *dk, *dv;
+    const float *state;
+    int64_t state_seg_stride;
+    float *agg_out;
+    int64_t N, seg_len;
+    int nseg;
+    float beta;
+    int causal;
+};
+
+// dY rows [0, nvalid) into DY128 ([128][64] SW128: dO/den) and DY32 ([128][16] SW32:
+// column 0 = -(dO.o)/den); zero rows beyond.  Threads 0..127 each build one row.
+__device__ __forceinline__ void build_dy(const __nv_bfloat16 *dout, const __nv_bfloat16 *o,
+                                         const float *den, int nvalid, uint8_t *dy128, uint8_t *dy32)
+{
+    if (threadIdx.x >= T) return;
+    const int r = threadIdx.x;
+    const uint32_t b128 = smem_u32(dy128), b32 = smem_u32(dy32);
+    if (r >= nvalid) {
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) st_shared_v4(b128 + sw128_off(r, ch), 0u, 0u, 0u, 0u);
+        st_shared_v4(b32 + sw32_off(r, 0), 0u, 0u, 0u, 0u);
+        st_shared_v4(b32 + sw32_off(r, 1), 0u, 0u, 0u, 0u);
+        return;
+    }
+    const float dn = den[r];
+    const float inv = dn != 0.f ? 1.f / dn : 0.f;
+    const uint4 *g4 = reinterpret_cast<const uint4 *>(dout + (int64_t)r * DH);
+    const uint4 *o4 = reinterpret_cast<const uint4 *>(o + (int64_t)r * DH);
+    float dot = 0.f;
+#pragma unroll
+    for (int ch = 0; ch < 8; ++ch) {
+        const uint4 g = g4[ch], ov = o4[ch];
+        const uint32_t gw[4] = {g.x, g.y, g.z, g.w}, ow[4] = {ov.x, ov.y, ov.z, ov.w};
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float g0 = bf16_lo(gw[i]), g1 = bf16_hi(gw[i]);
+            dot = fmaf(g0, bf16_lo(ow[i]), dot);
+            dot = fmaf(g1, bf16_hi(ow[i]), dot);
+            w[i] = pack_bf16x2(g0 * inv, g1 * inv);
+        }
+        st_shared_v4(b128 + sw128_off(r, ch), w[0], w[1], w[2], w[3]);
+    }
+    st_shared_v4(b32 + sw32_off(r, 0), pack_bf16x2(-dot * inv, 0.f), 0u, 0u, 0u);
+    st_shared_v4(b32 + sw32_off(r, 1), 0u, 0u, 0u, 0u);
+}
+
+// Like features_half, keeping u = tanh(proj/|x|) and t = tanh(beta u) of the 32
+// projections (8 tables) in registers for the feature-map VJP; phi may be null.
+__device__ __forceinline__ void features_half_keep(uint32_t tmem, uint32_t col0, int r, int h, float inv_norm,
+                                                   float beta, bool valid, uint8_t *phi, float (&u)[32],
+                                                   float (&t)[32])
+{
+    {
+        float a[16], b[16];
+        const uint32_t ta = tmem + (lane_base() << 16) + col0 + 32u * h;
+        tmem_ld16(ta, a);
+        tmem_ld16(ta + 16, b);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            u[i] = tanh_fast(a[i] * inv_norm);
+            u[16 + i] = tanh_fast(b[i] * inv_norm);
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) t[i] = tanh_fast(beta * u[i]);
+    }
+    if (!phi) return;
+    const uint32_t base = smem_u32(phi);
+#pragma unroll
+    for (int l = 0; l < 8; ++l) {
+        float f[16];
+        f[0] = 1.f;
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            const float s1 = 0.5f + 0.5f * t[4 * l + p], s0 = 0.5f - 0.5f * t[4 * l + p];
+            const int hh = 1 << p;
+#pragma unroll
+            for (int c = 0; c < hh; ++c) {
+                f[c + hh] = f[c] * s1;
+                f[c] *= s0;
+            }
+        }
+        uint32_t w[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) w[i] = valid ? pack_bf16x2(f[2 * i], f[2 * i + 1]) : 0u;
+        const int tl = 8 * h + l;
+        const uint32_t blk = base + (uint32_t)(tl >> 2) * TILE;
+        const int ch = (tl & 3) * 2;
+        st_shared_v4(blk + sw128_off(r, ch), w[0], w[1], w[2], w[3]);
+        st_shared_v4(blk + sw128_off(r, ch + 1), w[4], w[5], w[6], w[7]);
+    }
+}
+
+// Feature-map VJP for the 8 tables of half h: dphi from TMEM columns col0 + 128h .. (16 per
+// table), u and t from features_half_keep; writes dp~ (32 values) as bf16 into row r of
+// the DP tile ([128][64] SW128, projections 32h .. 32h+31).
+__device__ __forceinline__ void features_vjp_half(uint32_t tmem, uint32_t col0, int r, int h, float beta,
+                                                  bool valid, const float (&u)[32], const float (&t)[32],
+                                                  uint8_t *dp_tile)
+{
+    float dp[32];
+    const uint32_t ta = tmem + (lane_base() << 16) + col0 + 128u * h;
+#pragma unroll
+    for (int l = 0; l < 8; ++l) {
+        float g[16];
+        tmem_ld16(ta + 16 * l, g);
+        tmem_wait_ld();
+        float f[16];
+        f[0] = 1.f;
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            const float s1 = 0.5f + 0.5f * t[4 * l + p], s0 = 0.5f - 0.5f * t[4 * l + p];
+            const int hh = 1 << p;
+#pragma unroll
+            for (int c = 0; c < hh; ++c) {
+                f[c + hh] = f[c] * s1;
+                f[c] *= s0;
+            }
+        }
+        float dot = 0.f;
+#pragma unroll
+        for (int c = 0; c < 16; ++c) dot = fmaf(f[c], g[c], dot);
+        float du[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+            const float dz = f[c] * (g[c] - dot);
+#pragma unroll
+            for (int p = 0; p < 4; ++p) du[p] += ((c >> p) & 1) ? dz : -dz;
+        }
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            const float uu = u[4 * l + p];
+            dp[4 * l + p] = valid ? beta * du[p] * (1.f - uu * uu) : 0.f;
+        }
+    }
+    const uint32_t b = smem_u32(dp_tile);
+#pragma unroll
+    for (int ch = 0; ch < 4; ++ch)
+        st_shared_v4(b + sw128_off(r, 4 * h + ch), pack_bf16x2(dp[8 * ch], dp[8 * ch + 1]),
+                     pack_bf16x2(dp[8 * ch + 2], dp[8 * ch + 3]), pack_bf16x2(dp[8 * ch + 4], dp[8 * ch + 5]),
+                     pack_bf16x2(dp[8 * ch + 6], dp[8 * ch + 7]));
+}
+
+// D[128][64] = DP[128][64] (W_hi + W_lo): W as MN-major B (rows = projections, cols = d).
+__device__ __forceinline__ void issue_dxhat(uint32_t d, uint32_t dp, uint32_t whi, uint32_t wlo)
+{
+    constexpr uint32_t id = idesc_bf16(128, 64, 0, 1);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t a = sdesc(dp + kk * 32, 16, 1024, LAYOUT_SW128);
+        mma_bf16(d, a, sdesc(whi + kk * 2048, TILE, 1024, LAYOUT_SW128), id, kk > 0);
+        mma_bf16(d, a, sdesc(wlo + kk * 2048, TILE, 1024, LAYOUT_SW128), id, 1);
+    }
+}
+
+// D[128][N] (+)= A[128][80] B[N][80]^T, both K-major, K split as 64 (SW128) + 16 (SW32).
+__device__ __forceinline__ void issue_k80(uint32_t d, uint32_t a128, uint32_t a32, uint32_t b128, uint32_t b32,
+                                          uint32_t idesc, bool acc_first)
+{
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+        mma_bf16(d, sdesc(a128 + kk * 32, 16, 1024, LAYOUT_SW128), sdesc(b128 + kk * 32, 16, 1024, LAYOUT_SW128),
+                 idesc, (kk > 0 || acc_first) ? 1u : 0u);
+    mma_bf16(d, sdesc(a32, 16, 256, LAYOUT_SW32), sdesc(b32, 16, 256, LAYOUT_SW32), idesc, 1u);
+}
+
+// D[128][N] (+)= A[128][128] B where A = K-major bf16 [128][128] (2 tiles) and B is
+// MN-major [K=128 rows][N] spanning N/64 tiles (LBO = TILE).
+__device__ __forceinline__ void issue_tt_times(uint32_t d, uint32_t a, uint32_t b, uint32_t idesc, bool acc_first)
+{
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk)
+        mma_bf16(d, sdesc(a + (kk >> 2) * TILE + (kk & 3) * 32, 16, 1024, LAYOUT_SW128),
+                 sdesc(b + kk * 2048, TILE, 1024, LAYOUT_SW128), idesc, (kk > 0 || acc_first) ? 1u : 0u);
+}
+
+// Masked T x T block from TMEM (row r, columns col0 + 64h ..) to bf16 K-major tile h of dst.
+// keep_upper: keep column >= row (else column <= row).
+__device__ __forceinline__ void mask_block_to_smem(uint32_t tmem, uint32_t col0, int r, int h, bool keep_upper,
+                                                   uint8_t *dst)
+{
+    const uint32_t t = tmem + (lane_base() << 16) + col0 + 64u * h;
+    const uint32_t blk = smem_u32(dst) + (uint32_t)h * TILE;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        float x[16];
+        tmem_ld16(t + 16 * c, x);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int col = 64 * h + 16 * c + i;
+            if (keep_upper ? (col < r) : (col > r)) x[i] = 0.f;
+        }
+        st_shared_v4(blk + sw128_off(r, 2 * c), pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]),
+                     pack_bf16x2(x[4], x[5]), pack_bf16x2(x[6], x[7]));
+        st_shared_v4(blk + sw128_off(r, 2 * c + 1), pack_bf16x2(x[8], x[9]), pack_bf16x2(x[10], x[11]),
+                     pack_bf16x2(x[12], x[13]), pack_bf16x2(x[14], x[15]));
+    }
+}
+
+// dx = (dX^ - x^ (x^ . dX^)) / max(|x|, eps) for row r, columns 32h .. 32h+31; dX^ from TMEM
+// column col0; x re-read from global; the two halves exchange partial dots through xch.
+__device__ __forceinline__ void write_dx(uint32_t tmem, uint32_t col0, int r, int h, bool valid, float rawn,
+                                         const __nv_bfloat16 *xrow, __nv_bfloat16 *dst, float *xch)
+{
+    float g[32];
+    {
+        float a[16], b[16];
+        const uint32_t ta = tmem + (lane_base() << 16) + col0 + 32u * h;
+        tmem_ld16(ta, a);
+        tmem_ld16(ta + 16, b);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            g[i] = a[i];
+            g[16 + i] = b[i];
+        }
+    }
+    float x[32];
+    float dot = 0.f;
+    if (valid) {
+        const uint4 *x4 = reinterpret_cast<const uint4 *>(xrow + 32 * h);
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+            const uint4 w = x4[ch];
+            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                x[8 * ch + 2 * i] = bf16_lo(ws[i]);
+                x[8 * ch + 2 * i + 1] = bf16_hi(ws[i]);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) dot = fmaf(x[i], g[i], dot);
+    }
+    xch[threadIdx.x] = dot;
+    __syncthreads();
+    dot += xch[threadIdx.x ^ 128];
+    if (!valid) return;
+    const float n = fmaxf(rawn, kNormEps), inv = 1.f / n;
+    const float proj = rawn > kNormEps ? dot * inv * inv : 0.f;  // x^ . dX^ / |x|
+    uint4 *d4 = reinterpret_cast<uint4 *>(dst + 32 * h);
+#pragma unroll
+    for (int ch = 0; ch < 4; ++ch) {
+        float y[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) y[i] = (g[8 * ch + i] - x[8 * ch + i] * proj) * inv;
+        d4[ch] = make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
+                            pack_bf16x2(y[6], y[7]));
+    }
+}
+
+__device__ __forceinline__ void bseg_bounds(const BwdArgs &a, int seg, int64_t &t0, int64_t &t1)
+{
+    t0 = (int64_t)seg * a.seg_len;
+    t1 = t0 + a.seg_len;
+    if (t1 > a.N) t1 = a.N;
+}
+
+// Load a walk's start state (global fp32 [256][65] rows) into TMEM (two halves) and into
+// the bf16 staging tiles.
+__device__ __forceinline__ void load_start_state(const float *src_all, int h, int r, uint32_t tm, uint32_t htop,
+                                                 uint32_t hbot, uint8_t *s128, uint8_t *s32)
+{
+    const int m = 128 * h + r;
+    const float *src = src_all + (int64_t)m * DS;
+    float hv[80];
+#pragma unroll
+    for (int c = 0; c < 80; ++c) hv[c] = c < DS ? src[c] : 0.f;
+    const uint32_t t = tm + (lane_base() << 16) + (h ? hbot : htop);
+#pragma unroll
+    for (int c = 0; c < 5; ++c) {
+        float x[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) x[i] = hv[16 * c + i];
+        tmem_st16(t + 16 * c, x);
+    }
+    tmem_wait_st();
+    stage_state_row(hv, m, s128, s32);
+}
+
+// ------------------------------------------------------------------------------------------
+// Segment totals of the backward's key side: G_seg = sum_{i in segment} phi(q_i) dY_i^T
+// ------------------------------------------------------------------------------------------
+namespace aggq_smem {
+constexpr uint32_t PHQ = 0;
+constexpr uint32_t XQ = PHQ;
+constexpr uint32_t DY128 = PHQ + 4 * TILE;
+constexpr uint32_t DY32 = DY128 + TILE;
+constexpr uint32_t WHI = DY32 + 4096;
+constexpr uint32_t WLO = WHI + 8192;
+constexpr uint32_t BAR = WLO + 8192;
+constexpr uint32_t TOTAL = BAR + 64;
+}  // namespace aggq_smem
+
+__global__ void __launch_bounds__(NTH, 2) tc_agg_qdy(BwdArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = aligned_base(smem_raw);
+    using namespace aggq_smem;
+    Ctl *ctl = reinterpret_cast<Ctl *>(sm + BAR);
+    const int seg = blockIdx.x, bh = blockIdx.y;
+    const int r = threadIdx.x & 127, h = threadIdx.x >> 7;
+    const uint32_t sb = smem_u32(sm);
+    if (threadIdx.x == 0) {
+        mbar_init(&ctl->bar, 1);
+        ctl->abort = 0;
+    }
+    if (threadIdx.x < 32) tmem_alloc(&ctl->tmem, agg_tmem::NCOLS);
+    load_w_split(a.W, sm + WHI, sm + WLO);
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tm = ctl->tmem;
+    {
+        float z[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) z[i] = 0.f;
+        const uint32_t t = tm + (lane_base() << 16) + (h ? agg_tmem::HBOT : agg_tmem::HTOP);
+#pragma unroll
+        for (int c = 0; c < 5; ++c) tmem_st16(t + 16 * c, z);
+        tmem_wait_st();
+    }
+    int64_t t0, t1;
+    bseg_bounds(a, seg, t0, t1);
+    const int64_t base = (int64_t)bh * a.N;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int64_t c0 = t0; c0 < t1 && ok; c0 += T) {
+        const int nv = (int)(t1 - c0 < T ? t1 - c0 : T);
+        load_tile_async<NTH>(sm + XQ, a.q + (base + c0) * DH, nv);
+        cp_async_commit();
+        build_dy(a.dout + (base + c0) * DH, a.o + (base + c0) * DH, a.den + base + c0, nv, sm + DY128, sm + DY32);
+        cp_async_wait_all();
+        publish_smem();
+        if (threadIdx.x == 0) {
+            fence_after_sync();
+            issue_proj(tm + agg_tmem::PROJ, sb + XQ, sb + WHI, sb + WLO);
+            mma_commit(&ctl->bar);
+        }
+        const float inv = 1.f / fmaxf(sqrtf(row_sqnorm(sm + XQ, r)), kNormEps);
+        if (!(ok = wait_mma(ctl, phase))) break;
+        features_half(tm, agg_tmem::PROJ, r, h, inv, a.beta, r < nv, sm + PHQ);
+        publish_smem();
+        if (threadIdx.x == 0) {
+            fence_after_sync();
+            issue_state_update(tm, agg_tmem::HTOP, agg_tmem::HBOT, sb + PHQ, sb + DY128, sb + DY32);
+            mma_commit(&ctl->bar);
+        }
+        ok = wait_mma(ctl, phase);
+    }
+    if (ok) {
+        float hv[80];
+        read_state_row(tm, h ? agg_tmem::HBOT : agg_tmem::HTOP, hv);
+        const int m = 128 * h + r;
+        float *dst = a.agg_out + (((int64_t)bh * a.nseg + seg) * MF + m) * DS;
+#pragma unroll
+        for (int c = 0; c < DS; ++c) dst[c] = hv[c];
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (threadIdx.x < 32) tmem_dealloc(tm, agg_tmem::NCOLS);
+}
+
+// ------------------------------------------------------------------------------------------
+// dq walk (chunks in order, prefix state H)
+// ------------------------------------------------------------------------------------------
+namespace bq_smem {
+constexpr uint32_t RA = 0;               // k rows at load; Phi_K [128][256] after the features
+constexpr uint32_t XK = RA;
+constexpr uint32_t PHK = RA;
+constexpr uint32_t RB = 4 * TILE;        // q rows + W at load; masked P; dP~ + W at the end
+constexpr uint32_t XQ = RB;
+constexpr uint32_t PB = RB;
+constexpr uint32_t DP = RB;
+constexpr uint32_t WHI = RB + TILE;
+constexpr uint32_t WLO = RB + TILE + 8192;
+constexpr uint32_t V = RB + 2 * TILE;
+constexpr uint32_t ONES = V + TILE;
+constexpr uint32_t DY128 = ONES + 4096;
+constexpr uint32_t DY32 = DY128 + TILE;
+constexpr uint32_t HS128 = DY32 + 4096;
+constexpr uint32_t HS32 = HS128 + 2 * TILE;
+constexpr uint32_t XCH = HS32 + 8192;
+constexpr uint32_t BAR = XCH + 1024;
+constexpr uint32_t TOTAL = BAR + 64;
+}  // namespace bq_smem
+namespace bq_tmem {
+constexpr uint32_t PROJ = 0;   // q 0..63, k 64..127
+constexpr uint32_t P = 0;      // [128][128]
+constexpr uint32_t DPHI = 0;   // [128][256]
+constexpr uint32_t DX = 0;     // [128][64]
+constexpr uint32_t HTOP = 256;
+constexpr uint32_t HBOT = 336;
+constexpr uint32_t NCOLS = 512;
+}  // namespace bq_tmem
+
+__global__ void __launch_bounds__(NTH, 1) tc_bwd_q_walk(BwdArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = aligned_base(smem_raw);
+    using namespace bq_smem;
+    Ctl *ctl = reinterpret_cast<Ctl *>(sm + BAR);
+    float *xch = reinterpret_cast<float *>(sm + XCH);
+    const int seg = blockIdx.x, bh = blockIdx.y;
+    const int r = threadIdx.x & 127, h = threadIdx.x >> 7;
+    const uint32_t sb = smem_u32(sm);
+    const bool causal = a.causal != 0;
+    if (threadIdx.x == 0) {
+        mbar_init(&ctl->bar, 1);
+        ctl->abort = 0;
+    }
+    if (threadIdx.x < 32) tmem_alloc(&ctl->tmem, bq_tmem::NCOLS);
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tm = ctl->tmem;
+    load_start_state(a.state + (int64_t)bh * a.nseg * MF * DS + seg * a.state_seg_stride, h, r, tm,
+                     bq_tmem::HTOP, bq_tmem::HBOT, sm + HS128, sm + HS32);
+    int64_t t0, t1;
+    bseg_bounds(a, seg, t0, t1);
+    const int64_t base = (int64_t)bh * a.N;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int64_t c0 = t0; c0 < t1 && ok; c0 += T) {
+        const int nv = (int)(t1 - c0 < T ? t1 - c0 : T);
+        const bool valid = r < nv;
+        load_tile_async<NTH>(sm + XQ, a.q + (base + c0) * DH, nv);
+        if (causal) {
+            load_tile_async<NTH>(sm + XK, a.k + (base + c0) * DH, nv);
+            load_tile_async<NTH>(sm + V, a.v + (base + c0) * DH, nv);
+        }
+        cp_async_commit();
+        load_w_split(a.W, sm + WHI, sm + WLO);
+        if (causal) write_ones(sm + ONES, nv);
+        build_dy(a.dout + (base + c0) * DH, a.o + (base + c0) * DH, a.den + base + c0, nv, sm + DY128, sm + DY32);
+        cp_async_wait_all();
+        publish_smem();
+        if (threadIdx.x == 0) {
+            fence_after_sync();
+            issue_proj(tm + bq_tmem::PROJ, sb + XQ, sb + WHI, sb + WLO);
+            if (causal) issue_proj(tm + bq_tmem::PROJ + 64, sb + XK, sb + WHI, sb + WLO);
+            mma_commit(&ctl->bar);
+        }
+        const float raw_q = sqrtf(row_sqnorm(sm + XQ, r));
+        const float inv_q = 1.f / fmaxf(raw_q, kNormEps);
+        const float inv_k = causal ? 1.f / fmaxf(sqrtf(row_sqnorm(sm + XK, r)), kNormEps) : 0.f;
+        if (!(ok = wait_mma(ctl, phase))) break;
+        float u[32], t[32];
+        features_half_keep(tm, bq_tmem::PROJ, r, h, inv_q, a.beta, valid, nullptr, u, t);
+        if (causal) features_half(tm, bq_tmem::PROJ + 64, r, h, inv_k, a.beta, valid, sm + PHK);
+        publish_smem();
+        if (causal) {
+            if (threadIdx.x == 0) {  // P = dY V~^T
+                fence_after_sync();
+                issue_k80(tm + bq_tmem::P, sb + DY128, sb + DY32, sb + V, sb + ONES, idesc_bf16(128, 128, 0, 0),
+                          false);
+                mma_commit(&ctl->bar);
+            }
+            if (!(ok = wait_mma(ctl, phase))) break;
+            mask_block_to_smem(tm, bq_tmem::P, r, h, false, sm + PB);
+            publish_smem();
+        }
+        if (threadIdx.x == 0) {
+            fence_after_sync();
+            // dPhi_Q = dY H_prev^T (+ tril(P) Phi_K)
+            issue_k80(tm + bq_tmem::DPHI, sb + DY128, sb + DY32, sb + HS128, sb + HS32, idesc_bf16(128, 256, 0, 0),
+                      false);
+            if (causal) {
+                issue_tt_times(tm + bq_tmem::DPHI, sb + PB, sb + PHK, idesc_bf16(128, 256, 0, 1), true);
+                issue_state_update(tm, bq_tmem::HTOP, bq_tmem::HBOT, sb + PHK, sb + V, sb + ONES);
+            }
+            mma_commit(&ctl->bar);
+        }
+        if (!(ok = wait_mma(ctl, phase))) break;
+        features_vjp_half(tm, bq_tmem::DPHI, r, h, a.beta, valid, u, t, sm + DP);
+        load_w_split(a.W, sm + WHI, sm + WLO);
+        publish_smem();
+        if (threadIdx.x == 0) {
+            fence_after_sync();
+            issue_dxhat(tm + bq_tmem::DX, sb + DP, sb + WHI, sb + WLO);
+            mma_commit(&ctl->bar);
+        }
+        if (!(ok = wait_mma(ctl, phase))) break;
+        write_dx(tm, bq_tmem::DX, r, h, valid, raw_q, a.q + (base + c0 + r) * DH, a.dq + (base + c0 + r) * DH, xch);
+        if (causal) {
+            float hv[80];
+            read_state_row(tm, h ? bq_tmem::HBOT : bq_tmem::HTOP, hv);
+            stage_state_row(hv, 128 * h + r, sm + HS128, sm + HS32);
+        }
+        publish_smem();
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (threadIdx.x < 32) tmem_dealloc(tm, bq_tmem::NCOLS);
+}
+
+// ------------------------------------------------------------------------------------------
+// dk/dv walk (chunks in reverse, suffix state G)
+// ------------------------------------------------------------------------------------------
+namespace bkv_smem {
+constexpr uint32_t PHQ = 0;              // q rows + W at load; Phi_Q; dP~ + W at the end
+constexpr uint32_t XQ = PHQ;
+constexpr uint32_t WHI0 = PHQ + 2 * TILE;
+constexpr uint32_t WLO0 = WHI0 + 8192;
+constexpr uint32_t DP = PHQ;
+constexpr uint32_t WHI1 = PHQ + TILE;
+constexpr uint32_t WLO1 = WHI1 + 8192;
+constexpr uint32_t PHK = PHQ + 4 * TILE; // k rows at load; Phi_K; then masked S^T and P'
+constexpr uint32_t XK = PHK;
+constexpr uint32_t STB = PHK;            // tiles 0-1
+constexpr uint32_t PPB = PHK + 2 * TILE; // tiles 2-3
+constexpr uint32_t V = PHK + 4 * TILE;
+constexpr uint32_t ONES = V + TILE;
+constexpr uint32_t DY128 = ONES + 4096;
+constexpr uint32_t DY32 = DY128 + TILE;
+constexpr uint32_t GS128 = DY32 + 4096;
+constexpr uint32_t GS32 = GS128 + 2 * TILE;
+constexpr uint32_t XCH = GS32 + 8192;
+constexpr uint32_t BAR = XCH + 1024;
+constexpr uint32_t TOTAL = BAR + 64;
+}  // namespace bkv_smem
+namespace bkv_tmem {
+constexpr uint32_t PROJ = 0;    // q 0..63, k 64..127
+constexpr uint32_t ST = 0;      // S^T [128][128]
+constexpr uint32_t PP = 128;    // P'  [128][128]
+constexpr uint32_t DPHI = 0;    // [128][256]
+constexpr uint32_t DX = 0;      // [128][64]
+constexpr uint32_t GTOP = 256;
+constexpr uint32_t GBOT = 336;
+constexpr uint32_t DVT = 416;   // dV~[:, :64]
+constexpr uint32_t NCOLS = 512;
+}  // namespace bkv_tmem
+
+__global__ void __launch_bounds__(NTH, 1) tc_bwd_kv_walk(BwdArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = aligned_base(smem_raw);
+    using namespace bkv_smem;
+    Ctl *ctl = reinterpret_cast<Ctl *>(sm + BAR);
+    float *xch = reinterpret_cast<float *>(sm + XCH);
+    const int seg = blockIdx.x, bh = blockIdx.y;
+    const int r = threadIdx.x & 127, h = threadIdx.x >> 7;
+    const uint32_t sb = smem_u32(sm);
+    const bool causal = a.causal != 0;
+    if (threadIdx.x == 0) {
+        mbar_init(&ctl->bar, 1);
+        ctl->abort = 0;
+    }
+    if (threadIdx.x < 32) tmem_alloc(&ctl->tmem, bkv_tmem::NCOLS);
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tm = ctl->tmem;
+    load_start_state(a.state + (int64_t)bh * a.nseg * MF * DS + seg * a.state_seg_stride, h, r, tm,
+                     bkv_tmem::GTOP, bkv_tmem::GBOT, sm + GS128, sm + GS32);
+    int64_t t0, t1;
+    bseg_bounds(a, seg, t0, t1);
+    const int64_t base = (int64_t)bh * a.N;
+    const int64_t nchunks = (t1 - t0 + T - 1) / T;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int64_t ci = nchunks - 1; ci >= 0 && ok; --ci) {
+        const int64_t c0 = t0 + ci * T;
+        const int nv = (int)(t1 - c0 < T ? t1 - c0 : T);
+        const bool valid = r < nv;
+        load_tile_async<NTH>(sm + XK, a.k + (base + c0) * DH, nv);
+        load_tile_async<NTH>(sm + V, a.v + (base + c0) * DH, nv);
+        if (causal) load_tile_async<NTH>(sm + XQ, a.q + (base + c0) * DH, nv);
+        cp_async_commit();
+        load_w_split(a.W, sm + WHI0, sm + WLO0);
+        write_ones(sm + ONES, nv);
+        if (causal)
+            build_dy(a.dout + (base + c0) * DH, a.o + (base + c0) * DH, a.den + base + c0, nv, sm + DY128,
+                     sm + DY32);
+        cp_async_wait_all();
+        publish_smem();
+        if (threadIdx.x == 0) {
+            fence_after_sync();
+            issue_proj(tm + bkv_tmem::PROJ + 64, sb + XK, sb + WHI0, sb + WLO0);
+            if (causal) issue_proj(tm + bkv_tmem::PROJ, sb + XQ, sb + WHI0, sb + WLO0);
+            mma_commit(&ctl->bar);
+        }
+        const float raw_k = sqrtf(row_sqnorm(sm + XK, r));
+        const float inv_k = 1.f / fmaxf(raw_k, kNormEps);
+        const float inv_q = causal ? 1.f / fmaxf(sqrtf(row_sqnorm(sm + XQ, r)), kNormEps) : 0.f;
+        if (!(ok = wait_mma(ctl, phase))) break;
+        float u[32], t[32];
+        features_half_keep(tm, bkv_tmem::PROJ + 64, r, h, inv_k, a.beta, valid, sm + PHK, u, t);
+        if (causal) features_half(tm, bkv_tmem::PROJ, r, h, inv_q, a.beta, valid, sm + PHQ);
+        publish_smem();
+        if (threadIdx.x == 0) {
+            fence_after_sync();
+            // dV~ = Phi_K G_next (value columns 0..63)
+            {
+                constexpr uint32_t id = idesc_bf16(128, 64, 0, 1);
+#pragma unroll
+                for (int kk = 0; kk < 16; ++kk)
+                    mma_bf16(tm + bkv_tmem::DVT, sdesc(sb + PHK + (kk >> 2) * TILE + (kk & 3) * 32, 16, 1024, LAYOUT_SW128),
+                             sdesc(sb + GS128 + kk * 2048, TILE, 1024, LAYOUT_SW128), id, kk > 0);
+            }
+            if (causal) {
+                // S^T = Phi_K Phi_Q^T ; P' = V~ dY^T
+                constexpr uint32_t id = idesc_bf16(128, 128, 0, 0);
+#pragma unroll
+                for (int kk = 0; kk < 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * TILE + (kk & 3) * 32;
+                    mma_bf16(tm + bkv_tmem::ST, sdesc(sb + PHK + off, 16, 1024, LAYOUT_SW128),
+                             sdesc(sb + PHQ + off, 16, 1024, LAYOUT_SW128), id, kk > 0);
+                }
+                issue_k80(tm + bkv_tmem::PP, sb + V, sb + ONES, sb + DY128, sb + DY32, id, false);
+            }
+            mma_commit(&ctl->bar);
+        }
+        if (!(ok = wait_mma(ctl, phase))) break;
+        if (causal) {
+            mask_block_to_smem(tm, bkv_tmem::ST, r, h, true, sm + STB);
+            mask_block_to_smem(tm, bkv_tmem::PP, r, h, true, sm + PPB);
+        }
+        publish_smem();
+        if (threadIdx.x == 0) {
+            fence_after_sync();
+            if (causal)  // dV~ += triu(S^T) dY
+                issue_tt_times(tm + bkv_tmem::DVT, sb + STB, sb + DY128, idesc_bf16(128, 64, 0, 1), true);
+            // dPhi_K = V~ G_next^T (+ triu(P') Phi_Q)
+            issue_k80(tm + bkv_tmem::DPHI, sb + V, sb + ONES, sb + GS128, sb + GS32, idesc_bf16(128, 256, 0, 0),
+                      false);
+            if (causal) {
+                issue_tt_times(tm + bkv_tmem::DPHI, sb + PPB, sb + PHQ, idesc_bf16(128, 256, 0, 1), true);
+                issue_state_update(tm, bkv_tmem::GTOP, bkv_tmem::GBOT, sb + PHQ, sb + DY128, sb + DY32);
+            }
+            mma_commit(&ctl->bar);
+        }
+        if (!(ok = wait_mma(ctl, phase))) break;
+        {  // dv = dV~[:, :64], columns 32h .. 32h+31 of row r (TMEM loads are warp-collective:
+           // every lane loads, only valid rows store)
+            float a0[16], a1[16];
+            const uint32_t ta = tm + (lane_base() << 16) + bkv_tmem::DVT + 32u * h;
+            tmem_ld16(ta, a0);
+            tmem_ld16(ta + 16, a1);
+            tmem_wait_ld();
+            if (valid) {
+            uint4 *d4 = reinterpret_cast<uint4 *>(a.dv + (base + c0 + r) * DH + 32 * h);
+            d4[0] = make_uint4(pack_bf16x2(a0[0], a0[1]), pack_bf16x2(a0[2], a0[3]), pack_bf16x2(a0[4], a0[5]),
+                               pack_bf16x2(a0[6], a0[7]));
+            d4[1] = make_uint4(pack_bf16x2(a0[8], a0[9]), pack_bf16x2(a0[10], a0[11]), pack_bf16x2(a0[12], a0[13]),
+                               pack_bf16x2(a0[14], a0[15]));
+            d4[2] = make_uint4(pack_bf16x2(a1[0], a1[1]), pack_bf16x2(a1[2], a1[3]), pack_bf16x2(a1[4], a1[5]),
+                               pack_bf16x2(a1[6], a1[7]));
+            d4[3] = make_uint4(pack_bf16x2(a1[8], a1[9]), pack_bf16x2(a1[10], a1[11]), pack_bf16x2(a1[12], a1[13]),
+                               pack_bf16x2(a1[14], a1[15]));
+            }
+        }
+        features_vjp_half(tm, bkv_tmem::DPHI, r, h, a.beta, valid, u, t, sm + DP);
+        load_w_split(a.W, sm + WHI1, sm + WLO1);
+        publish_smem();
+        if (threadIdx.x == 0) {
+            fence_after_sync();
+            issue_dxhat(tm + bkv_tmem::DX, sb + DP, sb + WHI1, sb + WLO1);
+            mma_commit(&ctl->bar);
+        }
+        if (!(ok = wait_mma(ctl, phase))) break;
+        write_dx(tm, bkv_tmem::DX, r, h, valid, raw_k, a.k + (base + c0 + r) * DH, a.dk + (base + c0 + r) * DH, xch);
+        if (causal) {
+            float hv[80];
+            read_state_row(tm, h ? bkv_tmem::GBOT : bkv_tmem::GTOP, hv);
+            stage_state_row(hv, 128 * h + r, sm + GS128, sm + GS32);
+        }
+        publish_smem();
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (threadIdx.x < 32) tmem_dealloc(tm, bkv_tmem::NCOLS);
+}
+
 // ---- host side ---------------------------------------------------------------------------
 
 inline bool fast_path_ok(race_dtype_t dtype, int d, int L, int P, float tau)
