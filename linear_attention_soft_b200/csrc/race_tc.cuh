@@ -550,14 +550,22 @@ __global__ void __launch_bounds__(NTH, 1) tc_fwd_walk(Args a)
 }
 
 // ==========================================================================================
-// Backward.  With dY_i = [dO_i / den_i, -(dO_i . o_i) / den_i] (80 columns, 15 zero):
-//   dq side (prefix state H):   dPhi_Q = dY H_prev^T + tril(dY V~^T) Phi_K,   H += Phi_K^T V~
-//   dk/dv side (suffix state G, chunks walked backwards):
-//     dV~   = Phi_K G_next + triu(Phi_K Phi_Q^T) dY          (dv = dV~[:, :64])
-//     dPhi_K = V~ G_next^T + triu(V~ dY^T) Phi_Q,              G += Phi_Q^T dY
+// Backward.  With c_i = -(dO_i . o_i) and dY_i = [dO_i, c_i] / den_i (the gradient of
+// out_i = Y_i[:64] / Y_i[64] with respect to Y_i):
+//   dq side (prefix state H, chunks in order):
+//     dPhi_Q[i] = (dO_i H_prev[:, :64]^T + c_i H_prev[:, 64] + sum_{j<=i} (v_j.dO_i + c_i) Phi_K[j]) / den_i
+//     H += Phi_K^T [V | 1]
+//   dk/dv side (suffix state G = sum_i Phi_Q[i] dY_i^T, chunks walked backwards), with
+//   Phi_Q' = Phi_Q / den (row-scaled):
+//     dV[j]     = Phi_K[j] G_next[:, :64] + sum_{i>=j} (Phi_K[j].Phi_Q'[i]) dO_i
+//     dPhi_K[j] = [v_j, 1] G_next^T + sum_{i>=j} (v_j.dO_i + c_i) Phi_Q'[i]
+//     G += Phi_Q'^T [dO | c]
 //   feature-map VJP per table (CUDA cores): dz = phi (dphi - phi.dphi),
 //   du_p = beta sum_r c_rp dz_r, dp~ = du (1 - u^2); then dX^ = dP~ W (tcgen05) and
 //   dx = (dX^ - x^ (x^ . dX^)) / |x|.
+// The terms v_j.dO_i and c_i nearly cancel when o_i is close to v_j (short prefixes), so
+// they are formed in fp32 from exact bf16 inputs (dO, v), with c_i added in fp32, and the
+// dq side reads the state as a bf16 hi + lo pair.
 // ==========================================================================================
 
 struct BwdArgs {
@@ -573,70 +581,69 @@ struct BwdArgs {
     int causal;
 };
 
-// dY rows [0, nvalid) into DY128 ([128][64] SW128: dO/den) and DY32 ([128][16] SW32:
-// column 0 = -(dO.o)/den); zero rows beyond.  Threads 0..127 each build one row.
-__device__ __forceinline__ void build_dy(const __nv_bfloat16 *dout, const __nv_bfloat16 *o,
-                                         const float *den, int nvalid, uint8_t *dy128, uint8_t *dy32)
+// Per-row scalars of a chunk: rowc[r] = c_r = -(dO_r . o_r), rowinv[r] = 1/den_r (0 beyond
+// nvalid); dO read from its SW128 tile, o from global.  Optionally the SW32 block dc32
+// gets c_r (bf16) in column 0.  Threads 0..127, one row each.
+__device__ __forceinline__ void row_scalars(const uint8_t *do_tile, const __nv_bfloat16 *o, const float *den,
+                                            int nvalid, float *rowc, float *rowinv, uint8_t *dc32)
 {
     if (threadIdx.x >= T) return;
     const int r = threadIdx.x;
-    const uint32_t b128 = smem_u32(dy128), b32 = smem_u32(dy32);
-    if (r >= nvalid) {
+    float c = 0.f, inv = 0.f;
+    if (r < nvalid) {
+        const uint32_t a = smem_u32(do_tile);
+        const uint4 *o4 = reinterpret_cast<const uint4 *>(o + (int64_t)r * DH);
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) st_shared_v4(b128 + sw128_off(r, ch), 0u, 0u, 0u, 0u);
-        st_shared_v4(b32 + sw32_off(r, 0), 0u, 0u, 0u, 0u);
-        st_shared_v4(b32 + sw32_off(r, 1), 0u, 0u, 0u, 0u);
-        return;
-    }
-    const float dn = den[r];
-    const float inv = dn != 0.f ? 1.f / dn : 0.f;
-    const uint4 *g4 = reinterpret_cast<const uint4 *>(dout + (int64_t)r * DH);
-    const uint4 *o4 = reinterpret_cast<const uint4 *>(o + (int64_t)r * DH);
-    float dot = 0.f;
+        for (int ch = 0; ch < 8; ++ch) {
+            const uint4 g = ld_shared_v4(a + sw128_off(r, ch)), ov = o4[ch];
+            const uint32_t gw[4] = {g.x, g.y, g.z, g.w}, ow[4] = {ov.x, ov.y, ov.z, ov.w};
 #pragma unroll
-    for (int ch = 0; ch < 8; ++ch) {
-        const uint4 g = g4[ch], ov = o4[ch];
-        const uint32_t gw[4] = {g.x, g.y, g.z, g.w}, ow[4] = {ov.x, ov.y, ov.z, ov.w};
-        uint32_t w[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float g0 = bf16_lo(gw[i]), g1 = bf16_hi(gw[i]);
-            dot = fmaf(g0, bf16_lo(ow[i]), dot);
-            dot = fmaf(g1, bf16_hi(ow[i]), dot);
-            w[i] = pack_bf16x2(g0 * inv, g1 * inv);
+            for (int i = 0; i < 4; ++i) {
+                c = fmaf(bf16_lo(gw[i]), bf16_lo(ow[i]), c);
+                c = fmaf(bf16_hi(gw[i]), bf16_hi(ow[i]), c);
+            }
         }
-        st_shared_v4(b128 + sw128_off(r, ch), w[0], w[1], w[2], w[3]);
+        c = -c;
+        const float dn = den[r];
+        inv = dn != 0.f ? 1.f / dn : 0.f;
     }
-    st_shared_v4(b32 + sw32_off(r, 0), pack_bf16x2(-dot * inv, 0.f), 0u, 0u, 0u);
-    st_shared_v4(b32 + sw32_off(r, 1), 0u, 0u, 0u, 0u);
+    rowc[r] = c;
+    rowinv[r] = inv;
+    if (dc32) {
+        const uint32_t b = smem_u32(dc32);
+        st_shared_v4(b + sw32_off(r, 0), pack_bf16x2(c, 0.f), 0u, 0u, 0u);
+        st_shared_v4(b + sw32_off(r, 1), 0u, 0u, 0u, 0u);
+    }
 }
 
-// Like features_half, keeping u = tanh(proj/|x|) and t = tanh(beta u) of the 32
-// projections (8 tables) in registers for the feature-map VJP; phi may be null.
-__device__ __forceinline__ void features_half_keep(uint32_t tmem, uint32_t col0, int r, int h, float inv_norm,
-                                                   float beta, bool valid, uint8_t *phi, float (&u)[32],
-                                                   float (&t)[32])
+// u = tanh(proj / |x|) and t = tanh(beta u) of the 32 projections of half h (8 tables),
+// kept in registers for the feature-map VJP.
+__device__ __forceinline__ void proj_keep(uint32_t tmem, uint32_t col0, int h, float inv_norm, float beta,
+                                          float (&u)[32], float (&t)[32])
 {
-    {
-        float a[16], b[16];
-        const uint32_t ta = tmem + (lane_base() << 16) + col0 + 32u * h;
-        tmem_ld16(ta, a);
-        tmem_ld16(ta + 16, b);
-        tmem_wait_ld();
+    float a[16], b[16];
+    const uint32_t ta = tmem + (lane_base() << 16) + col0 + 32u * h;
+    tmem_ld16(ta, a);
+    tmem_ld16(ta + 16, b);
+    tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            u[i] = tanh_fast(a[i] * inv_norm);
-            u[16 + i] = tanh_fast(b[i] * inv_norm);
-        }
-#pragma unroll
-        for (int i = 0; i < 32; ++i) t[i] = tanh_fast(beta * u[i]);
+    for (int i = 0; i < 16; ++i) {
+        u[i] = tanh_fast(a[i] * inv_norm);
+        u[16 + i] = tanh_fast(b[i] * inv_norm);
     }
-    if (!phi) return;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) t[i] = tanh_fast(beta * u[i]);
+}
+
+// Features of the 8 tables of half h from t = tanh(beta u), times `scale`, as bf16 into row r
+// of the Phi tile [128][256].
+__device__ __forceinline__ void write_features(const float (&t)[32], int r, int h, float scale, uint8_t *phi)
+{
     const uint32_t base = smem_u32(phi);
 #pragma unroll
     for (int l = 0; l < 8; ++l) {
         float f[16];
-        f[0] = 1.f;
+        f[0] = scale;
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
             const float s1 = 0.5f + 0.5f * t[4 * l + p], s0 = 0.5f - 0.5f * t[4 * l + p];
@@ -647,22 +654,23 @@ __device__ __forceinline__ void features_half_keep(uint32_t tmem, uint32_t col0,
                 f[c] *= s0;
             }
         }
-        uint32_t w[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) w[i] = valid ? pack_bf16x2(f[2 * i], f[2 * i + 1]) : 0u;
         const int tl = 8 * h + l;
         const uint32_t blk = base + (uint32_t)(tl >> 2) * TILE;
         const int ch = (tl & 3) * 2;
-        st_shared_v4(blk + sw128_off(r, ch), w[0], w[1], w[2], w[3]);
-        st_shared_v4(blk + sw128_off(r, ch + 1), w[4], w[5], w[6], w[7]);
+        st_shared_v4(blk + sw128_off(r, ch), pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                     pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+        st_shared_v4(blk + sw128_off(r, ch + 1), pack_bf16x2(f[8], f[9]), pack_bf16x2(f[10], f[11]),
+                     pack_bf16x2(f[12], f[13]), pack_bf16x2(f[14], f[15]));
     }
 }
 
-// Feature-map VJP for the 8 tables of half h: dphi from TMEM columns col0 + 128h .. (16 per
-// table), u and t from features_half_keep; writes dp~ (32 values) as bf16 into row r of
-// the DP tile ([128][64] SW128, projections 32h .. 32h+31).
+// Feature-map VJP for the 8 tables of half h.  dphi[m] = (D[m] + add_scale * add_vec[m]) * mul
+// with D read from TMEM columns col0 + 128h .. (16 per table) and add_vec (features, fp32,
+// shared memory) optional; writes dp~ (32 values) as bf16 into row r of the DP tile
+// ([128][64] SW128, projections 32h .. 32h+31).
 __device__ __forceinline__ void features_vjp_half(uint32_t tmem, uint32_t col0, int r, int h, float beta,
                                                   bool valid, const float (&u)[32], const float (&t)[32],
+                                                  const float *add_vec, float add_scale, float mul,
                                                   uint8_t *dp_tile)
 {
     float dp[32];
@@ -672,6 +680,11 @@ __device__ __forceinline__ void features_vjp_half(uint32_t tmem, uint32_t col0, 
         float g[16];
         tmem_ld16(ta + 16 * l, g);
         tmem_wait_ld();
+        if (add_vec) {
+            const float *av = add_vec + 128 * h + 16 * l;
+#pragma unroll
+            for (int c = 0; c < 16; ++c) g[c] = fmaf(add_scale, av[c], g[c]) * mul;
+        }
         float f[16];
         f[0] = 1.f;
 #pragma unroll
@@ -720,14 +733,20 @@ __device__ __forceinline__ void issue_dxhat(uint32_t d, uint32_t dp, uint32_t wh
     }
 }
 
+// D[128][N] (+)= A[128][64] B[N][64]^T, both K-major SW128.
+__device__ __forceinline__ void issue_k64(uint32_t d, uint32_t a, uint32_t b, uint32_t idesc, bool acc_first)
+{
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+        mma_bf16(d, sdesc(a + kk * 32, 16, 1024, LAYOUT_SW128), sdesc(b + kk * 32, 16, 1024, LAYOUT_SW128), idesc,
+                 (kk > 0 || acc_first) ? 1u : 0u);
+}
+
 // D[128][N] (+)= A[128][80] B[N][80]^T, both K-major, K split as 64 (SW128) + 16 (SW32).
 __device__ __forceinline__ void issue_k80(uint32_t d, uint32_t a128, uint32_t a32, uint32_t b128, uint32_t b32,
                                           uint32_t idesc, bool acc_first)
 {
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(d, sdesc(a128 + kk * 32, 16, 1024, LAYOUT_SW128), sdesc(b128 + kk * 32, 16, 1024, LAYOUT_SW128),
-                 idesc, (kk > 0 || acc_first) ? 1u : 0u);
+    issue_k64(d, a128, b128, idesc, acc_first);
     mma_bf16(d, sdesc(a32, 16, 256, LAYOUT_SW32), sdesc(b32, 16, 256, LAYOUT_SW32), idesc, 1u);
 }
 
@@ -742,9 +761,10 @@ __device__ __forceinline__ void issue_tt_times(uint32_t d, uint32_t a, uint32_t 
 }
 
 // Masked T x T block from TMEM (row r, columns col0 + 64h ..) to bf16 K-major tile h of dst.
-// keep_upper: keep column >= row (else column <= row).
+// Adds add_row to every element of the row and add_col[col] per column (either optional)
+// before masking; keep_upper keeps column >= row (else column <= row).
 __device__ __forceinline__ void mask_block_to_smem(uint32_t tmem, uint32_t col0, int r, int h, bool keep_upper,
-                                                   uint8_t *dst)
+                                                   float add_row, const float *add_col, uint8_t *dst)
 {
     const uint32_t t = tmem + (lane_base() << 16) + col0 + 64u * h;
     const uint32_t blk = smem_u32(dst) + (uint32_t)h * TILE;
@@ -756,7 +776,9 @@ __device__ __forceinline__ void mask_block_to_smem(uint32_t tmem, uint32_t col0,
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             const int col = 64 * h + 16 * c + i;
-            if (keep_upper ? (col < r) : (col > r)) x[i] = 0.f;
+            float y = x[i] + add_row;
+            if (add_col) y += add_col[col];
+            x[i] = (keep_upper ? (col < r) : (col > r)) ? 0.f : y;
         }
         st_shared_v4(blk + sw128_off(r, 2 * c), pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]),
                      pack_bf16x2(x[4], x[5]), pack_bf16x2(x[6], x[7]));
@@ -824,14 +846,33 @@ __device__ __forceinline__ void bseg_bounds(const BwdArgs &a, int seg, int64_t &
     if (t1 > a.N) t1 = a.N;
 }
 
-// Load a walk's start state (global fp32 [256][65] rows) into TMEM (two halves) and into
-// the bf16 staging tiles.
-__device__ __forceinline__ void load_start_state(const float *src_all, int h, int r, uint32_t tm, uint32_t htop,
-                                                 uint32_t hbot, uint8_t *s128, uint8_t *s32)
+// Stage one state row (feature m) as a bf16 hi + lo pair of [256][64] SW128 tiles plus its
+// ones column in fp32.
+__device__ __forceinline__ void stage_state_hilo(const float (&hv)[80], int m, uint8_t *hi, uint8_t *lo, float *col64)
 {
-    const int m = 128 * h + r;
-    const float *src = src_all + (int64_t)m * DS;
-    float hv[80];
+    const uint32_t bh_ = smem_u32(hi) + (uint32_t)(m >> 7) * TILE, bl = smem_u32(lo) + (uint32_t)(m >> 7) * TILE;
+    const int rr = m & 127;
+#pragma unroll
+    for (int ch = 0; ch < 8; ++ch) {
+        uint32_t wh[4], wl[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float x0 = hv[8 * ch + 2 * i], x1 = hv[8 * ch + 2 * i + 1];
+            wh[i] = pack_bf16x2(x0, x1);
+            wl[i] = pack_bf16x2(x0 - bf16_lo(wh[i]), x1 - bf16_hi(wh[i]));
+        }
+        st_shared_v4(bh_ + sw128_off(rr, ch), wh[0], wh[1], wh[2], wh[3]);
+        st_shared_v4(bl + sw128_off(rr, ch), wl[0], wl[1], wl[2], wl[3]);
+    }
+    col64[m] = hv[64];
+}
+
+// A walk's start state row (global fp32 [256][65]) for feature m = 128h + r -> registers,
+// then into TMEM (the half's columns).
+__device__ __forceinline__ void load_start_row(const float *src_all, int h, int r, uint32_t tm, uint32_t htop,
+                                               uint32_t hbot, float (&hv)[80])
+{
+    const float *src = src_all + (int64_t)(128 * h + r) * DS;
 #pragma unroll
     for (int c = 0; c < 80; ++c) hv[c] = c < DS ? src[c] : 0.f;
     const uint32_t t = tm + (lane_base() << 16) + (h ? hbot : htop);
@@ -843,20 +884,22 @@ __device__ __forceinline__ void load_start_state(const float *src_all, int h, in
         tmem_st16(t + 16 * c, x);
     }
     tmem_wait_st();
-    stage_state_row(hv, m, s128, s32);
 }
 
 // ------------------------------------------------------------------------------------------
-// Segment totals of the backward's key side: G_seg = sum_{i in segment} phi(q_i) dY_i^T
+// Segment totals of the backward's key side: G_seg = sum_{i in segment} phi(q_i) dY_i^T,
+// formed as Phi_Q'^T [dO | c] with Phi_Q' = Phi_Q / den.
 // ------------------------------------------------------------------------------------------
 namespace aggq_smem {
 constexpr uint32_t PHQ = 0;
 constexpr uint32_t XQ = PHQ;
-constexpr uint32_t DY128 = PHQ + 4 * TILE;
-constexpr uint32_t DY32 = DY128 + TILE;
-constexpr uint32_t WHI = DY32 + 4096;
+constexpr uint32_t DO = PHQ + 4 * TILE;
+constexpr uint32_t DC32 = DO + TILE;
+constexpr uint32_t WHI = DC32 + 4096;
 constexpr uint32_t WLO = WHI + 8192;
-constexpr uint32_t BAR = WLO + 8192;
+constexpr uint32_t ROWC = WLO + 8192;
+constexpr uint32_t ROWINV = ROWC + 512;
+constexpr uint32_t BAR = ROWINV + 512;
 constexpr uint32_t TOTAL = BAR + 64;
 }  // namespace aggq_smem
 
@@ -866,6 +909,7 @@ __global__ void __launch_bounds__(NTH, 2) tc_agg_qdy(BwdArgs a)
     uint8_t *sm = aligned_base(smem_raw);
     using namespace aggq_smem;
     Ctl *ctl = reinterpret_cast<Ctl *>(sm + BAR);
+    float *rowc = reinterpret_cast<float *>(sm + ROWC), *rowinv = reinterpret_cast<float *>(sm + ROWINV);
     const int seg = blockIdx.x, bh = blockIdx.y;
     const int r = threadIdx.x & 127, h = threadIdx.x >> 7;
     const uint32_t sb = smem_u32(sm);
@@ -896,9 +940,11 @@ __global__ void __launch_bounds__(NTH, 2) tc_agg_qdy(BwdArgs a)
     for (int64_t c0 = t0; c0 < t1 && ok; c0 += T) {
         const int nv = (int)(t1 - c0 < T ? t1 - c0 : T);
         load_tile_async<NTH>(sm + XQ, a.q + (base + c0) * DH, nv);
+        load_tile_async<NTH>(sm + DO, a.dout + (base + c0) * DH, nv);
         cp_async_commit();
-        build_dy(a.dout + (base + c0) * DH, a.o + (base + c0) * DH, a.den + base + c0, nv, sm + DY128, sm + DY32);
         cp_async_wait_all();
+        __syncthreads();
+        row_scalars(sm + DO, a.o + (base + c0) * DH, a.den + base + c0, nv, rowc, rowinv, sm + DC32);
         publish_smem();
         if (threadIdx.x == 0) {
             fence_after_sync();
@@ -907,11 +953,15 @@ __global__ void __launch_bounds__(NTH, 2) tc_agg_qdy(BwdArgs a)
         }
         const float inv = 1.f / fmaxf(sqrtf(row_sqnorm(sm + XQ, r)), kNormEps);
         if (!(ok = wait_mma(ctl, phase))) break;
-        features_half(tm, agg_tmem::PROJ, r, h, inv, a.beta, r < nv, sm + PHQ);
+        {
+            float u[32], t[32];
+            proj_keep(tm, agg_tmem::PROJ, h, inv, a.beta, u, t);
+            write_features(t, r, h, r < nv ? rowinv[r] : 0.f, sm + PHQ);
+        }
         publish_smem();
         if (threadIdx.x == 0) {
             fence_after_sync();
-            issue_state_update(tm, agg_tmem::HTOP, agg_tmem::HBOT, sb + PHQ, sb + DY128, sb + DY32);
+            issue_state_update(tm, agg_tmem::HTOP, agg_tmem::HBOT, sb + PHQ, sb + DO, sb + DC32);
             mma_commit(&ctl->bar);
         }
         ok = wait_mma(ctl, phase);
@@ -936,7 +986,7 @@ namespace bq_smem {
 constexpr uint32_t RA = 0;               // k rows at load; Phi_K [128][256] after the features
 constexpr uint32_t XK = RA;
 constexpr uint32_t PHK = RA;
-constexpr uint32_t RB = 4 * TILE;        // q rows + W at load; masked P; dP~ + W at the end
+constexpr uint32_t RB = 4 * TILE;        // q rows + W at load; masked P''; dP~ + W at the end
 constexpr uint32_t XQ = RB;
 constexpr uint32_t PB = RB;
 constexpr uint32_t DP = RB;
@@ -944,11 +994,13 @@ constexpr uint32_t WHI = RB + TILE;
 constexpr uint32_t WLO = RB + TILE + 8192;
 constexpr uint32_t V = RB + 2 * TILE;
 constexpr uint32_t ONES = V + TILE;
-constexpr uint32_t DY128 = ONES + 4096;
-constexpr uint32_t DY32 = DY128 + TILE;
-constexpr uint32_t HS128 = DY32 + 4096;
-constexpr uint32_t HS32 = HS128 + 2 * TILE;
-constexpr uint32_t XCH = HS32 + 8192;
+constexpr uint32_t DO = ONES + 4096;     // dO rows [128][64]
+constexpr uint32_t HSHI = DO + TILE;     // staged H[:, :64], bf16 hi  [256][64]
+constexpr uint32_t HSLO = HSHI + 2 * TILE;  // and lo
+constexpr uint32_t HDEN = HSLO + 2 * TILE;  // H[:, 64] fp32 [256]
+constexpr uint32_t ROWC = HDEN + 1024;
+constexpr uint32_t ROWINV = ROWC + 512;
+constexpr uint32_t XCH = ROWINV + 512;
 constexpr uint32_t BAR = XCH + 1024;
 constexpr uint32_t TOTAL = BAR + 64;
 }  // namespace bq_smem
@@ -968,7 +1020,8 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_q_walk(BwdArgs a)
     uint8_t *sm = aligned_base(smem_raw);
     using namespace bq_smem;
     Ctl *ctl = reinterpret_cast<Ctl *>(sm + BAR);
-    float *xch = reinterpret_cast<float *>(sm + XCH);
+    float *xch = reinterpret_cast<float *>(sm + XCH), *hden = reinterpret_cast<float *>(sm + HDEN);
+    float *rowc = reinterpret_cast<float *>(sm + ROWC), *rowinv = reinterpret_cast<float *>(sm + ROWINV);
     const int seg = blockIdx.x, bh = blockIdx.y;
     const int r = threadIdx.x & 127, h = threadIdx.x >> 7;
     const uint32_t sb = smem_u32(sm);
@@ -982,8 +1035,12 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_q_walk(BwdArgs a)
     __syncthreads();
     fence_after_sync();
     const uint32_t tm = ctl->tmem;
-    load_start_state(a.state + (int64_t)bh * a.nseg * MF * DS + seg * a.state_seg_stride, h, r, tm,
-                     bq_tmem::HTOP, bq_tmem::HBOT, sm + HS128, sm + HS32);
+    {
+        float hv[80];
+        load_start_row(a.state + (int64_t)bh * a.nseg * MF * DS + seg * a.state_seg_stride, h, r, tm,
+                       bq_tmem::HTOP, bq_tmem::HBOT, hv);
+        stage_state_hilo(hv, 128 * h + r, sm + HSHI, sm + HSLO, hden);
+    }
     int64_t t0, t1;
     bseg_bounds(a, seg, t0, t1);
     const int64_t base = (int64_t)bh * a.N;
@@ -993,6 +1050,7 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_q_walk(BwdArgs a)
         const int nv = (int)(t1 - c0 < T ? t1 - c0 : T);
         const bool valid = r < nv;
         load_tile_async<NTH>(sm + XQ, a.q + (base + c0) * DH, nv);
+        load_tile_async<NTH>(sm + DO, a.dout + (base + c0) * DH, nv);
         if (causal) {
             load_tile_async<NTH>(sm + XK, a.k + (base + c0) * DH, nv);
             load_tile_async<NTH>(sm + V, a.v + (base + c0) * DH, nv);
@@ -1000,8 +1058,9 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_q_walk(BwdArgs a)
         cp_async_commit();
         load_w_split(a.W, sm + WHI, sm + WLO);
         if (causal) write_ones(sm + ONES, nv);
-        build_dy(a.dout + (base + c0) * DH, a.o + (base + c0) * DH, a.den + base + c0, nv, sm + DY128, sm + DY32);
         cp_async_wait_all();
+        __syncthreads();
+        row_scalars(sm + DO, a.o + (base + c0) * DH, a.den + base + c0, nv, rowc, rowinv, nullptr);
         publish_smem();
         if (threadIdx.x == 0) {
             fence_after_sync();
@@ -1012,27 +1071,27 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_q_walk(BwdArgs a)
         const float raw_q = sqrtf(row_sqnorm(sm + XQ, r));
         const float inv_q = 1.f / fmaxf(raw_q, kNormEps);
         const float inv_k = causal ? 1.f / fmaxf(sqrtf(row_sqnorm(sm + XK, r)), kNormEps) : 0.f;
+        const float c_r = rowc[r], invden_r = rowinv[r];
         if (!(ok = wait_mma(ctl, phase))) break;
         float u[32], t[32];
-        features_half_keep(tm, bq_tmem::PROJ, r, h, inv_q, a.beta, valid, nullptr, u, t);
+        proj_keep(tm, bq_tmem::PROJ, h, inv_q, a.beta, u, t);
         if (causal) features_half(tm, bq_tmem::PROJ + 64, r, h, inv_k, a.beta, valid, sm + PHK);
         publish_smem();
         if (causal) {
-            if (threadIdx.x == 0) {  // P = dY V~^T
+            if (threadIdx.x == 0) {  // P'' = dO V^T
                 fence_after_sync();
-                issue_k80(tm + bq_tmem::P, sb + DY128, sb + DY32, sb + V, sb + ONES, idesc_bf16(128, 128, 0, 0),
-                          false);
+                issue_k64(tm + bq_tmem::P, sb + DO, sb + V, idesc_bf16(128, 128, 0, 0), false);
                 mma_commit(&ctl->bar);
             }
             if (!(ok = wait_mma(ctl, phase))) break;
-            mask_block_to_smem(tm, bq_tmem::P, r, h, false, sm + PB);
+            mask_block_to_smem(tm, bq_tmem::P, r, h, false, c_r, nullptr, sm + PB);  // v_j.dO_i + c_i, j <= i
             publish_smem();
         }
         if (threadIdx.x == 0) {
             fence_after_sync();
-            // dPhi_Q = dY H_prev^T (+ tril(P) Phi_K)
-            issue_k80(tm + bq_tmem::DPHI, sb + DY128, sb + DY32, sb + HS128, sb + HS32, idesc_bf16(128, 256, 0, 0),
-                      false);
+            // D = dO H_prev[:, :64]^T (+ tril(P'') Phi_K)
+            issue_k64(tm + bq_tmem::DPHI, sb + DO, sb + HSHI, idesc_bf16(128, 256, 0, 0), false);
+            issue_k64(tm + bq_tmem::DPHI, sb + DO, sb + HSLO, idesc_bf16(128, 256, 0, 0), true);
             if (causal) {
                 issue_tt_times(tm + bq_tmem::DPHI, sb + PB, sb + PHK, idesc_bf16(128, 256, 0, 1), true);
                 issue_state_update(tm, bq_tmem::HTOP, bq_tmem::HBOT, sb + PHK, sb + V, sb + ONES);
@@ -1040,7 +1099,8 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_q_walk(BwdArgs a)
             mma_commit(&ctl->bar);
         }
         if (!(ok = wait_mma(ctl, phase))) break;
-        features_vjp_half(tm, bq_tmem::DPHI, r, h, a.beta, valid, u, t, sm + DP);
+        // dphi = (D + c_i H_prev[:, 64]) / den_i
+        features_vjp_half(tm, bq_tmem::DPHI, r, h, a.beta, valid, u, t, hden, c_r, invden_r, sm + DP);
         load_w_split(a.W, sm + WHI, sm + WLO);
         publish_smem();
         if (threadIdx.x == 0) {
@@ -1053,7 +1113,7 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_q_walk(BwdArgs a)
         if (causal) {
             float hv[80];
             read_state_row(tm, h ? bq_tmem::HBOT : bq_tmem::HTOP, hv);
-            stage_state_row(hv, 128 * h + r, sm + HS128, sm + HS32);
+            stage_state_hilo(hv, 128 * h + r, sm + HSHI, sm + HSLO, hden);
         }
         publish_smem();
     }
@@ -1066,36 +1126,38 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_q_walk(BwdArgs a)
 // dk/dv walk (chunks in reverse, suffix state G)
 // ------------------------------------------------------------------------------------------
 namespace bkv_smem {
-constexpr uint32_t PHQ = 0;              // q rows + W at load; Phi_Q; dP~ + W at the end
+constexpr uint32_t PHQ = 0;              // q rows + W at load; Phi_Q'; dP~ + W at the end
 constexpr uint32_t XQ = PHQ;
 constexpr uint32_t WHI0 = PHQ + 2 * TILE;
 constexpr uint32_t WLO0 = WHI0 + 8192;
 constexpr uint32_t DP = PHQ;
 constexpr uint32_t WHI1 = PHQ + TILE;
 constexpr uint32_t WLO1 = WHI1 + 8192;
-constexpr uint32_t PHK = PHQ + 4 * TILE; // k rows at load; Phi_K; then masked S^T and P'
+constexpr uint32_t PHK = PHQ + 4 * TILE; // k rows at load; Phi_K; then masked S'^T and P'
 constexpr uint32_t XK = PHK;
 constexpr uint32_t STB = PHK;            // tiles 0-1
 constexpr uint32_t PPB = PHK + 2 * TILE; // tiles 2-3
 constexpr uint32_t V = PHK + 4 * TILE;
 constexpr uint32_t ONES = V + TILE;
-constexpr uint32_t DY128 = ONES + 4096;
-constexpr uint32_t DY32 = DY128 + TILE;
-constexpr uint32_t GS128 = DY32 + 4096;
+constexpr uint32_t DO = ONES + 4096;     // dO rows [128][64]
+constexpr uint32_t DC32 = DO + TILE;     // c in column 0, [128][16] SW32
+constexpr uint32_t GS128 = DC32 + 4096;
 constexpr uint32_t GS32 = GS128 + 2 * TILE;
-constexpr uint32_t XCH = GS32 + 8192;
+constexpr uint32_t ROWC = GS32 + 8192;
+constexpr uint32_t ROWINV = ROWC + 512;
+constexpr uint32_t XCH = ROWINV + 512;
 constexpr uint32_t BAR = XCH + 1024;
 constexpr uint32_t TOTAL = BAR + 64;
 }  // namespace bkv_smem
 namespace bkv_tmem {
 constexpr uint32_t PROJ = 0;    // q 0..63, k 64..127
-constexpr uint32_t ST = 0;      // S^T [128][128]
-constexpr uint32_t PP = 128;    // P'  [128][128]
+constexpr uint32_t ST = 0;      // S'^T [128][128]
+constexpr uint32_t PP = 128;    // V dO^T [128][128]
 constexpr uint32_t DPHI = 0;    // [128][256]
 constexpr uint32_t DX = 0;      // [128][64]
 constexpr uint32_t GTOP = 256;
 constexpr uint32_t GBOT = 336;
-constexpr uint32_t DVT = 416;   // dV~[:, :64]
+constexpr uint32_t DVT = 416;   // dV [128][64]
 constexpr uint32_t NCOLS = 512;
 }  // namespace bkv_tmem
 
@@ -1106,6 +1168,7 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_kv_walk(BwdArgs a)
     using namespace bkv_smem;
     Ctl *ctl = reinterpret_cast<Ctl *>(sm + BAR);
     float *xch = reinterpret_cast<float *>(sm + XCH);
+    float *rowc = reinterpret_cast<float *>(sm + ROWC), *rowinv = reinterpret_cast<float *>(sm + ROWINV);
     const int seg = blockIdx.x, bh = blockIdx.y;
     const int r = threadIdx.x & 127, h = threadIdx.x >> 7;
     const uint32_t sb = smem_u32(sm);
@@ -1119,8 +1182,12 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_kv_walk(BwdArgs a)
     __syncthreads();
     fence_after_sync();
     const uint32_t tm = ctl->tmem;
-    load_start_state(a.state + (int64_t)bh * a.nseg * MF * DS + seg * a.state_seg_stride, h, r, tm,
-                     bkv_tmem::GTOP, bkv_tmem::GBOT, sm + GS128, sm + GS32);
+    {
+        float hv[80];
+        load_start_row(a.state + (int64_t)bh * a.nseg * MF * DS + seg * a.state_seg_stride, h, r, tm,
+                       bkv_tmem::GTOP, bkv_tmem::GBOT, hv);
+        stage_state_row(hv, 128 * h + r, sm + GS128, sm + GS32);
+    }
     int64_t t0, t1;
     bseg_bounds(a, seg, t0, t1);
     const int64_t base = (int64_t)bh * a.N;
@@ -1133,14 +1200,16 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_kv_walk(BwdArgs a)
         const bool valid = r < nv;
         load_tile_async<NTH>(sm + XK, a.k + (base + c0) * DH, nv);
         load_tile_async<NTH>(sm + V, a.v + (base + c0) * DH, nv);
-        if (causal) load_tile_async<NTH>(sm + XQ, a.q + (base + c0) * DH, nv);
+        if (causal) {
+            load_tile_async<NTH>(sm + XQ, a.q + (base + c0) * DH, nv);
+            load_tile_async<NTH>(sm + DO, a.dout + (base + c0) * DH, nv);
+        }
         cp_async_commit();
         load_w_split(a.W, sm + WHI0, sm + WLO0);
         write_ones(sm + ONES, nv);
-        if (causal)
-            build_dy(a.dout + (base + c0) * DH, a.o + (base + c0) * DH, a.den + base + c0, nv, sm + DY128,
-                     sm + DY32);
         cp_async_wait_all();
+        __syncthreads();
+        if (causal) row_scalars(sm + DO, a.o + (base + c0) * DH, a.den + base + c0, nv, rowc, rowinv, sm + DC32);
         publish_smem();
         if (threadIdx.x == 0) {
             fence_after_sync();
@@ -1151,14 +1220,20 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_kv_walk(BwdArgs a)
         const float raw_k = sqrtf(row_sqnorm(sm + XK, r));
         const float inv_k = 1.f / fmaxf(raw_k, kNormEps);
         const float inv_q = causal ? 1.f / fmaxf(sqrtf(row_sqnorm(sm + XQ, r)), kNormEps) : 0.f;
+        const float invden_r = causal ? rowinv[r] : 0.f;
         if (!(ok = wait_mma(ctl, phase))) break;
         float u[32], t[32];
-        features_half_keep(tm, bkv_tmem::PROJ + 64, r, h, inv_k, a.beta, valid, sm + PHK, u, t);
-        if (causal) features_half(tm, bkv_tmem::PROJ, r, h, inv_q, a.beta, valid, sm + PHQ);
+        proj_keep(tm, bkv_tmem::PROJ + 64, h, inv_k, a.beta, u, t);
+        write_features(t, r, h, valid ? 1.f : 0.f, sm + PHK);
+        if (causal) {  // Phi_Q' = Phi_Q / den
+            float uq[32], tq[32];
+            proj_keep(tm, bkv_tmem::PROJ, h, inv_q, a.beta, uq, tq);
+            write_features(tq, r, h, invden_r, sm + PHQ);
+        }
         publish_smem();
         if (threadIdx.x == 0) {
             fence_after_sync();
-            // dV~ = Phi_K G_next (value columns 0..63)
+            // dV = Phi_K G_next[:, :64]
             {
                 constexpr uint32_t id = idesc_bf16(128, 64, 0, 1);
 #pragma unroll
@@ -1167,7 +1242,7 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_kv_walk(BwdArgs a)
                              sdesc(sb + GS128 + kk * 2048, TILE, 1024, LAYOUT_SW128), id, kk > 0);
             }
             if (causal) {
-                // S^T = Phi_K Phi_Q^T ; P' = V~ dY^T
+                // S'^T = Phi_K Phi_Q'^T ; V dO^T
                 constexpr uint32_t id = idesc_bf16(128, 128, 0, 0);
 #pragma unroll
                 for (int kk = 0; kk < 16; ++kk) {
@@ -1175,50 +1250,50 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_kv_walk(BwdArgs a)
                     mma_bf16(tm + bkv_tmem::ST, sdesc(sb + PHK + off, 16, 1024, LAYOUT_SW128),
                              sdesc(sb + PHQ + off, 16, 1024, LAYOUT_SW128), id, kk > 0);
                 }
-                issue_k80(tm + bkv_tmem::PP, sb + V, sb + ONES, sb + DY128, sb + DY32, id, false);
+                issue_k64(tm + bkv_tmem::PP, sb + V, sb + DO, id, false);
             }
             mma_commit(&ctl->bar);
         }
         if (!(ok = wait_mma(ctl, phase))) break;
         if (causal) {
-            mask_block_to_smem(tm, bkv_tmem::ST, r, h, true, sm + STB);
-            mask_block_to_smem(tm, bkv_tmem::PP, r, h, true, sm + PPB);
+            mask_block_to_smem(tm, bkv_tmem::ST, r, h, true, 0.f, nullptr, sm + STB);
+            mask_block_to_smem(tm, bkv_tmem::PP, r, h, true, 0.f, rowc, sm + PPB);  // v_j.dO_i + c_i, i >= j
         }
         publish_smem();
         if (threadIdx.x == 0) {
             fence_after_sync();
-            if (causal)  // dV~ += triu(S^T) dY
-                issue_tt_times(tm + bkv_tmem::DVT, sb + STB, sb + DY128, idesc_bf16(128, 64, 0, 1), true);
-            // dPhi_K = V~ G_next^T (+ triu(P') Phi_Q)
+            if (causal)  // dV += triu(S'^T) dO
+                issue_tt_times(tm + bkv_tmem::DVT, sb + STB, sb + DO, idesc_bf16(128, 64, 0, 1), true);
+            // dPhi_K = [V | 1] G_next^T (+ triu(P') Phi_Q')
             issue_k80(tm + bkv_tmem::DPHI, sb + V, sb + ONES, sb + GS128, sb + GS32, idesc_bf16(128, 256, 0, 0),
                       false);
             if (causal) {
                 issue_tt_times(tm + bkv_tmem::DPHI, sb + PPB, sb + PHQ, idesc_bf16(128, 256, 0, 1), true);
-                issue_state_update(tm, bkv_tmem::GTOP, bkv_tmem::GBOT, sb + PHQ, sb + DY128, sb + DY32);
+                issue_state_update(tm, bkv_tmem::GTOP, bkv_tmem::GBOT, sb + PHQ, sb + DO, sb + DC32);
             }
             mma_commit(&ctl->bar);
         }
         if (!(ok = wait_mma(ctl, phase))) break;
-        {  // dv = dV~[:, :64], columns 32h .. 32h+31 of row r (TMEM loads are warp-collective:
-           // every lane loads, only valid rows store)
+        {  // dv, columns 32h .. 32h+31 of row r (TMEM loads are warp-collective: every lane
+           // loads, only valid rows store)
             float a0[16], a1[16];
             const uint32_t ta = tm + (lane_base() << 16) + bkv_tmem::DVT + 32u * h;
             tmem_ld16(ta, a0);
             tmem_ld16(ta + 16, a1);
             tmem_wait_ld();
             if (valid) {
-            uint4 *d4 = reinterpret_cast<uint4 *>(a.dv + (base + c0 + r) * DH + 32 * h);
-            d4[0] = make_uint4(pack_bf16x2(a0[0], a0[1]), pack_bf16x2(a0[2], a0[3]), pack_bf16x2(a0[4], a0[5]),
-                               pack_bf16x2(a0[6], a0[7]));
-            d4[1] = make_uint4(pack_bf16x2(a0[8], a0[9]), pack_bf16x2(a0[10], a0[11]), pack_bf16x2(a0[12], a0[13]),
-                               pack_bf16x2(a0[14], a0[15]));
-            d4[2] = make_uint4(pack_bf16x2(a1[0], a1[1]), pack_bf16x2(a1[2], a1[3]), pack_bf16x2(a1[4], a1[5]),
-                               pack_bf16x2(a1[6], a1[7]));
-            d4[3] = make_uint4(pack_bf16x2(a1[8], a1[9]), pack_bf16x2(a1[10], a1[11]), pack_bf16x2(a1[12], a1[13]),
-                               pack_bf16x2(a1[14], a1[15]));
+                uint4 *d4 = reinterpret_cast<uint4 *>(a.dv + (base + c0 + r) * DH + 32 * h);
+                d4[0] = make_uint4(pack_bf16x2(a0[0], a0[1]), pack_bf16x2(a0[2], a0[3]), pack_bf16x2(a0[4], a0[5]),
+                                   pack_bf16x2(a0[6], a0[7]));
+                d4[1] = make_uint4(pack_bf16x2(a0[8], a0[9]), pack_bf16x2(a0[10], a0[11]),
+                                   pack_bf16x2(a0[12], a0[13]), pack_bf16x2(a0[14], a0[15]));
+                d4[2] = make_uint4(pack_bf16x2(a1[0], a1[1]), pack_bf16x2(a1[2], a1[3]), pack_bf16x2(a1[4], a1[5]),
+                                   pack_bf16x2(a1[6], a1[7]));
+                d4[3] = make_uint4(pack_bf16x2(a1[8], a1[9]), pack_bf16x2(a1[10], a1[11]),
+                                   pack_bf16x2(a1[12], a1[13]), pack_bf16x2(a1[14], a1[15]));
             }
         }
-        features_vjp_half(tm, bkv_tmem::DPHI, r, h, a.beta, valid, u, t, sm + DP);
+        features_vjp_half(tm, bkv_tmem::DPHI, r, h, a.beta, valid, u, t, nullptr, 0.f, 1.f, sm + DP);
         load_w_split(a.W, sm + WHI1, sm + WLO1);
         publish_smem();
         if (threadIdx.x == 0) {

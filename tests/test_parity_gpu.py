@@ -56,21 +56,24 @@ def test_forward_backward_match_oracle(shape, dtype, causal):
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 def test_single_token_and_one_chunk_edges(dtype):
+    tol = TOL[dtype]
+    bad = {}
     for N in (1, 2, 31, 32, 33, 127, 128, 129, 512, 513):
         inp = make((1, 1, N, 64, 16, 4), dtype, seed=N)
         out, den, _ = gpu_forward(inp, 0.5, True)
         dq, dk, dv = gpu_backward(inp, out, den, 0.5, True)
         o_ref, den_ref = oracle_forward(inp, 0.5, True)
         dq_ref, dk_ref, dv_ref = oracle_backward(inp, 0.5, True)
-        tol = TOL[dtype]
         # with one token, out_0 = v_0 whatever q and k are: dq = dk = 0 exactly, so the
         # error is measured against the scale of dO instead
         fl = 1e-2 * float(inp["do"].abs().max())
-        assert rel_err(out, o_ref) <= tol and rel_err(den, den_ref) <= tol, N
-        assert rel_err(dq, dq_ref, fl) <= tol and rel_err(dk, dk_ref, fl) <= tol, N
-        assert rel_err(dv, dv_ref) <= tol, N
+        errs = {"out": rel_err(out, o_ref), "den": rel_err(den, den_ref), "dq": rel_err(dq, dq_ref, fl),
+                "dk": rel_err(dk, dk_ref, fl), "dv": rel_err(dv, dv_ref)}
         if N == 1:  # causal row 0 reads only its own key: out_0 = v_0
-            np.testing.assert_allclose(to64(out)[0, 0, 0], to64(inp["v"])[0, 0, 0], rtol=tol, atol=tol)
+            errs["out0_is_v0"] = rel_err(out[0, 0, 0], to64(inp["v"])[0, 0, 0])
+        if max(errs.values()) > tol:
+            bad[N] = errs
+    assert not bad, bad
 
 
 def test_empty_sequence_is_a_no_op():
