@@ -129,6 +129,32 @@ race_status_t race_attn_hash_indices(const void *x, const float *W, int32_t *idx
                                      race_stream_t stream);
 
 /*
+ * Forward pass that allocates nothing and takes no workspace (the method's description has
+ * no counterpart to this; it is a deployment convenience).  It is for callers that cannot
+ * obtain device memory on their own: code whose device memory is owned by a host
+ * framework's allocator that forbids other allocations, or loops that must not pay the
+ * device-wide synchronisation a cudaMalloc can cause.  The segment statistics that
+ * race_attn_forward keeps in its workspace live instead in one fixed buffer of
+ * RACE_NOALLOC_SCRATCH_BYTES that the library defines in device memory; every GPU that
+ * loads the library holds that buffer until the process exits.
+ *   Arguments as race_attn_forward (ctx is not offered).  Returns RACE_ERR_WORKSPACE, having
+ *   launched nothing, when race_attn_workspace_size(..., backward = 0) for these sizes
+ *   exceeds RACE_NOALLOC_SCRATCH_BYTES (for d = 64 and 2^P = 16, L = 16, that is roughly
+ *   B * H * min(N / 512, 296 / (B * H)) segment states of 66.5 KB each).
+ *   The first call on each device looks up the buffer's device address (a runtime call
+ *   with that device current); make that first call before any stream capture.
+ *   All calls share the buffer and it keeps the last call's contents: every element a call
+ *   reads is first written by the same call, so nothing needs clearing, but calls whose
+ *   executions overlap on the GPU (different streams, or several host threads) race on it
+ *   and must be serialised by the caller.
+ */
+#define RACE_NOALLOC_SCRATCH_BYTES ((size_t)24 << 20)
+race_status_t race_attn_forward_noalloc(const void *q, const void *k, const void *v,
+                                        const float *W, void *out, float *den, int B, int H,
+                                        int64_t N, int d, int L, int P, float tau, int causal,
+                                        race_dtype_t dtype, race_stream_t stream);
+
+/*
  * Opt-in kernel timing (a measurement aid; the method has no counterpart).  While enabled,
  * every kernel the library launches is bracketed by a pair of CUDA events recorded on the
  * launch stream; race_attn_profile_read waits for the recorded events, adds each

@@ -23,7 +23,7 @@ __all__ = [
     "race_status_string", "race_attn_workspace_size", "race_attn_ctx_size",
     "race_attn_forward", "race_attn_backward", "race_attn_hash_indices",
     "forward", "backward", "race_attn_profile_enable", "race_attn_profile_reset",
-    "race_attn_profile_read",
+    "race_attn_profile_read", "race_attn_forward_noalloc", "RACE_NOALLOC_SCRATCH_BYTES",
 ]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -31,6 +31,7 @@ _LIB_NAME = "librace_attn.so"
 
 RACE_OK, RACE_ERR_INVALID_ARG, RACE_ERR_UNSUPPORTED, RACE_ERR_WORKSPACE, RACE_ERR_CUDA = range(5)
 RACE_F32, RACE_BF16 = 0, 1
+RACE_NOALLOC_SCRATCH_BYTES = 24 << 20
 
 _vp = ctypes.c_void_p
 _i64 = ctypes.c_int64
@@ -77,6 +78,9 @@ def load_library():
     lib.race_attn_hash_indices.argtypes = [_vp, _vp, _vp, _int, _int, _i64, _int, _int, _int, _int,
                                            _vp]
     lib.race_attn_hash_indices.restype = _int
+    lib.race_attn_forward_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _i64, _int,
+                                              _int, _int, ctypes.c_float, _int, _int, _vp]
+    lib.race_attn_forward_noalloc.restype = _int
     lib.race_attn_profile_enable.argtypes = [_int]
     lib.race_attn_profile_enable.restype = None
     lib.race_attn_profile_reset.argtypes = []
@@ -173,6 +177,15 @@ def race_attn_hash_indices(x, W, idx, stream=None) -> None:
     _check(load_library().race_attn_hash_indices(
         _ptr(x), _ptr(W), _ptr(idx), B, H, N, d, L, P, _dtype_code(x), _stream(stream)),
         "race_attn_hash_indices")
+
+
+def race_attn_forward_noalloc(q, k, v, W, out, den, tau: float, causal: bool, stream=None) -> None:
+    """C ABI forward that takes no workspace: the library's fixed device buffer is used, so
+    nothing is allocated (for callers that cannot allocate device memory)."""
+    B, H, N, d, L, P = _dims(q, W)
+    _check(load_library().race_attn_forward_noalloc(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(W), _ptr(out), _ptr(den), B, H, N, d, L, P, float(tau),
+        int(bool(causal)), _dtype_code(q), _stream(stream)), "race_attn_forward_noalloc")
 
 
 def race_attn_profile_enable(on: bool) -> None:
