@@ -243,10 +243,63 @@ cudaError_t generic_backward(const Plan &p, Args a, const float *hstates, bool h
 
 // ---- the tensor-core path (bf16, d = 64, L = 16, P = 4) --------------------------------
 
+template <typename Kern>
+cudaError_t tc_prepare(Kern kernel, size_t smem)
+{
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+}
+
+// Segment totals of the key side: mode 0 = sum phi(k) [v, 1]^T, mode 1 = sum phi(q) dY^T.
+cudaError_t tc_segment_totals(const Plan &p, race::tc::BwdArgs a, int mode, float *out, cudaStream_t st)
+{
+    namespace tc = race::tc;
+    const dim3 grid((unsigned)p.nseg, (unsigned)p.BH);
+    const size_t sm = tc::smem_bytes(tc::agg_smem::TOTAL);
+    a.agg_out = out;
+    cudaError_t e;
+    if (mode == 0) {
+        if ((e = tc_prepare(tc::tc_agg<0>, sm)) != cudaSuccess) return e;
+        return timed("tc_agg_kv", st, [&] {
+            tc::tc_agg<0><<<grid, tc::NTH, sm, st>>>(a);
+            return cudaGetLastError();
+        });
+    }
+    if ((e = tc_prepare(tc::tc_agg<1>, sm)) != cudaSuccess) return e;
+    return timed("tc_agg_qdy", st, [&] {
+        tc::tc_agg<1><<<grid, tc::NTH, sm, st>>>(a);
+        return cudaGetLastError();
+    });
+}
+
+race::tc::BwdArgs tc_args(const Plan &p, const void *q, const void *k, const void *v, const float *W,
+                          const void *out, const float *den, const void *dout, float tau, int causal)
+{
+    race::tc::BwdArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.q = (const __nv_bfloat16 *)q;
+    a.k = (const __nv_bfloat16 *)k;
+    a.v = (const __nv_bfloat16 *)v;
+    a.o = (const __nv_bfloat16 *)out;
+    a.dout = (const __nv_bfloat16 *)dout;
+    a.den = den;
+    a.W = W;
+    a.N = p.N;
+    a.seg_len = p.seg_len;
+    a.nseg = p.nseg;
+    a.beta = 1.f / tau;
+    a.causal = causal;
+    return a;
+}
+
 cudaError_t tc_forward(const Plan &p, const void *q, const void *k, const void *v, const float *W,
                        void *out, float *den, float *states, float tau, int causal, cudaStream_t st)
 {
     namespace tc = race::tc;
+    cudaError_t e = tc_segment_totals(p, tc_args(p, q, k, v, W, nullptr, nullptr, nullptr, tau, causal), 0,
+                                      states, st);
+    if (e != cudaSuccess) return e;
+    e = launch_scan(states, p, causal ? gk::SCAN_EXCL_PREFIX : gk::SCAN_TOTAL, st);
+    if (e != cudaSuccess) return e;
     tc::Args a;
     std::memset(&a, 0, sizeof(a));
     a.q = (const __nv_bfloat16 *)q;
@@ -260,23 +313,11 @@ cudaError_t tc_forward(const Plan &p, const void *q, const void *k, const void *
     a.nseg = p.nseg;
     a.beta = 1.f / tau;
     a.causal = causal;
-    a.agg_out = states;
-    const dim3 grid((unsigned)p.nseg, (unsigned)p.BH);
-    const size_t sm_agg = tc::smem_bytes(tc::agg_smem::TOTAL);
-    const size_t sm_walk = tc::smem_bytes(tc::fwd_smem::TOTAL);
-    cudaError_t e = cudaFuncSetAttribute(tc::tc_agg_kv, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_agg);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(tc::tc_fwd_walk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_walk);
-    if (e != cudaSuccess) return e;
-    e = timed("tc_agg_kv", st, [&] {
-        tc::tc_agg_kv<<<grid, tc::NTH, sm_agg, st>>>(a);
-        return cudaGetLastError();
-    });
-    if (e != cudaSuccess) return e;
-    e = launch_scan(states, p, causal ? gk::SCAN_EXCL_PREFIX : gk::SCAN_TOTAL, st);
-    if (e != cudaSuccess) return e;
     a.state = states;
     a.state_seg_stride = causal ? (int64_t)p.M * p.D : 0;
+    const dim3 grid((unsigned)p.nseg, (unsigned)p.BH);
+    const size_t sm_walk = tc::smem_bytes(tc::fwd_smem::TOTAL);
+    if ((e = tc_prepare(tc::tc_fwd_walk, sm_walk)) != cudaSuccess) return e;
     return timed("tc_fwd_walk", st, [&] {
         tc::tc_fwd_walk<<<grid, tc::NTH, sm_walk, st>>>(a);
         return cudaGetLastError();
@@ -289,59 +330,23 @@ cudaError_t tc_backward(const Plan &p, const void *q, const void *k, const void 
 {
     namespace tc = race::tc;
     const dim3 grid((unsigned)p.nseg, (unsigned)p.BH);
-    cudaError_t e;
-    const float *hstates = ctx;
-    if (!hstates) {  // key-side prefix statistics, as the forward computes them
-        tc::Args fa;
-        std::memset(&fa, 0, sizeof(fa));
-        fa.k = (const __nv_bfloat16 *)k;
-        fa.v = (const __nv_bfloat16 *)v;
-        fa.W = W;
-        fa.N = p.N;
-        fa.seg_len = p.seg_len;
-        fa.nseg = p.nseg;
-        fa.beta = 1.f / tau;
-        fa.causal = causal;
-        fa.agg_out = hbuf;
-        const size_t sm_agg = tc::smem_bytes(tc::agg_smem::TOTAL);
-        e = cudaFuncSetAttribute(tc::tc_agg_kv, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_agg);
-        if (e != cudaSuccess) return e;
-        e = timed("tc_agg_kv", st, [&] {
-            tc::tc_agg_kv<<<grid, tc::NTH, sm_agg, st>>>(fa);
-            return cudaGetLastError();
-        });
-        if (e != cudaSuccess) return e;
-        e = launch_scan(hbuf, p, causal ? gk::SCAN_EXCL_PREFIX : gk::SCAN_TOTAL, st);
-        if (e != cudaSuccess) return e;
-        hstates = hbuf;
-    }
-    tc::BwdArgs a;
-    std::memset(&a, 0, sizeof(a));
-    a.q = (const __nv_bfloat16 *)q;
-    a.k = (const __nv_bfloat16 *)k;
-    a.v = (const __nv_bfloat16 *)v;
-    a.o = (const __nv_bfloat16 *)out;
-    a.dout = (const __nv_bfloat16 *)dout;
-    a.den = den;
-    a.W = W;
+    tc::BwdArgs a = tc_args(p, q, k, v, W, out, den, dout, tau, causal);
     a.dq = (__nv_bfloat16 *)dq;
     a.dk = (__nv_bfloat16 *)dk;
     a.dv = (__nv_bfloat16 *)dv;
-    a.N = p.N;
-    a.seg_len = p.seg_len;
-    a.nseg = p.nseg;
-    a.beta = 1.f / tau;
-    a.causal = causal;
+    cudaError_t e;
+    const float *hstates = ctx;
+    if (!hstates) {  // key-side prefix statistics, as the forward computes them
+        if ((e = tc_segment_totals(p, a, 0, hbuf, st)) != cudaSuccess) return e;
+        if ((e = launch_scan(hbuf, p, causal ? gk::SCAN_EXCL_PREFIX : gk::SCAN_TOTAL, st)) != cudaSuccess)
+            return e;
+        hstates = hbuf;
+    }
     const int64_t stride = causal ? (int64_t)p.M * p.D : 0;
     const size_t sm_q = tc::smem_bytes(tc::bq_smem::TOTAL);
-    const size_t sm_aq = tc::smem_bytes(tc::aggq_smem::TOTAL);
     const size_t sm_kv = tc::smem_bytes(tc::bkv_smem::TOTAL);
-    if ((e = cudaFuncSetAttribute(tc::tc_bwd_q_walk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_q)) !=
-            cudaSuccess ||
-        (e = cudaFuncSetAttribute(tc::tc_agg_qdy, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_aq)) !=
-            cudaSuccess ||
-        (e = cudaFuncSetAttribute(tc::tc_bwd_kv_walk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_kv)) !=
-            cudaSuccess)
+    if ((e = tc_prepare(tc::tc_bwd_q_walk, sm_q)) != cudaSuccess ||
+        (e = tc_prepare(tc::tc_bwd_kv_walk, sm_kv)) != cudaSuccess)
         return e;
     a.state = hstates;
     a.state_seg_stride = stride;
@@ -350,14 +355,8 @@ cudaError_t tc_backward(const Plan &p, const void *q, const void *k, const void 
         return cudaGetLastError();
     });
     if (e != cudaSuccess) return e;
-    a.agg_out = gbuf;
-    e = timed("tc_agg_qdy", st, [&] {
-        tc::tc_agg_qdy<<<grid, tc::NTH, sm_aq, st>>>(a);
-        return cudaGetLastError();
-    });
-    if (e != cudaSuccess) return e;
-    e = launch_scan(gbuf, p, causal ? gk::SCAN_EXCL_SUFFIX : gk::SCAN_TOTAL, st);
-    if (e != cudaSuccess) return e;
+    if ((e = tc_segment_totals(p, a, 1, gbuf, st)) != cudaSuccess) return e;
+    if ((e = launch_scan(gbuf, p, causal ? gk::SCAN_EXCL_SUFFIX : gk::SCAN_TOTAL, st)) != cudaSuccess) return e;
     a.state = gbuf;
     return timed("tc_bwd_kv_walk", st, [&] {
         tc::tc_bwd_kv_walk<<<grid, tc::NTH, sm_kv, st>>>(a);

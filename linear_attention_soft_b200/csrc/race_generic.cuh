@@ -522,22 +522,29 @@ __global__ void __launch_bounds__(NT) race_scan(float *buf, int nseg, int64_t MD
     const int64_t e = (int64_t)blockIdx.x * NT + threadIdx.x;
     if (e >= MD) return;
     float *b = buf + (int64_t)blockIdx.y * nseg * MD + e;
+    constexpr int K = 8;  // segments loaded together: independent loads in flight
     float run = 0.f;
-    if (mode == SCAN_EXCL_PREFIX) {
-        for (int s = 0; s < nseg; ++s) {
-            const float t = b[s * MD];
-            b[s * MD] = run;
-            run += t;
-        }
-    } else if (mode == SCAN_EXCL_SUFFIX) {
-        for (int s = nseg - 1; s >= 0; --s) {
-            const float t = b[s * MD];
-            b[s * MD] = run;
-            run += t;
-        }
-    } else {
+    if (mode == SCAN_TOTAL) {
         for (int s = 0; s < nseg; ++s) run += b[s * MD];
         b[0] = run;
+        return;
+    }
+    const bool rev = mode == SCAN_EXCL_SUFFIX;
+    for (int s0 = 0; s0 < nseg; s0 += K) {
+        float v[K];
+#pragma unroll
+        for (int i = 0; i < K; ++i) {
+            const int s = rev ? nseg - 1 - (s0 + i) : s0 + i;
+            v[i] = (s0 + i < nseg) ? b[(int64_t)s * MD] : 0.f;
+        }
+#pragma unroll
+        for (int i = 0; i < K; ++i) {
+            const int s = rev ? nseg - 1 - (s0 + i) : s0 + i;
+            if (s0 + i < nseg) {
+                b[(int64_t)s * MD] = run;
+                run += v[i];
+            }
+        }
     }
 }
 

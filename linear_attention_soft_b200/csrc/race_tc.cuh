@@ -14,11 +14,18 @@
 //     H     += Phi_K^T V~                   (causal; fp32 master copy stays in TMEM)
 //     out    = Y[:, :64] / Y[:, 64],  den = Y[:, 64]
 //
-// Every GEMM above is a tcgen05.mma with operands in shared memory (SW128 / SW32 swizzled
-// tiles) and the accumulator in tensor memory; one thread issues them, completion is
-// signalled through an mbarrier that the other threads wait on with a bounded poll.
-// One CTA of 256 threads walks one segment of one (b, h) sequence; thread t owns token
-// row t % 128 and the tables of half t / 128 (tables 0-7 or 8-15).
+// Every GEMM above is a tcgen05.mma with operands in shared memory and the accumulator in
+// tensor memory; one thread issues them and completion is signalled through an mbarrier
+// that one thread polls with a time limit.  One CTA of 512 threads walks one segment of
+// one (b, h) sequence.  Thread t owns token row r = t % 128 (its TMEM lane) and quarter
+// qd = t / 128 of every per-row job: tables 4qd .. 4qd+3 (feature block qd), a quarter of
+// the output columns, a quarter of the state rows.
+//
+// Shared-memory tile formats (bf16):
+//   K128 tile: [128 rows][64 cols], 128-byte rows, 16-byte chunks XOR-swizzled by row % 8.
+//   Value tile: [rows][16 * natoms] as natoms SW32 atoms of [rows][16] (32-byte rows); the
+//     value dimension of V~ = [V | 1], [dO | c] and of the staged states, so that one MMA
+//     covers all 80 (or 64) value columns, as the N side (MN-major) or the K side (K-major).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -33,15 +40,16 @@ namespace race {
 namespace tc {
 
 constexpr int T = 128;      // tokens per chunk (MMA M)
-constexpr int NTH = 256;    // threads per CTA
+constexpr int NTH = 512;    // threads per CTA
 constexpr int DH = 64;      // head dimension
 constexpr int NPROJ = 64;   // L * P projections
 constexpr int MF = 256;     // L * 2^P features
-constexpr int NV = 80;      // value columns: 64 of V, the ones column, 15 zero
 constexpr int DS = 65;      // state row length in global memory (64 + ones column)
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s: far above any chunk's MMA time
 
-constexpr uint32_t TILE = 16384;  // one [128][64] bf16 SW128 tile
+constexpr uint32_t TILE = 16384;   // one K128 tile
+constexpr uint32_t VA128 = 4096;   // one SW32 atom of 128 rows
+constexpr uint32_t VA256 = 8192;   // one SW32 atom of 256 rows
 
 // error word shared by all launches of this path (1 = an MMA completion wait timed out)
 __device__ int g_tc_error;
@@ -60,55 +68,26 @@ struct Args {
     int causal;
 };
 
-// ---- shared memory maps (byte offsets from a 1024-aligned base) -------------------------
-namespace fwd_smem {
-constexpr uint32_t PHQ = 0;                 // Phi_Q [128][256]: 4 SW128 tiles
-constexpr uint32_t XQ = PHQ;                // q rows during the projection
-constexpr uint32_t XK = PHQ + TILE;         // k rows during the projection
-constexpr uint32_t SB = PHQ;                // masked S as bf16 [128][128]: 2 tiles
-constexpr uint32_t PHK = PHQ + 4 * TILE;    // Phi_K [128][256]
-constexpr uint32_t HS128 = PHK + 4 * TILE;  // staged H[:, 0:64] as [256][64] SW128 (2 tiles)
-constexpr uint32_t HS32 = HS128 + 2 * TILE; // staged H[:, 64:80] as [256][16] SW32 (8 KB)
-constexpr uint32_t V = HS32 + 8192;         // v rows [128][64]
-constexpr uint32_t ONES = V + TILE;         // ones column block [128][16] SW32 (4 KB)
-constexpr uint32_t WHI = ONES + 4096;       // W hi [64][64]
-constexpr uint32_t WLO = WHI + 8192;        // W lo [64][64]
-constexpr uint32_t BAR = WLO + 8192;        // mbarrier, TMEM address, abort flag
-constexpr uint32_t TOTAL = BAR + 64;
-}  // namespace fwd_smem
-
-namespace agg_smem {
-constexpr uint32_t PHK = 0;                 // Phi_K, also k rows during the projection
-constexpr uint32_t XK = PHK;
-constexpr uint32_t V = PHK + 4 * TILE;
-constexpr uint32_t ONES = V + TILE;
-constexpr uint32_t WHI = ONES + 4096;
-constexpr uint32_t WLO = WHI + 8192;
-constexpr uint32_t BAR = WLO + 8192;
-constexpr uint32_t TOTAL = BAR + 64;
-}  // namespace agg_smem
-
-// TMEM columns
-namespace fwd_tmem {
-constexpr uint32_t PROJ = 0;    // [128][64] q projections, [128][64] k projections at +64
-constexpr uint32_t S = 0;       // [128][128] (reuses PROJ once the features are formed)
-constexpr uint32_t Y = 128;     // [128][80]
-constexpr uint32_t HTOP = 256;  // H rows 0..127   [128][80]
-constexpr uint32_t HBOT = 336;  // H rows 128..255 [128][80]
-constexpr uint32_t NCOLS = 512;
-}  // namespace fwd_tmem
-namespace agg_tmem {
-constexpr uint32_t PROJ = 0;
-constexpr uint32_t HTOP = 64;
-constexpr uint32_t HBOT = 144;
-constexpr uint32_t NCOLS = 256;
-}  // namespace agg_tmem
+struct BwdArgs {
+    const __nv_bfloat16 *q, *k, *v, *o, *dout;
+    const float *den, *W;
+    __nv_bfloat16 *dq, *dk, *dv;
+    const float *state;
+    int64_t state_seg_stride;
+    float *agg_out;
+    int64_t N, seg_len;
+    int nseg;
+    float beta;
+    int causal;
+};
 
 struct Ctl {
     uint64_t bar;
     uint32_t tmem;
     uint32_t abort;
 };
+
+// ---- small helpers ---------------------------------------------------------------------
 
 __device__ __forceinline__ uint8_t *aligned_base(uint8_t *raw)
 {
@@ -117,31 +96,67 @@ __device__ __forceinline__ uint8_t *aligned_base(uint8_t *raw)
 }
 
 __device__ __forceinline__ uint32_t lane_base() { return (uint32_t)((threadIdx.x >> 5) & 3) * 32u; }
+__device__ __forceinline__ uint32_t tlane(uint32_t tm, uint32_t col) { return tm + (lane_base() << 16) + col; }
 
-// W [64][64] fp32 -> two SW128 tiles of bf16 (hi = round(W), lo = round(W - hi)).
+// byte offset of 8-element chunk c8 of row `row` in a value tile with `rows` rows
+__device__ __forceinline__ uint32_t va_off(int row, int c8, uint32_t rows)
+{
+    return (uint32_t)(c8 >> 1) * rows * 32u + sw32_off(row, c8 & 1);
+}
+
+__device__ __forceinline__ void seg_bounds(int64_t seg_len, int64_t N, int seg, int64_t &t0, int64_t &t1)
+{
+    t0 = (int64_t)seg * seg_len;
+    t1 = t0 + seg_len;
+    if (t1 > N) t1 = N;
+}
+
+// W [64][64] fp32 -> two K128-format tiles [64][64] of bf16 (hi = round(W), lo = round(W - hi)).
 __device__ void load_w_split(const float *W, uint8_t *whi, uint8_t *wlo)
 {
-    for (int e = threadIdx.x; e < NPROJ * DH; e += NTH) {
-        const int n = e >> 6, c = e & 63;
-        const float w = W[e];
-        const __nv_bfloat16 hi = __float2bfloat16_rn(w);
-        const __nv_bfloat16 lo = __float2bfloat16_rn(w - __bfloat162float(hi));
+    for (int e = threadIdx.x; e < NPROJ * DH / 2; e += NTH) {
+        const float2 w = reinterpret_cast<const float2 *>(W)[e];
+        const int n = (2 * e) >> 6, c = (2 * e) & 63;
+        const uint32_t hi = pack_bf16x2(w.x, w.y);
+        const uint32_t lo = pack_bf16x2(w.x - bf16_lo(hi), w.y - bf16_hi(hi));
         const uint32_t off = sw128_off(n, c >> 3) + (c & 7) * 2;
-        *reinterpret_cast<__nv_bfloat16 *>(whi + off) = hi;
-        *reinterpret_cast<__nv_bfloat16 *>(wlo + off) = lo;
+        *reinterpret_cast<uint32_t *>(whi + off) = hi;
+        *reinterpret_cast<uint32_t *>(wlo + off) = lo;
     }
 }
 
-// Ones column block: row j holds 1 in column 0 when j < nvalid, zeros elsewhere.
-__device__ void write_ones(uint8_t *ones, int nvalid)
+// Rows [0, nvalid) of a [.., 64] bf16 tensor into a K128 tile (zero rows beyond).
+__device__ __forceinline__ void load_k128_async(uint8_t *tile, const __nv_bfloat16 *src, int nvalid)
 {
-    if (threadIdx.x < T) {
-        const int j = threadIdx.x;
-        const uint32_t one = j < nvalid ? 0x3F80u : 0u;  // bf16 1.0 in the low half
-        const uint32_t a = smem_u32(ones);
-        st_shared_v4(a + sw32_off(j, 0), one, 0u, 0u, 0u);
-        st_shared_v4(a + sw32_off(j, 1), 0u, 0u, 0u, 0u);
+    const uint32_t base = smem_u32(tile);
+#pragma unroll
+    for (int k = 0; k < 1024 / NTH; ++k) {
+        const int c = threadIdx.x + NTH * k;
+        const int row = c >> 3, ch = c & 7;
+        const bool ok = row < nvalid;
+        cp_async16(base + sw128_off(row, ch), src + (ok ? (int64_t)row * 64 + ch * 8 : 0), ok ? 16u : 0u);
     }
+}
+
+// Rows [0, nvalid) of a [.., 64] bf16 tensor into atoms 0..3 of a 128-row value tile.
+__device__ __forceinline__ void load_va_async(uint8_t *tile, const __nv_bfloat16 *src, int nvalid)
+{
+    const uint32_t base = smem_u32(tile);
+#pragma unroll
+    for (int k = 0; k < 1024 / NTH; ++k) {
+        const int c = threadIdx.x + NTH * k;
+        const int row = c >> 3, ch = c & 7;
+        const bool ok = row < nvalid;
+        cp_async16(base + va_off(row, ch, T), src + (ok ? (int64_t)row * 64 + ch * 8 : 0), ok ? 16u : 0u);
+    }
+}
+
+// Atom 4 of a 128-row value tile: column 64 = x (1 for the ones column), zeros elsewhere.
+__device__ __forceinline__ void write_col64(uint8_t *tile, int r, float x)
+{
+    const uint32_t b = smem_u32(tile) + 4 * VA128;
+    st_shared_v4(b + sw32_off(r, 0), pack_bf16x2(x, 0.f), 0u, 0u, 0u);
+    st_shared_v4(b + sw32_off(r, 1), 0u, 0u, 0u, 0u);
 }
 
 // Wait for the MMAs committed to ctl->bar; one thread polls (bounded), all learn the outcome.
@@ -167,8 +182,26 @@ __device__ __forceinline__ void publish_smem()
     __syncthreads();
 }
 
-// Squared L2 norm of row r of a [128][64] SW128 tile.
-__device__ __forceinline__ float row_sqnorm(const uint8_t *tile, int r)
+// L2 prefetch of the rows [row0, row0 + n) of up to five [.., 64] bf16 tensors and of a
+// per-token fp32 vector (threads 0..5 each take one), for the chunk after the current one.
+__device__ __forceinline__ void prefetch_chunk(int64_t row0, int n, const __nv_bfloat16 *t0_,
+                                               const __nv_bfloat16 *t1_, const __nv_bfloat16 *t2_,
+                                               const __nv_bfloat16 *t3_, const __nv_bfloat16 *t4_,
+                                               const float *f0)
+{
+    if (n <= 0 || threadIdx.x >= 6) return;
+    const __nv_bfloat16 *ts[5] = {t0_, t1_, t2_, t3_, t4_};
+    if (threadIdx.x < 5) {
+        if (ts[threadIdx.x]) prefetch_l2(ts[threadIdx.x] + row0 * DH, (uint32_t)n * DH * 2u);
+    } else if (f0) {  // shrink to 16-byte aligned bounds inside the range
+        const uintptr_t lo = ((uintptr_t)(f0 + row0) + 15u) & ~(uintptr_t)15u;
+        const uintptr_t hi = (uintptr_t)(f0 + row0 + n) & ~(uintptr_t)15u;
+        if (hi > lo) prefetch_l2((const void *)lo, (uint32_t)(hi - lo));
+    }
+}
+
+// Raw L2 norm of row r of a K128 tile.
+__device__ __forceinline__ float row_norm(const uint8_t *tile, int r)
 {
     const uint32_t a = smem_u32(tile);
     float s = 0.f;
@@ -183,206 +216,569 @@ __device__ __forceinline__ float row_sqnorm(const uint8_t *tile, int r)
             s = fmaf(x1, x1, s);
         }
     }
-    return s;
+    return sqrtf(s);
 }
 
-// Soft bucket assignment of the 8 tables of half h for token row r, from the 32
-// projections in TMEM (columns col0 + 32h ..), written as bf16 into the Phi tile
-// [128][256].  phi_l[r] = prod_p sigmoid(2 beta c_rp u_p) with u = tanh(proj / |x|): the
-// corner softmax of zh §2.2 in factorised form; sigmoid(2z) = (1 + tanh z) / 2.
-__device__ __forceinline__ void features_half(uint32_t tmem, uint32_t col0, int r, int h, float inv_norm,
-                                              float beta, bool valid, uint8_t *phi)
+// Per-row scalars of a chunk from the dO rows of a value tile and o from global:
+// rowc[r] = c_r = -(dO_r . o_r), rowinv[r] = 1/den_r (0 beyond nvalid); optionally c_r
+// into column 64 of the value tile.  One thread per row.
+__device__ __forceinline__ void row_scalars(int r, const uint8_t *doc, const __nv_bfloat16 *o, const float *den,
+                                            int nvalid, float *rowc, float *rowinv, uint8_t *doc_col64)
 {
-    float pr[32];
-    {
-        float a[16], b[16];
-        const uint32_t t = tmem + (lane_base() << 16) + col0 + 32u * h;
-        tmem_ld16(t, a);
-        tmem_ld16(t + 16, b);
-        tmem_wait_ld();
+    float c = 0.f, inv = 0.f;
+    if (r < nvalid) {
+        const uint32_t a = smem_u32(doc);
+        const uint4 *o4 = reinterpret_cast<const uint4 *>(o + (int64_t)r * DH);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            pr[i] = a[i];
-            pr[16 + i] = b[i];
-        }
-    }
-    const uint32_t base = smem_u32(phi);
+        for (int ch = 0; ch < 8; ++ch) {
+            const uint4 g = ld_shared_v4(a + va_off(r, ch, T)), ov = o4[ch];
+            const uint32_t gw[4] = {g.x, g.y, g.z, g.w}, ow[4] = {ov.x, ov.y, ov.z, ov.w};
 #pragma unroll
-    for (int l = 0; l < 8; ++l) {
-        float f[16];
-        f[0] = 1.f;
-#pragma unroll
-        for (int p = 0; p < 4; ++p) {
-            const float u = tanh_fast(pr[4 * l + p] * inv_norm);
-            const float t = tanh_fast(beta * u);
-            const float s1 = 0.5f + 0.5f * t, s0 = 0.5f - 0.5f * t;
-            const int hh = 1 << p;
-#pragma unroll
-            for (int c = 0; c < hh; ++c) {
-                f[c + hh] = f[c] * s1;
-                f[c] *= s0;
+            for (int i = 0; i < 4; ++i) {
+                c = fmaf(bf16_lo(gw[i]), bf16_lo(ow[i]), c);
+                c = fmaf(bf16_hi(gw[i]), bf16_hi(ow[i]), c);
             }
         }
-        uint32_t w[8];
+        c = -c;
+        const float dn = den[r];
+        inv = dn != 0.f ? 1.f / dn : 0.f;
+    }
+    rowc[r] = c;
+    rowinv[r] = inv;
+    if (doc_col64) write_col64(doc_col64, r, c);
+}
+
+// u = tanh(proj / |x|) and t = tanh(beta u) of this thread's 16 projections (tables
+// 4qd .. 4qd+3), read from TMEM columns col0 + 16qd.
+__device__ __forceinline__ void proj_tanh(uint32_t tm, uint32_t col0, int qd, float inv_norm, float beta,
+                                          float (&u)[16], float (&t)[16])
+{
+    uint32_t w[16];
+    tmem_ld16_nowait(tlane(tm, col0 + 16u * qd), w);
+    tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 8; ++i) w[i] = valid ? pack_bf16x2(f[2 * i], f[2 * i + 1]) : 0u;
-        const int tl = 8 * h + l;            // table 0..15 -> features 16 tl .. 16 tl + 15
-        const uint32_t blk = base + (uint32_t)(tl >> 2) * TILE;
-        const int ch = (tl & 3) * 2;
-        st_shared_v4(blk + sw128_off(r, ch), w[0], w[1], w[2], w[3]);
-        st_shared_v4(blk + sw128_off(r, ch + 1), w[4], w[5], w[6], w[7]);
+    for (int i = 0; i < 16; ++i) u[i] = tanh_fast(__uint_as_float(w[i]) * inv_norm);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) t[i] = tanh_fast(beta * u[i]);
+}
+
+// Corner weights of table l from t: phi_r = prod_p sigmoid(2 beta c_rp u_p) with
+// sigmoid(2z) = (1 + tanh z) / 2 -- the softmax over hypercube corners of zh §2.2 in its
+// factorised form.  Times `scale`.
+__device__ __forceinline__ void corner_weights(const float (&t)[16], int l, float scale, float (&f)[16])
+{
+    float a[4], b[4];
+    {
+        const float s1a = 0.5f + 0.5f * t[4 * l], s0a = 0.5f - 0.5f * t[4 * l];
+        const float s1b = 0.5f + 0.5f * t[4 * l + 1], s0b = 0.5f - 0.5f * t[4 * l + 1];
+        a[0] = s0a * s0b * scale;
+        a[1] = s1a * s0b * scale;
+        a[2] = s0a * s1b * scale;
+        a[3] = s1a * s1b * scale;
+    }
+    {
+        const float s1c = 0.5f + 0.5f * t[4 * l + 2], s0c = 0.5f - 0.5f * t[4 * l + 2];
+        const float s1d = 0.5f + 0.5f * t[4 * l + 3], s0d = 0.5f - 0.5f * t[4 * l + 3];
+        b[0] = s0c * s0d;
+        b[1] = s1c * s0d;
+        b[2] = s0c * s1d;
+        b[3] = s1c * s1d;
+    }
+#pragma unroll
+    for (int hi = 0; hi < 4; ++hi)
+#pragma unroll
+        for (int lo = 0; lo < 4; ++lo) f[4 * hi + lo] = a[lo] * b[hi];
+}
+
+// This thread's 64 features (feature block qd) of row r, times `scale`, into the Phi tile.
+__device__ __forceinline__ void write_features(const float (&t)[16], int r, int qd, float scale, uint8_t *phi)
+{
+    const uint32_t blk = smem_u32(phi) + (uint32_t)qd * TILE;
+#pragma unroll
+    for (int l = 0; l < 4; ++l) {
+        float f[16];
+        corner_weights(t, l, scale, f);
+        st_shared_v4(blk + sw128_off(r, 2 * l), pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                     pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+        st_shared_v4(blk + sw128_off(r, 2 * l + 1), pack_bf16x2(f[8], f[9]), pack_bf16x2(f[10], f[11]),
+                     pack_bf16x2(f[12], f[13]), pack_bf16x2(f[14], f[15]));
     }
 }
 
-// proj[128][64] (+)= X[128][64] (W_hi + W_lo)^T
+// Feature-map VJP for this thread's 4 tables: dphi[m] = (D[m] + add_scale * add_vec[m]) * mul
+// with D from TMEM columns col0 + 64qd (16 per table) and add_vec (fp32, shared memory,
+// indexed by feature) optional; dz = phi (dphi - phi.dphi), du_p = beta sum_r c_rp dz_r,
+// dp~ = du (1 - u^2) -> 16 values as bf16 into row r of the DP tile (projections 16qd ..).
+__device__ __forceinline__ void features_vjp(uint32_t tm, uint32_t col0, int r, int qd, float beta, bool valid,
+                                             const float (&u)[16], const float (&t)[16], const float *add_vec,
+                                             float add_scale, float mul, uint8_t *dp_tile)
+{
+    uint32_t g[4][16];
+#pragma unroll
+    for (int l = 0; l < 4; ++l) tmem_ld16_nowait(tlane(tm, col0 + 64u * qd + 16u * l), g[l]);
+    tmem_wait_ld();
+    float dp[16];
+#pragma unroll
+    for (int l = 0; l < 4; ++l) {
+        float gg[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) gg[c] = __uint_as_float(g[l][c]);
+        if (add_vec) {
+            const float *av = add_vec + 64 * qd + 16 * l;
+#pragma unroll
+            for (int c = 0; c < 16; ++c) gg[c] = fmaf(add_scale, av[c], gg[c]) * mul;
+        }
+        float f[16];
+        corner_weights(t, l, 1.f, f);
+        float dot = 0.f;
+#pragma unroll
+        for (int c = 0; c < 16; ++c) dot = fmaf(f[c], gg[c], dot);
+        float du[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+            const float dz = f[c] * (gg[c] - dot);
+#pragma unroll
+            for (int p = 0; p < 4; ++p) du[p] += ((c >> p) & 1) ? dz : -dz;
+        }
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            const float uu = u[4 * l + p];
+            dp[4 * l + p] = valid ? beta * du[p] * (1.f - uu * uu) : 0.f;
+        }
+    }
+    const uint32_t b = smem_u32(dp_tile);
+#pragma unroll
+    for (int ch = 0; ch < 2; ++ch)
+        st_shared_v4(b + sw128_off(r, 2 * qd + ch), pack_bf16x2(dp[8 * ch], dp[8 * ch + 1]),
+                     pack_bf16x2(dp[8 * ch + 2], dp[8 * ch + 3]), pack_bf16x2(dp[8 * ch + 4], dp[8 * ch + 5]),
+                     pack_bf16x2(dp[8 * ch + 6], dp[8 * ch + 7]));
+}
+
+// Masked T x T block from TMEM (row r, columns col0 + 32qd ..) to bf16 K128 tile (qd >> 1)
+// of dst.  Adds add_row to every element and add_col[col] per column (optional) before
+// masking; keep_upper keeps column >= row (else column <= row).
+__device__ __forceinline__ void mask_block(uint32_t tm, uint32_t col0, int r, int qd, bool keep_upper,
+                                           float add_row, const float *add_col, uint8_t *dst)
+{
+    uint32_t w[2][16];
+    tmem_ld16_nowait(tlane(tm, col0 + 32u * qd), w[0]);
+    tmem_ld16_nowait(tlane(tm, col0 + 32u * qd + 16u), w[1]);
+    tmem_wait_ld();
+    const uint32_t blk = smem_u32(dst) + (uint32_t)(qd >> 1) * TILE;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        float x[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int col = 32 * qd + 8 * c + i;
+            float y = __uint_as_float(w[c >> 1][8 * (c & 1) + i]) + add_row;
+            if (add_col) y += add_col[col];
+            x[i] = (keep_upper ? (col < r) : (col > r)) ? 0.f : y;
+        }
+        st_shared_v4(blk + sw128_off(r, 4 * (qd & 1) + c), pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]),
+                     pack_bf16x2(x[4], x[5]), pack_bf16x2(x[6], x[7]));
+    }
+}
+
+// This thread's 40 state columns (row m = 128 (qd & 1) + r of the state, columns
+// 40 (qd >> 1) .. +39) from TMEM (state halves at col_top / col_bot).
+__device__ __forceinline__ void read_state40(uint32_t tm, uint32_t col_top, uint32_t col_bot, int qd, float (&hv)[40])
+{
+    const uint32_t base = ((qd & 1) ? col_bot : col_top) + 40u * (qd >> 1);
+    uint32_t a[16], b[16], c[8];
+    tmem_ld16_nowait(tlane(tm, base), a);
+    tmem_ld16_nowait(tlane(tm, base + 16), b);
+    tmem_ld8_nowait(tlane(tm, base + 32), c);
+    tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        hv[i] = __uint_as_float(a[i]);
+        hv[16 + i] = __uint_as_float(b[i]);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) hv[32 + i] = __uint_as_float(c[i]);
+}
+
+// Stage those 40 columns as bf16 into a 256-row, 5-atom value tile.
+__device__ __forceinline__ void stage40(const float (&hv)[40], int m, int qd, uint8_t *va)
+{
+    const uint32_t b = smem_u32(va);
+#pragma unroll
+    for (int k = 0; k < 5; ++k) {
+        const int c8 = 5 * (qd >> 1) + k;
+        st_shared_v4(b + va_off(m, c8, 256), pack_bf16x2(hv[8 * k], hv[8 * k + 1]),
+                     pack_bf16x2(hv[8 * k + 2], hv[8 * k + 3]), pack_bf16x2(hv[8 * k + 4], hv[8 * k + 5]),
+                     pack_bf16x2(hv[8 * k + 6], hv[8 * k + 7]));
+    }
+}
+
+// Stage as a bf16 hi + lo pair of 4-atom value tiles (columns 0..63) plus column 64 in fp32.
+__device__ __forceinline__ void stage40_hilo(const float (&hv)[40], int m, int qd, uint8_t *hi, uint8_t *lo,
+                                             float *col64)
+{
+    const uint32_t bh_ = smem_u32(hi), bl = smem_u32(lo);
+#pragma unroll
+    for (int k = 0; k < 5; ++k) {
+        const int c8 = 5 * (qd >> 1) + k;
+        if (c8 >= 8) break;
+        uint32_t wh[4], wl[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float x0 = hv[8 * k + 2 * i], x1 = hv[8 * k + 2 * i + 1];
+            wh[i] = pack_bf16x2(x0, x1);
+            wl[i] = pack_bf16x2(x0 - bf16_lo(wh[i]), x1 - bf16_hi(wh[i]));
+        }
+        st_shared_v4(bh_ + va_off(m, c8, 256), wh[0], wh[1], wh[2], wh[3]);
+        st_shared_v4(bl + va_off(m, c8, 256), wl[0], wl[1], wl[2], wl[3]);
+    }
+    if (qd >> 1) col64[m] = hv[24];
+}
+
+// Start state: this thread's 40 columns of row m from global fp32 [256][65] into TMEM.
+__device__ __forceinline__ void load_state40(const float *src_all, int m, int qd, uint32_t tm, uint32_t col_top,
+                                             uint32_t col_bot, float (&hv)[40])
+{
+    const float *src = src_all + (int64_t)m * DS;
+    const int c0 = 40 * (qd >> 1);
+#pragma unroll
+    for (int i = 0; i < 40; ++i) hv[i] = (c0 + i < DS) ? src[c0 + i] : 0.f;
+    const uint32_t base = ((qd & 1) ? col_bot : col_top) + (uint32_t)c0;
+    float a[16], b[16], c[8];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        a[i] = hv[i];
+        b[i] = hv[16 + i];
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) c[i] = hv[32 + i];
+    tmem_st16(tlane(tm, base), a);
+    tmem_st16(tlane(tm, base + 16), b);
+    tmem_st8(tlane(tm, base + 32), c);
+    tmem_wait_st();
+}
+
+__device__ __forceinline__ void zero_state40(uint32_t tm, uint32_t col_top, uint32_t col_bot, int qd)
+{
+    const uint32_t base = ((qd & 1) ? col_bot : col_top) + 40u * (qd >> 1);
+    float z16[16], z8[8];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) z16[i] = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) z8[i] = 0.f;
+    tmem_st16(tlane(tm, base), z16);
+    tmem_st16(tlane(tm, base + 16), z16);
+    tmem_st8(tlane(tm, base + 32), z8);
+    tmem_wait_st();
+}
+
+// This thread's 40 state columns of row m to global fp32 [256][65].
+__device__ __forceinline__ void store_state40(const float (&hv)[40], float *dst_all, int m, int qd)
+{
+    float *dst = dst_all + (int64_t)m * DS;
+    const int c0 = 40 * (qd >> 1);
+#pragma unroll
+    for (int i = 0; i < 40; ++i)
+        if (c0 + i < DS) dst[c0 + i] = hv[i];
+}
+
+// dx = (dX^ - x^ (x^ . dX^)) / max(|x|, eps) for row r, columns 16qd .. 16qd+15; dX^ from
+// TMEM column col0; x re-read from global; the four quarters exchange partial dots.
+__device__ __forceinline__ void write_dx(uint32_t tm, uint32_t col0, int r, int qd, bool valid, float rawn,
+                                         const __nv_bfloat16 *xrow, __nv_bfloat16 *dst, float *xch)
+{
+    uint32_t w[16];
+    tmem_ld16_nowait(tlane(tm, col0 + 16u * qd), w);
+    float x[16];
+    if (valid) {
+        const uint4 *x4 = reinterpret_cast<const uint4 *>(xrow + 16 * qd);
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch) {
+            const uint4 v4 = x4[ch];
+            const uint32_t ws[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                x[8 * ch + 2 * i] = bf16_lo(ws[i]);
+                x[8 * ch + 2 * i + 1] = bf16_hi(ws[i]);
+            }
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) x[i] = 0.f;
+    }
+    tmem_wait_ld();
+    float dot = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) dot = fmaf(x[i], __uint_as_float(w[i]), dot);
+    xch[threadIdx.x] = dot;
+    __syncthreads();
+    dot = xch[r] + xch[128 + r] + xch[256 + r] + xch[384 + r];
+    if (!valid) return;
+    const float n = fmaxf(rawn, kNormEps), inv = 1.f / n;
+    const float pj = rawn > kNormEps ? dot * inv * inv : 0.f;  // x^ . dX^ / |x|
+    float y[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) y[i] = (__uint_as_float(w[i]) - x[i] * pj) * inv;
+    uint4 *d4 = reinterpret_cast<uint4 *>(dst + 16 * qd);
+    d4[0] = make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
+                       pack_bf16x2(y[6], y[7]));
+    d4[1] = make_uint4(pack_bf16x2(y[8], y[9]), pack_bf16x2(y[10], y[11]), pack_bf16x2(y[12], y[13]),
+                       pack_bf16x2(y[14], y[15]));
+}
+
+// 16 consecutive TMEM columns of row r (col0 + 16qd) as bf16 to global (16 values), scaled.
+__device__ __forceinline__ void store_row16(uint32_t tm, uint32_t col0, int qd, bool valid, float scale,
+                                            __nv_bfloat16 *dst)
+{
+    uint32_t w[16];
+    tmem_ld16_nowait(tlane(tm, col0 + 16u * qd), w);
+    tmem_wait_ld();
+    if (!valid) return;
+    float y[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) y[i] = __uint_as_float(w[i]) * scale;
+    uint4 *d4 = reinterpret_cast<uint4 *>(dst + 16 * qd);
+    d4[0] = make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
+                       pack_bf16x2(y[6], y[7]));
+    d4[1] = make_uint4(pack_bf16x2(y[8], y[9]), pack_bf16x2(y[10], y[11]), pack_bf16x2(y[12], y[13]),
+                       pack_bf16x2(y[14], y[15]));
+}
+
+// ---- MMA issue helpers (one thread) ------------------------------------------------------
+// Descriptors are built once and advanced by adding (byte offset >> 4) to the start field.
+
+// proj[128][64] = X[128][64] (W_hi + W_lo)^T       (X, W: K128 tiles, K-major)
 __device__ __forceinline__ void issue_proj(uint32_t d, uint32_t x, uint32_t whi, uint32_t wlo)
 {
     constexpr uint32_t id = idesc_bf16(128, 64, 0, 0);
+    const uint64_t ax = sdesc(x, 16, 1024, LAYOUT_SW128), bh = sdesc(whi, 16, 1024, LAYOUT_SW128),
+                   bl = sdesc(wlo, 16, 1024, LAYOUT_SW128);
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk) {
-        const uint64_t a = sdesc(x + kk * 32, 16, 1024, LAYOUT_SW128);
-        mma_bf16(d, a, sdesc(whi + kk * 32, 16, 1024, LAYOUT_SW128), id, kk > 0);
-        mma_bf16(d, a, sdesc(wlo + kk * 32, 16, 1024, LAYOUT_SW128), id, 1);
+        mma_bf16(d, ax + 2 * kk, bh + 2 * kk, id, kk > 0);
+        mma_bf16(d, ax + 2 * kk, bl + 2 * kk, id, 1);
     }
 }
 
-// D[128][80] (+)= A * [V | 1] with A given per K-step (16 tokens) by a_at(kk); B from the
-// V tile (MN-major SW128) and the ones block (MN-major SW32).
-template <typename AF>
-__device__ __forceinline__ void issue_times_vt(uint32_t d, AF a_at, int a_mn, uint32_t vt, uint32_t ones,
-                                               bool acc_first)
+// D[128][N] (+)= A[128][K=256] B^T, A K-major (4 K128 tiles), B K-major rows = N (4 tiles).
+__device__ __forceinline__ void issue_k256_kk(uint32_t d, uint32_t a, uint32_t b, uint32_t idesc, bool acc_first)
 {
-    const uint32_t i64 = idesc_bf16(128, 64, a_mn, 1), i16 = idesc_bf16(128, 16, a_mn, 1);
+    const uint64_t da = sdesc(a, 16, 1024, LAYOUT_SW128), db = sdesc(b, 16, 1024, LAYOUT_SW128);
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk) {
+        const uint32_t off = ((kk >> 2) * TILE + (kk & 3) * 32) >> 4;
+        mma_bf16(d, da + off, db + off, idesc, (kk > 0 || acc_first) ? 1u : 0u);
+    }
+}
+
+// D[128][N] (+)= A[128][K=256] B, A K-major (4 K128 tiles), B = value tile MN-major with
+// 256 K-rows (atom stride VA256, N = 16 * natoms).
+__device__ __forceinline__ void issue_k256_va(uint32_t d, uint32_t a, uint32_t b, uint32_t idesc, bool acc_first)
+{
+    const uint64_t da = sdesc(a, 16, 1024, LAYOUT_SW128), db = sdesc(b, VA256, 256, LAYOUT_SW32);
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk) {
+        const uint32_t off = ((kk >> 2) * TILE + (kk & 3) * 32) >> 4;
+        mma_bf16(d, da + off, db + kk * (512 >> 4), idesc, (kk > 0 || acc_first) ? 1u : 0u);
+    }
+}
+
+// D[128][N] (+)= A[128][K=128] B with A K-major (2 K128 tiles, a_mn = 0) or MN-major
+// (M spans tiles at LBO = TILE, a_mn = 1), B = 128-row value tile MN-major (N = 16 natoms).
+__device__ __forceinline__ void issue_k128_va(uint32_t d, uint32_t a, int a_mn, uint32_t b, uint32_t idesc,
+                                              bool acc_first)
+{
+    const uint64_t da = a_mn ? sdesc(a, TILE, 1024, LAYOUT_SW128) : sdesc(a, 16, 1024, LAYOUT_SW128);
+    const uint64_t db = sdesc(b, VA128, 256, LAYOUT_SW32);
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
-        const uint64_t a = a_at(kk);
-        const uint32_t acc = (kk > 0 || acc_first) ? 1u : 0u;
-        mma_bf16(d, a, sdesc(vt + kk * 2048, TILE, 1024, LAYOUT_SW128), i64, acc);
-        mma_bf16(d + 64, a, sdesc(ones + kk * 512, 4096, 256, LAYOUT_SW32), i16, acc);
+        const uint32_t aoff = a_mn ? (kk * 2048) >> 4 : ((kk >> 2) * TILE + (kk & 3) * 32) >> 4;
+        mma_bf16(d, da + aoff, db + kk * (512 >> 4), idesc, (kk > 0 || acc_first) ? 1u : 0u);
     }
 }
 
-// H (both halves) += Phi_K^T [V | 1]
-__device__ __forceinline__ void issue_state_update(uint32_t tm, uint32_t htop, uint32_t hbot, uint32_t phk,
-                                                   uint32_t vt, uint32_t ones)
+// D[128][N] (+)= A[128][K=128] B, A K-major (2 K128 tiles), B MN-major K128 tiles spanning
+// N / 64 tiles (LBO = TILE), K-rows = 128.
+__device__ __forceinline__ void issue_k128_k128mn(uint32_t d, uint32_t a, uint32_t b, uint32_t idesc,
+                                                  bool acc_first)
 {
-    issue_times_vt(tm + htop, [&](int kk) { return sdesc(phk + kk * 2048, TILE, 1024, LAYOUT_SW128); }, 1,
-                   vt, ones, true);
-    issue_times_vt(tm + hbot,
-                   [&](int kk) { return sdesc(phk + 2 * TILE + kk * 2048, TILE, 1024, LAYOUT_SW128); }, 1,
-                   vt, ones, true);
-}
-
-// Row of the state (lane r of the H half h: feature m = 128h + r), 80 columns -> regs.
-__device__ __forceinline__ void read_state_row(uint32_t tmem, uint32_t col, float (&hv)[80])
-{
-    const uint32_t t = tmem + (lane_base() << 16) + col;
+    const uint64_t da = sdesc(a, 16, 1024, LAYOUT_SW128), db = sdesc(b, TILE, 1024, LAYOUT_SW128);
 #pragma unroll
-    for (int c = 0; c < 5; ++c) {
-        float x[16];
-        tmem_ld16(t + 16 * c, x);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) hv[16 * c + i] = x[i];
+    for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t aoff = ((kk >> 2) * TILE + (kk & 3) * 32) >> 4;
+        mma_bf16(d, da + aoff, db + kk * (2048 >> 4), idesc, (kk > 0 || acc_first) ? 1u : 0u);
     }
-    tmem_wait_ld();
 }
 
-// Stage one state row (feature m) as bf16 into the [256][64] SW128 + [256][16] SW32 tiles.
-__device__ __forceinline__ void stage_state_row(const float (&hv)[80], int m, uint8_t *hs128, uint8_t *hs32)
+// D[128][N] (+)= A B^T with A = value tile K-major (rows 128, atom stride arows*32), B = value
+// tile K-major (rows = N, atom stride brows*32), K = 16 * natoms.
+__device__ __forceinline__ void issue_va_va(uint32_t d, uint32_t a, uint32_t arows, uint32_t b, uint32_t brows,
+                                            int natoms, uint32_t idesc, bool acc_first)
 {
-    const uint32_t b128 = smem_u32(hs128) + (uint32_t)(m >> 7) * TILE;
-    const int rr = m & 127;
-#pragma unroll
-    for (int ch = 0; ch < 8; ++ch)
-        st_shared_v4(b128 + sw128_off(rr, ch), pack_bf16x2(hv[8 * ch], hv[8 * ch + 1]),
-                     pack_bf16x2(hv[8 * ch + 2], hv[8 * ch + 3]), pack_bf16x2(hv[8 * ch + 4], hv[8 * ch + 5]),
-                     pack_bf16x2(hv[8 * ch + 6], hv[8 * ch + 7]));
-    const uint32_t b32 = smem_u32(hs32);
-#pragma unroll
-    for (int ch = 0; ch < 2; ++ch)
-        st_shared_v4(b32 + sw32_off(m, ch), pack_bf16x2(hv[64 + 8 * ch], hv[65 + 8 * ch]),
-                     pack_bf16x2(hv[66 + 8 * ch], hv[67 + 8 * ch]), pack_bf16x2(hv[68 + 8 * ch], hv[69 + 8 * ch]),
-                     pack_bf16x2(hv[70 + 8 * ch], hv[71 + 8 * ch]));
+    const uint64_t da = sdesc(a, 16, 256, LAYOUT_SW32), db = sdesc(b, 16, 256, LAYOUT_SW32);
+    for (int kk = 0; kk < natoms; ++kk)
+        mma_bf16(d, da + kk * ((arows * 32) >> 4), db + kk * ((brows * 32) >> 4), idesc,
+                 (kk > 0 || acc_first) ? 1u : 0u);
 }
 
-__device__ __forceinline__ void seg_bounds(const Args &a, int seg, int64_t &t0, int64_t &t1)
+// state (two halves of 128 rows) += Phi^T [B], Phi = [128 tokens][256] K128 tiles read
+// MN-major, B = 128-row value tile (N = 80) MN-major.
+__device__ __forceinline__ void issue_state_update(uint32_t tm, uint32_t htop, uint32_t hbot, uint32_t phi,
+                                                   uint32_t va)
 {
-    t0 = (int64_t)seg * a.seg_len;
-    t1 = t0 + a.seg_len;
-    if (t1 > a.N) t1 = a.N;
+    constexpr uint32_t id = idesc_bf16(128, 80, 1, 1);
+    issue_k128_va(tm + htop, phi, 1, va, id, true);
+    issue_k128_va(tm + hbot, phi + 2 * TILE, 1, va, id, true);
+}
+
+// ==========================================================================================
+// Forward
+// ==========================================================================================
+
+namespace agg_smem {  // used by both segment aggregates (x rows and value rows double-buffered)
+constexpr uint32_t X0 = 0;
+constexpr uint32_t X1 = TILE;
+constexpr uint32_t PHI = 2 * TILE;          // Phi [128][256]
+constexpr uint32_t VA0 = PHI + 4 * TILE;    // value tile [128][80] (5 atoms)
+constexpr uint32_t VA1 = VA0 + 5 * VA128;
+constexpr uint32_t WHI = VA1 + 5 * VA128;
+constexpr uint32_t WLO = WHI + 8192;
+constexpr uint32_t RN = WLO + 8192;         // row norms [128]
+constexpr uint32_t ROWC = RN + 512;
+constexpr uint32_t ROWINV = ROWC + 512;
+constexpr uint32_t BAR = ROWINV + 512;
+constexpr uint32_t TOTAL = BAR + 64;
+}  // namespace agg_smem
+namespace agg_tmem {
+constexpr uint32_t PROJ = 0;
+constexpr uint32_t HTOP = 64;
+constexpr uint32_t HBOT = 144;
+constexpr uint32_t NCOLS = 256;
+}  // namespace agg_tmem
+
+namespace fwd_smem {
+constexpr uint32_t PHQ = 0;                  // Phi_Q [128][256]
+constexpr uint32_t XQ = PHQ;                 // q rows during the projection
+constexpr uint32_t XK = PHQ + TILE;          // k rows during the projection
+constexpr uint32_t SB = PHQ;                 // masked S as bf16 [128][128]: 2 tiles
+constexpr uint32_t PHK = PHQ + 4 * TILE;     // Phi_K [128][256]
+constexpr uint32_t HS = PHK + 4 * TILE;      // staged H [256][80] value tile (5 atoms)
+constexpr uint32_t VA = HS + 5 * VA256;      // [V | 1] [128][80]
+constexpr uint32_t WHI = VA + 5 * VA128;
+constexpr uint32_t WLO = WHI + 8192;
+constexpr uint32_t RN = WLO + 8192;          // q norms [128], k norms [128]
+constexpr uint32_t BAR = RN + 1024;
+constexpr uint32_t TOTAL = BAR + 64;
+}  // namespace fwd_smem
+namespace fwd_tmem {
+constexpr uint32_t PROJ = 0;    // [128][64] q projections, [128][64] k projections at +64
+constexpr uint32_t S = 0;       // [128][128] (reuses PROJ once the features are formed)
+constexpr uint32_t Y = 128;     // [128][80]
+constexpr uint32_t HTOP = 256;  // H rows 0..127   [128][80]
+constexpr uint32_t HBOT = 336;  // H rows 128..255 [128][80]
+constexpr uint32_t NCOLS = 512;
+}  // namespace fwd_tmem
+
+// Common prologue: barrier, TMEM allocation, W tiles.
+__device__ __forceinline__ uint32_t kernel_setup(Ctl *ctl, uint32_t ncols, const float *W, uint8_t *whi,
+                                                 uint8_t *wlo)
+{
+    if (threadIdx.x == 0) {
+        mbar_init(&ctl->bar, 1);
+        ctl->abort = 0;
+    }
+    if (threadIdx.x < 32) tmem_alloc(&ctl->tmem, ncols);
+    if (whi) load_w_split(W, whi, wlo);
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    return ctl->tmem;
+}
+
+__device__ __forceinline__ void kernel_teardown(uint32_t tm, uint32_t ncols)
+{
+    fence_before_sync();
+    __syncthreads();
+    if (threadIdx.x < 32) tmem_dealloc(tm, ncols);
 }
 
 // ------------------------------------------------------------------------------------------
-// Segment totals: H_seg = sum_{j in segment} phi(k_j) [v_j, 1]^T   (grid: nseg x BH)
+// Segment totals.  MODE 0: H_seg = sum_j phi(k_j) [v_j, 1]^T (the bucket statistics A, B of
+// zh §2.2 over the segment).  MODE 1: G_seg = sum_i phi(q_i) dY_i^T = Phi_Q'^T [dO | c] with
+// Phi_Q' = Phi_Q / den (the backward's key-side statistics).   grid: nseg x BH
+// The next chunk's rows load while this chunk is processed (double-buffered tiles).
 // ------------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(NTH, 2) tc_agg_kv(Args a)
+template <int MODE>
+__global__ void __launch_bounds__(NTH, 1) tc_agg(BwdArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = aligned_base(smem_raw);
     using namespace agg_smem;
     Ctl *ctl = reinterpret_cast<Ctl *>(sm + BAR);
+    float *rn = reinterpret_cast<float *>(sm + RN);
+    float *rowc = reinterpret_cast<float *>(sm + ROWC), *rowinv = reinterpret_cast<float *>(sm + ROWINV);
     const int seg = blockIdx.x, bh = blockIdx.y;
-    const int r = threadIdx.x & 127, h = threadIdx.x >> 7;
+    const int r = threadIdx.x & 127, qd = threadIdx.x >> 7;
     const uint32_t sb = smem_u32(sm);
-    if (threadIdx.x == 0) {
-        mbar_init(&ctl->bar, 1);
-        ctl->abort = 0;
-    }
-    if (threadIdx.x < 32) tmem_alloc(&ctl->tmem, agg_tmem::NCOLS);
-    load_w_split(a.W, sm + WHI, sm + WLO);
-    fence_before_sync();
-    __syncthreads();
-    fence_after_sync();
-    const uint32_t tm = ctl->tmem;
-    {  // zero state
-        float z[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) z[i] = 0.f;
-        const uint32_t t = tm + (lane_base() << 16) + (h ? agg_tmem::HBOT : agg_tmem::HTOP);
-#pragma unroll
-        for (int c = 0; c < 5; ++c) tmem_st16(t + 16 * c, z);
-        tmem_wait_st();
-    }
+    const __nv_bfloat16 *xsrc = MODE == 0 ? a.k : a.q;
+    const __nv_bfloat16 *vsrc = MODE == 0 ? a.v : a.dout;
+    const uint32_t tm = kernel_setup(ctl, agg_tmem::NCOLS, a.W, sm + WHI, sm + WLO);
+    zero_state40(tm, agg_tmem::HTOP, agg_tmem::HBOT, qd);
     int64_t t0, t1;
-    seg_bounds(a, seg, t0, t1);
+    seg_bounds(a.seg_len, a.N, seg, t0, t1);
     const int64_t base = (int64_t)bh * a.N;
     uint32_t phase = 0;
     bool ok = true;
-    for (int64_t c0 = t0; c0 < t1 && ok; c0 += T) {
-        const int nv = (int)(t1 - c0 < T ? t1 - c0 : T);
-        load_tile_async<NTH>(sm + XK, a.k + (base + c0) * DH, nv);
-        load_tile_async<NTH>(sm + V, a.v + (base + c0) * DH, nv);
+    if (t0 < t1) {
+        load_k128_async(sm + X0, xsrc + (base + t0) * DH, (int)(t1 - t0 < T ? t1 - t0 : T));
+        load_va_async(sm + VA0, vsrc + (base + t0) * DH, (int)(t1 - t0 < T ? t1 - t0 : T));
         cp_async_commit();
-        write_ones(sm + ONES, nv);
+    }
+    int buf = 0;
+    for (int64_t c0 = t0; c0 < t1 && ok; c0 += T, buf ^= 1) {
+        const int nv = (int)(t1 - c0 < T ? t1 - c0 : T);
+        uint8_t *x = sm + (buf ? X1 : X0), *va = sm + (buf ? VA1 : VA0);
         cp_async_wait_all();
+        __syncthreads();
+        if (c0 + T < t1) {  // next chunk's rows into the other buffers (free: their MMAs completed)
+            const int nn = (int)(t1 - c0 - T < T ? t1 - c0 - T : T);
+            load_k128_async(sm + (buf ? X0 : X1), xsrc + (base + c0 + T) * DH, nn);
+            load_va_async(sm + (buf ? VA0 : VA1), vsrc + (base + c0 + T) * DH, nn);
+            cp_async_commit();
+            prefetch_chunk(base + c0 + 2 * T, (int)(t1 - c0 - 2 * T < T ? t1 - c0 - 2 * T : T), xsrc, vsrc,
+                           MODE ? a.o : nullptr, nullptr, nullptr, MODE ? a.den : nullptr);
+        }
+        if (qd == 0) rn[r] = row_norm(x, r);
+        if (MODE == 0 && qd == 1) write_col64(va, r, r < nv ? 1.f : 0.f);
+        if (MODE == 1 && qd == 2)
+            row_scalars(r, va, a.o + (base + c0) * DH, a.den + base + c0, nv, rowc, rowinv, va);
         publish_smem();
         if (threadIdx.x == 0) {
             fence_after_sync();
-            issue_proj(tm + agg_tmem::PROJ, sb + XK, sb + WHI, sb + WLO);
+            issue_proj(tm + agg_tmem::PROJ, smem_u32(x), sb + WHI, sb + WLO);
             mma_commit(&ctl->bar);
         }
-        const float inv = 1.f / fmaxf(sqrtf(row_sqnorm(sm + XK, r)), kNormEps);
         if (!(ok = wait_mma(ctl, phase))) break;
-        features_half(tm, agg_tmem::PROJ, r, h, inv, a.beta, r < nv, sm + PHK);
+        {
+            float u[16], t[16];
+            proj_tanh(tm, agg_tmem::PROJ, qd, 1.f / fmaxf(rn[r], kNormEps), a.beta, u, t);
+            const float sc = r < nv ? (MODE == 0 ? 1.f : rowinv[r]) : 0.f;
+            write_features(t, r, qd, sc, sm + PHI);
+        }
         publish_smem();
         if (threadIdx.x == 0) {
             fence_after_sync();
-            issue_state_update(tm, agg_tmem::HTOP, agg_tmem::HBOT, sb + PHK, sb + V, sb + ONES);
+            issue_state_update(tm, agg_tmem::HTOP, agg_tmem::HBOT, sb + PHI, smem_u32(va));
             mma_commit(&ctl->bar);
         }
         ok = wait_mma(ctl, phase);
     }
+    cp_async_wait_all();
     if (ok) {
-        float hv[80];
-        read_state_row(tm, h ? agg_tmem::HBOT : agg_tmem::HTOP, hv);
-        const int m = 128 * h + r;
-        float *dst = a.agg_out + (((int64_t)bh * a.nseg + seg) * MF + m) * DS;
-#pragma unroll
-        for (int c = 0; c < DS; ++c) dst[c] = hv[c];
+        float hv[40];
+        read_state40(tm, agg_tmem::HTOP, agg_tmem::HBOT, qd, hv);
+        store_state40(hv, a.agg_out + ((int64_t)bh * a.nseg + seg) * MF * DS, 128 * (qd & 1) + r, qd);
     }
-    fence_before_sync();
-    __syncthreads();
-    if (threadIdx.x < 32) tmem_dealloc(tm, agg_tmem::NCOLS);
+    kernel_teardown(tm, agg_tmem::NCOLS);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -394,52 +790,43 @@ __global__ void __launch_bounds__(NTH, 1) tc_fwd_walk(Args a)
     uint8_t *sm = aligned_base(smem_raw);
     using namespace fwd_smem;
     Ctl *ctl = reinterpret_cast<Ctl *>(sm + BAR);
+    float *rn = reinterpret_cast<float *>(sm + RN);
     const int seg = blockIdx.x, bh = blockIdx.y;
-    const int r = threadIdx.x & 127, h = threadIdx.x >> 7;
+    const int r = threadIdx.x & 127, qd = threadIdx.x >> 7;
     const uint32_t sb = smem_u32(sm);
     const bool causal = a.causal != 0;
-    if (threadIdx.x == 0) {
-        mbar_init(&ctl->bar, 1);
-        ctl->abort = 0;
-    }
-    if (threadIdx.x < 32) tmem_alloc(&ctl->tmem, fwd_tmem::NCOLS);
-    load_w_split(a.W, sm + WHI, sm + WLO);
-    fence_before_sync();
-    __syncthreads();
-    fence_after_sync();
-    const uint32_t tm = ctl->tmem;
-    {  // start state: fp32 master into TMEM, bf16 copy into the staging tiles
-        const int m = 128 * h + r;
-        const float *src = a.state + (int64_t)bh * a.nseg * MF * DS + seg * a.state_seg_stride + (int64_t)m * DS;
-        float hv[80];
-#pragma unroll
-        for (int c = 0; c < 80; ++c) hv[c] = c < DS ? src[c] : 0.f;
-        const uint32_t t = tm + (lane_base() << 16) + (h ? fwd_tmem::HBOT : fwd_tmem::HTOP);
-#pragma unroll
-        for (int c = 0; c < 5; ++c) {
-            float x[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) x[i] = hv[16 * c + i];
-            tmem_st16(t + 16 * c, x);
-        }
-        tmem_wait_st();
-        stage_state_row(hv, m, sm + HS128, sm + HS32);
+    const uint32_t tm = kernel_setup(ctl, fwd_tmem::NCOLS, a.W, sm + WHI, sm + WLO);
+    {  // start state: fp32 master into TMEM, bf16 copy into the staging tile
+        float hv[40];
+        load_state40(a.state + (int64_t)bh * a.nseg * MF * DS + seg * a.state_seg_stride, 128 * (qd & 1) + r, qd,
+                     tm, fwd_tmem::HTOP, fwd_tmem::HBOT, hv);
+        stage40(hv, 128 * (qd & 1) + r, qd, sm + HS);
     }
     int64_t t0, t1;
-    seg_bounds(a, seg, t0, t1);
+    seg_bounds(a.seg_len, a.N, seg, t0, t1);
     const int64_t base = (int64_t)bh * a.N;
     uint32_t phase = 0;
     bool ok = true;
-    for (int64_t c0 = t0; c0 < t1 && ok; c0 += T) {
-        const int nv = (int)(t1 - c0 < T ? t1 - c0 : T);
-        load_tile_async<NTH>(sm + XQ, a.q + (base + c0) * DH, nv);
+    auto issue_loads = [&](int64_t c) {
+        const int n = (int)(t1 - c < T ? t1 - c : T);
+        load_k128_async(sm + XQ, a.q + (base + c) * DH, n);
         if (causal) {
-            load_tile_async<NTH>(sm + XK, a.k + (base + c0) * DH, nv);
-            load_tile_async<NTH>(sm + V, a.v + (base + c0) * DH, nv);
+            load_k128_async(sm + XK, a.k + (base + c) * DH, n);
+            load_va_async(sm + VA, a.v + (base + c) * DH, n);
         }
         cp_async_commit();
-        if (causal) write_ones(sm + ONES, nv);
+        prefetch_chunk(base + c + T, (int)(t1 - c - T < T ? t1 - c - T : T), a.q, causal ? a.k : nullptr,
+                       causal ? a.v : nullptr, nullptr, nullptr, nullptr);
+    };
+    if (t0 < t1) issue_loads(t0);
+    for (int64_t c0 = t0; c0 < t1 && ok; c0 += T) {
+        const int nv = (int)(t1 - c0 < T ? t1 - c0 : T);
+        const bool valid = r < nv;
         cp_async_wait_all();
+        __syncthreads();
+        if (qd == 0) rn[r] = row_norm(sm + XQ, r);
+        if (causal && qd == 1) rn[128 + r] = row_norm(sm + XK, r);
+        if (causal && qd == 2) write_col64(sm + VA, r, valid ? 1.f : 0.f);
         publish_smem();
         if (threadIdx.x == 0) {
             fence_after_sync();
@@ -447,106 +834,60 @@ __global__ void __launch_bounds__(NTH, 1) tc_fwd_walk(Args a)
             if (causal) issue_proj(tm + fwd_tmem::PROJ + 64, sb + XK, sb + WHI, sb + WLO);
             mma_commit(&ctl->bar);
         }
-        const float inv_q = 1.f / fmaxf(sqrtf(row_sqnorm(sm + XQ, r)), kNormEps);
-        const float inv_k = causal ? 1.f / fmaxf(sqrtf(row_sqnorm(sm + XK, r)), kNormEps) : 0.f;
         if (!(ok = wait_mma(ctl, phase))) break;
-        features_half(tm, fwd_tmem::PROJ, r, h, inv_q, a.beta, r < nv, sm + PHQ);
-        if (causal) features_half(tm, fwd_tmem::PROJ + 64, r, h, inv_k, a.beta, r < nv, sm + PHK);
-        publish_smem();
-        if (threadIdx.x == 0) {
-            fence_after_sync();
-            if (causal) {  // S = Phi_Q Phi_K^T
-                constexpr uint32_t id = idesc_bf16(128, 128, 0, 0);
-#pragma unroll
-                for (int kk = 0; kk < 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * TILE + (kk & 3) * 32;
-                    mma_bf16(tm + fwd_tmem::S, sdesc(sb + PHQ + off, 16, 1024, LAYOUT_SW128),
-                             sdesc(sb + PHK + off, 16, 1024, LAYOUT_SW128), id, kk > 0);
-                }
-            }
-            {  // Y = Phi_Q H_prev
-                constexpr uint32_t i64 = idesc_bf16(128, 64, 0, 1), i16 = idesc_bf16(128, 16, 0, 1);
-#pragma unroll
-                for (int kk = 0; kk < 16; ++kk) {
-                    const uint64_t aq = sdesc(sb + PHQ + (kk >> 2) * TILE + (kk & 3) * 32, 16, 1024, LAYOUT_SW128);
-                    mma_bf16(tm + fwd_tmem::Y, aq, sdesc(sb + HS128 + kk * 2048, TILE, 1024, LAYOUT_SW128), i64,
-                             kk > 0);
-                    mma_bf16(tm + fwd_tmem::Y + 64, aq, sdesc(sb + HS32 + kk * 512, 8192, 256, LAYOUT_SW32), i16,
-                             kk > 0);
-                }
-            }
-            mma_commit(&ctl->bar);
+        {
+            float u[16], t[16];
+            proj_tanh(tm, fwd_tmem::PROJ, qd, 1.f / fmaxf(rn[r], kNormEps), a.beta, u, t);
+            write_features(t, r, qd, valid ? 1.f : 0.f, sm + PHQ);
         }
+        publish_smem();
+        if (threadIdx.x == 0) {  // Y = Phi_Q H_prev, while the key features are formed
+            fence_after_sync();
+            issue_k256_va(tm + fwd_tmem::Y, sb + PHQ, sb + HS, idesc_bf16(128, 80, 0, 1), false);
+        }
+        if (causal) {
+            {
+                float u[16], t[16];
+                proj_tanh(tm, fwd_tmem::PROJ + 64, qd, 1.f / fmaxf(rn[128 + r], kNormEps), a.beta, u, t);
+                write_features(t, r, qd, valid ? 1.f : 0.f, sm + PHK);
+            }
+            publish_smem();
+            if (threadIdx.x == 0) {  // S = Phi_Q Phi_K^T
+                fence_after_sync();
+                issue_k256_kk(tm + fwd_tmem::S, sb + PHQ, sb + PHK, idesc_bf16(128, 128, 0, 0), false);
+            }
+        }
+        if (threadIdx.x == 0) mma_commit(&ctl->bar);
         if (!(ok = wait_mma(ctl, phase))) break;
         if (causal) {
-            // masked S (j <= i) as bf16: row r, columns 64h .. 64h+63
-            const uint32_t t = tm + (lane_base() << 16) + fwd_tmem::S + 64u * h;
-            const uint32_t blk = sb + SB + (uint32_t)h * TILE;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                float x[16];
-                tmem_ld16(t + 16 * c, x);
-                tmem_wait_ld();
-#pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    if (64 * h + 16 * c + i > r) x[i] = 0.f;
-                st_shared_v4(blk + sw128_off(r, 2 * c), pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]),
-                             pack_bf16x2(x[4], x[5]), pack_bf16x2(x[6], x[7]));
-                st_shared_v4(blk + sw128_off(r, 2 * c + 1), pack_bf16x2(x[8], x[9]), pack_bf16x2(x[10], x[11]),
-                             pack_bf16x2(x[12], x[13]), pack_bf16x2(x[14], x[15]));
-            }
+            mask_block(tm, fwd_tmem::S, r, qd, false, 0.f, nullptr, sm + SB);  // j <= i
             publish_smem();
             if (threadIdx.x == 0) {
                 fence_after_sync();
-                // Y += S [V | 1]
-                issue_times_vt(tm + fwd_tmem::Y,
-                               [&](int kk) {
-                                   return sdesc(sb + SB + (kk >> 2) * TILE + (kk & 3) * 32, 16, 1024,
-                                                LAYOUT_SW128);
-                               },
-                               0, sb + V, sb + ONES, true);
-                // H += Phi_K^T [V | 1]
-                issue_state_update(tm, fwd_tmem::HTOP, fwd_tmem::HBOT, sb + PHK, sb + V, sb + ONES);
+                issue_k128_va(tm + fwd_tmem::Y, sb + SB, 0, sb + VA, idesc_bf16(128, 80, 0, 1), true);  // Y += S V~
+                issue_state_update(tm, fwd_tmem::HTOP, fwd_tmem::HBOT, sb + PHK, sb + VA);  // H += Phi_K^T V~
                 mma_commit(&ctl->bar);
             }
             if (!(ok = wait_mma(ctl, phase))) break;
         }
-        {  // out = Y[:, :64] / Y[:, 64]: this thread writes columns 32h .. 32h+31 of row r
-            float y[32], dn[16];
-            const uint32_t t = tm + (lane_base() << 16) + fwd_tmem::Y;
-            float y0[16], y1[16];
-            tmem_ld16(t + 32u * h, y0);
-            tmem_ld16(t + 32u * h + 16, y1);
-            tmem_ld16(t + 64, dn);
+        if (c0 + T < t1) issue_loads(c0 + T);  // next rows land while this chunk's results leave
+        {  // out = Y[:, :64] / Y[:, 64]: columns 16qd .. 16qd+15 of row r
+            uint32_t dn[16];
+            tmem_ld16_nowait(tlane(tm, fwd_tmem::Y + 64), dn);
             tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                y[i] = y0[i];
-                y[16 + i] = y1[i];
-            }
-            if (r < nv) {
-                const float d = dn[0];
-                const float inv = d != 0.f ? 1.f / d : 0.f;
-                uint4 *dst = reinterpret_cast<uint4 *>(a.out + (base + c0 + r) * DH + 32 * h);
-#pragma unroll
-                for (int v4 = 0; v4 < 4; ++v4)
-                    dst[v4] = make_uint4(pack_bf16x2(y[8 * v4] * inv, y[8 * v4 + 1] * inv),
-                                         pack_bf16x2(y[8 * v4 + 2] * inv, y[8 * v4 + 3] * inv),
-                                         pack_bf16x2(y[8 * v4 + 4] * inv, y[8 * v4 + 5] * inv),
-                                         pack_bf16x2(y[8 * v4 + 6] * inv, y[8 * v4 + 7] * inv));
-                if (h == 0 && a.den) a.den[base + c0 + r] = d;
-            }
+            const float d = __uint_as_float(dn[0]);
+            store_row16(tm, fwd_tmem::Y, qd, valid, d != 0.f ? 1.f / d : 0.f, a.out + (base + c0 + r) * DH);
+            if (qd == 0 && valid && a.den) a.den[base + c0 + r] = d;
         }
         if (causal) {  // stage the updated state for the next chunk's read-out
-            float hv[80];
-            read_state_row(tm, h ? fwd_tmem::HBOT : fwd_tmem::HTOP, hv);
-            stage_state_row(hv, 128 * h + r, sm + HS128, sm + HS32);
+            float hv[40];
+            read_state40(tm, fwd_tmem::HTOP, fwd_tmem::HBOT, qd, hv);
+            stage40(hv, 128 * (qd & 1) + r, qd, sm + HS);
         }
         publish_smem();
     }
-    fence_before_sync();
-    __syncthreads();
-    if (threadIdx.x < 32) tmem_dealloc(tm, fwd_tmem::NCOLS);
+    cp_async_wait_all();
+    kernel_teardown(tm, fwd_tmem::NCOLS);
 }
 
 // ==========================================================================================
@@ -568,440 +909,39 @@ __global__ void __launch_bounds__(NTH, 1) tc_fwd_walk(Args a)
 // dq side reads the state as a bf16 hi + lo pair.
 // ==========================================================================================
 
-struct BwdArgs {
-    const __nv_bfloat16 *q, *k, *v, *o, *dout;
-    const float *den, *W;
-    __nv_bfloat16 *dq, *dk, *dv;
-    const float *state;
-    int64_t state_seg_stride;
-    float *agg_out;
-    int64_t N, seg_len;
-    int nseg;
-    float beta;
-    int causal;
-};
-
-// Per-row scalars of a chunk: rowc[r] = c_r = -(dO_r . o_r), rowinv[r] = 1/den_r (0 beyond
-// nvalid); dO read from its SW128 tile, o from global.  Optionally the SW32 block dc32
-// gets c_r (bf16) in column 0.  Threads 0..127, one row each.
-__device__ __forceinline__ void row_scalars(const uint8_t *do_tile, const __nv_bfloat16 *o, const float *den,
-                                            int nvalid, float *rowc, float *rowinv, uint8_t *dc32)
-{
-    if (threadIdx.x >= T) return;
-    const int r = threadIdx.x;
-    float c = 0.f, inv = 0.f;
-    if (r < nvalid) {
-        const uint32_t a = smem_u32(do_tile);
-        const uint4 *o4 = reinterpret_cast<const uint4 *>(o + (int64_t)r * DH);
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-            const uint4 g = ld_shared_v4(a + sw128_off(r, ch)), ov = o4[ch];
-            const uint32_t gw[4] = {g.x, g.y, g.z, g.w}, ow[4] = {ov.x, ov.y, ov.z, ov.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                c = fmaf(bf16_lo(gw[i]), bf16_lo(ow[i]), c);
-                c = fmaf(bf16_hi(gw[i]), bf16_hi(ow[i]), c);
-            }
-        }
-        c = -c;
-        const float dn = den[r];
-        inv = dn != 0.f ? 1.f / dn : 0.f;
-    }
-    rowc[r] = c;
-    rowinv[r] = inv;
-    if (dc32) {
-        const uint32_t b = smem_u32(dc32);
-        st_shared_v4(b + sw32_off(r, 0), pack_bf16x2(c, 0.f), 0u, 0u, 0u);
-        st_shared_v4(b + sw32_off(r, 1), 0u, 0u, 0u, 0u);
-    }
-}
-
-// u = tanh(proj / |x|) and t = tanh(beta u) of the 32 projections of half h (8 tables),
-// kept in registers for the feature-map VJP.
-__device__ __forceinline__ void proj_keep(uint32_t tmem, uint32_t col0, int h, float inv_norm, float beta,
-                                          float (&u)[32], float (&t)[32])
-{
-    float a[16], b[16];
-    const uint32_t ta = tmem + (lane_base() << 16) + col0 + 32u * h;
-    tmem_ld16(ta, a);
-    tmem_ld16(ta + 16, b);
-    tmem_wait_ld();
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        u[i] = tanh_fast(a[i] * inv_norm);
-        u[16 + i] = tanh_fast(b[i] * inv_norm);
-    }
-#pragma unroll
-    for (int i = 0; i < 32; ++i) t[i] = tanh_fast(beta * u[i]);
-}
-
-// Features of the 8 tables of half h from t = tanh(beta u), times `scale`, as bf16 into row r
-// of the Phi tile [128][256].
-__device__ __forceinline__ void write_features(const float (&t)[32], int r, int h, float scale, uint8_t *phi)
-{
-    const uint32_t base = smem_u32(phi);
-#pragma unroll
-    for (int l = 0; l < 8; ++l) {
-        float f[16];
-        f[0] = scale;
-#pragma unroll
-        for (int p = 0; p < 4; ++p) {
-            const float s1 = 0.5f + 0.5f * t[4 * l + p], s0 = 0.5f - 0.5f * t[4 * l + p];
-            const int hh = 1 << p;
-#pragma unroll
-            for (int c = 0; c < hh; ++c) {
-                f[c + hh] = f[c] * s1;
-                f[c] *= s0;
-            }
-        }
-        const int tl = 8 * h + l;
-        const uint32_t blk = base + (uint32_t)(tl >> 2) * TILE;
-        const int ch = (tl & 3) * 2;
-        st_shared_v4(blk + sw128_off(r, ch), pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
-                     pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
-        st_shared_v4(blk + sw128_off(r, ch + 1), pack_bf16x2(f[8], f[9]), pack_bf16x2(f[10], f[11]),
-                     pack_bf16x2(f[12], f[13]), pack_bf16x2(f[14], f[15]));
-    }
-}
-
-// Feature-map VJP for the 8 tables of half h.  dphi[m] = (D[m] + add_scale * add_vec[m]) * mul
-// with D read from TMEM columns col0 + 128h .. (16 per table) and add_vec (features, fp32,
-// shared memory) optional; writes dp~ (32 values) as bf16 into row r of the DP tile
-// ([128][64] SW128, projections 32h .. 32h+31).
-__device__ __forceinline__ void features_vjp_half(uint32_t tmem, uint32_t col0, int r, int h, float beta,
-                                                  bool valid, const float (&u)[32], const float (&t)[32],
-                                                  const float *add_vec, float add_scale, float mul,
-                                                  uint8_t *dp_tile)
-{
-    float dp[32];
-    const uint32_t ta = tmem + (lane_base() << 16) + col0 + 128u * h;
-#pragma unroll
-    for (int l = 0; l < 8; ++l) {
-        float g[16];
-        tmem_ld16(ta + 16 * l, g);
-        tmem_wait_ld();
-        if (add_vec) {
-            const float *av = add_vec + 128 * h + 16 * l;
-#pragma unroll
-            for (int c = 0; c < 16; ++c) g[c] = fmaf(add_scale, av[c], g[c]) * mul;
-        }
-        float f[16];
-        f[0] = 1.f;
-#pragma unroll
-        for (int p = 0; p < 4; ++p) {
-            const float s1 = 0.5f + 0.5f * t[4 * l + p], s0 = 0.5f - 0.5f * t[4 * l + p];
-            const int hh = 1 << p;
-#pragma unroll
-            for (int c = 0; c < hh; ++c) {
-                f[c + hh] = f[c] * s1;
-                f[c] *= s0;
-            }
-        }
-        float dot = 0.f;
-#pragma unroll
-        for (int c = 0; c < 16; ++c) dot = fmaf(f[c], g[c], dot);
-        float du[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {
-            const float dz = f[c] * (g[c] - dot);
-#pragma unroll
-            for (int p = 0; p < 4; ++p) du[p] += ((c >> p) & 1) ? dz : -dz;
-        }
-#pragma unroll
-        for (int p = 0; p < 4; ++p) {
-            const float uu = u[4 * l + p];
-            dp[4 * l + p] = valid ? beta * du[p] * (1.f - uu * uu) : 0.f;
-        }
-    }
-    const uint32_t b = smem_u32(dp_tile);
-#pragma unroll
-    for (int ch = 0; ch < 4; ++ch)
-        st_shared_v4(b + sw128_off(r, 4 * h + ch), pack_bf16x2(dp[8 * ch], dp[8 * ch + 1]),
-                     pack_bf16x2(dp[8 * ch + 2], dp[8 * ch + 3]), pack_bf16x2(dp[8 * ch + 4], dp[8 * ch + 5]),
-                     pack_bf16x2(dp[8 * ch + 6], dp[8 * ch + 7]));
-}
-
 // D[128][64] = DP[128][64] (W_hi + W_lo): W as MN-major B (rows = projections, cols = d).
 __device__ __forceinline__ void issue_dxhat(uint32_t d, uint32_t dp, uint32_t whi, uint32_t wlo)
 {
     constexpr uint32_t id = idesc_bf16(128, 64, 0, 1);
+    const uint64_t da = sdesc(dp, 16, 1024, LAYOUT_SW128), bh = sdesc(whi, TILE, 1024, LAYOUT_SW128),
+                   bl = sdesc(wlo, TILE, 1024, LAYOUT_SW128);
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk) {
-        const uint64_t a = sdesc(dp + kk * 32, 16, 1024, LAYOUT_SW128);
-        mma_bf16(d, a, sdesc(whi + kk * 2048, TILE, 1024, LAYOUT_SW128), id, kk > 0);
-        mma_bf16(d, a, sdesc(wlo + kk * 2048, TILE, 1024, LAYOUT_SW128), id, 1);
+        mma_bf16(d, da + 2 * kk, bh + kk * (2048 >> 4), id, kk > 0);
+        mma_bf16(d, da + 2 * kk, bl + kk * (2048 >> 4), id, 1);
     }
 }
 
-// D[128][N] (+)= A[128][64] B[N][64]^T, both K-major SW128.
-__device__ __forceinline__ void issue_k64(uint32_t d, uint32_t a, uint32_t b, uint32_t idesc, bool acc_first)
-{
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(d, sdesc(a + kk * 32, 16, 1024, LAYOUT_SW128), sdesc(b + kk * 32, 16, 1024, LAYOUT_SW128), idesc,
-                 (kk > 0 || acc_first) ? 1u : 0u);
-}
-
-// D[128][N] (+)= A[128][80] B[N][80]^T, both K-major, K split as 64 (SW128) + 16 (SW32).
-__device__ __forceinline__ void issue_k80(uint32_t d, uint32_t a128, uint32_t a32, uint32_t b128, uint32_t b32,
-                                          uint32_t idesc, bool acc_first)
-{
-    issue_k64(d, a128, b128, idesc, acc_first);
-    mma_bf16(d, sdesc(a32, 16, 256, LAYOUT_SW32), sdesc(b32, 16, 256, LAYOUT_SW32), idesc, 1u);
-}
-
-// D[128][N] (+)= A[128][128] B where A = K-major bf16 [128][128] (2 tiles) and B is
-// MN-major [K=128 rows][N] spanning N/64 tiles (LBO = TILE).
-__device__ __forceinline__ void issue_tt_times(uint32_t d, uint32_t a, uint32_t b, uint32_t idesc, bool acc_first)
-{
-#pragma unroll
-    for (int kk = 0; kk < 8; ++kk)
-        mma_bf16(d, sdesc(a + (kk >> 2) * TILE + (kk & 3) * 32, 16, 1024, LAYOUT_SW128),
-                 sdesc(b + kk * 2048, TILE, 1024, LAYOUT_SW128), idesc, (kk > 0 || acc_first) ? 1u : 0u);
-}
-
-// Masked T x T block from TMEM (row r, columns col0 + 64h ..) to bf16 K-major tile h of dst.
-// Adds add_row to every element of the row and add_col[col] per column (either optional)
-// before masking; keep_upper keeps column >= row (else column <= row).
-__device__ __forceinline__ void mask_block_to_smem(uint32_t tmem, uint32_t col0, int r, int h, bool keep_upper,
-                                                   float add_row, const float *add_col, uint8_t *dst)
-{
-    const uint32_t t = tmem + (lane_base() << 16) + col0 + 64u * h;
-    const uint32_t blk = smem_u32(dst) + (uint32_t)h * TILE;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        float x[16];
-        tmem_ld16(t + 16 * c, x);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const int col = 64 * h + 16 * c + i;
-            float y = x[i] + add_row;
-            if (add_col) y += add_col[col];
-            x[i] = (keep_upper ? (col < r) : (col > r)) ? 0.f : y;
-        }
-        st_shared_v4(blk + sw128_off(r, 2 * c), pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]),
-                     pack_bf16x2(x[4], x[5]), pack_bf16x2(x[6], x[7]));
-        st_shared_v4(blk + sw128_off(r, 2 * c + 1), pack_bf16x2(x[8], x[9]), pack_bf16x2(x[10], x[11]),
-                     pack_bf16x2(x[12], x[13]), pack_bf16x2(x[14], x[15]));
-    }
-}
-
-// dx = (dX^ - x^ (x^ . dX^)) / max(|x|, eps) for row r, columns 32h .. 32h+31; dX^ from TMEM
-// column col0; x re-read from global; the two halves exchange partial dots through xch.
-__device__ __forceinline__ void write_dx(uint32_t tmem, uint32_t col0, int r, int h, bool valid, float rawn,
-                                         const __nv_bfloat16 *xrow, __nv_bfloat16 *dst, float *xch)
-{
-    float g[32];
-    {
-        float a[16], b[16];
-        const uint32_t ta = tmem + (lane_base() << 16) + col0 + 32u * h;
-        tmem_ld16(ta, a);
-        tmem_ld16(ta + 16, b);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            g[i] = a[i];
-            g[16 + i] = b[i];
-        }
-    }
-    float x[32];
-    float dot = 0.f;
-    if (valid) {
-        const uint4 *x4 = reinterpret_cast<const uint4 *>(xrow + 32 * h);
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-            const uint4 w = x4[ch];
-            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                x[8 * ch + 2 * i] = bf16_lo(ws[i]);
-                x[8 * ch + 2 * i + 1] = bf16_hi(ws[i]);
-            }
-        }
-#pragma unroll
-        for (int i = 0; i < 32; ++i) dot = fmaf(x[i], g[i], dot);
-    }
-    xch[threadIdx.x] = dot;
-    __syncthreads();
-    dot += xch[threadIdx.x ^ 128];
-    if (!valid) return;
-    const float n = fmaxf(rawn, kNormEps), inv = 1.f / n;
-    const float proj = rawn > kNormEps ? dot * inv * inv : 0.f;  // x^ . dX^ / |x|
-    uint4 *d4 = reinterpret_cast<uint4 *>(dst + 32 * h);
-#pragma unroll
-    for (int ch = 0; ch < 4; ++ch) {
-        float y[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) y[i] = (g[8 * ch + i] - x[8 * ch + i] * proj) * inv;
-        d4[ch] = make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
-                            pack_bf16x2(y[6], y[7]));
-    }
-}
-
-__device__ __forceinline__ void bseg_bounds(const BwdArgs &a, int seg, int64_t &t0, int64_t &t1)
-{
-    t0 = (int64_t)seg * a.seg_len;
-    t1 = t0 + a.seg_len;
-    if (t1 > a.N) t1 = a.N;
-}
-
-// Stage one state row (feature m) as a bf16 hi + lo pair of [256][64] SW128 tiles plus its
-// ones column in fp32.
-__device__ __forceinline__ void stage_state_hilo(const float (&hv)[80], int m, uint8_t *hi, uint8_t *lo, float *col64)
-{
-    const uint32_t bh_ = smem_u32(hi) + (uint32_t)(m >> 7) * TILE, bl = smem_u32(lo) + (uint32_t)(m >> 7) * TILE;
-    const int rr = m & 127;
-#pragma unroll
-    for (int ch = 0; ch < 8; ++ch) {
-        uint32_t wh[4], wl[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float x0 = hv[8 * ch + 2 * i], x1 = hv[8 * ch + 2 * i + 1];
-            wh[i] = pack_bf16x2(x0, x1);
-            wl[i] = pack_bf16x2(x0 - bf16_lo(wh[i]), x1 - bf16_hi(wh[i]));
-        }
-        st_shared_v4(bh_ + sw128_off(rr, ch), wh[0], wh[1], wh[2], wh[3]);
-        st_shared_v4(bl + sw128_off(rr, ch), wl[0], wl[1], wl[2], wl[3]);
-    }
-    col64[m] = hv[64];
-}
-
-// A walk's start state row (global fp32 [256][65]) for feature m = 128h + r -> registers,
-// then into TMEM (the half's columns).
-__device__ __forceinline__ void load_start_row(const float *src_all, int h, int r, uint32_t tm, uint32_t htop,
-                                               uint32_t hbot, float (&hv)[80])
-{
-    const float *src = src_all + (int64_t)(128 * h + r) * DS;
-#pragma unroll
-    for (int c = 0; c < 80; ++c) hv[c] = c < DS ? src[c] : 0.f;
-    const uint32_t t = tm + (lane_base() << 16) + (h ? hbot : htop);
-#pragma unroll
-    for (int c = 0; c < 5; ++c) {
-        float x[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) x[i] = hv[16 * c + i];
-        tmem_st16(t + 16 * c, x);
-    }
-    tmem_wait_st();
-}
-
-// ------------------------------------------------------------------------------------------
-// Segment totals of the backward's key side: G_seg = sum_{i in segment} phi(q_i) dY_i^T,
-// formed as Phi_Q'^T [dO | c] with Phi_Q' = Phi_Q / den.
-// ------------------------------------------------------------------------------------------
-namespace aggq_smem {
-constexpr uint32_t PHQ = 0;
-constexpr uint32_t XQ = PHQ;
-constexpr uint32_t DO = PHQ + 4 * TILE;
-constexpr uint32_t DC32 = DO + TILE;
-constexpr uint32_t WHI = DC32 + 4096;
-constexpr uint32_t WLO = WHI + 8192;
-constexpr uint32_t ROWC = WLO + 8192;
-constexpr uint32_t ROWINV = ROWC + 512;
-constexpr uint32_t BAR = ROWINV + 512;
-constexpr uint32_t TOTAL = BAR + 64;
-}  // namespace aggq_smem
-
-__global__ void __launch_bounds__(NTH, 2) tc_agg_qdy(BwdArgs a)
-{
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = aligned_base(smem_raw);
-    using namespace aggq_smem;
-    Ctl *ctl = reinterpret_cast<Ctl *>(sm + BAR);
-    float *rowc = reinterpret_cast<float *>(sm + ROWC), *rowinv = reinterpret_cast<float *>(sm + ROWINV);
-    const int seg = blockIdx.x, bh = blockIdx.y;
-    const int r = threadIdx.x & 127, h = threadIdx.x >> 7;
-    const uint32_t sb = smem_u32(sm);
-    if (threadIdx.x == 0) {
-        mbar_init(&ctl->bar, 1);
-        ctl->abort = 0;
-    }
-    if (threadIdx.x < 32) tmem_alloc(&ctl->tmem, agg_tmem::NCOLS);
-    load_w_split(a.W, sm + WHI, sm + WLO);
-    fence_before_sync();
-    __syncthreads();
-    fence_after_sync();
-    const uint32_t tm = ctl->tmem;
-    {
-        float z[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) z[i] = 0.f;
-        const uint32_t t = tm + (lane_base() << 16) + (h ? agg_tmem::HBOT : agg_tmem::HTOP);
-#pragma unroll
-        for (int c = 0; c < 5; ++c) tmem_st16(t + 16 * c, z);
-        tmem_wait_st();
-    }
-    int64_t t0, t1;
-    bseg_bounds(a, seg, t0, t1);
-    const int64_t base = (int64_t)bh * a.N;
-    uint32_t phase = 0;
-    bool ok = true;
-    for (int64_t c0 = t0; c0 < t1 && ok; c0 += T) {
-        const int nv = (int)(t1 - c0 < T ? t1 - c0 : T);
-        load_tile_async<NTH>(sm + XQ, a.q + (base + c0) * DH, nv);
-        load_tile_async<NTH>(sm + DO, a.dout + (base + c0) * DH, nv);
-        cp_async_commit();
-        cp_async_wait_all();
-        __syncthreads();
-        row_scalars(sm + DO, a.o + (base + c0) * DH, a.den + base + c0, nv, rowc, rowinv, sm + DC32);
-        publish_smem();
-        if (threadIdx.x == 0) {
-            fence_after_sync();
-            issue_proj(tm + agg_tmem::PROJ, sb + XQ, sb + WHI, sb + WLO);
-            mma_commit(&ctl->bar);
-        }
-        const float inv = 1.f / fmaxf(sqrtf(row_sqnorm(sm + XQ, r)), kNormEps);
-        if (!(ok = wait_mma(ctl, phase))) break;
-        {
-            float u[32], t[32];
-            proj_keep(tm, agg_tmem::PROJ, h, inv, a.beta, u, t);
-            write_features(t, r, h, r < nv ? rowinv[r] : 0.f, sm + PHQ);
-        }
-        publish_smem();
-        if (threadIdx.x == 0) {
-            fence_after_sync();
-            issue_state_update(tm, agg_tmem::HTOP, agg_tmem::HBOT, sb + PHQ, sb + DO, sb + DC32);
-            mma_commit(&ctl->bar);
-        }
-        ok = wait_mma(ctl, phase);
-    }
-    if (ok) {
-        float hv[80];
-        read_state_row(tm, h ? agg_tmem::HBOT : agg_tmem::HTOP, hv);
-        const int m = 128 * h + r;
-        float *dst = a.agg_out + (((int64_t)bh * a.nseg + seg) * MF + m) * DS;
-#pragma unroll
-        for (int c = 0; c < DS; ++c) dst[c] = hv[c];
-    }
-    fence_before_sync();
-    __syncthreads();
-    if (threadIdx.x < 32) tmem_dealloc(tm, agg_tmem::NCOLS);
-}
-
-// ------------------------------------------------------------------------------------------
-// dq walk (chunks in order, prefix state H)
-// ------------------------------------------------------------------------------------------
 namespace bq_smem {
-constexpr uint32_t RA = 0;               // k rows at load; Phi_K [128][256] after the features
+constexpr uint32_t RA = 0;                 // k rows at load; Phi_K [128][256] after the features
 constexpr uint32_t XK = RA;
 constexpr uint32_t PHK = RA;
-constexpr uint32_t RB = 4 * TILE;        // q rows + W at load; masked P''; dP~ + W at the end
+constexpr uint32_t RB = 4 * TILE;          // q rows + W at load; masked P''; dP~ + W at the end
 constexpr uint32_t XQ = RB;
 constexpr uint32_t PB = RB;
 constexpr uint32_t DP = RB;
 constexpr uint32_t WHI = RB + TILE;
 constexpr uint32_t WLO = RB + TILE + 8192;
-constexpr uint32_t V = RB + 2 * TILE;
-constexpr uint32_t ONES = V + TILE;
-constexpr uint32_t DO = ONES + 4096;     // dO rows [128][64]
-constexpr uint32_t HSHI = DO + TILE;     // staged H[:, :64], bf16 hi  [256][64]
-constexpr uint32_t HSLO = HSHI + 2 * TILE;  // and lo
-constexpr uint32_t HDEN = HSLO + 2 * TILE;  // H[:, 64] fp32 [256]
+constexpr uint32_t VA = RB + 2 * TILE;     // [V | 1] [128][80]
+constexpr uint32_t DOV = VA + 5 * VA128;   // dO [128][64] (4 atoms)
+constexpr uint32_t HSHI = DOV + 4 * VA128; // staged H[:, :64], bf16 hi  [256][64] (4 atoms)
+constexpr uint32_t HSLO = HSHI + 4 * VA256;  // and lo
+constexpr uint32_t HDEN = HSLO + 4 * VA256;  // H[:, 64] fp32 [256]
 constexpr uint32_t ROWC = HDEN + 1024;
 constexpr uint32_t ROWINV = ROWC + 512;
-constexpr uint32_t XCH = ROWINV + 512;
-constexpr uint32_t BAR = XCH + 1024;
+constexpr uint32_t RN = ROWINV + 512;
+constexpr uint32_t XCH = RN + 1024;
+constexpr uint32_t BAR = XCH + 2048;
 constexpr uint32_t TOTAL = BAR + 64;
 }  // namespace bq_smem
 namespace bq_tmem {
@@ -1014,6 +954,9 @@ constexpr uint32_t HBOT = 336;
 constexpr uint32_t NCOLS = 512;
 }  // namespace bq_tmem
 
+// ------------------------------------------------------------------------------------------
+// dq walk (chunks in order, prefix state H)
+// ------------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(NTH, 1) tc_bwd_q_walk(BwdArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
@@ -1022,45 +965,51 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_q_walk(BwdArgs a)
     Ctl *ctl = reinterpret_cast<Ctl *>(sm + BAR);
     float *xch = reinterpret_cast<float *>(sm + XCH), *hden = reinterpret_cast<float *>(sm + HDEN);
     float *rowc = reinterpret_cast<float *>(sm + ROWC), *rowinv = reinterpret_cast<float *>(sm + ROWINV);
+    float *rn = reinterpret_cast<float *>(sm + RN);
     const int seg = blockIdx.x, bh = blockIdx.y;
-    const int r = threadIdx.x & 127, h = threadIdx.x >> 7;
+    const int r = threadIdx.x & 127, qd = threadIdx.x >> 7;
     const uint32_t sb = smem_u32(sm);
     const bool causal = a.causal != 0;
-    if (threadIdx.x == 0) {
-        mbar_init(&ctl->bar, 1);
-        ctl->abort = 0;
-    }
-    if (threadIdx.x < 32) tmem_alloc(&ctl->tmem, bq_tmem::NCOLS);
-    fence_before_sync();
-    __syncthreads();
-    fence_after_sync();
-    const uint32_t tm = ctl->tmem;
+    const uint32_t tm = kernel_setup(ctl, bq_tmem::NCOLS, a.W, sm + WHI, sm + WLO);
     {
-        float hv[80];
-        load_start_row(a.state + (int64_t)bh * a.nseg * MF * DS + seg * a.state_seg_stride, h, r, tm,
-                       bq_tmem::HTOP, bq_tmem::HBOT, hv);
-        stage_state_hilo(hv, 128 * h + r, sm + HSHI, sm + HSLO, hden);
+        float hv[40];
+        load_state40(a.state + (int64_t)bh * a.nseg * MF * DS + seg * a.state_seg_stride, 128 * (qd & 1) + r, qd,
+                     tm, bq_tmem::HTOP, bq_tmem::HBOT, hv);
+        stage40_hilo(hv, 128 * (qd & 1) + r, qd, sm + HSHI, sm + HSLO, hden);
     }
     int64_t t0, t1;
-    bseg_bounds(a, seg, t0, t1);
+    seg_bounds(a.seg_len, a.N, seg, t0, t1);
     const int64_t base = (int64_t)bh * a.N;
     uint32_t phase = 0;
     bool ok = true;
+    auto issue_kv_do = [&](int64_t c) {  // k, v, dO rows of chunk c
+        const int n = (int)(t1 - c < T ? t1 - c : T);
+        load_va_async(sm + DOV, a.dout + (base + c) * DH, n);
+        if (causal) {
+            load_k128_async(sm + XK, a.k + (base + c) * DH, n);
+            load_va_async(sm + VA, a.v + (base + c) * DH, n);
+        }
+        cp_async_commit();
+        prefetch_chunk(base + c + T, (int)(t1 - c - T < T ? t1 - c - T : T), a.q, a.dout, a.o,
+                       causal ? a.k : nullptr, causal ? a.v : nullptr, a.den);
+    };
+    auto issue_q = [&](int64_t c) {
+        load_k128_async(sm + XQ, a.q + (base + c) * DH, (int)(t1 - c < T ? t1 - c : T));
+        cp_async_commit();
+    };
+    if (t0 < t1) {
+        issue_kv_do(t0);
+        issue_q(t0);
+    }
     for (int64_t c0 = t0; c0 < t1 && ok; c0 += T) {
         const int nv = (int)(t1 - c0 < T ? t1 - c0 : T);
         const bool valid = r < nv;
-        load_tile_async<NTH>(sm + XQ, a.q + (base + c0) * DH, nv);
-        load_tile_async<NTH>(sm + DO, a.dout + (base + c0) * DH, nv);
-        if (causal) {
-            load_tile_async<NTH>(sm + XK, a.k + (base + c0) * DH, nv);
-            load_tile_async<NTH>(sm + V, a.v + (base + c0) * DH, nv);
-        }
-        cp_async_commit();
-        load_w_split(a.W, sm + WHI, sm + WLO);
-        if (causal) write_ones(sm + ONES, nv);
         cp_async_wait_all();
         __syncthreads();
-        row_scalars(sm + DO, a.o + (base + c0) * DH, a.den + base + c0, nv, rowc, rowinv, nullptr);
+        if (qd == 0) rn[r] = row_norm(sm + XQ, r);
+        if (causal && qd == 1) rn[128 + r] = row_norm(sm + XK, r);
+        if (qd == 2) row_scalars(r, sm + DOV, a.o + (base + c0) * DH, a.den + base + c0, nv, rowc, rowinv, nullptr);
+        if (causal && qd == 3) write_col64(sm + VA, r, valid ? 1.f : 0.f);
         publish_smem();
         if (threadIdx.x == 0) {
             fence_after_sync();
@@ -1068,39 +1017,42 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_q_walk(BwdArgs a)
             if (causal) issue_proj(tm + bq_tmem::PROJ + 64, sb + XK, sb + WHI, sb + WLO);
             mma_commit(&ctl->bar);
         }
-        const float raw_q = sqrtf(row_sqnorm(sm + XQ, r));
-        const float inv_q = 1.f / fmaxf(raw_q, kNormEps);
-        const float inv_k = causal ? 1.f / fmaxf(sqrtf(row_sqnorm(sm + XK, r)), kNormEps) : 0.f;
-        const float c_r = rowc[r], invden_r = rowinv[r];
         if (!(ok = wait_mma(ctl, phase))) break;
-        float u[32], t[32];
-        proj_keep(tm, bq_tmem::PROJ, h, inv_q, a.beta, u, t);
-        if (causal) features_half(tm, bq_tmem::PROJ + 64, r, h, inv_k, a.beta, valid, sm + PHK);
+        const float raw_q = rn[r];
+        const float c_r = rowc[r], invden_r = rowinv[r];
+        float u[16], t[16];
+        proj_tanh(tm, bq_tmem::PROJ, qd, 1.f / fmaxf(raw_q, kNormEps), a.beta, u, t);
+        if (causal) {
+            float uk[16], tk[16];
+            proj_tanh(tm, bq_tmem::PROJ + 64, qd, 1.f / fmaxf(rn[128 + r], kNormEps), a.beta, uk, tk);
+            write_features(tk, r, qd, valid ? 1.f : 0.f, sm + PHK);
+        }
         publish_smem();
         if (causal) {
             if (threadIdx.x == 0) {  // P'' = dO V^T
                 fence_after_sync();
-                issue_k64(tm + bq_tmem::P, sb + DO, sb + V, idesc_bf16(128, 128, 0, 0), false);
+                issue_va_va(tm + bq_tmem::P, sb + DOV, T, sb + VA, T, 4, idesc_bf16(128, 128, 0, 0), false);
                 mma_commit(&ctl->bar);
             }
             if (!(ok = wait_mma(ctl, phase))) break;
-            mask_block_to_smem(tm, bq_tmem::P, r, h, false, c_r, nullptr, sm + PB);  // v_j.dO_i + c_i, j <= i
+            mask_block(tm, bq_tmem::P, r, qd, false, c_r, nullptr, sm + PB);  // v_j.dO_i + c_i, j <= i
             publish_smem();
         }
         if (threadIdx.x == 0) {
             fence_after_sync();
             // D = dO H_prev[:, :64]^T (+ tril(P'') Phi_K)
-            issue_k64(tm + bq_tmem::DPHI, sb + DO, sb + HSHI, idesc_bf16(128, 256, 0, 0), false);
-            issue_k64(tm + bq_tmem::DPHI, sb + DO, sb + HSLO, idesc_bf16(128, 256, 0, 0), true);
+            issue_va_va(tm + bq_tmem::DPHI, sb + DOV, T, sb + HSHI, 256, 4, idesc_bf16(128, 256, 0, 0), false);
+            issue_va_va(tm + bq_tmem::DPHI, sb + DOV, T, sb + HSLO, 256, 4, idesc_bf16(128, 256, 0, 0), true);
             if (causal) {
-                issue_tt_times(tm + bq_tmem::DPHI, sb + PB, sb + PHK, idesc_bf16(128, 256, 0, 1), true);
-                issue_state_update(tm, bq_tmem::HTOP, bq_tmem::HBOT, sb + PHK, sb + V, sb + ONES);
+                issue_k128_k128mn(tm + bq_tmem::DPHI, sb + PB, sb + PHK, idesc_bf16(128, 256, 0, 1), true);
+                issue_state_update(tm, bq_tmem::HTOP, bq_tmem::HBOT, sb + PHK, sb + VA);
             }
             mma_commit(&ctl->bar);
         }
         if (!(ok = wait_mma(ctl, phase))) break;
+        if (c0 + T < t1) issue_kv_do(c0 + T);  // Phi_K, V~ and dO are free now
         // dphi = (D + c_i H_prev[:, 64]) / den_i
-        features_vjp_half(tm, bq_tmem::DPHI, r, h, a.beta, valid, u, t, hden, c_r, invden_r, sm + DP);
+        features_vjp(tm, bq_tmem::DPHI, r, qd, a.beta, valid, u, t, hden, c_r, invden_r, sm + DP);
         load_w_split(a.W, sm + WHI, sm + WLO);
         publish_smem();
         if (threadIdx.x == 0) {
@@ -1109,44 +1061,37 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_q_walk(BwdArgs a)
             mma_commit(&ctl->bar);
         }
         if (!(ok = wait_mma(ctl, phase))) break;
-        write_dx(tm, bq_tmem::DX, r, h, valid, raw_q, a.q + (base + c0 + r) * DH, a.dq + (base + c0 + r) * DH, xch);
+        if (c0 + T < t1) issue_q(c0 + T);  // dP~ is consumed; W stays for the next projection
+        write_dx(tm, bq_tmem::DX, r, qd, valid, raw_q, a.q + (base + c0 + r) * DH, a.dq + (base + c0 + r) * DH, xch);
         if (causal) {
-            float hv[80];
-            read_state_row(tm, h ? bq_tmem::HBOT : bq_tmem::HTOP, hv);
-            stage_state_hilo(hv, 128 * h + r, sm + HSHI, sm + HSLO, hden);
+            float hv[40];
+            read_state40(tm, bq_tmem::HTOP, bq_tmem::HBOT, qd, hv);
+            stage40_hilo(hv, 128 * (qd & 1) + r, qd, sm + HSHI, sm + HSLO, hden);
         }
         publish_smem();
     }
-    fence_before_sync();
-    __syncthreads();
-    if (threadIdx.x < 32) tmem_dealloc(tm, bq_tmem::NCOLS);
+    cp_async_wait_all();
+    kernel_teardown(tm, bq_tmem::NCOLS);
 }
 
-// ------------------------------------------------------------------------------------------
-// dk/dv walk (chunks in reverse, suffix state G)
-// ------------------------------------------------------------------------------------------
 namespace bkv_smem {
-constexpr uint32_t PHQ = 0;              // q rows + W at load; Phi_Q'; dP~ + W at the end
+constexpr uint32_t PHQ = 0;                // q rows (tile 0) + W (tile 1) at load; Phi_Q'; dP~ + W at the end
 constexpr uint32_t XQ = PHQ;
-constexpr uint32_t WHI0 = PHQ + 2 * TILE;
-constexpr uint32_t WLO0 = WHI0 + 8192;
 constexpr uint32_t DP = PHQ;
-constexpr uint32_t WHI1 = PHQ + TILE;
-constexpr uint32_t WLO1 = WHI1 + 8192;
-constexpr uint32_t PHK = PHQ + 4 * TILE; // k rows at load; Phi_K; then masked S'^T and P'
+constexpr uint32_t WHI = PHQ + TILE;
+constexpr uint32_t WLO = WHI + 8192;
+constexpr uint32_t PHK = PHQ + 4 * TILE;   // k rows at load; Phi_K; then masked S'^T and P'
 constexpr uint32_t XK = PHK;
-constexpr uint32_t STB = PHK;            // tiles 0-1
-constexpr uint32_t PPB = PHK + 2 * TILE; // tiles 2-3
-constexpr uint32_t V = PHK + 4 * TILE;
-constexpr uint32_t ONES = V + TILE;
-constexpr uint32_t DO = ONES + 4096;     // dO rows [128][64]
-constexpr uint32_t DC32 = DO + TILE;     // c in column 0, [128][16] SW32
-constexpr uint32_t GS128 = DC32 + 4096;
-constexpr uint32_t GS32 = GS128 + 2 * TILE;
-constexpr uint32_t ROWC = GS32 + 8192;
+constexpr uint32_t STB = PHK;              // tiles 0-1
+constexpr uint32_t PPB = PHK + 2 * TILE;   // tiles 2-3
+constexpr uint32_t VA = PHK + 4 * TILE;    // [V | 1] [128][80]
+constexpr uint32_t DOC = VA + 5 * VA128;   // [dO | c] [128][80]
+constexpr uint32_t GS = DOC + 5 * VA128;   // staged G [256][80]
+constexpr uint32_t ROWC = GS + 5 * VA256;
 constexpr uint32_t ROWINV = ROWC + 512;
-constexpr uint32_t XCH = ROWINV + 512;
-constexpr uint32_t BAR = XCH + 1024;
+constexpr uint32_t RN = ROWINV + 512;
+constexpr uint32_t XCH = RN + 1024;
+constexpr uint32_t BAR = XCH + 2048;
 constexpr uint32_t TOTAL = BAR + 64;
 }  // namespace bkv_smem
 namespace bkv_tmem {
@@ -1161,158 +1106,134 @@ constexpr uint32_t DVT = 416;   // dV [128][64]
 constexpr uint32_t NCOLS = 512;
 }  // namespace bkv_tmem
 
+// ------------------------------------------------------------------------------------------
+// dk/dv walk (chunks in reverse, suffix state G)
+// ------------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(NTH, 1) tc_bwd_kv_walk(BwdArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = aligned_base(smem_raw);
     using namespace bkv_smem;
     Ctl *ctl = reinterpret_cast<Ctl *>(sm + BAR);
-    float *xch = reinterpret_cast<float *>(sm + XCH);
+    float *xch = reinterpret_cast<float *>(sm + XCH), *rn = reinterpret_cast<float *>(sm + RN);
     float *rowc = reinterpret_cast<float *>(sm + ROWC), *rowinv = reinterpret_cast<float *>(sm + ROWINV);
     const int seg = blockIdx.x, bh = blockIdx.y;
-    const int r = threadIdx.x & 127, h = threadIdx.x >> 7;
+    const int r = threadIdx.x & 127, qd = threadIdx.x >> 7;
     const uint32_t sb = smem_u32(sm);
     const bool causal = a.causal != 0;
-    if (threadIdx.x == 0) {
-        mbar_init(&ctl->bar, 1);
-        ctl->abort = 0;
-    }
-    if (threadIdx.x < 32) tmem_alloc(&ctl->tmem, bkv_tmem::NCOLS);
-    fence_before_sync();
-    __syncthreads();
-    fence_after_sync();
-    const uint32_t tm = ctl->tmem;
+    const uint32_t tm = kernel_setup(ctl, bkv_tmem::NCOLS, a.W, sm + WHI, sm + WLO);
     {
-        float hv[80];
-        load_start_row(a.state + (int64_t)bh * a.nseg * MF * DS + seg * a.state_seg_stride, h, r, tm,
-                       bkv_tmem::GTOP, bkv_tmem::GBOT, hv);
-        stage_state_row(hv, 128 * h + r, sm + GS128, sm + GS32);
+        float hv[40];
+        load_state40(a.state + (int64_t)bh * a.nseg * MF * DS + seg * a.state_seg_stride, 128 * (qd & 1) + r, qd,
+                     tm, bkv_tmem::GTOP, bkv_tmem::GBOT, hv);
+        stage40(hv, 128 * (qd & 1) + r, qd, sm + GS);
     }
     int64_t t0, t1;
-    bseg_bounds(a, seg, t0, t1);
+    seg_bounds(a.seg_len, a.N, seg, t0, t1);
     const int64_t base = (int64_t)bh * a.N;
     const int64_t nchunks = (t1 - t0 + T - 1) / T;
     uint32_t phase = 0;
     bool ok = true;
+    auto issue_kv_do = [&](int64_t c) {  // k, v, dO rows of chunk c
+        const int n = (int)(t1 - c < T ? t1 - c : T);
+        load_k128_async(sm + XK, a.k + (base + c) * DH, n);
+        load_va_async(sm + VA, a.v + (base + c) * DH, n);
+        if (causal) load_va_async(sm + DOC, a.dout + (base + c) * DH, n);
+        cp_async_commit();
+        if (c - T >= t0)
+            prefetch_chunk(base + c - T, T, a.k, a.v, causal ? a.q : nullptr, causal ? a.dout : nullptr,
+                           causal ? a.o : nullptr, causal ? a.den : nullptr);
+    };
+    auto issue_q = [&](int64_t c) {
+        if (causal) {
+            load_k128_async(sm + XQ, a.q + (base + c) * DH, (int)(t1 - c < T ? t1 - c : T));
+            cp_async_commit();
+        }
+    };
+    if (nchunks > 0) {
+        issue_kv_do(t0 + (nchunks - 1) * T);
+        issue_q(t0 + (nchunks - 1) * T);
+    }
     for (int64_t ci = nchunks - 1; ci >= 0 && ok; --ci) {
         const int64_t c0 = t0 + ci * T;
         const int nv = (int)(t1 - c0 < T ? t1 - c0 : T);
         const bool valid = r < nv;
-        load_tile_async<NTH>(sm + XK, a.k + (base + c0) * DH, nv);
-        load_tile_async<NTH>(sm + V, a.v + (base + c0) * DH, nv);
-        if (causal) {
-            load_tile_async<NTH>(sm + XQ, a.q + (base + c0) * DH, nv);
-            load_tile_async<NTH>(sm + DO, a.dout + (base + c0) * DH, nv);
-        }
-        cp_async_commit();
-        load_w_split(a.W, sm + WHI0, sm + WLO0);
-        write_ones(sm + ONES, nv);
         cp_async_wait_all();
         __syncthreads();
-        if (causal) row_scalars(sm + DO, a.o + (base + c0) * DH, a.den + base + c0, nv, rowc, rowinv, sm + DC32);
+        if (qd == 0) rn[128 + r] = row_norm(sm + XK, r);
+        if (causal && qd == 1) rn[r] = row_norm(sm + XQ, r);
+        if (causal && qd == 2)
+            row_scalars(r, sm + DOC, a.o + (base + c0) * DH, a.den + base + c0, nv, rowc, rowinv, sm + DOC);
+        if (qd == 3) write_col64(sm + VA, r, valid ? 1.f : 0.f);
         publish_smem();
         if (threadIdx.x == 0) {
             fence_after_sync();
-            issue_proj(tm + bkv_tmem::PROJ + 64, sb + XK, sb + WHI0, sb + WLO0);
-            if (causal) issue_proj(tm + bkv_tmem::PROJ, sb + XQ, sb + WHI0, sb + WLO0);
+            issue_proj(tm + bkv_tmem::PROJ + 64, sb + XK, sb + WHI, sb + WLO);
+            if (causal) issue_proj(tm + bkv_tmem::PROJ, sb + XQ, sb + WHI, sb + WLO);
             mma_commit(&ctl->bar);
         }
-        const float raw_k = sqrtf(row_sqnorm(sm + XK, r));
-        const float inv_k = 1.f / fmaxf(raw_k, kNormEps);
-        const float inv_q = causal ? 1.f / fmaxf(sqrtf(row_sqnorm(sm + XQ, r)), kNormEps) : 0.f;
-        const float invden_r = causal ? rowinv[r] : 0.f;
         if (!(ok = wait_mma(ctl, phase))) break;
-        float u[32], t[32];
-        proj_keep(tm, bkv_tmem::PROJ + 64, h, inv_k, a.beta, u, t);
-        write_features(t, r, h, valid ? 1.f : 0.f, sm + PHK);
+        const float raw_k = rn[128 + r];
+        float u[16], t[16];
+        proj_tanh(tm, bkv_tmem::PROJ + 64, qd, 1.f / fmaxf(raw_k, kNormEps), a.beta, u, t);
+        write_features(t, r, qd, valid ? 1.f : 0.f, sm + PHK);
         if (causal) {  // Phi_Q' = Phi_Q / den
-            float uq[32], tq[32];
-            proj_keep(tm, bkv_tmem::PROJ, h, inv_q, a.beta, uq, tq);
-            write_features(tq, r, h, invden_r, sm + PHQ);
+            float uq[16], tq[16];
+            proj_tanh(tm, bkv_tmem::PROJ, qd, 1.f / fmaxf(rn[r], kNormEps), a.beta, uq, tq);
+            write_features(tq, r, qd, rowinv[r], sm + PHQ);
         }
         publish_smem();
         if (threadIdx.x == 0) {
             fence_after_sync();
             // dV = Phi_K G_next[:, :64]
-            {
-                constexpr uint32_t id = idesc_bf16(128, 64, 0, 1);
-#pragma unroll
-                for (int kk = 0; kk < 16; ++kk)
-                    mma_bf16(tm + bkv_tmem::DVT, sdesc(sb + PHK + (kk >> 2) * TILE + (kk & 3) * 32, 16, 1024, LAYOUT_SW128),
-                             sdesc(sb + GS128 + kk * 2048, TILE, 1024, LAYOUT_SW128), id, kk > 0);
-            }
+            issue_k256_va(tm + bkv_tmem::DVT, sb + PHK, sb + GS, idesc_bf16(128, 64, 0, 1), false);
             if (causal) {
-                // S'^T = Phi_K Phi_Q'^T ; V dO^T
-                constexpr uint32_t id = idesc_bf16(128, 128, 0, 0);
-#pragma unroll
-                for (int kk = 0; kk < 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * TILE + (kk & 3) * 32;
-                    mma_bf16(tm + bkv_tmem::ST, sdesc(sb + PHK + off, 16, 1024, LAYOUT_SW128),
-                             sdesc(sb + PHQ + off, 16, 1024, LAYOUT_SW128), id, kk > 0);
-                }
-                issue_k64(tm + bkv_tmem::PP, sb + V, sb + DO, id, false);
+                issue_k256_kk(tm + bkv_tmem::ST, sb + PHK, sb + PHQ, idesc_bf16(128, 128, 0, 0), false);  // S'^T
+                issue_va_va(tm + bkv_tmem::PP, sb + VA, T, sb + DOC, T, 4, idesc_bf16(128, 128, 0, 0), false);  // V dO^T
             }
             mma_commit(&ctl->bar);
         }
         if (!(ok = wait_mma(ctl, phase))) break;
         if (causal) {
-            mask_block_to_smem(tm, bkv_tmem::ST, r, h, true, 0.f, nullptr, sm + STB);
-            mask_block_to_smem(tm, bkv_tmem::PP, r, h, true, 0.f, rowc, sm + PPB);  // v_j.dO_i + c_i, i >= j
+            mask_block(tm, bkv_tmem::ST, r, qd, true, 0.f, nullptr, sm + STB);
+            mask_block(tm, bkv_tmem::PP, r, qd, true, 0.f, rowc, sm + PPB);  // v_j.dO_i + c_i, i >= j
         }
         publish_smem();
         if (threadIdx.x == 0) {
             fence_after_sync();
             if (causal)  // dV += triu(S'^T) dO
-                issue_tt_times(tm + bkv_tmem::DVT, sb + STB, sb + DO, idesc_bf16(128, 64, 0, 1), true);
+                issue_k128_va(tm + bkv_tmem::DVT, sb + STB, 0, sb + DOC, idesc_bf16(128, 64, 0, 1), true);
             // dPhi_K = [V | 1] G_next^T (+ triu(P') Phi_Q')
-            issue_k80(tm + bkv_tmem::DPHI, sb + V, sb + ONES, sb + GS128, sb + GS32, idesc_bf16(128, 256, 0, 0),
-                      false);
+            issue_va_va(tm + bkv_tmem::DPHI, sb + VA, T, sb + GS, 256, 5, idesc_bf16(128, 256, 0, 0), false);
             if (causal) {
-                issue_tt_times(tm + bkv_tmem::DPHI, sb + PPB, sb + PHQ, idesc_bf16(128, 256, 0, 1), true);
-                issue_state_update(tm, bkv_tmem::GTOP, bkv_tmem::GBOT, sb + PHQ, sb + DO, sb + DC32);
+                issue_k128_k128mn(tm + bkv_tmem::DPHI, sb + PPB, sb + PHQ, idesc_bf16(128, 256, 0, 1), true);
+                issue_state_update(tm, bkv_tmem::GTOP, bkv_tmem::GBOT, sb + PHQ, sb + DOC);
             }
             mma_commit(&ctl->bar);
         }
         if (!(ok = wait_mma(ctl, phase))) break;
-        {  // dv, columns 32h .. 32h+31 of row r (TMEM loads are warp-collective: every lane
-           // loads, only valid rows store)
-            float a0[16], a1[16];
-            const uint32_t ta = tm + (lane_base() << 16) + bkv_tmem::DVT + 32u * h;
-            tmem_ld16(ta, a0);
-            tmem_ld16(ta + 16, a1);
-            tmem_wait_ld();
-            if (valid) {
-                uint4 *d4 = reinterpret_cast<uint4 *>(a.dv + (base + c0 + r) * DH + 32 * h);
-                d4[0] = make_uint4(pack_bf16x2(a0[0], a0[1]), pack_bf16x2(a0[2], a0[3]), pack_bf16x2(a0[4], a0[5]),
-                                   pack_bf16x2(a0[6], a0[7]));
-                d4[1] = make_uint4(pack_bf16x2(a0[8], a0[9]), pack_bf16x2(a0[10], a0[11]),
-                                   pack_bf16x2(a0[12], a0[13]), pack_bf16x2(a0[14], a0[15]));
-                d4[2] = make_uint4(pack_bf16x2(a1[0], a1[1]), pack_bf16x2(a1[2], a1[3]), pack_bf16x2(a1[4], a1[5]),
-                                   pack_bf16x2(a1[6], a1[7]));
-                d4[3] = make_uint4(pack_bf16x2(a1[8], a1[9]), pack_bf16x2(a1[10], a1[11]),
-                                   pack_bf16x2(a1[12], a1[13]), pack_bf16x2(a1[14], a1[15]));
-            }
-        }
-        features_vjp_half(tm, bkv_tmem::DPHI, r, h, a.beta, valid, u, t, nullptr, 0.f, 1.f, sm + DP);
-        load_w_split(a.W, sm + WHI1, sm + WLO1);
+        if (ci > 0) issue_kv_do(c0 - T);  // Phi_K / masks, V~ and [dO | c] are free now
+        store_row16(tm, bkv_tmem::DVT, qd, valid, 1.f, a.dv + (base + c0 + r) * DH);
+        features_vjp(tm, bkv_tmem::DPHI, r, qd, a.beta, valid, u, t, nullptr, 0.f, 1.f, sm + DP);
+        load_w_split(a.W, sm + WHI, sm + WLO);
         publish_smem();
         if (threadIdx.x == 0) {
             fence_after_sync();
-            issue_dxhat(tm + bkv_tmem::DX, sb + DP, sb + WHI1, sb + WLO1);
+            issue_dxhat(tm + bkv_tmem::DX, sb + DP, sb + WHI, sb + WLO);
             mma_commit(&ctl->bar);
         }
         if (!(ok = wait_mma(ctl, phase))) break;
-        write_dx(tm, bkv_tmem::DX, r, h, valid, raw_k, a.k + (base + c0 + r) * DH, a.dk + (base + c0 + r) * DH, xch);
+        if (ci > 0) issue_q(c0 - T);
+        write_dx(tm, bkv_tmem::DX, r, qd, valid, raw_k, a.k + (base + c0 + r) * DH, a.dk + (base + c0 + r) * DH, xch);
         if (causal) {
-            float hv[80];
-            read_state_row(tm, h ? bkv_tmem::GBOT : bkv_tmem::GTOP, hv);
-            stage_state_row(hv, 128 * h + r, sm + GS128, sm + GS32);
+            float hv[40];
+            read_state40(tm, bkv_tmem::GTOP, bkv_tmem::GBOT, qd, hv);
+            stage40(hv, 128 * (qd & 1) + r, qd, sm + GS);
         }
         publish_smem();
     }
-    fence_before_sync();
-    __syncthreads();
-    if (threadIdx.x < 32) tmem_dealloc(tm, bkv_tmem::NCOLS);
+    cp_async_wait_all();
+    kernel_teardown(tm, bkv_tmem::NCOLS);
 }
 
 // ---- host side ---------------------------------------------------------------------------
