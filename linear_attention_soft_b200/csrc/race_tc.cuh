@@ -219,19 +219,18 @@ __device__ __forceinline__ float row_norm(const uint8_t *tile, int r)
     return sqrtf(s);
 }
 
-// Per-row scalars of a chunk from the dO rows of a value tile and o from global:
+// Per-row scalars of a chunk from the dO rows (value tile) and o rows (K128 tile):
 // rowc[r] = c_r = -(dO_r . o_r), rowinv[r] = 1/den_r (0 beyond nvalid); optionally c_r
 // into column 64 of the value tile.  One thread per row.
-__device__ __forceinline__ void row_scalars(int r, const uint8_t *doc, const __nv_bfloat16 *o, const float *den,
+__device__ __forceinline__ void row_scalars(int r, const uint8_t *doc, const uint8_t *o_tile, const float *den,
                                             int nvalid, float *rowc, float *rowinv, uint8_t *doc_col64)
 {
     float c = 0.f, inv = 0.f;
     if (r < nvalid) {
-        const uint32_t a = smem_u32(doc);
-        const uint4 *o4 = reinterpret_cast<const uint4 *>(o + (int64_t)r * DH);
+        const uint32_t a = smem_u32(doc), ao = smem_u32(o_tile);
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) {
-            const uint4 g = ld_shared_v4(a + va_off(r, ch, T)), ov = o4[ch];
+            const uint4 g = ld_shared_v4(a + va_off(r, ch, T)), ov = ld_shared_v4(ao + sw128_off(r, ch));
             const uint32_t gw[4] = {g.x, g.y, g.z, g.w}, ow[4] = {ov.x, ov.y, ov.z, ov.w};
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
@@ -328,22 +327,30 @@ __device__ __forceinline__ void features_vjp(uint32_t tm, uint32_t col0, int r, 
 #pragma unroll
             for (int c = 0; c < 16; ++c) gg[c] = fmaf(add_scale, av[c], gg[c]) * mul;
         }
+        // Under phi the sign c_p has mean t_p = tanh(beta u_p), so
+        // du_p = beta sum_c c_cp phi_c (g_c - phi.g) = beta (2 A_p - (1 + t_p) phi.g),
+        // A_p = sum over the corners with bit p set of phi_c g_c.
         float f[16];
         corner_weights(t, l, 1.f, f);
-        float dot = 0.f;
+        float fg[16];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) dot = fmaf(f[c], gg[c], dot);
-        float du[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int c = 0; c < 16; ++c) fg[c] = f[c] * gg[c];
+        float s1[8], s2[4];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-            const float dz = f[c] * (gg[c] - dot);
+        for (int c = 0; c < 8; ++c) s1[c] = fg[2 * c] + fg[2 * c + 1];     // pairs over bit 0
 #pragma unroll
-            for (int p = 0; p < 4; ++p) du[p] += ((c >> p) & 1) ? dz : -dz;
-        }
+        for (int c = 0; c < 4; ++c) s2[c] = s1[2 * c] + s1[2 * c + 1];     // quads over bits 0-1
+        const float dot = (s2[0] + s2[1]) + (s2[2] + s2[3]);
+        float ap[4];
+        ap[0] = ((fg[1] + fg[3]) + (fg[5] + fg[7])) + ((fg[9] + fg[11]) + (fg[13] + fg[15]));
+        ap[1] = ((s1[1] + s1[3]) + (s1[5] + s1[7]));
+        ap[2] = s2[1] + s2[3];
+        ap[3] = s2[2] + s2[3];
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
             const float uu = u[4 * l + p];
-            dp[4 * l + p] = valid ? beta * du[p] * (1.f - uu * uu) : 0.f;
+            const float du = beta * (2.f * ap[p] - (1.f + t[4 * l + p]) * dot);
+            dp[4 * l + p] = valid ? du * (1.f - uu * uu) : 0.f;
         }
     }
     const uint32_t b = smem_u32(dp_tile);
@@ -482,19 +489,27 @@ __device__ __forceinline__ void store_state40(const float (&hv)[40], float *dst_
 }
 
 // dx = (dX^ - x^ (x^ . dX^)) / max(|x|, eps) for row r, columns 16qd .. 16qd+15; dX^ from
-// TMEM column col0; x re-read from global; the four quarters exchange partial dots.
+// TMEM column col0; x from a K128 tile in shared memory if xtile, else from global xrow;
+// the four quarters exchange partial dots.
 __device__ __forceinline__ void write_dx(uint32_t tm, uint32_t col0, int r, int qd, bool valid, float rawn,
-                                         const __nv_bfloat16 *xrow, __nv_bfloat16 *dst, float *xch)
+                                         const uint8_t *xtile, const __nv_bfloat16 *xrow, __nv_bfloat16 *dst,
+                                         float *xch)
 {
     uint32_t w[16];
     tmem_ld16_nowait(tlane(tm, col0 + 16u * qd), w);
     float x[16];
     if (valid) {
-        const uint4 *x4 = reinterpret_cast<const uint4 *>(xrow + 16 * qd);
+        uint4 v4[2];
+        if (xtile) {
+            v4[0] = ld_shared_v4(smem_u32(xtile) + sw128_off(r, 2 * qd));
+            v4[1] = ld_shared_v4(smem_u32(xtile) + sw128_off(r, 2 * qd + 1));
+        } else {
+            v4[0] = reinterpret_cast<const uint4 *>(xrow + 16 * qd)[0];
+            v4[1] = reinterpret_cast<const uint4 *>(xrow + 16 * qd)[1];
+        }
 #pragma unroll
         for (int ch = 0; ch < 2; ++ch) {
-            const uint4 v4 = x4[ch];
-            const uint32_t ws[4] = {v4.x, v4.y, v4.z, v4.w};
+            const uint32_t ws[4] = {v4[ch].x, v4[ch].y, v4[ch].z, v4[ch].w};
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 x[8 * ch + 2 * i] = bf16_lo(ws[i]);
@@ -645,7 +660,9 @@ constexpr uint32_t WLO = WHI + 8192;
 constexpr uint32_t RN = WLO + 8192;         // row norms [128]
 constexpr uint32_t ROWC = RN + 512;
 constexpr uint32_t ROWINV = ROWC + 512;
-constexpr uint32_t BAR = ROWINV + 512;
+constexpr uint32_t O0 = ROWINV + 512 + 512;  // o rows (backward aggregate), 1024-aligned
+constexpr uint32_t O1 = O0 + TILE;
+constexpr uint32_t BAR = O1 + TILE;
 constexpr uint32_t TOTAL = BAR + 64;
 }  // namespace agg_smem
 namespace agg_tmem {
@@ -731,6 +748,7 @@ __global__ void __launch_bounds__(NTH, 1) tc_agg(BwdArgs a)
     if (t0 < t1) {
         load_k128_async(sm + X0, xsrc + (base + t0) * DH, (int)(t1 - t0 < T ? t1 - t0 : T));
         load_va_async(sm + VA0, vsrc + (base + t0) * DH, (int)(t1 - t0 < T ? t1 - t0 : T));
+        if (MODE == 1) load_k128_async(sm + O0, a.o + (base + t0) * DH, (int)(t1 - t0 < T ? t1 - t0 : T));
         cp_async_commit();
     }
     int buf = 0;
@@ -743,6 +761,7 @@ __global__ void __launch_bounds__(NTH, 1) tc_agg(BwdArgs a)
             const int nn = (int)(t1 - c0 - T < T ? t1 - c0 - T : T);
             load_k128_async(sm + (buf ? X0 : X1), xsrc + (base + c0 + T) * DH, nn);
             load_va_async(sm + (buf ? VA0 : VA1), vsrc + (base + c0 + T) * DH, nn);
+            if (MODE == 1) load_k128_async(sm + (buf ? O0 : O1), a.o + (base + c0 + T) * DH, nn);
             cp_async_commit();
             prefetch_chunk(base + c0 + 2 * T, (int)(t1 - c0 - 2 * T < T ? t1 - c0 - 2 * T : T), xsrc, vsrc,
                            MODE ? a.o : nullptr, nullptr, nullptr, MODE ? a.den : nullptr);
@@ -750,7 +769,7 @@ __global__ void __launch_bounds__(NTH, 1) tc_agg(BwdArgs a)
         if (qd == 0) rn[r] = row_norm(x, r);
         if (MODE == 0 && qd == 1) write_col64(va, r, r < nv ? 1.f : 0.f);
         if (MODE == 1 && qd == 2)
-            row_scalars(r, va, a.o + (base + c0) * DH, a.den + base + c0, nv, rowc, rowinv, va);
+            row_scalars(r, va, sm + (buf ? O1 : O0), a.den + base + c0, nv, rowc, rowinv, va);
         publish_smem();
         if (threadIdx.x == 0) {
             fence_after_sync();
@@ -923,8 +942,9 @@ __device__ __forceinline__ void issue_dxhat(uint32_t d, uint32_t dp, uint32_t wh
 }
 
 namespace bq_smem {
-constexpr uint32_t RA = 0;                 // k rows at load; Phi_K [128][256] after the features
+constexpr uint32_t RA = 0;                 // k rows + o rows at load; Phi_K [128][256] after the features
 constexpr uint32_t XK = RA;
+constexpr uint32_t OT = RA + TILE;
 constexpr uint32_t PHK = RA;
 constexpr uint32_t RB = 4 * TILE;          // q rows + W at load; masked P''; dP~ + W at the end
 constexpr uint32_t XQ = RB;
@@ -941,12 +961,13 @@ constexpr uint32_t ROWC = HDEN + 1024;
 constexpr uint32_t ROWINV = ROWC + 512;
 constexpr uint32_t RN = ROWINV + 512;
 constexpr uint32_t XCH = RN + 1024;
-constexpr uint32_t BAR = XCH + 2048;
+constexpr uint32_t XQ2 = XCH + 2048 + 1024;  // q rows kept for dq (1024-aligned)
+constexpr uint32_t BAR = XQ2 + TILE;
 constexpr uint32_t TOTAL = BAR + 64;
 }  // namespace bq_smem
 namespace bq_tmem {
 constexpr uint32_t PROJ = 0;   // q 0..63, k 64..127
-constexpr uint32_t P = 0;      // [128][128]
+constexpr uint32_t P = 128;    // [128][128]
 constexpr uint32_t DPHI = 0;   // [128][256]
 constexpr uint32_t DX = 0;     // [128][64]
 constexpr uint32_t HTOP = 256;
@@ -982,9 +1003,10 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_q_walk(BwdArgs a)
     const int64_t base = (int64_t)bh * a.N;
     uint32_t phase = 0;
     bool ok = true;
-    auto issue_kv_do = [&](int64_t c) {  // k, v, dO rows of chunk c
+    auto issue_kv_do = [&](int64_t c) {  // k, v, dO, o rows of chunk c
         const int n = (int)(t1 - c < T ? t1 - c : T);
         load_va_async(sm + DOV, a.dout + (base + c) * DH, n);
+        load_k128_async(sm + OT, a.o + (base + c) * DH, n);
         if (causal) {
             load_k128_async(sm + XK, a.k + (base + c) * DH, n);
             load_va_async(sm + VA, a.v + (base + c) * DH, n);
@@ -993,13 +1015,18 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_q_walk(BwdArgs a)
         prefetch_chunk(base + c + T, (int)(t1 - c - T < T ? t1 - c - T : T), a.q, a.dout, a.o,
                        causal ? a.k : nullptr, causal ? a.v : nullptr, a.den);
     };
-    auto issue_q = [&](int64_t c) {
+    auto issue_q = [&](int64_t c) {  // q rows for the projection
         load_k128_async(sm + XQ, a.q + (base + c) * DH, (int)(t1 - c < T ? t1 - c : T));
+        cp_async_commit();
+    };
+    auto issue_q2 = [&](int64_t c) {  // q rows kept for dq
+        load_k128_async(sm + XQ2, a.q + (base + c) * DH, (int)(t1 - c < T ? t1 - c : T));
         cp_async_commit();
     };
     if (t0 < t1) {
         issue_kv_do(t0);
         issue_q(t0);
+        issue_q2(t0);
     }
     for (int64_t c0 = t0; c0 < t1 && ok; c0 += T) {
         const int nv = (int)(t1 - c0 < T ? t1 - c0 : T);
@@ -1008,13 +1035,17 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_q_walk(BwdArgs a)
         __syncthreads();
         if (qd == 0) rn[r] = row_norm(sm + XQ, r);
         if (causal && qd == 1) rn[128 + r] = row_norm(sm + XK, r);
-        if (qd == 2) row_scalars(r, sm + DOV, a.o + (base + c0) * DH, a.den + base + c0, nv, rowc, rowinv, nullptr);
+        if (qd == 2) row_scalars(r, sm + DOV, sm + OT, a.den + base + c0, nv, rowc, rowinv, nullptr);
         if (causal && qd == 3) write_col64(sm + VA, r, valid ? 1.f : 0.f);
         publish_smem();
         if (threadIdx.x == 0) {
             fence_after_sync();
             issue_proj(tm + bq_tmem::PROJ, sb + XQ, sb + WHI, sb + WLO);
-            if (causal) issue_proj(tm + bq_tmem::PROJ + 64, sb + XK, sb + WHI, sb + WLO);
+            if (causal) {
+                issue_proj(tm + bq_tmem::PROJ + 64, sb + XK, sb + WHI, sb + WLO);
+                // P'' = dO V^T (needs no features)
+                issue_va_va(tm + bq_tmem::P, sb + DOV, T, sb + VA, T, 4, idesc_bf16(128, 128, 0, 0), false);
+            }
             mma_commit(&ctl->bar);
         }
         if (!(ok = wait_mma(ctl, phase))) break;
@@ -1026,18 +1057,9 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_q_walk(BwdArgs a)
             float uk[16], tk[16];
             proj_tanh(tm, bq_tmem::PROJ + 64, qd, 1.f / fmaxf(rn[128 + r], kNormEps), a.beta, uk, tk);
             write_features(tk, r, qd, valid ? 1.f : 0.f, sm + PHK);
+            mask_block(tm, bq_tmem::P, r, qd, false, c_r, nullptr, sm + PB);  // v_j.dO_i + c_i, j <= i
         }
         publish_smem();
-        if (causal) {
-            if (threadIdx.x == 0) {  // P'' = dO V^T
-                fence_after_sync();
-                issue_va_va(tm + bq_tmem::P, sb + DOV, T, sb + VA, T, 4, idesc_bf16(128, 128, 0, 0), false);
-                mma_commit(&ctl->bar);
-            }
-            if (!(ok = wait_mma(ctl, phase))) break;
-            mask_block(tm, bq_tmem::P, r, qd, false, c_r, nullptr, sm + PB);  // v_j.dO_i + c_i, j <= i
-            publish_smem();
-        }
         if (threadIdx.x == 0) {
             fence_after_sync();
             // D = dO H_prev[:, :64]^T (+ tril(P'') Phi_K)
@@ -1062,7 +1084,9 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_q_walk(BwdArgs a)
         }
         if (!(ok = wait_mma(ctl, phase))) break;
         if (c0 + T < t1) issue_q(c0 + T);  // dP~ is consumed; W stays for the next projection
-        write_dx(tm, bq_tmem::DX, r, qd, valid, raw_q, a.q + (base + c0 + r) * DH, a.dq + (base + c0 + r) * DH, xch);
+        write_dx(tm, bq_tmem::DX, r, qd, valid, raw_q, sm + XQ2, nullptr, a.dq + (base + c0 + r) * DH, xch);
+        __syncthreads();  // every quarter has read its q rows
+        if (c0 + T < t1) issue_q2(c0 + T);
         if (causal) {
             float hv[40];
             read_state40(tm, bq_tmem::HTOP, bq_tmem::HBOT, qd, hv);
@@ -1080,6 +1104,7 @@ constexpr uint32_t XQ = PHQ;
 constexpr uint32_t DP = PHQ;
 constexpr uint32_t WHI = PHQ + TILE;
 constexpr uint32_t WLO = WHI + 8192;
+constexpr uint32_t OT = PHQ + 2 * TILE;    // o rows at load
 constexpr uint32_t PHK = PHQ + 4 * TILE;   // k rows at load; Phi_K; then masked S'^T and P'
 constexpr uint32_t XK = PHK;
 constexpr uint32_t STB = PHK;              // tiles 0-1
@@ -1138,7 +1163,10 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_kv_walk(BwdArgs a)
         const int n = (int)(t1 - c < T ? t1 - c : T);
         load_k128_async(sm + XK, a.k + (base + c) * DH, n);
         load_va_async(sm + VA, a.v + (base + c) * DH, n);
-        if (causal) load_va_async(sm + DOC, a.dout + (base + c) * DH, n);
+        if (causal) {
+            load_va_async(sm + DOC, a.dout + (base + c) * DH, n);
+            load_k128_async(sm + OT, a.o + (base + c) * DH, n);
+        }
         cp_async_commit();
         if (c - T >= t0)
             prefetch_chunk(base + c - T, T, a.k, a.v, causal ? a.q : nullptr, causal ? a.dout : nullptr,
@@ -1163,13 +1191,17 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_kv_walk(BwdArgs a)
         if (qd == 0) rn[128 + r] = row_norm(sm + XK, r);
         if (causal && qd == 1) rn[r] = row_norm(sm + XQ, r);
         if (causal && qd == 2)
-            row_scalars(r, sm + DOC, a.o + (base + c0) * DH, a.den + base + c0, nv, rowc, rowinv, sm + DOC);
+            row_scalars(r, sm + DOC, sm + OT, a.den + base + c0, nv, rowc, rowinv, sm + DOC);
         if (qd == 3) write_col64(sm + VA, r, valid ? 1.f : 0.f);
         publish_smem();
         if (threadIdx.x == 0) {
             fence_after_sync();
             issue_proj(tm + bkv_tmem::PROJ + 64, sb + XK, sb + WHI, sb + WLO);
-            if (causal) issue_proj(tm + bkv_tmem::PROJ, sb + XQ, sb + WHI, sb + WLO);
+            if (causal) {
+                issue_proj(tm + bkv_tmem::PROJ, sb + XQ, sb + WHI, sb + WLO);
+                // V dO^T (needs no features)
+                issue_va_va(tm + bkv_tmem::PP, sb + VA, T, sb + DOC, T, 4, idesc_bf16(128, 128, 0, 0), false);
+            }
             mma_commit(&ctl->bar);
         }
         if (!(ok = wait_mma(ctl, phase))) break;
@@ -1177,22 +1209,22 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_kv_walk(BwdArgs a)
         float u[16], t[16];
         proj_tanh(tm, bkv_tmem::PROJ + 64, qd, 1.f / fmaxf(raw_k, kNormEps), a.beta, u, t);
         write_features(t, r, qd, valid ? 1.f : 0.f, sm + PHK);
-        if (causal) {  // Phi_Q' = Phi_Q / den
-            float uq[16], tq[16];
-            proj_tanh(tm, bkv_tmem::PROJ, qd, 1.f / fmaxf(rn[r], kNormEps), a.beta, uq, tq);
-            write_features(tq, r, qd, rowinv[r], sm + PHQ);
-        }
+        float uq[16], tq[16];
+        if (causal) proj_tanh(tm, bkv_tmem::PROJ, qd, 1.f / fmaxf(rn[r], kNormEps), a.beta, uq, tq);
         publish_smem();
-        if (threadIdx.x == 0) {
+        if (threadIdx.x == 0) {  // dV = Phi_K G_next[:, :64], while Phi_Q' is formed
             fence_after_sync();
-            // dV = Phi_K G_next[:, :64]
             issue_k256_va(tm + bkv_tmem::DVT, sb + PHK, sb + GS, idesc_bf16(128, 64, 0, 1), false);
-            if (causal) {
-                issue_k256_kk(tm + bkv_tmem::ST, sb + PHK, sb + PHQ, idesc_bf16(128, 128, 0, 0), false);  // S'^T
-                issue_va_va(tm + bkv_tmem::PP, sb + VA, T, sb + DOC, T, 4, idesc_bf16(128, 128, 0, 0), false);  // V dO^T
-            }
-            mma_commit(&ctl->bar);
         }
+        if (causal) {
+            write_features(tq, r, qd, rowinv[r], sm + PHQ);  // Phi_Q' = Phi_Q / den
+            publish_smem();
+            if (threadIdx.x == 0) {
+                fence_after_sync();
+                issue_k256_kk(tm + bkv_tmem::ST, sb + PHK, sb + PHQ, idesc_bf16(128, 128, 0, 0), false);  // S'^T
+            }
+        }
+        if (threadIdx.x == 0) mma_commit(&ctl->bar);
         if (!(ok = wait_mma(ctl, phase))) break;
         if (causal) {
             mask_block(tm, bkv_tmem::ST, r, qd, true, 0.f, nullptr, sm + STB);
@@ -1224,7 +1256,8 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_kv_walk(BwdArgs a)
         }
         if (!(ok = wait_mma(ctl, phase))) break;
         if (ci > 0) issue_q(c0 - T);
-        write_dx(tm, bkv_tmem::DX, r, qd, valid, raw_k, a.k + (base + c0 + r) * DH, a.dk + (base + c0 + r) * DH, xch);
+        write_dx(tm, bkv_tmem::DX, r, qd, valid, raw_k, nullptr, a.k + (base + c0 + r) * DH, a.dk + (base + c0 + r) * DH,
+                 xch);
         if (causal) {
             float hv[40];
             read_state40(tm, bkv_tmem::GTOP, bkv_tmem::GBOT, qd, hv);
