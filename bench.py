@@ -74,6 +74,30 @@ def kernel_work(name: str, w: race_inputs.Workload):
     return None
 
 
+# DRAM bytes per token (read + write) per kernel from the ncu capture summarised in
+# profiles/tc_kernels_n1m_ncu_full.md (N = 2^20; traffic grows in proportion to the tokens),
+# valid only for the kernel sources it was taken on.
+NCU_TRAFFIC = {
+    "src_sha1": {"race_tc.cuh": "853b03348070471dae58f8da60afe06a175ac3f1",
+                 "race_tc_util.cuh": "ec7c601f16c5892d0fd431308161cd00e13fa94c"},
+    "bytes_per_token": {"tc_agg_kv": 273.0, "tc_fwd_walk": 514.0, "tc_bwd_q_walk": 780.0,
+                        "tc_agg_qdy": 404.0, "tc_bwd_kv_walk": 894.0},
+}
+
+
+def measured_traffic(name: str, tokens: int):
+    """DRAM bytes per launch of kernel `name` from the recorded ncu capture, or None when the
+    kernel sources changed since (the counters would describe another kernel)."""
+    import hashlib
+    csrc = os.path.join(ROOT, "linear_attention_soft_b200", "csrc")
+    for fn, sha in NCU_TRAFFIC["src_sha1"].items():
+        path = os.path.join(csrc, fn)
+        if not os.path.exists(path) or hashlib.sha1(open(path, "rb").read()).hexdigest() != sha:
+            return None
+    bpt = NCU_TRAFFIC["bytes_per_token"].get(name)
+    return None if bpt is None else bpt * tokens
+
+
 def is_tensor_core_kernel(name: str) -> bool:
     return name.startswith("tc_")
 
@@ -187,6 +211,30 @@ def run_reference(args, w):
     print(json.dumps(line), flush=True)
 
 
+# ---- multi-rank bookkeeping (weak scaling: one independent sequence per rank) ----------
+def rank_workload(w: race_inputs.Workload, rank: int) -> race_inputs.Workload:
+    """The workload rank `rank` runs: same shape, its own seed (independent sequences)."""
+    import dataclasses
+    return dataclasses.replace(w, seed=w.seed + 1000 * rank)
+
+
+def job_throughput(ms_local: float, tokens_local: int, world: int, device=None):
+    """(max ms over ranks, whole-job tokens/s): every rank's tokens over the slowest rank's
+    time.  Collective only when world > 1."""
+    t = torch.tensor([ms_local, float(tokens_local)], dtype=torch.float64,
+                     device=device if device is not None else "cpu")
+    if world > 1:
+        import torch.distributed as dist
+        mx = t.clone()
+        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
+        sm = t.clone()
+        dist.all_reduce(sm, op=dist.ReduceOp.SUM)
+        ms, tokens = float(mx[0]), float(sm[1])
+    else:
+        ms, tokens = float(t[0]), float(t[1])
+    return ms, tokens / (ms / 1e3)
+
+
 # ---- the CUDA library -------------------------------------------------------------------
 def run_ours(args, w):
     import linear_attention_soft_b200 as ra
@@ -202,9 +250,7 @@ def run_ours(args, w):
                                 device_id=dev)
     peaks = load_peaks()
     # each rank draws its own independent sequence (weak scaling)
-    import dataclasses
-    wr = dataclasses.replace(w, seed=w.seed + 1000 * rank)
-    inp = race_inputs.make_inputs(wr, dev)
+    inp = race_inputs.make_inputs(rank_workload(w, rank), dev)
     q, k, v, W, do = inp["q"], inp["k"], inp["v"], inp["W"], inp["do"]
     B, H, N, d = q.shape
     L, P = w.L, w.P
@@ -251,12 +297,8 @@ def run_ours(args, w):
     clk = clocks.stop()
     ms = e0.elapsed_time(e1) / args.steps
     prof = ra.race_attn_profile_read()
-    ms_t = torch.tensor([ms], device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(ms_t, op=torch.distributed.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
+    ms_max, value = job_throughput(ms, B * N, world, dev)
     tokens_all = B * N * world
-    value = tokens_all / (ms_max / 1e3)
 
     # ---- end to end through the C ABI with host buffers --------------------------------
     host = {n: t.cpu().pin_memory() for n, t in (("q", q), ("k", k), ("v", v), ("do", do))}
@@ -285,10 +327,7 @@ def run_ours(args, w):
     e1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
-    e2e_ms = torch.tensor([e0.elapsed_time(e1) / e2e_steps], device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(e2e_ms, op=torch.distributed.ReduceOp.MAX)
-    e2e_val = tokens_all / (float(e2e_ms.item()) / 1e3)
+    _, e2e_val = job_throughput(e0.elapsed_time(e1) / e2e_steps, B * N, world, dev)
 
     # ---- roofline of the dominant kernel and of the whole step ------------------------
     launches = sum(c for _, c in prof.values())
@@ -317,7 +356,7 @@ def run_ours(args, w):
                 roof = {"bound": "tensor" if is_tensor_core_kernel(name) else "alu",
                         "achieved": flops / per_launch_s / 1e12, "peak": peak_c, "unit": "TFLOP/s"}
             roof["frac"] = roof["achieved"] / roof["peak"]
-            roof["traffic"] = None
+            roof["traffic"] = measured_traffic(name, units)
             roof.update({"kernel": name, "ms_per_launch": per_launch_s * 1e3,
                          "share_of_step": share, "peak_source": peaks["source"]})
     sb, sf = step_work(w)

@@ -129,6 +129,22 @@ race_status_t race_attn_hash_indices(const void *x, const float *W, int32_t *idx
                                      race_stream_t stream);
 
 /*
+ * Device-side failure report (a robustness aid; the method has no counterpart).  Every wait
+ * of the tensor-core kernels on an MMA completion gives up after 2 s; a kernel that gave up
+ * skips the rest of its work, releases its tensor memory, returns, and sets a device error
+ * word.  race_attn_device_error waits for `stream`, writes that word to *flag (0 = no wait
+ * ever timed out, 1 = one did) and clears it.
+ */
+race_status_t race_attn_device_error(int *flag, race_stream_t stream);
+
+/*
+ * Self-test of that mechanism: launches one CTA that waits on a barrier nothing arrives on,
+ * for at most limit_ns nanoseconds (1 <= limit_ns <= 1e9), then records the timeout exactly
+ * as a stalled MMA would.  A following race_attn_device_error reports 1.
+ */
+race_status_t race_attn_selftest_wait_timeout(int64_t limit_ns, race_stream_t stream);
+
+/*
  * Forward pass that allocates nothing and takes no workspace (the method's description has
  * no counterpart to this; it is a deployment convenience).  It is for callers that cannot
  * obtain device memory on their own: code whose device memory is owned by a host

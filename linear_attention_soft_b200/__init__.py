@@ -24,6 +24,7 @@ __all__ = [
     "race_attn_forward", "race_attn_backward", "race_attn_hash_indices",
     "forward", "backward", "race_attn_profile_enable", "race_attn_profile_reset",
     "race_attn_profile_read", "race_attn_forward_noalloc", "RACE_NOALLOC_SCRATCH_BYTES",
+    "race_attn_device_error", "race_attn_selftest_wait_timeout",
 ]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -78,6 +79,10 @@ def load_library():
     lib.race_attn_hash_indices.argtypes = [_vp, _vp, _vp, _int, _int, _i64, _int, _int, _int, _int,
                                            _vp]
     lib.race_attn_hash_indices.restype = _int
+    lib.race_attn_device_error.argtypes = [ctypes.POINTER(_int), _vp]
+    lib.race_attn_device_error.restype = _int
+    lib.race_attn_selftest_wait_timeout.argtypes = [_i64, _vp]
+    lib.race_attn_selftest_wait_timeout.restype = _int
     lib.race_attn_forward_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _i64, _int,
                                               _int, _int, ctypes.c_float, _int, _int, _vp]
     lib.race_attn_forward_noalloc.restype = _int
@@ -186,6 +191,19 @@ def race_attn_forward_noalloc(q, k, v, W, out, den, tau: float, causal: bool, st
     _check(load_library().race_attn_forward_noalloc(
         _ptr(q), _ptr(k), _ptr(v), _ptr(W), _ptr(out), _ptr(den), B, H, N, d, L, P, float(tau),
         int(bool(causal)), _dtype_code(q), _stream(stream)), "race_attn_forward_noalloc")
+
+
+def race_attn_device_error(stream=None) -> int:
+    """1 if a tensor-core kernel gave up waiting on an MMA since the last call (and clear)."""
+    flag = _int()
+    _check(load_library().race_attn_device_error(ctypes.byref(flag), _stream(stream)),
+           "race_attn_device_error")
+    return flag.value
+
+
+def race_attn_selftest_wait_timeout(limit_ns: int, stream=None) -> None:
+    _check(load_library().race_attn_selftest_wait_timeout(int(limit_ns), _stream(stream)),
+           "race_attn_selftest_wait_timeout")
 
 
 def race_attn_profile_enable(on: bool) -> None:

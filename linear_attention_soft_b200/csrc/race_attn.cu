@@ -528,6 +528,26 @@ race_status_t race_attn_hash_indices(const void *x, const float *W, int32_t *idx
     return e == cudaSuccess ? RACE_OK : RACE_ERR_CUDA;
 }
 
+race_status_t race_attn_device_error(int *flag, race_stream_t stream)
+{
+    if (!flag) return RACE_ERR_INVALID_ARG;
+    int v = 0;
+    const int zero = 0;
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess ||
+        cudaMemcpyFromSymbol(&v, race::tc::g_tc_error, sizeof(int)) != cudaSuccess ||
+        cudaMemcpyToSymbol(race::tc::g_tc_error, &zero, sizeof(int)) != cudaSuccess)
+        return RACE_ERR_CUDA;
+    *flag = v;
+    return RACE_OK;
+}
+
+race_status_t race_attn_selftest_wait_timeout(int64_t limit_ns, race_stream_t stream)
+{
+    if (limit_ns < 1 || limit_ns > 1000000000) return RACE_ERR_INVALID_ARG;
+    race::tc::tc_wait_timeout_selftest<<<1, 32, 0, (cudaStream_t)stream>>>((uint64_t)limit_ns);
+    return cudaGetLastError() == cudaSuccess ? RACE_OK : RACE_ERR_CUDA;
+}
+
 void race_attn_profile_enable(int on) { g_prof_on = on != 0; }
 
 void race_attn_profile_reset(void)

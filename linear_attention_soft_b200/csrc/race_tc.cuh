@@ -1269,6 +1269,18 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_kv_walk(BwdArgs a)
     kernel_teardown(tm, bkv_tmem::NCOLS);
 }
 
+// Waits on a barrier that nothing arrives on, for at most limit_ns, and reports the timeout
+// the way the kernels above do.  One CTA of one warp.
+__global__ void tc_wait_timeout_selftest(uint64_t limit_ns)
+{
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        if (!mbar_wait(&bar, 0u, limit_ns)) atomicExch(&g_tc_error, 1);
+    }
+    __syncwarp();
+}
+
 // ---- host side ---------------------------------------------------------------------------
 
 inline bool fast_path_ok(race_dtype_t dtype, int d, int L, int P, float tau)
