@@ -62,8 +62,9 @@ const char *race_status_string(race_status_t status);
  * Device workspace, in bytes, that race_attn_forward (backward = 0) or
  * race_attn_backward (backward = 1) needs for these sizes, written to *bytes.
  * The workspace holds the per-segment bucket statistics of the chunked scan
- * (fp32, L*2^P x (d+1) per segment and head); it is scratch: its contents on entry
- * are ignored and on exit are unspecified.
+ * (fp32, L*2^P x (d+1) per segment and head; the backward needs two such buffers plus
+ * 16 KB and one fp32 per token for c_i = -(dO_i . o_i)); it is scratch: its contents on
+ * entry are ignored and on exit are unspecified.
  */
 race_status_t race_attn_workspace_size(int B, int H, int64_t N, int d, int L, int P, int causal,
                                        int backward, race_dtype_t dtype, size_t *bytes);

@@ -1,6 +1,7 @@
 // race_attn.cu -- C ABI of the RACE Attention library: argument checks, work planning and
 // kernel launches on the caller's stream.  Declarations and argument contracts are in
 // include/race_attn.h.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -71,6 +72,8 @@ using race::generic::Args;
 namespace gk = race::generic;
 
 constexpr int64_t kSegAlign = 128;     // segment lengths are multiples of this many tokens
+// so that only the last chunk of a head is ragged, where the TMA boxes read zeros past N
+static_assert(kSegAlign % race::tc::T == 0, "segments hold whole chunks");
 constexpr int64_t kMinSegTokens = 512;  // no segment shorter than this (unless N is)
 
 struct Plan {
@@ -133,6 +136,54 @@ Plan make_plan(int B, int H, int64_t N, int d, int L, int P)
 }
 
 bool aligned16(const void *ptr) { return ((uintptr_t)ptr & 15u) == 0; }
+
+// Backward workspace: key- and query-side segment states, then the W image of the tensor-core
+// path (16 KB), then c_i per token (fp32 [BH][N]).
+constexpr size_t kWImageBytes = 16384;
+size_t backward_workspace_bytes(const Plan &p)
+{
+    const size_t cbytes = ((size_t)p.BH * (size_t)p.N * sizeof(float) + 15) / 16 * 16;
+    return 2 * p.state_elems * sizeof(float) + kWImageBytes + cbytes;
+}
+
+// ---- tensor maps of the TMA loads ---------------------------------------------------------
+using EncodeTiled = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                 const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled encode_tiled()
+{
+    static const EncodeTiled fn = [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess) {
+            cudaGetLastError();
+            return (EncodeTiled) nullptr;
+        }
+        return (EncodeTiled)f;
+    }();
+    return fn;
+}
+
+// A [BH][N][64] bf16 tensor as a 3-D map (columns, rows, heads); boxes of 128 rows by
+// box_cols columns: 64 with the 128-byte swizzle (a K128 tile) or 16 with the 32-byte swizzle
+// (one value-tile atom).  Rows past N read as zero.
+cudaError_t bf16_map(CUtensorMap *m, const void *ptr, const Plan &p, bool value_atom)
+{
+    const EncodeTiled fn = encode_tiled();
+    if (!fn) return cudaErrorNotSupported;
+    const cuuint64_t dims[3] = {64, (cuuint64_t)p.N, (cuuint64_t)p.BH};
+    const cuuint64_t strides[2] = {128, (cuuint64_t)p.N * 128};
+    const cuuint32_t box[3] = {value_atom ? 16u : 64u, (cuuint32_t)race::tc::T, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          value_atom ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
 
 Args base_args(const Plan &p, const float *W, float tau)
 {
@@ -271,11 +322,16 @@ cudaError_t tc_segment_totals(const Plan &p, race::tc::BwdArgs a, int mode, floa
     });
 }
 
-race::tc::BwdArgs tc_args(const Plan &p, const void *q, const void *k, const void *v, const float *W,
-                          const void *out, const float *den, const void *dout, float tau, int causal)
+cudaError_t tc_args(race::tc::BwdArgs &a, const Plan &p, const void *q, const void *k, const void *v,
+                    const float *W, const void *out, const float *den, const void *dout, float tau, int causal)
 {
-    race::tc::BwdArgs a;
     std::memset(&a, 0, sizeof(a));
+    cudaError_t e;
+    if ((e = bf16_map(&a.tm_q, q, p, false)) != cudaSuccess || (e = bf16_map(&a.tm_k, k, p, false)) != cudaSuccess ||
+        (e = bf16_map(&a.tm_v_va, v, p, true)) != cudaSuccess)
+        return e;
+    if (out && (e = bf16_map(&a.tm_o, out, p, false)) != cudaSuccess) return e;
+    if (dout && (e = bf16_map(&a.tm_do_va, dout, p, true)) != cudaSuccess) return e;
     a.q = (const __nv_bfloat16 *)q;
     a.k = (const __nv_bfloat16 *)k;
     a.v = (const __nv_bfloat16 *)v;
@@ -288,20 +344,25 @@ race::tc::BwdArgs tc_args(const Plan &p, const void *q, const void *k, const voi
     a.nseg = p.nseg;
     a.beta = 1.f / tau;
     a.causal = causal;
-    return a;
+    return cudaSuccess;
 }
 
 cudaError_t tc_forward(const Plan &p, const void *q, const void *k, const void *v, const float *W,
                        void *out, float *den, float *states, float tau, int causal, cudaStream_t st)
 {
     namespace tc = race::tc;
-    cudaError_t e = tc_segment_totals(p, tc_args(p, q, k, v, W, nullptr, nullptr, nullptr, tau, causal), 0,
-                                      states, st);
+    tc::BwdArgs ka;
+    cudaError_t e = tc_args(ka, p, q, k, v, W, nullptr, nullptr, nullptr, tau, causal);
+    if (e != cudaSuccess) return e;
+    e = tc_segment_totals(p, ka, 0, states, st);
     if (e != cudaSuccess) return e;
     e = launch_scan(states, p, causal ? gk::SCAN_EXCL_PREFIX : gk::SCAN_TOTAL, st);
     if (e != cudaSuccess) return e;
     tc::Args a;
     std::memset(&a, 0, sizeof(a));
+    a.tm_q = ka.tm_q;
+    a.tm_k = ka.tm_k;
+    a.tm_v_va = ka.tm_v_va;
     a.q = (const __nv_bfloat16 *)q;
     a.k = (const __nv_bfloat16 *)k;
     a.v = (const __nv_bfloat16 *)v;
@@ -326,15 +387,24 @@ cudaError_t tc_forward(const Plan &p, const void *q, const void *k, const void *
 
 cudaError_t tc_backward(const Plan &p, const void *q, const void *k, const void *v, const float *W,
                         const void *out, const float *den, const void *dout, const float *ctx, float *hbuf,
-                        float *gbuf, void *dq, void *dk, void *dv, float tau, int causal, cudaStream_t st)
+                        float *gbuf, uint8_t *wimg, float *cbuf, void *dq, void *dk, void *dv, float tau,
+                        int causal, cudaStream_t st)
 {
     namespace tc = race::tc;
     const dim3 grid((unsigned)p.nseg, (unsigned)p.BH);
-    tc::BwdArgs a = tc_args(p, q, k, v, W, out, den, dout, tau, causal);
+    tc::BwdArgs a;
+    cudaError_t e = tc_args(a, p, q, k, v, W, out, den, dout, tau, causal);
+    if (e != cudaSuccess) return e;
     a.dq = (__nv_bfloat16 *)dq;
     a.dk = (__nv_bfloat16 *)dk;
     a.dv = (__nv_bfloat16 *)dv;
-    cudaError_t e;
+    a.wimg = wimg;
+    a.cbuf = cbuf;
+    e = timed("tc_w_image", st, [&] {
+        tc::tc_w_image<<<1, tc::NTH, 0, st>>>(W, wimg);
+        return cudaGetLastError();
+    });
+    if (e != cudaSuccess) return e;
     const float *hstates = ctx;
     if (!hstates) {  // key-side prefix statistics, as the forward computes them
         if ((e = tc_segment_totals(p, a, 0, hbuf, st)) != cudaSuccess) return e;
@@ -405,7 +475,7 @@ race_status_t race_attn_workspace_size(int B, int H, int64_t N, int d, int L, in
     race_status_t s = check_sizes(B, H, N, d, L, P);
     if (s != RACE_OK) return s;
     const Plan p = make_plan(B, H, N, d, L, P);
-    *bytes = p.state_elems * sizeof(float) * (backward ? 2 : 1);
+    *bytes = backward ? backward_workspace_bytes(p) : p.state_elems * sizeof(float);
     return RACE_OK;
 }
 
@@ -448,7 +518,7 @@ race_status_t race_attn_forward(const void *q, const void *k, const void *v, con
     float *states = ctx ? ctx : (float *)workspace;
     cudaStream_t st = (cudaStream_t)stream;
     cudaError_t e;
-    if (race::tc::fast_path_ok(dtype, d, L, P, tau) && g_tc_forward)
+    if (race::tc::fast_path_ok(dtype, d, L, P, tau, N) && g_tc_forward)
         e = tc_forward(p, q, k, v, W, out, den, states, tau, causal, st);
     else if (dtype == RACE_F32)
         e = dispatch_forward<float>(p, a, states, causal, st);
@@ -478,7 +548,7 @@ race_status_t race_attn_backward(const void *q, const void *k, const void *v, co
     if (ctx && !aligned16(ctx)) return RACE_ERR_INVALID_ARG;
     const Plan p = make_plan(B, H, N, d, L, P);
     const size_t one = p.state_elems * sizeof(float);
-    if (workspace_bytes < 2 * one) return RACE_ERR_WORKSPACE;
+    if (workspace_bytes < backward_workspace_bytes(p)) return RACE_ERR_WORKSPACE;
     if (ctx && ctx_bytes < one) return RACE_ERR_WORKSPACE;
     Args a = base_args(p, W, tau);
     a.q = q;
@@ -492,10 +562,12 @@ race_status_t race_attn_backward(const void *q, const void *k, const void *v, co
     a.dv = dv;
     float *hbuf = (float *)workspace;
     float *gbuf = hbuf + p.state_elems;
+    uint8_t *wimg = (uint8_t *)(gbuf + p.state_elems);
+    float *cbuf = (float *)(wimg + kWImageBytes);
     cudaStream_t st = (cudaStream_t)stream;
     cudaError_t e;
-    if (race::tc::fast_path_ok(dtype, d, L, P, tau) && g_tc_backward)
-        e = tc_backward(p, q, k, v, W, out, den, dout, ctx, hbuf, gbuf, dq, dk, dv, tau, causal, st);
+    if (race::tc::fast_path_ok(dtype, d, L, P, tau, N) && g_tc_backward)
+        e = tc_backward(p, q, k, v, W, out, den, dout, ctx, hbuf, gbuf, wimg, cbuf, dq, dk, dv, tau, causal, st);
     else if (dtype == RACE_F32)
         e = dispatch_backward<float>(p, a, ctx, hbuf, gbuf, causal, st);
     else

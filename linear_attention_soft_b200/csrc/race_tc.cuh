@@ -54,7 +54,12 @@ constexpr uint32_t VA256 = 8192;   // one SW32 atom of 256 rows
 // error word shared by all launches of this path (1 = an MMA completion wait timed out)
 __device__ int g_tc_error;
 
+// Tensor maps: every [B*H][N][64] bf16 tensor is described as a 3-D tensor (64 columns, N
+// rows, B*H heads) so that rows past a head's end read as zero; "k128" boxes are 128 rows x
+// 64 columns with the 128-byte swizzle (a K128 tile), "va" boxes 128 rows x 16 columns with
+// the 32-byte swizzle (one value-tile atom).
 struct Args {
+    CUtensorMap tm_q, tm_k, tm_v_va;
     const __nv_bfloat16 *q, *k, *v;
     const float *W;
     __nv_bfloat16 *out;
@@ -69,8 +74,11 @@ struct Args {
 };
 
 struct BwdArgs {
+    CUtensorMap tm_q, tm_k, tm_o, tm_v_va, tm_do_va;
     const __nv_bfloat16 *q, *k, *v, *o, *dout;
     const float *den, *W;
+    const uint8_t *wimg;       // W as the two bf16 K128 tiles (hi, lo) of load_w_split, 16 KB
+    float *cbuf;               // c_i = -(dO_i . o_i) per token [BH][N], written by the dq walk
     __nv_bfloat16 *dq, *dk, *dv;
     const float *state;
     int64_t state_seg_stride;
@@ -82,7 +90,8 @@ struct BwdArgs {
 };
 
 struct Ctl {
-    uint64_t bar;
+    uint64_t bar;    // MMA completion
+    uint64_t ld[4];  // TMA / bulk load completion, one per buffer set
     uint32_t tmem;
     uint32_t abort;
 };
@@ -125,30 +134,81 @@ __device__ void load_w_split(const float *W, uint8_t *whi, uint8_t *wlo)
     }
 }
 
-// Rows [0, nvalid) of a [.., 64] bf16 tensor into a K128 tile (zero rows beyond).
-__device__ __forceinline__ void load_k128_async(uint8_t *tile, const __nv_bfloat16 *src, int nvalid)
+// ---- asynchronous loads -----------------------------------------------------------------
+// Thread 0 issues every TMA / bulk load.  Barrier ctl->ld[b] has at most one load group in
+// flight; every thread keeps the same two bit masks, so the parity of the group in flight is
+// known everywhere (bit masks rather than counters: b is often a runtime value).
+struct Loads {
+    uint32_t odd;   // bit b: an odd number of groups has been issued on barrier b
+    uint32_t pend;  // bit b: the last group on barrier b has not been waited for
+};
+__device__ __forceinline__ uint32_t load_parity(const Loads &ld, int b) { return ((ld.odd >> b) & 1u) ^ 1u; }
+
+// Arm barrier b for `bytes` of traffic (thread 0) and count the group; the TMA copies that
+// follow, issued by thread 0, complete it.
+__device__ __forceinline__ uint64_t *arm_load(Ctl *ctl, Loads &ld, int b, uint32_t bytes)
 {
-    const uint32_t base = smem_u32(tile);
-#pragma unroll
-    for (int k = 0; k < 1024 / NTH; ++k) {
-        const int c = threadIdx.x + NTH * k;
-        const int row = c >> 3, ch = c & 7;
-        const bool ok = row < nvalid;
-        cp_async16(base + sw128_off(row, ch), src + (ok ? (int64_t)row * 64 + ch * 8 : 0), ok ? 16u : 0u);
-    }
+    if (threadIdx.x == 0) mbar_expect_tx(&ctl->ld[b], bytes);
+    ld.odd ^= 1u << b;
+    ld.pend |= 1u << b;
+    return &ctl->ld[b];
 }
 
-// Rows [0, nvalid) of a [.., 64] bf16 tensor into atoms 0..3 of a 128-row value tile.
-__device__ __forceinline__ void load_va_async(uint8_t *tile, const __nv_bfloat16 *src, int nvalid)
+// Rows [row0, row0 + 128) of head bh into a K128 tile (rows past the head's end read as 0).
+__device__ __forceinline__ void tma_k128(uint32_t dst, const CUtensorMap *m, int64_t row0, int bh, uint64_t *bar)
 {
-    const uint32_t base = smem_u32(tile);
+    tma_load3(dst, m, 0, (int)row0, bh, bar);
+}
+
+// Columns 0..63 of rows [row0, row0 + 128) of head bh into atoms 0..3 of a 128-row value tile.
+__device__ __forceinline__ void tma_va(uint32_t dst, const CUtensorMap *m, int64_t row0, int bh, uint64_t *bar)
+{
 #pragma unroll
-    for (int k = 0; k < 1024 / NTH; ++k) {
-        const int c = threadIdx.x + NTH * k;
-        const int row = c >> 3, ch = c & 7;
-        const bool ok = row < nvalid;
-        cp_async16(base + va_off(row, ch, T), src + (ok ? (int64_t)row * 64 + ch * 8 : 0), ok ? 16u : 0u);
+    for (int k = 0; k < 4; ++k) tma_load3(dst + (uint32_t)k * VA128, m, 16 * k, (int)row0, bh, bar);
+}
+
+// Every thread waits (bounded) for the groups in flight on the barriers in `mask`, then the
+// CTA syncs; false once the CTA has given up.
+__device__ __forceinline__ bool wait_loads(Ctl *ctl, Loads &ld, uint32_t mask)
+{
+    bool fail = false;
+    uint32_t todo = mask & ld.pend;
+    while (todo) {
+        const int b = __ffs(todo) - 1;
+        todo &= todo - 1u;
+        if (mbar_wait(&ctl->ld[b], load_parity(ld, b), WAIT_LIMIT_NS))
+            ld.pend &= ~(1u << b);
+        else
+            fail = true;
     }
+    if (fail) {
+        ctl->abort = 1u;
+        atomicExch(&g_tc_error, 1);
+    }
+    __syncthreads();
+    return *(volatile uint32_t *)&ctl->abort == 0u;
+}
+
+// Thread 0 alone waits for barrier b (data read by the tensor core only); false on timeout,
+// after marking the CTA as given up.
+__device__ __forceinline__ bool wait_load_t0(Ctl *ctl, Loads &ld, int b)
+{
+    if (!((ld.pend >> b) & 1u)) return true;
+    if (mbar_wait(&ctl->ld[b], load_parity(ld, b), WAIT_LIMIT_NS)) {
+        ld.pend &= ~(1u << b);
+        return true;
+    }
+    ctl->abort = 1u;
+    atomicExch(&g_tc_error, 1);
+    return false;
+}
+
+// Before exit: thread 0 waits (bounded) for every load group still in flight.
+__device__ __forceinline__ void drain_loads(Ctl *ctl, const Loads &ld)
+{
+    if (threadIdx.x != 0) return;
+    for (int b = 0; b < 4; ++b)
+        if ((ld.pend >> b) & 1u) mbar_wait(&ctl->ld[b], load_parity(ld, b), WAIT_LIMIT_NS);
 }
 
 // Atom 4 of a 128-row value tile: column 64 = x (1 for the ones column), zeros elsewhere.
@@ -162,7 +222,7 @@ __device__ __forceinline__ void write_col64(uint8_t *tile, int r, float x)
 // Wait for the MMAs committed to ctl->bar; one thread polls (bounded), all learn the outcome.
 __device__ __forceinline__ bool wait_mma(Ctl *ctl, uint32_t &phase)
 {
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 0 && ctl->abort == 0u) {
         if (!mbar_wait(&ctl->bar, phase & 1u, WAIT_LIMIT_NS)) {
             ctl->abort = 1u;
             atomicExch(&g_tc_error, 1);
@@ -182,20 +242,23 @@ __device__ __forceinline__ void publish_smem()
     __syncthreads();
 }
 
-// L2 prefetch of the rows [row0, row0 + n) of up to five [.., 64] bf16 tensors and of a
-// per-token fp32 vector (threads 0..5 each take one), for the chunk after the current one.
+// L2 prefetch of the rows [row0, row0 + n) of up to five [.., 64] bf16 tensors and of up to
+// two per-token fp32 vectors (threads 0..6 each take one), for a chunk ahead of the current one.
 __device__ __forceinline__ void prefetch_chunk(int64_t row0, int n, const __nv_bfloat16 *t0_,
                                                const __nv_bfloat16 *t1_, const __nv_bfloat16 *t2_,
                                                const __nv_bfloat16 *t3_, const __nv_bfloat16 *t4_,
-                                               const float *f0)
+                                               const float *f0, const float *f1 = nullptr)
 {
-    if (n <= 0 || threadIdx.x >= 6) return;
+    if (n <= 0 || threadIdx.x >= 7) return;
     const __nv_bfloat16 *ts[5] = {t0_, t1_, t2_, t3_, t4_};
     if (threadIdx.x < 5) {
         if (ts[threadIdx.x]) prefetch_l2(ts[threadIdx.x] + row0 * DH, (uint32_t)n * DH * 2u);
-    } else if (f0) {  // shrink to 16-byte aligned bounds inside the range
-        const uintptr_t lo = ((uintptr_t)(f0 + row0) + 15u) & ~(uintptr_t)15u;
-        const uintptr_t hi = (uintptr_t)(f0 + row0 + n) & ~(uintptr_t)15u;
+        return;
+    }
+    const float *f = threadIdx.x == 5 ? f0 : f1;
+    if (f) {  // shrink to 16-byte aligned bounds inside the range
+        const uintptr_t lo = ((uintptr_t)(f + row0) + 15u) & ~(uintptr_t)15u;
+        const uintptr_t hi = (uintptr_t)(f + row0 + n) & ~(uintptr_t)15u;
         if (hi > lo) prefetch_l2((const void *)lo, (uint32_t)(hi - lo));
     }
 }
@@ -245,6 +308,23 @@ __device__ __forceinline__ void row_scalars(int r, const uint8_t *doc, const uin
     rowc[r] = c;
     rowinv[r] = inv;
     if (doc_col64) write_col64(doc_col64, r, c);
+}
+
+// Per-row scalars of a chunk from the c_i the dq walk stored and den: rowc[r] = c_r,
+// rowinv[r] = 1/den_r (both 0 beyond the valid rows); c_r also into column 64 of the value
+// tile doc.  One thread per row.
+__device__ __forceinline__ void load_row_scalars(int r, bool valid, const float *c_row, const float *den_row,
+                                                 float *rowc, float *rowinv, uint8_t *doc)
+{
+    float c = 0.f, inv = 0.f;
+    if (valid) {
+        c = *c_row;
+        const float dn = *den_row;
+        inv = dn != 0.f ? 1.f / dn : 0.f;
+    }
+    rowc[r] = c;
+    rowinv[r] = inv;
+    write_col64(doc, r, c);
 }
 
 // u = tanh(proj / |x|) and t = tanh(beta u) of this thread's 16 projections (tables
@@ -660,9 +740,7 @@ constexpr uint32_t WLO = WHI + 8192;
 constexpr uint32_t RN = WLO + 8192;         // row norms [128]
 constexpr uint32_t ROWC = RN + 512;
 constexpr uint32_t ROWINV = ROWC + 512;
-constexpr uint32_t O0 = ROWINV + 512 + 512;  // o rows (backward aggregate), 1024-aligned
-constexpr uint32_t O1 = O0 + TILE;
-constexpr uint32_t BAR = O1 + TILE;
+constexpr uint32_t BAR = ROWINV + 512;
 constexpr uint32_t TOTAL = BAR + 64;
 }  // namespace agg_smem
 namespace agg_tmem {
@@ -701,6 +779,7 @@ __device__ __forceinline__ uint32_t kernel_setup(Ctl *ctl, uint32_t ncols, const
 {
     if (threadIdx.x == 0) {
         mbar_init(&ctl->bar, 1);
+        for (int b = 0; b < 4; ++b) mbar_init(&ctl->ld[b], 1);
         ctl->abort = 0;
     }
     if (threadIdx.x < 32) tmem_alloc(&ctl->tmem, ncols);
@@ -725,7 +804,7 @@ __device__ __forceinline__ void kernel_teardown(uint32_t tm, uint32_t ncols)
 // The next chunk's rows load while this chunk is processed (double-buffered tiles).
 // ------------------------------------------------------------------------------------------
 template <int MODE>
-__global__ void __launch_bounds__(NTH, 1) tc_agg(BwdArgs a)
+__global__ void __launch_bounds__(NTH, 1) tc_agg(const __grid_constant__ BwdArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = aligned_base(smem_raw);
@@ -738,6 +817,8 @@ __global__ void __launch_bounds__(NTH, 1) tc_agg(BwdArgs a)
     const uint32_t sb = smem_u32(sm);
     const __nv_bfloat16 *xsrc = MODE == 0 ? a.k : a.q;
     const __nv_bfloat16 *vsrc = MODE == 0 ? a.v : a.dout;
+    const CUtensorMap *xmap = MODE == 0 ? &a.tm_k : &a.tm_q;
+    const CUtensorMap *vmap = MODE == 0 ? &a.tm_v_va : &a.tm_do_va;
     const uint32_t tm = kernel_setup(ctl, agg_tmem::NCOLS, a.W, sm + WHI, sm + WLO);
     zero_state40(tm, agg_tmem::HTOP, agg_tmem::HBOT, qd);
     int64_t t0, t1;
@@ -745,31 +826,29 @@ __global__ void __launch_bounds__(NTH, 1) tc_agg(BwdArgs a)
     const int64_t base = (int64_t)bh * a.N;
     uint32_t phase = 0;
     bool ok = true;
-    if (t0 < t1) {
-        load_k128_async(sm + X0, xsrc + (base + t0) * DH, (int)(t1 - t0 < T ? t1 - t0 : T));
-        load_va_async(sm + VA0, vsrc + (base + t0) * DH, (int)(t1 - t0 < T ? t1 - t0 : T));
-        if (MODE == 1) load_k128_async(sm + O0, a.o + (base + t0) * DH, (int)(t1 - t0 < T ? t1 - t0 : T));
-        cp_async_commit();
-    }
+    Loads ld = {};
+    auto issue = [&](int64_t c, int b) {  // rows of chunk c into buffer set b
+        uint64_t *bar = arm_load(ctl, ld, b, 2u * TILE);
+        if (threadIdx.x == 0) {
+            tma_k128(sb + (b ? X1 : X0), xmap, c, bh, bar);
+            tma_va(sb + (b ? VA1 : VA0), vmap, c, bh, bar);
+        }
+    };
+    if (t0 < t1) issue(t0, 0);
     int buf = 0;
     for (int64_t c0 = t0; c0 < t1 && ok; c0 += T, buf ^= 1) {
         const int nv = (int)(t1 - c0 < T ? t1 - c0 : T);
         uint8_t *x = sm + (buf ? X1 : X0), *va = sm + (buf ? VA1 : VA0);
-        cp_async_wait_all();
-        __syncthreads();
+        if (!(ok = wait_loads(ctl, ld, 1u << buf))) break;
         if (c0 + T < t1) {  // next chunk's rows into the other buffers (free: their MMAs completed)
-            const int nn = (int)(t1 - c0 - T < T ? t1 - c0 - T : T);
-            load_k128_async(sm + (buf ? X0 : X1), xsrc + (base + c0 + T) * DH, nn);
-            load_va_async(sm + (buf ? VA0 : VA1), vsrc + (base + c0 + T) * DH, nn);
-            if (MODE == 1) load_k128_async(sm + (buf ? O0 : O1), a.o + (base + c0 + T) * DH, nn);
-            cp_async_commit();
+            issue(c0 + T, buf ^ 1);
             prefetch_chunk(base + c0 + 2 * T, (int)(t1 - c0 - 2 * T < T ? t1 - c0 - 2 * T : T), xsrc, vsrc,
-                           MODE ? a.o : nullptr, nullptr, nullptr, MODE ? a.den : nullptr);
+                           nullptr, nullptr, nullptr, MODE ? a.den : nullptr, MODE ? a.cbuf : nullptr);
         }
         if (qd == 0) rn[r] = row_norm(x, r);
         if (MODE == 0 && qd == 1) write_col64(va, r, r < nv ? 1.f : 0.f);
         if (MODE == 1 && qd == 2)
-            row_scalars(r, va, sm + (buf ? O1 : O0), a.den + base + c0, nv, rowc, rowinv, va);
+            load_row_scalars(r, r < nv, a.cbuf + base + c0 + r, a.den + base + c0 + r, rowc, rowinv, va);
         publish_smem();
         if (threadIdx.x == 0) {
             fence_after_sync();
@@ -791,7 +870,7 @@ __global__ void __launch_bounds__(NTH, 1) tc_agg(BwdArgs a)
         }
         ok = wait_mma(ctl, phase);
     }
-    cp_async_wait_all();
+    drain_loads(ctl, ld);
     if (ok) {
         float hv[40];
         read_state40(tm, agg_tmem::HTOP, agg_tmem::HBOT, qd, hv);
@@ -803,7 +882,7 @@ __global__ void __launch_bounds__(NTH, 1) tc_agg(BwdArgs a)
 // ------------------------------------------------------------------------------------------
 // Walk: causal (Algorithm 2) or bidirectional read-out (Algorithm 1).  grid: nseg x BH
 // ------------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(NTH, 1) tc_fwd_walk(Args a)
+__global__ void __launch_bounds__(NTH, 1) tc_fwd_walk(const __grid_constant__ Args a)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = aligned_base(smem_raw);
@@ -826,14 +905,16 @@ __global__ void __launch_bounds__(NTH, 1) tc_fwd_walk(Args a)
     const int64_t base = (int64_t)bh * a.N;
     uint32_t phase = 0;
     bool ok = true;
+    Loads ld = {};
     auto issue_loads = [&](int64_t c) {
-        const int n = (int)(t1 - c < T ? t1 - c : T);
-        load_k128_async(sm + XQ, a.q + (base + c) * DH, n);
-        if (causal) {
-            load_k128_async(sm + XK, a.k + (base + c) * DH, n);
-            load_va_async(sm + VA, a.v + (base + c) * DH, n);
+        uint64_t *bar = arm_load(ctl, ld, 0, (causal ? 3u : 1u) * TILE);
+        if (threadIdx.x == 0) {
+            tma_k128(sb + XQ, &a.tm_q, c, bh, bar);
+            if (causal) {
+                tma_k128(sb + XK, &a.tm_k, c, bh, bar);
+                tma_va(sb + VA, &a.tm_v_va, c, bh, bar);
+            }
         }
-        cp_async_commit();
         prefetch_chunk(base + c + T, (int)(t1 - c - T < T ? t1 - c - T : T), a.q, causal ? a.k : nullptr,
                        causal ? a.v : nullptr, nullptr, nullptr, nullptr);
     };
@@ -841,8 +922,7 @@ __global__ void __launch_bounds__(NTH, 1) tc_fwd_walk(Args a)
     for (int64_t c0 = t0; c0 < t1 && ok; c0 += T) {
         const int nv = (int)(t1 - c0 < T ? t1 - c0 : T);
         const bool valid = r < nv;
-        cp_async_wait_all();
-        __syncthreads();
+        if (!(ok = wait_loads(ctl, ld, 1u))) break;
         if (qd == 0) rn[r] = row_norm(sm + XQ, r);
         if (causal && qd == 1) rn[128 + r] = row_norm(sm + XK, r);
         if (causal && qd == 2) write_col64(sm + VA, r, valid ? 1.f : 0.f);
@@ -905,7 +985,7 @@ __global__ void __launch_bounds__(NTH, 1) tc_fwd_walk(Args a)
         }
         publish_smem();
     }
-    cp_async_wait_all();
+    drain_loads(ctl, ld);
     kernel_teardown(tm, fwd_tmem::NCOLS);
 }
 
@@ -978,7 +1058,7 @@ constexpr uint32_t NCOLS = 512;
 // ------------------------------------------------------------------------------------------
 // dq walk (chunks in order, prefix state H)
 // ------------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(NTH, 1) tc_bwd_q_walk(BwdArgs a)
+__global__ void __launch_bounds__(NTH, 1) tc_bwd_q_walk(const __grid_constant__ BwdArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = aligned_base(smem_raw);
@@ -1003,25 +1083,31 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_q_walk(BwdArgs a)
     const int64_t base = (int64_t)bh * a.N;
     uint32_t phase = 0;
     bool ok = true;
+    Loads ld = {};
     auto issue_kv_do = [&](int64_t c) {  // k, v, dO, o rows of chunk c
-        const int n = (int)(t1 - c < T ? t1 - c : T);
-        load_va_async(sm + DOV, a.dout + (base + c) * DH, n);
-        load_k128_async(sm + OT, a.o + (base + c) * DH, n);
-        if (causal) {
-            load_k128_async(sm + XK, a.k + (base + c) * DH, n);
-            load_va_async(sm + VA, a.v + (base + c) * DH, n);
+        uint64_t *bar = arm_load(ctl, ld, 0, (causal ? 4u : 2u) * TILE);
+        if (threadIdx.x == 0) {
+            tma_va(sb + DOV, &a.tm_do_va, c, bh, bar);
+            tma_k128(sb + OT, &a.tm_o, c, bh, bar);
+            if (causal) {
+                tma_k128(sb + XK, &a.tm_k, c, bh, bar);
+                tma_va(sb + VA, &a.tm_v_va, c, bh, bar);
+            }
         }
-        cp_async_commit();
         prefetch_chunk(base + c + T, (int)(t1 - c - T < T ? t1 - c - T : T), a.q, a.dout, a.o,
                        causal ? a.k : nullptr, causal ? a.v : nullptr, a.den);
     };
     auto issue_q = [&](int64_t c) {  // q rows for the projection
-        load_k128_async(sm + XQ, a.q + (base + c) * DH, (int)(t1 - c < T ? t1 - c : T));
-        cp_async_commit();
+        uint64_t *bar = arm_load(ctl, ld, 1, TILE);
+        if (threadIdx.x == 0) tma_k128(sb + XQ, &a.tm_q, c, bh, bar);
     };
     auto issue_q2 = [&](int64_t c) {  // q rows kept for dq
-        load_k128_async(sm + XQ2, a.q + (base + c) * DH, (int)(t1 - c < T ? t1 - c : T));
-        cp_async_commit();
+        uint64_t *bar = arm_load(ctl, ld, 2, TILE);
+        if (threadIdx.x == 0) tma_k128(sb + XQ2, &a.tm_q, c, bh, bar);
+    };
+    auto reload_w = [&]() {  // W tiles (hi, lo) back over the masked block
+        uint64_t *bar = arm_load(ctl, ld, 3, 2u * 8192u);
+        if (threadIdx.x == 0) bulk_load(sb + WHI, a.wimg, 2u * 8192u, bar);
     };
     if (t0 < t1) {
         issue_kv_do(t0);
@@ -1031,11 +1117,13 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_q_walk(BwdArgs a)
     for (int64_t c0 = t0; c0 < t1 && ok; c0 += T) {
         const int nv = (int)(t1 - c0 < T ? t1 - c0 : T);
         const bool valid = r < nv;
-        cp_async_wait_all();
-        __syncthreads();
+        if (!(ok = wait_loads(ctl, ld, 7u))) break;
         if (qd == 0) rn[r] = row_norm(sm + XQ, r);
         if (causal && qd == 1) rn[128 + r] = row_norm(sm + XK, r);
-        if (qd == 2) row_scalars(r, sm + DOV, sm + OT, a.den + base + c0, nv, rowc, rowinv, nullptr);
+        if (qd == 2) {
+            row_scalars(r, sm + DOV, sm + OT, a.den + base + c0, nv, rowc, rowinv, nullptr);
+            if (valid) a.cbuf[base + c0 + r] = rowc[r];  // for the key-side passes
+        }
         if (causal && qd == 3) write_col64(sm + VA, r, valid ? 1.f : 0.f);
         publish_smem();
         if (threadIdx.x == 0) {
@@ -1073,11 +1161,11 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_q_walk(BwdArgs a)
         }
         if (!(ok = wait_mma(ctl, phase))) break;
         if (c0 + T < t1) issue_kv_do(c0 + T);  // Phi_K, V~ and dO are free now
+        reload_w();
         // dphi = (D + c_i H_prev[:, 64]) / den_i
         features_vjp(tm, bq_tmem::DPHI, r, qd, a.beta, valid, u, t, hden, c_r, invden_r, sm + DP);
-        load_w_split(a.W, sm + WHI, sm + WLO);
         publish_smem();
-        if (threadIdx.x == 0) {
+        if (threadIdx.x == 0 && wait_load_t0(ctl, ld, 3)) {
             fence_after_sync();
             issue_dxhat(tm + bq_tmem::DX, sb + DP, sb + WHI, sb + WLO);
             mma_commit(&ctl->bar);
@@ -1094,7 +1182,7 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_q_walk(BwdArgs a)
         }
         publish_smem();
     }
-    cp_async_wait_all();
+    drain_loads(ctl, ld);
     kernel_teardown(tm, bq_tmem::NCOLS);
 }
 
@@ -1104,7 +1192,6 @@ constexpr uint32_t XQ = PHQ;
 constexpr uint32_t DP = PHQ;
 constexpr uint32_t WHI = PHQ + TILE;
 constexpr uint32_t WLO = WHI + 8192;
-constexpr uint32_t OT = PHQ + 2 * TILE;    // o rows at load
 constexpr uint32_t PHK = PHQ + 4 * TILE;   // k rows at load; Phi_K; then masked S'^T and P'
 constexpr uint32_t XK = PHK;
 constexpr uint32_t STB = PHK;              // tiles 0-1
@@ -1134,7 +1221,7 @@ constexpr uint32_t NCOLS = 512;
 // ------------------------------------------------------------------------------------------
 // dk/dv walk (chunks in reverse, suffix state G)
 // ------------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(NTH, 1) tc_bwd_kv_walk(BwdArgs a)
+__global__ void __launch_bounds__(NTH, 1) tc_bwd_kv_walk(const __grid_constant__ BwdArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = aligned_base(smem_raw);
@@ -1159,24 +1246,27 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_kv_walk(BwdArgs a)
     const int64_t nchunks = (t1 - t0 + T - 1) / T;
     uint32_t phase = 0;
     bool ok = true;
+    Loads ld = {};
     auto issue_kv_do = [&](int64_t c) {  // k, v, dO rows of chunk c
-        const int n = (int)(t1 - c < T ? t1 - c : T);
-        load_k128_async(sm + XK, a.k + (base + c) * DH, n);
-        load_va_async(sm + VA, a.v + (base + c) * DH, n);
-        if (causal) {
-            load_va_async(sm + DOC, a.dout + (base + c) * DH, n);
-            load_k128_async(sm + OT, a.o + (base + c) * DH, n);
+        uint64_t *bar = arm_load(ctl, ld, 0, (causal ? 3u : 2u) * TILE);
+        if (threadIdx.x == 0) {
+            tma_k128(sb + XK, &a.tm_k, c, bh, bar);
+            tma_va(sb + VA, &a.tm_v_va, c, bh, bar);
+            if (causal) tma_va(sb + DOC, &a.tm_do_va, c, bh, bar);
         }
-        cp_async_commit();
         if (c - T >= t0)
-            prefetch_chunk(base + c - T, T, a.k, a.v, causal ? a.q : nullptr, causal ? a.dout : nullptr,
-                           causal ? a.o : nullptr, causal ? a.den : nullptr);
+            prefetch_chunk(base + c - T, T, a.k, a.v, causal ? a.q : nullptr, causal ? a.dout : nullptr, nullptr,
+                           causal ? a.den : nullptr, causal ? a.cbuf : nullptr);
     };
     auto issue_q = [&](int64_t c) {
         if (causal) {
-            load_k128_async(sm + XQ, a.q + (base + c) * DH, (int)(t1 - c < T ? t1 - c : T));
-            cp_async_commit();
+            uint64_t *bar = arm_load(ctl, ld, 1, TILE);
+            if (threadIdx.x == 0) tma_k128(sb + XQ, &a.tm_q, c, bh, bar);
         }
+    };
+    auto reload_w = [&]() {  // W tiles (hi, lo) back over Phi_Q'
+        uint64_t *bar = arm_load(ctl, ld, 3, 2u * 8192u);
+        if (threadIdx.x == 0) bulk_load(sb + WHI, a.wimg, 2u * 8192u, bar);
     };
     if (nchunks > 0) {
         issue_kv_do(t0 + (nchunks - 1) * T);
@@ -1186,12 +1276,11 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_kv_walk(BwdArgs a)
         const int64_t c0 = t0 + ci * T;
         const int nv = (int)(t1 - c0 < T ? t1 - c0 : T);
         const bool valid = r < nv;
-        cp_async_wait_all();
-        __syncthreads();
+        if (!(ok = wait_loads(ctl, ld, 3u))) break;
         if (qd == 0) rn[128 + r] = row_norm(sm + XK, r);
         if (causal && qd == 1) rn[r] = row_norm(sm + XQ, r);
         if (causal && qd == 2)
-            row_scalars(r, sm + DOC, sm + OT, a.den + base + c0, nv, rowc, rowinv, sm + DOC);
+            load_row_scalars(r, valid, a.cbuf + base + c0 + r, a.den + base + c0 + r, rowc, rowinv, sm + DOC);
         if (qd == 3) write_col64(sm + VA, r, valid ? 1.f : 0.f);
         publish_smem();
         if (threadIdx.x == 0) {
@@ -1245,11 +1334,11 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_kv_walk(BwdArgs a)
         }
         if (!(ok = wait_mma(ctl, phase))) break;
         if (ci > 0) issue_kv_do(c0 - T);  // Phi_K / masks, V~ and [dO | c] are free now
+        reload_w();
         store_row16(tm, bkv_tmem::DVT, qd, valid, 1.f, a.dv + (base + c0 + r) * DH);
         features_vjp(tm, bkv_tmem::DPHI, r, qd, a.beta, valid, u, t, nullptr, 0.f, 1.f, sm + DP);
-        load_w_split(a.W, sm + WHI, sm + WLO);
         publish_smem();
-        if (threadIdx.x == 0) {
+        if (threadIdx.x == 0 && wait_load_t0(ctl, ld, 3)) {
             fence_after_sync();
             issue_dxhat(tm + bkv_tmem::DX, sb + DP, sb + WHI, sb + WLO);
             mma_commit(&ctl->bar);
@@ -1265,8 +1354,16 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_kv_walk(BwdArgs a)
         }
         publish_smem();
     }
-    cp_async_wait_all();
+    drain_loads(ctl, ld);
     kernel_teardown(tm, bkv_tmem::NCOLS);
+}
+
+// W [64][64] fp32 -> its two bf16 K128 tiles (hi, lo) in global memory, byte for byte as
+// load_w_split lays them out in shared memory, so that the walks reload them with one bulk
+// copy.  One CTA of NTH threads.
+__global__ void __launch_bounds__(NTH, 1) tc_w_image(const float *W, uint8_t *img)
+{
+    load_w_split(W, img, img + 8192);
 }
 
 // Waits on a barrier that nothing arrives on, for at most limit_ns, and reports the timeout
@@ -1283,12 +1380,29 @@ __global__ void tc_wait_timeout_selftest(uint64_t limit_ns)
 
 // ---- host side ---------------------------------------------------------------------------
 
-inline bool fast_path_ok(race_dtype_t dtype, int d, int L, int P, float tau)
+// Token coordinates of the TMA loads are 32-bit.
+inline bool fast_path_ok(race_dtype_t dtype, int d, int L, int P, float tau, int64_t N)
 {
-    return dtype == RACE_BF16 && d == 64 && L == 16 && P == 4 && tau > 0.f;
+    return dtype == RACE_BF16 && d == 64 && L == 16 && P == 4 && tau > 0.f && N < ((int64_t)1 << 31);
 }
 
 inline size_t smem_bytes(uint32_t total) { return total + 1024; }
+
+// TMA destinations: K128 tiles 1024-byte aligned (128-byte swizzle), value tiles 256-byte
+// aligned (32-byte swizzle); bulk copies 16-byte aligned.
+static_assert(agg_smem::X0 % 1024 == 0 && agg_smem::X1 % 1024 == 0, "agg tiles");
+static_assert(agg_smem::VA0 % 1024 == 0 && agg_smem::VA1 % 1024 == 0, "agg value tiles");
+static_assert(fwd_smem::XQ % 1024 == 0 && fwd_smem::XK % 1024 == 0 && fwd_smem::VA % 1024 == 0, "fwd tiles");
+static_assert(bq_smem::XQ % 1024 == 0 && bq_smem::XK % 1024 == 0 && bq_smem::OT % 1024 == 0 &&
+                  bq_smem::XQ2 % 1024 == 0 && bq_smem::VA % 1024 == 0 && bq_smem::DOV % 1024 == 0 &&
+                  bq_smem::WHI % 16 == 0,
+              "dq walk tiles");
+static_assert(bkv_smem::XQ % 1024 == 0 && bkv_smem::XK % 1024 == 0 && bkv_smem::VA % 1024 == 0 &&
+                  bkv_smem::DOC % 1024 == 0 && bkv_smem::WHI % 16 == 0,
+              "dk/dv walk tiles");
+static_assert(agg_smem::TOTAL + 1024 <= 232448 && fwd_smem::TOTAL + 1024 <= 232448 &&
+                  bq_smem::TOTAL + 1024 <= 232448 && bkv_smem::TOTAL + 1024 <= 232448,
+              "shared memory per CTA");
 
 }  // namespace tc
 }  // namespace race

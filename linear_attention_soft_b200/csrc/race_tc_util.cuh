@@ -1,7 +1,8 @@
 // race_tc_util.cuh -- sm_100a building blocks: UMMA descriptors, tcgen05 MMA / TMEM access,
-// bounded mbarrier waits, cp.async tile loads into swizzled shared memory.
+// bounded mbarrier waits, TMA and bulk copies into swizzled shared memory.
 #pragma once
 
+#include <cuda.h>  // CUtensorMap
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -177,6 +178,34 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64
         if (ok) return true;
         if ((it & 255u) == 255u && global_ns() - t0 > limit_ns) return false;
     }
+}
+
+// Arm an mbarrier for `bytes` of asynchronous-copy traffic (this thread's arrival included).
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+// ---- TMA / bulk copies (no multicast) -----------------------------------------------------
+// Box at coordinates (x, y, z) of a 3-D tensor map into shared memory at dst; completion is
+// counted on `bar`.  x * element size must be a multiple of 16 bytes.
+__device__ __forceinline__ void tma_load3(uint32_t dst, const CUtensorMap *map, int x, int y, int z, uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::
+            "r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// Contiguous global -> shared copy of `bytes` (both addresses 16-byte aligned, bytes a
+// multiple of 16); completion counted on `bar`.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint64_t *bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
 }
 
 // ---- cp.async ---------------------------------------------------------------------------

@@ -53,7 +53,8 @@ def test_workspace_queries(lib):
     fw = ra.race_attn_workspace_size(1, 1, 4096, 64, 16, 4, 1, 0, ra.RACE_BF16)
     bw = ra.race_attn_workspace_size(1, 1, 4096, 64, 16, 4, 1, 1, ra.RACE_BF16)
     cx = ra.race_attn_ctx_size(1, 1, 4096, 64, 16, 4, 1)
-    assert fw > 0 and bw == 2 * fw and cx == fw
+    # backward: both segment-state buffers, a 16 KB W image and c_i per token (fp32)
+    assert fw > 0 and bw == 2 * fw + 16384 + 4096 * 4 and cx == fw
     # state is [segments][L*R][d+1] fp32 per head: a multiple of that size
     assert fw % (256 * 65 * 4) == 0
     with pytest.raises(ra.RaceError) as e:
