@@ -74,6 +74,9 @@ def _load():
                                              ctypes.c_int, ctypes.c_double, ctypes.c_int,
                                              _dp, _dp, _dp]
         lib.race_oracle_backward.restype = ctypes.c_int
+        lib.race_oracle_state.argtypes = [_dp, _dp, _dp, ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
+                                          ctypes.c_int, ctypes.c_int, ctypes.c_double, _dp]
+        lib.race_oracle_state.restype = ctypes.c_int
         lib.race_oracle_num_threads.argtypes = []
         lib.race_oracle_num_threads.restype = ctypes.c_int
         _lib = lib
@@ -192,3 +195,19 @@ def backward(q, k, v, W, dout, tau: float, causal: bool):
     if rc != 0:
         raise RuntimeError("race_oracle_backward failed with code %d" % rc)
     return dq, dk, dv
+
+
+def state(k, v, W, tau: float) -> np.ndarray:
+    """Bucket statistics H[m, c] = sum_j phi(k_j)[m] [v_j, 1][c] over every key of each head
+    (zh §2.2: A = column d, B = columns 0..d-1 of every table).  k, v: [..., N, d];
+    returns [..., L*2^P, d+1]."""
+    k, v, W = _f64(k), _f64(v), _f64(W)
+    *lead, N, d = k.shape
+    BH = int(np.prod(lead)) if lead else 1
+    L, P, dw = W.shape
+    assert dw == d and v.shape == k.shape
+    H = np.empty((BH, L << P, d + 1), dtype=np.float64)
+    rc = _load().race_oracle_state(_ptr(k), _ptr(v), _ptr(W), BH, N, d, L, P, float(tau), _ptr(H))
+    if rc != 0:
+        raise RuntimeError("race_oracle_state failed with code %d" % rc)
+    return H.reshape(tuple(lead) + (L << P, d + 1))

@@ -334,6 +334,46 @@ int race_oracle_forward(const double *q, const double *k, const double *v, const
     return 0;
 }
 
+/* Bucket statistics of one head over all N keys, H[m][c] = sum_j phi(k_j)[m] v~_j[c]
+ * (zh §2.2, A and B of every table in one [M][d+1] array, m-major): the state Algorithm 2
+ * carries after token N-1, from which a streaming step continues. */
+static int state_head(const double *k, const double *v, const double *W, int64_t N, int d, int L,
+                      int P, double tau, double *H)
+{
+    const int M = L << P, D = d + 1;
+    const int hard = tau == 0.0;
+    const double beta = hard ? 0.0 : 1.0 / tau;
+    const int64_t NB = N < RACE_ORACLE_BLOCK ? (N > 0 ? N : 1) : RACE_ORACLE_BLOCK;
+    double *phik = (double *)malloc(sizeof(double) * (size_t)NB * M);
+    if (!phik) return 1;
+    memset(H, 0, sizeof(double) * (size_t)M * D);
+    for (int64_t t0 = 0; t0 < N; t0 += NB) {
+        const int64_t nt = (N - t0 < NB) ? N - t0 : NB;
+        features_block(k, t0, nt, d, W, L, P, beta, hard, phik);
+#pragma omp parallel for schedule(static)
+        for (int m = 0; m < M; ++m)
+            for (int64_t t = 0; t < nt; ++t) {
+                const double f = phik[t * M + m];
+                for (int c = 0; c < D; ++c) H[(size_t)m * D + c] += f * vt_at(v, t0 + t, d, c);
+            }
+    }
+    free(phik);
+    return 0;
+}
+
+int race_oracle_state(const double *k, const double *v, const double *W, int64_t BH, int64_t N,
+                      int d, int L, int P, double tau, double *H)
+{
+    if (BH < 0 || N < 0 || d < 1 || L < 1 || P < 1 || P > 6 || tau < 0.0) return 2;
+    const size_t MD = (size_t)(L << P) * (size_t)(d + 1);
+    for (int64_t bh = 0; bh < BH; ++bh) {
+        const size_t off = (size_t)bh * N * d;
+        int rc = state_head(k + off, v + off, W, N, d, L, P, tau, H + (size_t)bh * MD);
+        if (rc) return rc;
+    }
+    return 0;
+}
+
 /* ---------------------------------------------------------------------------------------- */
 /* Backward (chain rule through the forward above; soft hashing only)                      */
 /* ---------------------------------------------------------------------------------------- */

@@ -64,6 +64,11 @@ WORKLOADS: Dict[str, Workload] = {
     "c4_causal_h4_n12m_d128": Workload("c4_causal_h4_n12m_d128", 1, 4, 12_000_000, 128, 32, 5,
                                        0.5, True, "bf16", 3),
     "c5_sweep": Workload("c5_sweep", 1, 1, 1 << 20, 64, 16, 4, 0.5, True, "bf16", 4),
+    # bidirectional (Algorithm 1) forward + backward at the c2 and c3 sizes
+    "n1_noncausal_b2h8_n64k": Workload("n1_noncausal_b2h8_n64k", 2, 8, 65536, 64, 16, 4, 0.5, False,
+                                       "bf16", 5),
+    "n1_noncausal_n4m_clusters": Workload("n1_noncausal_n4m_clusters", 1, 1, 4_194_304, 64, 16, 4, 0.5,
+                                          False, "bf16", 6, "clusters"),
 }
 SWEEP_N = (1 << 20, 1 << 22, 1 << 24, 75_000_000)
 

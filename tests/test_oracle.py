@@ -317,3 +317,55 @@ def test_backward_spans_feature_blocks():
     dq2, _, _ = oracle.backward(q[:2100], k[:2100], v[:2100], W, do[:2100], 0.5, True)
     np.testing.assert_allclose(dq[:2100], dq2, rtol=1e-12, atol=1e-14)
     np.testing.assert_allclose(dv.sum(0), do.sum(0), rtol=1e-9, atol=1e-9)
+
+
+# ------------------------------------------------------------------------------------------
+# Bucket statistics (zh §2.2): the state a streaming (decode-time) step continues from
+# ------------------------------------------------------------------------------------------
+
+def test_state_hard_hash_sums_values_per_bucket():
+    """With hard hashing every key lands in one bucket per table, so each state row is the
+    sum of [v_j, 1] over the keys whose sign-hash index picks that corner."""
+    _, k, v, W = _case(N=200, d=6, L=3, P=3, seed=23)
+    L, P = W.shape[0], W.shape[1]
+    R = 1 << P
+    H = oracle.state(k, v, W, 0.0)
+    idx = oracle.hash_indices(k, W)
+    want = np.zeros((L * R, k.shape[1] + 1))
+    for j in range(k.shape[0]):
+        for l in range(L):
+            want[l * R + idx[j, l], :-1] += v[j]
+            want[l * R + idx[j, l], -1] += 1.0
+    np.testing.assert_allclose(H, want, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("tau", [0.25, 1.0])
+def test_state_tables_split_every_key_once(tau):
+    """A soft assignment is a distribution over each table's corners, so summed over the
+    corners of any one table the state counts every key once: sum_r A_l[r] = N and
+    sum_r B_l[r, :] = sum_j v_j."""
+    _, k, v, W = _case(N=150, d=5, L=4, P=3, seed=24)
+    L, P = W.shape[0], W.shape[1]
+    H = oracle.state(k, v, W, tau).reshape(L, 1 << P, -1).sum(1)
+    np.testing.assert_allclose(H[:, -1], k.shape[0], rtol=1e-12)
+    np.testing.assert_allclose(H[:, :-1], np.broadcast_to(v.sum(0), (L, v.shape[1])), rtol=1e-11, atol=1e-11)
+
+
+def test_state_is_additive_over_tokens():
+    """The statistics are a sum over keys: a run across the oracle's feature blocks equals the
+    sum of the states of its two parts."""
+    _, k, v, W = _case(N=4500, d=4, L=2, P=2, seed=25)
+    H = oracle.state(k, v, W, 0.5)
+    H2 = oracle.state(k[:2100], v[:2100], W, 0.5) + oracle.state(k[2100:], v[2100:], W, 0.5)
+    np.testing.assert_allclose(H, H2, rtol=1e-12, atol=1e-10)
+
+
+def test_state_read_out_is_the_last_causal_row():
+    """Algorithm 2 reads query i out of the statistics of keys 0..i: reading the last query
+    out of the state of the whole prefix gives the causal forward's last row."""
+    q, k, v, W = _case(N=40, d=6, L=3, P=2, seed=26)
+    H = oracle.state(k, v, W, 0.5)
+    y = oracle.features(q[-1], W, 0.5) @ H
+    out, den = oracle.forward(q, k, v, W, 0.5, True, rows=[39])
+    np.testing.assert_allclose(den[0], y[-1], rtol=1e-12)
+    np.testing.assert_allclose(out[0], y[:-1] / y[-1], rtol=1e-12)

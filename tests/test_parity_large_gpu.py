@@ -119,9 +119,10 @@ def _check(w, sampled=0, prefix_heads=(0,), prefix_n=4096, full_heads=()):
     try:
         for bh in full_heads:
             sl = lambda t: to64(t.view(w.B * w.H, w.N, -1)[bh])
-            o_ref, den_ref = oracle.forward(sl(inp["q"]), sl(inp["k"]), sl(inp["v"]), to64(inp["W"]), w.tau, True)
+            o_ref, den_ref = oracle.forward(sl(inp["q"]), sl(inp["k"]), sl(inp["v"]), to64(inp["W"]), w.tau,
+                                            w.causal)
             g_ref = oracle.backward(sl(inp["q"]), sl(inp["k"]), sl(inp["v"]), to64(inp["W"]), sl(inp["do"]),
-                                    w.tau, True)
+                                    w.tau, w.causal)
             got = [t.view(w.B * w.H, w.N, -1)[bh] for t in (out, dq, dk, dv)]
             m["h%d_out" % bh] = rel_err(got[0], o_ref)
             m["h%d_den" % bh] = rel_err(den.view(w.B * w.H, w.N)[bh], den_ref)
@@ -164,4 +165,19 @@ def test_c4_causal_h4_n12m_d128():
     """Workload c4 (B1 H4 N=12,000,000 d128 bf16, L32 P5 = 1024 features, tau 0.5)."""
     w = race_inputs.WORKLOADS["c4_causal_h4_n12m_d128"]
     m = _check(w, prefix_heads=(0, 3), prefix_n=2048)
+    assert max(m.values()) <= TOL, json.dumps(m)
+
+
+def test_n1_noncausal_b2h8_n64k_all_rows():
+    """Bidirectional (Algorithm 1) forward + backward, B2 H8 N65536 d64 bf16: every output of
+    two whole heads."""
+    w = race_inputs.WORKLOADS["n1_noncausal_b2h8_n64k"]
+    m = _check(w, prefix_n=0, full_heads=(0, w.B * w.H - 1))
+    assert max(m.values()) <= TOL, json.dumps(m)
+
+
+def test_n1_noncausal_n4m_clusters_full_size():
+    """Bidirectional forward + backward at N=4,194,304 (clustered Q/K): sampled forward rows
+    against the oracle (one streaming pass over the keys) and the gradient identities."""
+    m = _check(race_inputs.WORKLOADS["n1_noncausal_n4m_clusters"], sampled=2048, prefix_n=0)
     assert max(m.values()) <= TOL, json.dumps(m)
