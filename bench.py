@@ -63,9 +63,12 @@ def kernel_work(name: str, w: race_inputs.Workload):
     table = {
         "agg_kv": (2 * d * s, 2 * M * D + 2 * LP * d),
         "fwd_walk": (4 * d * s + 4, 4 * M * D + 4 * LP * d),
-        "bwd_q_walk": (6 * d * s + 4, 4 * M * D + 6 * LP * d),
-        "agg_qdy": (3 * d * s + 4, 2 * M * D + 2 * LP * d),
-        "bwd_kv_walk": (7 * d * s + 4, 6 * M * D + 6 * LP * d),
+        # q, k, v, o, dO, den in; dq and c_i out
+        "bwd_q_walk": (6 * d * s + 8, 4 * M * D + 6 * LP * d),
+        # q, dO, den, c_i in
+        "agg_qdy": (2 * d * s + 8, 2 * M * D + 2 * LP * d),
+        # q, k, v, dO, den, c_i in; dk, dv out
+        "bwd_kv_walk": (6 * d * s + 8, 6 * M * D + 6 * LP * d),
         "bwd_walk": (10 * d * s + 4, 10 * M * D + 12 * LP * d),
     }
     for key, val in table.items():
@@ -390,6 +393,89 @@ def run_ours(args, w):
         torch.distributed.destroy_process_group()
 
 
+# ---- decode-time streaming step ---------------------------------------------------------
+DECODE = {"B": 128, "H": 32, "d": 64, "L": 16, "P": 4, "tau": 0.5, "prompt": 256, "seed": 9}
+
+
+def run_decode(args):
+    """One step = race_attn_decode_step for every (b, h) (one new token per head).  The
+    B*H = 4096 states (272 MB fp32) exceed L2, so every step streams them from HBM."""
+    import linear_attention_soft_b200 as ra
+    c = DECODE
+    B, H, d, L, P, tau = c["B"], c["H"], c["d"], c["L"], c["P"], c["tau"]
+    BH, M, D = B * H, L << P, d + 1
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+    n_tok = args.warmup + args.steps
+    inp = race_inputs.small_normal(B, H, c["prompt"] + n_tok, d, L, P, c["seed"], dtype=torch.bfloat16, device=dev)
+    W = inp["W"]
+    state = ra.state(inp["k"][:, :, :c["prompt"]].contiguous(), inp["v"][:, :, :c["prompt"]].contiguous(), W, tau)
+    toks = {n: inp[n][:, :, c["prompt"]:].permute(2, 0, 1, 3).contiguous() for n in ("q", "k", "v")}
+    out = torch.empty((B, H, d), dtype=torch.bfloat16, device=dev)
+    den = torch.empty((B, H), dtype=torch.float32, device=dev)
+    ws = torch.empty(ra.race_attn_decode_workspace_size(B, H, d, L, P), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i, q=None, k=None, v=None):
+        ra.race_attn_decode_step(toks["q"][i] if q is None else q, toks["k"][i] if k is None else k,
+                                 toks["v"][i] if v is None else v, W, state, out, den, tau, ws, stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(0)
+    clocks.start()
+    time.sleep(0.3)
+    ra.race_attn_profile_reset()
+    ra.race_attn_profile_enable(True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.warmup, n_tok):
+        step(i)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ra.race_attn_profile_enable(False)
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    prof = ra.race_attn_profile_read()
+    # end to end: the step's tokens from pinned host memory in, out and den back
+    hq, hk, hv = (toks[n][0].cpu().pin_memory() for n in ("q", "k", "v"))
+    dq_, dk_, dv_ = (torch.empty_like(t, device=dev) for t in (hq, hk, hv))
+    ho = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    hd = torch.empty(den.shape, dtype=den.dtype, pin_memory=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        dq_.copy_(hq, non_blocking=True)
+        dk_.copy_(hk, non_blocking=True)
+        dv_.copy_(hv, non_blocking=True)
+        step(0, dq_, dk_, dv_)
+        ho.copy_(out, non_blocking=True)
+        hd.copy_(den, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / args.steps
+    upd_ms, upd_n = prof.get("decode_update", (0.0, 1))
+    per_launch_s = upd_ms / upd_n / 1e3
+    byts = BH * (2 * M * D * 4 + 3 * d * 2)      # the state read and written, the token read
+    roof = {"bound": "hbm", "achieved": byts / per_launch_s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "traffic": None, "kernel": "decode_update", "ms_per_launch": per_launch_s * 1e3,
+            "peak_source": peaks["source"]}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    line = {"metric": "RACE decode step tokens/s (one token per head, B*H=4096 heads, L16 P4 d64)",
+            "value": BH / (ms / 1e3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "decode_b128h32", "B": B, "H": H, "d": d, "L": L, "P": P, "tau": tau,
+                       "prompt": c["prompt"], "l2": "states larger than L2 (no flush)"},
+            "e2e": {"value": BH / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": 3 * BH * d * 2,
+                    "d2h_bytes_per_step": BH * d * 2 + BH * 4},
+            "gpu_launches": sum(n for _, n in prof.values()), "roofline": roof,
+            "kernels": {n: {"ms_total": t, "launches": k} for n, (t, k) in prof.items()},
+            "clocks": clk, "cpu_baseline": None}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -400,13 +486,17 @@ def main():
                     choices=sorted(race_inputs.WORKLOADS))
     ap.add_argument("--n", type=int, default=0, help="override the sequence length")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--decode", action="store_true",
+                    help="time the streaming decode step instead (one token per head, 4096 heads)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     w = race_inputs.WORKLOADS[args.workload]
     if args.n:
         w = w.with_n(args.n)
-    if args.impl == "reference":
+    if args.decode:
+        run_decode(args)
+    elif args.impl == "reference":
         run_reference(args, w)
     else:
         run_ours(args, w)

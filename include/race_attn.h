@@ -172,6 +172,48 @@ race_status_t race_attn_forward_noalloc(const void *q, const void *k, const void
                                         race_dtype_t dtype, race_stream_t stream);
 
 /*
+ * Bucket statistics of every key of each head: H[m][c] = sum_j phi(k_j)[m] [v_j, 1][c],
+ * m = l * 2^P + r, i.e. B_l (columns 0..d-1) and A_l (column d) of zh §2.2 for all tables in
+ * one array -- the running statistics of Algorithm 2 (zh §2.3) after the last token, which
+ * race_attn_decode_step continues from (a prompt of N tokens, then one token per step).
+ *   k, v       device, [B,H,N,d] in dtype, 16-byte aligned.
+ *   W          device fp32 [L,P,d], as race_attn_forward.
+ *   state      device fp32 [B*H][L*2^P][d+1], written (zero-filled when N = 0).
+ *   tau        >= 0 as race_attn_forward (0: hard sign hash).
+ *   workspace  device, workspace_bytes >= race_attn_workspace_size(..., backward = 0); scratch.
+ * Sizes and errors as race_attn_forward.  Asynchronous on `stream`.
+ */
+race_status_t race_attn_state(const void *k, const void *v, const float *W, float *state, int B,
+                              int H, int64_t N, int d, int L, int P, float tau,
+                              race_dtype_t dtype, void *workspace, size_t workspace_bytes,
+                              race_stream_t stream);
+
+/* Device workspace, in bytes, that race_attn_decode_step needs for these sizes. */
+race_status_t race_attn_decode_workspace_size(int B, int H, int d, int L, int P, size_t *bytes);
+
+/*
+ * One streaming (decode-time) step of Algorithm 2 (zh §2.3) for every (b, h): the new
+ * token joins the cumulative statistics, then its query is read out of them,
+ *   H += phi(k_t) [v_t, 1]^T;   Y = phi(q_t)^T H;   out_t = Y[:d] / Y[d],  den_t = Y[d]
+ * with the feature map of race_attn_forward, so that a prompt's race_attn_state followed by
+ * steps for tokens N, N+1, ... gives the causal forward's rows N, N+1, ... .
+ *   q, k, v    device, [B,H,d] in dtype: the new token of every head.
+ *   W          device fp32 [L,P,d].
+ *   state      device fp32 [B*H][L*2^P][d+1], read and updated in place.
+ *   out        device [B,H,d] in dtype, written; den device fp32 [B,H] or NULL.
+ *   tau        >= 0 (0: hard sign hash; a row whose buckets are all empty gets out = 0).
+ *   workspace  device, workspace_bytes >= race_attn_decode_workspace_size(...); scratch.
+ * Pointers 16-byte aligned.  Sizes as race_attn_forward (N does not apply).  Errors:
+ * RACE_ERR_INVALID_ARG (NULL or misaligned pointers, bad sizes or tau),
+ * RACE_ERR_UNSUPPORTED, RACE_ERR_WORKSPACE, RACE_ERR_CUDA.  Asynchronous on `stream`;
+ * calls on one state must be ordered (same stream).
+ */
+race_status_t race_attn_decode_step(const void *q, const void *k, const void *v, const float *W,
+                                    float *state, void *out, float *den, int B, int H, int d,
+                                    int L, int P, float tau, race_dtype_t dtype, void *workspace,
+                                    size_t workspace_bytes, race_stream_t stream);
+
+/*
  * Opt-in kernel timing (a measurement aid; the method has no counterpart).  While enabled,
  * every kernel the library launches is bracketed by a pair of CUDA events recorded on the
  * launch stream; race_attn_profile_read waits for the recorded events, adds each

@@ -24,7 +24,8 @@ __all__ = [
     "race_attn_forward", "race_attn_backward", "race_attn_hash_indices",
     "forward", "backward", "race_attn_profile_enable", "race_attn_profile_reset",
     "race_attn_profile_read", "race_attn_forward_noalloc", "RACE_NOALLOC_SCRATCH_BYTES",
-    "race_attn_device_error", "race_attn_selftest_wait_timeout",
+    "race_attn_device_error", "race_attn_selftest_wait_timeout", "race_attn_state",
+    "race_attn_decode_workspace_size", "race_attn_decode_step", "state", "decode_step",
 ]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -86,6 +87,14 @@ def load_library():
     lib.race_attn_forward_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _i64, _int,
                                               _int, _int, ctypes.c_float, _int, _int, _vp]
     lib.race_attn_forward_noalloc.restype = _int
+    lib.race_attn_state.argtypes = [_vp, _vp, _vp, _vp, _int, _int, _i64, _int, _int, _int,
+                                    ctypes.c_float, _int, _vp, _sz, _vp]
+    lib.race_attn_state.restype = _int
+    lib.race_attn_decode_workspace_size.argtypes = [_int, _int, _int, _int, _int, ctypes.POINTER(_sz)]
+    lib.race_attn_decode_workspace_size.restype = _int
+    lib.race_attn_decode_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int,
+                                          _int, ctypes.c_float, _int, _vp, _sz, _vp]
+    lib.race_attn_decode_step.restype = _int
     lib.race_attn_profile_enable.argtypes = [_int]
     lib.race_attn_profile_enable.restype = None
     lib.race_attn_profile_reset.argtypes = []
@@ -193,6 +202,34 @@ def race_attn_forward_noalloc(q, k, v, W, out, den, tau: float, causal: bool, st
         int(bool(causal)), _dtype_code(q), _stream(stream)), "race_attn_forward_noalloc")
 
 
+def race_attn_state(k, v, W, state, tau: float, workspace, stream=None) -> None:
+    """C ABI bucket statistics of every key: state is [B*H, L*2^P, d+1] fp32, written."""
+    B, H, N, d, L, P = _dims(k, W)
+    _check(load_library().race_attn_state(
+        _ptr(k), _ptr(v), _ptr(W), _ptr(state), B, H, N, d, L, P, float(tau), _dtype_code(k),
+        _ptr(workspace), _nbytes(workspace), _stream(stream)), "race_attn_state")
+
+
+def race_attn_decode_workspace_size(B, H, d, L, P) -> int:
+    out = _sz()
+    _check(load_library().race_attn_decode_workspace_size(B, H, d, L, P, ctypes.byref(out)),
+           "race_attn_decode_workspace_size")
+    return out.value
+
+
+def race_attn_decode_step(q, k, v, W, state, out, den, tau: float, workspace, stream=None) -> None:
+    """C ABI streaming step: q, k, v, out are [B,H,d]; den [B,H] fp32 or None; state is
+    updated in place."""
+    B, H, d = q.shape
+    L, P, dw = W.shape
+    if dw != d:
+        raise ValueError("W is [L, P, d] with the d of q")
+    _check(load_library().race_attn_decode_step(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(W), _ptr(state), _ptr(out), _ptr(den), B, H, d, L, P,
+        float(tau), _dtype_code(q), _ptr(workspace), _nbytes(workspace), _stream(stream)),
+        "race_attn_decode_step")
+
+
 def race_attn_device_error(stream=None) -> int:
     """1 if a tensor-core kernel gave up waiting on an MMA since the last call (and clear)."""
     flag = _int()
@@ -257,3 +294,24 @@ def backward(q, k, v, W, out, den, dout, tau: float, causal: bool, ctx=None, str
     race_attn_backward(q, k, v, W, out, den, dout, ctx, dq, dk, dv, tau, causal,
                        _workspace(q, W, causal, True), stream)
     return dq, dk, dv
+
+
+def state(k, v, W, tau: float, stream=None) -> torch.Tensor:
+    """Allocate and compute the bucket statistics of every key: [B*H, L*2^P, d+1] fp32."""
+    B, H, N, d, L, P = _dims(k, W)
+    st = torch.empty((B * H, L << P, d + 1), dtype=torch.float32, device=k.device)
+    race_attn_state(k, v, W, st, tau, _workspace(k, W, False, False), stream)
+    return st
+
+
+def decode_step(q, k, v, W, state, tau: float, stream=None):
+    """Allocate and run one streaming step ([B,H,d] q/k/v): returns (out, den); `state` is
+    updated in place."""
+    B, H, d = q.shape
+    L, P, _ = W.shape
+    out = torch.empty_like(q)
+    den = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    ws = torch.empty(max(race_attn_decode_workspace_size(B, H, d, L, P), 16), dtype=torch.uint8,
+                     device=q.device)
+    race_attn_decode_step(q, k, v, W, state, out, den, tau, ws, stream)
+    return out, den

@@ -11,6 +11,7 @@
 #include <vector>
 
 #include "race_attn.h"
+#include "race_decode.cuh"
 #include "race_generic.cuh"
 #include "race_tc.cuh"
 
@@ -450,6 +451,43 @@ cudaError_t dispatch_backward(const Plan &p, const Args &a, const float *ctx, fl
     return generic_backward<DT, 16>(p, a, ctx, ctx != nullptr, hbuf, gbuf, causal, st);
 }
 
+// Bucket statistics of every key of each head (Algorithm 1's A and B): segment totals of the
+// key side, summed over the segments into segment 0's slot of `tot`.
+template <typename DT, int T>
+cudaError_t generic_totals(const Plan &p, Args a, float *tot, cudaStream_t st)
+{
+    const size_t smem = gk::Smem(T, p.d, p.P).total * sizeof(float);
+    const dim3 grid((unsigned)p.G, (unsigned)p.nseg, (unsigned)p.BH);
+    a.causal = 0;
+    a.agg_out = tot;
+    return timed("generic_agg_kv", st, [&] { return launch(gk::race_agg<DT, T, gk::AGG_KV>, grid, 1, smem, st, a); });
+}
+
+template <typename DT>
+cudaError_t dispatch_totals(const Plan &p, const Args &a, float *tot, cudaStream_t st)
+{
+    if (p.d <= 64) return generic_totals<DT, 32>(p, a, tot, st);
+    return generic_totals<DT, 16>(p, a, tot, st);
+}
+
+// Decode step: rows of each head's state split over nsplit CTAs (about two CTAs per SM over
+// all heads, at least 32 rows per CTA).
+struct DecodePlan {
+    int nsplit, rows_per_split;
+};
+DecodePlan decode_plan(int BH, int M)
+{
+    const int target = 2 * device_sm_count();
+    int nsplit = (target + BH - 1) / BH;
+    const int maxsplit = (M + 31) / 32;
+    if (nsplit > maxsplit) nsplit = maxsplit;
+    if (nsplit < 1) nsplit = 1;
+    DecodePlan dp;
+    dp.rows_per_split = (M + nsplit - 1) / nsplit;
+    dp.nsplit = (M + dp.rows_per_split - 1) / dp.rows_per_split;
+    return dp;
+}
+
 }  // namespace
 
 extern "C" {
@@ -656,6 +694,116 @@ int race_attn_profile_read(char *names, float *ms, int64_t *launches, int max_ke
         if (launches) launches[i] = g_prof[i].launches;
     }
     return n;
+}
+
+}  // extern "C"
+
+extern "C" {
+
+race_status_t race_attn_state(const void *k, const void *v, const float *W, float *state, int B, int H,
+                              int64_t N, int d, int L, int P, float tau, race_dtype_t dtype, void *workspace,
+                              size_t workspace_bytes, race_stream_t stream)
+{
+    if (dtype != RACE_F32 && dtype != RACE_BF16) return RACE_ERR_INVALID_ARG;
+    if (!(tau >= 0.f) || !std::isfinite(tau)) return RACE_ERR_INVALID_ARG;
+    race_status_t s = check_sizes(B, H, N, d, L, P);
+    if (s != RACE_OK) return s;
+    if (!state || !W || !aligned16(state) || !aligned16(W)) return RACE_ERR_INVALID_ARG;
+    const Plan p = make_plan(B, H, N, d, L, P);
+    const size_t md = (size_t)p.M * p.D;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (N == 0)
+        return cudaMemsetAsync(state, 0, (size_t)p.BH * md * sizeof(float), st) == cudaSuccess ? RACE_OK
+                                                                                             : RACE_ERR_CUDA;
+    if (!k || !v || !workspace || !aligned16(k) || !aligned16(v) || !aligned16(workspace))
+        return RACE_ERR_INVALID_ARG;
+    if (workspace_bytes < p.state_elems * sizeof(float)) return RACE_ERR_WORKSPACE;
+    float *tot = (float *)workspace;
+    cudaError_t e;
+    if (race::tc::fast_path_ok(dtype, d, L, P, tau, N) && g_tc_forward) {
+        race::tc::BwdArgs ka;
+        e = tc_args(ka, p, k, k, v, W, nullptr, nullptr, nullptr, tau, 0);
+        if (e == cudaSuccess) e = tc_segment_totals(p, ka, 0, tot, st);
+    } else {
+        Args a = base_args(p, W, tau);
+        a.q = k;
+        a.k = k;
+        a.v = v;
+        e = dtype == RACE_F32 ? dispatch_totals<float>(p, a, tot, st) : dispatch_totals<__nv_bfloat16>(p, a, tot, st);
+    }
+    if (e == cudaSuccess) e = launch_scan(tot, p, gk::SCAN_TOTAL, st);
+    if (e == cudaSuccess)
+        e = cudaMemcpy2DAsync(state, md * sizeof(float), tot, (size_t)p.nseg * md * sizeof(float), md * sizeof(float),
+                              (size_t)p.BH, cudaMemcpyDeviceToDevice, st);
+    return e == cudaSuccess ? RACE_OK : RACE_ERR_CUDA;
+}
+
+race_status_t race_attn_decode_workspace_size(int B, int H, int d, int L, int P, size_t *bytes)
+{
+    if (!bytes) return RACE_ERR_INVALID_ARG;
+    race_status_t s = check_sizes(B, H, 1, d, L, P);
+    if (s != RACE_OK) return s;
+    const int M = L << P;
+    const DecodePlan dp = decode_plan(B * H, M);
+    *bytes = (size_t)B * H * dp.nsplit * (size_t)(d + 1) * sizeof(float);
+    return RACE_OK;
+}
+
+race_status_t race_attn_decode_step(const void *q, const void *k, const void *v, const float *W, float *state,
+                                    void *out, float *den, int B, int H, int d, int L, int P, float tau,
+                                    race_dtype_t dtype, void *workspace, size_t workspace_bytes,
+                                    race_stream_t stream)
+{
+    if (dtype != RACE_F32 && dtype != RACE_BF16) return RACE_ERR_INVALID_ARG;
+    if (!(tau >= 0.f) || !std::isfinite(tau)) return RACE_ERR_INVALID_ARG;
+    race_status_t s = check_sizes(B, H, 1, d, L, P);
+    if (s != RACE_OK) return s;
+    const void *ptrs[] = {q, k, v, W, state, out, workspace};
+    for (const void *ptr : ptrs)
+        if (!ptr || !aligned16(ptr)) return RACE_ERR_INVALID_ARG;
+    if (den && !aligned16(den)) return RACE_ERR_INVALID_ARG;
+    namespace dk = race::decode;
+    dk::Args a;
+    std::memset(&a, 0, sizeof(a));
+    const int BH = B * H;
+    a.q = q;
+    a.k = k;
+    a.v = v;
+    a.W = W;
+    a.state = state;
+    a.part = (float *)workspace;
+    a.out = out;
+    a.den = den;
+    a.d = d;
+    a.L = L;
+    a.P = P;
+    a.M = L << P;
+    a.D = d + 1;
+    const DecodePlan dp = decode_plan(BH, a.M);
+    a.nsplit = dp.nsplit;
+    a.rows_per_split = dp.rows_per_split;
+    a.hard = tau == 0.f;
+    a.beta = a.hard ? 0.f : 1.f / tau;
+    if (workspace_bytes < (size_t)BH * dp.nsplit * (size_t)a.D * sizeof(float)) return RACE_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    const size_t smem = (size_t)dk::update_smem_floats(d, a.D, dp.rows_per_split) * sizeof(float);
+    const dim3 grid((unsigned)dp.nsplit, (unsigned)BH);
+    cudaError_t e = timed("decode_update", st, [&] {
+        if (dtype == RACE_F32)
+            dk::race_decode_update<float><<<grid, dk::NT, smem, st>>>(a);
+        else
+            dk::race_decode_update<__nv_bfloat16><<<grid, dk::NT, smem, st>>>(a);
+        return cudaGetLastError();
+    });
+    if (e == cudaSuccess)
+        e = timed("decode_readout", st, [&] {
+            if (dtype == RACE_F32)
+                dk::race_decode_readout<float><<<BH, dk::NT, 0, st>>>(a);
+            else
+                dk::race_decode_readout<__nv_bfloat16><<<BH, dk::NT, 0, st>>>(a);
+            return cudaGetLastError();
+        });
+    return e == cudaSuccess ? RACE_OK : RACE_ERR_CUDA;
 }
 
 }  // extern "C"

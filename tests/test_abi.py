@@ -138,3 +138,34 @@ def test_product_path_has_no_cpu_fallback():
     assert "oracle" not in src.replace("oracle.", "")
     for f in os.listdir(os.path.join(ROOT, "linear_attention_soft_b200", "csrc")):
         assert "oracle" not in open(os.path.join(ROOT, "linear_attention_soft_b200", "csrc", f)).read().lower()
+
+
+def test_decode_entry_points_reject_bad_arguments_without_launching(lib):
+    import linear_attention_soft_b200 as ra
+    sz = ctypes.c_size_t()
+    assert lib.race_attn_decode_workspace_size(1, 1, 64, 16, 4, ctypes.byref(sz)) == ra.RACE_OK
+    # one share of d+1 fp32 per CTA of each head; at most one CTA per 32 state rows
+    assert sz.value % (65 * 4) == 0 and 0 < sz.value // (65 * 4) <= 256 // 32
+    assert lib.race_attn_decode_workspace_size(1, 1, 66, 16, 4, ctypes.byref(sz)) == ra.RACE_ERR_UNSUPPORTED
+    assert lib.race_attn_decode_workspace_size(1, 1, 64, 16, 6, ctypes.byref(sz)) == ra.RACE_ERR_UNSUPPORTED
+    f = lib.race_attn_decode_step
+    args = [16, 16, 16, 16, 16, 16, None, 1, 1, 64, 16, 4, ctypes.c_float(0.5), ra.RACE_BF16, 16, 1 << 20, None]
+    bad = list(args)
+    bad[0] = None                       # q
+    assert f(*bad) == ra.RACE_ERR_INVALID_ARG
+    bad = list(args)
+    bad[4] = 8                          # state not 16-byte aligned
+    assert f(*bad) == ra.RACE_ERR_INVALID_ARG
+    bad = list(args)
+    bad[12] = ctypes.c_float(-0.5)      # tau
+    assert f(*bad) == ra.RACE_ERR_INVALID_ARG
+    bad = list(args)
+    bad[15] = 16                        # workspace too small
+    assert f(*bad) == ra.RACE_ERR_WORKSPACE
+    g = lib.race_attn_state
+    assert g(16, 16, 16, None, 1, 1, 128, 64, 16, 4, ctypes.c_float(0.5), ra.RACE_BF16, 16, 1 << 30, None) == \
+        ra.RACE_ERR_INVALID_ARG         # state
+    assert g(16, 16, 16, 16, 1, 1, 128, 64, 16, 4, ctypes.c_float(0.5), 7, 16, 1 << 30, None) == \
+        ra.RACE_ERR_INVALID_ARG         # dtype
+    assert g(16, 16, 16, 16, 1, 1, 128, 64, 16, 4, ctypes.c_float(0.5), ra.RACE_BF16, 16, 16, None) == \
+        ra.RACE_ERR_WORKSPACE
