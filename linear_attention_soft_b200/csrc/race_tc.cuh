@@ -91,9 +91,11 @@ struct BwdArgs {
 
 struct Ctl {
     uint64_t bar;    // MMA completion
+    uint64_t bar_b;  // MMA completion of the second thread group (segment aggregates)
     uint64_t ld[4];  // TMA / bulk load completion, one per buffer set
     uint32_t tmem;
     uint32_t abort;
+    uint32_t abort_b;  // the second thread group's (segment aggregates)
 };
 
 // ---- small helpers ---------------------------------------------------------------------
@@ -144,11 +146,12 @@ struct Loads {
 };
 __device__ __forceinline__ uint32_t load_parity(const Loads &ld, int b) { return ((ld.odd >> b) & 1u) ^ 1u; }
 
-// Arm barrier b for `bytes` of traffic (thread 0) and count the group; the TMA copies that
-// follow, issued by thread 0, complete it.
-__device__ __forceinline__ uint64_t *arm_load(Ctl *ctl, Loads &ld, int b, uint32_t bytes)
+// Arm barrier b for `bytes` of traffic (by the issuing thread, thread 0 unless given) and
+// count the group; the TMA copies that follow, issued by the same thread, complete it.
+__device__ __forceinline__ uint64_t *arm_load(Ctl *ctl, Loads &ld, int b, uint32_t bytes,
+                                              bool issuer = threadIdx.x == 0)
 {
-    if (threadIdx.x == 0) mbar_expect_tx(&ctl->ld[b], bytes);
+    if (issuer) mbar_expect_tx(&ctl->ld[b], bytes);
     ld.odd ^= 1u << b;
     ld.pend |= 1u << b;
     return &ctl->ld[b];
@@ -729,25 +732,26 @@ __device__ __forceinline__ void issue_state_update(uint32_t tm, uint32_t htop, u
 // Forward
 // ==========================================================================================
 
-namespace agg_smem {  // used by both segment aggregates (x rows and value rows double-buffered)
-constexpr uint32_t X0 = 0;
-constexpr uint32_t X1 = TILE;
-constexpr uint32_t PHI = 2 * TILE;          // Phi [128][256]
-constexpr uint32_t VA0 = PHI + 4 * TILE;    // value tile [128][80] (5 atoms)
-constexpr uint32_t VA1 = VA0 + 5 * VA128;
-constexpr uint32_t WHI = VA1 + 5 * VA128;
+namespace agg_smem {  // two thread groups, each with its own rows, features and value tile
+constexpr uint32_t X = 0;                    // k or q rows [128][64]
+constexpr uint32_t PHI = TILE;               // Phi [128][256]
+constexpr uint32_t VA = 5 * TILE;            // value tile [128][80] (5 atoms)
+constexpr uint32_t GROUP = VA + 5 * VA128;   // bytes per group (a multiple of 1024)
+constexpr uint32_t WHI = 2 * GROUP;
 constexpr uint32_t WLO = WHI + 8192;
-constexpr uint32_t RN = WLO + 8192;         // row norms [128]
-constexpr uint32_t ROWC = RN + 512;
-constexpr uint32_t ROWINV = ROWC + 512;
-constexpr uint32_t BAR = ROWINV + 512;
+constexpr uint32_t RN = WLO + 8192;          // row norms [2][128]
+constexpr uint32_t ROWC = RN + 1024;         // c_i [2][128]
+constexpr uint32_t ROWINV = ROWC + 1024;     // 1 / den_i [2][128]
+constexpr uint32_t BAR = ROWINV + 1024;
 constexpr uint32_t TOTAL = BAR + 64;
+constexpr uint32_t RED = GROUP;              // at the end: group 1's state, fp32 [256][80]
+static_assert(256 * 80 * 4 <= GROUP, "reduction buffer");
 }  // namespace agg_smem
-namespace agg_tmem {
+namespace agg_tmem {  // per group, at 256 * group
 constexpr uint32_t PROJ = 0;
 constexpr uint32_t HTOP = 64;
 constexpr uint32_t HBOT = 144;
-constexpr uint32_t NCOLS = 256;
+constexpr uint32_t NCOLS = 512;
 }  // namespace agg_tmem
 
 namespace fwd_smem {
@@ -779,8 +783,10 @@ __device__ __forceinline__ uint32_t kernel_setup(Ctl *ctl, uint32_t ncols, const
 {
     if (threadIdx.x == 0) {
         mbar_init(&ctl->bar, 1);
+        mbar_init(&ctl->bar_b, 1);
         for (int b = 0; b < 4; ++b) mbar_init(&ctl->ld[b], 1);
         ctl->abort = 0;
+        ctl->abort_b = 0;
     }
     if (threadIdx.x < 32) tmem_alloc(&ctl->tmem, ncols);
     if (whi) load_w_split(W, whi, wlo);
@@ -797,11 +803,20 @@ __device__ __forceinline__ void kernel_teardown(uint32_t tm, uint32_t ncols)
     if (threadIdx.x < 32) tmem_dealloc(tm, ncols);
 }
 
+// Barrier of one 256-thread group (named barrier 1 + g).
+__device__ __forceinline__ void group_sync(int g)
+{
+    asm volatile("bar.sync %0, 256;" ::"r"(1 + g) : "memory");
+}
+
 // ------------------------------------------------------------------------------------------
 // Segment totals.  MODE 0: H_seg = sum_j phi(k_j) [v_j, 1]^T (the bucket statistics A, B of
 // zh §2.2 over the segment).  MODE 1: G_seg = sum_i phi(q_i) dY_i^T = Phi_Q'^T [dO | c] with
 // Phi_Q' = Phi_Q / den (the backward's key-side statistics).   grid: nseg x BH
-// The next chunk's rows load while this chunk is processed (double-buffered tiles).
+// The CTA's two groups of 256 threads take the segment's chunks alternately, each with its
+// own tiles, TMEM accumulator and barriers, so that one group's MMA and load waits overlap
+// the other group's feature math; the two partial sums are added at the end.  Thread
+// (r, h) of a group owns token row r and quarters 2h, 2h+1 of the per-row work.
 // ------------------------------------------------------------------------------------------
 template <int MODE>
 __global__ void __launch_bounds__(NTH, 1) tc_agg(const __grid_constant__ BwdArgs a)
@@ -810,71 +825,157 @@ __global__ void __launch_bounds__(NTH, 1) tc_agg(const __grid_constant__ BwdArgs
     uint8_t *sm = aligned_base(smem_raw);
     using namespace agg_smem;
     Ctl *ctl = reinterpret_cast<Ctl *>(sm + BAR);
-    float *rn = reinterpret_cast<float *>(sm + RN);
-    float *rowc = reinterpret_cast<float *>(sm + ROWC), *rowinv = reinterpret_cast<float *>(sm + ROWINV);
     const int seg = blockIdx.x, bh = blockIdx.y;
-    const int r = threadIdx.x & 127, qd = threadIdx.x >> 7;
-    const uint32_t sb = smem_u32(sm);
+    const int g = threadIdx.x >> 8, gt = threadIdx.x & 255;
+    const int r = gt & 127, h = gt >> 7;
+    const bool leader = gt == 0;
+    float *rn = reinterpret_cast<float *>(sm + RN) + 128 * g;
+    float *rowc = reinterpret_cast<float *>(sm + ROWC) + 128 * g;
+    float *rowinv = reinterpret_cast<float *>(sm + ROWINV) + 128 * g;
+    const uint32_t sb = smem_u32(sm), gb = sb + (uint32_t)g * GROUP;
+    uint8_t *xg = sm + g * GROUP + X, *vag = sm + g * GROUP + VA;
+    uint64_t *mbar = g ? &ctl->bar_b : &ctl->bar;
+    // each group decides on its own flag, read only after its own barrier, so that all its
+    // threads leave the loop together; the CTA checks both flags after the loops
+    volatile uint32_t *gabort = g ? &ctl->abort_b : &ctl->abort;
     const __nv_bfloat16 *xsrc = MODE == 0 ? a.k : a.q;
     const __nv_bfloat16 *vsrc = MODE == 0 ? a.v : a.dout;
     const CUtensorMap *xmap = MODE == 0 ? &a.tm_k : &a.tm_q;
     const CUtensorMap *vmap = MODE == 0 ? &a.tm_v_va : &a.tm_do_va;
     const uint32_t tm = kernel_setup(ctl, agg_tmem::NCOLS, a.W, sm + WHI, sm + WLO);
-    zero_state40(tm, agg_tmem::HTOP, agg_tmem::HBOT, qd);
+    const uint32_t tg = tm + 256u * g;  // this group's TMEM columns
+#pragma unroll
+    for (int qq = 0; qq < 2; ++qq) zero_state40(tg, agg_tmem::HTOP, agg_tmem::HBOT, 2 * h + qq);
     int64_t t0, t1;
     seg_bounds(a.seg_len, a.N, seg, t0, t1);
     const int64_t base = (int64_t)bh * a.N;
     uint32_t phase = 0;
     bool ok = true;
-    Loads ld = {};
-    auto issue = [&](int64_t c, int b) {  // rows of chunk c into buffer set b
-        uint64_t *bar = arm_load(ctl, ld, b, 2u * TILE);
-        if (threadIdx.x == 0) {
-            tma_k128(sb + (b ? X1 : X0), xmap, c, bh, bar);
-            tma_va(sb + (b ? VA1 : VA0), vmap, c, bh, bar);
-        }
+    Loads ld = {};  // barriers 2g (rows) and 2g + 1 (values) of this group
+    auto load_x = [&](int64_t c) {
+        uint64_t *bar = arm_load(ctl, ld, 2 * g, TILE, leader);
+        if (leader) tma_k128(gb + X, xmap, c, bh, bar);
     };
-    if (t0 < t1) issue(t0, 0);
-    int buf = 0;
-    for (int64_t c0 = t0; c0 < t1 && ok; c0 += T, buf ^= 1) {
-        const int nv = (int)(t1 - c0 < T ? t1 - c0 : T);
-        uint8_t *x = sm + (buf ? X1 : X0), *va = sm + (buf ? VA1 : VA0);
-        if (!(ok = wait_loads(ctl, ld, 1u << buf))) break;
-        if (c0 + T < t1) {  // next chunk's rows into the other buffers (free: their MMAs completed)
-            issue(c0 + T, buf ^ 1);
-            prefetch_chunk(base + c0 + 2 * T, (int)(t1 - c0 - 2 * T < T ? t1 - c0 - 2 * T : T), xsrc, vsrc,
-                           nullptr, nullptr, nullptr, MODE ? a.den : nullptr, MODE ? a.cbuf : nullptr);
+    auto load_v = [&](int64_t c) {
+        uint64_t *bar = arm_load(ctl, ld, 2 * g + 1, TILE, leader);
+        if (leader) tma_va(gb + VA, vmap, c, bh, bar);
+    };
+    // bounded wait on this group's MMA barrier, then the group syncs
+    auto wait_group_mma = [&]() {
+        if (leader && *gabort == 0u && !mbar_wait(mbar, phase & 1u, WAIT_LIMIT_NS)) {
+            *gabort = 1u;
+            atomicExch(&g_tc_error, 1);
         }
-        if (qd == 0) rn[r] = row_norm(x, r);
-        if (MODE == 0 && qd == 1) write_col64(va, r, r < nv ? 1.f : 0.f);
-        if (MODE == 1 && qd == 2)
-            load_row_scalars(r, r < nv, a.cbuf + base + c0 + r, a.den + base + c0 + r, rowc, rowinv, va);
-        publish_smem();
-        if (threadIdx.x == 0) {
-            fence_after_sync();
-            issue_proj(tm + agg_tmem::PROJ, smem_u32(x), sb + WHI, sb + WLO);
-            mma_commit(&ctl->bar);
+        ++phase;
+        group_sync(g);
+        fence_after_sync();
+        return *gabort == 0u;
+    };
+    auto wait_group_load = [&](int b) {
+        bool fail = false;
+        if ((ld.pend >> b) & 1u) {
+            if (mbar_wait(&ctl->ld[b], load_parity(ld, b), WAIT_LIMIT_NS))
+                ld.pend &= ~(1u << b);
+            else
+                fail = true;
         }
-        if (!(ok = wait_mma(ctl, phase))) break;
-        {
-            float u[16], t[16];
-            proj_tanh(tm, agg_tmem::PROJ, qd, 1.f / fmaxf(rn[r], kNormEps), a.beta, u, t);
-            const float sc = r < nv ? (MODE == 0 ? 1.f : rowinv[r]) : 0.f;
-            write_features(t, r, qd, sc, sm + PHI);
+        if (fail) {
+            *gabort = 1u;
+            atomicExch(&g_tc_error, 1);
         }
-        publish_smem();
-        if (threadIdx.x == 0) {
-            fence_after_sync();
-            issue_state_update(tm, agg_tmem::HTOP, agg_tmem::HBOT, sb + PHI, smem_u32(va));
-            mma_commit(&ctl->bar);
-        }
-        ok = wait_mma(ctl, phase);
+        group_sync(g);
+        return *gabort == 0u;
+    };
+    auto publish_group = [&]() {
+        fence_smem_async();
+        fence_before_sync();
+        group_sync(g);
+    };
+    int64_t c0 = t0 + (int64_t)g * T;  // this group's chunks: every other one of the segment
+    if (c0 < t1) {
+        load_x(c0);
+        load_v(c0);
     }
-    drain_loads(ctl, ld);
-    if (ok) {
-        float hv[40];
-        read_state40(tm, agg_tmem::HTOP, agg_tmem::HBOT, qd, hv);
-        store_state40(hv, a.agg_out + ((int64_t)bh * a.nseg + seg) * MF * DS, 128 * (qd & 1) + r, qd);
+    for (; c0 < t1 && ok; c0 += 2 * T) {
+        const int nv = (int)(t1 - c0 < T ? t1 - c0 : T);
+        const int64_t cn = c0 + 2 * T;  // this group's next chunk
+        if (!(ok = wait_group_load(2 * g))) break;
+        if (h == 0) rn[r] = row_norm(xg, r);
+        if (MODE == 0 && h == 1) write_col64(vag, r, r < nv ? 1.f : 0.f);
+        if (MODE == 1 && h == 1)
+            load_row_scalars(r, r < nv, a.cbuf + base + c0 + r, a.den + base + c0 + r, rowc, rowinv, vag);
+        publish_group();
+        if (leader) {
+            fence_after_sync();
+            issue_proj(tg + agg_tmem::PROJ, gb + X, sb + WHI, sb + WLO);
+            mma_commit(mbar);
+        }
+        if (!(ok = wait_group_mma())) break;
+        if (cn < t1) {  // the rows are consumed: the next chunk's rows come in during the features
+            load_x(cn);
+            const int64_t cp = cn + 2 * T;  // and the one after towards L2
+            if (gt < 4 && cp < t1) {
+                const int n = (int)(t1 - cp < T ? t1 - cp : T);
+                if (gt == 0) prefetch_l2(xsrc + (base + cp) * DH, (uint32_t)n * DH * 2u);
+                if (gt == 1) prefetch_l2(vsrc + (base + cp) * DH, (uint32_t)n * DH * 2u);
+                if (MODE == 1 && gt >= 2) {  // den, c_i: 16-byte aligned bounds inside the range
+                    const float *f = (gt == 2 ? a.den : a.cbuf) + base + cp;
+                    const uintptr_t lo = ((uintptr_t)f + 15u) & ~(uintptr_t)15u, hi = (uintptr_t)(f + n) & ~(uintptr_t)15u;
+                    if (hi > lo) prefetch_l2((const void *)lo, (uint32_t)(hi - lo));
+                }
+            }
+        }
+        {
+            const float inv = 1.f / fmaxf(rn[r], kNormEps);
+            const float sc = r < nv ? (MODE == 0 ? 1.f : rowinv[r]) : 0.f;
+#pragma unroll 1
+            for (int qq = 0; qq < 2; ++qq) {
+                float u[16], t[16];
+                proj_tanh(tg, agg_tmem::PROJ, 2 * h + qq, inv, a.beta, u, t);
+                write_features(t, r, 2 * h + qq, sc, sm + g * GROUP + PHI);
+            }
+        }
+        if (!(ok = wait_group_load(2 * g + 1))) break;  // this chunk's values (group-synced)
+        publish_group();
+        if (leader) {
+            fence_after_sync();
+            issue_state_update(tg, agg_tmem::HTOP, agg_tmem::HBOT, gb + PHI, gb + VA);
+            mma_commit(mbar);
+        }
+        if (!(ok = wait_group_mma())) break;
+        if (cn < t1) load_v(cn);
+    }
+    drain_loads(ctl, ld);  // thread 0 only; group 1's loads are drained by its own leader
+    if (g == 1 && leader)
+        for (int b = 2; b < 4; ++b)
+            if ((ld.pend >> b) & 1u) mbar_wait(&ctl->ld[b], load_parity(ld, b), WAIT_LIMIT_NS);
+    __syncthreads();
+    if (ctl->abort == 0u && ctl->abort_b == 0u) {  // H = group 0's sum + group 1's sum
+        float *red = reinterpret_cast<float *>(sm + RED);
+        if (g == 1) {
+#pragma unroll 1
+            for (int qq = 0; qq < 2; ++qq) {
+                const int qd = 2 * h + qq;
+                float hv[40];
+                read_state40(tg, agg_tmem::HTOP, agg_tmem::HBOT, qd, hv);
+                float *dst = red + (128 * (qd & 1) + r) * 80 + 40 * (qd >> 1);
+#pragma unroll
+                for (int i = 0; i < 40; ++i) dst[i] = hv[i];
+            }
+        }
+        __syncthreads();
+        if (g == 0) {
+#pragma unroll 1
+            for (int qq = 0; qq < 2; ++qq) {
+                const int qd = 2 * h + qq;
+                float hv[40];
+                read_state40(tg, agg_tmem::HTOP, agg_tmem::HBOT, qd, hv);
+                const float *src = red + (128 * (qd & 1) + r) * 80 + 40 * (qd >> 1);
+#pragma unroll
+                for (int i = 0; i < 40; ++i) hv[i] += src[i];
+                store_state40(hv, a.agg_out + ((int64_t)bh * a.nseg + seg) * MF * DS, 128 * (qd & 1) + r, qd);
+            }
+        }
     }
     kernel_teardown(tm, agg_tmem::NCOLS);
 }
@@ -1390,8 +1491,10 @@ inline size_t smem_bytes(uint32_t total) { return total + 1024; }
 
 // TMA destinations: K128 tiles 1024-byte aligned (128-byte swizzle), value tiles 256-byte
 // aligned (32-byte swizzle); bulk copies 16-byte aligned.
-static_assert(agg_smem::X0 % 1024 == 0 && agg_smem::X1 % 1024 == 0, "agg tiles");
-static_assert(agg_smem::VA0 % 1024 == 0 && agg_smem::VA1 % 1024 == 0, "agg value tiles");
+static_assert(agg_smem::X % 1024 == 0 && agg_smem::PHI % 1024 == 0 && agg_smem::VA % 1024 == 0 &&
+                  agg_smem::GROUP % 1024 == 0,
+              "agg tiles");
+static_assert(sizeof(Ctl) <= 64, "control block");
 static_assert(fwd_smem::XQ % 1024 == 0 && fwd_smem::XK % 1024 == 0 && fwd_smem::VA % 1024 == 0, "fwd tiles");
 static_assert(bq_smem::XQ % 1024 == 0 && bq_smem::XK % 1024 == 0 && bq_smem::OT % 1024 == 0 &&
                   bq_smem::XQ2 % 1024 == 0 && bq_smem::VA % 1024 == 0 && bq_smem::DOV % 1024 == 0 &&
