@@ -192,6 +192,24 @@ __device__ __forceinline__ bool wait_loads(Ctl *ctl, Loads &ld, uint32_t mask)
     return *(volatile uint32_t *)&ctl->abort == 0u;
 }
 
+// Every thread waits (bounded) for the groups in flight on the barriers in `mask`, without a
+// barrier: each thread observes the completion itself.  A timeout marks the CTA as given up,
+// which the next synchronised wait reports.
+__device__ __forceinline__ void wait_loads_nosync(Ctl *ctl, Loads &ld, uint32_t mask)
+{
+    uint32_t todo = mask & ld.pend;
+    while (todo) {
+        const int b = __ffs(todo) - 1;
+        todo &= todo - 1u;
+        if (mbar_wait(&ctl->ld[b], load_parity(ld, b), WAIT_LIMIT_NS)) {
+            ld.pend &= ~(1u << b);
+        } else {
+            ctl->abort = 1u;
+            atomicExch(&g_tc_error, 1);
+        }
+    }
+}
+
 // Thread 0 alone waits for barrier b (data read by the tensor core only); false on timeout,
 // after marking the CTA as given up.
 __device__ __forceinline__ bool wait_load_t0(Ctl *ctl, Loads &ld, int b)
@@ -790,6 +808,7 @@ __device__ __forceinline__ uint32_t kernel_setup(Ctl *ctl, uint32_t ncols, const
     }
     if (threadIdx.x < 32) tmem_alloc(&ctl->tmem, ncols);
     if (whi) load_w_split(W, whi, wlo);
+    fence_smem_async();  // W is read by the tensor core
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
@@ -900,16 +919,16 @@ __global__ void __launch_bounds__(NTH, 1) tc_agg(const __grid_constant__ BwdArgs
         const int nv = (int)(t1 - c0 < T ? t1 - c0 : T);
         const int64_t cn = c0 + 2 * T;  // this group's next chunk
         if (!(ok = wait_group_load(2 * g))) break;
-        if (h == 0) rn[r] = row_norm(xg, r);
-        if (MODE == 0 && h == 1) write_col64(vag, r, r < nv ? 1.f : 0.f);
-        if (MODE == 1 && h == 1)
-            load_row_scalars(r, r < nv, a.cbuf + base + c0 + r, a.den + base + c0 + r, rowc, rowinv, vag);
-        publish_group();
-        if (leader) {
+        if (leader) {  // the projection runs while the row norms are formed
             fence_after_sync();
             issue_proj(tg + agg_tmem::PROJ, gb + X, sb + WHI, sb + WLO);
             mma_commit(mbar);
         }
+        if (h == 0) rn[r] = row_norm(xg, r);
+        if (MODE == 0 && h == 1) write_col64(vag, r, r < nv ? 1.f : 0.f);
+        if (MODE == 1 && h == 1)
+            load_row_scalars(r, r < nv, a.cbuf + base + c0 + r, a.den + base + c0 + r, rowc, rowinv, vag);
+        fence_smem_async();
         if (!(ok = wait_group_mma())) break;
         if (cn < t1) {  // the rows are consumed: the next chunk's rows come in during the features
             load_x(cn);
@@ -1024,16 +1043,16 @@ __global__ void __launch_bounds__(NTH, 1) tc_fwd_walk(const __grid_constant__ Ar
         const int nv = (int)(t1 - c0 < T ? t1 - c0 : T);
         const bool valid = r < nv;
         if (!(ok = wait_loads(ctl, ld, 1u))) break;
-        if (qd == 0) rn[r] = row_norm(sm + XQ, r);
-        if (causal && qd == 1) rn[128 + r] = row_norm(sm + XK, r);
-        if (causal && qd == 2) write_col64(sm + VA, r, valid ? 1.f : 0.f);
-        publish_smem();
-        if (threadIdx.x == 0) {
+        if (threadIdx.x == 0) {  // the projections run while the row norms are formed
             fence_after_sync();
             issue_proj(tm + fwd_tmem::PROJ, sb + XQ, sb + WHI, sb + WLO);
             if (causal) issue_proj(tm + fwd_tmem::PROJ + 64, sb + XK, sb + WHI, sb + WLO);
             mma_commit(&ctl->bar);
         }
+        if (qd == 0) rn[r] = row_norm(sm + XQ, r);
+        if (causal && qd == 1) rn[128 + r] = row_norm(sm + XK, r);
+        if (causal && qd == 2) write_col64(sm + VA, r, valid ? 1.f : 0.f);
+        fence_smem_async();
         if (!(ok = wait_mma(ctl, phase))) break;
         {
             float u[16], t[16];
@@ -1218,16 +1237,8 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_q_walk(const __grid_constant__ 
     for (int64_t c0 = t0; c0 < t1 && ok; c0 += T) {
         const int nv = (int)(t1 - c0 < T ? t1 - c0 : T);
         const bool valid = r < nv;
-        if (!(ok = wait_loads(ctl, ld, 7u))) break;
-        if (qd == 0) rn[r] = row_norm(sm + XQ, r);
-        if (causal && qd == 1) rn[128 + r] = row_norm(sm + XK, r);
-        if (qd == 2) {
-            row_scalars(r, sm + DOV, sm + OT, a.den + base + c0, nv, rowc, rowinv, nullptr);
-            if (valid) a.cbuf[base + c0 + r] = rowc[r];  // for the key-side passes
-        }
-        if (causal && qd == 3) write_col64(sm + VA, r, valid ? 1.f : 0.f);
-        publish_smem();
-        if (threadIdx.x == 0) {
+        if (!(ok = wait_loads(ctl, ld, 3u))) break;  // the kept q rows (barrier 2) are waited for at dq
+        if (threadIdx.x == 0) {  // the projections and P'' run while the row scalars are formed
             fence_after_sync();
             issue_proj(tm + bq_tmem::PROJ, sb + XQ, sb + WHI, sb + WLO);
             if (causal) {
@@ -1237,6 +1248,14 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_q_walk(const __grid_constant__ 
             }
             mma_commit(&ctl->bar);
         }
+        if (qd == 0) rn[r] = row_norm(sm + XQ, r);
+        if (causal && qd == 1) rn[128 + r] = row_norm(sm + XK, r);
+        if (qd == 2) {
+            row_scalars(r, sm + DOV, sm + OT, a.den + base + c0, nv, rowc, rowinv, nullptr);
+            if (valid) a.cbuf[base + c0 + r] = rowc[r];  // for the key-side passes
+        }
+        if (causal && qd == 3) write_col64(sm + VA, r, valid ? 1.f : 0.f);
+        fence_smem_async();
         if (!(ok = wait_mma(ctl, phase))) break;
         const float raw_q = rn[r];
         const float c_r = rowc[r], invden_r = rowinv[r];
@@ -1273,6 +1292,7 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_q_walk(const __grid_constant__ 
         }
         if (!(ok = wait_mma(ctl, phase))) break;
         if (c0 + T < t1) issue_q(c0 + T);  // dP~ is consumed; W stays for the next projection
+        wait_loads_nosync(ctl, ld, 4u);     // this chunk's kept q rows
         write_dx(tm, bq_tmem::DX, r, qd, valid, raw_q, sm + XQ2, nullptr, a.dq + (base + c0 + r) * DH, xch);
         __syncthreads();  // every quarter has read its q rows
         if (c0 + T < t1) issue_q2(c0 + T);
@@ -1377,23 +1397,27 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_kv_walk(const __grid_constant__
         const int64_t c0 = t0 + ci * T;
         const int nv = (int)(t1 - c0 < T ? t1 - c0 : T);
         const bool valid = r < nv;
-        if (!(ok = wait_loads(ctl, ld, 3u))) break;
+        if (!(ok = wait_loads(ctl, ld, 1u))) break;
+        if (threadIdx.x == 0) {  // key projection and V dO^T run while the row scalars are formed
+            fence_after_sync();
+            issue_proj(tm + bkv_tmem::PROJ + 64, sb + XK, sb + WHI, sb + WLO);
+            if (causal)  // V dO^T (needs no features)
+                issue_va_va(tm + bkv_tmem::PP, sb + VA, T, sb + DOC, T, 4, idesc_bf16(128, 128, 0, 0), false);
+        }
         if (qd == 0) rn[128 + r] = row_norm(sm + XK, r);
-        if (causal && qd == 1) rn[r] = row_norm(sm + XQ, r);
         if (causal && qd == 2)
             load_row_scalars(r, valid, a.cbuf + base + c0 + r, a.den + base + c0 + r, rowc, rowinv, sm + DOC);
         if (qd == 3) write_col64(sm + VA, r, valid ? 1.f : 0.f);
-        publish_smem();
-        if (threadIdx.x == 0) {
-            fence_after_sync();
-            issue_proj(tm + bkv_tmem::PROJ + 64, sb + XK, sb + WHI, sb + WLO);
-            if (causal) {
+        if (causal) {  // the q rows, loaded last, feed the query projection
+            if (!(ok = wait_loads(ctl, ld, 2u))) break;
+            if (threadIdx.x == 0) {
+                fence_after_sync();
                 issue_proj(tm + bkv_tmem::PROJ, sb + XQ, sb + WHI, sb + WLO);
-                // V dO^T (needs no features)
-                issue_va_va(tm + bkv_tmem::PP, sb + VA, T, sb + DOC, T, 4, idesc_bf16(128, 128, 0, 0), false);
             }
-            mma_commit(&ctl->bar);
+            if (qd == 1) rn[r] = row_norm(sm + XQ, r);
         }
+        if (threadIdx.x == 0) mma_commit(&ctl->bar);
+        fence_smem_async();
         if (!(ok = wait_mma(ctl, phase))) break;
         const float raw_k = rn[128 + r];
         float u[16], t[16];
