@@ -81,10 +81,10 @@ def kernel_work(name: str, w: race_inputs.Workload):
 # profiles/tc_kernels_n1m_ncu_full.md (N = 2^20; traffic grows in proportion to the tokens),
 # valid only for the kernel sources it was taken on.
 NCU_TRAFFIC = {
-    "src_sha1": {"race_tc.cuh": "853b03348070471dae58f8da60afe06a175ac3f1",
-                 "race_tc_util.cuh": "ec7c601f16c5892d0fd431308161cd00e13fa94c"},
-    "bytes_per_token": {"tc_agg_kv": 273.0, "tc_fwd_walk": 514.0, "tc_bwd_q_walk": 780.0,
-                        "tc_agg_qdy": 404.0, "tc_bwd_kv_walk": 894.0},
+    "src_sha1": {"race_tc.cuh": "aff23352c7244a6da8b6fcf923fbf4d532845a48",
+                 "race_tc_util.cuh": "03e99a6c246f135995cac3020fdc856ef380f9fc"},
+    "bytes_per_token": {"tc_agg_kv": 269.6, "tc_fwd_walk": 514.2, "tc_bwd_q_walk": 782.2,
+                        "tc_agg_qdy": 277.3, "tc_bwd_kv_walk": 767.6},
 }
 
 
