@@ -172,6 +172,66 @@ race_status_t race_attn_forward_noalloc(const void *q, const void *k, const void
                                         race_dtype_t dtype, race_stream_t stream);
 
 /*
+ * ---- one sequence sharded over several devices -------------------------------------------
+ * The statistics of Algorithm 2 (zh §2.3) are sums over tokens, so a sequence split into
+ * contiguous shards (one per device, shard s holding tokens [s*n, (s+1)*n) of every head)
+ * needs from the other shards only their totals: the forward of shard s starts its causal
+ * scan from the key-side statistics of shards 0..s-1, and the backward's key side starts
+ * from the query-side statistics G of shards s+1.. (bidirectional: every other shard's).
+ * Each pass is split in two around that exchange, which the caller performs (an all-gather
+ * over the shards, e.g. NCCL, then race_attn_shard_combine).  The two halves of a pass
+ * must get the same ctx and workspace; in between, the caller may use the stream freely.
+ * A single device is the one-shard case: begin + end with NULL init equals the one-call
+ * entry point.
+ */
+
+/* Forward, first half: the key-side segment statistics into ctx (or the workspace) and
+ * this shard's total, h_total = sum over its keys of phi(k)[v, 1]^T, fp32
+ * [B*H][L*2^P][d+1] (required).  Other arguments as race_attn_forward. */
+race_status_t race_attn_forward_begin(const void *k, const void *v, const float *W, float *ctx,
+                                      size_t ctx_bytes, float *h_total, int B, int H, int64_t N,
+                                      int d, int L, int P, float tau, int causal,
+                                      race_dtype_t dtype, void *workspace,
+                                      size_t workspace_bytes, race_stream_t stream);
+
+/* Forward, second half: the scan starts from h_init ([B*H][L*2^P][d+1] fp32: the keys of
+ * the shards before this one, causal; of every other shard, bidirectional; NULL = none),
+ * then out, den (and ctx, which then includes h_init) as race_attn_forward. */
+race_status_t race_attn_forward_end(const void *q, const void *k, const void *v, const float *W,
+                                    const float *h_init, void *out, float *den, float *ctx,
+                                    size_t ctx_bytes, int B, int H, int64_t N, int d, int L, int P,
+                                    float tau, int causal, race_dtype_t dtype, void *workspace,
+                                    size_t workspace_bytes, race_stream_t stream);
+
+/* Backward, first half: dq, and this shard's query-side total g_total = sum over its
+ * queries of phi(q_i) dY_i^T, dY_i = [dO_i, c_i] / den_i, fp32 [B*H][L*2^P][d+1]
+ * (required).  With ctx from race_attn_forward_end the key-side statistics (h_init
+ * included) are read from it; without, they are recomputed starting from h_init. */
+race_status_t race_attn_backward_begin(const void *q, const void *k, const void *v,
+                                       const float *W, const void *out, const float *den,
+                                       const void *dout, const float *ctx, size_t ctx_bytes,
+                                       const float *h_init, void *dq, float *g_total, int B,
+                                       int H, int64_t N, int d, int L, int P, float tau,
+                                       int causal, race_dtype_t dtype, void *workspace,
+                                       size_t workspace_bytes, race_stream_t stream);
+
+/* Backward, second half: dk, dv with the key side's suffix statistics starting from g_init
+ * (the queries of the shards after this one, causal; of every other shard, bidirectional;
+ * NULL = none).  workspace: the one race_attn_backward_begin used, unchanged since. */
+race_status_t race_attn_backward_end(const void *q, const void *k, const void *v, const float *W,
+                                     const void *out, const float *den, const void *dout,
+                                     const float *g_init, void *dk, void *dv, int B, int H,
+                                     int64_t N, int d, int L, int P, float tau, int causal,
+                                     race_dtype_t dtype, void *workspace,
+                                     size_t workspace_bytes, race_stream_t stream);
+
+/* out[e] = sum over the selected shards s of gathered[s][e], in shard order: which = 0 the
+ * shards before `shard`, 1 those after it, 2 every other shard.  gathered: device fp32
+ * [nshards][elems] (the shards' totals side by side, as an all-gather leaves them). */
+race_status_t race_attn_shard_combine(const float *gathered, int nshards, int shard, int which,
+                                      int64_t elems, float *out, race_stream_t stream);
+
+/*
  * Bucket statistics of every key of each head: H[m][c] = sum_j phi(k_j)[m] [v_j, 1][c],
  * m = l * 2^P + r, i.e. B_l (columns 0..d-1) and A_l (column d) of zh §2.2 for all tables in
  * one array -- the running statistics of Algorithm 2 (zh §2.3) after the last token, which

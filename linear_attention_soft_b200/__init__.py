@@ -26,6 +26,8 @@ __all__ = [
     "race_attn_profile_read", "race_attn_forward_noalloc", "RACE_NOALLOC_SCRATCH_BYTES",
     "race_attn_device_error", "race_attn_selftest_wait_timeout", "race_attn_state",
     "race_attn_decode_workspace_size", "race_attn_decode_step", "state", "decode_step",
+    "race_attn_forward_begin", "race_attn_forward_end", "race_attn_backward_begin",
+    "race_attn_backward_end", "race_attn_shard_combine",
 ]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -95,6 +97,21 @@ def load_library():
     lib.race_attn_decode_step.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int,
                                           _int, ctypes.c_float, _int, _vp, _sz, _vp]
     lib.race_attn_decode_step.restype = _int
+    lib.race_attn_forward_begin.argtypes = [_vp, _vp, _vp, _vp, _sz, _vp, _int, _int, _i64, _int, _int, _int,
+                                            ctypes.c_float, _int, _int, _vp, _sz, _vp]
+    lib.race_attn_forward_begin.restype = _int
+    lib.race_attn_forward_end.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _int, _int, _i64, _int,
+                                          _int, _int, ctypes.c_float, _int, _int, _vp, _sz, _vp]
+    lib.race_attn_forward_end.restype = _int
+    lib.race_attn_backward_begin.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp, _vp, _int,
+                                             _int, _i64, _int, _int, _int, ctypes.c_float, _int, _int, _vp,
+                                             _sz, _vp]
+    lib.race_attn_backward_begin.restype = _int
+    lib.race_attn_backward_end.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _i64,
+                                           _int, _int, _int, ctypes.c_float, _int, _int, _vp, _sz, _vp]
+    lib.race_attn_backward_end.restype = _int
+    lib.race_attn_shard_combine.argtypes = [_vp, _int, _int, _int, _i64, _vp, _vp]
+    lib.race_attn_shard_combine.restype = _int
     lib.race_attn_profile_enable.argtypes = [_int]
     lib.race_attn_profile_enable.restype = None
     lib.race_attn_profile_reset.argtypes = []
@@ -228,6 +245,57 @@ def race_attn_decode_step(q, k, v, W, state, out, den, tau: float, workspace, st
         _ptr(q), _ptr(k), _ptr(v), _ptr(W), _ptr(state), _ptr(out), _ptr(den), B, H, d, L, P,
         float(tau), _dtype_code(q), _ptr(workspace), _nbytes(workspace), _stream(stream)),
         "race_attn_decode_step")
+
+
+def race_attn_forward_begin(k, v, W, ctx, h_total, tau: float, causal: bool, workspace, stream=None) -> None:
+    """C ABI forward, first half: h_total [B*H, L*2^P, d+1] fp32 receives this shard's
+    key-side total."""
+    B, H, N, d, L, P = _dims(k, W)
+    _check(load_library().race_attn_forward_begin(
+        _ptr(k), _ptr(v), _ptr(W), _ptr(ctx), _nbytes(ctx), _ptr(h_total), B, H, N, d, L, P, float(tau),
+        int(bool(causal)), _dtype_code(k), _ptr(workspace), _nbytes(workspace), _stream(stream)),
+        "race_attn_forward_begin")
+
+
+def race_attn_forward_end(q, k, v, W, h_init, out, den, ctx, tau: float, causal: bool, workspace,
+                          stream=None) -> None:
+    """C ABI forward, second half, from the other shards' key statistics h_init (or None)."""
+    B, H, N, d, L, P = _dims(q, W)
+    _check(load_library().race_attn_forward_end(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(W), _ptr(h_init), _ptr(out), _ptr(den), _ptr(ctx), _nbytes(ctx),
+        B, H, N, d, L, P, float(tau), int(bool(causal)), _dtype_code(q), _ptr(workspace), _nbytes(workspace),
+        _stream(stream)), "race_attn_forward_end")
+
+
+def race_attn_backward_begin(q, k, v, W, out, den, dout, ctx, h_init, dq, g_total, tau: float, causal: bool,
+                             workspace, stream=None) -> None:
+    """C ABI backward, first half: dq and this shard's query-side total g_total."""
+    B, H, N, d, L, P = _dims(q, W)
+    _check(load_library().race_attn_backward_begin(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(W), _ptr(out), _ptr(den), _ptr(dout), _ptr(ctx), _nbytes(ctx),
+        _ptr(h_init), _ptr(dq), _ptr(g_total), B, H, N, d, L, P, float(tau), int(bool(causal)),
+        _dtype_code(q), _ptr(workspace), _nbytes(workspace), _stream(stream)), "race_attn_backward_begin")
+
+
+def race_attn_backward_end(q, k, v, W, out, den, dout, g_init, dk, dv, tau: float, causal: bool, workspace,
+                           stream=None) -> None:
+    """C ABI backward, second half: dk, dv from the other shards' query statistics g_init."""
+    B, H, N, d, L, P = _dims(q, W)
+    _check(load_library().race_attn_backward_end(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(W), _ptr(out), _ptr(den), _ptr(dout), _ptr(g_init), _ptr(dk),
+        _ptr(dv), B, H, N, d, L, P, float(tau), int(bool(causal)), _dtype_code(q), _ptr(workspace),
+        _nbytes(workspace), _stream(stream)), "race_attn_backward_end")
+
+
+def race_attn_shard_combine(gathered, shard: int, which: int, out, stream=None) -> None:
+    """C ABI: out = sum of the selected shards of gathered [nshards, ...] in shard order
+    (which: 0 before `shard`, 1 after it, 2 every other)."""
+    n = gathered.shape[0]
+    elems = gathered.numel() // max(n, 1)
+    if out.numel() != elems:
+        raise ValueError("out holds one shard's elements")
+    _check(load_library().race_attn_shard_combine(_ptr(gathered), n, int(shard), int(which), elems, _ptr(out),
+                                                  _stream(stream)), "race_attn_shard_combine")
 
 
 def race_attn_device_error(stream=None) -> int:

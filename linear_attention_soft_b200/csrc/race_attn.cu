@@ -227,30 +227,51 @@ cudaError_t launch(Kern kernel, dim3 grid, int cluster_x, size_t smem, cudaStrea
     return cudaLaunchKernelEx(&cfg, kernel, a);
 }
 
-cudaError_t launch_scan(float *buf, const Plan &p, int mode, cudaStream_t st)
+cudaError_t launch_scan(float *buf, const Plan &p, int mode, cudaStream_t st, const float *init = nullptr,
+                        float *total_out = nullptr)
 {
     const int64_t MD = (int64_t)p.M * p.D;
     dim3 grid((unsigned)((MD + gk::NT - 1) / gk::NT), (unsigned)p.BH);
     return timed("segment_scan", st, [&] {
-        gk::race_scan<<<grid, gk::NT, 0, st>>>(buf, p.nseg, MD, mode);
+        gk::race_scan<<<grid, gk::NT, 0, st>>>(buf, p.nseg, MD, mode, init, total_out);
         return cudaGetLastError();
     });
 }
 
+// A pass split in two for a sequence sharded over several devices: BEGIN stops once the
+// local statistics the other shards need are known (h_total: key side, forward; g_total:
+// query side, backward), END continues from the other shards' statistics (h_init: the keys
+// before this shard -- every other shard's when bidirectional -- and g_init: the queries
+// after it).  ALL runs both halves with no other shards.
+enum Stage { STAGE_ALL = 0, STAGE_BEGIN = 1, STAGE_END = 2 };
+struct Shard {
+    int stage = STAGE_ALL;
+    const float *h_init = nullptr;
+    float *h_total = nullptr;
+    const float *g_init = nullptr;
+    float *g_total = nullptr;
+};
+
 // ---- the general path (every shape and dtype) ----------------------------------------
 
 template <typename DT, int T>
-cudaError_t generic_forward(const Plan &p, Args a, float *states, int causal, cudaStream_t st)
+cudaError_t generic_forward(const Plan &p, Args a, float *states, int causal, cudaStream_t st, const Shard &sh)
 {
     const size_t smem = gk::Smem(T, p.d, p.P).total * sizeof(float);
     const dim3 grid((unsigned)p.G, (unsigned)p.nseg, (unsigned)p.BH);
     a.causal = causal;
     a.agg_out = states;
-    cudaError_t e = timed("generic_agg_kv", st, [&] {
-        return launch(gk::race_agg<DT, T, gk::AGG_KV>, grid, 1, smem, st, a);
-    });
-    if (e != cudaSuccess) return e;
-    e = launch_scan(states, p, causal ? gk::SCAN_EXCL_PREFIX : gk::SCAN_TOTAL, st);
+    cudaError_t e;
+    if (sh.stage != STAGE_END) {
+        e = timed("generic_agg_kv", st, [&] {
+            return launch(gk::race_agg<DT, T, gk::AGG_KV>, grid, 1, smem, st, a);
+        });
+        if (e != cudaSuccess) return e;
+        if (sh.h_total && (e = launch_scan(states, p, gk::SCAN_TOTAL_ONLY, st, nullptr, sh.h_total)) != cudaSuccess)
+            return e;
+        if (sh.stage == STAGE_BEGIN) return cudaSuccess;
+    }
+    e = launch_scan(states, p, causal ? gk::SCAN_EXCL_PREFIX : gk::SCAN_TOTAL, st, sh.h_init);
     if (e != cudaSuccess) return e;
     a.state = states;
     a.state_seg_stride = causal ? (int64_t)p.M * p.D : 0;
@@ -260,35 +281,42 @@ cudaError_t generic_forward(const Plan &p, Args a, float *states, int causal, cu
 
 template <typename DT, int T>
 cudaError_t generic_backward(const Plan &p, Args a, const float *hstates, bool have_ctx,
-                             float *hbuf, float *gbuf, int causal, cudaStream_t st)
+                             float *hbuf, float *gbuf, int causal, cudaStream_t st, const Shard &sh)
 {
     const size_t smem = gk::Smem(T, p.d, p.P).total * sizeof(float);
     const dim3 grid((unsigned)p.G, (unsigned)p.nseg, (unsigned)p.BH);
+    const int64_t stride = causal ? (int64_t)p.M * p.D : 0;
     a.causal = causal;
     cudaError_t e;
-    if (!have_ctx) {
-        a.agg_out = hbuf;
-        e = timed("generic_agg_kv", st, [&] {
-            return launch(gk::race_agg<DT, T, gk::AGG_KV>, grid, 1, smem, st, a);
+    if (sh.stage != STAGE_END) {
+        if (!have_ctx) {  // key-side prefix statistics, as the forward computes them
+            a.agg_out = hbuf;
+            e = timed("generic_agg_kv", st, [&] {
+                return launch(gk::race_agg<DT, T, gk::AGG_KV>, grid, 1, smem, st, a);
+            });
+            if (e != cudaSuccess) return e;
+            e = launch_scan(hbuf, p, causal ? gk::SCAN_EXCL_PREFIX : gk::SCAN_TOTAL, st, sh.h_init);
+            if (e != cudaSuccess) return e;
+            hstates = hbuf;
+        }
+        a.state = hstates;
+        a.state_seg_stride = stride;
+        e = timed("generic_bwd_q_walk", st,
+                  [&] { return launch(gk::race_bwd_q_walk<DT, T>, grid, p.G, smem, st, a); });
+        if (e != cudaSuccess) return e;
+        a.agg_out = gbuf;
+        e = timed("generic_agg_qdy", st, [&] {
+            return launch(gk::race_agg<DT, T, gk::AGG_QDY>, grid, 1, smem, st, a);
         });
         if (e != cudaSuccess) return e;
-        e = launch_scan(hbuf, p, causal ? gk::SCAN_EXCL_PREFIX : gk::SCAN_TOTAL, st);
-        if (e != cudaSuccess) return e;
-        hstates = hbuf;
+        if (sh.g_total && (e = launch_scan(gbuf, p, gk::SCAN_TOTAL_ONLY, st, nullptr, sh.g_total)) != cudaSuccess)
+            return e;
+        if (sh.stage == STAGE_BEGIN) return cudaSuccess;
     }
-    a.state = hstates;
-    a.state_seg_stride = causal ? (int64_t)p.M * p.D : 0;
-    e = timed("generic_bwd_q_walk", st,
-              [&] { return launch(gk::race_bwd_q_walk<DT, T>, grid, p.G, smem, st, a); });
-    if (e != cudaSuccess) return e;
-    a.agg_out = gbuf;
-    e = timed("generic_agg_qdy", st, [&] {
-        return launch(gk::race_agg<DT, T, gk::AGG_QDY>, grid, 1, smem, st, a);
-    });
-    if (e != cudaSuccess) return e;
-    e = launch_scan(gbuf, p, causal ? gk::SCAN_EXCL_SUFFIX : gk::SCAN_TOTAL, st);
+    e = launch_scan(gbuf, p, causal ? gk::SCAN_EXCL_SUFFIX : gk::SCAN_TOTAL, st, sh.g_init);
     if (e != cudaSuccess) return e;
     a.state = gbuf;
+    a.state_seg_stride = stride;
     return timed("generic_bwd_kv_walk", st,
                  [&] { return launch(gk::race_bwd_kv_walk<DT, T>, grid, p.G, smem, st, a); });
 }
@@ -349,15 +377,20 @@ cudaError_t tc_args(race::tc::BwdArgs &a, const Plan &p, const void *q, const vo
 }
 
 cudaError_t tc_forward(const Plan &p, const void *q, const void *k, const void *v, const float *W,
-                       void *out, float *den, float *states, float tau, int causal, cudaStream_t st)
+                       void *out, float *den, float *states, float tau, int causal, cudaStream_t st, const Shard &sh)
 {
     namespace tc = race::tc;
     tc::BwdArgs ka;
     cudaError_t e = tc_args(ka, p, q, k, v, W, nullptr, nullptr, nullptr, tau, causal);
     if (e != cudaSuccess) return e;
-    e = tc_segment_totals(p, ka, 0, states, st);
-    if (e != cudaSuccess) return e;
-    e = launch_scan(states, p, causal ? gk::SCAN_EXCL_PREFIX : gk::SCAN_TOTAL, st);
+    if (sh.stage != STAGE_END) {
+        e = tc_segment_totals(p, ka, 0, states, st);
+        if (e != cudaSuccess) return e;
+        if (sh.h_total && (e = launch_scan(states, p, gk::SCAN_TOTAL_ONLY, st, nullptr, sh.h_total)) != cudaSuccess)
+            return e;
+        if (sh.stage == STAGE_BEGIN) return cudaSuccess;
+    }
+    e = launch_scan(states, p, causal ? gk::SCAN_EXCL_PREFIX : gk::SCAN_TOTAL, st, sh.h_init);
     if (e != cudaSuccess) return e;
     tc::Args a;
     std::memset(&a, 0, sizeof(a));
@@ -389,7 +422,7 @@ cudaError_t tc_forward(const Plan &p, const void *q, const void *k, const void *
 cudaError_t tc_backward(const Plan &p, const void *q, const void *k, const void *v, const float *W,
                         const void *out, const float *den, const void *dout, const float *ctx, float *hbuf,
                         float *gbuf, uint8_t *wimg, float *cbuf, void *dq, void *dk, void *dv, float tau,
-                        int causal, cudaStream_t st)
+                        int causal, cudaStream_t st, const Shard &sh)
 {
     namespace tc = race::tc;
     const dim3 grid((unsigned)p.nseg, (unsigned)p.BH);
@@ -406,29 +439,37 @@ cudaError_t tc_backward(const Plan &p, const void *q, const void *k, const void 
         return cudaGetLastError();
     });
     if (e != cudaSuccess) return e;
-    const float *hstates = ctx;
-    if (!hstates) {  // key-side prefix statistics, as the forward computes them
-        if ((e = tc_segment_totals(p, a, 0, hbuf, st)) != cudaSuccess) return e;
-        if ((e = launch_scan(hbuf, p, causal ? gk::SCAN_EXCL_PREFIX : gk::SCAN_TOTAL, st)) != cudaSuccess)
-            return e;
-        hstates = hbuf;
-    }
     const int64_t stride = causal ? (int64_t)p.M * p.D : 0;
     const size_t sm_q = tc::smem_bytes(tc::bq_smem::TOTAL);
     const size_t sm_kv = tc::smem_bytes(tc::bkv_smem::TOTAL);
     if ((e = tc_prepare(tc::tc_bwd_q_walk, sm_q)) != cudaSuccess ||
         (e = tc_prepare(tc::tc_bwd_kv_walk, sm_kv)) != cudaSuccess)
         return e;
-    a.state = hstates;
-    a.state_seg_stride = stride;
-    e = timed("tc_bwd_q_walk", st, [&] {
-        tc::tc_bwd_q_walk<<<grid, tc::NTH, sm_q, st>>>(a);
-        return cudaGetLastError();
-    });
-    if (e != cudaSuccess) return e;
-    if ((e = tc_segment_totals(p, a, 1, gbuf, st)) != cudaSuccess) return e;
-    if ((e = launch_scan(gbuf, p, causal ? gk::SCAN_EXCL_SUFFIX : gk::SCAN_TOTAL, st)) != cudaSuccess) return e;
+    if (sh.stage != STAGE_END) {
+        const float *hstates = ctx;
+        if (!hstates) {  // key-side prefix statistics, as the forward computes them
+            if ((e = tc_segment_totals(p, a, 0, hbuf, st)) != cudaSuccess) return e;
+            if ((e = launch_scan(hbuf, p, causal ? gk::SCAN_EXCL_PREFIX : gk::SCAN_TOTAL, st, sh.h_init)) !=
+                cudaSuccess)
+                return e;
+            hstates = hbuf;
+        }
+        a.state = hstates;
+        a.state_seg_stride = stride;
+        e = timed("tc_bwd_q_walk", st, [&] {
+            tc::tc_bwd_q_walk<<<grid, tc::NTH, sm_q, st>>>(a);
+            return cudaGetLastError();
+        });
+        if (e != cudaSuccess) return e;
+        if ((e = tc_segment_totals(p, a, 1, gbuf, st)) != cudaSuccess) return e;
+        if (sh.g_total && (e = launch_scan(gbuf, p, gk::SCAN_TOTAL_ONLY, st, nullptr, sh.g_total)) != cudaSuccess)
+            return e;
+        if (sh.stage == STAGE_BEGIN) return cudaSuccess;
+    }
+    if ((e = launch_scan(gbuf, p, causal ? gk::SCAN_EXCL_SUFFIX : gk::SCAN_TOTAL, st, sh.g_init)) != cudaSuccess)
+        return e;
     a.state = gbuf;
+    a.state_seg_stride = stride;
     return timed("tc_bwd_kv_walk", st, [&] {
         tc::tc_bwd_kv_walk<<<grid, tc::NTH, sm_kv, st>>>(a);
         return cudaGetLastError();
@@ -436,19 +477,19 @@ cudaError_t tc_backward(const Plan &p, const void *q, const void *k, const void 
 }
 
 template <typename DT>
-cudaError_t dispatch_forward(const Plan &p, const Args &a, float *states, int causal,
-                             cudaStream_t st)
+cudaError_t dispatch_forward(const Plan &p, const Args &a, float *states, int causal, cudaStream_t st,
+                             const Shard &sh)
 {
-    if (p.d <= 64) return generic_forward<DT, 32>(p, a, states, causal, st);
-    return generic_forward<DT, 16>(p, a, states, causal, st);
+    if (p.d <= 64) return generic_forward<DT, 32>(p, a, states, causal, st, sh);
+    return generic_forward<DT, 16>(p, a, states, causal, st, sh);
 }
 
 template <typename DT>
 cudaError_t dispatch_backward(const Plan &p, const Args &a, const float *ctx, float *hbuf,
-                              float *gbuf, int causal, cudaStream_t st)
+                              float *gbuf, int causal, cudaStream_t st, const Shard &sh)
 {
-    if (p.d <= 64) return generic_backward<DT, 32>(p, a, ctx, ctx != nullptr, hbuf, gbuf, causal, st);
-    return generic_backward<DT, 16>(p, a, ctx, ctx != nullptr, hbuf, gbuf, causal, st);
+    if (p.d <= 64) return generic_backward<DT, 32>(p, a, ctx, ctx != nullptr, hbuf, gbuf, causal, st, sh);
+    return generic_backward<DT, 16>(p, a, ctx, ctx != nullptr, hbuf, gbuf, causal, st, sh);
 }
 
 // Bucket statistics of every key of each head (Algorithm 1's A and B): segment totals of the
@@ -528,25 +569,37 @@ race_status_t race_attn_ctx_size(int B, int H, int64_t N, int d, int L, int P, i
     return RACE_OK;
 }
 
-race_status_t race_attn_forward(const void *q, const void *k, const void *v, const float *W,
-                                void *out, float *den, float *ctx, size_t ctx_bytes, int B,
-                                int H, int64_t N, int d, int L, int P, float tau, int causal,
-                                race_dtype_t dtype, void *workspace, size_t workspace_bytes,
-                                race_stream_t stream)
+}  // extern "C"
+
+namespace {
+
+race_status_t forward_impl(const void *q, const void *k, const void *v, const float *W, void *out, float *den,
+                           float *ctx, size_t ctx_bytes, int B, int H, int64_t N, int d, int L, int P, float tau,
+                           int causal, race_dtype_t dtype, void *workspace, size_t workspace_bytes,
+                           race_stream_t stream, const Shard &sh)
 {
     if (dtype != RACE_F32 && dtype != RACE_BF16) return RACE_ERR_INVALID_ARG;
     if (!(tau >= 0.f) || !std::isfinite(tau)) return RACE_ERR_INVALID_ARG;
     race_status_t s = check_sizes(B, H, N, d, L, P);
     if (s != RACE_OK) return s;
-    if (N == 0) return RACE_OK;
-    if (!q || !k || !v || !W || !out || !workspace) return RACE_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(W) || !aligned16(out) ||
-        !aligned16(workspace) || (den && !aligned16(den)) || (ctx && !aligned16(ctx)))
+    if (N == 0) {  // an empty shard contributes zero statistics
+        if (sh.h_total)
+            return cudaMemsetAsync(sh.h_total, 0, (size_t)B * H * (L << P) * (d + 1) * sizeof(float),
+                                   (cudaStream_t)stream) == cudaSuccess ? RACE_OK : RACE_ERR_CUDA;
+        return RACE_OK;
+    }
+    const bool walk = sh.stage != STAGE_BEGIN;
+    if (!k || !v || !W || !workspace || (walk && (!q || !out)) || (sh.stage == STAGE_BEGIN && !sh.h_total))
+        return RACE_ERR_INVALID_ARG;
+    if (!aligned16(k) || !aligned16(v) || !aligned16(W) || !aligned16(workspace) || (q && !aligned16(q)) ||
+        (out && !aligned16(out)) || (den && !aligned16(den)) || (ctx && !aligned16(ctx)) ||
+        (sh.h_init && !aligned16(sh.h_init)) || (sh.h_total && !aligned16(sh.h_total)))
         return RACE_ERR_INVALID_ARG;
     const Plan p = make_plan(B, H, N, d, L, P);
     const size_t need = p.state_elems * sizeof(float);
     if (workspace_bytes < need) return RACE_ERR_WORKSPACE;
     if (ctx && ctx_bytes < need) return RACE_ERR_WORKSPACE;
+    if (!q) q = k;  // the first half reads keys and values only
     Args a = base_args(p, W, tau);
     a.q = q;
     a.k = k;
@@ -557,33 +610,41 @@ race_status_t race_attn_forward(const void *q, const void *k, const void *v, con
     cudaStream_t st = (cudaStream_t)stream;
     cudaError_t e;
     if (race::tc::fast_path_ok(dtype, d, L, P, tau, N) && g_tc_forward)
-        e = tc_forward(p, q, k, v, W, out, den, states, tau, causal, st);
+        e = tc_forward(p, q, k, v, W, out, den, states, tau, causal, st, sh);
     else if (dtype == RACE_F32)
-        e = dispatch_forward<float>(p, a, states, causal, st);
+        e = dispatch_forward<float>(p, a, states, causal, st, sh);
     else
-        e = dispatch_forward<__nv_bfloat16>(p, a, states, causal, st);
+        e = dispatch_forward<__nv_bfloat16>(p, a, states, causal, st, sh);
     return e == cudaSuccess ? RACE_OK : RACE_ERR_CUDA;
 }
 
-race_status_t race_attn_backward(const void *q, const void *k, const void *v, const float *W,
-                                 const void *out, const float *den, const void *dout,
-                                 const float *ctx, size_t ctx_bytes, void *dq, void *dk,
-                                 void *dv, int B, int H, int64_t N, int d, int L, int P,
-                                 float tau, int causal, race_dtype_t dtype, void *workspace,
-                                 size_t workspace_bytes, race_stream_t stream)
+race_status_t backward_impl(const void *q, const void *k, const void *v, const float *W, const void *out,
+                            const float *den, const void *dout, const float *ctx, size_t ctx_bytes, void *dq,
+                            void *dk, void *dv, int B, int H, int64_t N, int d, int L, int P, float tau, int causal,
+                            race_dtype_t dtype, void *workspace, size_t workspace_bytes, race_stream_t stream,
+                            const Shard &sh)
 {
     if (dtype != RACE_F32 && dtype != RACE_BF16) return RACE_ERR_INVALID_ARG;
     if (!(tau >= 0.f) || !std::isfinite(tau)) return RACE_ERR_INVALID_ARG;
     race_status_t s = check_sizes(B, H, N, d, L, P);
     if (s != RACE_OK) return s;
     if (tau == 0.f) return RACE_ERR_UNSUPPORTED;
-    if (N == 0) return RACE_OK;
-    if (!q || !k || !v || !W || !out || !den || !dout || !dq || !dk || !dv || !workspace)
+    if (N == 0) {  // an empty shard contributes zero statistics
+        if (sh.g_total)
+            return cudaMemsetAsync(sh.g_total, 0, (size_t)B * H * (L << P) * (d + 1) * sizeof(float),
+                                   (cudaStream_t)stream) == cudaSuccess ? RACE_OK : RACE_ERR_CUDA;
+        return RACE_OK;
+    }
+    const bool first = sh.stage != STAGE_END, second = sh.stage != STAGE_BEGIN;
+    if (!q || !k || !v || !W || !out || !den || !dout || !workspace || (first && !dq) || (second && (!dk || !dv)) ||
+        (sh.stage == STAGE_BEGIN && !sh.g_total))
         return RACE_ERR_INVALID_ARG;
-    const void *ptrs[] = {q, k, v, W, out, den, dout, dq, dk, dv, workspace};
+    const void *ptrs[] = {q, k, v, W, out, den, dout, workspace};
     for (const void *ptr : ptrs)
         if (!aligned16(ptr)) return RACE_ERR_INVALID_ARG;
-    if (ctx && !aligned16(ctx)) return RACE_ERR_INVALID_ARG;
+    const void *opt[] = {ctx, dq, dk, dv, sh.h_init, sh.g_init, sh.g_total};
+    for (const void *ptr : opt)
+        if (ptr && !aligned16(ptr)) return RACE_ERR_INVALID_ARG;
     const Plan p = make_plan(B, H, N, d, L, P);
     const size_t one = p.state_elems * sizeof(float);
     if (workspace_bytes < backward_workspace_bytes(p)) return RACE_ERR_WORKSPACE;
@@ -605,11 +666,105 @@ race_status_t race_attn_backward(const void *q, const void *k, const void *v, co
     cudaStream_t st = (cudaStream_t)stream;
     cudaError_t e;
     if (race::tc::fast_path_ok(dtype, d, L, P, tau, N) && g_tc_backward)
-        e = tc_backward(p, q, k, v, W, out, den, dout, ctx, hbuf, gbuf, wimg, cbuf, dq, dk, dv, tau, causal, st);
+        e = tc_backward(p, q, k, v, W, out, den, dout, ctx, hbuf, gbuf, wimg, cbuf, dq, dk, dv, tau, causal, st,
+                        sh);
     else if (dtype == RACE_F32)
-        e = dispatch_backward<float>(p, a, ctx, hbuf, gbuf, causal, st);
+        e = dispatch_backward<float>(p, a, ctx, hbuf, gbuf, causal, st, sh);
     else
-        e = dispatch_backward<__nv_bfloat16>(p, a, ctx, hbuf, gbuf, causal, st);
+        e = dispatch_backward<__nv_bfloat16>(p, a, ctx, hbuf, gbuf, causal, st, sh);
+    return e == cudaSuccess ? RACE_OK : RACE_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+race_status_t race_attn_forward(const void *q, const void *k, const void *v, const float *W,
+                                void *out, float *den, float *ctx, size_t ctx_bytes, int B,
+                                int H, int64_t N, int d, int L, int P, float tau, int causal,
+                                race_dtype_t dtype, void *workspace, size_t workspace_bytes,
+                                race_stream_t stream)
+{
+    return forward_impl(q, k, v, W, out, den, ctx, ctx_bytes, B, H, N, d, L, P, tau, causal, dtype, workspace,
+                        workspace_bytes, stream, Shard());
+}
+
+race_status_t race_attn_backward(const void *q, const void *k, const void *v, const float *W,
+                                 const void *out, const float *den, const void *dout,
+                                 const float *ctx, size_t ctx_bytes, void *dq, void *dk,
+                                 void *dv, int B, int H, int64_t N, int d, int L, int P,
+                                 float tau, int causal, race_dtype_t dtype, void *workspace,
+                                 size_t workspace_bytes, race_stream_t stream)
+{
+    return backward_impl(q, k, v, W, out, den, dout, ctx, ctx_bytes, dq, dk, dv, B, H, N, d, L, P, tau, causal,
+                         dtype, workspace, workspace_bytes, stream, Shard());
+}
+
+race_status_t race_attn_forward_begin(const void *k, const void *v, const float *W, float *ctx, size_t ctx_bytes,
+                                      float *h_total, int B, int H, int64_t N, int d, int L, int P, float tau,
+                                      int causal, race_dtype_t dtype, void *workspace, size_t workspace_bytes,
+                                      race_stream_t stream)
+{
+    Shard sh;
+    sh.stage = STAGE_BEGIN;
+    sh.h_total = h_total;
+    return forward_impl(nullptr, k, v, W, nullptr, nullptr, ctx, ctx_bytes, B, H, N, d, L, P, tau, causal, dtype,
+                        workspace, workspace_bytes, stream, sh);
+}
+
+race_status_t race_attn_forward_end(const void *q, const void *k, const void *v, const float *W,
+                                    const float *h_init, void *out, float *den, float *ctx, size_t ctx_bytes, int B,
+                                    int H, int64_t N, int d, int L, int P, float tau, int causal,
+                                    race_dtype_t dtype, void *workspace, size_t workspace_bytes,
+                                    race_stream_t stream)
+{
+    Shard sh;
+    sh.stage = STAGE_END;
+    sh.h_init = h_init;
+    return forward_impl(q, k, v, W, out, den, ctx, ctx_bytes, B, H, N, d, L, P, tau, causal, dtype, workspace,
+                        workspace_bytes, stream, sh);
+}
+
+race_status_t race_attn_backward_begin(const void *q, const void *k, const void *v, const float *W,
+                                       const void *out, const float *den, const void *dout, const float *ctx,
+                                       size_t ctx_bytes, const float *h_init, void *dq, float *g_total, int B,
+                                       int H, int64_t N, int d, int L, int P, float tau, int causal,
+                                       race_dtype_t dtype, void *workspace, size_t workspace_bytes,
+                                       race_stream_t stream)
+{
+    Shard sh;
+    sh.stage = STAGE_BEGIN;
+    sh.h_init = h_init;
+    sh.g_total = g_total;
+    return backward_impl(q, k, v, W, out, den, dout, ctx, ctx_bytes, dq, nullptr, nullptr, B, H, N, d, L, P, tau,
+                         causal, dtype, workspace, workspace_bytes, stream, sh);
+}
+
+race_status_t race_attn_backward_end(const void *q, const void *k, const void *v, const float *W,
+                                     const void *out, const float *den, const void *dout, const float *g_init,
+                                     void *dk, void *dv, int B, int H, int64_t N, int d, int L, int P, float tau,
+                                     int causal, race_dtype_t dtype, void *workspace, size_t workspace_bytes,
+                                     race_stream_t stream)
+{
+    Shard sh;
+    sh.stage = STAGE_END;
+    sh.g_init = g_init;
+    return backward_impl(q, k, v, W, out, den, dout, nullptr, 0, nullptr, dk, dv, B, H, N, d, L, P, tau, causal,
+                         dtype, workspace, workspace_bytes, stream, sh);
+}
+
+race_status_t race_attn_shard_combine(const float *gathered, int nshards, int shard, int which, int64_t elems,
+                                      float *out, race_stream_t stream)
+{
+    if (!gathered || !out || nshards < 1 || shard < 0 || shard >= nshards || which < 0 || which > 2 || elems < 0)
+        return RACE_ERR_INVALID_ARG;
+    if (elems == 0) return RACE_OK;
+    const unsigned blocks = (unsigned)((elems + gk::NT - 1) / gk::NT);
+    cudaError_t e = timed("shard_combine", (cudaStream_t)stream, [&] {
+        gk::race_shard_combine<<<blocks, gk::NT, 0, (cudaStream_t)stream>>>(gathered, nshards, shard, which, elems,
+                                                                             out);
+        return cudaGetLastError();
+    });
     return e == cudaSuccess ? RACE_OK : RACE_ERR_CUDA;
 }
 

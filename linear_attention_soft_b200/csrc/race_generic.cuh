@@ -44,7 +44,7 @@ constexpr int MAXG = 8;   // groups per cluster (portable cluster size)
 constexpr int CSLOT = 5;  // column slots of 32: D = d + 1 <= 160
 
 enum AggMode { AGG_KV = 0, AGG_QDY = 1 };
-enum ScanMode { SCAN_EXCL_PREFIX = 0, SCAN_EXCL_SUFFIX = 1, SCAN_TOTAL = 2 };
+enum ScanMode { SCAN_EXCL_PREFIX = 0, SCAN_EXCL_SUFFIX = 1, SCAN_TOTAL = 2, SCAN_TOTAL_ONLY = 3 };
 
 struct Args {
     const void *q, *k, *v, *o, *dout;
@@ -515,18 +515,27 @@ __global__ void __launch_bounds__(NT) race_agg(Args a)
 
 // ------------------------------------------------------------------------------------
 // race_scan: over the segments of each (b, h), element-wise on the [M][D] states.
+//   SCAN_EXCL_PREFIX / SUFFIX: each segment's slot becomes the sum of the segments before
+//     (after) it, starting from init (statistics of tokens held elsewhere, e.g. earlier or
+//     later shards of the sequence; null = zero);
+//   SCAN_TOTAL: slot 0 becomes init + the sum of all segments;
+//   SCAN_TOTAL_ONLY: the buffer is left as it is.
+// total_out (optional) receives the sum of all segments (plus init, except TOTAL_ONLY).
 // grid (ceil(M*D / NT), BH)
 // ------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(NT) race_scan(float *buf, int nseg, int64_t MD, int mode)
+__global__ void __launch_bounds__(NT) race_scan(float *buf, int nseg, int64_t MD, int mode, const float *init,
+                                                float *total_out)
 {
     const int64_t e = (int64_t)blockIdx.x * NT + threadIdx.x;
     if (e >= MD) return;
     float *b = buf + (int64_t)blockIdx.y * nseg * MD + e;
+    const int64_t oe = (int64_t)blockIdx.y * MD + e;
     constexpr int K = 8;  // segments loaded together: independent loads in flight
-    float run = 0.f;
-    if (mode == SCAN_TOTAL) {
-        for (int s = 0; s < nseg; ++s) run += b[s * MD];
-        b[0] = run;
+    float run = (init && mode != SCAN_TOTAL_ONLY) ? init[oe] : 0.f;
+    if (mode == SCAN_TOTAL || mode == SCAN_TOTAL_ONLY) {
+        for (int s = 0; s < nseg; ++s) run += b[(int64_t)s * MD];
+        if (mode == SCAN_TOTAL) b[0] = run;
+        if (total_out) total_out[oe] = run;
         return;
     }
     const bool rev = mode == SCAN_EXCL_SUFFIX;
@@ -546,6 +555,25 @@ __global__ void __launch_bounds__(NT) race_scan(float *buf, int nseg, int64_t MD
             }
         }
     }
+    if (total_out) total_out[oe] = run;
+}
+
+// ------------------------------------------------------------------------------------
+// race_shard_combine: out = sum of the selected shards' statistics, in shard order:
+// which = 0 the shards before `shard`, 1 those after it, 2 every other shard.
+// gathered is [nshards][elems].  grid ceil(elems / NT)
+// ------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(NT) race_shard_combine(const float *gathered, int nshards, int shard, int which,
+                                                         int64_t elems, float *out)
+{
+    const int64_t e = (int64_t)blockIdx.x * NT + threadIdx.x;
+    if (e >= elems) return;
+    float run = 0.f;
+    for (int s = 0; s < nshards; ++s) {
+        const bool take = which == 0 ? s < shard : which == 1 ? s > shard : s != shard;
+        if (take) run += gathered[(int64_t)s * elems + e];
+    }
+    out[e] = run;
 }
 
 __device__ inline void load_state(const Args &a, int g, int seg, int bh, int Mg, float *st)

@@ -169,3 +169,22 @@ def test_decode_entry_points_reject_bad_arguments_without_launching(lib):
         ra.RACE_ERR_INVALID_ARG         # dtype
     assert g(16, 16, 16, 16, 1, 1, 128, 64, 16, 4, ctypes.c_float(0.5), ra.RACE_BF16, 16, 16, None) == \
         ra.RACE_ERR_WORKSPACE
+
+
+def test_shard_entry_points_reject_bad_arguments_without_launching(lib):
+    import linear_attention_soft_b200 as ra
+    f = lib.race_attn_shard_combine
+    assert f(None, 2, 0, 0, 8, 16, None) == ra.RACE_ERR_INVALID_ARG
+    assert f(16, 2, 2, 0, 8, 16, None) == ra.RACE_ERR_INVALID_ARG      # shard out of range
+    assert f(16, 2, 0, 3, 8, 16, None) == ra.RACE_ERR_INVALID_ARG      # which
+    assert f(16, 2, 0, 0, 0, 16, None) == ra.RACE_OK                   # nothing to sum
+    fb = lib.race_attn_forward_begin
+    args = [16, 16, 16, None, 0, None, 1, 1, 256, 64, 16, 4, ctypes.c_float(0.5), 1, ra.RACE_BF16, 16, 1 << 30,
+            None]
+    assert fb(*args) == ra.RACE_ERR_INVALID_ARG                        # h_total is required
+    args[5] = 8
+    assert fb(*args) == ra.RACE_ERR_INVALID_ARG                        # misaligned
+    bb = lib.race_attn_backward_begin
+    bargs = [16] * 8 + [0, None, 16, None, 1, 1, 256, 64, 16, 4, ctypes.c_float(0.5), 1, ra.RACE_BF16, 16,
+                        1 << 30, None]
+    assert bb(*bargs) == ra.RACE_ERR_INVALID_ARG                       # g_total is required
