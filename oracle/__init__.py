@@ -72,7 +72,7 @@ def _load():
         lib.race_oracle_backward.argtypes = [_dp, _dp, _dp, _dp, _dp, ctypes.c_int64,
                                              ctypes.c_int64, ctypes.c_int, ctypes.c_int,
                                              ctypes.c_int, ctypes.c_double, ctypes.c_int,
-                                             _dp, _dp, _dp]
+                                             _dp, _dp, _dp, _dp]
         lib.race_oracle_backward.restype = ctypes.c_int
         lib.race_oracle_state.argtypes = [_dp, _dp, _dp, ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
                                           ctypes.c_int, ctypes.c_int, ctypes.c_double, _dp]
@@ -180,8 +180,10 @@ def forward(q, k, v, W, tau: float, causal: bool, rows=None):
     return out.reshape(tuple(lead) + (n, d)), den.reshape(tuple(lead) + (n,))
 
 
-def backward(q, k, v, W, dout, tau: float, causal: bool):
-    """Gradients (dq, dk, dv) of sum(out * dout) for the forward above (soft hashing)."""
+def backward(q, k, v, W, dout, tau: float, causal: bool, with_dw: bool = False):
+    """Gradients (dq, dk, dv) of sum(out * dout) for the forward above (soft hashing); with
+    ``with_dw`` also dW [L, P, d], the gradient with respect to the hyperplanes (shared by
+    every head, so summed over them)."""
     q, k, v, W, dout = _f64(q), _f64(k), _f64(v), _f64(W), _f64(dout)
     *lead, N, d = q.shape
     BH = int(np.prod(lead)) if lead else 1
@@ -189,13 +191,14 @@ def backward(q, k, v, W, dout, tau: float, causal: bool):
     dq = np.empty_like(q)
     dk = np.empty_like(k)
     dv = np.empty_like(v)
+    dW = np.empty_like(W) if with_dw else None
     rc = _load().race_oracle_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(W), _ptr(dout), BH, N, d,
                                       L, P, float(tau), int(bool(causal)),
-                                      _ptr(dq), _ptr(dk), _ptr(dv))
+                                      _ptr(dq), _ptr(dk), _ptr(dv),
+                                      _ptr(dW) if with_dw else ctypes.cast(None, _dp))
     if rc != 0:
         raise RuntimeError("race_oracle_backward failed with code %d" % rc)
-    return dq, dk, dv
-
+    return (dq, dk, dv, dW) if with_dw else (dq, dk, dv)
 
 def state(k, v, W, tau: float) -> np.ndarray:
     """Bucket statistics H[m, c] = sum_j phi(k_j)[m] [v_j, 1][c] over every key of each head

@@ -134,9 +134,10 @@ void race_oracle_hash_indices(const double *x, int d, const double *W, int L, in
 
 /* Vector-Jacobian product of the feature map: given dphi = dLoss/dphi(x), return
  * dx = dLoss/dx through softmax, the corner logits, tanh, the projection and the
- * normalisation (soft hashing only). */
-void race_oracle_features_backward(const double *x, int d, const double *W, int L, int P,
-                                   double beta, const double *dphi, double *dx)
+ * normalisation (soft hashing only); dp (optional, [L*P]) receives dLoss/dp for the
+ * projections p = W_l x^, from which the gradient of W follows (dW_lp += dp_lp x^). */
+static void features_vjp(const double *x, int d, const double *W, int L, int P, double beta,
+                         const double *dphi, double *dx, double *dp_out)
 {
     const int R = 1 << P;
     double s2 = 0.0;
@@ -180,6 +181,7 @@ void race_oracle_features_backward(const double *x, int d, const double *W, int 
             for (int r = 0; r < R; ++r) s += corner_sign(r, p) * dz[r];
             du[p] = beta * s;
             dp[p] = du[p] * (1.0 - u[p] * u[p]);
+            if (dp_out) dp_out[l * P + p] = dp[p];
         }
         /* proj = W_l x^ */
         for (int p = 0; p < P; ++p) {
@@ -198,6 +200,31 @@ void race_oracle_features_backward(const double *x, int d, const double *W, int 
     free(xh);
     free(dxh);
     free(phi);
+}
+
+void race_oracle_features_backward(const double *x, int d, const double *W, int L, int P,
+                                   double beta, const double *dphi, double *dx)
+{
+    if (d < 1) return;
+    features_vjp(x, d, W, L, P, beta, dphi, dx, NULL);
+}
+
+/* dW[l][p][:] += sum over the tokens t0..t0+nt-1 of dp[t][l*P+p] x^_t, x^ = x / max(|x|, eps),
+ * every element summed in token order. */
+static void accumulate_dw(const double *x, int64_t t0, int64_t nt, int d, int LP, const double *dp,
+                          double *dW)
+{
+    double *inv = (double *)malloc(sizeof(double) * (size_t)(nt > 0 ? nt : 1));
+    if (!inv) return;
+    for (int64_t t = 0; t < nt; ++t) inv[t] = 1.0 / row_norm(x + (t0 + t) * d, d);
+#pragma omp parallel for schedule(static)
+    for (int e = 0; e < LP * d; ++e) {
+        const int lp = e / d, c = e % d;
+        double s = dW[e];
+        for (int64_t t = 0; t < nt; ++t) s += dp[t * LP + lp] * x[(t0 + t) * d + c] * inv[t];
+        dW[e] = s;
+    }
+    free(inv);
 }
 
 /* ---------------------------------------------------------------------------------------- */
@@ -387,7 +414,7 @@ int race_oracle_state(const double *k, const double *v, const double *W, int64_t
  */
 static int backward_head(const double *q, const double *k, const double *v, const double *W,
                          const double *dout, int64_t N, int d, int L, int P, double tau,
-                         int causal, double *dq, double *dk, double *dv)
+                         int causal, double *dq, double *dk, double *dv, double *dW)
 {
     const int M = L << P, D = d + 1;
     const double beta = 1.0 / tau;
@@ -401,8 +428,9 @@ static int backward_head(const double *q, const double *k, const double *v, cons
     double *phik = (double *)malloc(sizeof(double) * (size_t)NB * M);
     double *phiq = (double *)malloc(sizeof(double) * (size_t)NB * M);
     double *dphi = (double *)malloc(sizeof(double) * (size_t)NB * M);
+    double *dpb = dW ? (double *)malloc(sizeof(double) * (size_t)NB * L * P) : NULL;
     int rc = 0;
-    if (!o || !den || !dY || !Hm || !Gm || !Gc || !phik || !phiq || !dphi) { rc = 1; goto done; }
+    if (!o || !den || !dY || !Hm || !Gm || !Gc || !phik || !phiq || !dphi || (dW && !dpb)) { rc = 1; goto done; }
 
     rc = forward_head(q, k, v, W, N, d, L, P, tau, causal, 0, NULL, o, den);
     if (rc) goto done;
@@ -442,8 +470,9 @@ static int backward_head(const double *q, const double *k, const double *v, cons
         }
 #pragma omp parallel for schedule(static)
         for (int64_t t = 0; t < nt; ++t)
-            race_oracle_features_backward(q + (t0 + t) * d, d, W, L, P, beta, dphi + t * M,
-                                          dq + (t0 + t) * d);
+            features_vjp(q + (t0 + t) * d, d, W, L, P, beta, dphi + t * M, dq + (t0 + t) * d,
+                         dpb ? dpb + t * L * P : NULL);
+        if (dW) accumulate_dw(q, t0, nt, d, L * P, dpb, dW);
     }
 
     /* ---- dk, dv: suffix (causal) or total (bidirectional) state G */
@@ -496,25 +525,30 @@ static int backward_head(const double *q, const double *k, const double *v, cons
         }
 #pragma omp parallel for schedule(static)
         for (int64_t t = 0; t < nt; ++t)
-            race_oracle_features_backward(k + (t0 + t) * d, d, W, L, P, beta, dphi + t * M,
-                                          dk + (t0 + t) * d);
+            features_vjp(k + (t0 + t) * d, d, W, L, P, beta, dphi + t * M, dk + (t0 + t) * d,
+                         dpb ? dpb + t * L * P : NULL);
+        if (dW) accumulate_dw(k, t0, nt, d, L * P, dpb, dW);
     }
 
 done:
     free(o); free(den); free(dY); free(Hm); free(Gm); free(Gc);
-    free(phik); free(phiq); free(dphi);
+    free(phik); free(phiq); free(dphi); free(dpb);
     return rc;
 }
 
+/* dW (optional, [L][P][d], zeroed here) receives the gradient with respect to the
+ * hyperplanes, summed over every head (W is shared by all of them): p = W_l x^ for every
+ * q and k row, so dW_lp = sum over rows of dLoss/dp_lp x^. */
 int race_oracle_backward(const double *q, const double *k, const double *v, const double *W,
                          const double *dout, int64_t BH, int64_t N, int d, int L, int P,
-                         double tau, int causal, double *dq, double *dk, double *dv)
+                         double tau, int causal, double *dq, double *dk, double *dv, double *dW)
 {
     if (BH < 0 || N < 0 || d < 1 || L < 1 || P < 1 || P > 6 || !(tau > 0.0)) return 2;
+    if (dW) memset(dW, 0, sizeof(double) * (size_t)L * P * d);
     for (int64_t bh = 0; bh < BH; ++bh) {
         const size_t off = (size_t)bh * N * d;
         int rc = backward_head(q + off, k + off, v + off, W, dout + off, N, d, L, P, tau, causal,
-                               dq + off, dk + off, dv + off);
+                               dq + off, dk + off, dv + off, dW);
         if (rc) return rc;
     }
     return 0;

@@ -369,3 +369,58 @@ def test_state_read_out_is_the_last_causal_row():
     out, den = oracle.forward(q, k, v, W, 0.5, True, rows=[39])
     np.testing.assert_allclose(den[0], y[-1], rtol=1e-12)
     np.testing.assert_allclose(out[0], y[:-1] / y[-1], rtol=1e-12)
+
+
+# ------------------------------------------------------------------------------------------
+# Gradient with respect to the hyperplanes W (chain rule through p = W_l x^; the pages
+# treat W as fixed random projections, zh §2.2, so this is the learnable-W variant)
+# ------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("tau", [0.5, 1.0])
+def test_hyperplane_gradient_matches_finite_differences(causal, tau):
+    q, k, v, W = _case(N=9, d=4, L=2, P=2, seed=27)
+    do = np.random.default_rng(28).standard_normal(q.shape)
+    dq, dk, dv, dW = oracle.backward(q, k, v, W, do, tau, causal, with_dw=True)
+    h = 1e-6
+    fd = np.zeros_like(W)
+    for idx in np.ndindex(W.shape):
+        Wp, Wm = W.copy(), W.copy()
+        Wp[idx] += h
+        Wm[idx] -= h
+        lp = float((oracle.forward(q, k, v, Wp, tau, causal)[0] * do).sum())
+        lm = float((oracle.forward(q, k, v, Wm, tau, causal)[0] * do).sum())
+        fd[idx] = (lp - lm) / (2 * h)
+    np.testing.assert_allclose(dW, fd, rtol=1e-6, atol=1e-8 * np.abs(fd).max())
+    # the other gradients are unchanged by asking for dW
+    for a, b in zip((dq, dk, dv), oracle.backward(q, k, v, W, do, tau, causal)):
+        np.testing.assert_array_equal(a, b)
+
+
+def test_hyperplane_gradient_sums_over_heads_and_blocks():
+    """W is shared by every head, so the batch's dW is the sum of the heads' dW; a run longer
+    than the oracle's feature block accumulates across blocks."""
+    rng = np.random.default_rng(29)
+    q, k, v, do = (rng.standard_normal((2, 2100, 4)) for _ in range(4))
+    W = rng.standard_normal((2, 2, 4))
+    dW = oracle.backward(q, k, v, W, do, 0.5, True, with_dw=True)[3]
+    parts = [oracle.backward(q[h], k[h], v[h], W, do[h], 0.5, True, with_dw=True)[3] for h in range(2)]
+    np.testing.assert_allclose(dW, parts[0] + parts[1], rtol=1e-12, atol=1e-12)
+
+
+def test_hyperplane_gradient_of_a_scale_free_loss():
+    """Scaling one hyperplane row W_lp by a > 0 changes p_lp = W_lp x^ by the same factor;
+    the loss's derivative along that direction, sum_c W_lpc dW_lpc, must equal
+    d/da L(a W_lp) at a = 1 (a directional check of every row at once)."""
+    q, k, v, W = _case(N=20, d=5, L=3, P=2, seed=30)
+    do = np.random.default_rng(31).standard_normal(q.shape)
+    dW = oracle.backward(q, k, v, W, do, 0.5, True, with_dw=True)[3]
+    h = 1e-6
+    for l in range(W.shape[0]):
+        for p in range(W.shape[1]):
+            Wp, Wm = W.copy(), W.copy()
+            Wp[l, p] *= 1 + h
+            Wm[l, p] *= 1 - h
+            lp = float((oracle.forward(q, k, v, Wp, 0.5, True)[0] * do).sum())
+            lm = float((oracle.forward(q, k, v, Wm, 0.5, True)[0] * do).sum())
+            np.testing.assert_allclose((W[l, p] * dW[l, p]).sum(), (lp - lm) / (2 * h), rtol=1e-6, atol=1e-9)
