@@ -263,16 +263,22 @@ def run_ours(args, w):
     code = ra.RACE_F32 if w.dtype == "f32" else ra.RACE_BF16
     ws_f = torch.empty(ra.race_attn_workspace_size(B, H, N, d, L, P, w.causal, 0, code),
                        dtype=torch.uint8, device=dev)
-    ws_b = torch.empty(ra.race_attn_workspace_size(B, H, N, d, L, P, w.causal, 1, code),
+    ws_b = torch.empty(ra.race_attn_dw_workspace_size(B, H, N, d, L, P, w.causal, code) if args.dw else
+                       ra.race_attn_workspace_size(B, H, N, d, L, P, w.causal, 1, code),
                        dtype=torch.uint8, device=dev)
+    dW = torch.empty(W.shape, dtype=torch.float32, device=dev)
     ctx = torch.empty(ra.race_attn_ctx_size(B, H, N, d, L, P, w.causal) // 4,
                       dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     def step(qq=q, kk=k, vv=v, dd=do):
         ra.race_attn_forward(qq, kk, vv, W, out, den, ctx, w.tau, w.causal, ws_f, stream)
-        ra.race_attn_backward(qq, kk, vv, W, out, den, dd, ctx, dq, dk, dv, w.tau, w.causal,
-                              ws_b, stream)
+        if args.dw:
+            ra.race_attn_backward_dw(qq, kk, vv, W, out, den, dd, ctx, dq, dk, dv, dW, w.tau, w.causal, ws_b,
+                                     stream)
+        else:
+            ra.race_attn_backward(qq, kk, vv, W, out, den, dd, ctx, dq, dk, dv, w.tau, w.causal,
+                                  ws_b, stream)
 
     def barrier():
         if world > 1:
@@ -379,7 +385,7 @@ def run_ours(args, w):
                 "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
                 "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
                            "L": w.L, "P": w.P, "tau": w.tau, "causal": w.causal,
-                           "dist": w.dist, "l2": "inputs larger than L2 (no flush)",
+                           "dist": w.dist, "l2": "inputs larger than L2 (no flush)", "dW": bool(args.dw),
                            "head_tokens_per_s": B * H * N * world / (ms_max / 1e3)},
                 "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                         "d2h_bytes_per_step": d2h},
@@ -486,6 +492,7 @@ def main():
                     choices=sorted(race_inputs.WORKLOADS))
     ap.add_argument("--n", type=int, default=0, help="override the sequence length")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--dw", action="store_true", help="also compute the gradient of the hyperplanes W")
     ap.add_argument("--decode", action="store_true",
                     help="time the streaming decode step instead (one token per head, 4096 heads)")
     args = ap.parse_args()

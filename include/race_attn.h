@@ -172,6 +172,26 @@ race_status_t race_attn_forward_noalloc(const void *q, const void *k, const void
                                         race_dtype_t dtype, race_stream_t stream);
 
 /*
+ * Backward that also returns the gradient with respect to the hyperplanes, for the variant
+ * in which W is learned (the pages treat W as fixed Gaussian hyperplanes, zh §2.2; this is
+ * the chain rule through p_l = W_l x^ for every q and k row):
+ *   dW[l][p][:] = sum over heads and rows of dLoss/dp_lp * x^,   x^ = x / max(|x|, 1e-12).
+ *   dW         device fp32 [L,P,d], written (not accumulated; zero when N = 0).
+ *   workspace  workspace_bytes >= race_attn_dw_workspace_size(...); scratch.
+ * Other arguments, results and errors as race_attn_backward.  dW is summed over rows in a
+ * fixed order (per split, then over the splits), so repeated calls give the same bits.
+ */
+race_status_t race_attn_dw_workspace_size(int B, int H, int64_t N, int d, int L, int P, int causal,
+                                          race_dtype_t dtype, size_t *bytes);
+race_status_t race_attn_backward_dw(const void *q, const void *k, const void *v, const float *W,
+                                    const void *out, const float *den, const void *dout,
+                                    const float *ctx, size_t ctx_bytes, void *dq, void *dk,
+                                    void *dv, float *dW, int B, int H, int64_t N, int d, int L,
+                                    int P, float tau, int causal, race_dtype_t dtype,
+                                    void *workspace, size_t workspace_bytes,
+                                    race_stream_t stream);
+
+/*
  * ---- one sequence sharded over several devices -------------------------------------------
  * The statistics of Algorithm 2 (zh §2.3) are sums over tokens, so a sequence split into
  * contiguous shards (one per device, shard s holding tokens [s*n, (s+1)*n) of every head)

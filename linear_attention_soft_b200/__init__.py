@@ -27,7 +27,8 @@ __all__ = [
     "race_attn_device_error", "race_attn_selftest_wait_timeout", "race_attn_state",
     "race_attn_decode_workspace_size", "race_attn_decode_step", "state", "decode_step",
     "race_attn_forward_begin", "race_attn_forward_end", "race_attn_backward_begin",
-    "race_attn_backward_end", "race_attn_shard_combine",
+    "race_attn_backward_end", "race_attn_shard_combine", "race_attn_dw_workspace_size",
+    "race_attn_backward_dw", "backward_dw",
 ]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -110,6 +111,11 @@ def load_library():
     lib.race_attn_backward_end.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _i64,
                                            _int, _int, _int, ctypes.c_float, _int, _int, _vp, _sz, _vp]
     lib.race_attn_backward_end.restype = _int
+    lib.race_attn_dw_workspace_size.argtypes = [_int, _int, _i64, _int, _int, _int, _int, _int, ctypes.POINTER(_sz)]
+    lib.race_attn_dw_workspace_size.restype = _int
+    lib.race_attn_backward_dw.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp, _vp, _vp, _int, _int,
+                                          _i64, _int, _int, _int, ctypes.c_float, _int, _int, _vp, _sz, _vp]
+    lib.race_attn_backward_dw.restype = _int
     lib.race_attn_shard_combine.argtypes = [_vp, _int, _int, _int, _i64, _vp, _vp]
     lib.race_attn_shard_combine.restype = _int
     lib.race_attn_profile_enable.argtypes = [_int]
@@ -298,6 +304,23 @@ def race_attn_shard_combine(gathered, shard: int, which: int, out, stream=None) 
                                                   _stream(stream)), "race_attn_shard_combine")
 
 
+def race_attn_dw_workspace_size(B, H, N, d, L, P, causal, dtype) -> int:
+    out = _sz()
+    _check(load_library().race_attn_dw_workspace_size(B, H, N, d, L, P, int(causal), int(dtype), ctypes.byref(out)),
+           "race_attn_dw_workspace_size")
+    return out.value
+
+
+def race_attn_backward_dw(q, k, v, W, out, den, dout, ctx, dq, dk, dv, dW, tau: float, causal: bool, workspace,
+                          stream=None) -> None:
+    """C ABI backward that also writes dW [L, P, d] fp32 (gradient of the hyperplanes)."""
+    B, H, N, d, L, P = _dims(q, W)
+    _check(load_library().race_attn_backward_dw(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(W), _ptr(out), _ptr(den), _ptr(dout), _ptr(ctx), _nbytes(ctx),
+        _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dW), B, H, N, d, L, P, float(tau), int(bool(causal)), _dtype_code(q),
+        _ptr(workspace), _nbytes(workspace), _stream(stream)), "race_attn_backward_dw")
+
+
 def race_attn_device_error(stream=None) -> int:
     """1 if a tensor-core kernel gave up waiting on an MMA since the last call (and clear)."""
     flag = _int()
@@ -383,3 +406,14 @@ def decode_step(q, k, v, W, state, tau: float, stream=None):
                      device=q.device)
     race_attn_decode_step(q, k, v, W, state, out, den, tau, ws, stream)
     return out, den
+
+
+def backward_dw(q, k, v, W, out, den, dout, tau: float, causal: bool, ctx=None, stream=None):
+    """Allocate and run the backward with the hyperplane gradient: (dq, dk, dv, dW)."""
+    B, H, N, d, L, P = _dims(q, W)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dW = torch.empty(W.shape, dtype=torch.float32, device=q.device)
+    ws = torch.empty(max(race_attn_dw_workspace_size(B, H, N, d, L, P, causal, _dtype_code(q)), 16),
+                     dtype=torch.uint8, device=q.device)
+    race_attn_backward_dw(q, k, v, W, out, den, dout, ctx, dq, dk, dv, dW, tau, causal, ws, stream)
+    return dq, dk, dv, dW

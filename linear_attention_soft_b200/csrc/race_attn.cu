@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -250,6 +251,7 @@ struct Shard {
     float *h_total = nullptr;
     const float *g_init = nullptr;
     float *g_total = nullptr;
+    void *dpq = nullptr, *dpk = nullptr;  // backward: dLoss/dp / |x| per row, for dW (optional)
 };
 
 // ---- the general path (every shape and dtype) ----------------------------------------
@@ -287,6 +289,8 @@ cudaError_t generic_backward(const Plan &p, Args a, const float *hstates, bool h
     const dim3 grid((unsigned)p.G, (unsigned)p.nseg, (unsigned)p.BH);
     const int64_t stride = causal ? (int64_t)p.M * p.D : 0;
     a.causal = causal;
+    a.dpq = (float *)sh.dpq;
+    a.dpk = (float *)sh.dpk;
     cudaError_t e;
     if (sh.stage != STAGE_END) {
         if (!have_ctx) {  // key-side prefix statistics, as the forward computes them
@@ -434,6 +438,8 @@ cudaError_t tc_backward(const Plan &p, const void *q, const void *k, const void 
     a.dv = (__nv_bfloat16 *)dv;
     a.wimg = wimg;
     a.cbuf = cbuf;
+    a.dpq = (__nv_bfloat16 *)sh.dpq;
+    a.dpk = (__nv_bfloat16 *)sh.dpk;
     e = timed("tc_w_image", st, [&] {
         tc::tc_w_image<<<1, tc::NTH, 0, st>>>(W, wimg);
         return cudaGetLastError();
@@ -675,9 +681,137 @@ race_status_t backward_impl(const void *q, const void *k, const void *v, const f
     return e == cudaSuccess ? RACE_OK : RACE_ERR_CUDA;
 }
 
+// ---- gradient of W (the learnable-hyperplane variant) -----------------------------------
+// Workspace after the backward's own: dLoss/dp / |x| for the q rows and the k rows (sized for
+// the general path's fp32 [rows][L*P]; the tensor-core path uses bf16 [rows][64] of it), then
+// the per-split partial sums of dW.
+struct DwPlan {
+    size_t dp_bytes;     // one side
+    int tc_nblk;         // tensor-core reduction: CTAs
+    int64_t tc_chunks_per_cta;
+    int ksplit;          // general reduction: row splits
+    int64_t rows_per_split;
+    size_t partial_bytes;
+};
+DwPlan dw_plan(const Plan &p)
+{
+    DwPlan dp;
+    const int64_t rows = (int64_t)p.BH * p.N;
+    const int LP = p.L * p.P;
+    dp.dp_bytes = ((size_t)rows * LP * sizeof(float) + 255) / 256 * 256;
+    const int sms = device_sm_count();
+    const int64_t cps = (int64_t)p.BH * ((p.N + race::tc::T - 1) / race::tc::T);
+    dp.tc_nblk = (int)std::max<int64_t>(1, std::min<int64_t>(2 * sms, 2 * cps));
+    dp.tc_chunks_per_cta = (2 * cps + dp.tc_nblk - 1) / dp.tc_nblk;
+    const int tiles = ((LP + 63) / 64) * ((p.d + 63) / 64);
+    dp.ksplit = (int)std::max<int64_t>(1, std::min<int64_t>((2 * sms + tiles - 1) / tiles, (2 * rows + 15) / 16));
+    dp.rows_per_split = ((2 * rows + dp.ksplit - 1) / dp.ksplit + 15) / 16 * 16;
+    const size_t tc_part = (size_t)dp.tc_nblk * 64 * 64 * sizeof(float);
+    const size_t gen_part = (size_t)dp.ksplit * LP * p.d * sizeof(float);
+    dp.partial_bytes = std::max(tc_part, gen_part);
+    return dp;
+}
+
+cudaError_t tc_dw(const Plan &p, const DwPlan &dp, const void *q, const void *k, const void *dpq, const void *dpk,
+                  float *partial, float *dW, cudaStream_t st)
+{
+    namespace tc = race::tc;
+    tc::DwArgs a;
+    std::memset(&a, 0, sizeof(a));
+    cudaError_t e;
+    if ((e = bf16_map(&a.tm_dp[0], dpq, p, false)) != cudaSuccess || (e = bf16_map(&a.tm_dp[1], dpk, p, false)) != cudaSuccess ||
+        (e = bf16_map(&a.tm_x[0], q, p, false)) != cudaSuccess || (e = bf16_map(&a.tm_x[1], k, p, false)) != cudaSuccess)
+        return e;
+    a.chunks_per_head = (p.N + tc::T - 1) / tc::T;
+    a.chunks_per_side = (int64_t)p.BH * a.chunks_per_head;
+    a.chunks_per_cta = dp.tc_chunks_per_cta;
+    a.partial = partial;
+    const size_t sm = tc::smem_bytes(tc::dw_smem::TOTAL);
+    if ((e = tc_prepare(tc::tc_dw, sm)) != cudaSuccess) return e;
+    e = timed("tc_dw", st, [&] {
+        tc::tc_dw<<<dp.tc_nblk, 128, sm, st>>>(a);
+        return cudaGetLastError();
+    });
+    if (e != cudaSuccess) return e;
+    return timed("dw_sum", st, [&] {
+        tc::tc_dw_reduce<<<16, 256, 0, st>>>(partial, dp.tc_nblk, dW);
+        return cudaGetLastError();
+    });
+}
+
+template <typename DT>
+cudaError_t generic_dw(const Plan &p, const DwPlan &dp, const void *q, const void *k, const float *dpq,
+                       const float *dpk, float *partial, float *dW, cudaStream_t st)
+{
+    const int LP = p.L * p.P;
+    const dim3 grid((unsigned)dp.ksplit, (unsigned)((LP + 63) / 64), (unsigned)((p.d + 63) / 64));
+    cudaError_t e = timed("generic_dw", st, [&] {
+        gk::race_dw_partial<DT><<<grid, gk::NT, 0, st>>>(dpq, dpk, (const DT *)q, (const DT *)k, (int64_t)p.BH * p.N,
+                                                         LP, p.d, dp.rows_per_split, partial);
+        return cudaGetLastError();
+    });
+    if (e != cudaSuccess) return e;
+    const int64_t n = (int64_t)LP * p.d;
+    return timed("dw_sum", st, [&] {
+        gk::race_dw_sum<<<(unsigned)((n + gk::NT - 1) / gk::NT), gk::NT, 0, st>>>(partial, dp.ksplit, n, dW);
+        return cudaGetLastError();
+    });
+}
+
 }  // namespace
 
 extern "C" {
+
+race_status_t race_attn_dw_workspace_size(int B, int H, int64_t N, int d, int L, int P, int causal,
+                                          race_dtype_t dtype, size_t *bytes)
+{
+    (void)causal;
+    if (!bytes) return RACE_ERR_INVALID_ARG;
+    if (dtype != RACE_F32 && dtype != RACE_BF16) return RACE_ERR_INVALID_ARG;
+    race_status_t s = check_sizes(B, H, N, d, L, P);
+    if (s != RACE_OK) return s;
+    const Plan p = make_plan(B, H, N, d, L, P);
+    const DwPlan dp = dw_plan(p);
+    *bytes = backward_workspace_bytes(p) + 2 * dp.dp_bytes + dp.partial_bytes;
+    return RACE_OK;
+}
+
+race_status_t race_attn_backward_dw(const void *q, const void *k, const void *v, const float *W, const void *out,
+                                    const float *den, const void *dout, const float *ctx, size_t ctx_bytes,
+                                    void *dq, void *dk, void *dv, float *dW, int B, int H, int64_t N, int d, int L,
+                                    int P, float tau, int causal, race_dtype_t dtype, void *workspace,
+                                    size_t workspace_bytes, race_stream_t stream)
+{
+    if (!dW || !aligned16(dW)) return RACE_ERR_INVALID_ARG;
+    if (dtype != RACE_F32 && dtype != RACE_BF16) return RACE_ERR_INVALID_ARG;
+    race_status_t s = check_sizes(B, H, N, d, L, P);
+    if (s != RACE_OK) return s;
+    if (!(tau > 0.f) || !std::isfinite(tau)) return tau == 0.f ? RACE_ERR_UNSUPPORTED : RACE_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (N == 0)
+        return cudaMemsetAsync(dW, 0, (size_t)L * P * d * sizeof(float), st) == cudaSuccess ? RACE_OK : RACE_ERR_CUDA;
+    const Plan p = make_plan(B, H, N, d, L, P);
+    const DwPlan dp = dw_plan(p);
+    const size_t bw = backward_workspace_bytes(p);
+    if (!workspace) return RACE_ERR_INVALID_ARG;
+    if (workspace_bytes < bw + 2 * dp.dp_bytes + dp.partial_bytes) return RACE_ERR_WORKSPACE;
+    uint8_t *wsb = (uint8_t *)workspace;
+    Shard sh;
+    sh.dpq = wsb + bw;
+    sh.dpk = wsb + bw + dp.dp_bytes;
+    float *partial = (float *)(wsb + bw + 2 * dp.dp_bytes);
+    s = backward_impl(q, k, v, W, out, den, dout, ctx, ctx_bytes, dq, dk, dv, B, H, N, d, L, P, tau, causal, dtype,
+                      workspace, bw, stream, sh);
+    if (s != RACE_OK) return s;
+    cudaError_t e;
+    if (race::tc::fast_path_ok(dtype, d, L, P, tau, N) && g_tc_backward)
+        e = tc_dw(p, dp, q, k, sh.dpq, sh.dpk, partial, dW, st);
+    else if (dtype == RACE_F32)
+        e = generic_dw<float>(p, dp, q, k, (const float *)sh.dpq, (const float *)sh.dpk, partial, dW, st);
+    else
+        e = generic_dw<__nv_bfloat16>(p, dp, q, k, (const float *)sh.dpq, (const float *)sh.dpk, partial, dW, st);
+    return e == cudaSuccess ? RACE_OK : RACE_ERR_CUDA;
+}
 
 race_status_t race_attn_forward(const void *q, const void *k, const void *v, const float *W,
                                 void *out, float *den, float *ctx, size_t ctx_bytes, int B,

@@ -61,6 +61,7 @@ struct Args {
     int hard, causal;
     int64_t seg_len;
     int nseg;
+    float *dpq, *dpk;  // optional: dLoss/dp / |x| per q (k) row [BH*N][L*P] fp32, for dW
 };
 
 // Shared-memory carve-up, in floats.  Identical on host and device.
@@ -243,6 +244,18 @@ __device__ void group_features_bwd(const float *phi, const float *dphi, const fl
             const float up = u[i * (tg * P) + l * P + p];
             o[p] = beta * du[p] * (1.f - up * up);
         }
+    }
+}
+
+// dp[T][tg*P] of this group's tables, divided by |x| of each row, into rows [0, nvalid) of a
+// [rows][LP] buffer at the group's first projection (for the gradient of W).
+template <int T>
+__device__ void store_dp(const float *dp, const float *rawn, int nvalid, int tg, int P, int g, int LP, float *dst)
+{
+    const int n = tg * P, lp0 = g * (MG >> P) * P;
+    for (int e = threadIdx.x; e < nvalid * n; e += NT) {
+        const int i = e / n, j = e - i * n;
+        dst[(int64_t)i * LP + lp0 + j] = dp[i * n + j] / fmaxf(rawn[i], kNormEps);
     }
 }
 
@@ -559,6 +572,78 @@ __global__ void __launch_bounds__(NT) race_scan(float *buf, int nseg, int64_t MD
 }
 
 // ------------------------------------------------------------------------------------
+// Gradient of W: dW[lp][c] = sum over rows of dp[row][lp] x[row][c] (dp = dLoss/dp / |x|),
+// over the q rows then the k rows.  CTA (ks, i, j) sums its share of the rows into the
+// 64 x 64 output tile (i, j); race_dw_sum adds the shares in ks order.  16 x 16 threads,
+// each a 4 x 4 block of the tile, rows staged 16 at a time.
+// grid (ksplit, ceil(LP / 64), ceil(d / 64))
+// ------------------------------------------------------------------------------------
+template <typename DT>
+__global__ void __launch_bounds__(NT) race_dw_partial(const float *dpq, const float *dpk, const DT *q, const DT *k,
+                                                      int64_t rows, int LP, int d, int64_t rows_per_split,
+                                                      float *partial)
+{
+    __shared__ float As[16][64], Bs[16][64];
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    const int lp0 = blockIdx.y * 64, c0 = blockIdx.z * 64;
+    float acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+    int64_t r0 = (int64_t)blockIdx.x * rows_per_split, r1 = r0 + rows_per_split;
+    if (r1 > 2 * rows) r1 = 2 * rows;
+    for (int64_t rb = r0; rb < r1; rb += 16) {
+        for (int e = threadIdx.x; e < 16 * 64; e += NT) {
+            const int rr = e >> 6, cc = e & 63;
+            const int64_t row = rb + rr;
+            float av = 0.f, bv = 0.f;
+            if (row < r1) {
+                const bool kside = row >= rows;
+                const int64_t rw = kside ? row - rows : row;
+                if (lp0 + cc < LP) av = (kside ? dpk : dpq)[rw * LP + lp0 + cc];
+                if (c0 + cc < d) bv = to_f32((kside ? k : q)[rw * d + c0 + cc]);
+            }
+            As[rr][cc] = av;
+            Bs[rr][cc] = bv;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int kk = 0; kk < 16; ++kk) {
+            float av[4], bv[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                av[i] = As[kk][ty * 4 + i];
+                bv[i] = Bs[kk][tx * 4 + i];
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+        }
+        __syncthreads();
+    }
+    float *dst = partial + (int64_t)blockIdx.x * LP * d;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int lp = lp0 + ty * 4 + i, c = c0 + tx * 4 + j;
+            if (lp < LP && c < d) dst[(int64_t)lp * d + c] = acc[i][j];
+        }
+}
+
+// dW[e] = sum over the splits of partial[s][e], in split order.
+__global__ void __launch_bounds__(NT) race_dw_sum(const float *partial, int nsplit, int64_t n, float *dW)
+{
+    const int64_t e = (int64_t)blockIdx.x * NT + threadIdx.x;
+    if (e >= n) return;
+    float s = 0.f;
+    for (int k = 0; k < nsplit; ++k) s += partial[(int64_t)k * n + e];
+    dW[e] = s;
+}
+
+// ------------------------------------------------------------------------------------
 // race_shard_combine: out = sum of the selected shards' statistics, in shard order:
 // which = 0 the shards before `shard`, 1 those after it, 2 every other shard.
 // gathered is [nshards][elems].  grid ceil(elems / NT)
@@ -716,6 +801,7 @@ __global__ void __launch_bounds__(NT) race_bwd_q_walk(Args a)
         if (a.causal) md_update<T>(st, phk, vt, Mg, D);
         group_features_bwd<T>(phq, dph, ub, nv, tg, a.P, a.beta, dpb);
         __syncthreads();
+        if (a.dpq) store_dp<T>(dpb, nq, nv, tg, a.P, g, a.L * a.P, a.dpq + ((int64_t)bh * a.N + c0) * (a.L * a.P));
         float *part = red + buf * T * d;
         group_dxhat<T>(wg, dpb, tg, a.P, d, part);
         cl.sync();
@@ -799,6 +885,7 @@ __global__ void __launch_bounds__(NT) race_bwd_kv_walk(Args a)
                 if (c < D) pv[(ty * RPT + r) * D + c] = acc[r][s];
             }
         __syncthreads();
+        if (a.dpk) store_dp<T>(dpb, nk, nv, tg, a.P, g, a.L * a.P, a.dpk + ((int64_t)bh * a.N + c0) * (a.L * a.P));
         float *px = redx + buf * T * d;
         group_dxhat<T>(wg, dpb, tg, a.P, d, px);
         cl.sync();

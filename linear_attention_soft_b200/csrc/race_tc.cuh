@@ -79,6 +79,7 @@ struct BwdArgs {
     const float *den, *W;
     const uint8_t *wimg;       // W as the two bf16 K128 tiles (hi, lo) of load_w_split, 16 KB
     float *cbuf;               // c_i = -(dO_i . o_i) per token [BH][N], written by the dq walk
+    __nv_bfloat16 *dpq, *dpk;  // optional: dLoss/dp / |x| per q (k) row [BH*N][64], for dW
     __nv_bfloat16 *dq, *dk, *dv;
     const float *state;
     int64_t state_seg_stride;
@@ -411,7 +412,8 @@ __device__ __forceinline__ void write_features(const float (&t)[16], int r, int 
 // dp~ = du (1 - u^2) -> 16 values as bf16 into row r of the DP tile (projections 16qd ..).
 __device__ __forceinline__ void features_vjp(uint32_t tm, uint32_t col0, int r, int qd, float beta, bool valid,
                                              const float (&u)[16], const float (&t)[16], const float *add_vec,
-                                             float add_scale, float mul, uint8_t *dp_tile)
+                                             float add_scale, float mul, uint8_t *dp_tile,
+                                             __nv_bfloat16 *dp_row = nullptr, float dp_scale = 0.f)
 {
     uint32_t g[4][16];
 #pragma unroll
@@ -460,6 +462,15 @@ __device__ __forceinline__ void features_vjp(uint32_t tm, uint32_t col0, int r, 
         st_shared_v4(b + sw128_off(r, 2 * qd + ch), pack_bf16x2(dp[8 * ch], dp[8 * ch + 1]),
                      pack_bf16x2(dp[8 * ch + 2], dp[8 * ch + 3]), pack_bf16x2(dp[8 * ch + 4], dp[8 * ch + 5]),
                      pack_bf16x2(dp[8 * ch + 6], dp[8 * ch + 7]));
+    if (dp_row && valid) {  // dLoss/dp / |x| of this row's 16 projections, for the gradient of W
+        uint4 *d4 = reinterpret_cast<uint4 *>(dp_row + 16 * qd);
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch)
+            d4[ch] = make_uint4(pack_bf16x2(dp[8 * ch] * dp_scale, dp[8 * ch + 1] * dp_scale),
+                                pack_bf16x2(dp[8 * ch + 2] * dp_scale, dp[8 * ch + 3] * dp_scale),
+                                pack_bf16x2(dp[8 * ch + 4] * dp_scale, dp[8 * ch + 5] * dp_scale),
+                                pack_bf16x2(dp[8 * ch + 6] * dp_scale, dp[8 * ch + 7] * dp_scale));
+    }
 }
 
 // Masked T x T block from TMEM (row r, columns col0 + 32qd ..) to bf16 K128 tile (qd >> 1)
@@ -1283,7 +1294,8 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_q_walk(const __grid_constant__ 
         if (c0 + T < t1) issue_kv_do(c0 + T);  // Phi_K, V~ and dO are free now
         reload_w();
         // dphi = (D + c_i H_prev[:, 64]) / den_i
-        features_vjp(tm, bq_tmem::DPHI, r, qd, a.beta, valid, u, t, hden, c_r, invden_r, sm + DP);
+        features_vjp(tm, bq_tmem::DPHI, r, qd, a.beta, valid, u, t, hden, c_r, invden_r, sm + DP,
+                     a.dpq ? a.dpq + (base + c0 + r) * DH : nullptr, 1.f / fmaxf(raw_q, kNormEps));
         publish_smem();
         if (threadIdx.x == 0 && wait_load_t0(ctl, ld, 3)) {
             fence_after_sync();
@@ -1461,7 +1473,8 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_kv_walk(const __grid_constant__
         if (ci > 0) issue_kv_do(c0 - T);  // Phi_K / masks, V~ and [dO | c] are free now
         reload_w();
         store_row16(tm, bkv_tmem::DVT, qd, valid, 1.f, a.dv + (base + c0 + r) * DH);
-        features_vjp(tm, bkv_tmem::DPHI, r, qd, a.beta, valid, u, t, nullptr, 0.f, 1.f, sm + DP);
+        features_vjp(tm, bkv_tmem::DPHI, r, qd, a.beta, valid, u, t, nullptr, 0.f, 1.f, sm + DP,
+                     a.dpk ? a.dpk + (base + c0 + r) * DH : nullptr, 1.f / fmaxf(raw_k, kNormEps));
         publish_smem();
         if (threadIdx.x == 0 && wait_load_t0(ctl, ld, 3)) {
             fence_after_sync();
@@ -1481,6 +1494,122 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_kv_walk(const __grid_constant__
     }
     drain_loads(ctl, ld);
     kernel_teardown(tm, bkv_tmem::NCOLS);
+}
+
+// ------------------------------------------------------------------------------------------
+// Gradient of W (the learnable-hyperplane variant): p = W_l x^ for every q and k row, so
+// dW = sum over rows of (dLoss/dp / |x|) x^T with the raw rows x.  The walks leave
+// dLoss/dp / |x| per row ([rows][64] bf16); here each CTA sums a range of 128-row chunks of
+// the q side then the k side on the tensor core, D[64 projections][64] += dp^T x, and
+// writes its partial; tc_dw_reduce adds the partials in CTA order.  The MMA's M is 128:
+// rows 64..127 of the accumulator come from the x tile placed after the dp tile and are
+// not read.   grid: nblk, 128 threads
+// ------------------------------------------------------------------------------------------
+struct DwArgs {
+    CUtensorMap tm_dp[2], tm_x[2];  // [BH][N][64] bf16 as 3-D maps, K128 boxes (q side, k side)
+    int64_t chunks_per_head;        // ceil(N / 128)
+    int64_t chunks_per_side;        // BH * chunks_per_head
+    int64_t chunks_per_cta;
+    float *partial;                 // [nblk][64][64]
+};
+
+namespace dw_smem {
+constexpr uint32_t STAGE = 2 * TILE;  // dp tile, then x tile
+constexpr uint32_t BAR = 2 * STAGE;   // 2 stages
+constexpr uint32_t TOTAL = BAR + 64;
+}  // namespace dw_smem
+
+__global__ void __launch_bounds__(128, 1) tc_dw(const __grid_constant__ DwArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = aligned_base(smem_raw);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + dw_smem::BAR);  // tma[2], mma[2]
+    __shared__ uint32_t tmem_slot;
+    __shared__ uint32_t failed;
+    const uint32_t sb = smem_u32(sm);
+    const int64_t c_begin = (int64_t)blockIdx.x * a.chunks_per_cta;
+    int64_t c_end = c_begin + a.chunks_per_cta;
+    if (c_end > 2 * a.chunks_per_side) c_end = 2 * a.chunks_per_side;
+    const int n = c_end > c_begin ? (int)(c_end - c_begin) : 0;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
+        failed = 0;
+    }
+    if (threadIdx.x < 32) tmem_alloc(&tmem_slot, 64);
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tm = tmem_slot;
+    if (threadIdx.x == 0 && n > 0) {
+        constexpr uint32_t id = idesc_bf16(128, 64, 1, 1);
+        auto load = [&](int i) {
+            const int64_t c = c_begin + i;
+            const int side = c >= a.chunks_per_side ? 1 : 0;
+            const int64_t hc = c - side * a.chunks_per_side;
+            const int head = (int)(hc / a.chunks_per_head), row = (int)((hc % a.chunks_per_head) * T);
+            const uint32_t st = sb + (uint32_t)(i & 1) * dw_smem::STAGE;
+            mbar_expect_tx(&bars[i & 1], 2 * TILE);
+            tma_load3(st, &a.tm_dp[side], 0, row, head, &bars[i & 1]);
+            tma_load3(st + TILE, &a.tm_x[side], 0, row, head, &bars[i & 1]);
+        };
+        bool ok = true;
+        load(0);
+        for (int i = 0; i < n && ok; ++i) {
+            if (i + 1 < n) {
+                if (i >= 1 && !mbar_wait(&bars[2 + ((i + 1) & 1)], ((i - 1) >> 1) & 1, WAIT_LIMIT_NS)) {
+                    ok = false;  // the stage's previous MMAs never completed
+                    break;
+                }
+                load(i + 1);
+            }
+            if (!mbar_wait(&bars[i & 1], (i >> 1) & 1, WAIT_LIMIT_NS)) {
+                ok = false;
+                break;
+            }
+            fence_after_sync();
+            const uint32_t st = sb + (uint32_t)(i & 1) * dw_smem::STAGE;
+            const uint64_t da = sdesc(st, TILE, 1024, LAYOUT_SW128), db = sdesc(st + TILE, TILE, 1024, LAYOUT_SW128);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+                mma_bf16(tm, da + kk * (2048 >> 4), db + kk * (2048 >> 4), id, (i > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(&bars[2 + (i & 1)]);
+        }
+        // the last commit covers every MMA issued before it; then every load in flight
+        if (ok && !mbar_wait(&bars[2 + ((n - 1) & 1)], ((n - 1) >> 1) & 1, WAIT_LIMIT_NS)) ok = false;
+        if (!ok) {
+            failed = 1;
+            atomicExch(&g_tc_error, 1);
+            for (int s = 0; s < 2; ++s) mbar_wait(&bars[s], 0, WAIT_LIMIT_NS);  // bounded drain
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    float *dst = a.partial + (int64_t)blockIdx.x * 64 * 64;
+    if (threadIdx.x < 64) {  // rows 0..63 of the accumulator: warps 0 and 1
+#pragma unroll 1
+        for (int c0 = 0; c0 < 64; c0 += 16) {
+            uint32_t w[16];
+            tmem_ld16_nowait(tlane(tm, (uint32_t)c0), w);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                dst[threadIdx.x * 64 + c0 + i] = (n > 0 && !failed) ? __uint_as_float(w[i]) : 0.f;
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (threadIdx.x < 32) tmem_dealloc(tm, 64);
+}
+
+// dW[e] = sum over the CTAs of partial[b][e], in CTA order.
+__global__ void tc_dw_reduce(const float *partial, int nblk, float *dW)
+{
+    const int e = blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= 64 * 64) return;
+    float s = 0.f;
+    for (int b = 0; b < nblk; ++b) s += partial[(int64_t)b * 64 * 64 + e];
+    dW[e] = s;
 }
 
 // W [64][64] fp32 -> its two bf16 K128 tiles (hi, lo) in global memory, byte for byte as

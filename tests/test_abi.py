@@ -188,3 +188,21 @@ def test_shard_entry_points_reject_bad_arguments_without_launching(lib):
     bargs = [16] * 8 + [0, None, 16, None, 1, 1, 256, 64, 16, 4, ctypes.c_float(0.5), 1, ra.RACE_BF16, 16,
                         1 << 30, None]
     assert bb(*bargs) == ra.RACE_ERR_INVALID_ARG                       # g_total is required
+
+
+def test_dw_entry_points_reject_bad_arguments_without_launching(lib):
+    import linear_attention_soft_b200 as ra
+    bw = ra.race_attn_workspace_size(1, 1, 4096, 64, 16, 4, 1, 1, ra.RACE_BF16)
+    dw = ra.race_attn_dw_workspace_size(1, 1, 4096, 64, 16, 4, 1, ra.RACE_BF16)
+    # the backward's workspace, then dLoss/dp of the q and k rows (fp32 [rows][L*P] each)
+    assert dw >= bw + 2 * 4096 * 64 * 4
+    f = lib.race_attn_backward_dw
+    args = [16] * 7 + [None, 0, 16, 16, 16, None, 1, 1, 4096, 64, 16, 4, ctypes.c_float(0.5), 1, ra.RACE_BF16, 16,
+                       dw, None]
+    assert f(*args) == ra.RACE_ERR_INVALID_ARG                    # dW missing
+    args[12] = 16
+    args[19] = ctypes.c_float(0.0)
+    assert f(*args) == ra.RACE_ERR_UNSUPPORTED                    # hard hashing has no gradient
+    args[19] = ctypes.c_float(0.5)
+    args[23] = dw - 1
+    assert f(*args) == ra.RACE_ERR_WORKSPACE
