@@ -176,14 +176,24 @@ cudaError_t bf16_map(CUtensorMap *m, const void *ptr, const Plan &p, bool value_
 {
     const EncodeTiled fn = encode_tiled();
     if (!fn) return cudaErrorNotSupported;
-    const cuuint64_t dims[3] = {64, (cuuint64_t)p.N, (cuuint64_t)p.BH};
-    const cuuint64_t strides[2] = {128, (cuuint64_t)p.N * 128};
-    const cuuint32_t box[3] = {value_atom ? 16u : 64u, (cuuint32_t)race::tc::T, 1};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
-                          CU_TENSOR_MAP_INTERLEAVE_NONE,
-                          value_atom ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_128B,
-                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    CUresult r;
+    if (value_atom) {  // (16 columns, rows, 4 atoms, heads): one box fills a whole value tile
+        const cuuint64_t dims[4] = {16, (cuuint64_t)p.N, 4, (cuuint64_t)p.BH};
+        const cuuint64_t strides[3] = {128, 32, (cuuint64_t)p.N * 128};
+        const cuuint32_t box[4] = {16, (cuuint32_t)race::tc::T, 4, 1};
+        const cuuint32_t estr[4] = {1, 1, 1, 1};
+        r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(ptr), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    } else {
+        const cuuint64_t dims[3] = {64, (cuuint64_t)p.N, (cuuint64_t)p.BH};
+        const cuuint64_t strides[2] = {128, (cuuint64_t)p.N * 128};
+        const cuuint32_t box[3] = {64, (cuuint32_t)race::tc::T, 1};
+        const cuuint32_t estr[3] = {1, 1, 1};
+        r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    }
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 

@@ -164,11 +164,12 @@ __device__ __forceinline__ void tma_k128(uint32_t dst, const CUtensorMap *m, int
     tma_load3(dst, m, 0, (int)row0, bh, bar);
 }
 
-// Columns 0..63 of rows [row0, row0 + 128) of head bh into atoms 0..3 of a 128-row value tile.
+// Columns 0..63 of rows [row0, row0 + 128) of head bh into atoms 0..3 of a 128-row value tile:
+// one box of a 4-D map (16 columns, rows, 4 atoms of 16 columns, heads) whose shared-memory
+// image is the four atoms one after another.
 __device__ __forceinline__ void tma_va(uint32_t dst, const CUtensorMap *m, int64_t row0, int bh, uint64_t *bar)
 {
-#pragma unroll
-    for (int k = 0; k < 4; ++k) tma_load3(dst + (uint32_t)k * VA128, m, 16 * k, (int)row0, bh, bar);
+    tma_load4(dst, m, 0, (int)row0, 0, bh, bar);
 }
 
 // Every thread waits (bounded) for the groups in flight on the barriers in `mask`, then the

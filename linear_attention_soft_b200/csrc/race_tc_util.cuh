@@ -199,6 +199,17 @@ __device__ __forceinline__ void tma_load3(uint32_t dst, const CUtensorMap *map, 
         : "memory");
 }
 
+// Box at coordinates (x, y, z, w) of a 4-D tensor map into shared memory at dst.
+__device__ __forceinline__ void tma_load4(uint32_t dst, const CUtensorMap *map, int x, int y, int z, int w,
+                                          uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], [%6];" ::
+            "r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(bar))
+        : "memory");
+}
+
 // Contiguous global -> shared copy of `bytes` (both addresses 16-byte aligned, bytes a
 // multiple of 16); completion counted on `bar`.
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint64_t *bar)
