@@ -265,27 +265,6 @@ __device__ __forceinline__ void publish_smem()
     __syncthreads();
 }
 
-// L2 prefetch of the rows [row0, row0 + n) of up to five [.., 64] bf16 tensors and of up to
-// two per-token fp32 vectors (threads 0..6 each take one), for a chunk ahead of the current one.
-__device__ __forceinline__ void prefetch_chunk(int64_t row0, int n, const __nv_bfloat16 *t0_,
-                                               const __nv_bfloat16 *t1_, const __nv_bfloat16 *t2_,
-                                               const __nv_bfloat16 *t3_, const __nv_bfloat16 *t4_,
-                                               const float *f0, const float *f1 = nullptr)
-{
-    if (n <= 0 || threadIdx.x >= 7) return;
-    const __nv_bfloat16 *ts[5] = {t0_, t1_, t2_, t3_, t4_};
-    if (threadIdx.x < 5) {
-        if (ts[threadIdx.x]) prefetch_l2(ts[threadIdx.x] + row0 * DH, (uint32_t)n * DH * 2u);
-        return;
-    }
-    const float *f = threadIdx.x == 5 ? f0 : f1;
-    if (f) {  // shrink to 16-byte aligned bounds inside the range
-        const uintptr_t lo = ((uintptr_t)(f + row0) + 15u) & ~(uintptr_t)15u;
-        const uintptr_t hi = (uintptr_t)(f + row0 + n) & ~(uintptr_t)15u;
-        if (hi > lo) prefetch_l2((const void *)lo, (uint32_t)(hi - lo));
-    }
-}
-
 // Raw L2 norm of row r of a K128 tile.
 __device__ __forceinline__ float row_norm(const uint8_t *tile, int r)
 {
@@ -942,20 +921,7 @@ __global__ void __launch_bounds__(NTH, 1) tc_agg(const __grid_constant__ BwdArgs
             load_row_scalars(r, r < nv, a.cbuf + base + c0 + r, a.den + base + c0 + r, rowc, rowinv, vag);
         fence_smem_async();
         if (!(ok = wait_group_mma())) break;
-        if (cn < t1) {  // the rows are consumed: the next chunk's rows come in during the features
-            load_x(cn);
-            const int64_t cp = cn + 2 * T;  // and the one after towards L2
-            if (gt < 4 && cp < t1) {
-                const int n = (int)(t1 - cp < T ? t1 - cp : T);
-                if (gt == 0) prefetch_l2(xsrc + (base + cp) * DH, (uint32_t)n * DH * 2u);
-                if (gt == 1) prefetch_l2(vsrc + (base + cp) * DH, (uint32_t)n * DH * 2u);
-                if (MODE == 1 && gt >= 2) {  // den, c_i: 16-byte aligned bounds inside the range
-                    const float *f = (gt == 2 ? a.den : a.cbuf) + base + cp;
-                    const uintptr_t lo = ((uintptr_t)f + 15u) & ~(uintptr_t)15u, hi = (uintptr_t)(f + n) & ~(uintptr_t)15u;
-                    if (hi > lo) prefetch_l2((const void *)lo, (uint32_t)(hi - lo));
-                }
-            }
-        }
+        if (cn < t1) load_x(cn);  // the rows are consumed: the next chunk's rows come in during the features
         {
             const float inv = 1.f / fmaxf(rn[r], kNormEps);
             const float sc = r < nv ? (MODE == 0 ? 1.f : rowinv[r]) : 0.f;
@@ -1047,8 +1013,6 @@ __global__ void __launch_bounds__(NTH, 1) tc_fwd_walk(const __grid_constant__ Ar
                 tma_va(sb + VA, &a.tm_v_va, c, bh, bar);
             }
         }
-        prefetch_chunk(base + c + T, (int)(t1 - c - T < T ? t1 - c - T : T), a.q, causal ? a.k : nullptr,
-                       causal ? a.v : nullptr, nullptr, nullptr, nullptr);
     };
     if (t0 < t1) issue_loads(t0);
     for (int64_t c0 = t0; c0 < t1 && ok; c0 += T) {
@@ -1226,8 +1190,6 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_q_walk(const __grid_constant__ 
                 tma_va(sb + VA, &a.tm_v_va, c, bh, bar);
             }
         }
-        prefetch_chunk(base + c + T, (int)(t1 - c - T < T ? t1 - c - T : T), a.q, a.dout, a.o,
-                       causal ? a.k : nullptr, causal ? a.v : nullptr, a.den);
     };
     auto issue_q = [&](int64_t c) {  // q rows for the projection
         uint64_t *bar = arm_load(ctl, ld, 1, TILE);
@@ -1388,9 +1350,6 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_kv_walk(const __grid_constant__
             tma_va(sb + VA, &a.tm_v_va, c, bh, bar);
             if (causal) tma_va(sb + DOC, &a.tm_do_va, c, bh, bar);
         }
-        if (c - T >= t0)
-            prefetch_chunk(base + c - T, T, a.k, a.v, causal ? a.q : nullptr, causal ? a.dout : nullptr, nullptr,
-                           causal ? a.den : nullptr, causal ? a.cbuf : nullptr);
     };
     auto issue_q = [&](int64_t c) {
         if (causal) {

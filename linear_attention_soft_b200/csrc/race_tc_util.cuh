@@ -93,19 +93,6 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
 }
 
 // 16 consecutive fp32 columns of this thread's lane (warp w reads lanes 32*(w%4)..+31).
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16])
-{
-    uint32_t r[16];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, "
-        "[%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-          "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr));
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
-}
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16])
 {
     asm volatile(
@@ -217,37 +204,6 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
                  "l"(src), "r"(bytes), "r"(smem_u32(bar))
                  : "memory");
-}
-
-// ---- cp.async ---------------------------------------------------------------------------
-// 16-byte async copy global -> shared; src_bytes = 0 zero-fills the destination.
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes)
-{
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
-
-// Rows [0, nvalid) of a [.., 64] bf16 tensor into a [128][64] SW128 tile (zero rows beyond).
-template <int NTH>
-__device__ __forceinline__ void load_tile_async(uint8_t *tile, const __nv_bfloat16 *src, int nvalid)
-{
-    const uint32_t base = smem_u32(tile);
-#pragma unroll
-    for (int k = 0; k < 1024 / NTH; ++k) {
-        const int c = threadIdx.x + NTH * k;
-        const int row = c >> 3, ch = c & 7;
-        const bool ok = row < nvalid;
-        const __nv_bfloat16 *g = src + (ok ? (int64_t)row * 64 + ch * 8 : 0);
-        cp_async16(base + sw128_off(row, ch), g, ok ? 16u : 0u);
-    }
-}
-
-// Bring [p, p + bytes) towards L2 ahead of use (p 16-byte aligned, bytes a multiple of 16).
-__device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes)
-{
-    if (bytes) asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
