@@ -81,10 +81,10 @@ def kernel_work(name: str, w: race_inputs.Workload):
 # profiles/tc_kernels_n1m_ncu_full.md (N = 2^20; traffic grows in proportion to the tokens),
 # valid only for the kernel sources it was taken on.
 NCU_TRAFFIC = {
-    "src_sha1": {"race_tc.cuh": "aff23352c7244a6da8b6fcf923fbf4d532845a48",
-                 "race_tc_util.cuh": "03e99a6c246f135995cac3020fdc856ef380f9fc"},
-    "bytes_per_token": {"tc_agg_kv": 269.6, "tc_fwd_walk": 514.2, "tc_bwd_q_walk": 782.2,
-                        "tc_agg_qdy": 277.3, "tc_bwd_kv_walk": 767.6},
+    "src_sha1": {"race_tc.cuh": "cef874770fb57746d6eb7b4c10ba7f751aa54a04",
+                 "race_tc_util.cuh": "590acb8de31114ff59b949728d33097de70d0401"},
+    "bytes_per_token": {"tc_agg_kv": 269.5, "tc_fwd_walk": 513.9, "tc_bwd_q_walk": 781.8,
+                        "tc_agg_qdy": 278.3, "tc_bwd_kv_walk": 765.3},
 }
 
 
