@@ -8,7 +8,8 @@ import torch
 import linear_attention_soft_b200 as ra
 import oracle
 
-# spec tolerances: normwise max relative error
+# parity tolerances: normwise max relative error (fp32 inputs: fp32 arithmetic; bf16 inputs:
+# bf16 operands with fp32 accumulation)
 TOL = {torch.float32: 1e-4, torch.bfloat16: 2e-2}
 
 

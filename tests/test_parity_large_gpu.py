@@ -13,7 +13,7 @@ a time, plus identities that hold at any size:
   sum_j dv_j = sum_i dO_i; the output ignores the scale of q and k rows, so every
   dq_i is orthogonal to q_i and every dk_j to k_j.
 
-Tolerances are the spec ones (normwise max relative error 2e-2 for bf16).
+Tolerance: normwise max relative error 2e-2 for bf16 inputs (fp32 accumulation).
 """
 import gc
 import json
