@@ -22,7 +22,7 @@ namespace decode {
 constexpr int NT = 256;    // threads per CTA
 constexpr int NW = NT / 32;
 constexpr int CS = 5;      // column slots of 32: d + 1 <= 160
-constexpr int RB = 4;      // state rows a warp loads before it updates them
+constexpr int RB = 8;      // state rows a warp loads before it updates them
 
 struct Args {
     const void *q, *k, *v;  // [BH][d]
@@ -76,8 +76,8 @@ __device__ inline void table_features(const float *x, float rawn, const float *W
         for (int r = 0; r < R; ++r) f[r] = r == rs ? 1.f : 0.f;
 }
 
-// grid (nsplit, BH): rows [m0, m1) of head bh's state.
-template <typename DT>
+// grid (nsplit, BH): rows [m0, m1) of head bh's state.  NS column slots of 32 cover d + 1.
+template <typename DT, int NS>
 __global__ void __launch_bounds__(NT) race_decode_update(Args a)
 {
     extern __shared__ float sm[];
@@ -123,17 +123,17 @@ __global__ void __launch_bounds__(NT) race_decode_update(Args a)
     __syncthreads();
     // H[m] += phi_k[m] v~ and this CTA's share of Y = sum_m phi_q[m] H[m]; warp w takes rows
     // m0 + w, m0 + w + NW, ..., RB of them loaded before any is written back
-    float y[CS];
+    float y[NS];
 #pragma unroll
-    for (int s = 0; s < CS; ++s) y[s] = 0.f;
+    for (int s = 0; s < NS; ++s) y[s] = 0.f;
     float *H = a.state + (int64_t)bh * a.M * D;
     for (int i0 = warp; i0 < m1 - m0; i0 += NW * RB) {
-        float h[RB][CS];
+        float h[RB][NS];
 #pragma unroll
         for (int b = 0; b < RB; ++b) {
             const int i = i0 + b * NW;
 #pragma unroll
-            for (int s = 0; s < CS; ++s) {
+            for (int s = 0; s < NS; ++s) {
                 const int c = lane + 32 * s;
                 h[b][s] = (i < m1 - m0 && c < D) ? H[(int64_t)(m0 + i) * D + c] : 0.f;
             }
@@ -144,7 +144,7 @@ __global__ void __launch_bounds__(NT) race_decode_update(Args a)
             if (i >= m1 - m0) break;
             const float fk = phk[i], fq = phq[i];
 #pragma unroll
-            for (int s = 0; s < CS; ++s) {
+            for (int s = 0; s < NS; ++s) {
                 const int c = lane + 32 * s;
                 if (c < D) {
                     const float hn = fmaf(fk, vt[c], h[b][s]);
@@ -155,7 +155,7 @@ __global__ void __launch_bounds__(NT) race_decode_update(Args a)
         }
     }
 #pragma unroll
-    for (int s = 0; s < CS; ++s) {
+    for (int s = 0; s < NS; ++s) {
         const int c = lane + 32 * s;
         if (c < D) red[warp * D + c] = y[s];
     }
