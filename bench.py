@@ -271,13 +271,14 @@ def run_ours(args, w):
                       dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step(qq=q, kk=k, vv=v, dd=do):
-        ra.race_attn_forward(qq, kk, vv, W, out, den, ctx, w.tau, w.causal, ws_f, stream)
+    def step(qq=q, kk=k, vv=v, dd=do, res=None):
+        o_, den_, dq_, dk_, dv_ = res if res is not None else (out, den, dq, dk, dv)
+        ra.race_attn_forward(qq, kk, vv, W, o_, den_, ctx, w.tau, w.causal, ws_f, stream)
         if args.dw:
-            ra.race_attn_backward_dw(qq, kk, vv, W, out, den, dd, ctx, dq, dk, dv, dW, w.tau, w.causal, ws_b,
+            ra.race_attn_backward_dw(qq, kk, vv, W, o_, den_, dd, ctx, dq_, dk_, dv_, dW, w.tau, w.causal, ws_b,
                                      stream)
         else:
-            ra.race_attn_backward(qq, kk, vv, W, out, den, dd, ctx, dq, dk, dv, w.tau, w.causal,
+            ra.race_attn_backward(qq, kk, vv, W, o_, den_, dd, ctx, dq_, dk_, dv_, w.tau, w.causal,
                                   ws_b, stream)
 
     def barrier():
@@ -310,29 +311,54 @@ def run_ours(args, w):
     tokens_all = B * N * world
 
     # ---- end to end through the C ABI with host buffers --------------------------------
+    # Every step copies its inputs in from pinned host memory and its results out, on their
+    # own streams: step i+1's inputs go in and step i-1's results go out while step i
+    # computes (two device buffer sets, ordered by events).
     host = {n: t.cpu().pin_memory() for n, t in (("q", q), ("k", k), ("v", v), ("do", do))}
     host_out = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
                 for n, t in (("out", out), ("dq", dq), ("dk", dk), ("dv", dv))}
-    dq_in = {n: torch.empty_like(host[n], device=dev) for n in host}
+    dev_in = [{n: torch.empty_like(host[n], device=dev) for n in host} for _ in range(2)]
+    dev_res = [(out, den, dq, dk, dv),
+               (torch.empty_like(out), torch.empty_like(den), torch.empty_like(dq), torch.empty_like(dk),
+                torch.empty_like(dv))]
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = sum(t.numel() * t.element_size() for t in host_out.values())
     e2e_steps = max(2, min(args.steps, 5))
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_done = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
 
-    def e2e_step():
-        for n in host:
-            dq_in[n].copy_(host[n], non_blocking=True)
-        step(dq_in["q"], dq_in["k"], dq_in["v"], dq_in["do"])
-        host_out["out"].copy_(out, non_blocking=True)
-        host_out["dq"].copy_(dq, non_blocking=True)
-        host_out["dk"].copy_(dk, non_blocking=True)
-        host_out["dv"].copy_(dv, non_blocking=True)
+    def e2e_run(n_steps):
+        s_in.wait_stream(stream)  # nothing of the run starts before what the stream already holds
+        for i in range(n_steps):
+            b = i & 1
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(ev_done[b])  # step i-2 has finished reading these inputs
+                for n in host:
+                    dev_in[b][n].copy_(host[n], non_blocking=True)
+                ev_in[b].record(s_in)
+            stream.wait_event(ev_in[b])
+            if i >= 2:
+                stream.wait_event(ev_out[b])    # step i-2's results are out
+            step(dev_in[b]["q"], dev_in[b]["k"], dev_in[b]["v"], dev_in[b]["do"], dev_res[b])
+            ev_done[b].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_done[b])
+                o_, _, dq_, dk_, dv_ = dev_res[b]
+                host_out["out"].copy_(o_, non_blocking=True)
+                host_out["dq"].copy_(dq_, non_blocking=True)
+                host_out["dk"].copy_(dk_, non_blocking=True)
+                host_out["dv"].copy_(dv_, non_blocking=True)
+                ev_out[b].record(s_out)
+        stream.wait_event(ev_out[(n_steps - 1) & 1])
 
-    e2e_step()
+    e2e_run(2)
     torch.cuda.synchronize(dev)
     barrier()
     e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
+    e2e_run(e2e_steps)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
