@@ -30,7 +30,9 @@
  *     RACE_ERR_CUDA (the runtime's own error stays readable with cudaGetLastError()).
  *   - Supported: B, H >= 1; N >= 0 (N = 0 is a no-op); d a multiple of 8 in [8, 128];
  *     1 <= P <= 5; L >= 1 with L * 2^P <= 1024; tau >= 0 and finite; dtype RACE_F32 or
- *     RACE_BF16 (arithmetic is fp32 either way, with fp32 accumulation).
+ *     RACE_BF16.  fp32 inputs are computed in fp32; bf16 inputs of the shape d = 64, L = 16,
+ *     P = 4 run on the tensor cores with bf16 operands (features, the staged statistics,
+ *     W as a bf16 hi + lo pair) and fp32 accumulation, other bf16 shapes in fp32.
  */
 #ifndef RACE_ATTN_H
 #define RACE_ATTN_H
@@ -103,8 +105,8 @@ race_status_t race_attn_forward(const void *q, const void *k, const void *v, con
 /*
  * Backward pass: gradients of sum(out * dout) with respect to q, k and v, by the chain
  * rule through the forward above (the pages state the method is differentiable end to
- * end, es §2.3; they print no gradient formula).  W gets no gradient: it is a fixed
- * random projection (zh §2.2).
+ * end, es §2.3; they print no gradient formula).  W gets no gradient here: it is a fixed
+ * random projection (zh §2.2); race_attn_backward_dw also returns it, for a learned W.
  *   q, k, v, W, out, den   the forward's inputs and outputs (den must not be NULL).
  *   dout       device, [B,H,N,d] of `dtype`.
  *   ctx        NULL, or the buffer a forward call with the same arguments filled.
@@ -131,9 +133,9 @@ race_status_t race_attn_hash_indices(const void *x, const float *W, int32_t *idx
 
 /*
  * Device-side failure report (a robustness aid; the method has no counterpart).  Every wait
- * of the tensor-core kernels on an MMA completion gives up after 2 s; a kernel that gave up
- * skips the rest of its work, releases its tensor memory, returns, and sets a device error
- * word.  race_attn_device_error waits for `stream`, writes that word to *flag (0 = no wait
+ * of the tensor-core kernels on an MMA or load completion gives up after 2 s; a kernel that
+ * gave up skips the rest of its work, waits (again bounded) for its loads in flight, releases
+ * its tensor memory, returns, and sets a device error word.  race_attn_device_error waits for `stream`, writes that word to *flag (0 = no wait
  * ever timed out, 1 = one did) and clears it.
  */
 race_status_t race_attn_device_error(int *flag, race_stream_t stream);
