@@ -83,3 +83,34 @@ def test_one_shard_equals_the_single_call():
     torch.cuda.synchronize()
     for n, ref in (("out", out), ("den", den), ("dq", dq), ("dk", dk), ("dv", dv)):
         assert torch.equal(got[n], ref), n
+
+
+def test_driver_on_one_rank_equals_the_single_call():
+    """linear_attention_soft_b200.sharded through a one-rank NCCL group: the exchange leaves
+    zero statistics from other shards, so the result is the single-call pass bit for bit."""
+    import os
+    import socket
+
+    import torch.distributed as dist
+
+    from linear_attention_soft_b200 import sharded
+
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("nccl", rank=0, world_size=1, device_id=torch.device(DEV, 0))
+    try:
+        inp = race_inputs.small_normal(1, 2, 900, 64, 16, 4, seed=4, dtype=torch.bfloat16, device=DEV)
+        q, k, v, W, do = (inp[n] for n in ("q", "k", "v", "W", "do"))
+        out, den, ctx = sharded.forward(q, k, v, W, 0.5, True)
+        dq, dk, dv = sharded.backward(q, k, v, W, out, den, do, 0.5, True, ctx)
+        ro, rd, rc = ra.forward(q, k, v, W, 0.5, True, save_ctx=True)
+        rq, rk, rv = ra.backward(q, k, v, W, ro, rd, do, 0.5, True, ctx=rc)
+        torch.cuda.synchronize()
+        for a, b in ((out, ro), (den, rd), (dq, rq), (dk, rk), (dv, rv)):
+            assert torch.equal(a, b)
+    finally:
+        dist.destroy_process_group()
