@@ -351,11 +351,11 @@ __device__ __forceinline__ void corner_weights(const float (&t)[16], int l, floa
     float a[4], b[4];
     {
         const float s1a = 0.5f + 0.5f * t[4 * l], s0a = 0.5f - 0.5f * t[4 * l];
-        const float s1b = 0.5f + 0.5f * t[4 * l + 1], s0b = 0.5f - 0.5f * t[4 * l + 1];
-        a[0] = s0a * s0b * scale;
-        a[1] = s1a * s0b * scale;
-        a[2] = s0a * s1b * scale;
-        a[3] = s1a * s1b * scale;
+        const float s1b = (0.5f + 0.5f * t[4 * l + 1]) * scale, s0b = (0.5f - 0.5f * t[4 * l + 1]) * scale;
+        a[0] = s0a * s0b;
+        a[1] = s1a * s0b;
+        a[2] = s0a * s1b;
+        a[3] = s1a * s1b;
     }
     {
         const float s1c = 0.5f + 0.5f * t[4 * l + 2], s0c = 0.5f - 0.5f * t[4 * l + 2];
@@ -454,25 +454,37 @@ __device__ __forceinline__ void features_vjp(uint32_t tm, uint32_t col0, int r, 
 }
 
 // Masked T x T block from TMEM (row r, columns col0 + 32qd ..) to bf16 K128 tile (qd >> 1)
-// of dst.  Adds add_row to every element and add_col[col] per column (optional) before
-// masking; keep_upper keeps column >= row (else column <= row).
-__device__ __forceinline__ void mask_block(uint32_t tm, uint32_t col0, int r, int qd, bool keep_upper,
-                                           float add_row, const float *add_col, uint8_t *dst)
+// of dst.  Adds add_row to every element (ADD_ROW) and add_col[col] per column (ADD_COL)
+// before masking; UPPER keeps column >= row (else column <= row).  A warp's 32 rows and
+// 32 columns lie wholly on one side of the diagonal unless its row block is the quarter's
+// own, so only those warps compare element by element; the warps wholly outside the
+// kept triangle store zeros without reading TMEM.
+template <bool UPPER, bool ADD_ROW, bool ADD_COL>
+__device__ __forceinline__ void mask_block(uint32_t tm, uint32_t col0, int r, int qd, float add_row,
+                                           const float *add_col, uint8_t *dst)
 {
+    const uint32_t blk = smem_u32(dst) + (uint32_t)(qd >> 1) * TILE;
+    const int rb = (int)((threadIdx.x >> 5) & 3);  // this warp's 32-row block
+    const bool all_zero = UPPER ? rb > qd : rb < qd, diag = rb == qd;
+    if (all_zero) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) st_shared_v4(blk + sw128_off(r, 4 * (qd & 1) + c), 0u, 0u, 0u, 0u);
+        return;
+    }
     uint32_t w[2][16];
     tmem_ld16_nowait(tlane(tm, col0 + 32u * qd), w[0]);
     tmem_ld16_nowait(tlane(tm, col0 + 32u * qd + 16u), w[1]);
     tmem_wait_ld();
-    const uint32_t blk = smem_u32(dst) + (uint32_t)(qd >> 1) * TILE;
+    const int lim = r - 32 * qd;  // column offset of the diagonal within this warp's 32 columns
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
         float x[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            const int col = 32 * qd + 8 * c + i;
-            float y = __uint_as_float(w[c >> 1][8 * (c & 1) + i]) + add_row;
-            if (add_col) y += add_col[col];
-            x[i] = (keep_upper ? (col < r) : (col > r)) ? 0.f : y;
+            float y = __uint_as_float(w[c >> 1][8 * (c & 1) + i]);
+            if (ADD_ROW) y += add_row;
+            if (ADD_COL) y += add_col[32 * qd + 8 * c + i];
+            x[i] = (diag && (UPPER ? (8 * c + i < lim) : (8 * c + i > lim))) ? 0.f : y;
         }
         st_shared_v4(blk + sw128_off(r, 4 * (qd & 1) + c), pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]),
                      pack_bf16x2(x[4], x[5]), pack_bf16x2(x[6], x[7]));
@@ -848,8 +860,6 @@ __global__ void __launch_bounds__(NTH, 1) tc_agg(const __grid_constant__ BwdArgs
     // each group decides on its own flag, read only after its own barrier, so that all its
     // threads leave the loop together; the CTA checks both flags after the loops
     volatile uint32_t *gabort = g ? &ctl->abort_b : &ctl->abort;
-    const __nv_bfloat16 *xsrc = MODE == 0 ? a.k : a.q;
-    const __nv_bfloat16 *vsrc = MODE == 0 ? a.v : a.dout;
     const CUtensorMap *xmap = MODE == 0 ? &a.tm_k : &a.tm_q;
     const CUtensorMap *vmap = MODE == 0 ? &a.tm_v_va : &a.tm_do_va;
     const uint32_t tm = kernel_setup(ctl, agg_tmem::NCOLS, a.W, sm + WHI, sm + WLO);
@@ -1055,7 +1065,7 @@ __global__ void __launch_bounds__(NTH, 1) tc_fwd_walk(const __grid_constant__ Ar
         if (threadIdx.x == 0) mma_commit(&ctl->bar);
         if (!(ok = wait_mma(ctl, phase))) break;
         if (causal) {
-            mask_block(tm, fwd_tmem::S, r, qd, false, 0.f, nullptr, sm + SB);  // j <= i
+            mask_block<false, false, false>(tm, fwd_tmem::S, r, qd, 0.f, nullptr, sm + SB);  // j <= i
             publish_smem();
             if (threadIdx.x == 0) {
                 fence_after_sync();
@@ -1239,7 +1249,7 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_q_walk(const __grid_constant__ 
             float uk[16], tk[16];
             proj_tanh(tm, bq_tmem::PROJ + 64, qd, 1.f / fmaxf(rn[128 + r], kNormEps), a.beta, uk, tk);
             write_features(tk, r, qd, valid ? 1.f : 0.f, sm + PHK);
-            mask_block(tm, bq_tmem::P, r, qd, false, c_r, nullptr, sm + PB);  // v_j.dO_i + c_i, j <= i
+            mask_block<false, true, false>(tm, bq_tmem::P, r, qd, c_r, nullptr, sm + PB);  // v_j.dO_i + c_i, j <= i
         }
         publish_smem();
         if (threadIdx.x == 0) {
@@ -1413,8 +1423,8 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_kv_walk(const __grid_constant__
         if (threadIdx.x == 0) mma_commit(&ctl->bar);
         if (!(ok = wait_mma(ctl, phase))) break;
         if (causal) {
-            mask_block(tm, bkv_tmem::ST, r, qd, true, 0.f, nullptr, sm + STB);
-            mask_block(tm, bkv_tmem::PP, r, qd, true, 0.f, rowc, sm + PPB);  // v_j.dO_i + c_i, i >= j
+            mask_block<true, false, false>(tm, bkv_tmem::ST, r, qd, 0.f, nullptr, sm + STB);
+            mask_block<true, false, true>(tm, bkv_tmem::PP, r, qd, 0.f, rowc, sm + PPB);  // v_j.dO_i + c_i, i >= j
         }
         publish_smem();
         if (threadIdx.x == 0) {
