@@ -1085,7 +1085,7 @@ race_status_t race_attn_decode_step(const void *q, const void *k, const void *v,
     a.beta = a.hard ? 0.f : 1.f / tau;
     if (workspace_bytes < (size_t)BH * dp.nsplit * (size_t)a.D * sizeof(float)) return RACE_ERR_WORKSPACE;
     cudaStream_t st = (cudaStream_t)stream;
-    const size_t smem = (size_t)dk::update_smem_floats(d, a.D, dp.rows_per_split) * sizeof(float);
+    const size_t smem = (size_t)dk::update_smem_floats(d, a.D, dp.rows_per_split, P) * sizeof(float);
     const dim3 grid((unsigned)dp.nsplit, (unsigned)BH);
     cudaError_t e = timed("decode_update", st, [&] {
         const bool narrow = a.D <= 96;  // three column slots of 32 cover d + 1
@@ -1102,7 +1102,7 @@ race_status_t race_attn_decode_step(const void *q, const void *k, const void *v,
         }
         return cudaGetLastError();
     });
-    if (e == cudaSuccess)
+    if (e == cudaSuccess && dp.nsplit > 1)  // one split per head writes out_t itself
         e = timed("decode_readout", st, [&] {
             if (dtype == RACE_F32)
                 dk::race_decode_readout<float><<<BH, dk::NT, 0, st>>>(a);

@@ -11,7 +11,14 @@
 // The step is bound by reading and writing H (2 * L*2^P * (d+1) * 4 bytes per head).  The
 // rows of H are split over `nsplit` CTAs per head (grid nsplit x B*H) so that a few heads
 // still fill the GPU; each CTA forms the features of its rows for q_t and k_t, updates its
-// rows and writes its share of Y; a second kernel sums the shares in a fixed order.
+// rows and writes its share of Y; a second kernel sums the shares in a fixed order.  With
+// one CTA per head (many heads) the CTA writes out_t itself and the second kernel is not
+// launched.
+//
+// Features: every warp takes whole rows W_lp (coalesced), dotted with q_t and k_t at once;
+// lane pairs of the butterfly sums then apply the nonlinearity of one projection each, and
+// every thread multiplies out the corner weights of its rows.  So no thread runs a long
+// dependent chain of loads before the first row of H is read.
 #pragma once
 
 #include "race_common.cuh"
@@ -23,12 +30,13 @@ constexpr int NT = 256;    // threads per CTA
 constexpr int NW = NT / 32;
 constexpr int CS = 5;      // column slots of 32: d + 1 <= 160
 constexpr int RB = 8;      // state rows a warp loads before it updates them
+constexpr int PB = 4;      // projections a warp forms together
 
 struct Args {
     const void *q, *k, *v;  // [BH][d]
     const float *W;         // [L][P][d]
     float *state;           // [BH][M][D]
-    float *part;            // [BH][nsplit][D] shares of Y
+    float *part;            // [BH][nsplit][D] shares of Y (unused when nsplit = 1)
     void *out;              // [BH][d]
     float *den;             // [BH] or null
     int d, L, P, M, D;
@@ -37,48 +45,32 @@ struct Args {
     int hard;
 };
 
+// Tables that the rows [m0, m0 + rows_per_split) of one split can touch.
+__host__ __device__ inline int split_tables(int rows_per_split, int P) { return rows_per_split / (1 << P) + 2; }
+
 // Shared memory of race_decode_update, in floats.
-__host__ __device__ inline int update_smem_floats(int d, int D, int rows_per_split)
+__host__ __device__ inline int update_smem_floats(int d, int D, int rows_per_split, int P)
 {
-    return 2 * d + D + 2 + 2 * rows_per_split + NW * D;
+    return 2 * d + D + 2 + 2 * rows_per_split + NW * D + D + 4 * P * split_tables(rows_per_split, P);
 }
 
-// The 2^P corner weights of table l for the normalised row x^ = x / |x| (x in shared
-// memory, rawn = |x|): prod_p sigmoid(2 beta c_rp tanh(W_lp . x^)), or the one-hot sign
-// hash when hard.
-__device__ inline void table_features(const float *x, float rawn, const float *Wl, int P, int d, float beta,
-                                      int hard, float (&f)[32])
+// sigmoid(2 beta c u) for the two signs c = -1, +1 of one projection pr = W_lp . x^, with
+// u = tanh(pr) (zh §2.2); the sign hash (0 / 1 by the sign of pr) when hard.
+__device__ inline float2 corner_pair(float pr, float beta, int hard)
 {
-    const float inv = 1.f / fmaxf(rawn, kNormEps);
-    const int R = 1 << P;
-    f[0] = 1.f;
-    int rs = 0;
-    for (int p = 0; p < P; ++p) {
-        const float *w = Wl + p * d;
-        float s = 0.f;
-        for (int c = 0; c < d; ++c) s = fmaf(w[c], x[c], s);
-        const float pr = s * inv;
-        if (hard) {
-            if (pr > 0.f) rs |= 1 << p;
-            continue;
-        }
-        const float up = tanhf(pr);
-        const float e = expf(-2.f * beta * fabsf(up));
-        const float big = 1.f / (1.f + e), small = e * big;
-        const float s1 = up >= 0.f ? big : small, s0 = up >= 0.f ? small : big;
-        const int h = 1 << p;
-        for (int r = 0; r < h; ++r) {
-            f[r + h] = f[r] * s1;
-            f[r] *= s0;
-        }
+    if (hard) {
+        const float s1 = pr > 0.f ? 1.f : 0.f;
+        return make_float2(1.f - s1, s1);
     }
-    if (hard)
-        for (int r = 0; r < R; ++r) f[r] = r == rs ? 1.f : 0.f;
+    const float up = tanhf(pr);
+    const float e = expf(-2.f * beta * fabsf(up));
+    const float big = 1.f / (1.f + e), small = e * big;
+    return up >= 0.f ? make_float2(small, big) : make_float2(big, small);
 }
 
 // grid (nsplit, BH): rows [m0, m1) of head bh's state.  NS column slots of 32 cover d + 1.
 template <typename DT, int NS>
-__global__ void __launch_bounds__(NT) race_decode_update(Args a)
+__global__ void __launch_bounds__(NT, NS <= 3 ? 4 : 2) race_decode_update(Args a)
 {
     extern __shared__ float sm[];
     const int split = blockIdx.x, bh = blockIdx.y;
@@ -86,8 +78,9 @@ __global__ void __launch_bounds__(NT) race_decode_update(Args a)
     const int d = a.d, D = a.D, P = a.P, R = 1 << P;
     const int m0 = split * a.rows_per_split;
     const int m1 = min(a.M, m0 + a.rows_per_split);
+    const int l0 = m0 / R, nl = m0 < m1 ? (m1 - 1) / R - l0 + 1 : 0;
     float *xq = sm, *xk = xq + d, *vt = xk + d, *nrm = vt + D, *phq = nrm + 2, *phk = phq + a.rows_per_split,
-          *red = phk + a.rows_per_split;
+          *red = phk + a.rows_per_split, *ysm = red + NW * D, *sg = ysm + D;  // sg: [2][nl][P] pairs
     const DT *q = reinterpret_cast<const DT *>(a.q) + (int64_t)bh * d;
     const DT *k = reinterpret_cast<const DT *>(a.k) + (int64_t)bh * d;
     const DT *v = reinterpret_cast<const DT *>(a.v) + (int64_t)bh * d;
@@ -106,19 +99,53 @@ __global__ void __launch_bounds__(NT) race_decode_update(Args a)
         if (lane == 0) nrm[warp] = sqrtf(s);
     }
     __syncthreads();
-    // features of this CTA's rows: one (table, q|k) item per thread
-    if (m0 < m1) {
-        const int l0 = m0 / R, l1 = (m1 - 1) / R;
-        for (int item = tid; item < 2 * (l1 - l0 + 1); item += NT) {
-            const int which = item & 1, l = l0 + (item >> 1);
-            float f[32];
-            table_features(which ? xk : xq, nrm[which], a.W + (int64_t)l * P * d, P, d, a.beta, a.hard, f);
-            float *dst = which ? phk : phq;
-            for (int r = 0; r < R; ++r) {
-                const int m = l * R + r;
-                if (m >= m0 && m < m1) dst[m - m0] = f[r];
+    // projections W_lp . q^ and W_lp . k^ of this CTA's tables: warp w takes PB rows of W at
+    // a time (rows j = w, w + NW, ...), every lane its columns c = lane + 32i
+    const int nproj = nl * P;
+    const float *Wc = a.W + (int64_t)l0 * P * d;
+    const float invq = 1.f / fmaxf(nrm[0], kNormEps), invk = 1.f / fmaxf(nrm[1], kNormEps);
+    for (int j0 = warp; j0 < nproj; j0 += NW * PB) {
+        float s[2 * PB];
+#pragma unroll
+        for (int b = 0; b < 2 * PB; ++b) s[b] = 0.f;
+        for (int c = lane; c < d; c += 32) {
+            const float xqc = xq[c], xkc = xk[c];
+#pragma unroll
+            for (int b = 0; b < PB; ++b) {
+                const int j = j0 + b * NW;
+                const float w = j < nproj ? Wc[(int64_t)j * d + c] : 0.f;
+                s[b] = fmaf(w, xqc, s[b]);
+                s[PB + b] = fmaf(w, xkc, s[PB + b]);
             }
         }
+#pragma unroll
+        for (int b = 0; b < 2 * PB; ++b) s[b] = warp_sum(s[b]);
+        // lane i < 2 PB: sum i (q for i < PB, k above) of row j0 + (i % PB) NW
+        if (lane < 2 * PB) {
+            float x = s[0];
+#pragma unroll
+            for (int b = 1; b < 2 * PB; ++b) x = lane == b ? s[b] : x;
+            const int which = lane >= PB, j = j0 + (lane % PB) * NW;
+            if (j < nproj) {
+                const float2 c2 = corner_pair(x * (which ? invk : invq), a.beta, a.hard);
+                reinterpret_cast<float2 *>(sg)[which * nproj + j] = c2;
+            }
+        }
+    }
+    __syncthreads();
+    // corner weights of this CTA's rows: phi_r = prod_p sigmoid(2 beta c_rp u_p), c_rp the
+    // sign of bit p of r (one-hot when hard)
+    const int nrows = m1 > m0 ? m1 - m0 : 0;
+    for (int i = tid; i < 2 * nrows; i += NT) {
+        const int which = i >= nrows, mi = which ? i - nrows : i;
+        const int m = m0 + mi, rr = m & (R - 1);
+        const float2 *sp = reinterpret_cast<const float2 *>(sg) + which * nproj + (m / R - l0) * P;
+        float f = 1.f;
+        for (int p = 0; p < P; ++p) {
+            const float2 c2 = sp[p];
+            f *= (rr >> p) & 1 ? c2.y : c2.x;
+        }
+        (which ? phk : phq)[mi] = f;
     }
     __syncthreads();
     // H[m] += phi_k[m] v~ and this CTA's share of Y = sum_m phi_q[m] H[m]; warp w takes rows
@@ -163,8 +190,17 @@ __global__ void __launch_bounds__(NT) race_decode_update(Args a)
     for (int c = tid; c < D; c += NT) {
         float t = 0.f;
         for (int w = 0; w < NW; ++w) t += red[w * D + c];
-        a.part[((int64_t)bh * a.nsplit + split) * D + c] = t;
+        if (a.nsplit == 1)
+            ysm[c] = t;
+        else
+            a.part[((int64_t)bh * a.nsplit + split) * D + c] = t;
     }
+    if (a.nsplit != 1) return;
+    __syncthreads();  // one split: out = Y[:d] / Y[d] here (0 where Y[d] = 0)
+    const float dn = ysm[d];
+    DT *out = reinterpret_cast<DT *>(a.out) + (int64_t)bh * d;
+    for (int c = tid; c < d; c += NT) store_as(out + c, dn != 0.f ? ysm[c] / dn : 0.f);
+    if (tid == 0 && a.den) a.den[bh] = dn;
 }
 
 // grid BH: Y = sum of the shares (split order), out = Y[:d] / Y[d] (0 where Y[d] = 0).
