@@ -1088,17 +1088,17 @@ race_status_t race_attn_decode_step(const void *q, const void *k, const void *v,
     const size_t smem = (size_t)dk::update_smem_floats(d, a.D, dp.rows_per_split, P) * sizeof(float);
     const dim3 grid((unsigned)dp.nsplit, (unsigned)BH);
     cudaError_t e = timed("decode_update", st, [&] {
-        const bool narrow = a.D <= 96;  // three column slots of 32 cover d + 1
+        const bool narrow = d <= 64;  // two column slots of 32 cover d (else four: d <= 128)
         if (dtype == RACE_F32) {
             if (narrow)
-                dk::race_decode_update<float, 3><<<grid, dk::NT, smem, st>>>(a);
+                dk::race_decode_update<float, 2><<<grid, dk::NT, smem, st>>>(a);
             else
-                dk::race_decode_update<float, dk::CS><<<grid, dk::NT, smem, st>>>(a);
+                dk::race_decode_update<float, 4><<<grid, dk::NT, smem, st>>>(a);
         } else {
             if (narrow)
-                dk::race_decode_update<__nv_bfloat16, 3><<<grid, dk::NT, smem, st>>>(a);
+                dk::race_decode_update<__nv_bfloat16, 2><<<grid, dk::NT, smem, st>>>(a);
             else
-                dk::race_decode_update<__nv_bfloat16, dk::CS><<<grid, dk::NT, smem, st>>>(a);
+                dk::race_decode_update<__nv_bfloat16, 4><<<grid, dk::NT, smem, st>>>(a);
         }
         return cudaGetLastError();
     });

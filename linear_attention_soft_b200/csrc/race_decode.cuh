@@ -29,7 +29,6 @@ namespace decode {
 constexpr int NT = 256;    // threads per CTA
 constexpr int NW = NT / 32;
 constexpr int CS = 5;      // column slots of 32: d + 1 <= 160
-constexpr int RB = 8;      // state rows a warp loads before it updates them
 constexpr int PB = 4;      // projections a warp forms together
 
 struct Args {
@@ -68,9 +67,9 @@ __device__ inline float2 corner_pair(float pr, float beta, int hard)
     return up >= 0.f ? make_float2(small, big) : make_float2(big, small);
 }
 
-// grid (nsplit, BH): rows [m0, m1) of head bh's state.  NS column slots of 32 cover d + 1.
+// grid (nsplit, BH): rows [m0, m1) of head bh's state.  NS column slots of 32 cover d.
 template <typename DT, int NS>
-__global__ void __launch_bounds__(NT, NS <= 3 ? 4 : 2) race_decode_update(Args a)
+__global__ void __launch_bounds__(NT, NS <= 2 ? 4 : 2) race_decode_update(Args a)
 {
     extern __shared__ float sm[];
     const int split = blockIdx.x, bh = blockIdx.y;
@@ -149,12 +148,15 @@ __global__ void __launch_bounds__(NT, NS <= 3 ? 4 : 2) race_decode_update(Args a
     }
     __syncthreads();
     // H[m] += phi_k[m] v~ and this CTA's share of Y = sum_m phi_q[m] H[m]; warp w takes rows
-    // m0 + w, m0 + w + NW, ..., RB of them loaded before any is written back
-    float y[NS];
+    // m0 + w, m0 + w + NW, ..., RB of them loaded before any is written back.  Columns
+    // c = lane + 32 s (< d) sit in slots; column d (the A statistic) of the batch's row b sits
+    // in lane b.
+    constexpr int RB = NS <= 2 ? 16 : 8;
+    float y[NS], ydn = 0.f;
 #pragma unroll
     for (int s = 0; s < NS; ++s) y[s] = 0.f;
-    float *H = a.state + (int64_t)bh * a.M * D;
-    for (int i0 = warp; i0 < m1 - m0; i0 += NW * RB) {
+    float *H = a.state + ((int64_t)bh * a.M + m0) * D;
+    for (int i0 = warp; i0 < nrows; i0 += NW * RB) {
         float h[RB][NS];
 #pragma unroll
         for (int b = 0; b < RB; ++b) {
@@ -162,30 +164,40 @@ __global__ void __launch_bounds__(NT, NS <= 3 ? 4 : 2) race_decode_update(Args a
 #pragma unroll
             for (int s = 0; s < NS; ++s) {
                 const int c = lane + 32 * s;
-                h[b][s] = (i < m1 - m0 && c < D) ? H[(int64_t)(m0 + i) * D + c] : 0.f;
+                h[b][s] = (i < nrows && c < d) ? H[(int64_t)i * D + c] : 0.f;
             }
         }
+        const int id = i0 + lane * NW;  // this lane's row for column d
+        const bool has_d = lane < RB && id < nrows;
+        const float hd = has_d ? H[(int64_t)id * D + d] : 0.f;
 #pragma unroll
         for (int b = 0; b < RB; ++b) {
             const int i = i0 + b * NW;
-            if (i >= m1 - m0) break;
+            if (i >= nrows) break;
             const float fk = phk[i], fq = phq[i];
 #pragma unroll
             for (int s = 0; s < NS; ++s) {
                 const int c = lane + 32 * s;
-                if (c < D) {
+                if (c < d) {
                     const float hn = fmaf(fk, vt[c], h[b][s]);
-                    H[(int64_t)(m0 + i) * D + c] = hn;
+                    H[(int64_t)i * D + c] = hn;
                     y[s] = fmaf(fq, hn, y[s]);
                 }
             }
+        }
+        if (has_d) {
+            const float hn = fmaf(phk[id], vt[d], hd);
+            H[(int64_t)id * D + d] = hn;
+            ydn = fmaf(phq[id], hn, ydn);
         }
     }
 #pragma unroll
     for (int s = 0; s < NS; ++s) {
         const int c = lane + 32 * s;
-        if (c < D) red[warp * D + c] = y[s];
+        if (c < d) red[warp * D + c] = y[s];
     }
+    ydn = warp_sum(ydn);
+    if (lane == 0) red[warp * D + d] = ydn;
     __syncthreads();
     for (int c = tid; c < D; c += NT) {
         float t = 0.f;
