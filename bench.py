@@ -81,10 +81,10 @@ def kernel_work(name: str, w: race_inputs.Workload):
 # profiles/tc_kernels_n1m_ncu_full.md (N = 2^20; traffic grows in proportion to the tokens),
 # valid only for the kernel sources it was taken on.
 NCU_TRAFFIC = {
-    "src_sha1": {"race_tc.cuh": "cef874770fb57746d6eb7b4c10ba7f751aa54a04",
+    "src_sha1": {"race_tc.cuh": "82d96ff09d7d64b5616df11716bbadee49d126c4",
                  "race_tc_util.cuh": "590acb8de31114ff59b949728d33097de70d0401"},
-    "bytes_per_token": {"tc_agg_kv": 269.5, "tc_fwd_walk": 513.9, "tc_bwd_q_walk": 781.8,
-                        "tc_agg_qdy": 278.3, "tc_bwd_kv_walk": 765.3},
+    "bytes_per_token": {"tc_agg_kv": 271.2, "tc_fwd_walk": 515.6, "tc_bwd_q_walk": 785.3,
+                        "tc_agg_qdy": 280.3, "tc_bwd_kv_walk": 764.9},
 }
 
 
