@@ -593,11 +593,11 @@ __device__ __forceinline__ void store_state40(const float (&hv)[40], float *dst_
 }
 
 // dx = (dX^ - x^ (x^ . dX^)) / max(|x|, eps) for row r, columns 16qd .. 16qd+15; dX^ from
-// TMEM column col0; x from a K128 tile in shared memory if xtile, else from global xrow;
+// TMEM column col0; x from a K128 tile in shared memory if xtile, else the two 16-byte
+// words xpre the caller loaded;
 // the four quarters exchange partial dots.
 __device__ __forceinline__ void write_dx(uint32_t tm, uint32_t col0, int r, int qd, bool valid, float rawn,
-                                         const uint8_t *xtile, const __nv_bfloat16 *xrow, __nv_bfloat16 *dst,
-                                         float *xch)
+                                         const uint8_t *xtile, const uint4 *xpre, __nv_bfloat16 *dst, float *xch)
 {
     uint32_t w[16];
     tmem_ld16_nowait(tlane(tm, col0 + 16u * qd), w);
@@ -608,8 +608,8 @@ __device__ __forceinline__ void write_dx(uint32_t tm, uint32_t col0, int r, int 
             v4[0] = ld_shared_v4(smem_u32(xtile) + sw128_off(r, 2 * qd));
             v4[1] = ld_shared_v4(smem_u32(xtile) + sw128_off(r, 2 * qd + 1));
         } else {
-            v4[0] = reinterpret_cast<const uint4 *>(xrow + 16 * qd)[0];
-            v4[1] = reinterpret_cast<const uint4 *>(xrow + 16 * qd)[1];
+            v4[0] = xpre[0];
+            v4[1] = xpre[1];
         }
 #pragma unroll
         for (int ch = 0; ch < 2; ++ch) {
@@ -1451,15 +1451,20 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_kv_walk(const __grid_constant__
             issue_dxhat(tm + bkv_tmem::DX, sb + DP, sb + WHI, sb + WLO);
             mma_commit(&ctl->bar);
         }
-        if (!(ok = wait_mma(ctl, phase))) break;
-        if (ci > 0) issue_q(c0 - T);
-        write_dx(tm, bkv_tmem::DX, r, qd, valid, raw_k, nullptr, a.k + (base + c0 + r) * DH, a.dk + (base + c0 + r) * DH,
-                 xch);
-        if (causal) {
+        uint4 xk4[2];  // this row's k values (its tile is being reloaded), fetched while dX^ runs
+        if (valid) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(a.k + (base + c0 + r) * DH + 16 * qd);
+            xk4[0] = src[0];
+            xk4[1] = src[1];
+        }
+        if (causal) {  // the updated state is staged while dX^ runs
             float hv[40];
             read_state40(tm, bkv_tmem::GTOP, bkv_tmem::GBOT, qd, hv);
             stage40(hv, 128 * (qd & 1) + r, qd, sm + GS);
         }
+        if (!(ok = wait_mma(ctl, phase))) break;
+        if (ci > 0) issue_q(c0 - T);
+        write_dx(tm, bkv_tmem::DX, r, qd, valid, raw_k, nullptr, xk4, a.dk + (base + c0 + r) * DH, xch);
         publish_smem();
     }
     drain_loads(ctl, ld);
