@@ -63,6 +63,8 @@ def kernel_work(name: str, w: race_inputs.Workload):
     table = {
         "agg_kv": (2 * d * s, 2 * M * D + 2 * LP * d),
         "fwd_walk": (4 * d * s + 4, 4 * M * D + 4 * LP * d),
+        # bidirectional read-out: q in, out and den out
+        "readout": (2 * d * s + 4, 2 * M * D + 2 * LP * d),
         # q, k, v, o, dO, den in; dq and c_i out
         "bwd_q_walk": (6 * d * s + 8, 4 * M * D + 6 * LP * d),
         # q, dO, den, c_i in

@@ -425,6 +425,14 @@ cudaError_t tc_forward(const Plan &p, const void *q, const void *k, const void *
     a.state = states;
     a.state_seg_stride = causal ? (int64_t)p.M * p.D : 0;
     const dim3 grid((unsigned)p.nseg, (unsigned)p.BH);
+    if (!causal) {  // every chunk reads the total state: two chunks in flight per CTA
+        const size_t sm_ro = tc::smem_bytes(tc::ro_smem::TOTAL);
+        if ((e = tc_prepare(tc::tc_readout, sm_ro)) != cudaSuccess) return e;
+        return timed("tc_readout", st, [&] {
+            tc::tc_readout<<<grid, tc::NTH, sm_ro, st>>>(a);
+            return cudaGetLastError();
+        });
+    }
     const size_t sm_walk = tc::smem_bytes(tc::fwd_smem::TOTAL);
     if ((e = tc_prepare(tc::tc_fwd_walk, sm_walk)) != cudaSuccess) return e;
     return timed("tc_fwd_walk", st, [&] {

@@ -1095,6 +1095,138 @@ __global__ void __launch_bounds__(NTH, 1) tc_fwd_walk(const __grid_constant__ Ar
     kernel_teardown(tm, fwd_tmem::NCOLS);
 }
 
+// ------------------------------------------------------------------------------------------
+// Bidirectional read-out (Algorithm 1, zh §2.2): Y_i = Phi(q_i)^T H with the head's total
+// state H, out_i = Y_i[:64] / Y_i[64].  No chunk depends on another, so the CTA's two
+// 256-thread groups take alternate chunks of the segment, as the segment aggregates do:
+// while one group waits for its MMA or its rows, the other forms features.  Both read one
+// bf16 copy of H staged at the start.   grid: nseg x BH
+// ------------------------------------------------------------------------------------------
+namespace ro_smem {
+constexpr uint32_t X = 0;             // q rows [128][64] (per group)
+constexpr uint32_t PHI = TILE;        // Phi_Q [128][256] (per group)
+constexpr uint32_t GROUP = 5 * TILE;  // bytes per group
+constexpr uint32_t HS = 2 * GROUP;    // H as a bf16 value tile [256][80] (5 atoms)
+constexpr uint32_t WHI = HS + 5 * VA256;
+constexpr uint32_t WLO = WHI + 8192;
+constexpr uint32_t RN = WLO + 8192;   // row norms [2][128]
+constexpr uint32_t BAR = RN + 1024;
+constexpr uint32_t TOTAL = BAR + 64;
+}  // namespace ro_smem
+namespace ro_tmem {  // per group, at 256 * group
+constexpr uint32_t PROJ = 0;  // [128][64]
+constexpr uint32_t Y = 64;    // [128][80]
+constexpr uint32_t NCOLS = 512;
+}  // namespace ro_tmem
+
+__global__ void __launch_bounds__(NTH, 1) tc_readout(const __grid_constant__ Args a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = aligned_base(smem_raw);
+    using namespace ro_smem;
+    Ctl *ctl = reinterpret_cast<Ctl *>(sm + BAR);
+    const int seg = blockIdx.x, bh = blockIdx.y;
+    const int g = threadIdx.x >> 8, gt = threadIdx.x & 255;
+    const int r = gt & 127, h = gt >> 7;
+    const bool leader = gt == 0;
+    float *rn = reinterpret_cast<float *>(sm + RN) + 128 * g;
+    const uint32_t sb = smem_u32(sm), gb = sb + (uint32_t)g * GROUP;
+    uint8_t *xg = sm + g * GROUP + X, *phig = sm + g * GROUP + PHI;
+    uint64_t *mbar = g ? &ctl->bar_b : &ctl->bar;
+    volatile uint32_t *gabort = g ? &ctl->abort_b : &ctl->abort;  // as in the segment aggregates
+    const uint32_t tm = kernel_setup(ctl, ro_tmem::NCOLS, a.W, sm + WHI, sm + WLO);
+    const uint32_t tg = tm + 256u * g;  // this group's TMEM columns
+    {  // H into the value tile: quarter qd = 2g + h takes 40 columns of state row 128 (qd & 1) + r
+        const int qd = 2 * g + h, m = 128 * (qd & 1) + r, c0 = 40 * (qd >> 1);
+        const float *src = a.state + (int64_t)bh * a.nseg * MF * DS + seg * a.state_seg_stride + (int64_t)m * DS;
+        float hv[40];
+#pragma unroll
+        for (int i = 0; i < 40; ++i) hv[i] = (c0 + i < DS) ? src[c0 + i] : 0.f;
+        stage40(hv, m, qd, sm + HS);
+    }
+    publish_smem();
+    int64_t t0, t1;
+    seg_bounds(a.seg_len, a.N, seg, t0, t1);
+    const int64_t base = (int64_t)bh * a.N;
+    uint32_t phase = 0;
+    bool ok = true;
+    Loads ld = {};  // barrier g: this group's rows
+    auto load_x = [&](int64_t c) {
+        uint64_t *bar = arm_load(ctl, ld, g, TILE, leader);
+        if (leader) tma_k128(gb + X, &a.tm_q, c, bh, bar);
+    };
+    auto wait_group_mma = [&]() {  // bounded, then the group syncs
+        if (leader && *gabort == 0u && !mbar_wait(mbar, phase & 1u, WAIT_LIMIT_NS)) {
+            *gabort = 1u;
+            atomicExch(&g_tc_error, 1);
+        }
+        ++phase;
+        group_sync(g);
+        fence_after_sync();
+        return *gabort == 0u;
+    };
+    auto wait_group_load = [&]() {
+        if ((ld.pend >> g) & 1u) {
+            if (mbar_wait(&ctl->ld[g], load_parity(ld, g), WAIT_LIMIT_NS)) {
+                ld.pend &= ~(1u << g);
+            } else {
+                *gabort = 1u;
+                atomicExch(&g_tc_error, 1);
+            }
+        }
+        group_sync(g);
+        return *gabort == 0u;
+    };
+    int64_t c0 = t0 + (int64_t)g * T;  // this group's chunks: every other one of the segment
+    if (c0 < t1) load_x(c0);
+    for (; c0 < t1 && ok; c0 += 2 * T) {
+        const int nv = (int)(t1 - c0 < T ? t1 - c0 : T);
+        const bool valid = r < nv;
+        const int64_t cn = c0 + 2 * T;
+        if (!(ok = wait_group_load())) break;
+        if (leader) {  // the projection runs while the row norms are formed
+            fence_after_sync();
+            issue_proj(tg + ro_tmem::PROJ, gb + X, sb + WHI, sb + WLO);
+            mma_commit(mbar);
+        }
+        if (h == 0) rn[r] = row_norm(xg, r);
+        if (!(ok = wait_group_mma())) break;
+        if (cn < t1) load_x(cn);  // the rows are consumed: the next ones come in meanwhile
+        {
+            const float inv = 1.f / fmaxf(rn[r], kNormEps);
+#pragma unroll 1
+            for (int qq = 0; qq < 2; ++qq) {
+                float u[16], t[16];
+                proj_tanh(tg, ro_tmem::PROJ, 2 * h + qq, inv, a.beta, u, t);
+                write_features(t, r, 2 * h + qq, valid ? 1.f : 0.f, phig);
+            }
+        }
+        fence_smem_async();
+        fence_before_sync();
+        group_sync(g);
+        if (leader) {  // Y = Phi_Q H
+            fence_after_sync();
+            issue_k256_va(tg + ro_tmem::Y, gb + PHI, sb + HS, idesc_bf16(128, 80, 0, 1), false);
+            mma_commit(mbar);
+        }
+        if (!(ok = wait_group_mma())) break;
+        {  // out = Y[:, :64] / Y[:, 64]: columns 16 (2h + qq) .. of row r
+            uint32_t dn[16];
+            tmem_ld16_nowait(tlane(tg, ro_tmem::Y + 64), dn);
+            tmem_wait_ld();
+            const float dd = __uint_as_float(dn[0]);
+#pragma unroll 1
+            for (int qq = 0; qq < 2; ++qq)
+                store_row16(tg, ro_tmem::Y, 2 * h + qq, valid, dd != 0.f ? 1.f / dd : 0.f,
+                            a.out + (base + c0 + r) * DH);
+            if (h == 0 && valid && a.den) a.den[base + c0 + r] = dd;
+        }
+        fence_before_sync();  // the read-out of Y precedes the next chunk's MMAs
+    }
+    if (leader && ((ld.pend >> g) & 1u)) mbar_wait(&ctl->ld[g], load_parity(ld, g), WAIT_LIMIT_NS);
+    kernel_teardown(tm, ro_tmem::NCOLS);
+}
+
 // ==========================================================================================
 // Backward.  With c_i = -(dO_i . o_i) and dY_i = [dO_i, c_i] / den_i (the gradient of
 // out_i = Y_i[:64] / Y_i[64] with respect to Y_i):
@@ -1631,8 +1763,12 @@ static_assert(bq_smem::XQ % 1024 == 0 && bq_smem::XK % 1024 == 0 && bq_smem::OT 
 static_assert(bkv_smem::XQ % 1024 == 0 && bkv_smem::XK % 1024 == 0 && bkv_smem::VA % 1024 == 0 &&
                   bkv_smem::DOC % 1024 == 0 && bkv_smem::WHI % 16 == 0,
               "dk/dv walk tiles");
+static_assert(ro_smem::X % 1024 == 0 && ro_smem::PHI % 1024 == 0 && ro_smem::GROUP % 1024 == 0 &&
+                  ro_smem::HS % 1024 == 0 && ro_smem::WHI % 1024 == 0,
+              "read-out tiles");
 static_assert(agg_smem::TOTAL + 1024 <= 232448 && fwd_smem::TOTAL + 1024 <= 232448 &&
-                  bq_smem::TOTAL + 1024 <= 232448 && bkv_smem::TOTAL + 1024 <= 232448,
+                  bq_smem::TOTAL + 1024 <= 232448 && bkv_smem::TOTAL + 1024 <= 232448 &&
+                  ro_smem::TOTAL + 1024 <= 232448,
               "shared memory per CTA");
 
 }  // namespace tc
