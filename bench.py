@@ -83,10 +83,10 @@ def kernel_work(name: str, w: race_inputs.Workload):
 # profiles/tc_kernels_n1m_ncu_full.md (N = 2^20; traffic grows in proportion to the tokens),
 # valid only for the kernel sources it was taken on.
 NCU_TRAFFIC = {
-    "src_sha1": {"race_tc.cuh": "82d96ff09d7d64b5616df11716bbadee49d126c4",
+    "src_sha1": {"race_tc.cuh": "ecc9fd019c9af601a2d2535eafb8e3f135eb257d",
                  "race_tc_util.cuh": "590acb8de31114ff59b949728d33097de70d0401"},
-    "bytes_per_token": {"tc_agg_kv": 271.2, "tc_fwd_walk": 515.6, "tc_bwd_q_walk": 785.3,
-                        "tc_agg_qdy": 280.3, "tc_bwd_kv_walk": 764.9},
+    "bytes_per_token": {"tc_agg_kv": 269.5, "tc_fwd_walk": 513.7, "tc_bwd_q_walk": 782.3,
+                        "tc_agg_qdy": 277.4, "tc_bwd_kv_walk": 766.5, "tc_readout": 213.2},
 }
 
 
@@ -325,7 +325,7 @@ def run_ours(args, w):
                 torch.empty_like(dv))]
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = sum(t.numel() * t.element_size() for t in host_out.values())
-    e2e_steps = max(2, min(args.steps, 5))
+    e2e_steps = max(2, args.steps)  # the same K steps as the device-timed leg
     s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     ev_in = [torch.cuda.Event() for _ in range(2)]
     ev_done = [torch.cuda.Event() for _ in range(2)]
