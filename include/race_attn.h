@@ -158,8 +158,10 @@ race_status_t race_attn_selftest_wait_timeout(int64_t limit_ns, race_stream_t st
  * loads the library holds that buffer until the process exits.
  *   Arguments as race_attn_forward (ctx is not offered).  Returns RACE_ERR_WORKSPACE, having
  *   launched nothing, when race_attn_workspace_size(..., backward = 0) for these sizes
- *   exceeds RACE_NOALLOC_SCRATCH_BYTES (for d = 64 and 2^P = 16, L = 16, that is roughly
- *   B * H * min(N / 512, 296 / (B * H)) segment states of 66.5 KB each).
+ *   exceeds RACE_NOALLOC_SCRATCH_BYTES (for d = 64 and 2^P = 16, L = 16, that is B * H * nseg
+ *   segment states of 66.5 KB each, nseg being the segments the library plans per sequence:
+ *   at most N / 512, usually about (SM count) / (B * H); race_attn_workspace_size gives
+ *   the exact figure).
  *   The first call on each device looks up the buffer's device address (a runtime call
  *   with that device current); make that first call before any stream capture.
  *   All calls share the buffer and it keeps the last call's contents: every element a call

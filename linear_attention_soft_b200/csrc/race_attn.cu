@@ -120,18 +120,31 @@ Plan make_plan(int B, int H, int64_t N, int d, int L, int P)
     p.M = L * p.R;
     p.D = d + 1;
     p.G = (p.M + gk::MG - 1) / gk::MG;
-    // Segments per sequence: about two CTAs per SM over all heads, none shorter than
-    // kMinSegTokens, lengths a multiple of kSegAlign.
-    const int64_t target = 2 * (int64_t)device_sm_count();
-    int64_t nseg = (target + p.BH - 1) / p.BH;
-    const int64_t maxseg = (N + kMinSegTokens - 1) / kMinSegTokens;
-    if (nseg > maxseg) nseg = maxseg;
-    if (nseg < 1) nseg = 1;
-    int64_t len = (N + nseg - 1) / nseg;
-    len = (len + kSegAlign - 1) / kSegAlign * kSegAlign;
-    if (len < kSegAlign) len = kSegAlign;
-    p.seg_len = len;
-    p.nseg = (int)((N + len - 1) / len);
+    // Segments per sequence.  One CTA walks one segment and holds its SM, so a pass takes
+    // ceil(nseg * BH / SMs) waves, each as long as a segment's chunks plus a fixed cost per
+    // CTA (TMEM, W and the start state: about two chunks).  The count that minimises this
+    // is taken, with no segment shorter than kMinSegTokens (unless N is) and lengths a
+    // multiple of kSegAlign; ties go to fewer segments (less scan work).
+    const int64_t sms = device_sm_count();
+    auto seg_len_for = [&](int64_t n) {
+        int64_t len = (N + n - 1) / n;
+        len = (len + kSegAlign - 1) / kSegAlign * kSegAlign;
+        return len < kSegAlign ? kSegAlign : len;
+    };
+    int64_t maxseg = (N + kMinSegTokens - 1) / kMinSegTokens;
+    if (maxseg > 4 * sms) maxseg = 4 * sms;
+    int64_t best_len = seg_len_for(1), best_cost = -1;
+    for (int64_t n = 1; n <= maxseg; ++n) {
+        const int64_t len = seg_len_for(n), segs = (N + len - 1) / len;
+        const int64_t waves = (segs * p.BH + sms - 1) / sms;
+        const int64_t cost = waves * (len / kSegAlign + 2);
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
+            best_len = len;
+        }
+    }
+    p.seg_len = best_len;
+    p.nseg = (int)((N + best_len - 1) / best_len);
     if (p.nseg < 1) p.nseg = 1;
     p.state_elems = (size_t)p.BH * p.nseg * p.M * p.D;
     return p;

@@ -43,7 +43,7 @@ def test_hyperplane_gradient_matches_oracle(dtype, shape, causal):
 
 
 def test_hyperplane_gradient_at_size():
-    """N = 524,288 (4096 chunks over 296 segments) on the tensor-core path, clustered q/k."""
+    """N = 524,288 (4096 chunks over 147 segments) on the tensor-core path, clustered q/k."""
     w = race_inputs.WORKLOADS["c3_causal_n4m_clusters"].with_n(1 << 19)
     inp = race_inputs.make_inputs(w, DEV)
     (dq, dk, dv, dW), _ = _run(inp, w.tau, True)
