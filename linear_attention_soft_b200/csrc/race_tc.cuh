@@ -912,26 +912,34 @@ __global__ void __launch_bounds__(NTH, 1) tc_agg(const __grid_constant__ BwdArgs
         group_sync(g);
     };
     int64_t c0 = t0 + (int64_t)g * T;  // this group's chunks: every other one of the segment
-    if (c0 < t1) {
-        load_x(c0);
-        load_v(c0);
-    }
+    if (c0 < t1) load_x(c0);
+    bool pending = false;  // a state update of this group is in flight
     for (; c0 < t1 && ok; c0 += 2 * T) {
         const int nv = (int)(t1 - c0 < T ? t1 - c0 : T);
         const int64_t cn = c0 + 2 * T;  // this group's next chunk
         if (!(ok = wait_group_load(2 * g))) break;
-        if (leader) {  // the projection runs while the row norms are formed
+        if (leader) {  // the projection runs while the row norms are formed; it completes after
+                       // the previous state update (MMAs complete in order)
             fence_after_sync();
             issue_proj(tg + agg_tmem::PROJ, gb + X, sb + WHI, sb + WLO);
             mma_commit(mbar);
         }
         if (h == 0) rn[r] = row_norm(xg, r);
-        if (MODE == 0 && h == 1) write_col64(vag, r, r < nv ? 1.f : 0.f);
-        if (MODE == 1 && h == 1)
-            load_row_scalars(r, r < nv, a.cbuf + base + c0 + r, a.den + base + c0 + r, rowc, rowinv, vag);
-        fence_smem_async();
+        if (MODE == 1 && h == 1) {  // c_i and 1/den_i (0 beyond the valid rows)
+            float c = 0.f, inv = 0.f;
+            if (r < nv) {
+                c = a.cbuf[base + c0 + r];
+                const float dn = a.den[base + c0 + r];
+                inv = dn != 0.f ? 1.f / dn : 0.f;
+            }
+            rowc[r] = c;
+            rowinv[r] = inv;
+        }
         if (!(ok = wait_group_mma())) break;
+        pending = false;
+        load_v(c0);               // the previous state update has read the value tile
         if (cn < t1) load_x(cn);  // the rows are consumed: the next chunk's rows come in during the features
+        if (h == 1) write_col64(vag, r, MODE == 0 ? (r < nv ? 1.f : 0.f) : rowc[r]);  // [v | 1] or [dO | c]
         {
             const float inv = 1.f / fmaxf(rn[r], kNormEps);
             const float sc = r < nv ? (MODE == 0 ? 1.f : rowinv[r]) : 0.f;
@@ -944,13 +952,15 @@ __global__ void __launch_bounds__(NTH, 1) tc_agg(const __grid_constant__ BwdArgs
         }
         if (!(ok = wait_group_load(2 * g + 1))) break;  // this chunk's values (group-synced)
         publish_group();
-        if (leader) {
+        if (leader) {  // not committed: the next projection's commit covers it
             fence_after_sync();
             issue_state_update(tg, agg_tmem::HTOP, agg_tmem::HBOT, gb + PHI, gb + VA);
-            mma_commit(mbar);
         }
-        if (!(ok = wait_group_mma())) break;
-        if (cn < t1) load_v(cn);
+        pending = true;
+    }
+    if (pending && ok) {  // the group's last state update
+        if (leader) mma_commit(mbar);
+        ok = wait_group_mma();
     }
     drain_loads(ctl, ld);  // thread 0 only; group 1's loads are drained by its own leader
     if (g == 1 && leader)
