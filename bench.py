@@ -81,12 +81,13 @@ def kernel_work(name: str, w: race_inputs.Workload):
 
 # DRAM bytes per token (read + write) per kernel from the ncu capture summarised in
 # profiles/tc_kernels_n1m_ncu_full.md (N = 2^20; traffic grows in proportion to the tokens),
-# valid only for the kernel sources it was taken on.
+# valid only for the kernel sources and the segment planner it was taken on.
 NCU_TRAFFIC = {
-    "src_sha1": {"race_tc.cuh": "ecc9fd019c9af601a2d2535eafb8e3f135eb257d",
-                 "race_tc_util.cuh": "590acb8de31114ff59b949728d33097de70d0401"},
-    "bytes_per_token": {"tc_agg_kv": 269.5, "tc_fwd_walk": 513.7, "tc_bwd_q_walk": 782.3,
-                        "tc_agg_qdy": 277.4, "tc_bwd_kv_walk": 766.5, "tc_readout": 213.2},
+    "src_sha1": {"race_tc.cuh": "a463bede8b6dc60ff685b1df83325cdb4e49d2ec",
+                 "race_tc_util.cuh": "590acb8de31114ff59b949728d33097de70d0401",
+                 "race_attn.cu": "d18b7d867333c53b74e090c8e6ea14a7bfd3a24b"},
+    "bytes_per_token": {"tc_agg_kv": 259.7, "tc_fwd_walk": 504.9, "tc_bwd_q_walk": 772.2,
+                        "tc_agg_qdy": 267.6, "tc_bwd_kv_walk": 756.7, "tc_readout": 215.2},
 }
 
 
