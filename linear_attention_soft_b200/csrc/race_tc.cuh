@@ -257,6 +257,20 @@ __device__ __forceinline__ bool wait_mma(Ctl *ctl, uint32_t &phase)
     return *(volatile uint32_t *)&ctl->abort == 0u;
 }
 
+// Every thread waits (bounded) for the MMAs committed to ctl->bar itself, with no CTA
+// barrier, so no warp waits for another.  Used where what follows reads no shared memory
+// that other threads wrote since the last barrier.  A timeout marks the CTA as given up,
+// which the next synchronised wait reports (the control flow does not depend on it).
+__device__ __forceinline__ void wait_mma_each(Ctl *ctl, uint32_t &phase)
+{
+    if (*(volatile uint32_t *)&ctl->abort == 0u && !mbar_wait(&ctl->bar, phase & 1u, WAIT_LIMIT_NS)) {
+        ctl->abort = 1u;
+        atomicExch(&g_tc_error, 1);
+    }
+    ++phase;
+    fence_after_sync();
+}
+
 // Hand the shared-memory tiles written so far to the tensor core and sync the CTA.
 __device__ __forceinline__ void publish_smem()
 {
@@ -1073,7 +1087,7 @@ __global__ void __launch_bounds__(NTH, 1) tc_fwd_walk(const __grid_constant__ Ar
             }
         }
         if (threadIdx.x == 0) mma_commit(&ctl->bar);
-        if (!(ok = wait_mma(ctl, phase))) break;
+        wait_mma_each(ctl, phase);
         if (causal) {
             mask_block<false, false, false>(tm, fwd_tmem::S, r, qd, 0.f, nullptr, sm + SB);  // j <= i
             publish_smem();
@@ -1083,7 +1097,7 @@ __global__ void __launch_bounds__(NTH, 1) tc_fwd_walk(const __grid_constant__ Ar
                 issue_state_update(tm, fwd_tmem::HTOP, fwd_tmem::HBOT, sb + PHK, sb + VA);  // H += Phi_K^T V~
                 mma_commit(&ctl->bar);
             }
-            if (!(ok = wait_mma(ctl, phase))) break;
+            wait_mma_each(ctl, phase);
         }
         if (c0 + T < t1) issue_loads(c0 + T);  // next rows land while this chunk's results leave
         {  // out = Y[:, :64] / Y[:, 64]: columns 16qd .. 16qd+15 of row r
@@ -1405,7 +1419,7 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_q_walk(const __grid_constant__ 
             }
             mma_commit(&ctl->bar);
         }
-        if (!(ok = wait_mma(ctl, phase))) break;
+        wait_mma_each(ctl, phase);
         if (c0 + T < t1) issue_kv_do(c0 + T);  // Phi_K, V~ and dO are free now
         reload_w();
         // dphi = (D + c_i H_prev[:, 64]) / den_i
@@ -1417,7 +1431,7 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_q_walk(const __grid_constant__ 
             issue_dxhat(tm + bq_tmem::DX, sb + DP, sb + WHI, sb + WLO);
             mma_commit(&ctl->bar);
         }
-        if (!(ok = wait_mma(ctl, phase))) break;
+        wait_mma_each(ctl, phase);
         if (c0 + T < t1) issue_q(c0 + T);  // dP~ is consumed; W stays for the next projection
         wait_loads_nosync(ctl, ld, 4u);     // this chunk's kept q rows
         write_dx(tm, bq_tmem::DX, r, qd, valid, raw_q, sm + XQ2, nullptr, a.dq + (base + c0 + r) * DH, xch);
@@ -1563,7 +1577,7 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_kv_walk(const __grid_constant__
             }
         }
         if (threadIdx.x == 0) mma_commit(&ctl->bar);
-        if (!(ok = wait_mma(ctl, phase))) break;
+        wait_mma_each(ctl, phase);
         if (causal) {
             mask_block<true, false, false>(tm, bkv_tmem::ST, r, qd, 0.f, nullptr, sm + STB);
             mask_block<true, false, true>(tm, bkv_tmem::PP, r, qd, 0.f, rowc, sm + PPB);  // v_j.dO_i + c_i, i >= j
@@ -1581,7 +1595,7 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_kv_walk(const __grid_constant__
             }
             mma_commit(&ctl->bar);
         }
-        if (!(ok = wait_mma(ctl, phase))) break;
+        wait_mma_each(ctl, phase);
         if (ci > 0) issue_kv_do(c0 - T);  // Phi_K / masks, V~ and [dO | c] are free now
         reload_w();
         store_row16(tm, bkv_tmem::DVT, qd, valid, 1.f, a.dv + (base + c0 + r) * DH);
@@ -1604,7 +1618,7 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_kv_walk(const __grid_constant__
             read_state40(tm, bkv_tmem::GTOP, bkv_tmem::GBOT, qd, hv);
             stage40(hv, 128 * (qd & 1) + r, qd, sm + GS);
         }
-        if (!(ok = wait_mma(ctl, phase))) break;
+        wait_mma_each(ctl, phase);
         if (ci > 0) issue_q(c0 - T);
         write_dx(tm, bkv_tmem::DX, r, qd, valid, raw_k, nullptr, xk4, a.dk + (base + c0 + r) * DH, xch);
         publish_smem();
