@@ -83,11 +83,11 @@ def kernel_work(name: str, w: race_inputs.Workload):
 # profiles/tc_kernels_n1m_ncu_full.md (N = 2^20; traffic grows in proportion to the tokens),
 # valid only for the kernel sources and the segment planner it was taken on.
 NCU_TRAFFIC = {
-    "src_sha1": {"race_tc.cuh": "a463bede8b6dc60ff685b1df83325cdb4e49d2ec",
+    "src_sha1": {"race_tc.cuh": "19588ad4a06ec2b36d33e7ca166006aa14986e43",
                  "race_tc_util.cuh": "590acb8de31114ff59b949728d33097de70d0401",
                  "race_attn.cu": "d18b7d867333c53b74e090c8e6ea14a7bfd3a24b"},
-    "bytes_per_token": {"tc_agg_kv": 259.7, "tc_fwd_walk": 504.9, "tc_bwd_q_walk": 772.2,
-                        "tc_agg_qdy": 267.6, "tc_bwd_kv_walk": 756.7, "tc_readout": 215.2},
+    "bytes_per_token": {"tc_agg_kv": 261.3, "tc_fwd_walk": 505.2, "tc_bwd_q_walk": 772.6,
+                        "tc_agg_qdy": 267.6, "tc_bwd_kv_walk": 757.3, "tc_readout": 217.3},
 }
 
 
