@@ -81,24 +81,34 @@ def kernel_work(name: str, w: race_inputs.Workload):
 
 # DRAM bytes per token (read + write) per kernel from the ncu capture summarised in
 # profiles/tc_kernels_n1m_ncu_full.md (N = 2^20; traffic grows in proportion to the tokens),
-# valid only for the kernel sources and the segment planner it was taken on.
+# valid only for the kernel code and the segment planner it was taken on: the sha1 of each
+# source with its comments and whitespace removed.
 NCU_TRAFFIC = {
-    "src_sha1": {"race_tc.cuh": "19588ad4a06ec2b36d33e7ca166006aa14986e43",
-                 "race_tc_util.cuh": "590acb8de31114ff59b949728d33097de70d0401",
-                 "race_attn.cu": "d18b7d867333c53b74e090c8e6ea14a7bfd3a24b"},
+    "code_sha1": {"race_tc.cuh": "3c4244b479fc7fa149759ccbe94acfc59cc6d723",
+                  "race_tc_util.cuh": "f1810754d25d46a51618b9ee942bf40fdca2da55",
+                  "race_attn.cu": "cb5e5418250397230de02e0f99e24c931c3ba18e"},
     "bytes_per_token": {"tc_agg_kv": 261.3, "tc_fwd_walk": 505.2, "tc_bwd_q_walk": 772.6,
                         "tc_agg_qdy": 267.6, "tc_bwd_kv_walk": 757.3, "tc_readout": 217.3},
 }
 
 
+def code_sha1(path: str) -> str:
+    """sha1 of a C++ source without its comments and whitespace (what the compiler sees)."""
+    import hashlib
+    import re
+    src = open(path, encoding="utf-8").read()
+    src = re.sub(r"//[^\n]*", "", src)
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return hashlib.sha1(re.sub(r"\s+", "", src).encode()).hexdigest()
+
+
 def measured_traffic(name: str, tokens: int):
     """DRAM bytes per launch of kernel `name` from the recorded ncu capture, or None when the
-    kernel sources changed since (the counters would describe another kernel)."""
-    import hashlib
+    kernel code changed since (the counters would describe another kernel)."""
     csrc = os.path.join(ROOT, "linear_attention_soft_b200", "csrc")
-    for fn, sha in NCU_TRAFFIC["src_sha1"].items():
+    for fn, sha in NCU_TRAFFIC["code_sha1"].items():
         path = os.path.join(csrc, fn)
-        if not os.path.exists(path) or hashlib.sha1(open(path, "rb").read()).hexdigest() != sha:
+        if not os.path.exists(path) or code_sha1(path) != sha:
             return None
     bpt = NCU_TRAFFIC["bytes_per_token"].get(name)
     return None if bpt is None else bpt * tokens

@@ -15,9 +15,11 @@
 //     out    = Y[:, :64] / Y[:, 64],  den = Y[:, 64]
 //
 // Every GEMM above is a tcgen05.mma with operands in shared memory and the accumulator in
-// tensor memory; one thread issues them and completion is signalled through an mbarrier
-// that one thread polls with a time limit.  One CTA of 512 threads walks one segment of
-// one (b, h) sequence.  Thread t owns token row r = t % 128 (its TMEM lane) and quarter
+// tensor memory; one thread issues them and completion is signalled through an mbarrier,
+// polled with a time limit (by one thread before a CTA barrier where other threads' shared
+// data is read next, else by every thread).  One CTA of 512 threads walks one segment of
+// one (b, h) sequence; the segment aggregates and the bidirectional read-out split the CTA
+// into two 256-thread groups that take alternate chunks.  Thread t owns token row r = t % 128 (its TMEM lane) and quarter
 // qd = t / 128 of every per-row job: tables 4qd .. 4qd+3 (feature block qd), a quarter of
 // the output columns, a quarter of the state rows.
 //
@@ -51,7 +53,7 @@ constexpr uint32_t TILE = 16384;   // one K128 tile
 constexpr uint32_t VA128 = 4096;   // one SW32 atom of 128 rows
 constexpr uint32_t VA256 = 8192;   // one SW32 atom of 256 rows
 
-// error word shared by all launches of this path (1 = an MMA completion wait timed out)
+// error word shared by all launches of this path (1 = an MMA or load completion wait timed out)
 __device__ int g_tc_error;
 
 // Tensor maps: every [B*H][N][64] bf16 tensor is described as a 3-D tensor (64 columns, N
