@@ -71,6 +71,33 @@ def test_workspace_queries(lib):
     assert e.value.status == ra.RACE_ERR_INVALID_ARG
 
 
+
+def _segments(ra, B, H, N):
+    """Segments per sequence the library plans, read off the forward workspace size
+    (B*H*nseg states of [L*R][d+1] fp32 for d = 64, L = 16, P = 4)."""
+    fw = ra.race_attn_workspace_size(B, H, N, 64, 16, 4, 1, 0, ra.RACE_BF16)
+    per = B * H * 256 * 65 * 4
+    assert fw % per == 0
+    return fw // per
+
+
+def test_segment_plan_fills_whole_waves(lib):
+    """One CTA walks one segment and holds its SM, so the planner picks the segment count
+    that wastes the fewest CTA slots: one wave when the heads alone do not fill the GPU."""
+    import torch
+    import linear_attention_soft_b200 as ra
+    sms = torch.cuda.get_device_properties(0).multi_processor_count if torch.cuda.is_available() else 148
+    # one long head: one segment per SM
+    assert _segments(ra, 1, 1, 1 << 22) == sms
+    # 16 heads of 65,536 tokens: one wave (at most sms CTAs), not a nearly empty second one
+    n = _segments(ra, 2, 8, 65536)
+    assert 16 * n <= sms and 16 * (n + 1) > sms
+    # more heads than SMs: one segment each
+    assert _segments(ra, 64, 64, 4096) == 1
+    # never a segment shorter than 512 tokens (unless N is)
+    for N in (1, 300, 1000, 5000, 70000):
+        assert 1 <= _segments(ra, 1, 1, N) <= max(1, -(-N // 512))
+
 def _fwd(lib, **kw):
     a = dict(q=16, k=16, v=16, W=16, out=16, den=16, ctx=None, ctx_bytes=0, B=1, H=1, N=256, d=64,
              L=16, P=4, tau=0.5, causal=1, dtype=1, ws=16, ws_bytes=1 << 40, stream=None)
