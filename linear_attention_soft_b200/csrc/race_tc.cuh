@@ -1088,7 +1088,11 @@ __global__ void __launch_bounds__(NTH, 1) tc_fwd_walk(const __grid_constant__ Ar
                 issue_k256_kk(tm + fwd_tmem::S, sb + PHQ, sb + PHK, idesc_bf16(128, 128, 0, 0), false);
             }
         }
-        if (threadIdx.x == 0) mma_commit(&ctl->bar);
+        if (threadIdx.x == 0) {
+            mma_commit(&ctl->bar);
+            if (causal)  // H += Phi_K^T V~ runs under the masking; the next commit reports it too
+                issue_state_update(tm, fwd_tmem::HTOP, fwd_tmem::HBOT, sb + PHK, sb + VA);
+        }
         wait_mma_each(ctl, phase);
         if (causal) {
             mask_block<false, false, false>(tm, fwd_tmem::S, r, qd, 0.f, nullptr, sm + SB);  // j <= i
@@ -1096,7 +1100,6 @@ __global__ void __launch_bounds__(NTH, 1) tc_fwd_walk(const __grid_constant__ Ar
             if (threadIdx.x == 0) {
                 fence_after_sync();
                 issue_k128_va(tm + fwd_tmem::Y, sb + SB, 0, sb + VA, idesc_bf16(128, 80, 0, 1), true);  // Y += S V~
-                issue_state_update(tm, fwd_tmem::HTOP, fwd_tmem::HBOT, sb + PHK, sb + VA);  // H += Phi_K^T V~
                 mma_commit(&ctl->bar);
             }
             wait_mma_each(ctl, phase);
