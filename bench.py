@@ -84,11 +84,11 @@ def kernel_work(name: str, w: race_inputs.Workload):
 # valid only for the kernel code and the segment planner it was taken on: the sha1 of each
 # source with its comments and whitespace removed.
 NCU_TRAFFIC = {
-    "code_sha1": {"race_tc.cuh": "3c4244b479fc7fa149759ccbe94acfc59cc6d723",
+    "code_sha1": {"race_tc.cuh": "8a4adcc53785c191b40ed6e9f8ebe41bde032597",
                   "race_tc_util.cuh": "f1810754d25d46a51618b9ee942bf40fdca2da55",
                   "race_attn.cu": "cb5e5418250397230de02e0f99e24c931c3ba18e"},
-    "bytes_per_token": {"tc_agg_kv": 261.3, "tc_fwd_walk": 505.2, "tc_bwd_q_walk": 772.6,
-                        "tc_agg_qdy": 267.6, "tc_bwd_kv_walk": 757.3, "tc_readout": 217.3},
+    "bytes_per_token": {"tc_agg_kv": 261.9, "tc_fwd_walk": 501.5, "tc_bwd_q_walk": 768.9,
+                        "tc_agg_qdy": 264.6, "tc_bwd_kv_walk": 753.1, "tc_readout": 217.3},
 }
 
 
