@@ -853,8 +853,10 @@ __device__ __forceinline__ void group_sync(int g)
 // Phi_Q' = Phi_Q / den (the backward's key-side statistics).   grid: nseg x BH
 // The CTA's two groups of 256 threads take the segment's chunks alternately, each with its
 // own tiles, TMEM accumulator and barriers, so that one group's MMA and load waits overlap
-// the other group's feature math; the two partial sums are added at the end.  Thread
-// (r, h) of a group owns token row r and quarters 2h, 2h+1 of the per-row work.
+// the other group's feature math; the two partial sums are added at the end.  A group's
+// state update is not committed on its own: the next chunk's projection commit reports it
+// too, since MMAs complete in issue order.  Thread (r, h) of a group owns token row r and
+// quarters 2h, 2h+1 of the per-row work.
 // ------------------------------------------------------------------------------------------
 template <int MODE>
 __global__ void __launch_bounds__(NTH, 1) tc_agg(const __grid_constant__ BwdArgs a)
