@@ -233,3 +233,23 @@ def test_dw_entry_points_reject_bad_arguments_without_launching(lib):
     args[19] = ctypes.c_float(0.5)
     args[23] = dw - 1
     assert f(*args) == ra.RACE_ERR_WORKSPACE
+
+
+def test_header_is_plain_c_and_links(lib, tmp_path):
+    """A C99 program that includes only the header compiles with gcc -Werror, links against
+    the library and gets the documented statuses back (argument checks launch nothing)."""
+    import shutil
+    import subprocess
+    import linear_attention_soft_b200 as ra
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    libdir = os.path.dirname(ra.library_path())
+    exe = str(tmp_path / "abi_from_c")
+    src = os.path.join(os.path.dirname(__file__), "c", "abi_from_c.c")
+    inc = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", inc, src, "-o", exe, "-L", libdir,
+                    "-l:" + os.path.basename(ra.library_path()), "-Wl,-rpath," + libdir], check=True)
+    p = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert p.returncode == 0, p.stderr
+    assert "abi_from_c ok" in p.stdout
+
