@@ -8,10 +8,13 @@ so no L2 flush is needed between steps).  Prints one JSON line on rank 0.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
-With N > 1 (torchrun) every rank runs its own independent sequence (weak scaling, no
-collective on the data path); the timed region is bracketed by barriers and the time is
-the max over ranks.  ``--impl reference`` times the fp64 CPU oracle instead, on a bounded
-prefix of the same workload, on rank 0 only.
+With N > 1 (torchrun, one process per GPU, NCCL) the ranks run ONE sequence of N times the
+workload's tokens, cut into contiguous slices in rank order, through the sequence-sharded
+passes (one all-gather of per-slice bucket statistics per pass): weak scaling, the tokens
+per rank fixed.  ``--independent`` runs N independent sequences instead (no collective on
+the data path).  The timed region is bracketed by barriers and the time is the max over
+ranks.  ``--impl reference`` times the fp64 CPU oracle instead, on a bounded prefix of the
+same workload, on rank 0 only.
 """
 from __future__ import annotations
 
@@ -79,10 +82,10 @@ def kernel_work(name: str, w: race_inputs.Workload):
     return None
 
 
-# DRAM bytes per token (read + write) per kernel from the ncu capture summarised in
-# profiles/tc_kernels_n1m_ncu_full.md (N = 2^20; traffic grows in proportion to the tokens),
-# valid only for the kernel code and the segment planner it was taken on: the sha1 of each
-# source with its comments and whitespace removed.
+# DRAM bytes per token (dram__bytes_read.sum + dram__bytes_write.sum) per kernel, from one
+# ncu capture of the causal forward + backward at B1 H1 N = 2^20 d64 (traffic grows in
+# proportion to the tokens), valid only for the kernel code and the segment planner it was
+# taken on: the sha1 of each source with its comments and whitespace removed.
 NCU_TRAFFIC = {
     "code_sha1": {"race_tc.cuh": "8a4adcc53785c191b40ed6e9f8ebe41bde032597",
                   "race_tc_util.cuh": "f1810754d25d46a51618b9ee942bf40fdca2da55",
@@ -227,11 +230,30 @@ def run_reference(args, w):
     print(json.dumps(line), flush=True)
 
 
-# ---- multi-rank bookkeeping (weak scaling: one independent sequence per rank) ----------
+# ---- multi-rank bookkeeping ----------------------------------------------------------------
 def rank_workload(w: race_inputs.Workload, rank: int) -> race_inputs.Workload:
-    """The workload rank `rank` runs: same shape, its own seed (independent sequences)."""
+    """The workload rank `rank` runs with --independent: same shape, its own seed."""
     import dataclasses
     return dataclasses.replace(w, seed=w.seed + 1000 * rank)
+
+
+def shard_inputs(w: race_inputs.Workload, rank: int, device):
+    """Rank `rank`'s slice (tokens [rank N, (rank + 1) N) of every head) of one sequence of
+    world * N tokens: the hyperplanes W are the same on every rank, the rows are the slice's
+    own draw."""
+    return race_inputs.make_inputs(w, device, slice_index=rank)
+
+
+def sharded_step(inp, w: race_inputs.Workload, lib=None, events=None):
+    """One forward + backward of this rank's slice through the sequence-sharded passes (one
+    all-gather per pass).  `lib` replaces the CUDA library (a CPU stand-in in the tests);
+    `events` collects CUDA event pairs around each exchange."""
+    from linear_attention_soft_b200 import sharded
+    out, den, ctx = sharded.forward(inp["q"], inp["k"], inp["v"], inp["W"], w.tau, w.causal, lib=lib,
+                                    events=events)
+    dq, dk, dv = sharded.backward(inp["q"], inp["k"], inp["v"], inp["W"], out, den, inp["do"], w.tau,
+                                  w.causal, ctx, lib=lib, events=events)
+    return out, den, dq, dk, dv
 
 
 def job_throughput(ms_local: float, tokens_local: int, world: int, device=None):
@@ -265,8 +287,11 @@ def run_ours(args, w):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
     peaks = load_peaks()
-    # each rank draws its own independent sequence (weak scaling)
-    inp = race_inputs.make_inputs(rank_workload(w, rank), dev)
+    sharded_mode = world > 1 and not args.independent
+    if sharded_mode and args.dw:
+        raise SystemExit("--dw is not offered by the sequence-sharded passes; use --independent")
+    # one sequence sliced over the ranks, or (--independent) one sequence per rank
+    inp = shard_inputs(w, rank, dev) if sharded_mode else race_inputs.make_inputs(rank_workload(w, rank), dev)
     q, k, v, W, do = inp["q"], inp["k"], inp["v"], inp["W"], inp["do"]
     B, H, N, d = q.shape
     L, P = w.L, w.P
@@ -284,7 +309,10 @@ def run_ours(args, w):
                       dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step(qq=q, kk=k, vv=v, dd=do, res=None):
+    def step(qq=q, kk=k, vv=v, dd=do, res=None, events=None):
+        """One forward + backward; returns the five result tensors."""
+        if sharded_mode:
+            return sharded_step({"q": qq, "k": kk, "v": vv, "do": dd, "W": W}, w, events=events)
         o_, den_, dq_, dk_, dv_ = res if res is not None else (out, den, dq, dk, dv)
         ra.race_attn_forward(qq, kk, vv, W, o_, den_, ctx, w.tau, w.causal, ws_f, stream)
         if args.dw:
@@ -293,6 +321,7 @@ def run_ours(args, w):
         else:
             ra.race_attn_backward(qq, kk, vv, W, o_, den_, dd, ctx, dq_, dk_, dv_, w.tau, w.causal,
                                   ws_b, stream)
+        return o_, den_, dq_, dk_, dv_
 
     def barrier():
         if world > 1:
@@ -310,9 +339,10 @@ def run_ours(args, w):
     torch.cuda.synchronize(dev)
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    xevents = [] if sharded_mode else None
     e0.record(stream)
     for _ in range(args.steps):
-        step()
+        step(events=xevents)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
@@ -321,61 +351,70 @@ def run_ours(args, w):
     ms = e0.elapsed_time(e1) / args.steps
     prof = ra.race_attn_profile_read()
     ms_max, value = job_throughput(ms, B * N, world, dev)
-    tokens_all = B * N * world
+    # the exchanges (all-gather + shard-order combine), timed on this rank, max over ranks
+    x_ms_max = None
+    if sharded_mode:
+        x_ms = sum(a.elapsed_time(b) for a, b in xevents) / args.steps
+        x_ms_max = job_throughput(x_ms, 0, world, dev)[0]
 
     # ---- end to end through the C ABI with host buffers --------------------------------
-    # Every step copies its inputs in from pinned host memory and its results out, on their
-    # own streams: step i+1's inputs go in and step i-1's results go out while step i
-    # computes (two device buffer sets, ordered by events).
-    host = {n: t.cpu().pin_memory() for n, t in (("q", q), ("k", k), ("v", v), ("do", do))}
-    host_out = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
-                for n, t in (("out", out), ("dq", dq), ("dk", dk), ("dv", dv))}
-    dev_in = [{n: torch.empty_like(host[n], device=dev) for n in host} for _ in range(2)]
-    dev_res = [(out, den, dq, dk, dv),
-               (torch.empty_like(out), torch.empty_like(den), torch.empty_like(dq), torch.empty_like(dk),
-                torch.empty_like(dv))]
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
-    e2e_steps = max(2, args.steps)  # the same K steps as the device-timed leg
-    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-    ev_in = [torch.cuda.Event() for _ in range(2)]
-    ev_done = [torch.cuda.Event() for _ in range(2)]
-    ev_out = [torch.cuda.Event() for _ in range(2)]
+    e2e_val = h2d = d2h = None
+    if not args.no_e2e:
+        # Every step copies its inputs in from pinned host memory and its results out, on their
+        # own streams: step i+1's inputs go in and step i-1's results go out while step i
+        # computes (two device buffer sets, ordered by events).
+        host = {n: t.cpu().pin_memory() for n, t in (("q", q), ("k", k), ("v", v), ("do", do))}
+        host_out = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+                    for n, t in (("out", out), ("dq", dq), ("dk", dk), ("dv", dv))}
+        dev_in = [{n: torch.empty_like(host[n], device=dev) for n in host} for _ in range(2)]
+        dev_res = [(out, den, dq, dk, dv),
+                   (torch.empty_like(out), torch.empty_like(den), torch.empty_like(dq), torch.empty_like(dk),
+                    torch.empty_like(dv))]
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+        e2e_steps = max(2, args.steps)  # the same K steps as the device-timed leg
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_done = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
 
-    def e2e_run(n_steps):
-        s_in.wait_stream(stream)  # nothing of the run starts before what the stream already holds
-        for i in range(n_steps):
-            b = i & 1
-            with torch.cuda.stream(s_in):
+        def e2e_run(n_steps):
+            s_in.wait_stream(stream)  # nothing of the run starts before what the stream already holds
+            for i in range(n_steps):
+                b = i & 1
+                with torch.cuda.stream(s_in):
+                    if i >= 2:
+                        s_in.wait_event(ev_done[b])  # step i-2 has finished reading these inputs
+                    for n in host:
+                        dev_in[b][n].copy_(host[n], non_blocking=True)
+                    ev_in[b].record(s_in)
+                stream.wait_event(ev_in[b])
                 if i >= 2:
-                    s_in.wait_event(ev_done[b])  # step i-2 has finished reading these inputs
-                for n in host:
-                    dev_in[b][n].copy_(host[n], non_blocking=True)
-                ev_in[b].record(s_in)
-            stream.wait_event(ev_in[b])
-            if i >= 2:
-                stream.wait_event(ev_out[b])    # step i-2's results are out
-            step(dev_in[b]["q"], dev_in[b]["k"], dev_in[b]["v"], dev_in[b]["do"], dev_res[b])
-            ev_done[b].record(stream)
-            with torch.cuda.stream(s_out):
-                s_out.wait_event(ev_done[b])
-                o_, _, dq_, dk_, dv_ = dev_res[b]
-                host_out["out"].copy_(o_, non_blocking=True)
-                host_out["dq"].copy_(dq_, non_blocking=True)
-                host_out["dk"].copy_(dk_, non_blocking=True)
-                host_out["dv"].copy_(dv_, non_blocking=True)
-                ev_out[b].record(s_out)
-        stream.wait_event(ev_out[(n_steps - 1) & 1])
+                    stream.wait_event(ev_out[b])    # step i-2's results are out
+                res = step(dev_in[b]["q"], dev_in[b]["k"], dev_in[b]["v"], dev_in[b]["do"], dev_res[b])
+                ev_done[b].record(stream)
+                with torch.cuda.stream(s_out):
+                    s_out.wait_event(ev_done[b])
+                    o_, _, dq_, dk_, dv_ = res
+                    if sharded_mode:  # the driver's own results, made on the compute stream
+                        for t in res:
+                            t.record_stream(s_out)
+                    host_out["out"].copy_(o_, non_blocking=True)
+                    host_out["dq"].copy_(dq_, non_blocking=True)
+                    host_out["dk"].copy_(dk_, non_blocking=True)
+                    host_out["dv"].copy_(dv_, non_blocking=True)
+                    ev_out[b].record(s_out)
+            stream.wait_event(ev_out[(n_steps - 1) & 1])
 
-    e2e_run(2)
-    torch.cuda.synchronize(dev)
-    barrier()
-    e0.record(stream)
-    e2e_run(e2e_steps)
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier()
-    _, e2e_val = job_throughput(e0.elapsed_time(e1) / e2e_steps, B * N, world, dev)
+        e2e_run(2)
+        torch.cuda.synchronize(dev)
+        barrier()
+        e0.record(stream)
+        e2e_run(e2e_steps)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        _, e2e_val = job_throughput(e0.elapsed_time(e1) / e2e_steps, B * N, world, dev)
 
     # ---- roofline of the dominant kernel and of the whole step ------------------------
     launches = sum(c for _, c in prof.values())
@@ -425,9 +464,14 @@ def run_ours(args, w):
                 "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
                            "L": w.L, "P": w.P, "tau": w.tau, "causal": w.causal,
                            "dist": w.dist, "l2": "inputs larger than L2 (no flush)", "dW": bool(args.dw),
-                           "head_tokens_per_s": B * H * N * world / (ms_max / 1e3)},
-                "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                        "d2h_bytes_per_step": d2h},
+                           "head_tokens_per_s": B * H * N * world / (ms_max / 1e3),
+                           "parallelism": ("sequence sharded over %d ranks (%d tokens each, one all-gather "
+                                           "per pass)" % (world, N)) if sharded_mode else
+                                          ("%d independent sequences" % world if world > 1 else "one GPU"),
+                           "exchange_ms_per_step": x_ms_max,
+                           "exchange_share_of_step": x_ms_max / ms_max if sharded_mode else None},
+                "e2e": None if args.no_e2e else {"value": e2e_val, "unit": "tokens/s",
+                                                  "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
                 "gpu_launches": launches,
                 "roofline": roof, "step_roofline": step_roof,
                 "kernels": {n: {"ms_total": t, "launches": c} for n, (t, c) in prof.items()},
@@ -531,7 +575,12 @@ def main():
                     choices=sorted(race_inputs.WORKLOADS))
     ap.add_argument("--n", type=int, default=0, help="override the sequence length")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true",
+                    help="skip the end-to-end leg (it holds a second device copy of inputs and results)")
     ap.add_argument("--dw", action="store_true", help="also compute the gradient of the hyperplanes W")
+    ap.add_argument("--independent", action="store_true",
+                    help="with several ranks: one independent sequence per rank instead of one "
+                         "sequence sharded over the ranks")
     ap.add_argument("--decode", action="store_true",
                     help="time the streaming decode step instead (one token per head, 4096 heads)")
     args = ap.parse_args()

@@ -20,8 +20,12 @@
  *   - Layout: q, k, v, out, dout, dq, dk, dv are [B, H, N, d] row-major (d fastest),
  *     contiguous; den is [B, H, N]; W is [L, P, d] fp32 and is shared by every (b, h).
  *   - Every pointer named "device" must point to memory of the current CUDA device,
- *     16-byte aligned.  The caller owns all buffers, workspaces included; the library
- *     allocates no memory and keeps no state between calls.
+ *     16-byte aligned.  The caller owns all buffers, workspaces included; no entry point
+ *     allocates memory.  The library's own state is small and fixed: one device error word
+ *     (race_attn_device_error), the kernel timers of race_attn_profile_* (host side, off
+ *     unless enabled), and the fixed device buffer of race_attn_forward_noalloc, which is
+ *     part of the library's device code and is held by every GPU that loads it.  Apart from
+ *     those, nothing persists from one call to the next.
  *   - Execution is asynchronous on `stream` (a cudaStream_t; NULL = legacy default
  *     stream).  Nothing synchronises the host.
  *   - Arguments are validated before anything is launched; a rejected call launches
@@ -163,7 +167,13 @@ race_status_t race_attn_selftest_wait_timeout(int64_t limit_ns, race_stream_t st
  *   at most N / 512, usually about (SM count) / (B * H); race_attn_workspace_size gives
  *   the exact figure).
  *   The first call on each device looks up the buffer's device address (a runtime call
- *   with that device current); make that first call before any stream capture.
+ *   with that device current).  With CUDA's default lazy module loading, that first call is
+ *   also when the library's device code, and with it this buffer, is loaded onto the device,
+ *   so it is the one call that can fail for lack of device memory (RACE_ERR_CUDA).  Make one
+ *   warm-up call at set-up, on every device, before any stream capture and before a host
+ *   framework reserves the device's memory; later calls only reuse the buffer.  The address
+ *   is remembered per device together with the ID of the context it belongs to, so after a
+ *   cudaDeviceReset the next call looks it up again (and is such a first call again).
  *   All calls share the buffer and it keeps the last call's contents: every element a call
  *   reads is first written by the same call, so nothing needs clearing, but calls whose
  *   executions overlap on the GPU (different streams, or several host threads) race on it

@@ -49,16 +49,24 @@ class Library:
         race_attn_shard_combine(gathered, shard, which, out)
 
 
-def exchange(local: torch.Tensor, which: int, group=None, lib=None) -> torch.Tensor:
+def exchange(local: torch.Tensor, which: int, group=None, lib=None, events=None) -> torch.Tensor:
     """All-gather every rank's `local` statistics and return the sum of the ranks selected by
-    `which` (BEFORE, AFTER or OTHERS this rank), in rank order."""
+    `which` (BEFORE, AFTER or OTHERS this rank), in rank order.  With `events` (a list), a
+    pair of CUDA events recorded on the current stream around the exchange is appended, so a
+    caller can time it."""
     lib = lib or Library()
     world = dist.get_world_size(group)
     rank = dist.get_rank(group)
+    if events is not None:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
     gathered = torch.empty((world,) + tuple(local.shape), dtype=local.dtype, device=local.device)
     dist.all_gather(list(gathered.unbind(0)), local.contiguous(), group=group)
     out = torch.empty_like(local)
     lib.combine(gathered, rank, which, out)
+    if events is not None:
+        e1.record()
+        events.append((e0, e1))
     return out
 
 
@@ -67,9 +75,9 @@ def _state_shape(q, W):
     return (B * H, L << P, d + 1)
 
 
-def forward(q, k, v, W, tau: float, causal: bool, group=None, lib=None):
+def forward(q, k, v, W, tau: float, causal: bool, group=None, lib=None, events=None):
     """Forward of this rank's shard ([B, H, n, d]): returns (out, den, ctx); ctx is kept for
-    the backward."""
+    the backward.  `events`: as for exchange."""
     lib = lib or Library()
     B, H, N, d, L, P = _dims(q, W)
     ctx = torch.empty(max(race_attn_ctx_size(B, H, N, d, L, P, causal) // 4, 4), dtype=torch.float32,
@@ -78,15 +86,16 @@ def forward(q, k, v, W, tau: float, causal: bool, group=None, lib=None):
                      dtype=torch.uint8, device=q.device)
     h_total = torch.empty(_state_shape(q, W), dtype=torch.float32, device=q.device)
     lib.forward_begin(k, v, W, ctx, h_total, tau, causal, ws)
-    h_init = exchange(h_total, BEFORE if causal else OTHERS, group, lib)
+    h_init = exchange(h_total, BEFORE if causal else OTHERS, group, lib, events)
     out = torch.empty_like(q)
     den = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
     lib.forward_end(q, k, v, W, h_init, out, den, ctx, tau, causal, ws)
     return out, den, ctx
 
 
-def backward(q, k, v, W, out, den, dout, tau: float, causal: bool, ctx, group=None, lib=None):
-    """Backward of this rank's shard, with the ctx its forward returned: (dq, dk, dv)."""
+def backward(q, k, v, W, out, den, dout, tau: float, causal: bool, ctx, group=None, lib=None, events=None):
+    """Backward of this rank's shard, with the ctx its forward returned: (dq, dk, dv).
+    `events`: as for exchange."""
     lib = lib or Library()
     B, H, N, d, L, P = _dims(q, W)
     ws = torch.empty(max(race_attn_workspace_size(B, H, N, d, L, P, causal, True, _dtype_code(q)), 16),
@@ -94,7 +103,7 @@ def backward(q, k, v, W, out, den, dout, tau: float, causal: bool, ctx, group=No
     dq = torch.empty_like(q)
     g_total = torch.empty(_state_shape(q, W), dtype=torch.float32, device=q.device)
     lib.backward_begin(q, k, v, W, out, den, dout, ctx, dq, g_total, tau, causal, ws)
-    g_init = exchange(g_total, AFTER if causal else OTHERS, group, lib)
+    g_init = exchange(g_total, AFTER if causal else OTHERS, group, lib, events)
     dk, dv = torch.empty_like(k), torch.empty_like(v)
     lib.backward_end(q, k, v, W, out, den, dout, g_init, dk, dv, tau, causal, ws)
     return dq, dk, dv

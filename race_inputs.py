@@ -97,10 +97,13 @@ def _cluster_rows(gen, centres: torch.Tensor, rows: int, device, dtype) -> torch
     return out
 
 
-def make_inputs(w: Workload, device="cpu", with_grad_out: Optional[bool] = None):
+def make_inputs(w: Workload, device="cpu", with_grad_out: Optional[bool] = None, slice_index: int = 0):
     """Draw W, q, k, v (and dO) for workload ``w`` on ``device``.
 
     Sequence tensors are [B, H, N, d] in the workload's dtype; W is [L, P, d] fp32.
+    ``slice_index`` s > 0 draws slice s of a longer sequence cut into slices of N tokens:
+    W (and the cluster centres) as for slice 0, the rows from a generator reseeded with
+    seed + 1000 s.  Slice 0 is the workload itself.
     """
     device = torch.device(device)
     gen = torch.Generator(device=device)
@@ -108,8 +111,12 @@ def make_inputs(w: Workload, device="cpu", with_grad_out: Optional[bool] = None)
     dt = torch_dtype(w)
     rows = w.B * w.H * w.N
     W = torch.randn((w.L, w.P, w.d), generator=gen, device=device, dtype=torch.float32)
+    centres = None
     if w.dist == "clusters":
         centres = torch.randn((256, w.d), generator=gen, device=device, dtype=torch.float32)
+    if slice_index:
+        gen.manual_seed(w.seed + 1000 * slice_index)
+    if w.dist == "clusters":
         q = _cluster_rows(gen, centres, rows, device, dt)
         k = _cluster_rows(gen, centres, rows, device, dt)
     elif w.dist == "normal":

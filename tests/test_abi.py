@@ -253,3 +253,13 @@ def test_header_is_plain_c_and_links(lib, tmp_path):
     assert p.returncode == 0, p.stderr
     assert "abi_from_c ok" in p.stdout
 
+
+
+def test_noalloc_buffer_size_matches_the_header():
+    """The binding's copy of RACE_NOALLOC_SCRATCH_BYTES equals the header's definition (the
+    refusal of larger sizes is tested where a GPU runs the entry point)."""
+    import linear_attention_soft_b200 as ra
+    src = open(os.path.join(ROOT, "include", "race_attn.h")).read()
+    m = re.search(r"#define\s+RACE_NOALLOC_SCRATCH_BYTES\s+\(\(size_t\)(\d+)\s*<<\s*(\d+)\)", src)
+    assert m, "RACE_NOALLOC_SCRATCH_BYTES not found in the header"
+    assert ra.RACE_NOALLOC_SCRATCH_BYTES == int(m.group(1)) << int(m.group(2))
