@@ -449,7 +449,7 @@ cudaError_t tc_forward(const Plan &p, const void *q, const void *k, const void *
     const size_t sm_walk = tc::smem_bytes(tc::fwd_smem::TOTAL);
     if ((e = tc_prepare(tc::tc_fwd_walk, sm_walk)) != cudaSuccess) return e;
     return timed("tc_fwd_walk", st, [&] {
-        tc::tc_fwd_walk<<<grid, tc::NTH, sm_walk, st>>>(a);
+        tc::tc_fwd_walk<<<grid, tc::NTH + 32, sm_walk, st>>>(a);
         return cudaGetLastError();
     });
 }

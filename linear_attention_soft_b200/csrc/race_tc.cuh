@@ -244,10 +244,11 @@ __device__ __forceinline__ void write_col64(uint8_t *tile, int r, float x)
     st_shared_v4(b + sw32_off(r, 1), 0u, 0u, 0u, 0u);
 }
 
-// Wait for the MMAs committed to ctl->bar; one thread polls (bounded), all learn the outcome.
-__device__ __forceinline__ bool wait_mma(Ctl *ctl, uint32_t &phase)
+// Wait for the MMAs committed to ctl->bar; one thread (`poller`) polls (bounded), all learn the
+// outcome.
+__device__ __forceinline__ bool wait_mma(Ctl *ctl, uint32_t &phase, unsigned poller = 0)
 {
-    if (threadIdx.x == 0 && ctl->abort == 0u) {
+    if (threadIdx.x == poller && ctl->abort == 0u) {
         if (!mbar_wait(&ctl->bar, phase & 1u, WAIT_LIMIT_NS)) {
             ctl->abort = 1u;
             atomicExch(&g_tc_error, 1);
@@ -399,6 +400,26 @@ __device__ __forceinline__ void write_features(const float (&t)[16], int r, int 
                      pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
         st_shared_v4(blk + sw128_off(r, 2 * l + 1), pack_bf16x2(f[8], f[9]), pack_bf16x2(f[10], f[11]),
                      pack_bf16x2(f[12], f[13]), pack_bf16x2(f[14], f[15]));
+    }
+}
+
+// This thread's 64 features of row r (feature block qd), times `scale`, as bf16 pairs into
+// its TMEM lane at columns col0 + 32qd .. +31 (feature f of the row at column col0 + f/2,
+// lower half for even f): the A operand layout of a tensor-memory MMA.
+__device__ __forceinline__ void write_features_tmem(const float (&t)[16], int qd, float scale, uint32_t tm,
+                                                    uint32_t col0)
+{
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {  // tables 2h, 2h+1: 16 columns
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            float f[16];
+            corner_weights(t, 2 * h + e, scale, f);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) w[8 * e + c] = pack_bf16x2(f[2 * c], f[2 * c + 1]);
+        }
+        tmem_st16u(tlane(tm, col0 + 32u * qd + 16u * h), w);
     }
 }
 
@@ -678,6 +699,37 @@ __device__ __forceinline__ void store_row16(uint32_t tm, uint32_t col0, int qd, 
                        pack_bf16x2(y[14], y[15]));
 }
 
+// out = Y[:, 16 qq ..] / Y[:, 64] for the quarters qq of `qds` (n of them) of row r, with Y at
+// TMEM column ycol: the quarters' columns and column 64 come in with one TMEM round trip.
+// Returns den = Y[r, 64].
+template <int NQ>
+__device__ __forceinline__ float store_out_quarters(uint32_t tm, uint32_t ycol, const int (&qds)[NQ], bool valid,
+                                                   __nv_bfloat16 *dst)
+{
+    uint32_t w[NQ][16], dn[8];
+#pragma unroll
+    for (int i = 0; i < NQ; ++i) tmem_ld16_nowait(tlane(tm, ycol + 16u * qds[i]), w[i]);
+    tmem_ld8_nowait(tlane(tm, ycol + 64u), dn);
+    tmem_wait_ld();
+    const float d = __uint_as_float(dn[0]);
+    if (valid) {
+        const float2 sc = dup2(d != 0.f ? 1.f / d : 0.f);
+#pragma unroll
+        for (int i = 0; i < NQ; ++i) {
+            uint32_t pk[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const float2 y = mul2(make_float2(__uint_as_float(w[i][2 * k]), __uint_as_float(w[i][2 * k + 1])), sc);
+                pk[k] = pack_bf16x2(y.x, y.y);
+            }
+            uint4 *d4 = reinterpret_cast<uint4 *>(dst + 16 * qds[i]);
+            d4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        }
+    }
+    return d;
+}
+
 // ---- MMA issue helpers (one thread) ------------------------------------------------------
 // Descriptors are built once and advanced by adding (byte offset >> 4) to the start field.
 
@@ -715,6 +767,27 @@ __device__ __forceinline__ void issue_k256_va(uint32_t d, uint32_t a, uint32_t b
         const uint32_t off = ((kk >> 2) * TILE + (kk & 3) * 32) >> 4;
         mma_bf16(d, da + off, db + kk * (512 >> 4), idesc, (kk > 0 || acc_first) ? 1u : 0u);
     }
+}
+
+// D[128][N] (+)= A[128][K=256] B^T with A in TMEM (128 columns of bf16 pairs from a_tmem) and
+// B K-major rows = N (4 K128 tiles).
+__device__ __forceinline__ void issue_k256_tkk(uint32_t d, uint32_t a_tmem, uint32_t b, uint32_t idesc)
+{
+    const uint64_t db = sdesc(b, 16, 1024, LAYOUT_SW128);
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk) {
+        const uint32_t off = ((kk >> 2) * TILE + (kk & 3) * 32) >> 4;
+        mma_bf16_ts(d, a_tmem + 8u * kk, db + off, idesc, kk > 0 ? 1u : 0u);
+    }
+}
+
+// D[128][N] (+)= A[128][K=256] B with A in TMEM and B a value tile MN-major with 256 K-rows
+// (atom stride VA256, N = 16 * natoms).
+__device__ __forceinline__ void issue_k256_tva(uint32_t d, uint32_t a_tmem, uint32_t b, uint32_t idesc)
+{
+    const uint64_t db = sdesc(b, VA256, 256, LAYOUT_SW32);
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk) mma_bf16_ts(d, a_tmem + 8u * kk, db + kk * (512 >> 4), idesc, kk > 0 ? 1u : 0u);
 }
 
 // D[128][N] (+)= A[128][K=128] B with A K-major (2 K128 tiles, a_mn = 0) or MN-major
@@ -780,7 +853,8 @@ constexpr uint32_t RN = WLO + 8192;          // row norms [2][128]
 constexpr uint32_t ROWC = RN + 1024;         // c_i [2][128]
 constexpr uint32_t ROWINV = ROWC + 1024;     // 1 / den_i [2][128]
 constexpr uint32_t BAR = ROWINV + 1024;
-constexpr uint32_t TOTAL = BAR + 64;
+constexpr uint32_t VBAR = BAR + 64;          // per group: its state update is done (value tile free)
+constexpr uint32_t TOTAL = VBAR + 64;
 constexpr uint32_t RED = GROUP;              // at the end: group 1's state, fp32 [256][80]
 static_assert(256 * 80 * 4 <= GROUP, "reduction buffer");
 }  // namespace agg_smem
@@ -792,25 +866,27 @@ constexpr uint32_t NCOLS = 512;
 }  // namespace agg_tmem
 
 namespace fwd_smem {
-constexpr uint32_t PHQ = 0;                  // Phi_Q [128][256]
-constexpr uint32_t XQ = PHQ;                 // q rows during the projection
-constexpr uint32_t XK = PHQ + TILE;          // k rows during the projection
-constexpr uint32_t SB = PHQ;                 // masked S as bf16 [128][128]: 2 tiles
-constexpr uint32_t PHK = PHQ + 4 * TILE;     // Phi_K [128][256]
-constexpr uint32_t HS = PHK + 4 * TILE;      // staged H [256][80] value tile (5 atoms)
-constexpr uint32_t VA = HS + 5 * VA256;      // [V | 1] [128][80]
-constexpr uint32_t WHI = VA + 5 * VA128;
+constexpr uint32_t PHK = 0;                  // Phi_K [128][256]
+constexpr uint32_t SB = 4 * TILE;            // masked S as bf16 [128][128]: 2 tiles
+constexpr uint32_t XQ = SB + 2 * TILE;       // q rows of the next chunk (loaded a chunk ahead)
+constexpr uint32_t XK = XQ + TILE;           // k rows likewise
+constexpr uint32_t VA0 = XK + TILE;          // [V | 1] [128][80], two buffers (chunk parity)
+constexpr uint32_t VA1 = VA0 + 5 * VA128;
+constexpr uint32_t HS = VA1 + 5 * VA128;     // staged H [256][80] value tile (5 atoms)
+constexpr uint32_t WHI = HS + 5 * VA256;
 constexpr uint32_t WLO = WHI + 8192;
 constexpr uint32_t RN = WLO + 8192;          // q norms [128], k norms [128]
 constexpr uint32_t BAR = RN + 1024;
-constexpr uint32_t TOTAL = BAR + 64;
+constexpr uint32_t FB = BAR + 64;            // the walk's own mbarriers (FwdBars)
+constexpr uint32_t TOTAL = FB + 128;
 }  // namespace fwd_smem
 namespace fwd_tmem {
 constexpr uint32_t PROJ = 0;    // [128][64] q projections, [128][64] k projections at +64
 constexpr uint32_t S = 0;       // [128][128] (reuses PROJ once the features are formed)
 constexpr uint32_t Y = 128;     // [128][80]
-constexpr uint32_t HTOP = 256;  // H rows 0..127   [128][80]
-constexpr uint32_t HBOT = 336;  // H rows 128..255 [128][80]
+constexpr uint32_t HTOP = 208;  // H rows 0..127   [128][80]
+constexpr uint32_t HBOT = 288;  // H rows 128..255 [128][80]
+constexpr uint32_t PHQ = 368;   // Phi_Q [128][256] as bf16 pairs (128 columns): the A operand
 constexpr uint32_t NCOLS = 512;
 }  // namespace fwd_tmem
 
@@ -880,6 +956,11 @@ __global__ void __launch_bounds__(NTH, 1) tc_agg(const __grid_constant__ BwdArgs
     volatile uint32_t *gabort = g ? &ctl->abort_b : &ctl->abort;
     const CUtensorMap *xmap = MODE == 0 ? &a.tm_k : &a.tm_q;
     const CUtensorMap *vmap = MODE == 0 ? &a.tm_v_va : &a.tm_do_va;
+    uint64_t *vbar = reinterpret_cast<uint64_t *>(sm + VBAR) + g;
+    if (threadIdx.x == 0) {
+        mbar_init(reinterpret_cast<uint64_t *>(sm + VBAR), 1);
+        mbar_init(reinterpret_cast<uint64_t *>(sm + VBAR) + 1, 1);
+    }
     const uint32_t tm = kernel_setup(ctl, agg_tmem::NCOLS, a.W, sm + WHI, sm + WLO);
     const uint32_t tg = tm + 256u * g;  // this group's TMEM columns
 #pragma unroll
@@ -930,14 +1011,25 @@ __global__ void __launch_bounds__(NTH, 1) tc_agg(const __grid_constant__ BwdArgs
         group_sync(g);
     };
     int64_t c0 = t0 + (int64_t)g * T;  // this group's chunks: every other one of the segment
-    if (c0 < t1) load_x(c0);
+    if (c0 < t1) {
+        load_x(c0);
+        load_v(c0);
+    }
     bool pending = false;  // a state update of this group is in flight
+    uint32_t vphase = 0;   // phase of vbar (waited on by the leader)
     for (; c0 < t1 && ok; c0 += 2 * T) {
         const int nv = (int)(t1 - c0 < T ? t1 - c0 : T);
         const int64_t cn = c0 + 2 * T;  // this group's next chunk
+        if (pending) {  // the value tile comes in as soon as the last state update has read it
+            if (leader && *gabort == 0u && !mbar_wait(vbar, vphase & 1u, WAIT_LIMIT_NS)) {
+                *gabort = 1u;
+                atomicExch(&g_tc_error, 1);
+            }
+            ++vphase;
+            load_v(c0);
+        }
         if (!(ok = wait_group_load(2 * g))) break;
-        if (leader) {  // the projection runs while the row norms are formed; it completes after
-                       // the previous state update (MMAs complete in order)
+        if (leader) {  // the projection runs while the row norms are formed
             fence_after_sync();
             issue_proj(tg + agg_tmem::PROJ, gb + X, sb + WHI, sb + WLO);
             mma_commit(mbar);
@@ -955,7 +1047,6 @@ __global__ void __launch_bounds__(NTH, 1) tc_agg(const __grid_constant__ BwdArgs
         }
         if (!(ok = wait_group_mma())) break;
         pending = false;
-        load_v(c0);               // the previous state update has read the value tile
         if (cn < t1) load_x(cn);  // the rows are consumed: the next chunk's rows come in during the features
         if (h == 1) write_col64(vag, r, MODE == 0 ? (r < nv ? 1.f : 0.f) : rowc[r]);  // [v | 1] or [dO | c]
         {
@@ -970,15 +1061,21 @@ __global__ void __launch_bounds__(NTH, 1) tc_agg(const __grid_constant__ BwdArgs
         }
         if (!(ok = wait_group_load(2 * g + 1))) break;  // this chunk's values (group-synced)
         publish_group();
-        if (leader) {  // not committed: the next projection's commit covers it
+        if (leader) {
             fence_after_sync();
             issue_state_update(tg, agg_tmem::HTOP, agg_tmem::HBOT, gb + PHI, gb + VA);
+            mma_commit(vbar);
         }
         pending = true;
     }
     if (pending && ok) {  // the group's last state update
-        if (leader) mma_commit(mbar);
-        ok = wait_group_mma();
+        if (leader && *gabort == 0u && !mbar_wait(vbar, vphase & 1u, WAIT_LIMIT_NS)) {
+            *gabort = 1u;
+            atomicExch(&g_tc_error, 1);
+        }
+        group_sync(g);
+        fence_after_sync();
+        ok = *gabort == 0u;
     }
     drain_loads(ctl, ld);  // thread 0 only; group 1's loads are drained by its own leader
     if (g == 1 && leader)
@@ -1016,113 +1113,202 @@ __global__ void __launch_bounds__(NTH, 1) tc_agg(const __grid_constant__ BwdArgs
 }
 
 // ------------------------------------------------------------------------------------------
-// Walk: causal (Algorithm 2) or bidirectional read-out (Algorithm 1).  grid: nseg x BH
+// Causal walk (Algorithm 2, zh §2.3).  grid: nseg x BH, NTH + 32 threads.
+// Phi_Q lives in tensor memory as the A operand of S = Phi_Q Phi_K^T and Y = Phi_Q H_prev, so
+// shared memory holds dedicated q / k row tiles and two [V | 1] tiles: every load of the
+// next chunk is issued a whole chunk ahead.  Threads 0..NTH-1 compute; one lane of the last
+// warp issues every TMA load and MMA (an issuing thread is held until the tensor core's queue
+// takes its last MMA, so no computing warp issues).  The two sides hand over through
+// mbarriers: the computing warps arrive (one lane per warp) when a tile is ready, the issuer
+// commits MMAs to barriers the computing threads poll.  The next chunk's projections are
+// issued as soon as the mask has read S (they share its tensor-memory columns), so they run
+// under this chunk's S V~ product and read-out.
 // ------------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(NTH, 1) tc_fwd_walk(const __grid_constant__ Args a)
+struct FwdBars {
+    uint64_t rows, v[2];                     // TMA: q and k rows; value tile p
+    uint64_t proj, s, sv;                    // MMA commits
+    uint64_t norm, phiq, phik, sbar, done;   // the computing warps' hand-overs (16 arrivals)
+};
+static_assert(sizeof(FwdBars) <= 128, "walk barriers");
+
+__global__ void __launch_bounds__(NTH + 32, 1) tc_fwd_walk(const __grid_constant__ Args a)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = aligned_base(smem_raw);
     using namespace fwd_smem;
     Ctl *ctl = reinterpret_cast<Ctl *>(sm + BAR);
+    FwdBars *fb = reinterpret_cast<FwdBars *>(sm + FB);
     float *rn = reinterpret_cast<float *>(sm + RN);
     const int seg = blockIdx.x, bh = blockIdx.y;
-    const int r = threadIdx.x & 127, qd = threadIdx.x >> 7;
+    const bool issuer_warp = threadIdx.x >= NTH;
+    const int r = threadIdx.x & 127, qd = (threadIdx.x >> 7) & 3;
     const uint32_t sb = smem_u32(sm);
-    const bool causal = a.causal != 0;
-    const uint32_t tm = kernel_setup(ctl, fwd_tmem::NCOLS, a.W, sm + WHI, sm + WLO);
-    {  // start state: fp32 master into TMEM, bf16 copy into the staging tile
-        float hv[40];
-        load_state40(a.state + (int64_t)bh * a.nseg * MF * DS + seg * a.state_seg_stride, 128 * (qd & 1) + r, qd,
-                     tm, fwd_tmem::HTOP, fwd_tmem::HBOT, hv);
-        stage40(hv, 128 * (qd & 1) + r, qd, sm + HS);
+    if (threadIdx.x == 0) {
+        mbar_init(&fb->rows, 1);
+        mbar_init(&fb->v[0], 1);
+        mbar_init(&fb->v[1], 1);
+        mbar_init(&fb->proj, 1);
+        mbar_init(&fb->s, 1);
+        mbar_init(&fb->sv, 1);
+        mbar_init(&fb->norm, NTH / 32);
+        mbar_init(&fb->phiq, NTH / 32);
+        mbar_init(&fb->phik, NTH / 32);
+        mbar_init(&fb->sbar, NTH / 32);
+        mbar_init(&fb->done, NTH / 32);
     }
+    const uint32_t tm = kernel_setup(ctl, fwd_tmem::NCOLS, a.W, sm + WHI, sm + WLO);
     int64_t t0, t1;
     seg_bounds(a.seg_len, a.N, seg, t0, t1);
     const int64_t base = (int64_t)bh * a.N;
-    uint32_t phase = 0;
-    bool ok = true;
-    Loads ld = {};
-    auto issue_loads = [&](int64_t c) {
-        uint64_t *bar = arm_load(ctl, ld, 0, (causal ? 3u : 1u) * TILE);
-        if (threadIdx.x == 0) {
-            tma_k128(sb + XQ, &a.tm_q, c, bh, bar);
-            if (causal) {
-                tma_k128(sb + XK, &a.tm_k, c, bh, bar);
-                tma_va(sb + VA, &a.tm_v_va, c, bh, bar);
-            }
+    volatile uint32_t *abort_flag = &ctl->abort;
+    // bounded wait on a barrier phase; a timeout marks the CTA as given up (every later wait
+    // then returns at once) and the walk loops below leave
+    auto wait = [&](uint64_t *bar, uint32_t &ph) {
+        bool good = *abort_flag == 0u && mbar_wait(bar, ph & 1u, WAIT_LIMIT_NS);
+        ++ph;
+        if (!good && *abort_flag == 0u) {
+            *abort_flag = 1u;
+            atomicExch(&g_tc_error, 1);
         }
+        return *abort_flag == 0u;
     };
-    if (t0 < t1) issue_loads(t0);
-    for (int64_t c0 = t0; c0 < t1 && ok; c0 += T) {
-        const int nv = (int)(t1 - c0 < T ? t1 - c0 : T);
-        const bool valid = r < nv;
-        if (!(ok = wait_loads(ctl, ld, 1u))) break;
-        if (threadIdx.x == 0) {  // the projections run while the row norms are formed
-            fence_after_sync();
-            issue_proj(tm + fwd_tmem::PROJ, sb + XQ, sb + WHI, sb + WLO);
-            if (causal) issue_proj(tm + fwd_tmem::PROJ + 64, sb + XK, sb + WHI, sb + WLO);
-            mma_commit(&ctl->bar);
+    if (issuer_warp) {
+        if (threadIdx.x == NTH) {  // the issuing lane
+            uint32_t ph_rows = 0, ph_v[2] = {0, 0}, ph_proj = 0, ph_norm = 0, ph_phiq = 0, ph_phik = 0,
+                     ph_sb = 0, ph_done = 0;
+            auto issue_rows = [&](int64_t c) {
+                mbar_expect_tx(&fb->rows, 2u * TILE);
+                tma_k128(sb + XQ, &a.tm_q, c, bh, &fb->rows);
+                tma_k128(sb + XK, &a.tm_k, c, bh, &fb->rows);
+            };
+            auto issue_v = [&](int64_t c, int p) {
+                mbar_expect_tx(&fb->v[p], TILE);
+                tma_va(sb + (p ? VA1 : VA0), &a.tm_v_va, c, bh, &fb->v[p]);
+            };
+            auto issue_proj_of = [&](int p) {  // the rows and value tile p of the chunk have landed
+                if (!wait(&fb->rows, ph_rows) || !wait(&fb->v[p], ph_v[p])) return false;
+                fence_after_sync();
+                issue_proj(tm + fwd_tmem::PROJ, sb + XQ, sb + WHI, sb + WLO);
+                issue_proj(tm + fwd_tmem::PROJ + 64, sb + XK, sb + WHI, sb + WLO);
+                mma_commit(&fb->proj);
+                return true;
+            };
+            int rows_pending = 0, v_pending[2] = {0, 0};  // TMA groups issued, not yet waited for
+            bool ok = true;
+            if (t0 < t1) {
+                issue_rows(t0);
+                issue_v(t0, 0);
+                rows_pending = 1;
+                v_pending[0] = 1;
+                ok = issue_proj_of(0);
+                rows_pending = v_pending[0] = 0;
+            }
+            int par = 0;
+            for (int64_t c0 = t0; c0 < t1 && ok; c0 += T, par ^= 1) {
+                const bool more = c0 + T < t1;
+                // the q / k rows are read by the projections and the row norms
+                if (!(ok = wait(&fb->norm, ph_norm) && wait(&fb->proj, ph_proj))) break;
+                if (more) {
+                    issue_rows(c0 + T);
+                    issue_v(c0 + T, par ^ 1);  // last read by the previous chunk's MMAs
+                    rows_pending = 1;
+                    v_pending[par ^ 1] = 1;
+                }
+                if (!(ok = wait(&fb->phiq, ph_phiq))) break;
+                fence_after_sync();  // Y = Phi_Q H_prev
+                issue_k256_tva(tm + fwd_tmem::Y, tm + fwd_tmem::PHQ, sb + HS, idesc_bf16(128, 80, 0, 1));
+                if (!(ok = wait(&fb->phik, ph_phik))) break;
+                fence_after_sync();  // S = Phi_Q Phi_K^T, then H += Phi_K^T V~
+                issue_k256_tkk(tm + fwd_tmem::S, tm + fwd_tmem::PHQ, sb + PHK, idesc_bf16(128, 128, 0, 0));
+                mma_commit(&fb->s);
+                issue_state_update(tm, fwd_tmem::HTOP, fwd_tmem::HBOT, sb + PHK, sb + (par ? VA1 : VA0));
+                if (!(ok = wait(&fb->sbar, ph_sb))) break;
+                fence_after_sync();  // Y += tril(S) V~
+                issue_k128_va(tm + fwd_tmem::Y, sb + SB, 0, sb + (par ? VA1 : VA0), idesc_bf16(128, 80, 0, 1), true);
+                mma_commit(&fb->sv);
+                if (more) {  // the next chunk's projections: S has been read, the rows are (being) loaded
+                    ok = issue_proj_of(par ^ 1);
+                    rows_pending = v_pending[par ^ 1] = 0;
+                    if (!ok) break;
+                }
+                if (!(ok = wait(&fb->done, ph_done))) break;
+            }
+            // leave nothing in flight: every MMA issued has been committed; wait (bounded) for
+            // the last commit and for any load group not yet waited for
+            mma_commit(&fb->proj);
+            mbar_wait(&fb->proj, ph_proj & 1u, WAIT_LIMIT_NS);
+            if (rows_pending) mbar_wait(&fb->rows, ph_rows & 1u, WAIT_LIMIT_NS);
+            for (int p = 0; p < 2; ++p)
+                if (v_pending[p]) mbar_wait(&fb->v[p], ph_v[p] & 1u, WAIT_LIMIT_NS);
         }
-        if (qd == 0) rn[r] = row_norm(sm + XQ, r);
-        if (causal && qd == 1) rn[128 + r] = row_norm(sm + XK, r);
-        if (causal && qd == 2) write_col64(sm + VA, r, valid ? 1.f : 0.f);
+    } else {
+        {  // start state: fp32 master into TMEM, bf16 copy into the staging tile
+            float hv[40];
+            load_state40(a.state + (int64_t)bh * a.nseg * MF * DS + seg * a.state_seg_stride, 128 * (qd & 1) + r,
+                         qd, tm, fwd_tmem::HTOP, fwd_tmem::HBOT, hv);
+            stage40(hv, 128 * (qd & 1) + r, qd, sm + HS);
+        }
         fence_smem_async();
-        if (!(ok = wait_mma(ctl, phase))) break;
-        {
-            float u[16], t[16];
-            proj_tanh(tm, fwd_tmem::PROJ, qd, 1.f / fmaxf(rn[r], kNormEps), a.beta, u, t);
-            write_features(t, r, qd, valid ? 1.f : 0.f, sm + PHQ);
-        }
-        publish_smem();
-        if (threadIdx.x == 0) {  // Y = Phi_Q H_prev, while the key features are formed
-            fence_after_sync();
-            issue_k256_va(tm + fwd_tmem::Y, sb + PHQ, sb + HS, idesc_bf16(128, 80, 0, 1), false);
-        }
-        if (causal) {
+        fence_before_sync();
+        asm volatile("bar.sync 1, %0;" ::"n"(NTH) : "memory");  // the staged state before the first Y
+        uint32_t ph_rows = 0, ph_proj = 0, ph_s = 0, ph_sv = 0;
+        const bool elect = (threadIdx.x & 31) == 0;
+        auto hand_over = [&](uint64_t *bar) {  // this warp's writes are complete: one arrival
+            __syncwarp();
+            if (elect) mbar_arrive(bar);
+        };
+        int par = 0;
+        bool ok = true;
+        for (int64_t c0 = t0; c0 < t1 && ok; c0 += T, par ^= 1) {
+            const int nv = (int)(t1 - c0 < T ? t1 - c0 : T);
+            const bool valid = r < nv;
+            if (!(ok = wait(&fb->rows, ph_rows))) break;
+            if (qd == 0) rn[r] = row_norm(sm + XQ, r);
+            if (qd == 1) rn[128 + r] = row_norm(sm + XK, r);
+            if (qd == 2) write_col64(sm + (par ? VA1 : VA0), r, valid ? 1.f : 0.f);
+            fence_smem_async();
+            hand_over(&fb->norm);
+            if (!(ok = wait(&fb->proj, ph_proj))) break;
+            asm volatile("bar.sync 1, %0;" ::"n"(NTH) : "memory");  // the row norms
+            {  // Phi_Q into tensor memory
+                float u[16], t[16];
+                proj_tanh(tm, fwd_tmem::PROJ, qd, 1.f / fmaxf(rn[r], kNormEps), a.beta, u, t);
+                write_features_tmem(t, qd, valid ? 1.f : 0.f, tm, fwd_tmem::PHQ);
+            }
+            tmem_wait_st();
+            fence_before_sync();
+            hand_over(&fb->phiq);
             {
                 float u[16], t[16];
                 proj_tanh(tm, fwd_tmem::PROJ + 64, qd, 1.f / fmaxf(rn[128 + r], kNormEps), a.beta, u, t);
                 write_features(t, r, qd, valid ? 1.f : 0.f, sm + PHK);
             }
-            publish_smem();
-            if (threadIdx.x == 0) {  // S = Phi_Q Phi_K^T
-                fence_after_sync();
-                issue_k256_kk(tm + fwd_tmem::S, sb + PHQ, sb + PHK, idesc_bf16(128, 128, 0, 0), false);
-            }
-        }
-        if (threadIdx.x == 0) {
-            mma_commit(&ctl->bar);
-            if (causal)  // H += Phi_K^T V~ runs under the masking; the next commit reports it too
-                issue_state_update(tm, fwd_tmem::HTOP, fwd_tmem::HBOT, sb + PHK, sb + VA);
-        }
-        wait_mma_each(ctl, phase);
-        if (causal) {
+            fence_smem_async();
+            fence_before_sync();
+            hand_over(&fb->phik);
+            if (!(ok = wait(&fb->s, ph_s))) break;
+            fence_after_sync();
             mask_block<false, false, false>(tm, fwd_tmem::S, r, qd, 0.f, nullptr, sm + SB);  // j <= i
-            publish_smem();
-            if (threadIdx.x == 0) {
-                fence_after_sync();
-                issue_k128_va(tm + fwd_tmem::Y, sb + SB, 0, sb + VA, idesc_bf16(128, 80, 0, 1), true);  // Y += S V~
-                mma_commit(&ctl->bar);
+            fence_smem_async();
+            fence_before_sync();
+            hand_over(&fb->sbar);
+            if (!(ok = wait(&fb->sv, ph_sv))) break;
+            fence_after_sync();
+            {  // out = Y[:, :64] / Y[:, 64]: columns 16qd .. 16qd+15 of row r
+                const int qds[1] = {qd};
+                const float d = store_out_quarters<1>(tm, fwd_tmem::Y, qds, valid, a.out + (base + c0 + r) * DH);
+                if (qd == 0 && valid && a.den) a.den[base + c0 + r] = d;
             }
-            wait_mma_each(ctl, phase);
+            {  // stage the updated state for the next chunk's read-out
+                float hv[40];
+                read_state40(tm, fwd_tmem::HTOP, fwd_tmem::HBOT, qd, hv);
+                stage40(hv, 128 * (qd & 1) + r, qd, sm + HS);
+            }
+            fence_smem_async();
+            fence_before_sync();
+            hand_over(&fb->done);
         }
-        if (c0 + T < t1) issue_loads(c0 + T);  // next rows land while this chunk's results leave
-        {  // out = Y[:, :64] / Y[:, 64]: columns 16qd .. 16qd+15 of row r
-            uint32_t dn[16];
-            tmem_ld16_nowait(tlane(tm, fwd_tmem::Y + 64), dn);
-            tmem_wait_ld();
-            const float d = __uint_as_float(dn[0]);
-            store_row16(tm, fwd_tmem::Y, qd, valid, d != 0.f ? 1.f / d : 0.f, a.out + (base + c0 + r) * DH);
-            if (qd == 0 && valid && a.den) a.den[base + c0 + r] = d;
-        }
-        if (causal) {  // stage the updated state for the next chunk's read-out
-            float hv[40];
-            read_state40(tm, fwd_tmem::HTOP, fwd_tmem::HBOT, qd, hv);
-            stage40(hv, 128 * (qd & 1) + r, qd, sm + HS);
-        }
-        publish_smem();
     }
-    drain_loads(ctl, ld);
     kernel_teardown(tm, fwd_tmem::NCOLS);
 }
 
@@ -1242,14 +1428,8 @@ __global__ void __launch_bounds__(NTH, 1) tc_readout(const __grid_constant__ Arg
         }
         if (!(ok = wait_group_mma())) break;
         {  // out = Y[:, :64] / Y[:, 64]: columns 16 (2h + qq) .. of row r
-            uint32_t dn[16];
-            tmem_ld16_nowait(tlane(tg, ro_tmem::Y + 64), dn);
-            tmem_wait_ld();
-            const float dd = __uint_as_float(dn[0]);
-#pragma unroll 1
-            for (int qq = 0; qq < 2; ++qq)
-                store_row16(tg, ro_tmem::Y, 2 * h + qq, valid, dd != 0.f ? 1.f / dd : 0.f,
-                            a.out + (base + c0 + r) * DH);
+            const int qds[2] = {2 * h, 2 * h + 1};
+            const float dd = store_out_quarters<2>(tg, ro_tmem::Y, qds, valid, a.out + (base + c0 + r) * DH);
             if (h == 0 && valid && a.den) a.den[base + c0 + r] = dd;
         }
         fence_before_sync();  // the read-out of Y precedes the next chunk's MMAs
@@ -1291,12 +1471,12 @@ __device__ __forceinline__ void issue_dxhat(uint32_t d, uint32_t dp, uint32_t wh
 }
 
 namespace bq_smem {
-constexpr uint32_t RA = 0;                 // k rows + o rows at load; Phi_K [128][256] after the features
+constexpr uint32_t RA = 0;                 // k, o, q rows at load; Phi_K [128][256] after the features
 constexpr uint32_t XK = RA;
 constexpr uint32_t OT = RA + TILE;
+constexpr uint32_t XQ = RA + 2 * TILE;
 constexpr uint32_t PHK = RA;
-constexpr uint32_t RB = 4 * TILE;          // q rows + W at load; masked P''; dP~ + W at the end
-constexpr uint32_t XQ = RB;
+constexpr uint32_t RB = 4 * TILE;          // W at load; masked P''; dP~ + W at the end
 constexpr uint32_t PB = RB;
 constexpr uint32_t DP = RB;
 constexpr uint32_t WHI = RB + TILE;
@@ -1353,20 +1533,17 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_q_walk(const __grid_constant__ 
     uint32_t phase = 0;
     bool ok = true;
     Loads ld = {};
-    auto issue_kv_do = [&](int64_t c) {  // k, v, dO, o rows of chunk c
-        uint64_t *bar = arm_load(ctl, ld, 0, (causal ? 4u : 2u) * TILE);
+    auto issue_kv_do = [&](int64_t c) {  // q, k, v, dO, o rows of chunk c
+        uint64_t *bar = arm_load(ctl, ld, 0, (causal ? 5u : 3u) * TILE);
         if (threadIdx.x == 0) {
             tma_va(sb + DOV, &a.tm_do_va, c, bh, bar);
             tma_k128(sb + OT, &a.tm_o, c, bh, bar);
+            tma_k128(sb + XQ, &a.tm_q, c, bh, bar);
             if (causal) {
                 tma_k128(sb + XK, &a.tm_k, c, bh, bar);
                 tma_va(sb + VA, &a.tm_v_va, c, bh, bar);
             }
         }
-    };
-    auto issue_q = [&](int64_t c) {  // q rows for the projection
-        uint64_t *bar = arm_load(ctl, ld, 1, TILE);
-        if (threadIdx.x == 0) tma_k128(sb + XQ, &a.tm_q, c, bh, bar);
     };
     auto issue_q2 = [&](int64_t c) {  // q rows kept for dq
         uint64_t *bar = arm_load(ctl, ld, 2, TILE);
@@ -1378,14 +1555,15 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_q_walk(const __grid_constant__ 
     };
     if (t0 < t1) {
         issue_kv_do(t0);
-        issue_q(t0);
         issue_q2(t0);
     }
     for (int64_t c0 = t0; c0 < t1 && ok; c0 += T) {
         const int nv = (int)(t1 - c0 < T ? t1 - c0 : T);
         const bool valid = r < nv;
-        if (!(ok = wait_loads(ctl, ld, 3u))) break;  // the kept q rows (barrier 2) are waited for at dq
-        if (threadIdx.x == 0) {  // the projections and P'' run while the row scalars are formed
+        if (!(ok = wait_loads(ctl, ld, 1u))) break;  // the kept q rows (barrier 2) are waited for at dq
+        if (threadIdx.x == 3 * 128) {  // the projections and P'' run while quarters 0-2 form the row norms
+                                       // and scalars (a thread issuing MMAs is held until the tensor
+                                       // core's queue takes the last one)
             fence_after_sync();
             issue_proj(tm + bq_tmem::PROJ, sb + XQ, sb + WHI, sb + WLO);
             if (causal) {
@@ -1403,7 +1581,7 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_q_walk(const __grid_constant__ 
         }
         if (causal && qd == 3) write_col64(sm + VA, r, valid ? 1.f : 0.f);
         fence_smem_async();
-        if (!(ok = wait_mma(ctl, phase))) break;
+        if (!(ok = wait_mma(ctl, phase, 3 * 128))) break;
         const float raw_q = rn[r];
         const float c_r = rowc[r], invden_r = rowinv[r];
         float u[16], t[16];
@@ -1427,7 +1605,7 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_q_walk(const __grid_constant__ 
             mma_commit(&ctl->bar);
         }
         wait_mma_each(ctl, phase);
-        if (c0 + T < t1) issue_kv_do(c0 + T);  // Phi_K, V~ and dO are free now
+        if (c0 + T < t1) issue_kv_do(c0 + T);  // Phi_K (where the q, k, o rows go), V~ and dO are free now
         reload_w();
         // dphi = (D + c_i H_prev[:, 64]) / den_i
         features_vjp(tm, bq_tmem::DPHI, r, qd, a.beta, valid, u, t, hden, c_r, invden_r, sm + DP,
@@ -1439,7 +1617,6 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_q_walk(const __grid_constant__ 
             mma_commit(&ctl->bar);
         }
         wait_mma_each(ctl, phase);
-        if (c0 + T < t1) issue_q(c0 + T);  // dP~ is consumed; W stays for the next projection
         wait_loads_nosync(ctl, ld, 4u);     // this chunk's kept q rows
         write_dx(tm, bq_tmem::DX, r, qd, valid, raw_q, sm + XQ2, nullptr, a.dq + (base + c0 + r) * DH, xch);
         __syncthreads();  // every quarter has read its q rows
@@ -1456,13 +1633,13 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_q_walk(const __grid_constant__ 
 }
 
 namespace bkv_smem {
-constexpr uint32_t PHQ = 0;                // q rows (tile 0) + W (tile 1) at load; Phi_Q'; dP~ + W at the end
-constexpr uint32_t XQ = PHQ;
+constexpr uint32_t PHQ = 0;                // W (tile 1) at load; Phi_Q'; dP~ + W at the end
 constexpr uint32_t DP = PHQ;
 constexpr uint32_t WHI = PHQ + TILE;
 constexpr uint32_t WLO = WHI + 8192;
-constexpr uint32_t PHK = PHQ + 4 * TILE;   // k rows at load; Phi_K; then masked S'^T and P'
+constexpr uint32_t PHK = PHQ + 4 * TILE;   // k rows (tile 0), q rows (tile 1) at load; Phi_K; then masked S'^T and P'
 constexpr uint32_t XK = PHK;
+constexpr uint32_t XQ = PHK + TILE;
 constexpr uint32_t STB = PHK;              // tiles 0-1
 constexpr uint32_t PPB = PHK + 2 * TILE;   // tiles 2-3
 constexpr uint32_t VA = PHK + 4 * TILE;    // [V | 1] [128][80]
@@ -1516,54 +1693,45 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_kv_walk(const __grid_constant__
     uint32_t phase = 0;
     bool ok = true;
     Loads ld = {};
-    auto issue_kv_do = [&](int64_t c) {  // k, v, dO rows of chunk c
-        uint64_t *bar = arm_load(ctl, ld, 0, (causal ? 3u : 2u) * TILE);
+    auto issue_kv_do = [&](int64_t c) {  // k, v, dO (and q) rows of chunk c
+        uint64_t *bar = arm_load(ctl, ld, 0, (causal ? 4u : 2u) * TILE);
         if (threadIdx.x == 0) {
             tma_k128(sb + XK, &a.tm_k, c, bh, bar);
             tma_va(sb + VA, &a.tm_v_va, c, bh, bar);
-            if (causal) tma_va(sb + DOC, &a.tm_do_va, c, bh, bar);
-        }
-    };
-    auto issue_q = [&](int64_t c) {
-        if (causal) {
-            uint64_t *bar = arm_load(ctl, ld, 1, TILE);
-            if (threadIdx.x == 0) tma_k128(sb + XQ, &a.tm_q, c, bh, bar);
+            if (causal) {
+                tma_va(sb + DOC, &a.tm_do_va, c, bh, bar);
+                tma_k128(sb + XQ, &a.tm_q, c, bh, bar);
+            }
         }
     };
     auto reload_w = [&]() {  // W tiles (hi, lo) back over Phi_Q'
         uint64_t *bar = arm_load(ctl, ld, 3, 2u * 8192u);
         if (threadIdx.x == 0) bulk_load(sb + WHI, a.wimg, 2u * 8192u, bar);
     };
-    if (nchunks > 0) {
-        issue_kv_do(t0 + (nchunks - 1) * T);
-        issue_q(t0 + (nchunks - 1) * T);
-    }
+    if (nchunks > 0) issue_kv_do(t0 + (nchunks - 1) * T);
     for (int64_t ci = nchunks - 1; ci >= 0 && ok; --ci) {
         const int64_t c0 = t0 + ci * T;
         const int nv = (int)(t1 - c0 < T ? t1 - c0 : T);
         const bool valid = r < nv;
         if (!(ok = wait_loads(ctl, ld, 1u))) break;
-        if (threadIdx.x == 0) {  // key projection and V dO^T run while the row scalars are formed
+        if (threadIdx.x == 3 * 128) {  // projections and V dO^T run while quarters 0-2 form the row norms
+                                       // and scalars (a thread issuing MMAs is held until the tensor
+                                       // core's queue takes the last one)
             fence_after_sync();
             issue_proj(tm + bkv_tmem::PROJ + 64, sb + XK, sb + WHI, sb + WLO);
-            if (causal)  // V dO^T (needs no features)
+            if (causal) {
                 issue_va_va(tm + bkv_tmem::PP, sb + VA, T, sb + DOC, T, 4, idesc_bf16(128, 128, 0, 0), false);
-        }
-        if (qd == 0) rn[128 + r] = row_norm(sm + XK, r);
-        if (causal && qd == 2)
-            load_row_scalars(r, valid, a.cbuf + base + c0 + r, a.den + base + c0 + r, rowc, rowinv, sm + DOC);
-        if (qd == 3) write_col64(sm + VA, r, valid ? 1.f : 0.f);
-        if (causal) {  // the q rows, loaded last, feed the query projection
-            if (!(ok = wait_loads(ctl, ld, 2u))) break;
-            if (threadIdx.x == 0) {
-                fence_after_sync();
                 issue_proj(tm + bkv_tmem::PROJ, sb + XQ, sb + WHI, sb + WLO);
             }
-            if (qd == 1) rn[r] = row_norm(sm + XQ, r);
+            mma_commit(&ctl->bar);
         }
-        if (threadIdx.x == 0) mma_commit(&ctl->bar);
+        if (qd == 0) rn[128 + r] = row_norm(sm + XK, r);
+        if (causal && qd == 1) rn[r] = row_norm(sm + XQ, r);
+        if (causal && qd == 2)
+            load_row_scalars(r, valid, a.cbuf + base + c0 + r, a.den + base + c0 + r, rowc, rowinv, sm + DOC);
+        if (qd == 2) write_col64(sm + VA, r, valid ? 1.f : 0.f);
         fence_smem_async();
-        if (!(ok = wait_mma(ctl, phase))) break;
+        if (!(ok = wait_mma(ctl, phase, 3 * 128))) break;
         const float raw_k = rn[128 + r];
         float u[16], t[16];
         proj_tanh(tm, bkv_tmem::PROJ + 64, qd, 1.f / fmaxf(raw_k, kNormEps), a.beta, u, t);
@@ -1583,6 +1751,7 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_kv_walk(const __grid_constant__
                 issue_k256_kk(tm + bkv_tmem::ST, sb + PHK, sb + PHQ, idesc_bf16(128, 128, 0, 0), false);  // S'^T
             }
         }
+        // the commit reports dV too: it is complete before the masks overwrite Phi_K
         if (threadIdx.x == 0) mma_commit(&ctl->bar);
         wait_mma_each(ctl, phase);
         if (causal) {
@@ -1626,7 +1795,6 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_kv_walk(const __grid_constant__
             stage40(hv, 128 * (qd & 1) + r, qd, sm + GS);
         }
         wait_mma_each(ctl, phase);
-        if (ci > 0) issue_q(c0 - T);
         write_dx(tm, bkv_tmem::DX, r, qd, valid, raw_k, nullptr, xk4, a.dk + (base + c0 + r) * DH, xch);
         publish_smem();
     }
@@ -1786,7 +1954,9 @@ static_assert(agg_smem::X % 1024 == 0 && agg_smem::PHI % 1024 == 0 && agg_smem::
                   agg_smem::GROUP % 1024 == 0,
               "agg tiles");
 static_assert(sizeof(Ctl) <= 64, "control block");
-static_assert(fwd_smem::XQ % 1024 == 0 && fwd_smem::XK % 1024 == 0 && fwd_smem::VA % 1024 == 0, "fwd tiles");
+static_assert(fwd_smem::XQ % 1024 == 0 && fwd_smem::XK % 1024 == 0 && fwd_smem::VA0 % 1024 == 0 &&
+                  fwd_smem::VA1 % 1024 == 0 && fwd_smem::HS % 1024 == 0 && fwd_smem::SB % 1024 == 0,
+              "fwd tiles");
 static_assert(bq_smem::XQ % 1024 == 0 && bq_smem::XK % 1024 == 0 && bq_smem::OT % 1024 == 0 &&
                   bq_smem::XQ2 % 1024 == 0 && bq_smem::VA % 1024 == 0 && bq_smem::DOV % 1024 == 0 &&
                   bq_smem::WHI % 16 == 0,
