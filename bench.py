@@ -63,17 +63,21 @@ def kernel_work(name: str, w: race_inputs.Workload):
     """(algorithmic bytes, algorithmic flops) per token per head of one kernel launch."""
     s = 4 if w.dtype == "f32" else 2
     M, d, LP, D = w.L * w.R, w.d, w.L * w.P, w.d + 1
+    if w.causal:
+        q_walk = (6 * d * s + 8, 4 * M * D + 6 * LP * d)    # q, k, v, o, dO, den in; dq, c_i out
+        kv_walk = (6 * d * s + 8, 6 * M * D + 6 * LP * d)   # q, k, v, dO, den, c_i in; dk, dv out
+    else:  # against the total statistics: no key (query) rows on the query (key) side
+        q_walk = (4 * d * s + 8, 2 * M * D + 4 * LP * d)    # q, o, dO, den in; dq, c_i out
+        kv_walk = (4 * d * s, 4 * M * D + 4 * LP * d)       # k, v in; dk, dv out
     table = {
         "agg_kv": (2 * d * s, 2 * M * D + 2 * LP * d),
         "fwd_walk": (4 * d * s + 4, 4 * M * D + 4 * LP * d),
         # bidirectional read-out: q in, out and den out
         "readout": (2 * d * s + 4, 2 * M * D + 2 * LP * d),
-        # q, k, v, o, dO, den in; dq and c_i out
-        "bwd_q_walk": (6 * d * s + 8, 4 * M * D + 6 * LP * d),
+        "bwd_q_walk": q_walk,
         # q, dO, den, c_i in
         "agg_qdy": (2 * d * s + 8, 2 * M * D + 2 * LP * d),
-        # q, k, v, dO, den, c_i in; dk, dv out
-        "bwd_kv_walk": (6 * d * s + 8, 6 * M * D + 6 * LP * d),
+        "bwd_kv_walk": kv_walk,
         "bwd_walk": (10 * d * s + 4, 10 * M * D + 12 * LP * d),
     }
     for key, val in table.items():
@@ -87,11 +91,11 @@ def kernel_work(name: str, w: race_inputs.Workload):
 # proportion to the tokens), valid only for the kernel code and the segment planner it was
 # taken on: the sha1 of each source with its comments and whitespace removed.
 NCU_TRAFFIC = {
-    "code_sha1": {"race_tc.cuh": "8a4adcc53785c191b40ed6e9f8ebe41bde032597",
-                  "race_tc_util.cuh": "f1810754d25d46a51618b9ee942bf40fdca2da55",
-                  "race_attn.cu": "cb5e5418250397230de02e0f99e24c931c3ba18e"},
-    "bytes_per_token": {"tc_agg_kv": 261.9, "tc_fwd_walk": 501.5, "tc_bwd_q_walk": 768.9,
-                        "tc_agg_qdy": 264.6, "tc_bwd_kv_walk": 753.1, "tc_readout": 217.3},
+    "code_sha1": {"race_tc.cuh": "811f0d281e43d1c1dc96e41f9c0a9321a3c22d6b",
+                  "race_tc_util.cuh": "aed713e09ad44ad8a535b2b1684d92827ba3f9e2",
+                  "race_attn.cu": "03ee1618da5e4c2fe4d5522b24e7912942df6cd3"},
+    "bytes_per_token": {"tc_agg_kv": 262.0, "tc_fwd_walk": 500.4, "tc_bwd_q_walk": 768.4,
+                        "tc_agg_qdy": 264.6, "tc_bwd_kv_walk": 752.4},
 }
 
 
@@ -105,9 +109,12 @@ def code_sha1(path: str) -> str:
     return hashlib.sha1(re.sub(r"\s+", "", src).encode()).hexdigest()
 
 
-def measured_traffic(name: str, tokens: int):
-    """DRAM bytes per launch of kernel `name` from the recorded ncu capture, or None when the
-    kernel code changed since (the counters would describe another kernel)."""
+def measured_traffic(name: str, tokens: int, causal: bool = True):
+    """DRAM bytes per launch of kernel `name` from the recorded ncu capture (a causal pass),
+    or None for a bidirectional pass or when the kernel code changed since (the counters
+    would describe another kernel)."""
+    if not causal:
+        return None
     csrc = os.path.join(ROOT, "linear_attention_soft_b200", "csrc")
     for fn, sha in NCU_TRAFFIC["code_sha1"].items():
         path = os.path.join(csrc, fn)
@@ -443,7 +450,7 @@ def run_ours(args, w):
                 roof = {"bound": "tensor" if is_tensor_core_kernel(name) else "alu",
                         "achieved": flops / per_launch_s / 1e12, "peak": peak_c, "unit": "TFLOP/s"}
             roof["frac"] = roof["achieved"] / roof["peak"]
-            roof["traffic"] = measured_traffic(name, units)
+            roof["traffic"] = measured_traffic(name, units, w.causal)
             roof.update({"kernel": name, "ms_per_launch": per_launch_s * 1e3,
                          "share_of_step": share, "peak_source": peaks["source"]})
     sb, sf = step_work(w)
