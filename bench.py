@@ -91,11 +91,11 @@ def kernel_work(name: str, w: race_inputs.Workload):
 # proportion to the tokens), valid only for the kernel code and the segment planner it was
 # taken on: the sha1 of each source with its comments and whitespace removed.
 NCU_TRAFFIC = {
-    "code_sha1": {"race_tc.cuh": "811f0d281e43d1c1dc96e41f9c0a9321a3c22d6b",
+    "code_sha1": {"race_tc.cuh": "71a47b360be9e900d79a057bcbb1ffaf3015d976",
                   "race_tc_util.cuh": "aed713e09ad44ad8a535b2b1684d92827ba3f9e2",
                   "race_attn.cu": "03ee1618da5e4c2fe4d5522b24e7912942df6cd3"},
-    "bytes_per_token": {"tc_agg_kv": 262.0, "tc_fwd_walk": 500.4, "tc_bwd_q_walk": 768.4,
-                        "tc_agg_qdy": 264.6, "tc_bwd_kv_walk": 752.4},
+    "bytes_per_token": {"tc_agg_kv": 259.5, "tc_fwd_walk": 499.5, "tc_bwd_q_walk": 769.4,
+                        "tc_agg_qdy": 265.0, "tc_bwd_kv_walk": 753.0},
 }
 
 

@@ -632,7 +632,7 @@ __device__ __forceinline__ void store_state40(const float (&hv)[40], float *dst_
 // dx = (dX^ - x^ (x^ . dX^)) / max(|x|, eps) for row r, columns 16qd .. 16qd+15; dX^ from
 // TMEM column col0; x from a K128 tile in shared memory if xtile, else the two 16-byte
 // words xpre the caller loaded;
-// the four quarters exchange partial dots.
+// the four quarters exchange partial dots (named barriers 1..4, one per 32-row block).
 __device__ __forceinline__ void write_dx(uint32_t tm, uint32_t col0, int r, int qd, bool valid, float rawn,
                                          const uint8_t *xtile, const uint4 *xpre, __nv_bfloat16 *dst, float *xch)
 {
@@ -666,7 +666,8 @@ __device__ __forceinline__ void write_dx(uint32_t tm, uint32_t col0, int r, int 
 #pragma unroll
     for (int i = 0; i < 16; ++i) dot = fmaf(x[i], __uint_as_float(w[i]), dot);
     xch[threadIdx.x] = dot;
-    __syncthreads();
+    // the four quarters of this thread's 32 rows are the warps w, w+4, w+8, w+12: they alone meet
+    asm volatile("bar.sync %0, 128;" ::"r"(1 + (int)((threadIdx.x >> 5) & 3)) : "memory");
     dot = xch[r] + xch[128 + r] + xch[256 + r] + xch[384 + r];
     if (!valid) return;
     const float n = fmaxf(rawn, kNormEps), inv = 1.f / n;
@@ -1561,6 +1562,7 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_q_walk(const __grid_constant__ 
         const int nv = (int)(t1 - c0 < T ? t1 - c0 : T);
         const bool valid = r < nv;
         if (!(ok = wait_loads(ctl, ld, 1u))) break;  // the kept q rows (barrier 2) are waited for at dq
+        if (c0 > t0) issue_q2(c0);  // after the barrier: the last chunk's dx has read the kept rows
         if (threadIdx.x == 3 * 128) {  // the projections and P'' run while quarters 0-2 form the row norms
                                        // and scalars (a thread issuing MMAs is held until the tensor
                                        // core's queue takes the last one)
@@ -1619,14 +1621,14 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_q_walk(const __grid_constant__ 
         wait_mma_each(ctl, phase);
         wait_loads_nosync(ctl, ld, 4u);     // this chunk's kept q rows
         write_dx(tm, bq_tmem::DX, r, qd, valid, raw_q, sm + XQ2, nullptr, a.dq + (base + c0 + r) * DH, xch);
-        __syncthreads();  // every quarter has read its q rows
-        if (c0 + T < t1) issue_q2(c0 + T);
         if (causal) {
             float hv[40];
             read_state40(tm, bq_tmem::HTOP, bq_tmem::HBOT, qd, hv);
             stage40_hilo(hv, 128 * (qd & 1) + r, qd, sm + HSHI, sm + HSLO, hden);
         }
-        publish_smem();
+        // the staged state and the TMEM reads are handed over by the next chunk's first barrier
+        fence_smem_async();
+        fence_before_sync();
     }
     drain_loads(ctl, ld);
     kernel_teardown(tm, bq_tmem::NCOLS);
@@ -1796,7 +1798,9 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_kv_walk(const __grid_constant__
         }
         wait_mma_each(ctl, phase);
         write_dx(tm, bkv_tmem::DX, r, qd, valid, raw_k, nullptr, xk4, a.dk + (base + c0 + r) * DH, xch);
-        publish_smem();
+        // the staged state and the TMEM reads are handed over by the next chunk's first barrier
+        fence_smem_async();
+        fence_before_sync();
     }
     drain_loads(ctl, ld);
     kernel_teardown(tm, bkv_tmem::NCOLS);
