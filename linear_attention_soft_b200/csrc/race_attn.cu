@@ -15,6 +15,7 @@
 #include "race_decode.cuh"
 #include "race_generic.cuh"
 #include "race_tc.cuh"
+#include "race_tc_wide.cuh"
 
 namespace {
 
@@ -513,6 +514,297 @@ cudaError_t tc_backward(const Plan &p, const void *q, const void *k, const void 
     });
 }
 
+// ---- the tensor-core path for d = 128, P = 5 (feature groups x value halves) -------------
+namespace wd = race::tc::wide;
+
+bool wide_ok(race_dtype_t dtype, int d, int L, int P, float tau, int causal, int64_t N)
+{
+    return dtype == RACE_BF16 && d == wd::WD && P == wd::WP && L % 8 == 0 && L >= 8 && L <= 32 && tau > 0.f &&
+           causal && N < ((int64_t)1 << 31);
+}
+
+size_t align256(size_t b) { return (b + 255) / 256 * 256; }
+
+// One head at a time: the segment plan is that of a single head, and the per-head arrays
+// (projections, dLoss/dp^, fp32 sums over the groups) are reused for every head.
+struct WidePlan {
+    Plan p;
+    int G, npw, npwp, ntile;
+    size_t state_bytes;  // one head's segment states [2G][nseg][256][65] fp32
+    size_t p_bytes;      // one side's projections [N][npwp] fp32
+    size_t acc_bytes;    // [N][128] fp32 sums over the groups (when G > 1)
+    size_t dacc_bytes;   // [N] fp32
+};
+
+WidePlan wide_plan(int64_t N, int d, int L, int P)
+{
+    WidePlan w;
+    w.p = make_plan(1, 1, N, d, L, P);
+    w.G = L / 8;
+    w.npw = L * P;
+    w.npwp = (w.npw + 15) / 16 * 16;
+    w.ntile = (int)((N + race::tc::T - 1) / race::tc::T);
+    w.state_bytes = align256((size_t)2 * w.G * w.p.nseg * race::tc::MF * race::tc::DS * sizeof(float));
+    w.p_bytes = align256((size_t)N * w.npwp * sizeof(float));
+    w.acc_bytes = w.G > 1 ? align256((size_t)N * wd::WD * sizeof(float)) : 0;
+    w.dacc_bytes = align256((size_t)N * sizeof(float));
+    return w;
+}
+
+size_t wide_forward_bytes(const WidePlan &w) { return w.state_bytes + 2 * w.p_bytes + w.acc_bytes + w.dacc_bytes; }
+// states of both sides, projections and dLoss/dp^ of both sides, the dv sums, c of the head
+size_t wide_backward_bytes(const WidePlan &w)
+{
+    return 2 * w.state_bytes + 4 * w.p_bytes + w.acc_bytes + w.dacc_bytes;
+}
+
+cudaError_t map_2d(CUtensorMap *m, CUtensorMapDataType dt, const void *ptr, uint64_t cols, uint64_t rows,
+                   uint64_t row_bytes, uint32_t box_cols, CUtensorMapSwizzle sw)
+{
+    const EncodeTiled fn = encode_tiled();
+    if (!fn) return cudaErrorNotSupported;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {row_bytes};
+    const cuuint32_t box[2] = {box_cols, (cuuint32_t)race::tc::T};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(m, dt, 2, const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+// One head's [N][128] bf16 as (16 columns, N rows, 8 atoms): a box of 4 atoms is one value half.
+cudaError_t value_map_128(CUtensorMap *m, const void *ptr, int64_t N)
+{
+    const EncodeTiled fn = encode_tiled();
+    if (!fn) return cudaErrorNotSupported;
+    const cuuint64_t dims[3] = {16, (cuuint64_t)N, 8};
+    const cuuint64_t strides[2] = {256, 32};
+    const cuuint32_t box[3] = {16, (cuuint32_t)race::tc::T, 4};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+cudaError_t launch_scan_passes(float *buf, int npass, int nseg, int mode, cudaStream_t st)
+{
+    const int64_t MD = (int64_t)race::tc::MF * race::tc::DS;
+    dim3 grid((unsigned)((MD + gk::NT - 1) / gk::NT), (unsigned)npass);
+    return timed("segment_scan", st, [&] {
+        gk::race_scan<<<grid, gk::NT, 0, st>>>(buf, nseg, MD, mode, nullptr, nullptr);
+        return cudaGetLastError();
+    });
+}
+
+// p^ of the q and k rows of one head (bf16 [N][128] each) into pq, pk.
+cudaError_t wide_projections(const WidePlan &w, const void *qh, const void *kh, const float *W, float *pq, float *pk,
+                             cudaStream_t st)
+{
+    namespace tc = race::tc;
+    wd::ProjArgs pa;
+    std::memset(&pa, 0, sizeof(pa));
+    cudaError_t e;
+    if ((e = map_2d(&pa.tm_x[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, qh, wd::WD, (uint64_t)w.p.N, 256, 64,
+                    CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess ||
+        (e = map_2d(&pa.tm_x[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kh, wd::WD, (uint64_t)w.p.N, 256, 64,
+                    CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess)
+        return e;
+    pa.W = W;
+    pa.p[0] = pq;
+    pa.p[1] = pk;
+    pa.N = w.p.N;
+    pa.ntile = w.ntile;
+    pa.npw = w.npw;
+    pa.npwp = w.npwp;
+    const size_t sm = tc::smem_bytes(wd::proj_smem::TOTAL);
+    if ((e = tc_prepare(wd::wide_proj, sm)) != cudaSuccess) return e;
+    const int grid = (int)std::min<int64_t>(2 * (int64_t)w.ntile, device_sm_count());
+    return timed("wide_proj", st, [&] {
+        wd::wide_proj<<<grid, tc::NTH, sm, st>>>(pa);
+        return cudaGetLastError();
+    });
+}
+
+cudaError_t wide_args(wd::WideArgs &a, const WidePlan &w, const float *pq, const float *pk, const void *vh,
+                      const void *doh, float tau)
+{
+    std::memset(&a, 0, sizeof(a));
+    cudaError_t e;
+    const uint64_t N = (uint64_t)w.p.N, rb = (uint64_t)w.npwp * sizeof(float);
+    if ((e = map_2d(&a.tm_pq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, pq, (uint64_t)w.npwp, N, rb, wd::WPROJ,
+                    CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess ||
+        (e = map_2d(&a.tm_pk, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, pk, (uint64_t)w.npwp, N, rb, wd::WPROJ,
+                    CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess ||
+        (e = value_map_128(&a.tm_v, vh, w.p.N)) != cudaSuccess)
+        return e;
+    if (doh && (e = value_map_128(&a.tm_do, doh, w.p.N)) != cudaSuccess) return e;
+    a.N = w.p.N;
+    a.seg_len = w.p.seg_len;
+    a.nseg = w.p.nseg;
+    a.npwp = w.npwp;
+    a.beta = 1.f / tau;
+    return cudaSuccess;
+}
+
+// Segment totals of every (group, half) pass of one head (mode 0: key side, 1: query side).
+cudaError_t wide_segment_totals(const WidePlan &w, wd::WideArgs a, int mode, float *out, cudaStream_t st)
+{
+    namespace tc = race::tc;
+    const size_t sm = tc::smem_bytes(wd::wagg_smem::TOTAL);
+    const dim3 grid((unsigned)w.p.nseg, (unsigned)(2 * w.G));
+    a.agg_out = out;
+    cudaError_t e;
+    if (mode == 0) {
+        if ((e = tc_prepare(wd::wide_agg<0>, sm)) != cudaSuccess) return e;
+        return timed("wide_agg_kv", st, [&] {
+            wd::wide_agg<0><<<grid, tc::NTH, sm, st>>>(a);
+            return cudaGetLastError();
+        });
+    }
+    if ((e = tc_prepare(wd::wide_agg<1>, sm)) != cudaSuccess) return e;
+    return timed("wide_agg_qdy", st, [&] {
+        wd::wide_agg<1><<<grid, tc::NTH, sm, st>>>(a);
+        return cudaGetLastError();
+    });
+}
+
+cudaError_t wide_forward(int BH, int64_t N, int d, int L, int P, const void *q, const void *k, const void *v,
+                         const float *W, void *out, float *den, float tau, void *workspace, cudaStream_t st)
+{
+    namespace tc = race::tc;
+    const WidePlan w = wide_plan(N, d, L, P);
+    uint8_t *ws = (uint8_t *)workspace;
+    float *states = (float *)ws;
+    float *pq = (float *)(ws + w.state_bytes);
+    float *pk = (float *)(ws + w.state_bytes + w.p_bytes);
+    float *acc = w.acc_bytes ? (float *)(ws + w.state_bytes + 2 * w.p_bytes) : nullptr;
+    float *dacc = (float *)(ws + w.state_bytes + 2 * w.p_bytes + w.acc_bytes);
+    const size_t sm_walk = tc::smem_bytes(wd::wfwd_smem::TOTAL);
+    cudaError_t e;
+    if ((e = tc_prepare(wd::wide_fwd_walk, sm_walk)) != cudaSuccess) return e;
+    const size_t row_bytes = (size_t)N * wd::WD * sizeof(__nv_bfloat16);
+    for (int bh = 0; bh < BH; ++bh) {
+        const uint8_t *qh = (const uint8_t *)q + bh * row_bytes, *kh = (const uint8_t *)k + bh * row_bytes;
+        const uint8_t *vh = (const uint8_t *)v + bh * row_bytes;
+        if ((e = wide_projections(w, qh, kh, W, pq, pk, st)) != cudaSuccess) return e;
+        wd::WideArgs a;
+        if ((e = wide_args(a, w, pq, pk, vh, nullptr, tau)) != cudaSuccess) return e;
+        if ((e = wide_segment_totals(w, a, 0, states, st)) != cudaSuccess) return e;
+        if ((e = launch_scan_passes(states, 2 * w.G, w.p.nseg, gk::SCAN_EXCL_PREFIX, st)) != cudaSuccess) return e;
+        a.state = states;
+        a.acc = acc;
+        a.dacc = dacc;
+        a.out = (__nv_bfloat16 *)((uint8_t *)out + bh * row_bytes);
+        a.den_out = den ? den + (int64_t)bh * N : nullptr;
+        for (int g = 0; g < w.G; ++g) {
+            a.g = g;
+            a.first = g == 0;
+            a.last = g == w.G - 1;
+            e = timed("wide_fwd_walk", st, [&] {
+                wd::wide_fwd_walk<<<dim3((unsigned)w.p.nseg, 2), tc::NTH + 32, sm_walk, st>>>(a);
+                return cudaGetLastError();
+            });
+            if (e != cudaSuccess) return e;
+        }
+    }
+    return cudaSuccess;
+}
+
+cudaError_t wide_backward(int BH, int64_t N, int d, int L, int P, const void *q, const void *k, const void *v,
+                          const float *W, const void *out, const float *den, const void *dout, void *dq, void *dk,
+                          void *dv, float tau, void *workspace, cudaStream_t st)
+{
+    namespace tc = race::tc;
+    const WidePlan w = wide_plan(N, d, L, P);
+    uint8_t *ws = (uint8_t *)workspace;
+    float *hstates = (float *)ws;
+    float *gstates = (float *)(ws + w.state_bytes);
+    uint8_t *arr = ws + 2 * w.state_bytes;
+    float *pq = (float *)arr, *pk = (float *)(arr + w.p_bytes);
+    float *dpq = (float *)(arr + 2 * w.p_bytes), *dpk = (float *)(arr + 3 * w.p_bytes);
+    float *acc = w.acc_bytes ? (float *)(arr + 4 * w.p_bytes) : nullptr;
+    float *cbuf = (float *)(arr + 4 * w.p_bytes + w.acc_bytes);
+    const size_t sm_q = tc::smem_bytes(wd::wbq_smem::TOTAL), sm_kv = tc::smem_bytes(wd::wbkv_smem::TOTAL);
+    const size_t sm_dx = tc::smem_bytes(wd::dx_smem::TOTAL);
+    cudaError_t e;
+    if ((e = tc_prepare(wd::wide_bwd_q_walk, sm_q)) != cudaSuccess ||
+        (e = tc_prepare(wd::wide_bwd_kv_walk, sm_kv)) != cudaSuccess || (e = tc_prepare(wd::wide_dx, sm_dx)) != cudaSuccess)
+        return e;
+    const size_t row_bytes = (size_t)N * wd::WD * sizeof(__nv_bfloat16);
+    for (int bh = 0; bh < BH; ++bh) {
+        const size_t off = bh * row_bytes;
+        const uint8_t *qh = (const uint8_t *)q + off, *kh = (const uint8_t *)k + off, *vh = (const uint8_t *)v + off;
+        const uint8_t *oh = (const uint8_t *)out + off, *doh = (const uint8_t *)dout + off;
+        if ((e = wide_projections(w, qh, kh, W, pq, pk, st)) != cudaSuccess) return e;
+        e = timed("wide_rowc", st, [&] {
+            const int64_t threads = N * 16;
+            wd::wide_rowc<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(
+                (const __nv_bfloat16 *)oh, (const __nv_bfloat16 *)doh, cbuf, N);
+            return cudaGetLastError();
+        });
+        if (e != cudaSuccess) return e;
+        wd::WideArgs a;
+        if ((e = wide_args(a, w, pq, pk, vh, doh, tau)) != cudaSuccess) return e;
+        a.den = den + (int64_t)bh * N;
+        a.cbuf = cbuf;
+        // query side: key-side prefix statistics, then the dq walks of half 0 and half 1
+        if ((e = wide_segment_totals(w, a, 0, hstates, st)) != cudaSuccess) return e;
+        if ((e = launch_scan_passes(hstates, 2 * w.G, w.p.nseg, gk::SCAN_EXCL_PREFIX, st)) != cudaSuccess) return e;
+        a.state = hstates;
+        a.dp = dpq;
+        for (int h = 0; h < 2; ++h) {
+            a.h = h;
+            e = timed("wide_bwd_q_walk", st, [&] {
+                wd::wide_bwd_q_walk<<<dim3((unsigned)w.p.nseg, (unsigned)w.G), tc::NTH, sm_q, st>>>(a);
+                return cudaGetLastError();
+            });
+            if (e != cudaSuccess) return e;
+        }
+        // key side: query-side suffix statistics, then the dk/dv walk of every (group, half)
+        if ((e = wide_segment_totals(w, a, 1, gstates, st)) != cudaSuccess) return e;
+        if ((e = launch_scan_passes(gstates, 2 * w.G, w.p.nseg, gk::SCAN_EXCL_SUFFIX, st)) != cudaSuccess) return e;
+        a.state = gstates;
+        a.dp = dpk;
+        a.acc = acc;
+        a.out = (__nv_bfloat16 *)((uint8_t *)dv + off);
+        for (int g = 0; g < w.G; ++g) {
+            for (int h = 0; h < 2; ++h) {
+                a.g = g;
+                a.h = h;
+                a.first = g == 0;
+                a.last = g == w.G - 1;
+                e = timed("wide_bwd_kv_walk", st, [&] {
+                    wd::wide_bwd_kv_walk<<<(unsigned)w.p.nseg, tc::NTH, sm_kv, st>>>(a);
+                    return cudaGetLastError();
+                });
+                if (e != cudaSuccess) return e;
+            }
+        }
+        wd::DxArgs xa;
+        std::memset(&xa, 0, sizeof(xa));
+        xa.x[0] = (const __nv_bfloat16 *)qh;
+        xa.x[1] = (const __nv_bfloat16 *)kh;
+        xa.dp[0] = dpq;
+        xa.dp[1] = dpk;
+        xa.W = W;
+        xa.dx[0] = (__nv_bfloat16 *)((uint8_t *)dq + off);
+        xa.dx[1] = (__nv_bfloat16 *)((uint8_t *)dk + off);
+        xa.N = N;
+        xa.ntile = w.ntile;
+        xa.npw = w.npw;
+        xa.npwp = w.npwp;
+        xa.kp = (w.npwp + 63) / 64 * 64;
+        const int grid = (int)std::min<int64_t>(2 * (int64_t)w.ntile, device_sm_count());
+        e = timed("wide_dx", st, [&] {
+            wd::wide_dx<<<grid, tc::NTH, sm_dx, st>>>(xa);
+            return cudaGetLastError();
+        });
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
 template <typename DT>
 cudaError_t dispatch_forward(const Plan &p, const Args &a, float *states, int causal, cudaStream_t st,
                              const Shard &sh)
@@ -585,13 +877,16 @@ const char *race_status_string(race_status_t s)
 race_status_t race_attn_workspace_size(int B, int H, int64_t N, int d, int L, int P, int causal,
                                        int backward, race_dtype_t dtype, size_t *bytes)
 {
-    (void)causal;
     if (!bytes) return RACE_ERR_INVALID_ARG;
     if (dtype != RACE_F32 && dtype != RACE_BF16) return RACE_ERR_INVALID_ARG;
     race_status_t s = check_sizes(B, H, N, d, L, P);
     if (s != RACE_OK) return s;
     const Plan p = make_plan(B, H, N, d, L, P);
     *bytes = backward ? backward_workspace_bytes(p) : p.state_elems * sizeof(float);
+    if (wide_ok(dtype, d, L, P, 1.f, causal, N)) {  // room for the feature-group path too
+        const WidePlan w = wide_plan(N, d, L, P);
+        *bytes = std::max(*bytes, backward ? wide_backward_bytes(w) : wide_forward_bytes(w));
+    }
     return RACE_OK;
 }
 
@@ -634,7 +929,11 @@ race_status_t forward_impl(const void *q, const void *k, const void *v, const fl
         return RACE_ERR_INVALID_ARG;
     const Plan p = make_plan(B, H, N, d, L, P);
     const size_t need = p.state_elems * sizeof(float);
-    if (workspace_bytes < need) return RACE_ERR_WORKSPACE;
+    // d = 128, P = 5: the feature-group path when the workspace holds its arrays (it leaves
+    // ctx untouched; the backward recomputes what it needs)
+    const bool wide = sh.stage == STAGE_ALL && wide_ok(dtype, d, L, P, tau, causal, N) &&
+                      workspace_bytes >= wide_forward_bytes(wide_plan(N, d, L, P));
+    if (workspace_bytes < need && !wide) return RACE_ERR_WORKSPACE;
     if (ctx && ctx_bytes < need) return RACE_ERR_WORKSPACE;
     if (!q) q = k;  // the first half reads keys and values only
     Args a = base_args(p, W, tau);
@@ -646,7 +945,9 @@ race_status_t forward_impl(const void *q, const void *k, const void *v, const fl
     float *states = ctx ? ctx : (float *)workspace;
     cudaStream_t st = (cudaStream_t)stream;
     cudaError_t e;
-    if (race::tc::fast_path_ok(dtype, d, L, P, tau, N) && g_tc_forward)
+    if (wide && g_tc_forward)
+        e = wide_forward(B * H, N, d, L, P, q, k, v, W, out, den, tau, workspace, st);
+    else if (race::tc::fast_path_ok(dtype, d, L, P, tau, N) && g_tc_forward)
         e = tc_forward(p, q, k, v, W, out, den, states, tau, causal, st, sh);
     else if (dtype == RACE_F32)
         e = dispatch_forward<float>(p, a, states, causal, st, sh);
@@ -684,8 +985,13 @@ race_status_t backward_impl(const void *q, const void *k, const void *v, const f
         if (ptr && !aligned16(ptr)) return RACE_ERR_INVALID_ARG;
     const Plan p = make_plan(B, H, N, d, L, P);
     const size_t one = p.state_elems * sizeof(float);
-    if (workspace_bytes < backward_workspace_bytes(p)) return RACE_ERR_WORKSPACE;
+    const bool wide = sh.stage == STAGE_ALL && !sh.dpq && wide_ok(dtype, d, L, P, tau, causal, N) &&
+                      workspace_bytes >= wide_backward_bytes(wide_plan(N, d, L, P));
+    if (!wide && workspace_bytes < backward_workspace_bytes(p)) return RACE_ERR_WORKSPACE;
     if (ctx && ctx_bytes < one) return RACE_ERR_WORKSPACE;
+    // the feature-group forward leaves ctx untouched, so for its shapes the statistics are
+    // recomputed rather than read from a context it may not have written
+    if (wide_ok(dtype, d, L, P, tau, causal, N)) ctx = nullptr;
     Args a = base_args(p, W, tau);
     a.q = q;
     a.k = k;
@@ -702,7 +1008,9 @@ race_status_t backward_impl(const void *q, const void *k, const void *v, const f
     float *cbuf = (float *)(wimg + kWImageBytes);
     cudaStream_t st = (cudaStream_t)stream;
     cudaError_t e;
-    if (race::tc::fast_path_ok(dtype, d, L, P, tau, N) && g_tc_backward)
+    if (wide && g_tc_backward)
+        e = wide_backward(B * H, N, d, L, P, q, k, v, W, out, den, dout, dq, dk, dv, tau, workspace, st);
+    else if (race::tc::fast_path_ok(dtype, d, L, P, tau, N) && g_tc_backward)
         e = tc_backward(p, q, k, v, W, out, den, dout, ctx, hbuf, gbuf, wimg, cbuf, dq, dk, dv, tau, causal, st,
                         sh);
     else if (dtype == RACE_F32)
