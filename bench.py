@@ -60,9 +60,24 @@ def step_work(w: race_inputs.Workload):
 
 
 def kernel_work(name: str, w: race_inputs.Workload):
-    """(algorithmic bytes, algorithmic flops) per token per head of one kernel launch."""
+    """(algorithmic bytes, algorithmic flops) per token per head of one kernel over a step
+    (all its launches: one per step for the d = 64 kernels; for the feature-group kernels of
+    d = 128 one per head and pass, whose shares add up to these figures)."""
     s = 4 if w.dtype == "f32" else 2
     M, d, LP, D = w.L * w.R, w.d, w.L * w.P, w.d + 1
+    pb = 4 * LP  # one side's projections p^ (fp32), the feature-group path's intermediate
+    wide = {
+        "wide_proj": (2 * d * s + 2 * pb, 4 * LP * d),                    # q, k in; p^ out
+        "wide_agg_kv": (pb + d * s, 2 * M * D),                          # p^_k, v in
+        "wide_fwd_walk": (2 * pb + 2 * d * s + 4, 4 * M * D),            # p^, v in; out, den out
+        "wide_rowc": (2 * d * s + 4, 2 * d),                             # o, dO in; c out
+        "wide_agg_qdy": (pb + d * s + 8, 2 * M * D),                     # p^_q, dO, den, c in
+        "wide_bwd_q_walk": (3 * pb + 2 * d * s + 8, 4 * M * D),          # p^, v, dO, den, c in; dp^ out
+        "wide_bwd_kv_walk": (3 * pb + 3 * d * s + 8, 6 * M * D),         # and dv out
+        "wide_dx": (2 * pb + 4 * d * s, 4 * LP * d),                     # dp^, x in; dx out (both sides)
+    }
+    if name in wide:
+        return wide[name]
     if w.causal:
         q_walk = (6 * d * s + 8, 4 * M * D + 6 * LP * d)    # q, k, v, o, dO, den in; dq, c_i out
         kv_walk = (6 * d * s + 8, 6 * M * D + 6 * LP * d)   # q, k, v, dO, den, c_i in; dk, dv out
@@ -125,7 +140,7 @@ def measured_traffic(name: str, tokens: int, causal: bool = True):
 
 
 def is_tensor_core_kernel(name: str) -> bool:
-    return name.startswith("tc_")
+    return name.startswith("tc_") or (name.startswith("wide_") and name != "wide_rowc")
 
 
 # ---- clocks ----------------------------------------------------------------------------
@@ -306,11 +321,11 @@ def run_ours(args, w):
     den = torch.empty((B, H, N), dtype=torch.float32, device=dev)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     code = ra.RACE_F32 if w.dtype == "f32" else ra.RACE_BF16
-    ws_f = torch.empty(ra.race_attn_workspace_size(B, H, N, d, L, P, w.causal, 0, code),
-                       dtype=torch.uint8, device=dev)
-    ws_b = torch.empty(ra.race_attn_dw_workspace_size(B, H, N, d, L, P, w.causal, code) if args.dw else
-                       ra.race_attn_workspace_size(B, H, N, d, L, P, w.causal, 1, code),
-                       dtype=torch.uint8, device=dev)
+    # one scratch buffer serves the forward and the backward, which run in turn on one stream
+    ws_f = ws_b = torch.empty(max(ra.race_attn_workspace_size(B, H, N, d, L, P, w.causal, 0, code),
+                                  ra.race_attn_dw_workspace_size(B, H, N, d, L, P, w.causal, code) if args.dw
+                                  else ra.race_attn_workspace_size(B, H, N, d, L, P, w.causal, 1, code)),
+                              dtype=torch.uint8, device=dev)
     dW = torch.empty(W.shape, dtype=torch.float32, device=dev)
     ctx = torch.empty(ra.race_attn_ctx_size(B, H, N, d, L, P, w.causal) // 4,
                       dtype=torch.float32, device=dev)
@@ -430,6 +445,7 @@ def run_ours(args, w):
     if top:
         name, (tot_ms, cnt) = top
         per_launch_s = tot_ms / cnt / 1e3
+        per_step_s = tot_ms / args.steps / 1e3  # all the kernel's launches in one step
         work = kernel_work(name, w)
         units = B * H * N
         share = tot_ms / sum(t for t, _ in prof.values())
@@ -444,14 +460,15 @@ def run_ours(args, w):
                 t_c = flops / (peak_c * 1e12)
             t_m = byts / (peaks["hbm_gbs"] * 1e9)
             if t_m >= t_c:
-                roof = {"bound": "hbm", "achieved": byts / per_launch_s / 1e9,
+                roof = {"bound": "hbm", "achieved": byts / per_step_s / 1e9,
                         "peak": peaks["hbm_gbs"], "unit": "GB/s"}
             else:
                 roof = {"bound": "tensor" if is_tensor_core_kernel(name) else "alu",
-                        "achieved": flops / per_launch_s / 1e12, "peak": peak_c, "unit": "TFLOP/s"}
+                        "achieved": flops / per_step_s / 1e12, "peak": peak_c, "unit": "TFLOP/s"}
             roof["frac"] = roof["achieved"] / roof["peak"]
             roof["traffic"] = measured_traffic(name, units, w.causal)
             roof.update({"kernel": name, "ms_per_launch": per_launch_s * 1e3,
+                         "launches_per_step": cnt / args.steps,
                          "share_of_step": share, "peak_source": peaks["source"]})
     sb, sf = step_work(w)
     t_step_roof = max(sb * B * H * N / (peaks["hbm_gbs"] * 1e9),

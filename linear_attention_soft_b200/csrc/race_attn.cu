@@ -552,10 +552,11 @@ WidePlan wide_plan(int64_t N, int d, int L, int P)
 }
 
 size_t wide_forward_bytes(const WidePlan &w) { return w.state_bytes + 2 * w.p_bytes + w.acc_bytes + w.dacc_bytes; }
-// states of both sides, projections and dLoss/dp^ of both sides, the dv sums, c of the head
+// states of both sides, projections of both sides, dLoss/dp^ of one side at a time, the dv
+// sums, c of the head
 size_t wide_backward_bytes(const WidePlan &w)
 {
-    return 2 * w.state_bytes + 4 * w.p_bytes + w.acc_bytes + w.dacc_bytes;
+    return 2 * w.state_bytes + 3 * w.p_bytes + w.acc_bytes + w.dacc_bytes;
 }
 
 cudaError_t map_2d(CUtensorMap *m, CUtensorMapDataType dt, const void *ptr, uint64_t cols, uint64_t rows,
@@ -722,9 +723,9 @@ cudaError_t wide_backward(int BH, int64_t N, int d, int L, int P, const void *q,
     float *gstates = (float *)(ws + w.state_bytes);
     uint8_t *arr = ws + 2 * w.state_bytes;
     float *pq = (float *)arr, *pk = (float *)(arr + w.p_bytes);
-    float *dpq = (float *)(arr + 2 * w.p_bytes), *dpk = (float *)(arr + 3 * w.p_bytes);
-    float *acc = w.acc_bytes ? (float *)(arr + 4 * w.p_bytes) : nullptr;
-    float *cbuf = (float *)(arr + 4 * w.p_bytes + w.acc_bytes);
+    float *dp = (float *)(arr + 2 * w.p_bytes);  // the q side's, then the k side's
+    float *acc = w.acc_bytes ? (float *)(arr + 3 * w.p_bytes) : nullptr;
+    float *cbuf = (float *)(arr + 3 * w.p_bytes + w.acc_bytes);
     const size_t sm_q = tc::smem_bytes(wd::wbq_smem::TOTAL), sm_kv = tc::smem_bytes(wd::wbkv_smem::TOTAL);
     const size_t sm_dx = tc::smem_bytes(wd::dx_smem::TOTAL);
     cudaError_t e;
@@ -732,6 +733,25 @@ cudaError_t wide_backward(int BH, int64_t N, int d, int L, int P, const void *q,
         (e = tc_prepare(wd::wide_bwd_kv_walk, sm_kv)) != cudaSuccess || (e = tc_prepare(wd::wide_dx, sm_dx)) != cudaSuccess)
         return e;
     const size_t row_bytes = (size_t)N * wd::WD * sizeof(__nv_bfloat16);
+    const int dx_grid = (int)std::min<int64_t>(w.ntile, device_sm_count());
+    auto launch_dx = [&](const void *xh, void *dxh) {  // dx of one side from dp
+        wd::DxArgs xa;
+        std::memset(&xa, 0, sizeof(xa));
+        xa.x[0] = (const __nv_bfloat16 *)xh;
+        xa.dp[0] = dp;
+        xa.dx[0] = (__nv_bfloat16 *)dxh;
+        xa.W = W;
+        xa.N = N;
+        xa.nsides = 1;
+        xa.ntile = w.ntile;
+        xa.npw = w.npw;
+        xa.npwp = w.npwp;
+        xa.kp = (w.npwp + 63) / 64 * 64;
+        return timed("wide_dx", st, [&] {
+            wd::wide_dx<<<dx_grid, tc::NTH, sm_dx, st>>>(xa);
+            return cudaGetLastError();
+        });
+    };
     for (int bh = 0; bh < BH; ++bh) {
         const size_t off = bh * row_bytes;
         const uint8_t *qh = (const uint8_t *)q + off, *kh = (const uint8_t *)k + off, *vh = (const uint8_t *)v + off;
@@ -752,7 +772,7 @@ cudaError_t wide_backward(int BH, int64_t N, int d, int L, int P, const void *q,
         if ((e = wide_segment_totals(w, a, 0, hstates, st)) != cudaSuccess) return e;
         if ((e = launch_scan_passes(hstates, 2 * w.G, w.p.nseg, gk::SCAN_EXCL_PREFIX, st)) != cudaSuccess) return e;
         a.state = hstates;
-        a.dp = dpq;
+        a.dp = dp;
         for (int h = 0; h < 2; ++h) {
             a.h = h;
             e = timed("wide_bwd_q_walk", st, [&] {
@@ -761,11 +781,12 @@ cudaError_t wide_backward(int BH, int64_t N, int d, int L, int P, const void *q,
             });
             if (e != cudaSuccess) return e;
         }
+        if ((e = launch_dx(qh, (uint8_t *)dq + off)) != cudaSuccess) return e;
         // key side: query-side suffix statistics, then the dk/dv walk of every (group, half)
         if ((e = wide_segment_totals(w, a, 1, gstates, st)) != cudaSuccess) return e;
         if ((e = launch_scan_passes(gstates, 2 * w.G, w.p.nseg, gk::SCAN_EXCL_SUFFIX, st)) != cudaSuccess) return e;
         a.state = gstates;
-        a.dp = dpk;
+        a.dp = dp;
         a.acc = acc;
         a.out = (__nv_bfloat16 *)((uint8_t *)dv + off);
         for (int g = 0; g < w.G; ++g) {
@@ -781,26 +802,7 @@ cudaError_t wide_backward(int BH, int64_t N, int d, int L, int P, const void *q,
                 if (e != cudaSuccess) return e;
             }
         }
-        wd::DxArgs xa;
-        std::memset(&xa, 0, sizeof(xa));
-        xa.x[0] = (const __nv_bfloat16 *)qh;
-        xa.x[1] = (const __nv_bfloat16 *)kh;
-        xa.dp[0] = dpq;
-        xa.dp[1] = dpk;
-        xa.W = W;
-        xa.dx[0] = (__nv_bfloat16 *)((uint8_t *)dq + off);
-        xa.dx[1] = (__nv_bfloat16 *)((uint8_t *)dk + off);
-        xa.N = N;
-        xa.ntile = w.ntile;
-        xa.npw = w.npw;
-        xa.npwp = w.npwp;
-        xa.kp = (w.npwp + 63) / 64 * 64;
-        const int grid = (int)std::min<int64_t>(2 * (int64_t)w.ntile, device_sm_count());
-        e = timed("wide_dx", st, [&] {
-            wd::wide_dx<<<grid, tc::NTH, sm_dx, st>>>(xa);
-            return cudaGetLastError();
-        });
-        if (e != cudaSuccess) return e;
+        if ((e = launch_dx(kh, (uint8_t *)dk + off)) != cudaSuccess) return e;
     }
     return cudaSuccess;
 }

@@ -1111,18 +1111,18 @@ __global__ void __launch_bounds__(NTH, 1) wide_bwd_kv_walk(const __grid_constant
 }
 
 // ------------------------------------------------------------------------------------------
-// dx of the q and k rows of one head from dLoss/dp^ (p^ = W x^, x^ = x / max(|x|, eps)):
-// dX^ = dp^ W on the tensor core (dp^ and W each as bf16 hi + lo; the lo x lo product is
-// left out), then dx = (dX^ - x^ (x^ . dX^)) / |x|.  Persistent over 128-row tiles of the q
-// rows, then the k rows.   grid: min(tiles, SMs), 512 threads
+// dx of the rows of one head (one or two sides: q, k) from dLoss/dp^ (p^ = W x^,
+// x^ = x / max(|x|, eps)): dX^ = dp^ W on the tensor core (dp^ and W each as bf16 hi + lo;
+// the lo x lo product is left out), then dx = (dX^ - x^ (x^ . dX^)) / |x|.  Persistent over
+// the 128-row tiles of side 0, then side 1.   grid: min(tiles, SMs), 512 threads
 // ------------------------------------------------------------------------------------------
 struct DxArgs {
-    const __nv_bfloat16 *x[2];  // q, k rows of the head [N][128]
-    const float *dp[2];         // [N][npwp] dLoss/dp^
+    const __nv_bfloat16 *x[2];  // rows of the head [N][128] per side
+    const float *dp[2];         // [N][npwp] dLoss/dp^ per side
     const float *W;             // [npw][128]
-    __nv_bfloat16 *dx[2];       // dq, dk of the head [N][128]
+    __nv_bfloat16 *dx[2];       // gradient of the rows [N][128] per side
     int64_t N;
-    int ntile, npw, npwp, kp;   // kp = npwp rounded up to 64: the MMA's K
+    int nsides, ntile, npw, npwp, kp;  // kp = npwp rounded up to 64: the MMA's K
 };
 
 constexpr uint32_t BT_MAX = 192u * 128u;  // one N-half of W as MN-major rows [kp <= 192][64]
@@ -1158,7 +1158,7 @@ __global__ void __launch_bounds__(NTH, 1) wide_dx(const __grid_constant__ DxArgs
         *reinterpret_cast<uint32_t *>(sm + BLO + off) = lo;
     }
     const uint32_t tm = kernel_setup(ctl, 128, nullptr, nullptr, nullptr);
-    const int ntiles = 2 * a.ntile, kp8 = a.kp >> 3, np8 = a.npwp >> 3;
+    const int ntiles = a.nsides * a.ntile, kp8 = a.kp >> 3, np8 = a.npwp >> 3;
     const uint32_t idesc = idesc_bf16(128, 128, 0, 1);
     uint32_t phase = 0;
     for (int i = blockIdx.x; i < ntiles; i += gridDim.x) {
