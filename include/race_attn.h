@@ -70,7 +70,12 @@ const char *race_status_string(race_status_t status);
  * The workspace holds the per-segment bucket statistics of the chunked scan
  * (fp32, L*2^P x (d+1) per segment and head; the backward needs two such buffers plus
  * 16 KB and one fp32 per token for c_i = -(dO_i . o_i)); it is scratch: its contents on
- * entry are ignored and on exit are unspecified.
+ * entry are ignored and on exit are unspecified.  For bf16 inputs with d = 128, P = 5,
+ * L a multiple of 8 up to 32, causal, the size also covers the per-head arrays of the
+ * feature-group tensor-core path (the normalised projections of q and k, one side's
+ * dLoss/dp and fp32 sums over the feature groups: about (4 * L * P * 3 + 516) bytes per
+ * token of one head in the backward); with a smaller workspace that still holds the
+ * statistics, those shapes run on the general path.
  */
 race_status_t race_attn_workspace_size(int B, int H, int64_t N, int d, int L, int P, int causal,
                                        int backward, race_dtype_t dtype, size_t *bytes);
@@ -81,7 +86,8 @@ race_status_t race_attn_workspace_size(int B, int H, int64_t N, int d, int L, in
  * segment (the running sums A_cum, B_cum of Algorithm 2, zh §2.3, at each segment
  * start; for the bidirectional form, the totals A, B of Algorithm 1); handing the same
  * buffer to race_attn_backward with the same q, k, v, W and sizes saves the backward
- * pass one read of k and v.
+ * pass one read of k and v.  For the shapes of the feature-group path (bf16, d = 128,
+ * P = 5, causal) ctx is left untouched and every backward recomputes the statistics.
  */
 race_status_t race_attn_ctx_size(int B, int H, int64_t N, int d, int L, int P, int causal,
                                  size_t *bytes);
@@ -164,8 +170,9 @@ race_status_t race_attn_selftest_wait_timeout(int64_t limit_ns, race_stream_t st
  *   launched nothing, when race_attn_workspace_size(..., backward = 0) for these sizes
  *   exceeds RACE_NOALLOC_SCRATCH_BYTES (for d = 64 and 2^P = 16, L = 16, that is B * H * nseg
  *   segment states of 66.5 KB each, nseg being the segments the library plans per sequence:
- *   at most N / 512, usually about (SM count) / (B * H); race_attn_workspace_size gives
- *   the exact figure).
+ *   at most N / 512, usually about (SM count) / (B * H); for bf16, d = 128, P = 5,
+ *   causal, it includes the per-head arrays of the feature-group path, about
+ *   (4 * L * P * 2 + 516) bytes per token; race_attn_workspace_size gives the exact figure).
  *   The first call on each device looks up the buffer's device address (a runtime call
  *   with that device current).  With CUDA's default lazy module loading, that first call is
  *   also when the library's device code, and with it this buffer, is loaded onto the device,
