@@ -532,7 +532,7 @@ struct WidePlan {
     int G, npw, npwp, ntile;
     size_t state_bytes;  // one head's segment states [2G][nseg][256][65] fp32
     size_t p_bytes;      // one side's projections [N][npwp] fp32
-    size_t acc_bytes;    // [N][128] fp32 sums over the groups (when G > 1)
+    size_t acc_bytes;    // [N][128] fp32 sums over the groups
     size_t dacc_bytes;   // [N] fp32
 };
 
@@ -546,7 +546,7 @@ WidePlan wide_plan(int64_t N, int d, int L, int P)
     w.ntile = (int)((N + race::tc::T - 1) / race::tc::T);
     w.state_bytes = align256((size_t)2 * w.G * w.p.nseg * race::tc::MF * race::tc::DS * sizeof(float));
     w.p_bytes = align256((size_t)N * w.npwp * sizeof(float));
-    w.acc_bytes = w.G > 1 ? align256((size_t)N * wd::WD * sizeof(float)) : 0;
+    w.acc_bytes = align256((size_t)N * wd::WD * sizeof(float));
     w.dacc_bytes = align256((size_t)N * sizeof(float));
     return w;
 }
@@ -653,7 +653,7 @@ cudaError_t wide_segment_totals(const WidePlan &w, wd::WideArgs a, int mode, flo
 {
     namespace tc = race::tc;
     const size_t sm = tc::smem_bytes(wd::wagg_smem::TOTAL);
-    const dim3 grid((unsigned)w.p.nseg, (unsigned)(2 * w.G));
+    const dim3 grid((unsigned)(2 * w.G), (unsigned)w.p.nseg);
     a.agg_out = out;
     cudaError_t e;
     if (mode == 0) {
@@ -679,7 +679,7 @@ cudaError_t wide_forward(int BH, int64_t N, int d, int L, int P, const void *q, 
     float *states = (float *)ws;
     float *pq = (float *)(ws + w.state_bytes);
     float *pk = (float *)(ws + w.state_bytes + w.p_bytes);
-    float *acc = w.acc_bytes ? (float *)(ws + w.state_bytes + 2 * w.p_bytes) : nullptr;
+    float *acc = (float *)(ws + w.state_bytes + 2 * w.p_bytes);
     float *dacc = (float *)(ws + w.state_bytes + 2 * w.p_bytes + w.acc_bytes);
     const size_t sm_walk = tc::smem_bytes(wd::wfwd_smem::TOTAL);
     cudaError_t e;
@@ -696,18 +696,22 @@ cudaError_t wide_forward(int BH, int64_t N, int d, int L, int P, const void *q, 
         a.state = states;
         a.acc = acc;
         a.dacc = dacc;
-        a.out = (__nv_bfloat16 *)((uint8_t *)out + bh * row_bytes);
-        a.den_out = den ? den + (int64_t)bh * N : nullptr;
         for (int g = 0; g < w.G; ++g) {
             a.g = g;
             a.first = g == 0;
-            a.last = g == w.G - 1;
             e = timed("wide_fwd_walk", st, [&] {
-                wd::wide_fwd_walk<<<dim3((unsigned)w.p.nseg, 2), tc::NTH + 32, sm_walk, st>>>(a);
+                wd::wide_fwd_walk<<<dim3(2, (unsigned)w.p.nseg), tc::NTH + 32, sm_walk, st>>>(a);
                 return cudaGetLastError();
             });
             if (e != cudaSuccess) return e;
         }
+        e = timed("wide_finish", st, [&] {
+            wd::wide_finish<<<(unsigned)((N * 16 + 255) / 256), 256, 0, st>>>(
+                acc, dacc, (__nv_bfloat16 *)((uint8_t *)out + bh * row_bytes), den ? den + (int64_t)bh * N : nullptr,
+                N);
+            return cudaGetLastError();
+        });
+        if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
 }
@@ -724,7 +728,7 @@ cudaError_t wide_backward(int BH, int64_t N, int d, int L, int P, const void *q,
     uint8_t *arr = ws + 2 * w.state_bytes;
     float *pq = (float *)arr, *pk = (float *)(arr + w.p_bytes);
     float *dp = (float *)(arr + 2 * w.p_bytes);  // the q side's, then the k side's
-    float *acc = w.acc_bytes ? (float *)(arr + 3 * w.p_bytes) : nullptr;
+    float *acc = (float *)(arr + 3 * w.p_bytes);
     float *cbuf = (float *)(arr + 3 * w.p_bytes + w.acc_bytes);
     const size_t sm_q = tc::smem_bytes(wd::wbq_smem::TOTAL), sm_kv = tc::smem_bytes(wd::wbkv_smem::TOTAL);
     const size_t sm_dx = tc::smem_bytes(wd::dx_smem::TOTAL);
@@ -768,40 +772,40 @@ cudaError_t wide_backward(int BH, int64_t N, int d, int L, int P, const void *q,
         if ((e = wide_args(a, w, pq, pk, vh, doh, tau)) != cudaSuccess) return e;
         a.den = den + (int64_t)bh * N;
         a.cbuf = cbuf;
-        // query side: key-side prefix statistics, then the dq walks of half 0 and half 1
+        // query side: key-side prefix statistics, then the dq walks of every (group, half)
         if ((e = wide_segment_totals(w, a, 0, hstates, st)) != cudaSuccess) return e;
         if ((e = launch_scan_passes(hstates, 2 * w.G, w.p.nseg, gk::SCAN_EXCL_PREFIX, st)) != cudaSuccess) return e;
         a.state = hstates;
-        a.dp = dp;
-        for (int h = 0; h < 2; ++h) {
-            a.h = h;
-            e = timed("wide_bwd_q_walk", st, [&] {
-                wd::wide_bwd_q_walk<<<dim3((unsigned)w.p.nseg, (unsigned)w.G), tc::NTH, sm_q, st>>>(a);
-                return cudaGetLastError();
-            });
-            if (e != cudaSuccess) return e;
-        }
+        a.dp = dp;  // the walks add their shares of dLoss/dp^ onto zeros
+        if ((e = cudaMemsetAsync(dp, 0, (size_t)N * w.npwp * sizeof(float), st)) != cudaSuccess) return e;
+        e = timed("wide_bwd_q_walk", st, [&] {
+            wd::wide_bwd_q_walk<<<dim3((unsigned)(2 * w.G), (unsigned)w.p.nseg), tc::NTH, sm_q, st>>>(a);
+            return cudaGetLastError();
+        });
+        if (e != cudaSuccess) return e;
         if ((e = launch_dx(qh, (uint8_t *)dq + off)) != cudaSuccess) return e;
-        // key side: query-side suffix statistics, then the dk/dv walk of every (group, half)
+        // key side: query-side suffix statistics, then the dk/dv walks, one group at a time
         if ((e = wide_segment_totals(w, a, 1, gstates, st)) != cudaSuccess) return e;
         if ((e = launch_scan_passes(gstates, 2 * w.G, w.p.nseg, gk::SCAN_EXCL_SUFFIX, st)) != cudaSuccess) return e;
         a.state = gstates;
         a.dp = dp;
         a.acc = acc;
-        a.out = (__nv_bfloat16 *)((uint8_t *)dv + off);
+        if ((e = cudaMemsetAsync(dp, 0, (size_t)N * w.npwp * sizeof(float), st)) != cudaSuccess) return e;
         for (int g = 0; g < w.G; ++g) {
-            for (int h = 0; h < 2; ++h) {
-                a.g = g;
-                a.h = h;
-                a.first = g == 0;
-                a.last = g == w.G - 1;
-                e = timed("wide_bwd_kv_walk", st, [&] {
-                    wd::wide_bwd_kv_walk<<<(unsigned)w.p.nseg, tc::NTH, sm_kv, st>>>(a);
-                    return cudaGetLastError();
-                });
-                if (e != cudaSuccess) return e;
-            }
+            a.g = g;
+            a.first = g == 0;
+            e = timed("wide_bwd_kv_walk", st, [&] {
+                wd::wide_bwd_kv_walk<<<dim3(2, (unsigned)w.p.nseg), tc::NTH, sm_kv, st>>>(a);
+                return cudaGetLastError();
+            });
+            if (e != cudaSuccess) return e;
         }
+        e = timed("wide_finish", st, [&] {
+            wd::wide_finish<<<(unsigned)((N * 16 + 255) / 256), 256, 0, st>>>(
+                acc, nullptr, (__nv_bfloat16 *)((uint8_t *)dv + off), nullptr, N);
+            return cudaGetLastError();
+        });
+        if (e != cudaSuccess) return e;
         if ((e = launch_dx(kh, (uint8_t *)dk + off)) != cudaSuccess) return e;
     }
     return cudaSuccess;

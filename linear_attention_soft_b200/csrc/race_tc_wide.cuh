@@ -16,8 +16,9 @@
 //                 128-row tile (x bf16 exact, W as bf16 hi + lo), fp32 [N][npwp]
 //   wide_agg<0>   per (group, half) segment totals sum_j phi_g(k_j) [v_j,h | 1]^T
 //   wide_agg<1>   per (group, half) sum_i phi_g(q_i) / den_i [dO_i,h | c_i]^T (c only in half 0)
-//   wide_fwd_walk one (group, half) causal walk: partial numerator and den, summed over the
-//                 groups in fp32; the last group divides and writes out and den
+//   wide_fwd_walk one group's causal walk for both halves: partial numerator and den, summed
+//                 over the groups in fp32 in memory
+//   wide_finish   out = numerator / den (forward) or dv (backward) from the fp32 sums
 //   wide_rowc     c_i = -(dO_i . o_i) over all 128 columns
 //   wide_bwd_q_walk / wide_bwd_kv_walk: the dq / dk,dv walks of one (group, half)
 //   wide_dx       dx = (dX^ - x^ (x^ . dX^)) / |x| with dX^ = dp^ W on the tensor core
@@ -48,15 +49,13 @@ struct WideArgs {
     const float *cbuf;       // [N] c_i (backward)
     float *acc;              // [N][128] fp32: numerator (forward) or dv (backward) over the groups so far
     float *dacc;             // [N] fp32: den over the groups so far (forward)
-    __nv_bfloat16 *out;      // [N][128]: out (forward) or dv (backward), written by the last group
-    float *den_out;          // [N] (forward, last group; may be null)
-    float *dp;               // [N][npwp] dLoss/dp^ of the walk's side (backward)
+    float *dp;               // [N][npwp] dLoss/dp^ of the walk's side (backward; zero before the walk)
     const float *state;      // walk start states [2 * groups][nseg][256][65]
     float *agg_out;          // segment totals [2 * groups][nseg][256][65]
     int64_t N, seg_len;
     int nseg, npwp;
-    int g, h;                // the launch's feature group and value half (where not from blockIdx.y)
-    int first, last;         // the launch is the first / the last of its accumulation
+    int g;                   // the launch's feature group (walks launched once per group)
+    int first;               // the launch is the first of its group sum (stores instead of adding)
     float beta;
 };
 
@@ -215,38 +214,41 @@ __device__ __forceinline__ void features_vjp10(uint32_t tm, uint32_t col0, int q
     }
 }
 
-// 10 fp32 values to dst (8-byte aligned): stored, or added to what is there.
-__device__ __forceinline__ void put10(float *dst, const float (&v)[10], bool add)
+// Partial sums to global memory without reading it back: stored (the first contribution)
+// or added there by the memory system (red.global.add, no value returned), so no thread
+// waits on the round trip.  Each element receives one contribution per launch, or two that
+// commute exactly (a + b onto zero), so the sums do not depend on scheduling.
+__device__ __forceinline__ void red_add_v4(float *p, float a, float b, float c, float d)
 {
-    float2 *d2 = reinterpret_cast<float2 *>(dst);
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
+}
+__device__ __forceinline__ void red_add_v2(float *p, float a, float b)
+{
+    asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(p), "f"(a), "f"(b) : "memory");
+}
+__device__ __forceinline__ void red_add_f32(float *p, float a)
+{
+    asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(a) : "memory");
+}
+
+// 16 fp32 values to dst (16-byte aligned): stored, or added in memory.
+__device__ __forceinline__ void put16(float *dst, const float (&v)[16], bool add)
+{
 #pragma unroll
-    for (int i = 0; i < 5; ++i) {
-        float2 x = make_float2(v[2 * i], v[2 * i + 1]);
-        if (add) {
-            const float2 o = d2[i];
-            x.x += o.x;
-            x.y += o.y;
-        }
-        d2[i] = x;
+    for (int i = 0; i < 4; ++i) {
+        if (add)
+            red_add_v4(dst + 4 * i, v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        else
+            reinterpret_cast<float4 *>(dst)[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
     }
 }
 
-// 16 fp32 values to dst (16-byte aligned): stored, or added to what is there.
-__device__ __forceinline__ void put16(float *dst, const float (&v)[16], bool add)
+// 10 fp32 values added in memory at dst (8-byte aligned).
+__device__ __forceinline__ void add10(float *dst, const float (&v)[10])
 {
-    float4 *d4 = reinterpret_cast<float4 *>(dst);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        float4 x = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-        if (add) {
-            const float4 o = d4[i];
-            x.x += o.x;
-            x.y += o.y;
-            x.z += o.z;
-            x.w += o.w;
-        }
-        d4[i] = x;
-    }
+    for (int i = 0; i < 5; ++i) red_add_v2(dst + 2 * i, v[2 * i], v[2 * i + 1]);
 }
 
 __device__ __forceinline__ void store_bf16x16(__nv_bfloat16 *dst, const float (&y)[16])
@@ -410,7 +412,8 @@ __global__ void __launch_bounds__(NTH, 1) wide_proj(const __grid_constant__ Proj
 // Segment totals of one (group, half) pass.  MODE 0: H_seg = sum_j phi_g(k_j) [v_j,h | 1]^T
 // (the bucket statistics A, B of zh §2.2 over the segment, for the group's tables and the
 // half's value columns).  MODE 1: G_seg = sum_i phi_g(q_i) / den_i [dO_i,h | c_i]^T, with c
-// in half 0 only (the backward's query-side statistics).   grid: nseg x (2 * groups)
+// in half 0 only (the backward's query-side statistics).   grid: (2 * groups) x nseg: the
+// passes of a segment side by side, so that they read the segment's rows from L2 together.
 // As in the 256-feature kernels, the CTA's two groups of 256 threads take alternate chunks,
 // each with its own tiles, TMEM accumulator and barriers, and the two sums are added at the
 // end.  Thread (r, hh) of a thread group owns row r and quarters 2hh, 2hh+1 of the features.
@@ -434,7 +437,7 @@ __global__ void __launch_bounds__(NTH, 1) wide_agg(const __grid_constant__ WideA
     uint8_t *sm = aligned_base(smem_raw);
     using namespace wagg_smem;
     Ctl *ctl = reinterpret_cast<Ctl *>(sm + BAR);
-    const int seg = blockIdx.x, pass = blockIdx.y, g = pass >> 1, hv = pass & 1;
+    const int seg = blockIdx.y, pass = blockIdx.x, g = pass >> 1, hv = pass & 1;
     const int gi = threadIdx.x >> 8, gt = threadIdx.x & 255;
     const int r = gt & 127, hh = gt >> 7;
     const bool leader = gt == 0;
@@ -576,13 +579,13 @@ __global__ void __launch_bounds__(NTH, 1) wide_agg(const __grid_constant__ WideA
 }
 
 // ------------------------------------------------------------------------------------------
-// Causal walk of one (group, half) pass (Algorithm 2, zh §2.3).   grid: nseg x 2 (value
-// halves), NTH + 32 threads; launched once per group, group 0 first.
+// Causal walk of one (group, half) pass (Algorithm 2, zh §2.3).   grid: 2 (value halves) x
+// nseg, NTH + 32 threads; launched once per group, group 0 first.
 // The structure is that of the 256-feature walk: Phi_Q in tensor memory, one lane of the last
 // warp issuing every TMA load and MMA, hand-overs through mbarriers.  The chunk's projections
 // come as two [128][40] fp32 tiles (q, k), loaded a chunk ahead once the features of the
 // current chunk have been formed.  Each pass adds its partial numerator Y[:, :64] and den
-// Y[:, 64] to fp32 sums over the groups; the last group divides.
+// Y[:, 64] to fp32 sums over the groups (group 0 stores); wide_finish divides.
 // ------------------------------------------------------------------------------------------
 namespace wfwd_smem {
 constexpr uint32_t PHK = 0;                // Phi_K [128][256]
@@ -619,7 +622,7 @@ __global__ void __launch_bounds__(NTH + 32, 1) wide_fwd_walk(const __grid_consta
     namespace tmc = wfwd_tmem;
     Ctl *ctl = reinterpret_cast<Ctl *>(sm + BAR);
     WFwdBars *fb = reinterpret_cast<WFwdBars *>(sm + FB);
-    const int seg = blockIdx.x, h = blockIdx.y, g = a.g;
+    const int seg = blockIdx.y, h = blockIdx.x, g = a.g;
     const bool issuer_warp = threadIdx.x >= NTH;
     const int r = threadIdx.x & 127, qd = (threadIdx.x >> 7) & 3;
     const uint32_t sb = smem_u32(sm);
@@ -753,29 +756,13 @@ __global__ void __launch_bounds__(NTH + 32, 1) wide_fwd_walk(const __grid_consta
                     float y[16];
 #pragma unroll
                     for (int i = 0; i < 16; ++i) y[i] = __uint_as_float(w[i]);
-                    float dn = __uint_as_float(dn8[0]);
-                    float *accp = a.acc + row * WD + 64 * h + 16 * qd;
-                    if (!a.last) {
-                        put16(accp, y, !a.first);
-                        if (h == 0 && qd == 0) a.dacc[row] = a.first ? dn : a.dacc[row] + dn;
-                    } else {
-                        if (!a.first) {
-                            const float4 *s4 = reinterpret_cast<const float4 *>(accp);
-#pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                const float4 o = s4[i];
-                                y[4 * i] += o.x;
-                                y[4 * i + 1] += o.y;
-                                y[4 * i + 2] += o.z;
-                                y[4 * i + 3] += o.w;
-                            }
-                            dn += a.dacc[row];
-                        }
-                        const float inv = dn != 0.f ? 1.f / dn : 0.f;
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) y[i] *= inv;
-                        store_bf16x16(a.out + row * WD + 64 * h + 16 * qd, y);
-                        if (h == 0 && qd == 0 && a.den_out) a.den_out[row] = dn;
+                    const float dn = __uint_as_float(dn8[0]);
+                    put16(a.acc + row * WD + 64 * h + 16 * qd, y, !a.first);
+                    if (h == 0 && qd == 0) {
+                        if (a.first)
+                            a.dacc[row] = dn;
+                        else
+                            red_add_f32(a.dacc + row, dn);
                     }
                 }
             }
@@ -853,8 +840,8 @@ constexpr uint32_t HBOT = 336;
 }  // namespace wbq_tmem
 
 // ------------------------------------------------------------------------------------------
-// dq walk of the value half a.h for every group (chunks in order, prefix state H).
-// grid: nseg x groups; launched for half 0, then half 1.
+// dq walk of every (group, half) pass (chunks in order, prefix state H).   grid: (2 * groups)
+// x nseg.  The two halves' shares of dLoss/dp^ are added in memory onto zeros.
 // ------------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(NTH, 1) wide_bwd_q_walk(const __grid_constant__ WideArgs a)
 {
@@ -865,7 +852,7 @@ __global__ void __launch_bounds__(NTH, 1) wide_bwd_q_walk(const __grid_constant_
     Ctl *ctl = reinterpret_cast<Ctl *>(sm + BAR);
     float *hden = reinterpret_cast<float *>(sm + HDEN);
     float *rowc = reinterpret_cast<float *>(sm + ROWC), *rowinv = reinterpret_cast<float *>(sm + ROWINV);
-    const int seg = blockIdx.x, g = blockIdx.y, h = a.h;
+    const int seg = blockIdx.y, g = blockIdx.x >> 1, h = blockIdx.x & 1;
     const int r = threadIdx.x & 127, qd = threadIdx.x >> 7;
     const uint32_t sb = smem_u32(sm);
     const uint32_t tm = kernel_setup(ctl, 512, nullptr, nullptr, nullptr);
@@ -933,7 +920,7 @@ __global__ void __launch_bounds__(NTH, 1) wide_bwd_q_walk(const __grid_constant_
         {  // dphi = (D + c'_i H_prev[:, 64]) / den_i -> dLoss/dp^ of the group's projections
             float dp[10];
             features_vjp10(tm, tmc::DPHI, qd, a.beta, valid, u, t, hden + 256 * par, c_r, invden_r, dp);
-            if (valid) put10(a.dp + (c0 + r) * a.npwp + WPROJ * g + 10 * qd, dp, h != 0);
+            if (valid) add10(a.dp + (c0 + r) * a.npwp + WPROJ * g + 10 * qd, dp);
         }
         {  // the updated state, staged for the next chunk (its den column into the other buffer)
             float hv[40];
@@ -973,8 +960,9 @@ constexpr uint32_t DVT = 416;   // dV_h [128][64]
 }  // namespace wbkv_tmem
 
 // ------------------------------------------------------------------------------------------
-// dk/dv walk of one (group, half) pass (chunks in reverse, suffix state G).   grid: nseg;
-// launched for every group and half in the order (g, h) = (0, 0), (0, 1), (1, 0), ...
+// dk/dv walk of one group for both halves (chunks in reverse, suffix state G).   grid: 2
+// (value halves) x nseg; launched once per group, group 0 first.  dv is summed over the
+// groups (group 0 stores), dLoss/dp^ over the halves (added onto zeros).
 // ------------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(NTH, 1) wide_bwd_kv_walk(const __grid_constant__ WideArgs a)
 {
@@ -984,7 +972,7 @@ __global__ void __launch_bounds__(NTH, 1) wide_bwd_kv_walk(const __grid_constant
     namespace tmc = wbkv_tmem;
     Ctl *ctl = reinterpret_cast<Ctl *>(sm + BAR);
     float *rowc = reinterpret_cast<float *>(sm + ROWC), *rowinv = reinterpret_cast<float *>(sm + ROWINV);
-    const int seg = blockIdx.x, g = a.g, h = a.h;
+    const int seg = blockIdx.y, g = a.g, h = blockIdx.x;
     const int r = threadIdx.x & 127, qd = threadIdx.x >> 7;
     const uint32_t sb = smem_u32(sm);
     const uint32_t tm = kernel_setup(ctl, 512, nullptr, nullptr, nullptr);
@@ -1073,29 +1061,13 @@ __global__ void __launch_bounds__(NTH, 1) wide_bwd_kv_walk(const __grid_constant
                 float y[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) y[i] = __uint_as_float(w[i]);
-                float *accp = a.acc + row * WD + 64 * h + 16 * qd;
-                if (!a.last) {
-                    put16(accp, y, !a.first);
-                } else {
-                    if (!a.first) {
-                        const float4 *s4 = reinterpret_cast<const float4 *>(accp);
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const float4 o = s4[i];
-                            y[4 * i] += o.x;
-                            y[4 * i + 1] += o.y;
-                            y[4 * i + 2] += o.z;
-                            y[4 * i + 3] += o.w;
-                        }
-                    }
-                    store_bf16x16(a.out + row * WD + 64 * h + 16 * qd, y);
-                }
+                put16(a.acc + row * WD + 64 * h + 16 * qd, y, !a.first);
             }
         }
         {
             float dp[10];
             features_vjp10(tm, tmc::DPHI, qd, a.beta, valid, u, t, nullptr, 0.f, 1.f, dp);
-            if (valid) put10(a.dp + (c0 + r) * a.npwp + WPROJ * g + 10 * qd, dp, h != 0);
+            if (valid) add10(a.dp + (c0 + r) * a.npwp + WPROJ * g + 10 * qd, dp);
         }
         {
             float hv[40];
@@ -1111,10 +1083,35 @@ __global__ void __launch_bounds__(NTH, 1) wide_bwd_kv_walk(const __grid_constant
 }
 
 // ------------------------------------------------------------------------------------------
+// From the fp32 sums over the feature groups of one head: out = num / den in bf16 and den
+// (den_out, may be null) when den is given, else dv = the sum in bf16.  16 threads per row.
+// ------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) wide_finish(const float *acc, const float *den, __nv_bfloat16 *dst,
+                                                   float *den_out, int64_t rows)
+{
+    const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t row = t >> 4;
+    const int part = (int)(t & 15);
+    if (row >= rows) return;
+    const float4 *src = reinterpret_cast<const float4 *>(acc + row * WD) + 2 * part;
+    const float4 x0 = src[0], x1 = src[1];
+    float sc = 1.f;
+    if (den) {
+        const float dn = den[row];
+        sc = dn != 0.f ? 1.f / dn : 0.f;
+        if (den_out && part == 0) den_out[row] = dn;
+    }
+    reinterpret_cast<uint4 *>(dst + row * WD)[part] =
+        make_uint4(pack_bf16x2(x0.x * sc, x0.y * sc), pack_bf16x2(x0.z * sc, x0.w * sc),
+                   pack_bf16x2(x1.x * sc, x1.y * sc), pack_bf16x2(x1.z * sc, x1.w * sc));
+}
+
+// ------------------------------------------------------------------------------------------
 // dx of the rows of one head (one or two sides: q, k) from dLoss/dp^ (p^ = W x^,
 // x^ = x / max(|x|, eps)): dX^ = dp^ W on the tensor core (dp^ and W each as bf16 hi + lo;
 // the lo x lo product is left out), then dx = (dX^ - x^ (x^ . dX^)) / |x|.  Persistent over
-// the 128-row tiles of side 0, then side 1.   grid: min(tiles, SMs), 512 threads
+// the 128-row tiles of side 0, then side 1.
+// grid: min(tiles, SMs), 512 threads
 // ------------------------------------------------------------------------------------------
 struct DxArgs {
     const __nv_bfloat16 *x[2];  // rows of the head [N][128] per side
@@ -1165,23 +1162,29 @@ __global__ void __launch_bounds__(NTH, 1) wide_dx(const __grid_constant__ DxArgs
         const int side = i >= a.ntile ? 1 : 0;
         const int64_t row = (int64_t)(i - side * a.ntile) * T + r;
         const bool valid = row < a.N;
-        // this thread's 8-column chunks qd, qd + 4, ... of the row's dp^ as hi + lo
-        for (int c8 = qd; c8 < kp8; c8 += 4) {
-            float v[8];
+        // this thread's 8-column chunks qd, qd + 4, ... (at most 6) of the row's dp^ as hi + lo
+        float4 v[6][2];
+#pragma unroll
+        for (int k = 0; k < 6; ++k) {
+            const int c8 = qd + 4 * k;
             if (valid && c8 < np8) {
                 const float4 *src = reinterpret_cast<const float4 *>(a.dp[side] + row * a.npwp + 8 * c8);
-                const float4 x0 = src[0], x1 = src[1];
-                v[0] = x0.x; v[1] = x0.y; v[2] = x0.z; v[3] = x0.w;
-                v[4] = x1.x; v[5] = x1.y; v[6] = x1.z; v[7] = x1.w;
+                v[k][0] = src[0];
+                v[k][1] = src[1];
             } else {
-#pragma unroll
-                for (int k = 0; k < 8; ++k) v[k] = 0.f;
+                v[k][0] = v[k][1] = make_float4(0.f, 0.f, 0.f, 0.f);
             }
+        }
+#pragma unroll
+        for (int k = 0; k < 6; ++k) {
+            const int c8 = qd + 4 * k;
+            if (c8 >= kp8) break;
+            const float x[8] = {v[k][0].x, v[k][0].y, v[k][0].z, v[k][0].w, v[k][1].x, v[k][1].y, v[k][1].z, v[k][1].w};
             uint32_t wh[4], wl[4];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                wh[k] = pack_bf16x2(v[2 * k], v[2 * k + 1]);
-                wl[k] = pack_bf16x2(v[2 * k] - bf16_lo(wh[k]), v[2 * k + 1] - bf16_hi(wh[k]));
+            for (int m = 0; m < 4; ++m) {
+                wh[m] = pack_bf16x2(x[2 * m], x[2 * m + 1]);
+                wl[m] = pack_bf16x2(x[2 * m] - bf16_lo(wh[m]), x[2 * m + 1] - bf16_hi(wh[m]));
             }
             const uint32_t off = (uint32_t)(c8 >> 3) * TILE + sw128_off(r, c8 & 7);
             st_shared_v4(sb + AHI + off, wh[0], wh[1], wh[2], wh[3]);
