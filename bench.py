@@ -104,21 +104,26 @@ def kernel_work(name: str, w: race_inputs.Workload):
 # DRAM bytes per token (dram__bytes_read.sum + dram__bytes_write.sum) per kernel, from one
 # ncu capture of the causal forward + backward at B1 H1 N = 2^20 d64 (traffic grows in
 # proportion to the tokens), valid only for the kernel code and the segment planner it was
-# taken on: the sha1 of each source with its comments and whitespace removed.
+# taken on: the sha1 of the d = 64 kernel sources and of the planner, comments and
+# whitespace removed.
 NCU_TRAFFIC = {
     "code_sha1": {"race_tc.cuh": "71a47b360be9e900d79a057bcbb1ffaf3015d976",
                   "race_tc_util.cuh": "aed713e09ad44ad8a535b2b1684d92827ba3f9e2",
-                  "race_attn.cu": "03ee1618da5e4c2fe4d5522b24e7912942df6cd3"},
+                  "race_attn.cu:make_plan": "368b30caf4555ce78bb0b9b31efea22157570d7e"},
     "bytes_per_token": {"tc_agg_kv": 259.5, "tc_fwd_walk": 499.5, "tc_bwd_q_walk": 769.4,
                         "tc_agg_qdy": 265.0, "tc_bwd_kv_walk": 753.0},
 }
 
 
-def code_sha1(path: str) -> str:
-    """sha1 of a C++ source without its comments and whitespace (what the compiler sees)."""
+def code_sha1(path: str, function: str = "") -> str:
+    """sha1 of a C++ source (or of one function in it: from its signature to the first line
+    that closes it) without comments and whitespace: what the compiler sees."""
     import hashlib
     import re
     src = open(path, encoding="utf-8").read()
+    if function:
+        i = src.index(function)
+        src = src[i:src.index("\n}\n", i) + 3]
     src = re.sub(r"//[^\n]*", "", src)
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
     return hashlib.sha1(re.sub(r"\s+", "", src).encode()).hexdigest()
@@ -131,9 +136,10 @@ def measured_traffic(name: str, tokens: int, causal: bool = True):
     if not causal:
         return None
     csrc = os.path.join(ROOT, "linear_attention_soft_b200", "csrc")
-    for fn, sha in NCU_TRAFFIC["code_sha1"].items():
+    for key, sha in NCU_TRAFFIC["code_sha1"].items():
+        fn, _, function = key.partition(":")
         path = os.path.join(csrc, fn)
-        if not os.path.exists(path) or code_sha1(path) != sha:
+        if not os.path.exists(path) or code_sha1(path, ("Plan " + function + "(") if function else "") != sha:
             return None
     bpt = NCU_TRAFFIC["bytes_per_token"].get(name)
     return None if bpt is None else bpt * tokens

@@ -696,6 +696,9 @@ cudaError_t wide_forward(int BH, int64_t N, int d, int L, int P, const void *q, 
         a.state = states;
         a.acc = acc;
         a.dacc = dacc;
+        if ((e = map_2d(&a.tm_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, acc, wd::WD, (uint64_t)N, wd::WD * sizeof(float),
+                        32, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess)
+            return e;
         for (int g = 0; g < w.G; ++g) {
             a.g = g;
             a.first = g == 0;
@@ -790,6 +793,9 @@ cudaError_t wide_backward(int BH, int64_t N, int d, int L, int P, const void *q,
         a.state = gstates;
         a.dp = dp;
         a.acc = acc;
+        if ((e = map_2d(&a.tm_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, acc, wd::WD, (uint64_t)N, wd::WD * sizeof(float),
+                        32, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess)
+            return e;
         if ((e = cudaMemsetAsync(dp, 0, (size_t)N * w.npwp * sizeof(float), st)) != cudaSuccess) return e;
         for (int g = 0; g < w.G; ++g) {
             a.g = g;

@@ -45,6 +45,7 @@ constexpr uint32_t WTILE_MAX = 160u * 128u;        // one K-half of W as K-major
 // of 4 atoms with the 32-byte swizzle (one value half); rows past N read as zero.
 struct WideArgs {
     CUtensorMap tm_pq, tm_pk, tm_v, tm_do;
+    CUtensorMap tm_acc;      // acc as 2-D fp32 (128 columns, N rows), boxes 32 x 128, 128-byte swizzle
     const float *den;        // [N] (backward)
     const float *cbuf;       // [N] c_i (backward)
     float *acc;              // [N][128] fp32: numerator (forward) or dv (backward) over the groups so far
@@ -218,11 +219,6 @@ __device__ __forceinline__ void features_vjp10(uint32_t tm, uint32_t col0, int q
 // or added there by the memory system (red.global.add, no value returned), so no thread
 // waits on the round trip.  Each element receives one contribution per launch, or two that
 // commute exactly (a + b onto zero), so the sums do not depend on scheduling.
-__device__ __forceinline__ void red_add_v4(float *p, float a, float b, float c, float d)
-{
-    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
-                 : "memory");
-}
 __device__ __forceinline__ void red_add_v2(float *p, float a, float b)
 {
     asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(p), "f"(a), "f"(b) : "memory");
@@ -232,16 +228,50 @@ __device__ __forceinline__ void red_add_f32(float *p, float a)
     asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(a) : "memory");
 }
 
-// 16 fp32 values to dst (16-byte aligned): stored, or added in memory.
-__device__ __forceinline__ void put16(float *dst, const float (&v)[16], bool add)
+// ---- bulk stores and reductions from shared memory (TMA, no multicast) ---------------------
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, int x, int y, uint32_t src)
+{
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%1, %2}], [%3];" ::"l"(map),
+                 "r"(x), "r"(y), "r"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void tma_add_2d(const CUtensorMap *map, int x, int y, uint32_t src)
+{
+    asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                     map),
+                 "r"(x), "r"(y), "r"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// the shared-memory sources of the committed bulk groups may be overwritten
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// the committed bulk groups are complete
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// 16 fp32 values of row r, value columns 16qd .. 16qd+15 of a half, into a [128][64] fp32
+// staging tile laid out as the TMA image of two boxes of [128][32] with the 128-byte swizzle.
+__device__ __forceinline__ void stage_row16(uint32_t stage, int r, int qd, const float (&y)[16])
+{
+    const uint32_t box = stage + (uint32_t)(qd >> 1) * TILE;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        st_shared_v4(box + sw128_off(r, 4 * (qd & 1) + i), __float_as_uint(y[4 * i]), __float_as_uint(y[4 * i + 1]),
+                     __float_as_uint(y[4 * i + 2]), __float_as_uint(y[4 * i + 3]));
+}
+
+// The staged tile into columns 64h .. 64h+63 of rows row0 .. row0+127 of an fp32 [N][128]
+// array, stored or added (one writer per element per launch; rows past N are left out), as
+// one committed bulk group.  Issued by one thread after the staging is published.
+__device__ __forceinline__ void put_tile64(const CUtensorMap *map, uint32_t stage, int h, int row0, bool add)
 {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int b = 0; b < 2; ++b) {
         if (add)
-            red_add_v4(dst + 4 * i, v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            tma_add_2d(map, 64 * h + 32 * b, row0, stage + (uint32_t)b * TILE);
         else
-            reinterpret_cast<float4 *>(dst)[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            tma_store_2d(map, 64 * h + 32 * b, row0, stage + (uint32_t)b * TILE);
     }
+    bulk_commit();
 }
 
 // 10 fp32 values added in memory at dst (8-byte aligned).
@@ -277,9 +307,9 @@ __device__ __forceinline__ bool wait_one_load(Ctl *ctl, Loads &ld, int b, volati
 // ------------------------------------------------------------------------------------------
 // Projections p^ = W x / max(|x|, eps) of every q and k row of one head: the normalised
 // projections of the soft hash (zh §2.2) before the squash.  Persistent: CTA b takes the
-// 128-row tiles b, b + gridDim.x, ... of the q rows, then of the k rows; the rows of the tile
-// after next load while this one is read out, into the other of two row buffers and two
-// accumulators.   grid: min(tiles, SMs), 512 threads
+// 128-row tiles b, b + gridDim.x, ... of the q rows, then of the k rows; while one tile is
+// read out, the next tile's projection runs into the other accumulator and the rows of the
+// tile after it load into the other row buffer.   grid: min(tiles, SMs), 512 threads
 // ------------------------------------------------------------------------------------------
 namespace proj_smem {
 constexpr uint32_t X0 = 0;                     // a tile's rows: 2 K128 tiles (columns 0-63, 64-127)
@@ -333,8 +363,28 @@ __global__ void __launch_bounds__(NTH, 1) wide_proj(const __grid_constant__ Proj
             tma_load2(dst + TILE, &a.tm_x[side], 64, row0, bar);
         }
     };
+    // thread 0: once tile j's rows are in, issue its projection into accumulator j & 1
+    auto issue_mma = [&](int j) {
+        const int b = j & 1;
+        if (*(volatile uint32_t *)&ctl->abort != 0u || !wait_one_load(ctl, ld, b, &ctl->abort)) return;
+        fence_after_sync();
+        const uint32_t xs = sb + (b ? X1 : X0), d = tm + (uint32_t)b * 256u;
+#pragma unroll
+        for (int kh = 0; kh < 2; ++kh) {
+            const uint64_t ax = sdesc(xs + kh * TILE, 16, 1024, LAYOUT_SW128);
+            const uint64_t bh = sdesc(sb + WHI + kh * WTILE_MAX, 16, 1024, LAYOUT_SW128);
+            const uint64_t bl = sdesc(sb + WLO + kh * WTILE_MAX, 16, 1024, LAYOUT_SW128);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                mma_bf16(d, ax + 2 * kk, bh + 2 * kk, idesc, (kh | kk) != 0 ? 1u : 0u);
+                mma_bf16(d, ax + 2 * kk, bl + 2 * kk, idesc, 1u);
+            }
+        }
+        mma_commit(&mb[b]);
+    };
     if (tile_of(0) < ntiles) issue_load(0);
     if (tile_of(1) < ntiles) issue_load(1);
+    if (threadIdx.x == 0 && tile_of(0) < ntiles) issue_mma(0);
     for (int j = 0; tile_of(j) < ntiles; ++j) {
         const int i = tile_of(j), side = i >= a.ntile ? 1 : 0, b = j & 1;
         const int64_t row0 = (int64_t)(i - side * a.ntile) * T;
@@ -356,30 +406,17 @@ __global__ void __launch_bounds__(NTH, 1) wide_proj(const __grid_constant__ Proj
             }
             rn[(b * 4 + qd) * 128 + r] = s;
         }
-        if (threadIdx.x == 0 && *(volatile uint32_t *)&ctl->abort == 0u) {
-            fence_after_sync();
-            const uint32_t d = tm + (uint32_t)b * 256u;
-#pragma unroll
-            for (int kh = 0; kh < 2; ++kh) {
-                const uint64_t ax = sdesc(xs + kh * TILE, 16, 1024, LAYOUT_SW128);
-                const uint64_t bh = sdesc(sb + WHI + kh * WTILE_MAX, 16, 1024, LAYOUT_SW128);
-                const uint64_t bl = sdesc(sb + WLO + kh * WTILE_MAX, 16, 1024, LAYOUT_SW128);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    mma_bf16(d, ax + 2 * kk, bh + 2 * kk, idesc, (kh | kk) != 0 ? 1u : 0u);
-                    mma_bf16(d, ax + 2 * kk, bl + 2 * kk, idesc, 1u);
-                }
-            }
-            mma_commit(&mb[b]);
-        }
         if (*(volatile uint32_t *)&ctl->abort == 0u && !mbar_wait(&mb[b], (uint32_t)(j >> 1) & 1u, WAIT_LIMIT_NS)) {
             ctl->abort = 1u;
             atomicExch(&g_tc_error, 1);
         }
         fence_after_sync();
-        __syncthreads();  // the norms are complete; the MMA has read the rows buffer
+        // the norms are complete, tile j's MMA has read its rows buffer, and every thread has
+        // read accumulator (j + 1) & 1 for tile j - 1
+        __syncthreads();
         if (*(volatile uint32_t *)&ctl->abort != 0u) break;
         if (tile_of(j + 2) < ntiles) issue_load(j + 2);
+        if (threadIdx.x == 0 && tile_of(j + 1) < ntiles) issue_mma(j + 1);  // runs under this tile's read-out
         const float n2 = (rn[b * 512 + r] + rn[b * 512 + 128 + r]) + (rn[b * 512 + 256 + r] + rn[b * 512 + 384 + r]);
         const float inv = 1.f / fmaxf(sqrtf(n2), kNormEps);
         uint32_t w[5][8];
@@ -670,7 +707,7 @@ __global__ void __launch_bounds__(NTH + 32, 1) wide_fwd_walk(const __grid_consta
                 issue_rows(t0);
                 issue_v(t0, 0);
             }
-            bool ok = true;
+            bool ok = true, staged = false;  // staged: a Y tile is being written out from SB
             int par = 0;
             for (int64_t c0 = t0; c0 < t1 && ok; c0 += T, par ^= 1) {
                 const bool more = c0 + T < t1;
@@ -681,6 +718,10 @@ __global__ void __launch_bounds__(NTH + 32, 1) wide_fwd_walk(const __grid_consta
                 if (!(ok = wait(&fb->phik, ph_phik))) break;
                 if (more) issue_rows(c0 + T);  // both projection tiles have been read
                 if (!(ok = wait(&fb->v[par], ph_v[par]))) break;
+                if (staged) {  // the mask after this S overwrites SB: the last Y tile has left it
+                    bulk_wait_read();
+                    staged = false;
+                }
                 fence_after_sync();  // S = Phi_Q Phi_K^T, then H += Phi_K^T V~
                 issue_k256_tkk(tm + tmc::S, tm + tmc::PHQ, sb + PHK, idesc_bf16(128, 128, 0, 0));
                 mma_commit(&fb->s);
@@ -690,7 +731,10 @@ __global__ void __launch_bounds__(NTH + 32, 1) wide_fwd_walk(const __grid_consta
                 issue_k128_va(tm + tmc::Y, sb + SB, 0, sb + (par ? VA1 : VA0), idesc_bf16(128, 80, 0, 1), true);
                 mma_commit(&fb->sv);
                 if (!(ok = wait(&fb->done, ph_done))) break;
+                put_tile64(&a.tm_acc, sb + SB, h, (int)c0, !a.first);  // Y[:, :64], staged in SB
+                staged = true;
             }
+            bulk_wait_all();
             // leave nothing in flight: the last commit covers every MMA issued; then every load
             // group issued has completed (a wait on the parity of the last phase returns at once
             // when that phase is over)
@@ -751,19 +795,16 @@ __global__ void __launch_bounds__(NTH + 32, 1) wide_fwd_walk(const __grid_consta
                 tmem_ld16_nowait(tlane(tm, tmc::Y + 16u * qd), w);
                 tmem_ld8_nowait(tlane(tm, tmc::Y + 64u), dn8);
                 tmem_wait_ld();
-                if (valid) {
-                    const int64_t row = c0 + r;
-                    float y[16];
+                float y[16];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) y[i] = __uint_as_float(w[i]);
+                for (int i = 0; i < 16; ++i) y[i] = __uint_as_float(w[i]);
+                stage_row16(sb + SB, r, qd, y);  // the issuer writes the tile out (SB is free: S V~ is done)
+                if (valid && h == 0 && qd == 0) {
                     const float dn = __uint_as_float(dn8[0]);
-                    put16(a.acc + row * WD + 64 * h + 16 * qd, y, !a.first);
-                    if (h == 0 && qd == 0) {
-                        if (a.first)
-                            a.dacc[row] = dn;
-                        else
-                            red_add_f32(a.dacc + row, dn);
-                    }
+                    if (a.first)
+                        a.dacc[c0 + r] = dn;
+                    else
+                        red_add_f32(a.dacc + c0 + r, dn);
                 }
             }
             {  // stage the updated state for the next chunk's read-out
@@ -962,7 +1003,8 @@ constexpr uint32_t DVT = 416;   // dV_h [128][64]
 // ------------------------------------------------------------------------------------------
 // dk/dv walk of one group for both halves (chunks in reverse, suffix state G).   grid: 2
 // (value halves) x nseg; launched once per group, group 0 first.  dv is summed over the
-// groups (group 0 stores), dLoss/dp^ over the halves (added onto zeros).
+// groups (group 0 stores) by TMA from a staged tile, dLoss/dp^ over the halves (added onto
+// zeros).
 // ------------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(NTH, 1) wide_bwd_kv_walk(const __grid_constant__ WideArgs a)
 {
@@ -997,11 +1039,14 @@ __global__ void __launch_bounds__(NTH, 1) wide_bwd_kv_walk(const __grid_constant
         }
     };
     if (nchunks > 0) issue_loads(t0 + (nchunks - 1) * T);
+    int64_t staged_row0 = -1;  // the previous chunk's dV tile, staged in PHQ, not yet written out
     for (int64_t ci = nchunks - 1; ci >= 0 && ok; --ci) {
         const int64_t c0 = t0 + ci * T;
         const int nv = (int)(t1 - c0 < T ? t1 - c0 : T);
         const bool valid = r < nv;
         if (!(ok = wait_loads(ctl, ld, 1u))) break;
+        if (threadIdx.x == 0 && staged_row0 >= 0)  // the barrier above published it
+            put_tile64(&a.tm_acc, sb + PHQ, h, (int)staged_row0, !a.first);
         if (threadIdx.x == 3 * 128) {  // P' = V dO^T while the features are formed
             fence_after_sync();
             issue_va_va(tm + tmc::PP, sb + VA, T, sb + DOC, T, 4, idesc_bf16(128, 128, 0, 0), false);
@@ -1025,6 +1070,8 @@ __global__ void __launch_bounds__(NTH, 1) wide_bwd_kv_walk(const __grid_constant
         fence_smem_async();
         if (!(ok = wait_mma(ctl, phase, 3 * 128))) break;  // every thread has read the projection tiles
         write_features64(t, r, qd, valid ? 1.f : 0.f, sm + PHK);
+        if (threadIdx.x == 0 && staged_row0 >= 0) bulk_wait_read();  // PHQ is rewritten next
+        staged_row0 = -1;
         publish_smem();
         if (threadIdx.x == 0) {  // dV = Phi_K G_next[:, :64], while Phi_Q' is formed
             fence_after_sync();
@@ -1056,13 +1103,11 @@ __global__ void __launch_bounds__(NTH, 1) wide_bwd_kv_walk(const __grid_constant
             uint32_t w[16];
             tmem_ld16_nowait(tlane(tm, tmc::DVT + 16u * qd), w);
             tmem_wait_ld();
-            if (valid) {
-                const int64_t row = c0 + r;
-                float y[16];
+            float y[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) y[i] = __uint_as_float(w[i]);
-                put16(a.acc + row * WD + 64 * h + 16 * qd, y, !a.first);
-            }
+            for (int i = 0; i < 16; ++i) y[i] = __uint_as_float(w[i]);
+            stage_row16(sb + PHQ, r, qd, y);  // Phi_Q' has been read; written out at the next barrier
+            staged_row0 = c0;
         }
         {
             float dp[10];
@@ -1077,6 +1122,11 @@ __global__ void __launch_bounds__(NTH, 1) wide_bwd_kv_walk(const __grid_constant
         // the staged state and the TMEM reads are handed over by the next chunk's first barrier
         fence_smem_async();
         fence_before_sync();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        if (ok && staged_row0 >= 0) put_tile64(&a.tm_acc, sb + PHQ, h, (int)staged_row0, !a.first);
+        bulk_wait_all();
     }
     drain_loads(ctl, ld);
     kernel_teardown(tm, 512);
