@@ -86,8 +86,11 @@ race_status_t race_attn_workspace_size(int B, int H, int64_t N, int d, int L, in
  * segment (the running sums A_cum, B_cum of Algorithm 2, zh §2.3, at each segment
  * start; for the bidirectional form, the totals A, B of Algorithm 1); handing the same
  * buffer to race_attn_backward with the same q, k, v, W and sizes saves the backward
- * pass one read of k and v.  For the shapes of the feature-group path (bf16, d = 128,
- * P = 5, causal) ctx is left untouched and every backward recomputes the statistics.
+ * pass one read of k and v.  For the shapes of the feature-group tensor-core path (d = 128,
+ * P = 5, L a multiple of 8, causal) the size leaves room for either path's statistics and a
+ * 16-byte tag after them: that path's forward keeps its own layout there and sets the tag,
+ * every other forward clears it; the feature-group backward checks the tag on the device
+ * and otherwise recomputes, and every other backward recomputes for these shapes.
  */
 race_status_t race_attn_ctx_size(int B, int H, int64_t N, int d, int L, int P, int causal,
                                  size_t *bytes);

@@ -552,6 +552,18 @@ WidePlan wide_plan(int64_t N, int d, int L, int P)
 }
 
 size_t wide_forward_bytes(const WidePlan &w) { return w.state_bytes + 2 * w.p_bytes + w.acc_bytes + w.dacc_bytes; }
+
+// Context of the shapes this path can take (d = 128, P = 5, L a multiple of 8 up to 32,
+// causal): room for either path's states, then a tag (kCtxTag when this path's forward left
+// its scanned key-side states [BH][2G][nseg][256][65] there, 0 otherwise).
+bool wide_shape(int d, int L, int P, int causal)
+{
+    return d == wd::WD && P == wd::WP && L % 8 == 0 && L >= 8 && L <= 32 && causal;
+}
+size_t wide_ctx_tag_offset(const Plan &p, const WidePlan &w)
+{
+    return align256(std::max(p.state_elems * sizeof(float), (size_t)p.BH * w.state_bytes));
+}
 // states of both sides, projections of both sides, dLoss/dp^ of one side at a time, the dv
 // sums, c of the head
 size_t wide_backward_bytes(const WidePlan &w)
@@ -588,12 +600,13 @@ cudaError_t value_map_128(CUtensorMap *m, const void *ptr, int64_t N)
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-cudaError_t launch_scan_passes(float *buf, int npass, int nseg, int mode, cudaStream_t st)
+cudaError_t launch_scan_passes(float *buf, int npass, int nseg, int mode, cudaStream_t st,
+                               const uint32_t *skip_if = nullptr)
 {
     const int64_t MD = (int64_t)race::tc::MF * race::tc::DS;
     dim3 grid((unsigned)((MD + gk::NT - 1) / gk::NT), (unsigned)npass);
     return timed("segment_scan", st, [&] {
-        gk::race_scan<<<grid, gk::NT, 0, st>>>(buf, nseg, MD, mode, nullptr, nullptr);
+        gk::race_scan<<<grid, gk::NT, 0, st>>>(buf, nseg, MD, mode, nullptr, nullptr, skip_if, wd::kCtxTag);
         return cudaGetLastError();
     });
 }
@@ -670,8 +683,10 @@ cudaError_t wide_segment_totals(const WidePlan &w, wd::WideArgs a, int mode, flo
     });
 }
 
+// ctx_tag: non-null when ctx (room for BH heads' states) receives them, with the tag set at the end.
 cudaError_t wide_forward(int BH, int64_t N, int d, int L, int P, const void *q, const void *k, const void *v,
-                         const float *W, void *out, float *den, float tau, void *workspace, cudaStream_t st)
+                         const float *W, void *out, float *den, float tau, void *workspace, float *ctx,
+                         uint32_t *ctx_tag, cudaStream_t st)
 {
     namespace tc = race::tc;
     const WidePlan w = wide_plan(N, d, L, P);
@@ -685,7 +700,9 @@ cudaError_t wide_forward(int BH, int64_t N, int d, int L, int P, const void *q, 
     cudaError_t e;
     if ((e = tc_prepare(wd::wide_fwd_walk, sm_walk)) != cudaSuccess) return e;
     const size_t row_bytes = (size_t)N * wd::WD * sizeof(__nv_bfloat16);
+    if (ctx_tag && (e = cudaMemsetAsync(ctx_tag, 0, 16, st)) != cudaSuccess) return e;
     for (int bh = 0; bh < BH; ++bh) {
+        if (ctx_tag) states = (float *)((uint8_t *)ctx + bh * w.state_bytes);  // kept for the backward
         const uint8_t *qh = (const uint8_t *)q + bh * row_bytes, *kh = (const uint8_t *)k + bh * row_bytes;
         const uint8_t *vh = (const uint8_t *)v + bh * row_bytes;
         if ((e = wide_projections(w, qh, kh, W, pq, pk, st)) != cudaSuccess) return e;
@@ -716,12 +733,15 @@ cudaError_t wide_forward(int BH, int64_t N, int d, int L, int P, const void *q, 
         });
         if (e != cudaSuccess) return e;
     }
+    if (ctx_tag && (e = cudaMemsetAsync(ctx_tag, 0x5A, 16, st)) != cudaSuccess) return e;
     return cudaSuccess;
 }
 
+// ctx_tag: non-null when ctx may hold the forward's key-side states (decided on the device).
 cudaError_t wide_backward(int BH, int64_t N, int d, int L, int P, const void *q, const void *k, const void *v,
                           const float *W, const void *out, const float *den, const void *dout, void *dq, void *dk,
-                          void *dv, float tau, void *workspace, cudaStream_t st)
+                          void *dv, float tau, void *workspace, const float *ctx, const uint32_t *ctx_tag,
+                          cudaStream_t st)
 {
     namespace tc = race::tc;
     const WidePlan w = wide_plan(N, d, L, P);
@@ -775,9 +795,14 @@ cudaError_t wide_backward(int BH, int64_t N, int d, int L, int P, const void *q,
         if ((e = wide_args(a, w, pq, pk, vh, doh, tau)) != cudaSuccess) return e;
         a.den = den + (int64_t)bh * N;
         a.cbuf = cbuf;
-        // query side: key-side prefix statistics, then the dq walks of every (group, half)
+        a.ctx_tag = ctx_tag;
+        a.ctx_states = ctx_tag ? (const float *)((const uint8_t *)ctx + bh * w.state_bytes) : nullptr;
+        // query side: key-side prefix statistics (from the context when the forward left them
+        // there), then the dq walks of every (group, half)
         if ((e = wide_segment_totals(w, a, 0, hstates, st)) != cudaSuccess) return e;
-        if ((e = launch_scan_passes(hstates, 2 * w.G, w.p.nseg, gk::SCAN_EXCL_PREFIX, st)) != cudaSuccess) return e;
+        if ((e = launch_scan_passes(hstates, 2 * w.G, w.p.nseg, gk::SCAN_EXCL_PREFIX, st, ctx_tag)) != cudaSuccess)
+            return e;
+        a.ctx_tag = nullptr;
         a.state = hstates;
         a.dp = dp;  // the walks add their shares of dLoss/dp^ onto zeros
         if ((e = cudaMemsetAsync(dp, 0, (size_t)N * w.npwp * sizeof(float), st)) != cudaSuccess) return e;
@@ -905,11 +930,12 @@ race_status_t race_attn_workspace_size(int B, int H, int64_t N, int d, int L, in
 race_status_t race_attn_ctx_size(int B, int H, int64_t N, int d, int L, int P, int causal,
                                  size_t *bytes)
 {
-    (void)causal;
     if (!bytes) return RACE_ERR_INVALID_ARG;
     race_status_t s = check_sizes(B, H, N, d, L, P);
     if (s != RACE_OK) return s;
-    *bytes = make_plan(B, H, N, d, L, P).state_elems * sizeof(float);
+    const Plan p = make_plan(B, H, N, d, L, P);
+    *bytes = p.state_elems * sizeof(float);
+    if (wide_shape(d, L, P, causal)) *bytes = wide_ctx_tag_offset(p, wide_plan(N, d, L, P)) + 256;
     return RACE_OK;
 }
 
@@ -957,8 +983,16 @@ race_status_t forward_impl(const void *q, const void *k, const void *v, const fl
     float *states = ctx ? ctx : (float *)workspace;
     cudaStream_t st = (cudaStream_t)stream;
     cudaError_t e;
+    // for the shapes of the feature-group path, the tag after the states in ctx says whether
+    // they are that path's (set by its forward) or not (cleared by every other forward)
+    uint32_t *tag = nullptr;
+    if (ctx && wide_shape(d, L, P, causal)) {
+        const size_t off = wide_ctx_tag_offset(p, wide_plan(N, d, L, P));
+        if (ctx_bytes >= off + 16) tag = (uint32_t *)((uint8_t *)ctx + off);
+    }
+    if (tag && !(wide && g_tc_forward) && cudaMemsetAsync(tag, 0, 16, st) != cudaSuccess) return RACE_ERR_CUDA;
     if (wide && g_tc_forward)
-        e = wide_forward(B * H, N, d, L, P, q, k, v, W, out, den, tau, workspace, st);
+        e = wide_forward(B * H, N, d, L, P, q, k, v, W, out, den, tau, workspace, ctx, tag, st);
     else if (race::tc::fast_path_ok(dtype, d, L, P, tau, N) && g_tc_forward)
         e = tc_forward(p, q, k, v, W, out, den, states, tau, causal, st, sh);
     else if (dtype == RACE_F32)
@@ -1001,9 +1035,18 @@ race_status_t backward_impl(const void *q, const void *k, const void *v, const f
                       workspace_bytes >= wide_backward_bytes(wide_plan(N, d, L, P));
     if (!wide && workspace_bytes < backward_workspace_bytes(p)) return RACE_ERR_WORKSPACE;
     if (ctx && ctx_bytes < one) return RACE_ERR_WORKSPACE;
-    // the feature-group forward leaves ctx untouched, so for its shapes the statistics are
-    // recomputed rather than read from a context it may not have written
-    if (wide_ok(dtype, d, L, P, tau, causal, N)) ctx = nullptr;
+    // for the shapes of the feature-group path the context may hold that path's states: only
+    // that path reads it (after checking the tag on the device); the others recompute
+    const float *wctx = nullptr;
+    const uint32_t *tag = nullptr;
+    if (ctx && wide_shape(d, L, P, causal)) {
+        const size_t off = wide_ctx_tag_offset(p, wide_plan(N, d, L, P));
+        if (ctx_bytes >= off + 16) {
+            wctx = ctx;
+            tag = (const uint32_t *)((const uint8_t *)ctx + off);
+        }
+        ctx = nullptr;
+    }
     Args a = base_args(p, W, tau);
     a.q = q;
     a.k = k;
@@ -1021,7 +1064,7 @@ race_status_t backward_impl(const void *q, const void *k, const void *v, const f
     cudaStream_t st = (cudaStream_t)stream;
     cudaError_t e;
     if (wide && g_tc_backward)
-        e = wide_backward(B * H, N, d, L, P, q, k, v, W, out, den, dout, dq, dk, dv, tau, workspace, st);
+        e = wide_backward(B * H, N, d, L, P, q, k, v, W, out, den, dout, dq, dk, dv, tau, workspace, wctx, tag, st);
     else if (race::tc::fast_path_ok(dtype, d, L, P, tau, N) && g_tc_backward)
         e = tc_backward(p, q, k, v, W, out, den, dout, ctx, hbuf, gbuf, wimg, cbuf, dq, dk, dv, tau, causal, st,
                         sh);

@@ -534,13 +534,16 @@ __global__ void __launch_bounds__(NT) race_agg(Args a)
 //   SCAN_TOTAL: slot 0 becomes init + the sum of all segments;
 //   SCAN_TOTAL_ONLY: the buffer is left as it is.
 // total_out (optional) receives the sum of all segments (plus init, except TOTAL_ONLY).
+// skip_if (optional): the scan does nothing when *skip_if == skip_tag (the buffer already
+// holds the scanned states, decided on the device).
 // grid (ceil(M*D / NT), BH)
 // ------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(NT) race_scan(float *buf, int nseg, int64_t MD, int mode, const float *init,
-                                                float *total_out)
+                                                float *total_out, const uint32_t *skip_if = nullptr,
+                                                uint32_t skip_tag = 0)
 {
     const int64_t e = (int64_t)blockIdx.x * NT + threadIdx.x;
-    if (e >= MD) return;
+    if (e >= MD || (skip_if && *skip_if == skip_tag)) return;
     float *b = buf + (int64_t)blockIdx.y * nseg * MD + e;
     const int64_t oe = (int64_t)blockIdx.y * MD + e;
     constexpr int K = 8;  // segments loaded together: independent loads in flight

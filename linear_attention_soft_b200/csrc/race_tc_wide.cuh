@@ -39,6 +39,7 @@ constexpr int WP = 5;                              // hyperplanes per table
 constexpr int WPROJ = 40;                          // projections of a feature group (8 tables)
 constexpr uint32_t PTILE = 128u * WPROJ * 4u;      // one chunk's projections of a group, fp32 [128][40]
 constexpr uint32_t WTILE_MAX = 160u * 128u;        // one K-half of W as K-major bf16 rows [npwp <= 160][64]
+constexpr uint32_t kCtxTag = 0x5A5A5A5Au;          // a context holds this path's key-side states
 
 // Per head.  Tensor maps: p^ as 2-D fp32 (npwp columns, N rows), boxes of 40 columns x 128
 // rows (no swizzle); v and dO as 3-D bf16 (16 columns, N rows, 8 atoms of 16 columns), boxes
@@ -53,6 +54,8 @@ struct WideArgs {
     float *dp;               // [N][npwp] dLoss/dp^ of the walk's side (backward; zero before the walk)
     const float *state;      // walk start states [2 * groups][nseg][256][65]
     float *agg_out;          // segment totals [2 * groups][nseg][256][65]
+    const float *ctx_states; // a saved context's scanned key-side states of the head, laid out as state
+    const uint32_t *ctx_tag; // == kCtxTag when ctx_states holds them (written by this path's forward)
     int64_t N, seg_len;
     int nseg, npwp;
     int g;                   // the launch's feature group (walks launched once per group)
@@ -475,6 +478,11 @@ __global__ void __launch_bounds__(NTH, 1) wide_agg(const __grid_constant__ WideA
     using namespace wagg_smem;
     Ctl *ctl = reinterpret_cast<Ctl *>(sm + BAR);
     const int seg = blockIdx.y, pass = blockIdx.x, g = pass >> 1, hv = pass & 1;
+    if (MODE == 0 && a.ctx_tag && *a.ctx_tag == kCtxTag) {  // the forward saved them (already scanned)
+        const int64_t off = ((int64_t)pass * a.nseg + seg) * MF * DS;
+        for (int i = threadIdx.x; i < MF * DS; i += NTH) a.agg_out[off + i] = a.ctx_states[off + i];
+        return;
+    }
     const int gi = threadIdx.x >> 8, gt = threadIdx.x & 255;
     const int r = gt & 127, hh = gt >> 7;
     const bool leader = gt == 0;

@@ -112,3 +112,30 @@ def test_backward_with_a_saved_context():
     g2 = gpu_backward(inp, out, den, 0.5, True)
     torch.cuda.synchronize()
     assert all(torch.equal(a, b) for a, b in zip(g1, g2))
+
+
+def test_context_left_by_another_path_is_not_read():
+    """A forward that cannot take the feature-group path (its workspace holds only the segment
+    statistics) leaves ctx in the general layout and clears the tag that the feature-group
+    forward sets; the feature-group backward then recomputes the statistics."""
+    B, H, N, L = 1, 1, 1500, 16
+    inp = _inputs(B, H, N, L, seed=12)
+    q, k, v, W = inp["q"], inp["k"], inp["v"], inp["W"]
+    code = ra.RACE_BF16
+    full = torch.empty(ra.race_attn_workspace_size(B, H, N, 128, L, 5, 1, 0, code), dtype=torch.uint8, device=DEV)
+    small = torch.empty(ra.race_attn_workspace_size(B, H, N, 128, L, 5, 0, 0, code), dtype=torch.uint8,
+                        device=DEV)  # the general path's need (bidirectional sizes)
+    assert small.numel() < full.numel()
+    ctx = torch.empty(ra.race_attn_ctx_size(B, H, N, 128, L, 5, 1) // 4, dtype=torch.float32, device=DEV)
+    out, den = torch.empty_like(q), torch.empty((B, H, N), dtype=torch.float32, device=DEV)
+    ra.race_attn_forward(q, k, v, W, out, den, ctx, 0.5, True, full)     # feature-group path: tag set
+    g_ctx = gpu_backward(inp, out, den, 0.5, True, ctx=ctx)
+    g_none = gpu_backward(inp, out, den, 0.5, True)
+    torch.cuda.synchronize()
+    assert all(torch.equal(a, b) for a, b in zip(g_ctx, g_none))
+    out2, den2 = torch.empty_like(q), torch.empty_like(den)
+    ra.race_attn_forward(q, k, v, W, out2, den2, ctx, 0.5, True, small)  # general path: tag cleared
+    g_ctx2 = gpu_backward(inp, out, den, 0.5, True, ctx=ctx)
+    torch.cuda.synchronize()
+    assert rel_err(out2, out.float().cpu().numpy()) <= TOL[torch.bfloat16]
+    assert all(torch.equal(a, b) for a, b in zip(g_ctx2, g_none))
