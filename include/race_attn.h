@@ -20,7 +20,10 @@
  *   - Layout: q, k, v, out, dout, dq, dk, dv are [B, H, N, d] row-major (d fastest),
  *     contiguous; den is [B, H, N]; W is [L, P, d] fp32 and is shared by every (b, h).
  *   - Every pointer named "device" must point to memory of the current CUDA device,
- *     16-byte aligned.  The caller owns all buffers, workspaces included; no entry point
+ *     16-byte aligned.  The tensor-core paths move rows in 32-byte accesses and run only
+ *     when the buffers of the call are 32-byte aligned (every cudaMalloc or torch
+ *     allocation is); with buffers that are only 16-byte aligned the general path gives the
+ *     same results, more slowly.  The caller owns all buffers, workspaces included; no entry point
  *     allocates memory.  The library's own state is small and fixed: one device error word
  *     (race_attn_device_error), the kernel timers of race_attn_profile_* (host side, off
  *     unless enabled), and the fixed device buffer of race_attn_forward_noalloc, which is

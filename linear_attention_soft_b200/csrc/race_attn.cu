@@ -8,6 +8,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <initializer_list>
 #include <string>
 #include <vector>
 
@@ -152,6 +153,15 @@ Plan make_plan(int B, int H, int64_t N, int d, int L, int P)
 }
 
 bool aligned16(const void *ptr) { return ((uintptr_t)ptr & 15u) == 0; }
+// The tensor-core paths move rows in 32-byte accesses: they run only when every buffer they
+// touch is 32-byte aligned (as every cudaMalloc or torch allocation is); otherwise the
+// general path runs.
+bool aligned32(std::initializer_list<const void *> ptrs)
+{
+    for (const void *p : ptrs)
+        if (p && ((uintptr_t)p & 31u) != 0) return false;
+    return true;
+}
 
 // Backward workspace: key- and query-side segment states, then the W image of the tensor-core
 // path (16 KB), then c_i per token (fp32 [BH][N]).
@@ -969,7 +979,8 @@ race_status_t forward_impl(const void *q, const void *k, const void *v, const fl
     const size_t need = p.state_elems * sizeof(float);
     // d = 128, P = 5: the feature-group path when the workspace holds its arrays (it leaves
     // ctx untouched; the backward recomputes what it needs)
-    const bool wide = sh.stage == STAGE_ALL && wide_ok(dtype, d, L, P, tau, causal, N) &&
+    const bool al32 = aligned32({q, k, v, out, workspace, ctx});
+    const bool wide = sh.stage == STAGE_ALL && wide_ok(dtype, d, L, P, tau, causal, N) && al32 &&
                       workspace_bytes >= wide_forward_bytes(wide_plan(N, d, L, P));
     if (workspace_bytes < need && !wide) return RACE_ERR_WORKSPACE;
     if (ctx && ctx_bytes < need) return RACE_ERR_WORKSPACE;
@@ -993,7 +1004,7 @@ race_status_t forward_impl(const void *q, const void *k, const void *v, const fl
     if (tag && !(wide && g_tc_forward) && cudaMemsetAsync(tag, 0, 16, st) != cudaSuccess) return RACE_ERR_CUDA;
     if (wide && g_tc_forward)
         e = wide_forward(B * H, N, d, L, P, q, k, v, W, out, den, tau, workspace, ctx, tag, st);
-    else if (race::tc::fast_path_ok(dtype, d, L, P, tau, N) && g_tc_forward)
+    else if (race::tc::fast_path_ok(dtype, d, L, P, tau, N) && al32 && g_tc_forward)
         e = tc_forward(p, q, k, v, W, out, den, states, tau, causal, st, sh);
     else if (dtype == RACE_F32)
         e = dispatch_forward<float>(p, a, states, causal, st, sh);
@@ -1031,7 +1042,8 @@ race_status_t backward_impl(const void *q, const void *k, const void *v, const f
         if (ptr && !aligned16(ptr)) return RACE_ERR_INVALID_ARG;
     const Plan p = make_plan(B, H, N, d, L, P);
     const size_t one = p.state_elems * sizeof(float);
-    const bool wide = sh.stage == STAGE_ALL && !sh.dpq && wide_ok(dtype, d, L, P, tau, causal, N) &&
+    const bool al32 = aligned32({q, k, v, out, dout, dq, dk, dv, workspace, ctx});
+    const bool wide = sh.stage == STAGE_ALL && !sh.dpq && wide_ok(dtype, d, L, P, tau, causal, N) && al32 &&
                       workspace_bytes >= wide_backward_bytes(wide_plan(N, d, L, P));
     if (!wide && workspace_bytes < backward_workspace_bytes(p)) return RACE_ERR_WORKSPACE;
     if (ctx && ctx_bytes < one) return RACE_ERR_WORKSPACE;
@@ -1065,7 +1077,7 @@ race_status_t backward_impl(const void *q, const void *k, const void *v, const f
     cudaError_t e;
     if (wide && g_tc_backward)
         e = wide_backward(B * H, N, d, L, P, q, k, v, W, out, den, dout, dq, dk, dv, tau, workspace, wctx, tag, st);
-    else if (race::tc::fast_path_ok(dtype, d, L, P, tau, N) && g_tc_backward)
+    else if (race::tc::fast_path_ok(dtype, d, L, P, tau, N) && al32 && g_tc_backward)
         e = tc_backward(p, q, k, v, W, out, den, dout, ctx, hbuf, gbuf, wimg, cbuf, dq, dk, dv, tau, causal, st,
                         sh);
     else if (dtype == RACE_F32)
@@ -1198,7 +1210,9 @@ race_status_t race_attn_backward_dw(const void *q, const void *k, const void *v,
                       workspace, bw, stream, sh);
     if (s != RACE_OK) return s;
     cudaError_t e;
-    if (race::tc::fast_path_ok(dtype, d, L, P, tau, N) && g_tc_backward)
+    // the same choice of path as the backward above made (it left dp in that path's format)
+    if (race::tc::fast_path_ok(dtype, d, L, P, tau, N) && aligned32({q, k, v, out, dout, dq, dk, dv, workspace, ctx}) &&
+        g_tc_backward)
         e = tc_dw(p, dp, q, k, sh.dpq, sh.dpk, partial, dW, st);
     else if (dtype == RACE_F32)
         e = generic_dw<float>(p, dp, q, k, (const float *)sh.dpq, (const float *)sh.dpk, partial, dW, st);

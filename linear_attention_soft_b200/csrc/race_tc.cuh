@@ -480,13 +480,10 @@ __device__ __forceinline__ void features_vjp(uint32_t tm, uint32_t col0, int r, 
                      pack_bf16x2(dp[8 * ch + 2], dp[8 * ch + 3]), pack_bf16x2(dp[8 * ch + 4], dp[8 * ch + 5]),
                      pack_bf16x2(dp[8 * ch + 6], dp[8 * ch + 7]));
     if (dp_row && valid) {  // dLoss/dp / |x| of this row's 16 projections, for the gradient of W
-        uint4 *d4 = reinterpret_cast<uint4 *>(dp_row + 16 * qd);
+        uint32_t pk[8];
 #pragma unroll
-        for (int ch = 0; ch < 2; ++ch)
-            d4[ch] = make_uint4(pack_bf16x2(dp[8 * ch] * dp_scale, dp[8 * ch + 1] * dp_scale),
-                                pack_bf16x2(dp[8 * ch + 2] * dp_scale, dp[8 * ch + 3] * dp_scale),
-                                pack_bf16x2(dp[8 * ch + 4] * dp_scale, dp[8 * ch + 5] * dp_scale),
-                                pack_bf16x2(dp[8 * ch + 6] * dp_scale, dp[8 * ch + 7] * dp_scale));
+        for (int k = 0; k < 8; ++k) pk[k] = pack_bf16x2(dp[2 * k] * dp_scale, dp[2 * k + 1] * dp_scale);
+        st_global_v8(dp_row + 16 * qd, pk);
     }
 }
 
@@ -675,11 +672,10 @@ __device__ __forceinline__ void write_dx(uint32_t tm, uint32_t col0, int r, int 
     float y[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) y[i] = (__uint_as_float(w[i]) - x[i] * pj) * inv;
-    uint4 *d4 = reinterpret_cast<uint4 *>(dst + 16 * qd);
-    d4[0] = make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
-                       pack_bf16x2(y[6], y[7]));
-    d4[1] = make_uint4(pack_bf16x2(y[8], y[9]), pack_bf16x2(y[10], y[11]), pack_bf16x2(y[12], y[13]),
-                       pack_bf16x2(y[14], y[15]));
+    uint32_t pk[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) pk[k] = pack_bf16x2(y[2 * k], y[2 * k + 1]);
+    st_global_v8(dst + 16 * qd, pk);
 }
 
 // 16 consecutive TMEM columns of row r (col0 + 16qd) as bf16 to global (16 values), scaled.
@@ -690,14 +686,10 @@ __device__ __forceinline__ void store_row16(uint32_t tm, uint32_t col0, int qd, 
     tmem_ld16_nowait(tlane(tm, col0 + 16u * qd), w);
     tmem_wait_ld();
     if (!valid) return;
-    float y[16];
+    uint32_t pk[8];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) y[i] = __uint_as_float(w[i]) * scale;
-    uint4 *d4 = reinterpret_cast<uint4 *>(dst + 16 * qd);
-    d4[0] = make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
-                       pack_bf16x2(y[6], y[7]));
-    d4[1] = make_uint4(pack_bf16x2(y[8], y[9]), pack_bf16x2(y[10], y[11]), pack_bf16x2(y[12], y[13]),
-                       pack_bf16x2(y[14], y[15]));
+    for (int k = 0; k < 8; ++k) pk[k] = pack_bf16x2(__uint_as_float(w[2 * k]) * scale, __uint_as_float(w[2 * k + 1]) * scale);
+    st_global_v8(dst + 16 * qd, pk);
 }
 
 // out = Y[:, 16 qq ..] / Y[:, 64] for the quarters qq of `qds` (n of them) of row r, with Y at
@@ -723,9 +715,7 @@ __device__ __forceinline__ float store_out_quarters(uint32_t tm, uint32_t ycol, 
                 const float2 y = mul2(make_float2(__uint_as_float(w[i][2 * k]), __uint_as_float(w[i][2 * k + 1])), sc);
                 pk[k] = pack_bf16x2(y.x, y.y);
             }
-            uint4 *d4 = reinterpret_cast<uint4 *>(dst + 16 * qds[i]);
-            d4[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            d4[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            st_global_v8(dst + 16 * qds[i], pk);
         }
     }
     return d;
@@ -1787,9 +1777,10 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_kv_walk(const __grid_constant__
         }
         uint4 xk4[2];  // this row's k values (its tile is being reloaded), fetched while dX^ runs
         if (valid) {
-            const uint4 *src = reinterpret_cast<const uint4 *>(a.k + (base + c0 + r) * DH + 16 * qd);
-            xk4[0] = src[0];
-            xk4[1] = src[1];
+            uint32_t w8[8];
+            ld_global_v8(a.k + (base + c0 + r) * DH + 16 * qd, w8);
+            xk4[0] = make_uint4(w8[0], w8[1], w8[2], w8[3]);
+            xk4[1] = make_uint4(w8[4], w8[5], w8[6], w8[7]);
         }
         if (causal) {  // the updated state is staged while dX^ runs
             float hv[40];

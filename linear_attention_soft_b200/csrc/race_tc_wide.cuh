@@ -284,14 +284,6 @@ __device__ __forceinline__ void add10(float *dst, const float (&v)[10])
     for (int i = 0; i < 5; ++i) red_add_v2(dst + 2 * i, v[2 * i], v[2 * i + 1]);
 }
 
-__device__ __forceinline__ void store_bf16x16(__nv_bfloat16 *dst, const float (&y)[16])
-{
-    uint4 *d4 = reinterpret_cast<uint4 *>(dst);
-    d4[0] = make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
-                       pack_bf16x2(y[6], y[7]));
-    d4[1] = make_uint4(pack_bf16x2(y[8], y[9]), pack_bf16x2(y[10], y[11]), pack_bf16x2(y[12], y[13]),
-                       pack_bf16x2(y[14], y[15]));
-}
 
 // Bounded wait on one TMA barrier by the calling thread alone; false on timeout (after
 // marking the CTA, or the thread group behind `flag`, as given up).
@@ -436,11 +428,10 @@ __global__ void __launch_bounds__(NTH, 1) wide_proj(const __grid_constant__ Proj
             for (int k = 0; k < 5; ++k) {
                 const int c8 = qd + 4 * k;
                 if (c8 >= npw8) break;
-                float4 *d4 = reinterpret_cast<float4 *>(dst + 8 * c8);
-                d4[0] = make_float4(__uint_as_float(w[k][0]) * inv, __uint_as_float(w[k][1]) * inv,
-                                    __uint_as_float(w[k][2]) * inv, __uint_as_float(w[k][3]) * inv);
-                d4[1] = make_float4(__uint_as_float(w[k][4]) * inv, __uint_as_float(w[k][5]) * inv,
-                                    __uint_as_float(w[k][6]) * inv, __uint_as_float(w[k][7]) * inv);
+                uint32_t o[8];
+#pragma unroll
+                for (int m = 0; m < 8; ++m) o[m] = __float_as_uint(__uint_as_float(w[k][m]) * inv);
+                st_global_v8(dst + 8 * c8, o);
             }
         }
     }
@@ -1151,8 +1142,12 @@ __global__ void __launch_bounds__(256) wide_finish(const float *acc, const float
     const int64_t row = t >> 4;
     const int part = (int)(t & 15);
     if (row >= rows) return;
-    const float4 *src = reinterpret_cast<const float4 *>(acc + row * WD) + 2 * part;
-    const float4 x0 = src[0], x1 = src[1];
+    uint32_t w8[8];
+    ld_global_v8(acc + row * WD + 8 * part, w8);
+    const float4 x0 = make_float4(__uint_as_float(w8[0]), __uint_as_float(w8[1]), __uint_as_float(w8[2]),
+                                  __uint_as_float(w8[3]));
+    const float4 x1 = make_float4(__uint_as_float(w8[4]), __uint_as_float(w8[5]), __uint_as_float(w8[6]),
+                                  __uint_as_float(w8[7]));
     float sc = 1.f;
     if (den) {
         const float dn = den[row];
@@ -1226,9 +1221,12 @@ __global__ void __launch_bounds__(NTH, 1) wide_dx(const __grid_constant__ DxArgs
         for (int k = 0; k < 6; ++k) {
             const int c8 = qd + 4 * k;
             if (valid && c8 < np8) {
-                const float4 *src = reinterpret_cast<const float4 *>(a.dp[side] + row * a.npwp + 8 * c8);
-                v[k][0] = src[0];
-                v[k][1] = src[1];
+                uint32_t w8[8];
+                ld_global_v8(a.dp[side] + row * a.npwp + 8 * c8, w8);
+                v[k][0] = make_float4(__uint_as_float(w8[0]), __uint_as_float(w8[1]), __uint_as_float(w8[2]),
+                                      __uint_as_float(w8[3]));
+                v[k][1] = make_float4(__uint_as_float(w8[4]), __uint_as_float(w8[5]), __uint_as_float(w8[6]),
+                                      __uint_as_float(w8[7]));
             } else {
                 v[k][0] = v[k][1] = make_float4(0.f, 0.f, 0.f, 0.f);
             }
@@ -1303,11 +1301,13 @@ __global__ void __launch_bounds__(NTH, 1) wide_dx(const __grid_constant__ DxArgs
 #pragma unroll
             for (int k = 0; k < 32; ++k) y[k] = (__uint_as_float(w[k >> 4][k & 15]) - x[k] * pj) * inv;
             __nv_bfloat16 *dst = a.dx[side] + row * WD + 32 * qd;
-            uint4 *d4 = reinterpret_cast<uint4 *>(dst);
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-                d4[k] = make_uint4(pack_bf16x2(y[8 * k], y[8 * k + 1]), pack_bf16x2(y[8 * k + 2], y[8 * k + 3]),
-                                   pack_bf16x2(y[8 * k + 4], y[8 * k + 5]), pack_bf16x2(y[8 * k + 6], y[8 * k + 7]));
+            for (int k = 0; k < 2; ++k) {
+                uint32_t pk[8];
+#pragma unroll
+                for (int m = 0; m < 8; ++m) pk[m] = pack_bf16x2(y[16 * k + 2 * m], y[16 * k + 2 * m + 1]);
+                st_global_v8(dst + 16 * k, pk);
+            }
         }
     }
     kernel_teardown(tm, 128);

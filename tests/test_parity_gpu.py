@@ -10,6 +10,7 @@ import pytest
 import torch
 
 import oracle
+import linear_attention_soft_b200 as ra
 import race_inputs
 from parity import (TOL, gpu_backward, gpu_forward, oracle_backward, oracle_forward,
                     projection_margin, rel_err, to64)
@@ -170,3 +171,33 @@ def test_causal_output_ignores_later_tokens():
     # the chunked scan sums the same prefix in the same order whatever follows
     assert torch.equal(out[..., :cut, :], out2[..., :cut, :])
     assert torch.equal(den[..., :cut], den2[..., :cut])
+
+
+@pytest.mark.parametrize("shape", [(1, 1, 700, 64, 16, 4), (1, 1, 300, 128, 16, 5)])
+def test_sixteen_byte_aligned_buffers_take_the_general_path(shape):
+    """The tensor-core paths move rows in 32-byte accesses; with tensors only 16-byte aligned
+    (valid for the ABI) the library runs the general path, with the same results."""
+    B, H, N, d, L, P = shape
+    inp = make(shape, torch.bfloat16, seed=77, scale_qk=2.0)
+
+    def off16(t):  # the same values at an address 16 bytes past a 32-byte boundary
+        raw = torch.empty(t.numel() + 16, dtype=t.dtype, device=DEV)
+        v = raw[8:8 + t.numel()].view(t.shape)
+        v.copy_(t)
+        return v
+
+    shifted = {n: (off16(x) if n != "W" else x) for n, x in inp.items()}
+    assert shifted["q"].data_ptr() % 32 == 16
+    ra.race_attn_profile_reset()
+    ra.race_attn_profile_enable(True)
+    out, den, _ = gpu_forward(shifted, 0.5, True)
+    dq, dk, dv = gpu_backward(shifted, out, den, 0.5, True)
+    torch.cuda.synchronize()
+    prof = ra.race_attn_profile_read()
+    ra.race_attn_profile_enable(False)
+    assert not any(n.startswith(("tc_", "wide_")) for n in prof), prof
+    o_ref, den_ref = oracle_forward(inp, 0.5, True)
+    dq_ref, dk_ref, dv_ref = oracle_backward(inp, 0.5, True)
+    errs = {"out": rel_err(out, o_ref), "den": rel_err(den, den_ref), "dq": rel_err(dq, dq_ref),
+            "dk": rel_err(dk, dk_ref), "dv": rel_err(dv, dv_ref)}
+    assert max(errs.values()) <= TOL[torch.bfloat16], errs
