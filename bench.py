@@ -107,11 +107,11 @@ def kernel_work(name: str, w: race_inputs.Workload):
 # taken on: the sha1 of the d = 64 kernel sources and of the planner, comments and
 # whitespace removed.
 NCU_TRAFFIC = {
-    "code_sha1": {"race_tc.cuh": "71a47b360be9e900d79a057bcbb1ffaf3015d976",
-                  "race_tc_util.cuh": "aed713e09ad44ad8a535b2b1684d92827ba3f9e2",
+    "code_sha1": {"race_tc.cuh": "3e07af0a038427dd7415d5d6ab85476f21ff4df5",
+                  "race_tc_util.cuh": "66584d04b44755793b5fb474adf462b16315bf95",
                   "race_attn.cu:make_plan": "368b30caf4555ce78bb0b9b31efea22157570d7e"},
-    "bytes_per_token": {"tc_agg_kv": 259.5, "tc_fwd_walk": 499.5, "tc_bwd_q_walk": 769.4,
-                        "tc_agg_qdy": 265.0, "tc_bwd_kv_walk": 753.0},
+    "bytes_per_token": {"tc_agg_kv": 259.3, "tc_fwd_walk": 502.5, "tc_bwd_q_walk": 769.7,
+                        "tc_agg_qdy": 264.4, "tc_bwd_kv_walk": 756.0},
 }
 
 
