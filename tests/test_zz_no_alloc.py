@@ -5,9 +5,9 @@ Some callers cannot allocate device memory (their device memory belongs to a hos
 framework's allocator, or they cannot afford the synchronisation an allocation may cause),
 so this entry point keeps its scratch in a fixed buffer inside the library.  The test calls
 it through the C ABI twice in a row per case, on different inputs, and compares each result
-with race_attn_forward given its own workspace and with the oracle, on the tensor-core path
-(bf16, d64 L16 P4) and on the general path (fp32, and bf16 with 1,024 features over a
-thread-block cluster).  After the first call it checks that further calls change neither
+with race_attn_forward given its own workspace and with the oracle, on the tensor-core paths
+(bf16 d64 L16 P4; bf16 d128 L32 P5 causal, the feature-group path) and on the general path
+(fp32, and bf16 bidirectional with 1,024 features over a thread-block cluster).  After the first call it checks that further calls change neither
 the device's free memory nor torch's allocations, and that sizes needing more scratch than
 the fixed buffer are refused before anything runs.  This file is collected last so a
 failure here comes after every other test has run.
@@ -23,13 +23,15 @@ from parity import TOL, rel_err, to64
 pytestmark = pytest.mark.gpu
 
 # (B, H, N, d, L, P, tau, causal, dtype): tensor-core path causal and bidirectional, the
-# general fp32 path, and the general bf16 path with L * 2^P = 1024 features (8 cluster CTAs)
+# general fp32 path, the feature-group tensor-core path (d128 L32 P5 causal) and the general
+# bf16 path with L * 2^P = 1024 features (bidirectional: 8 cluster CTAs)
 CASES = [
     (1, 2, 3000, 64, 16, 4, 0.5, True, torch.bfloat16),
     (2, 1, 1300, 64, 16, 4, 0.5, False, torch.bfloat16),
     (1, 2, 2500, 64, 8, 4, 1.0, True, torch.float32),
     (2, 1, 1000, 32, 8, 3, 0.5, False, torch.float32),
     (1, 1, 1500, 128, 32, 5, 0.5, True, torch.bfloat16),
+    (1, 1, 1200, 128, 32, 5, 0.5, False, torch.bfloat16),
 ]
 
 
