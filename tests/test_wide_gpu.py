@@ -139,3 +139,18 @@ def test_context_left_by_another_path_is_not_read():
     torch.cuda.synchronize()
     assert rel_err(out2, out.float().cpu().numpy()) <= TOL[torch.bfloat16]
     assert all(torch.equal(a, b) for a, b in zip(g_ctx2, g_none))
+
+
+@pytest.mark.parametrize("tau", [0.25, 1.0, 3.0])
+def test_other_temperatures(tau):
+    """beta = 1 / tau enters the soft hash and its VJP: forward and backward at three more
+    temperatures."""
+    inp = _inputs(1, 1, 700, 16, seed=int(100 * tau))
+    out, den, _ = gpu_forward(inp, tau, True)
+    dq, dk, dv = gpu_backward(inp, out, den, tau, True)
+    torch.cuda.synchronize()
+    o_ref, den_ref = oracle_forward(inp, tau, True)
+    dq_ref, dk_ref, dv_ref = oracle_backward(inp, tau, True)
+    errs = {"out": rel_err(out, o_ref), "den": rel_err(den, den_ref), "dq": rel_err(dq, dq_ref),
+            "dk": rel_err(dk, dk_ref), "dv": rel_err(dv, dv_ref)}
+    assert max(errs.values()) <= TOL[torch.bfloat16], errs
