@@ -20,7 +20,7 @@
 //                 over the groups in fp32 in memory
 //   wide_finish   out = numerator / den (forward) or dv (backward) from the fp32 sums
 //   wide_rowc     c_i = -(dO_i . o_i) over all 128 columns
-//   wide_bwd_q_walk / wide_bwd_kv_walk: the dq / dk,dv walks of one (group, half)
+//   wide_bwd_q_walk / wide_bwd_kv_walk: the dq / dk,dv walks of the (group, half) passes
 //   wide_dx       dx = (dX^ - x^ (x^ . dX^)) / |x| with dX^ = dp^ W on the tensor core
 //
 // Projections of the group come from shared memory (a [128][40] fp32 tile per chunk and
@@ -1098,7 +1098,7 @@ __global__ void __launch_bounds__(NTH, 1) wide_bwd_kv_walk(const __grid_constant
         }
         wait_mma_each(ctl, phase);
         if (ci > 0) issue_loads(c0 - T);  // Phi_K / masks, V~ and [dO | c'] have been read
-        {  // this pass's dV[:, 16qd ..] into the sum over the groups; the last group writes dv
+        {  // this pass's dV[:, 16qd ..], staged for the sum over the groups (wide_finish writes dv)
             uint32_t w[16];
             tmem_ld16_nowait(tlane(tm, tmc::DVT + 16u * qd), w);
             tmem_wait_ld();
