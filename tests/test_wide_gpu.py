@@ -154,3 +154,20 @@ def test_other_temperatures(tau):
     errs = {"out": rel_err(out, o_ref), "den": rel_err(den, den_ref), "dq": rel_err(dq, dq_ref),
             "dk": rel_err(dk, dk_ref), "dv": rel_err(dv, dv_ref)}
     assert max(errs.values()) <= TOL[torch.bfloat16], errs
+
+
+def test_chunk_and_segment_edges():
+    """Lengths at the edges of a 128-token chunk and of the 512-token minimum segment."""
+    bad = {}
+    for N in (2, 127, 128, 129, 255, 256, 511, 512, 513, 1024, 1025):
+        inp = _inputs(1, 1, N, 8, seed=N)
+        out, den, _ = gpu_forward(inp, 0.5, True)
+        dq, dk, dv = gpu_backward(inp, out, den, 0.5, True)
+        torch.cuda.synchronize()
+        o_ref, den_ref = oracle_forward(inp, 0.5, True)
+        dq_ref, dk_ref, dv_ref = oracle_backward(inp, 0.5, True)
+        errs = {"out": rel_err(out, o_ref), "den": rel_err(den, den_ref), "dq": rel_err(dq, dq_ref),
+                "dk": rel_err(dk, dk_ref), "dv": rel_err(dv, dv_ref)}
+        if max(errs.values()) > TOL[torch.bfloat16]:
+            bad[N] = errs
+    assert not bad, bad
