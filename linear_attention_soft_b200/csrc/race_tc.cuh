@@ -442,10 +442,16 @@ __device__ __forceinline__ void features_vjp(uint32_t tm, uint32_t col0, int r, 
         float gg[16];
 #pragma unroll
         for (int c = 0; c < 16; ++c) gg[c] = __uint_as_float(g[l][c]);
-        if (add_vec) {
-            const float *av = add_vec + 64 * qd + 16 * l;
+        if (add_vec) {  // 16-byte loads (the vector is read by every thread of a quarter)
+            const float4 *av4 = reinterpret_cast<const float4 *>(add_vec + 64 * qd + 16 * l);
 #pragma unroll
-            for (int c = 0; c < 16; ++c) gg[c] = fmaf(add_scale, av[c], gg[c]) * mul;
+            for (int c4 = 0; c4 < 4; ++c4) {
+                const float4 av = av4[c4];
+                gg[4 * c4] = fmaf(add_scale, av.x, gg[4 * c4]) * mul;
+                gg[4 * c4 + 1] = fmaf(add_scale, av.y, gg[4 * c4 + 1]) * mul;
+                gg[4 * c4 + 2] = fmaf(add_scale, av.z, gg[4 * c4 + 2]) * mul;
+                gg[4 * c4 + 3] = fmaf(add_scale, av.w, gg[4 * c4 + 3]) * mul;
+            }
         }
         // Under phi the sign c_p has mean t_p = tanh(beta u_p), so
         // du_p = beta sum_c c_cp phi_c (g_c - phi.g) = beta (2 A_p - (1 + t_p) phi.g),
@@ -512,12 +518,18 @@ __device__ __forceinline__ void mask_block(uint32_t tm, uint32_t col0, int r, in
     const int lim = r - 32 * qd;  // column offset of the diagonal within this warp's 32 columns
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-        float x[8];
+        float x[8], ac[8];
+        if (ADD_COL) {  // 16-byte loads of the per-column terms
+            const float4 a0 = reinterpret_cast<const float4 *>(add_col + 32 * qd + 8 * c)[0];
+            const float4 a1 = reinterpret_cast<const float4 *>(add_col + 32 * qd + 8 * c)[1];
+            ac[0] = a0.x; ac[1] = a0.y; ac[2] = a0.z; ac[3] = a0.w;
+            ac[4] = a1.x; ac[5] = a1.y; ac[6] = a1.z; ac[7] = a1.w;
+        }
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             float y = __uint_as_float(w[c >> 1][8 * (c & 1) + i]);
             if (ADD_ROW) y += add_row;
-            if (ADD_COL) y += add_col[32 * qd + 8 * c + i];
+            if (ADD_COL) y += ac[i];
             x[i] = (diag && (UPPER ? (8 * c + i < lim) : (8 * c + i > lim))) ? 0.f : y;
         }
         st_shared_v4(blk + sw128_off(r, 4 * (qd & 1) + c), pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]),

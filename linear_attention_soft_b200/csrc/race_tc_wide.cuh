@@ -91,17 +91,29 @@ __device__ __forceinline__ const float *state_of(const WideArgs &a, int pass, in
 // 10qd .. 10qd+9 and features 64qd .. 64qd+63 (feature 32e + c of table 2qd+e, corner c).
 
 // u = tanh(p^) and t = tanh(beta u) of this thread's 10 projections, from row r of a [128][40]
-// fp32 tile.
+// fp32 tile.  The 40 bytes start 16-byte aligned for even qd and 8 bytes past for odd qd: two
+// 16-byte loads and one 8-byte load.
 __device__ __forceinline__ void proj_tanh10(const uint8_t *ptile, int r, int qd, float beta, float (&u)[10],
                                             float (&t)[10])
 {
-    const float2 *row = reinterpret_cast<const float2 *>(ptile + (uint32_t)(r * WPROJ + 10 * qd) * 4u);
-#pragma unroll
-    for (int i = 0; i < 5; ++i) {
-        const float2 p = row[i];
-        u[2 * i] = tanh_fast(p.x);
-        u[2 * i + 1] = tanh_fast(p.y);
+    const uint32_t a = smem_u32(ptile) + (uint32_t)(r * WPROJ + 10 * qd) * 4u;
+    float p[10];
+    if ((qd & 1) == 0) {
+        const uint4 x0 = ld_shared_v4(a), x1 = ld_shared_v4(a + 16);
+        const float2 x2 = *reinterpret_cast<const float2 *>(ptile + (uint32_t)(r * WPROJ + 10 * qd + 8) * 4u);
+        p[0] = __uint_as_float(x0.x); p[1] = __uint_as_float(x0.y); p[2] = __uint_as_float(x0.z);
+        p[3] = __uint_as_float(x0.w); p[4] = __uint_as_float(x1.x); p[5] = __uint_as_float(x1.y);
+        p[6] = __uint_as_float(x1.z); p[7] = __uint_as_float(x1.w); p[8] = x2.x; p[9] = x2.y;
+    } else {
+        const float2 x0 = *reinterpret_cast<const float2 *>(ptile + (uint32_t)(r * WPROJ + 10 * qd) * 4u);
+        const uint4 x1 = ld_shared_v4(a + 8), x2 = ld_shared_v4(a + 24);
+        p[0] = x0.x; p[1] = x0.y;
+        p[2] = __uint_as_float(x1.x); p[3] = __uint_as_float(x1.y); p[4] = __uint_as_float(x1.z);
+        p[5] = __uint_as_float(x1.w); p[6] = __uint_as_float(x2.x); p[7] = __uint_as_float(x2.y);
+        p[8] = __uint_as_float(x2.z); p[9] = __uint_as_float(x2.w);
     }
+#pragma unroll
+    for (int i = 0; i < 10; ++i) u[i] = tanh_fast(p[i]);
 #pragma unroll
     for (int i = 0; i < 10; ++i) t[i] = tanh_fast(beta * u[i]);
 }
@@ -185,10 +197,19 @@ __device__ __forceinline__ void features_vjp10(uint32_t tm, uint32_t col0, int q
         corner_weights32(t, e, 1.f, f);
         float fg[32];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-            float gg = __uint_as_float(g[c >> 4][c & 15]);
-            if (add_vec) gg = fmaf(add_scale, add_vec[64 * qd + 32 * e + c], gg) * mul;
-            fg[c] = f[c] * gg;
+        for (int c4 = 0; c4 < 8; ++c4) {
+            float av[4] = {0.f, 0.f, 0.f, 0.f};
+            if (add_vec) {  // 16-byte loads (the vector is read by every thread of a quarter)
+                const float4 a4 = reinterpret_cast<const float4 *>(add_vec + 64 * qd + 32 * e)[c4];
+                av[0] = a4.x; av[1] = a4.y; av[2] = a4.z; av[3] = a4.w;
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int c = 4 * c4 + k;
+                float gg = __uint_as_float(g[c >> 4][c & 15]);
+                if (add_vec) gg = fmaf(add_scale, av[k], gg) * mul;
+                fg[c] = f[c] * gg;
+            }
         }
         float s1[16], s2[8], s3[4];
 #pragma unroll
@@ -222,6 +243,11 @@ __device__ __forceinline__ void features_vjp10(uint32_t tm, uint32_t col0, int q
 // or added there by the memory system (red.global.add, no value returned), so no thread
 // waits on the round trip.  Each element receives one contribution per launch, or two that
 // commute exactly (a + b onto zero), so the sums do not depend on scheduling.
+__device__ __forceinline__ void red_add_v4(float *p, float a, float b, float c, float d)
+{
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
+}
 __device__ __forceinline__ void red_add_v2(float *p, float a, float b)
 {
     asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(p), "f"(a), "f"(b) : "memory");
@@ -277,11 +303,20 @@ __device__ __forceinline__ void put_tile64(const CUtensorMap *map, uint32_t stag
     bulk_commit();
 }
 
-// 10 fp32 values added in memory at dst (8-byte aligned).
-__device__ __forceinline__ void add10(float *dst, const float (&v)[10])
+// 10 fp32 values added in memory at dst, 16-byte aligned for even qd and 8 bytes past a
+// 16-byte boundary for odd qd (dst = row base + 40 bytes x qd): two 16-byte and one 8-byte
+// reduction.
+__device__ __forceinline__ void add10(float *dst, const float (&v)[10], int qd)
 {
-#pragma unroll
-    for (int i = 0; i < 5; ++i) red_add_v2(dst + 2 * i, v[2 * i], v[2 * i + 1]);
+    if ((qd & 1) == 0) {
+        red_add_v4(dst, v[0], v[1], v[2], v[3]);
+        red_add_v4(dst + 4, v[4], v[5], v[6], v[7]);
+        red_add_v2(dst + 8, v[8], v[9]);
+    } else {
+        red_add_v2(dst, v[0], v[1]);
+        red_add_v4(dst + 2, v[2], v[3], v[4], v[5]);
+        red_add_v4(dst + 6, v[6], v[7], v[8], v[9]);
+    }
 }
 
 
@@ -960,7 +995,7 @@ __global__ void __launch_bounds__(NTH, 1) wide_bwd_q_walk(const __grid_constant_
         {  // dphi = (D + c'_i H_prev[:, 64]) / den_i -> dLoss/dp^ of the group's projections
             float dp[10];
             features_vjp10(tm, tmc::DPHI, qd, a.beta, valid, u, t, hden + 256 * par, c_r, invden_r, dp);
-            if (valid) add10(a.dp + (c0 + r) * a.npwp + WPROJ * g + 10 * qd, dp);
+            if (valid) add10(a.dp + (c0 + r) * a.npwp + WPROJ * g + 10 * qd, dp, qd);
         }
         {  // the updated state, staged for the next chunk (its den column into the other buffer)
             float hv[40];
@@ -1111,7 +1146,7 @@ __global__ void __launch_bounds__(NTH, 1) wide_bwd_kv_walk(const __grid_constant
         {
             float dp[10];
             features_vjp10(tm, tmc::DPHI, qd, a.beta, valid, u, t, nullptr, 0.f, 1.f, dp);
-            if (valid) add10(a.dp + (c0 + r) * a.npwp + WPROJ * g + 10 * qd, dp);
+            if (valid) add10(a.dp + (c0 + r) * a.npwp + WPROJ * g + 10 * qd, dp, qd);
         }
         {
             float hv[40];
