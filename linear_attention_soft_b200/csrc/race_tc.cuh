@@ -1493,8 +1493,7 @@ constexpr uint32_t ROWC = HDEN + 1024;
 constexpr uint32_t ROWINV = ROWC + 512;
 constexpr uint32_t RN = ROWINV + 512;
 constexpr uint32_t XCH = RN + 1024;
-constexpr uint32_t XQ2 = XCH + 2048 + 1024;  // q rows kept for dq (1024-aligned)
-constexpr uint32_t BAR = XQ2 + TILE;
+constexpr uint32_t BAR = XCH + 2048;
 constexpr uint32_t TOTAL = BAR + 64;
 }  // namespace bq_smem
 namespace bq_tmem {
@@ -1548,23 +1547,17 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_q_walk(const __grid_constant__ 
             }
         }
     };
-    auto issue_q2 = [&](int64_t c) {  // q rows kept for dq
-        uint64_t *bar = arm_load(ctl, ld, 2, TILE);
-        if (threadIdx.x == 0) tma_k128(sb + XQ2, &a.tm_q, c, bh, bar);
-    };
     auto reload_w = [&]() {  // W tiles (hi, lo) back over the masked block
         uint64_t *bar = arm_load(ctl, ld, 3, 2u * 8192u);
         if (threadIdx.x == 0) bulk_load(sb + WHI, a.wimg, 2u * 8192u, bar);
     };
     if (t0 < t1) {
         issue_kv_do(t0);
-        issue_q2(t0);
     }
     for (int64_t c0 = t0; c0 < t1 && ok; c0 += T) {
         const int nv = (int)(t1 - c0 < T ? t1 - c0 : T);
         const bool valid = r < nv;
-        if (!(ok = wait_loads(ctl, ld, 1u))) break;  // the kept q rows (barrier 2) are waited for at dq
-        if (c0 > t0) issue_q2(c0);  // after the barrier: the last chunk's dx has read the kept rows
+        if (!(ok = wait_loads(ctl, ld, 1u))) break;
         if (threadIdx.x == 3 * 128) {  // the projections and P'' run while quarters 0-2 form the row norms
                                        // and scalars (a thread issuing MMAs is held until the tensor
                                        // core's queue takes the last one)
@@ -1620,9 +1613,15 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_q_walk(const __grid_constant__ 
             issue_dxhat(tm + bq_tmem::DX, sb + DP, sb + WHI, sb + WLO);
             mma_commit(&ctl->bar);
         }
+        uint4 xq4[2];  // this row's q values, fetched while dX^ runs
+        if (valid) {
+            uint32_t w8[8];
+            ld_global_v8(a.q + (base + c0 + r) * DH + 16 * qd, w8);
+            xq4[0] = make_uint4(w8[0], w8[1], w8[2], w8[3]);
+            xq4[1] = make_uint4(w8[4], w8[5], w8[6], w8[7]);
+        }
         wait_mma_each(ctl, phase);
-        wait_loads_nosync(ctl, ld, 4u);     // this chunk's kept q rows
-        write_dx(tm, bq_tmem::DX, r, qd, valid, raw_q, sm + XQ2, nullptr, a.dq + (base + c0 + r) * DH, xch);
+        write_dx(tm, bq_tmem::DX, r, qd, valid, raw_q, nullptr, xq4, a.dq + (base + c0 + r) * DH, xch);
         if (causal) {
             float hv[40];
             read_state40(tm, bq_tmem::HTOP, bq_tmem::HBOT, qd, hv);
@@ -1965,7 +1964,7 @@ static_assert(fwd_smem::XQ % 1024 == 0 && fwd_smem::XK % 1024 == 0 && fwd_smem::
                   fwd_smem::VA1 % 1024 == 0 && fwd_smem::HS % 1024 == 0 && fwd_smem::SB % 1024 == 0,
               "fwd tiles");
 static_assert(bq_smem::XQ % 1024 == 0 && bq_smem::XK % 1024 == 0 && bq_smem::OT % 1024 == 0 &&
-                  bq_smem::XQ2 % 1024 == 0 && bq_smem::VA % 1024 == 0 && bq_smem::DOV % 1024 == 0 &&
+                  bq_smem::VA % 1024 == 0 && bq_smem::DOV % 1024 == 0 &&
                   bq_smem::WHI % 16 == 0,
               "dq walk tiles");
 static_assert(bkv_smem::XQ % 1024 == 0 && bkv_smem::XK % 1024 == 0 && bkv_smem::VA % 1024 == 0 &&
