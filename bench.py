@@ -107,11 +107,11 @@ def kernel_work(name: str, w: race_inputs.Workload):
 # taken on: the sha1 of the d = 64 kernel sources and of the planner, comments and
 # whitespace removed.
 NCU_TRAFFIC = {
-    "code_sha1": {"race_tc.cuh": "737e1cf72b849a2a43ce65d0cf1891b9db60c1f7",
+    "code_sha1": {"race_tc.cuh": "e896e02c7b81127a93bf92eedc49a3905110e92a",
                   "race_tc_util.cuh": "66584d04b44755793b5fb474adf462b16315bf95",
                   "race_attn.cu:make_plan": "368b30caf4555ce78bb0b9b31efea22157570d7e"},
-    "bytes_per_token": {"tc_agg_kv": 259.3, "tc_fwd_walk": 502.8, "tc_bwd_q_walk": 769.5,
-                        "tc_agg_qdy": 264.2, "tc_bwd_kv_walk": 756.3},
+    "bytes_per_token": {"tc_agg_kv": 259.4, "tc_fwd_walk": 502.8, "tc_bwd_q_walk": 770.3,
+                        "tc_agg_qdy": 264.6, "tc_bwd_kv_walk": 756.4},
 }
 
 
