@@ -34,6 +34,15 @@ sys.path.insert(0, ROOT)
 import race_inputs  # noqa: E402
 
 METRIC = "causal RACE attn fwd+bwd tokens/s at N=4M,d=64 (1 B200); % of roofline"
+METRIC_FWD = "RACE attn forward tokens/s (1 B200); % of roofline"  # forward-only workloads
+
+
+def metric_of(w):
+    return METRIC if w.backward else METRIC_FWD
+
+
+def pass_name(w):
+    return "%s %s" % ("causal" if w.causal else "bidirectional", "fwd+bwd" if w.backward else "forward")
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
                   "sm_max_mhz": 1965.0}
 FP32_LANES_PER_SM = 128  # FMA units per SM (4 partitions x 32)
@@ -54,6 +63,8 @@ def load_peaks():
 def step_work(w: race_inputs.Workload):
     s = 4 if w.dtype == "f32" else 2
     M, d, LP = w.L * w.R, w.d, w.L * w.P
+    if not w.backward:  # q, k, v in; out and den out; projections, aggregate, read-out
+        return 4 * d * s + 4, 4 * M * (d + 1) + 4 * LP * d
     byts = 12 * d * s + 8
     flops = 12 * M * (d + 1) + 12 * LP * d
     return byts, flops
@@ -86,7 +97,9 @@ def kernel_work(name: str, w: race_inputs.Workload):
         kv_walk = (4 * d * s, 4 * M * D + 4 * LP * d)       # k, v in; dk, dv out
     table = {
         "agg_kv": (2 * d * s, 2 * M * D + 2 * LP * d),
-        "fwd_walk": (4 * d * s + 4, 4 * M * D + 4 * LP * d),
+        # causal walk: q, k, v in, out and den out; the general path's bidirectional pass of
+        # the same name is a read-out (q in, out and den out)
+        "fwd_walk": (4 * d * s + 4, 4 * M * D + 4 * LP * d) if w.causal else (2 * d * s + 4, 2 * M * D + 2 * LP * d),
         # bidirectional read-out: q in, out and den out
         "readout": (2 * d * s + 4, 2 * M * D + 2 * LP * d),
         "bwd_q_walk": q_walk,
@@ -202,11 +215,13 @@ class ClockSampler:
 def oracle_step(inp_cpu, w, n):
     import numpy as np
     import oracle
-    q, k, v, do = (inp_cpu[x][0, 0, :n].to(torch.float64).numpy() for x in ("q", "k", "v", "do"))
+    q, k, v = (inp_cpu[x][0, 0, :n].to(torch.float64).numpy() for x in ("q", "k", "v"))
+    do = inp_cpu["do"][0, 0, :n].to(torch.float64).numpy() if w.backward else None
     W = inp_cpu["W"].to(torch.float64).numpy()
     t0 = time.perf_counter()
     oracle.forward(q, k, v, W, w.tau, w.causal)
-    oracle.backward(q, k, v, W, do, w.tau, w.causal)
+    if w.backward:
+        oracle.backward(q, k, v, W, do, w.tau, w.causal)
     return time.perf_counter() - t0
 
 
@@ -224,8 +239,8 @@ def cpu_baseline(w, target_s=12.0):
     n = oracle_sample_size(small, w, target_s)
     t = oracle_step(small, w, n)
     return {"value": n / t, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": "causal fwd+bwd of the first %d tokens of head 0 (inputs drawn with the "
-                      "workload's recipe), fp64, wall clock %.1f s" % (n, t)}
+            "sample": "%s of the first %d tokens of head 0 (inputs drawn with the "
+                      "workload's recipe), fp64, wall clock %.1f s" % (pass_name(w), n, t)}
 
 
 def run_reference(args, w):
@@ -242,7 +257,7 @@ def run_reference(args, w):
     times = [oracle_step(small, w, n) for _ in range(args.steps)]
     t = statistics.mean(times)
     val = n / t
-    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s",
+    line = {"impl": "reference", "metric": metric_of(w), "value": val, "unit": "tokens/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -251,8 +266,8 @@ def run_reference(args, w):
                        "sample_tokens_per_step": n},
             "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": oracle.num_threads(),
                              "kind": "oracle",
-                             "sample": "causal fwd+bwd of the first %d tokens of head 0 per step"
-                                       % n},
+                             "sample": "%s of the first %d tokens of head 0 per step"
+                                       % (pass_name(w), n)},
             "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -279,6 +294,8 @@ def sharded_step(inp, w: race_inputs.Workload, lib=None, events=None):
     from linear_attention_soft_b200 import sharded
     out, den, ctx = sharded.forward(inp["q"], inp["k"], inp["v"], inp["W"], w.tau, w.causal, lib=lib,
                                     events=events)
+    if not w.backward:
+        return out, den, None, None, None
     dq, dk, dv = sharded.backward(inp["q"], inp["k"], inp["v"], inp["W"], out, den, inp["do"], w.tau,
                                   w.causal, ctx, lib=lib, events=events)
     return out, den, dq, dk, dv
@@ -320,7 +337,7 @@ def run_ours(args, w):
         raise SystemExit("--dw is not offered by the sequence-sharded passes; use --independent")
     # one sequence sliced over the ranks, or (--independent) one sequence per rank
     inp = shard_inputs(w, rank, dev) if sharded_mode else race_inputs.make_inputs(rank_workload(w, rank), dev)
-    q, k, v, W, do = inp["q"], inp["k"], inp["v"], inp["W"], inp["do"]
+    q, k, v, W, do = inp["q"], inp["k"], inp["v"], inp["W"], inp.get("do")
     B, H, N, d = q.shape
     L, P = w.L, w.P
     out = torch.empty_like(q)
@@ -338,11 +355,14 @@ def run_ours(args, w):
     stream = torch.cuda.current_stream(dev)
 
     def step(qq=q, kk=k, vv=v, dd=do, res=None, events=None):
-        """One forward + backward; returns the five result tensors."""
+        """One forward + backward (a forward alone for forward-only workloads); returns the
+        five result tensors."""
         if sharded_mode:
             return sharded_step({"q": qq, "k": kk, "v": vv, "do": dd, "W": W}, w, events=events)
         o_, den_, dq_, dk_, dv_ = res if res is not None else (out, den, dq, dk, dv)
         ra.race_attn_forward(qq, kk, vv, W, o_, den_, ctx, w.tau, w.causal, ws_f, stream)
+        if not w.backward:
+            return o_, den_, dq_, dk_, dv_
         if args.dw:
             ra.race_attn_backward_dw(qq, kk, vv, W, o_, den_, dd, ctx, dq_, dk_, dv_, dW, w.tau, w.causal, ws_b,
                                      stream)
@@ -391,9 +411,11 @@ def run_ours(args, w):
         # Every step copies its inputs in from pinned host memory and its results out, on their
         # own streams: step i+1's inputs go in and step i-1's results go out while step i
         # computes (two device buffer sets, ordered by events).
-        host = {n: t.cpu().pin_memory() for n, t in (("q", q), ("k", k), ("v", v), ("do", do))}
+        host = {n: t.cpu().pin_memory() for n, t in (("q", q), ("k", k), ("v", v), ("do", do))
+                if t is not None}
         host_out = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
-                    for n, t in (("out", out), ("dq", dq), ("dk", dk), ("dv", dv))}
+                    for n, t in ((("out", out), ("dq", dq), ("dk", dk), ("dv", dv)) if w.backward
+                                 else (("out", out),))}
         dev_in = [{n: torch.empty_like(host[n], device=dev) for n in host} for _ in range(2)]
         dev_res = [(out, den, dq, dk, dv),
                    (torch.empty_like(out), torch.empty_like(den), torch.empty_like(dq), torch.empty_like(dk),
@@ -419,18 +441,17 @@ def run_ours(args, w):
                 stream.wait_event(ev_in[b])
                 if i >= 2:
                     stream.wait_event(ev_out[b])    # step i-2's results are out
-                res = step(dev_in[b]["q"], dev_in[b]["k"], dev_in[b]["v"], dev_in[b]["do"], dev_res[b])
+                res = step(dev_in[b]["q"], dev_in[b]["k"], dev_in[b]["v"], dev_in[b].get("do"), dev_res[b])
                 ev_done[b].record(stream)
                 with torch.cuda.stream(s_out):
                     s_out.wait_event(ev_done[b])
-                    o_, _, dq_, dk_, dv_ = res
                     if sharded_mode:  # the driver's own results, made on the compute stream
                         for t in res:
-                            t.record_stream(s_out)
-                    host_out["out"].copy_(o_, non_blocking=True)
-                    host_out["dq"].copy_(dq_, non_blocking=True)
-                    host_out["dk"].copy_(dk_, non_blocking=True)
-                    host_out["dv"].copy_(dv_, non_blocking=True)
+                            if t is not None:
+                                t.record_stream(s_out)
+                    for n, t in zip(("out", None, "dq", "dk", "dv"), res):
+                        if n in host_out:
+                            host_out[n].copy_(t, non_blocking=True)
                     ev_out[b].record(s_out)
             stream.wait_event(ev_out[(n_steps - 1) & 1])
 
@@ -487,7 +508,7 @@ def run_ours(args, w):
         cpu = cpu_baseline(w)
 
     if rank == 0:
-        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        line = {"metric": metric_of(w), "value": value, "unit": "tokens/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",

@@ -42,3 +42,31 @@ def test_reference_arm_other_ranks_exit_quietly():
     p = _run({"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
     assert p.returncode == 0, p.stderr[-2000:]
     assert not [l for l in p.stdout.splitlines() if l.startswith("{")]
+
+
+def test_reference_arm_forward_only_workload():
+    """The forward-only workload (bidirectional fp32 forward at N = 1024) is timed as a forward
+    pass alone, under its own metric name."""
+    p = _run(args=("--workload", "c1_noncausal_fwd_f32", "--steps", "2", "--warmup", "3"))
+    assert p.returncode == 0, p.stderr[-2000:]
+    lines = [l for l in p.stdout.strip().splitlines() if l.startswith("{")]
+    assert len(lines) == 1, p.stdout
+    d = json.loads(lines[0])
+    assert d["metric"].startswith("RACE attn forward tokens/s")
+    assert d["config"]["workload"] == "c1_noncausal_fwd_f32" and d["config"]["N"] == 1024
+    assert d["cpu_baseline"]["sample"].startswith("bidirectional forward of the first 1024 tokens")
+
+
+def test_step_work_of_forward_only_and_full_steps():
+    """Algorithmic bytes and flops per token: a forward reads q, k, v and writes out and den;
+    forward + backward also reads dO, out and den twice over and writes dq, dk, dv."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import race_inputs
+    c1 = race_inputs.WORKLOADS["c1_noncausal_fwd_f32"]
+    M, D, LP, d = c1.L * c1.R, c1.d + 1, c1.L * c1.P, c1.d
+    assert bench.step_work(c1) == (4 * d * 4 + 4, 4 * M * D + 4 * LP * d)
+    c3 = race_inputs.WORKLOADS["c3_causal_n4m_clusters"]
+    assert bench.step_work(c3) == (1544, 248832)
+    # the general path's bidirectional pass named fwd_walk is a read-out
+    assert bench.kernel_work("generic_fwd_walk", c1) == (2 * d * 4 + 4, 2 * M * D + 2 * LP * d)
