@@ -78,7 +78,7 @@ namespace gk = race::generic;
 constexpr int64_t kSegAlign = 128;     // segment lengths are multiples of this many tokens
 // so that only the last chunk of a head is ragged, where the TMA boxes read zeros past N
 static_assert(kSegAlign % race::tc::T == 0, "segments hold whole chunks");
-constexpr int64_t kMinSegTokens = 512;  // no segment shorter than this (unless N is)
+constexpr int64_t kMinSegTokens = 128;  // no segment shorter than this (unless N is)
 
 struct Plan {
     int BH;

@@ -1776,6 +1776,10 @@ __global__ void __launch_bounds__(NTH, 1) tc_bwd_kv_walk(const __grid_constant__
         }
         wait_mma_each(ctl, phase);
         if (ci > 0) issue_kv_do(c0 - T);  // Phi_K / masks, V~ and [dO | c] are free now
+        if (causal && ci > 0 && qd == 2) {  // the next chunk's c_i and den_i into L2
+            prefetch_l2(a.cbuf + base + c0 - T + r);
+            prefetch_l2(a.den + base + c0 - T + r);
+        }
         reload_w();
         store_row16(tm, bkv_tmem::DVT, qd, valid, 1.f, a.dv + (base + c0 + r) * DH);
         features_vjp(tm, bkv_tmem::DPHI, r, qd, a.beta, valid, u, t, nullptr, 0.f, 1.f, sm + DP,

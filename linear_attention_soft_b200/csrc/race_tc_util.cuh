@@ -263,6 +263,9 @@ __device__ __forceinline__ void st_global_v8(void *dst, const uint32_t (&w)[8])
                  "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
                  : "memory");
 }
+// Bring the 128-byte line holding p into L2 (no register written, nothing waited for).
+__device__ __forceinline__ void prefetch_l2(const void *p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
+
 __device__ __forceinline__ void ld_global_v8(const void *src, uint32_t (&w)[8])
 {
     asm volatile("ld.global.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"

@@ -1133,6 +1133,10 @@ __global__ void __launch_bounds__(NTH, 1) wide_bwd_kv_walk(const __grid_constant
         }
         wait_mma_each(ctl, phase);
         if (ci > 0) issue_loads(c0 - T);  // Phi_K / masks, V~ and [dO | c'] have been read
+        if (ci > 0 && qd == 2) {  // the next chunk's c_i and den_i into L2
+            prefetch_l2(a.cbuf + c0 - T + r);
+            prefetch_l2(a.den + c0 - T + r);
+        }
         {  // this pass's dV[:, 16qd ..], staged for the sum over the groups (wide_finish writes dv)
             uint32_t w[16];
             tmem_ld16_nowait(tlane(tm, tmc::DVT + 16u * qd), w);

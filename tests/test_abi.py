@@ -94,9 +94,11 @@ def test_segment_plan_fills_whole_waves(lib):
     assert 16 * n <= sms and 16 * (n + 1) > sms
     # more heads than SMs: one segment each
     assert _segments(ra, 64, 64, 4096) == 1
-    # never a segment shorter than 512 tokens (unless N is)
+    # never a segment shorter than one 128-token chunk (unless N is); a short head is cut
+    # into chunk-long segments, one CTA each
     for N in (1, 300, 1000, 5000, 70000):
-        assert 1 <= _segments(ra, 1, 1, N) <= max(1, -(-N // 512))
+        assert 1 <= _segments(ra, 1, 1, N) <= max(1, -(-N // 128))
+    assert _segments(ra, 1, 1, 1024) == 8
 
 def _fwd(lib, **kw):
     a = dict(q=16, k=16, v=16, W=16, out=16, den=16, ctx=None, ctx_bytes=0, B=1, H=1, N=256, d=64,

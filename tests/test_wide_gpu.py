@@ -16,7 +16,7 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 # (B, H, N, L): one to four feature groups; N spans one chunk, several segments (segments
-# hold at least 512 tokens) and ragged tails
+# hold whole 128-token chunks) and ragged tails
 CASES = [
     (1, 1, 1, 8),
     (1, 1, 129, 16),
@@ -157,7 +157,7 @@ def test_other_temperatures(tau):
 
 
 def test_chunk_and_segment_edges():
-    """Lengths at the edges of a 128-token chunk and of the 512-token minimum segment."""
+    """Lengths at the edges of a 128-token chunk and of segments of one to four chunks."""
     bad = {}
     for N in (2, 127, 128, 129, 255, 256, 511, 512, 513, 1024, 1025):
         inp = _inputs(1, 1, N, 8, seed=N)
