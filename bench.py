@@ -120,11 +120,11 @@ def kernel_work(name: str, w: race_inputs.Workload):
 # taken on: the sha1 of the d = 64 kernel sources and of the planner, comments and
 # whitespace removed.
 NCU_TRAFFIC = {
-    "code_sha1": {"race_tc.cuh": "e896e02c7b81127a93bf92eedc49a3905110e92a",
-                  "race_tc_util.cuh": "66584d04b44755793b5fb474adf462b16315bf95",
+    "code_sha1": {"race_tc.cuh": "d23e4f78ca71d55d8b4f97c61a71751a45d11b0d",
+                  "race_tc_util.cuh": "574225aad3a9d82eef836e6f2c9f235ec0df8d12",
                   "race_attn.cu:make_plan": "368b30caf4555ce78bb0b9b31efea22157570d7e"},
-    "bytes_per_token": {"tc_agg_kv": 259.4, "tc_fwd_walk": 502.8, "tc_bwd_q_walk": 770.3,
-                        "tc_agg_qdy": 264.6, "tc_bwd_kv_walk": 756.4},
+    "bytes_per_token": {"tc_agg_kv": 259.4, "tc_fwd_walk": 502.1, "tc_bwd_q_walk": 769.8,
+                        "tc_agg_qdy": 264.5, "tc_bwd_kv_walk": 757.1},
 }
 
 
