@@ -176,7 +176,7 @@ race_status_t race_attn_selftest_wait_timeout(int64_t limit_ns, race_stream_t st
  *   launched nothing, when race_attn_workspace_size(..., backward = 0) for these sizes
  *   exceeds RACE_NOALLOC_SCRATCH_BYTES (for d = 64 and 2^P = 16, L = 16, that is B * H * nseg
  *   segment states of 66.5 KB each, nseg being the segments the library plans per sequence:
- *   at most N / 512, usually about (SM count) / (B * H); for bf16, d = 128, P = 5,
+ *   at most N / 128, usually about (SM count) / (B * H); for bf16, d = 128, P = 5,
  *   causal, it includes the per-head arrays of the feature-group path, about
  *   (4 * L * P * 2 + 516) bytes per token; race_attn_workspace_size gives the exact figure).
  *   The first call on each device looks up the buffer's device address (a runtime call
