@@ -1254,6 +1254,18 @@ __global__ void __launch_bounds__(NTH, 1) wide_dx(const __grid_constant__ DxArgs
         const int side = i >= a.ntile ? 1 : 0;
         const int64_t row = (int64_t)(i - side * a.ntile) * T + r;
         const bool valid = row < a.N;
+        {  // this CTA's next tile: its dp^ and x rows into L2 while this one is worked on
+            const int in = i + (int)gridDim.x;
+            const int sn = in >= a.ntile ? 1 : 0;
+            const int64_t rn = (int64_t)(in - sn * a.ntile) * T + r;
+            if (in < ntiles && rn < a.N) {
+                const char *pd = reinterpret_cast<const char *>(a.dp[sn] + rn * a.npwp);
+                const int bytes = 4 * a.npwp;
+                for (int off = 128 * qd; off < bytes; off += 512) prefetch_l2(pd + off);
+                if (qd == 3) prefetch_l2(pd + bytes - 4);  // the row's last line, if it starts mid-line
+                if (qd < 2) prefetch_l2(a.x[sn] + rn * WD + 64 * qd);
+            }
+        }
         // this thread's 8-column chunks qd, qd + 4, ... (at most 6) of the row's dp^ as hi + lo
         float4 v[6][2];
 #pragma unroll
