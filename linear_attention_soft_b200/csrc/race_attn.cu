@@ -241,7 +241,7 @@ Args base_args(const Plan &p, const float *W, float tau)
 
 template <typename Kern>
 cudaError_t launch(Kern kernel, dim3 grid, int cluster_x, size_t smem, cudaStream_t st,
-                   const Args &a)
+                   const Args &a, int cluster_y = 1)
 {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
@@ -255,7 +255,7 @@ cudaError_t launch(Kern kernel, dim3 grid, int cluster_x, size_t smem, cudaStrea
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = cluster_x;
-    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.y = cluster_y;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
@@ -290,6 +290,22 @@ struct Shard {
 
 // ---- the general path (every shape and dtype) ----------------------------------------
 
+// Segment totals on the general path.  When the segments leave most SMs idle (short
+// sequences), the chunks of each segment are split over a cluster of up to 8 CTAs along y
+// (one CTA per SM); the partial sums are added in rank order, so the result does not depend
+// on the timing.
+template <typename Kern>
+cudaError_t launch_agg(Kern kernel, const Plan &p, size_t smem, cudaStream_t st, Args a, int T)
+{
+    const int64_t chunks = (p.seg_len + T - 1) / T;
+    const int64_t ctas = (int64_t)p.G * p.nseg * p.BH;
+    int64_t split = std::min<int64_t>({8, chunks, device_sm_count() / std::max<int64_t>(1, ctas)});
+    if (split < 2) split = 1;
+    a.agg_split = (int)split;
+    const dim3 grid((unsigned)p.G, (unsigned)(p.nseg * split), (unsigned)p.BH);
+    return launch(kernel, grid, 1, smem, st, a, (int)split);
+}
+
 template <typename DT, int T>
 cudaError_t generic_forward(const Plan &p, Args a, float *states, int causal, cudaStream_t st, const Shard &sh)
 {
@@ -300,7 +316,7 @@ cudaError_t generic_forward(const Plan &p, Args a, float *states, int causal, cu
     cudaError_t e;
     if (sh.stage != STAGE_END) {
         e = timed("generic_agg_kv", st, [&] {
-            return launch(gk::race_agg<DT, T, gk::AGG_KV>, grid, 1, smem, st, a);
+            return launch_agg(gk::race_agg<DT, T, gk::AGG_KV>, p, smem, st, a, T);
         });
         if (e != cudaSuccess) return e;
         if (sh.h_total && (e = launch_scan(states, p, gk::SCAN_TOTAL_ONLY, st, nullptr, sh.h_total)) != cudaSuccess)
@@ -311,8 +327,19 @@ cudaError_t generic_forward(const Plan &p, Args a, float *states, int causal, cu
     if (e != cudaSuccess) return e;
     a.state = states;
     a.state_seg_stride = causal ? (int64_t)p.M * p.D : 0;
+    dim3 wgrid = grid;
+    if (!causal) {  // the read-out needs no segments: split the rows over as many CTAs as fill the
+                    // GPU once (one CTA per SM), whole T-token chunks each
+        const int64_t chunks = (p.N + T - 1) / T;
+        int64_t n = std::max<int64_t>(1, device_sm_count() / ((int64_t)p.G * p.BH));
+        n = std::min(n, chunks);
+        if (n > p.nseg) {
+            a.ro_seg_len = (chunks + n - 1) / n * T;
+            wgrid.y = (unsigned)((p.N + a.ro_seg_len - 1) / a.ro_seg_len);
+        }
+    }
     return timed("generic_fwd_walk", st,
-                 [&] { return launch(gk::race_fwd_walk<DT, T>, grid, p.G, smem, st, a); });
+                 [&] { return launch(gk::race_fwd_walk<DT, T>, wgrid, p.G, smem, st, a); });
 }
 
 template <typename DT, int T>
@@ -330,7 +357,7 @@ cudaError_t generic_backward(const Plan &p, Args a, const float *hstates, bool h
         if (!have_ctx) {  // key-side prefix statistics, as the forward computes them
             a.agg_out = hbuf;
             e = timed("generic_agg_kv", st, [&] {
-                return launch(gk::race_agg<DT, T, gk::AGG_KV>, grid, 1, smem, st, a);
+                return launch_agg(gk::race_agg<DT, T, gk::AGG_KV>, p, smem, st, a, T);
             });
             if (e != cudaSuccess) return e;
             e = launch_scan(hbuf, p, causal ? gk::SCAN_EXCL_PREFIX : gk::SCAN_TOTAL, st, sh.h_init);
@@ -344,7 +371,7 @@ cudaError_t generic_backward(const Plan &p, Args a, const float *hstates, bool h
         if (e != cudaSuccess) return e;
         a.agg_out = gbuf;
         e = timed("generic_agg_qdy", st, [&] {
-            return launch(gk::race_agg<DT, T, gk::AGG_QDY>, grid, 1, smem, st, a);
+            return launch_agg(gk::race_agg<DT, T, gk::AGG_QDY>, p, smem, st, a, T);
         });
         if (e != cudaSuccess) return e;
         if (sh.g_total && (e = launch_scan(gbuf, p, gk::SCAN_TOTAL_ONLY, st, nullptr, sh.g_total)) != cudaSuccess)
@@ -874,10 +901,9 @@ template <typename DT, int T>
 cudaError_t generic_totals(const Plan &p, Args a, float *tot, cudaStream_t st)
 {
     const size_t smem = gk::Smem(T, p.d, p.P).total * sizeof(float);
-    const dim3 grid((unsigned)p.G, (unsigned)p.nseg, (unsigned)p.BH);
     a.causal = 0;
     a.agg_out = tot;
-    return timed("generic_agg_kv", st, [&] { return launch(gk::race_agg<DT, T, gk::AGG_KV>, grid, 1, smem, st, a); });
+    return timed("generic_agg_kv", st, [&] { return launch_agg(gk::race_agg<DT, T, gk::AGG_KV>, p, smem, st, a, T); });
 }
 
 template <typename DT>

@@ -62,6 +62,8 @@ struct Args {
     int64_t seg_len;
     int nseg;
     float *dpq, *dpk;  // optional: dLoss/dp / |x| per q (k) row [BH*N][L*P] fp32, for dW
+    int64_t ro_seg_len;  // bidirectional read-out only: tokens per CTA (0: the segments)
+    int agg_split;       // race_agg: CTAs per segment, a cluster along y (0 or 1: one)
 };
 
 // Shared-memory carve-up, in floats.  Identical on host and device.
@@ -493,7 +495,10 @@ __global__ void __launch_bounds__(NT) race_agg(Args a)
 {
     extern __shared__ float sm[];
     const Smem L(T, a.d, a.P);
-    const int g = blockIdx.x, seg = blockIdx.y, bh = blockIdx.z;
+    // with S = agg_split > 1 the S CTAs of a cluster along y share a segment: CTA `sub` takes
+    // its chunks sub, sub + S, ... and rank 0 adds the S partial states in rank order
+    const int S = a.agg_split > 1 ? a.agg_split : 1;
+    const int g = blockIdx.x, seg = blockIdx.y / S, sub = blockIdx.y % S, bh = blockIdx.z;
     const int d = a.d, D = d + 1, R = 1 << a.P;
     const int Mg = min(MG, a.M - g * MG), tg = Mg / R;
     const int64_t base = (int64_t)bh * a.N * d;
@@ -503,7 +508,7 @@ __global__ void __launch_bounds__(NT) race_agg(Args a)
     for (int e = threadIdx.x; e < MG * D; e += NT) st[e] = 0.f;
     int64_t t0, t1;
     seg_range(a, seg, t0, t1);
-    for (int64_t c0 = t0; c0 < t1; c0 += T) {
+    for (int64_t c0 = t0 + (int64_t)sub * T; c0 < t1; c0 += (int64_t)S * T) {
         const int nv = (int)(t1 - c0 < T ? t1 - c0 : (int64_t)T);
         __syncthreads();
         if (MODE == AGG_KV) {
@@ -523,7 +528,19 @@ __global__ void __launch_bounds__(NT) race_agg(Args a)
     }
     __syncthreads();
     float *dst = a.agg_out + (((int64_t)bh * a.nseg + seg) * a.M + (int64_t)g * MG) * D;
-    for (int e = threadIdx.x; e < Mg * D; e += NT) dst[e] = st[e];
+    if (S == 1) {
+        for (int e = threadIdx.x; e < Mg * D; e += NT) dst[e] = st[e];
+        return;
+    }
+    cg::cluster_group cl = cg::this_cluster();
+    cl.sync();  // every partial state is complete
+    if (cl.block_rank() == 0)
+        for (int e = threadIdx.x; e < Mg * D; e += NT) {
+            float acc = st[e];
+            for (int q = 1; q < S; ++q) acc += cl.map_shared_rank(st, q)[e];
+            dst[e] = acc;
+        }
+    cl.sync();  // no CTA leaves while rank 0 still reads its shared memory
 }
 
 // ------------------------------------------------------------------------------------
@@ -696,7 +713,12 @@ __global__ void __launch_bounds__(NT) race_fwd_walk(Args a)
     load_w_group(a.W, g, a.P, d, tg, wg);
     load_state(a, g, seg, bh, Mg, st);
     int64_t t0, t1;
-    seg_range(a, seg, t0, t1);
+    if (!a.causal && a.ro_seg_len > 0) {  // every row reads the same total state: any split works
+        t0 = (int64_t)seg * a.ro_seg_len;
+        t1 = t0 + a.ro_seg_len < a.N ? t0 + a.ro_seg_len : a.N;
+    } else {
+        seg_range(a, seg, t0, t1);
+    }
     int buf = 0;
     for (int64_t c0 = t0; c0 < t1; c0 += T) {
         const int nv = (int)(t1 - c0 < T ? t1 - c0 : (int64_t)T);
