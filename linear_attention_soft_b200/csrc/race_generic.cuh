@@ -189,33 +189,40 @@ __device__ void group_features(const float *x, const float *rawn, int nvalid, co
         }
         const float *xr = x + i * D;
         const float inv = 1.f / fmaxf(rawn[i], kNormEps);
+        // the plane loop is unrolled to its maximum (P <= 5) so that every index into f is a
+        // compile-time constant and f stays in registers
         float f[32];
         f[0] = 1.f;
         int rs = 0;
-        for (int p = 0; p < P; ++p) {
+#pragma unroll
+        for (int p = 0; p < 5; ++p) {
+            if (p >= P) break;
             const float *w = wg + (l * P + p) * d;
             float s = 0.f;
             for (int c = 0; c < d; ++c) s = fmaf(w[c], xr[c], s);
             const float pr = s * inv;
             if (hard) {
                 if (pr > 0.f) rs |= 1 << p;
-                continue;
-            }
-            const float up = tanhf(pr);
-            if (u) u[i * (tg * P) + l * P + p] = up;
-            const float e = expf(-2.f * beta * fabsf(up));
-            const float big = 1.f / (1.f + e), small = e * big;
-            const float s1 = up >= 0.f ? big : small, s0 = up >= 0.f ? small : big;
-            const int h = 1 << p;
-            for (int r = 0; r < h; ++r) {
-                f[r + h] = f[r] * s1;
-                f[r] *= s0;
+            } else {
+                const float up = tanhf(pr);
+                if (u) u[i * (tg * P) + l * P + p] = up;
+                const float e = expf(-2.f * beta * fabsf(up));
+                const float big = 1.f / (1.f + e), small = e * big;
+                const float s1 = up >= 0.f ? big : small, s0 = up >= 0.f ? small : big;
+#pragma unroll
+                for (int r = 0; r < (1 << p); ++r) {
+                    f[r + (1 << p)] = f[r] * s1;
+                    f[r] *= s0;
+                }
             }
         }
-        if (hard)
+        if (hard) {
             for (int r = 0; r < R; ++r) out[r] = r == rs ? 1.f : 0.f;
-        else
-            for (int r = 0; r < R; ++r) out[r] = f[r];
+        } else {
+#pragma unroll
+            for (int r = 0; r < 32; ++r)
+                if (r < R) out[r] = f[r];
+        }
     }
 }
 
@@ -237,12 +244,16 @@ __device__ void group_features_bwd(const float *phi, const float *dphi, const fl
         const float *g = dphi + i * (MG + 1) + l * R;
         float dot = 0.f;
         for (int r = 0; r < R; ++r) dot = fmaf(f[r], g[r], dot);
-        float du[5] = {0.f, 0.f, 0.f, 0.f, 0.f};
+        float du[5] = {0.f, 0.f, 0.f, 0.f, 0.f};  // unrolled to P <= 5: kept in registers
         for (int r = 0; r < R; ++r) {
             const float dz = f[r] * (g[r] - dot);
-            for (int p = 0; p < P; ++p) du[p] += ((r >> p) & 1) ? dz : -dz;
+#pragma unroll
+            for (int p = 0; p < 5; ++p)
+                if (p < P) du[p] += ((r >> p) & 1) ? dz : -dz;
         }
-        for (int p = 0; p < P; ++p) {
+#pragma unroll
+        for (int p = 0; p < 5; ++p) {
+            if (p >= P) break;
             const float up = u[i * (tg * P) + l * P + p];
             o[p] = beta * du[p] * (1.f - up * up);
         }

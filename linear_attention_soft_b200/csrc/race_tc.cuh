@@ -1177,7 +1177,9 @@ __global__ void __launch_bounds__(NTH + 32, 1) tc_fwd_walk(const __grid_constant
     };
     if (issuer_warp) {
         if (threadIdx.x == NTH) {  // the issuing lane
-            uint32_t ph_rows = 0, ph_v[2] = {0, 0}, ph_proj = 0, ph_norm = 0, ph_phiq = 0, ph_phik = 0,
+            // phases and pending flags as scalars: arrays indexed by the chunk parity would live in
+            // local memory
+            uint32_t ph_rows = 0, ph_v0 = 0, ph_v1 = 0, ph_proj = 0, ph_norm = 0, ph_phiq = 0, ph_phik = 0,
                      ph_sb = 0, ph_done = 0;
             auto issue_rows = [&](int64_t c) {
                 mbar_expect_tx(&fb->rows, 2u * TILE);
@@ -1189,22 +1191,22 @@ __global__ void __launch_bounds__(NTH + 32, 1) tc_fwd_walk(const __grid_constant
                 tma_va(sb + (p ? VA1 : VA0), &a.tm_v_va, c, bh, &fb->v[p]);
             };
             auto issue_proj_of = [&](int p) {  // the rows and value tile p of the chunk have landed
-                if (!wait(&fb->rows, ph_rows) || !wait(&fb->v[p], ph_v[p])) return false;
+                if (!wait(&fb->rows, ph_rows) || !(p ? wait(&fb->v[1], ph_v1) : wait(&fb->v[0], ph_v0))) return false;
                 fence_after_sync();
                 issue_proj(tm + fwd_tmem::PROJ, sb + XQ, sb + WHI, sb + WLO);
                 issue_proj(tm + fwd_tmem::PROJ + 64, sb + XK, sb + WHI, sb + WLO);
                 mma_commit(&fb->proj);
                 return true;
             };
-            int rows_pending = 0, v_pending[2] = {0, 0};  // TMA groups issued, not yet waited for
+            int rows_pending = 0, v_pend0 = 0, v_pend1 = 0;  // TMA groups issued, not yet waited for
             bool ok = true;
             if (t0 < t1) {
                 issue_rows(t0);
                 issue_v(t0, 0);
                 rows_pending = 1;
-                v_pending[0] = 1;
+                v_pend0 = 1;
                 ok = issue_proj_of(0);
-                rows_pending = v_pending[0] = 0;
+                rows_pending = v_pend0 = 0;
             }
             int par = 0;
             for (int64_t c0 = t0; c0 < t1 && ok; c0 += T, par ^= 1) {
@@ -1215,7 +1217,8 @@ __global__ void __launch_bounds__(NTH + 32, 1) tc_fwd_walk(const __grid_constant
                     issue_rows(c0 + T);
                     issue_v(c0 + T, par ^ 1);  // last read by the previous chunk's MMAs
                     rows_pending = 1;
-                    v_pending[par ^ 1] = 1;
+                    if (par) v_pend0 = 1;
+                    else v_pend1 = 1;
                 }
                 if (!(ok = wait(&fb->phiq, ph_phiq))) break;
                 fence_after_sync();  // Y = Phi_Q H_prev
@@ -1231,7 +1234,9 @@ __global__ void __launch_bounds__(NTH + 32, 1) tc_fwd_walk(const __grid_constant
                 mma_commit(&fb->sv);
                 if (more) {  // the next chunk's projections: S has been read, the rows are (being) loaded
                     ok = issue_proj_of(par ^ 1);
-                    rows_pending = v_pending[par ^ 1] = 0;
+                    rows_pending = 0;
+                    if (par) v_pend0 = 0;
+                    else v_pend1 = 0;
                     if (!ok) break;
                 }
                 if (!(ok = wait(&fb->done, ph_done))) break;
@@ -1241,8 +1246,8 @@ __global__ void __launch_bounds__(NTH + 32, 1) tc_fwd_walk(const __grid_constant
             mma_commit(&fb->proj);
             mbar_wait(&fb->proj, ph_proj & 1u, WAIT_LIMIT_NS);
             if (rows_pending) mbar_wait(&fb->rows, ph_rows & 1u, WAIT_LIMIT_NS);
-            for (int p = 0; p < 2; ++p)
-                if (v_pending[p]) mbar_wait(&fb->v[p], ph_v[p] & 1u, WAIT_LIMIT_NS);
+            if (v_pend0) mbar_wait(&fb->v[0], ph_v0 & 1u, WAIT_LIMIT_NS);
+            if (v_pend1) mbar_wait(&fb->v[1], ph_v1 & 1u, WAIT_LIMIT_NS);
         }
     } else {
         {  // start state: fp32 master into TMEM, bf16 copy into the staging tile

@@ -724,8 +724,9 @@ __global__ void __launch_bounds__(NTH + 32, 1) wide_fwd_walk(const __grid_consta
     };
     if (issuer_warp) {
         if (threadIdx.x == NTH) {  // the issuing lane
-            uint32_t ph_v[2] = {0, 0}, ph_phiq = 0, ph_phik = 0, ph_sb = 0, ph_done = 0;
-            uint32_t n_rows = 0, n_v[2] = {0, 0};  // loads issued per barrier
+            // scalars, not arrays indexed by the chunk parity (those would live in local memory)
+            uint32_t ph_v0 = 0, ph_v1 = 0, ph_phiq = 0, ph_phik = 0, ph_sb = 0, ph_done = 0;
+            uint32_t n_rows = 0, n_v0 = 0, n_v1 = 0;  // loads issued per barrier
             auto issue_rows = [&](int64_t c) {
                 mbar_expect_tx(&fb->rows, 2u * PTILE);
                 tma_load2(sb + PQ, &a.tm_pq, WPROJ * g, (int)c, &fb->rows);
@@ -735,7 +736,8 @@ __global__ void __launch_bounds__(NTH + 32, 1) wide_fwd_walk(const __grid_consta
             auto issue_v = [&](int64_t c, int p) {
                 mbar_expect_tx(&fb->v[p], TILE);
                 tma_load3(sb + (p ? VA1 : VA0), &a.tm_v, 0, (int)c, 4 * h, &fb->v[p]);
-                ++n_v[p];
+                if (p) ++n_v1;
+                else ++n_v0;
             };
             if (t0 < t1) {
                 issue_rows(t0);
@@ -751,7 +753,7 @@ __global__ void __launch_bounds__(NTH + 32, 1) wide_fwd_walk(const __grid_consta
                 issue_k256_tva(tm + tmc::Y, tm + tmc::PHQ, sb + HS, idesc_bf16(128, 80, 0, 1));
                 if (!(ok = wait(&fb->phik, ph_phik))) break;
                 if (more) issue_rows(c0 + T);  // both projection tiles have been read
-                if (!(ok = wait(&fb->v[par], ph_v[par]))) break;
+                if (!(ok = par ? wait(&fb->v[1], ph_v1) : wait(&fb->v[0], ph_v0))) break;
                 if (staged) {  // the mask after this S overwrites SB: the last Y tile has left it
                     bulk_wait_read();
                     staged = false;
@@ -775,8 +777,8 @@ __global__ void __launch_bounds__(NTH + 32, 1) wide_fwd_walk(const __grid_consta
             mma_commit(&fb->fin);
             mbar_wait(&fb->fin, 0u, WAIT_LIMIT_NS);
             if (n_rows) mbar_wait(&fb->rows, (n_rows - 1u) & 1u, WAIT_LIMIT_NS);
-            for (int p = 0; p < 2; ++p)
-                if (n_v[p]) mbar_wait(&fb->v[p], (n_v[p] - 1u) & 1u, WAIT_LIMIT_NS);
+            if (n_v0) mbar_wait(&fb->v[0], (n_v0 - 1u) & 1u, WAIT_LIMIT_NS);
+            if (n_v1) mbar_wait(&fb->v[1], (n_v1 - 1u) & 1u, WAIT_LIMIT_NS);
         }
     } else {
         {  // start state: fp32 master into TMEM, bf16 copy into the staging tile
