@@ -120,11 +120,11 @@ def kernel_work(name: str, w: race_inputs.Workload):
 # taken on: the sha1 of the d = 64 kernel sources and of the planner, comments and
 # whitespace removed.
 NCU_TRAFFIC = {
-    "code_sha1": {"race_tc.cuh": "d23e4f78ca71d55d8b4f97c61a71751a45d11b0d",
+    "code_sha1": {"race_tc.cuh": "9f7bf0221539d6a3842be7ef8a0990eddbcd37bf",
                   "race_tc_util.cuh": "574225aad3a9d82eef836e6f2c9f235ec0df8d12",
                   "race_attn.cu:make_plan": "368b30caf4555ce78bb0b9b31efea22157570d7e"},
-    "bytes_per_token": {"tc_agg_kv": 259.4, "tc_fwd_walk": 502.1, "tc_bwd_q_walk": 769.8,
-                        "tc_agg_qdy": 264.5, "tc_bwd_kv_walk": 757.1},
+    "bytes_per_token": {"tc_agg_kv": 259.9, "tc_fwd_walk": 502.3, "tc_bwd_q_walk": 769.9,
+                        "tc_agg_qdy": 264.3, "tc_bwd_kv_walk": 756.6},
 }
 
 
